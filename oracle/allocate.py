@@ -1,0 +1,112 @@
+"""Retained-rank allocation: LoRAForge-U and LoRAForge-S, in float64.
+
+Sources
+-------
+* LoRAForge abstract (mlinfo.pages.dev, arXiv 2611.01256): two policies share
+  one backend -- uniform retention ratios (U) and spectral-energy budget
+  allocation (S); the S "floored" configuration exports at 1/12 of rank with a
+  rank floor.
+* LoRAForge (kongchang.com), section "LoRAForge's Core Design: Explicit
+  Retained-Rank Representation and Dual Strategies": U applies one retained
+  ratio to every module; S allocates a total budget by each module's spectral
+  energy accumulation curve, where spectral energy is the sum of squared
+  singular values and each direction carries sigma_j^2 of it.
+
+Readings (the pages give no formula):
+* U: k = round-half-up(num * r / den), clamped to [floor, r].
+* S: budget in rank units per adapter (module ``group``):
+  K = floor(num * sum_i r_i / den).  Every module first receives ``floor``.
+  The remaining K - floor * M slots go to the candidates (i, j), j >= floor,
+  with the largest normalised energy e_ij = sigma_ij^2 / sum_j sigma_ij^2
+  (one module's accumulation curve, read per direction).  Candidates with
+  e_ij = 0 are never taken, so budget can stay unused.  Equal energies are
+  ordered by lower module index, then lower j.  Because e_ij does not increase
+  with j, the chosen set is a prefix of every module, and the greedy choice
+  maximises sum_i (retained energy fraction of module i) under sum_i k_i <= K.
+  If K < floor * M every module keeps ``floor`` (budget exceeded, reported).
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+
+def uniform_rank(r: int, num: int, den: int, floor: int) -> int:
+    """LoRAForge-U retained rank of a rank-r module."""
+    k = (num * r + den // 2) // den
+    return min(r, max(floor, k))
+
+
+def energies(sigma, r: int) -> np.ndarray:
+    """Normalised spectral energies e_j = sigma_j^2 / sum sigma^2 (zeros for a zero module)."""
+    s = np.asarray(sigma, dtype=np.float64)[:r]
+    sq = s * s
+    tot = math.fsum(sq.tolist())
+    if tot == 0.0:
+        return np.zeros(r)
+    return sq / tot
+
+
+def spectral_ranks(sigma_rows, r, group, num: int, den: int, floor: int):
+    """LoRAForge-S ranks for every module.
+
+    sigma_rows: n x r_max array, row i holds module i's singular values in
+    descending order (entries past r_i ignored).
+    Returns (ranks int32[n], info) where info[g] = dict(K, selected, gap_rel,
+    over_budget) per group; gap_rel is the relative energy gap between the last
+    selected and the first unselected candidate (inf if either does not exist).
+    """
+    sigma_rows = np.asarray(sigma_rows, dtype=np.float64)
+    r = np.asarray(r); group = np.asarray(group)
+    n = len(r)
+    ranks = np.zeros(n, dtype=np.int32)
+    info = {}
+    for g in sorted(set(int(x) for x in group)):
+        mods = [i for i in range(n) if int(group[i]) == g]
+        K = (num * int(sum(int(r[i]) for i in mods))) // den
+        extra = K - floor * len(mods)
+        cands = []
+        for i in mods:
+            ri = int(r[i])
+            if floor > ri:
+                raise ValueError("floor exceeds module rank")
+            e = energies(sigma_rows[i], ri)
+            for j in range(floor, ri):
+                if e[j] > 0.0:
+                    cands.append((-e[j], i, j))
+        cands.sort()
+        take = max(extra, 0)
+        chosen = cands[:take]
+        for i in mods:
+            ranks[i] = floor
+        for _, i, _ in chosen:
+            ranks[i] += 1
+        last = -chosen[-1][0] if chosen else None
+        first_out = -cands[take][0] if take < len(cands) else None
+        gap = math.inf
+        if last is not None and first_out is not None and last > 0:
+            gap = (last - first_out) / last
+        info[g] = dict(K=K, selected=len(chosen), gap_rel=gap, over_budget=extra < 0)
+    return ranks, info
+
+
+def brute_force_ranks(sigma_rows, r, num: int, den: int, floor: int):
+    """Exhaustive search for one group (tiny cases only): every rank vector with
+    floor <= k_i <= r_i and sum k_i <= K; returns (best objective, list of optimal
+    rank tuples) for the objective sum_i sum_{j<k_i} e_ij."""
+    import itertools
+    sigma_rows = np.asarray(sigma_rows, dtype=np.float64)
+    r = [int(x) for x in r]
+    K = (num * sum(r)) // den
+    E = [energies(sigma_rows[i], r[i]) for i in range(len(r))]
+    best, arg = -1.0, []
+    for ks in itertools.product(*[range(floor, ri + 1) for ri in r]):
+        if sum(ks) > max(K, floor * len(r)):
+            continue
+        val = math.fsum(math.fsum(E[i][:ks[i]].tolist()) for i in range(len(r)))
+        if val > best + 1e-15:
+            best, arg = val, [ks]
+        elif abs(val - best) <= 1e-15:
+            arg.append(ks)
+    return best, arg

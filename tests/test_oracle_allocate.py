@@ -1,0 +1,76 @@
+"""Pins for oracle.allocate: hand-worked fixtures, brute force, invariants."""
+import json
+import os
+
+import numpy as np
+import pytest
+
+from oracle import allocate as AL
+from tests.conftest import GOLDEN
+
+GOLD = json.load(open(os.path.join(GOLDEN, "allocation_cases.json")))
+
+
+@pytest.mark.parametrize("case", GOLD["uniform"])
+def test_uniform_closed_form(case):
+    assert AL.uniform_rank(case["r"], case["num"], case["den"], case["floor"]) == case["k"]
+
+
+@pytest.mark.parametrize("case", GOLD["spectral"], ids=[c["name"] for c in GOLD["spectral"]])
+def test_spectral_hand_cases(case):
+    ranks, info = AL.spectral_ranks(np.array(case["sigma"], dtype=float), case["r"], case["group"],
+                                    case["num"], case["den"], case["floor"])
+    assert ranks.tolist() == case["ranks"]
+
+
+def test_below_floor_flagged():
+    case = [c for c in GOLD["spectral"] if c["name"] == "below-floor-budget"][0]
+    _, info = AL.spectral_ranks(np.array(case["sigma"], float), case["r"], case["group"],
+                                case["num"], case["den"], case["floor"])
+    assert info[0]["over_budget"]
+
+
+def random_sigma(g, n, r):
+    s = np.sort(np.abs(g.standard_normal((n, r))) * g.uniform(0.1, 3, size=(n, 1)), axis=1)[:, ::-1]
+    return s
+
+
+@pytest.mark.parametrize("seed", range(12))
+def test_greedy_equals_brute_force(seed):
+    g = np.random.default_rng(100 + seed)
+    n, r = int(g.integers(2, 5)), 4
+    sig = random_sigma(g, n, r)
+    num, den = int(g.integers(1, 4)), 4
+    floor = int(g.integers(1, 3))
+    ranks, _ = AL.spectral_ranks(sig, [r] * n, [0] * n, num, den, floor)
+    best, opts = AL.brute_force_ranks(sig, [r] * n, num, den, floor)
+    E = [AL.energies(sig[i], r) for i in range(n)]
+    val = sum(E[i][:ranks[i]].sum() for i in range(n))
+    assert val == pytest.approx(best, abs=1e-12)
+    assert tuple(int(k) for k in ranks) in opts
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_invariants_and_monotone(seed):
+    g = np.random.default_rng(200 + seed)
+    n, r = 30, 16
+    sig = random_sigma(g, n, r)
+    grp = np.repeat([0, 1, 2], 10)
+    prev = None
+    for num in range(1, 13):
+        ranks, info = AL.spectral_ranks(sig, [r] * n, grp, num, 12, 1)
+        assert np.all(ranks >= 1) and np.all(ranks <= r)
+        for gi in range(3):
+            K = (num * r * 10) // 12
+            assert ranks[grp == gi].sum() <= max(K, 10)
+        if prev is not None:
+            assert np.all(ranks >= prev)  # more budget never lowers a rank
+        prev = ranks
+
+
+def test_prefix_closed_with_ties():
+    # equal energies inside one module are taken in j order
+    sig = np.array([[2.0, 1.0, 1.0, 1.0, 1.0]])
+    for num in range(1, 6):
+        ranks, _ = AL.spectral_ranks(sig, [5], [0], num, 5, 1)
+        assert ranks[0] == max(1, num)

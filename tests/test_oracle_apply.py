@@ -1,0 +1,89 @@
+"""Pins for oracle.apply: hand case, brute force, routing by bucket loop, invariants."""
+import json
+import os
+
+import numpy as np
+import pytest
+
+from oracle import apply as AP
+from tests.conftest import GOLDEN
+
+GOLD = json.load(open(os.path.join(GOLDEN, "small_factors.json")))
+
+
+@pytest.mark.parametrize("case", GOLD["apply"])
+def test_apply_hand_case(case):
+    y = AP.lora_apply(np.array(case["x"], float), np.array(case["y0"], float), case["ids"],
+                      case["ranks"], [0], [0], np.array(case["A_pool"], float),
+                      np.array(case["Bt_pool"], float), case["scale"])
+    np.testing.assert_array_equal(y, np.array(case["y"], float))
+
+
+def bucket_route(ids, n):
+    buckets = [[] for _ in range(n)]
+    for t, a in enumerate(ids):
+        if a >= 0:
+            buckets[a].append(t)
+    segs, perm = [], []
+    for a in range(n):
+        if buckets[a]:
+            segs.append((a, len(perm), len(buckets[a])))
+            perm.extend(buckets[a])
+    return segs, perm
+
+
+@pytest.mark.parametrize("seed", range(5))
+def test_route_matches_bucket_loop(seed):
+    g = np.random.default_rng(seed)
+    n = int(g.integers(1, 20))
+    ids = g.integers(-1, n, size=int(g.integers(0, 300)))
+    segs, perm = AP.route(ids, n)
+    s2, p2 = bucket_route(ids.tolist(), n)
+    assert [tuple(s) for s in segs.tolist()] == s2
+    assert perm.tolist() == p2
+
+
+def test_route_rejects_bad_ids():
+    with pytest.raises(ValueError):
+        AP.route([0, 3], 3)
+    with pytest.raises(ValueError):
+        AP.route([0, -2], 3)
+
+
+def make_pools(g, n, d_in, d_out, ranks):
+    offA = np.zeros(n, np.int64); offB = np.zeros(n, np.int64)
+    ta = tb = 0
+    for a in range(n):
+        offA[a], offB[a] = ta, tb
+        ta += ranks[a] * d_in; tb += ranks[a] * d_out
+    return offA, offB, g.standard_normal(ta), g.standard_normal(tb)
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_apply_matches_dense_delta_w(seed):
+    g = np.random.default_rng(10 + seed)
+    n, d_in, d_out, T = 5, 24, 40, 33
+    ranks = g.integers(1, 7, size=n)
+    offA, offB, Ap, Bt = make_pools(g, n, d_in, d_out, ranks)
+    x = g.standard_normal((T, d_in)); y0 = g.standard_normal((T, d_out))
+    ids = g.integers(-1, n, size=T)
+    y1 = AP.lora_apply(x, y0, ids, ranks, offA, offB, Ap, Bt, 1.5)
+    y2 = AP.lora_apply_dense(x, y0, ids, ranks, offA, offB, Ap, Bt, 1.5)
+    np.testing.assert_allclose(y1, y2, atol=1e-12)
+    # rows without an adapter are untouched, bit for bit
+    np.testing.assert_array_equal(y1[ids < 0], y0[ids < 0])
+    # s = 0 leaves y as it is
+    np.testing.assert_array_equal(AP.lora_apply(x, y0, ids, ranks, offA, offB, Ap, Bt, 0.0), y0)
+    # linear in x
+    z = AP.lora_apply(2 * x, 0 * y0, ids, ranks, offA, offB, Ap, Bt, 1.5)
+    z1 = AP.lora_apply(x, 0 * y0, ids, ranks, offA, offB, Ap, Bt, 1.5)
+    np.testing.assert_allclose(z, 2 * z1, atol=1e-12)
+    # permuting tokens permutes the output
+    p = g.permutation(T)
+    y3 = AP.lora_apply(x[p], y0[p], ids[p], ranks, offA, offB, Ap, Bt, 1.5)
+    np.testing.assert_allclose(y3, y1[p], atol=1e-12)
+
+
+def test_empty_batch():
+    y = AP.lora_apply(np.zeros((0, 4)), np.zeros((0, 6)), [], [1], [0], [0], np.ones(4), np.ones(6), 2.0)
+    assert y.shape == (0, 6)
