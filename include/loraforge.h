@@ -1,0 +1,183 @@
+/*
+ * loraforge.h -- C ABI of libloraforge.so, the sm_100a hot path of LoRAForge-style
+ * post-hoc LoRA compression and multi-LoRA serving.
+ *
+ * What the method computes (sources are named by page title and section):
+ *  - "Compress then Serve" (academ.us/article/2407.00066), section 3: a module's
+ *    LoRA update is dW = B A with B (d_out x r) and A (r x d_in); the adapted
+ *    output is (W0 + B A) x.  Section 4, eq. 4: the per-module truncated SVD
+ *    U_k S_k V_k^T is the best rank-k approximation (Eckart-Young), with S_k V_k^T
+ *    stored as one matrix.
+ *  - LoRAForge (kongchang.com), section "FlashTSQR: An Accelerator for Batched
+ *    Factor Construction": factor construction runs a tall-skinny QR (local QR of
+ *    row blocks, then merging) batched across modules and row tiles.
+ *  - LoRAForge abstract (mlinfo.pages.dev, arXiv 2611.01256) and the kongchang.com
+ *    section "LoRAForge's Core Design: Explicit Retained-Rank Representation and
+ *    Dual Strategies": retained ranks come from a uniform ratio (LoRAForge-U) or a
+ *    spectral-energy budget with a per-module floor (LoRAForge-S) and are carried
+ *    as an explicit retained-rank table to rank-specialised kernels, never padded.
+ *  - "Compress then Serve", section 13.4 "Punica": the side path is buffer = A x
+ *    (fp32 buffer, rows selected per token by an adapter index), then
+ *    y += scale * B buffer.
+ *
+ * Conventions shared by every entry point:
+ *  - All pointers are DEVICE pointers unless marked [host].  Matrices are
+ *    row-major.  The caller owns all memory; the library allocates nothing.
+ *    Scratch memory ("workspace") is passed in; its size comes from the matching
+ *    *_workspace_size query.
+ *  - Every call is asynchronous on `stream` (a cudaStream_t; 0 = legacy default).
+ *    Argument errors are found on the host before any launch and returned as an
+ *    lf_status; nothing is launched in that case.  Errors that only the device can
+ *    see (an adapter id out of range, a non-finite value, a pool that is too small,
+ *    a misaligned device offset) are latched into a per-device error word that
+ *    lf_get_device_status() returns and clears.  Kernels never trap.
+ *  - Results are bitwise reproducible from run to run: no floating-point atomics,
+ *    fixed reduction orders.
+ *  - Device pointers to fp32 data must be 16-byte aligned; factor offsets (in
+ *    elements) must be multiples of 4; bf16 rows (x, y, pools) must be 16-byte
+ *    aligned and d_in, d_out multiples of 8.  Violations return LF_ERR_ALIGNMENT.
+ */
+#ifndef LORAFORGE_H
+#define LORAFORGE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* lf_stream_t; /* the same handle as cudaStream_t */
+
+typedef enum {
+    LF_OK = 0,
+    LF_ERR_INVALID_ARG = 1, /* null pointer, negative count, bad policy fields      */
+    LF_ERR_SHAPE = 2,       /* r < 1, r > 64, r > min(d_in, d_out), floor > r ...    */
+    LF_ERR_BAD_INDEX = 3,   /* (device) adapter id < -1 or >= n_adapters             */
+    LF_ERR_WORKSPACE = 4,   /* workspace or output pool smaller than required        */
+    LF_ERR_NUMERIC = 5,     /* (device) non-finite input or singular value           */
+    LF_ERR_TIMEOUT = 6,     /* (device) a bounded wait ran out                       */
+    LF_ERR_CUDA = 7,        /* a CUDA runtime call failed                            */
+    LF_ERR_ALIGNMENT = 8    /* pointer/offset/leading dimension not aligned          */
+} lf_status;
+
+/* One LoRA module (B: d_out x r, A: r x d_in), "Compress then Serve" section 3.
+ * group = adapter id: the scope of the LoRAForge-S budget.
+ * B_off / A_off = element offsets of B and A inside the B_base / A_base buffers. */
+typedef struct {
+    int32_t d_out, d_in, r, group;
+    int64_t B_off, A_off;
+} lf_module;
+
+/* Allocation policy.  kind 0 = LoRAForge-U, kind 1 = LoRAForge-S.
+ * ratio = ratio_num / ratio_den (exact integers, e.g. 1/4, 1/12); floor >= 1.
+ *  U: k = clamp(floor(ratio_num*r/ratio_den + 1/2), floor, r).
+ *  S: per group, K = floor(ratio_num * sum r / ratio_den); every module gets
+ *     `floor`; the remaining K - floor*M slots go to the largest normalised
+ *     energies e_ij = sigma_ij^2 / sum_j sigma_ij^2 (j >= floor, e_ij > 0),
+ *     ties to the lower module index, then lower j. */
+typedef struct {
+    int32_t kind, ratio_num, ratio_den, floor;
+} lf_policy;
+
+/* Largest r over the modules: the stride used by the per-module r x r outputs. */
+int32_t lf_rank_stride(const lf_module* mods /*[host]*/, int32_t n);
+
+/* ---- Factor construction (FlashTSQR + small SVD) -----------------------------
+ * For every module i, with X_B = B_i (d_out x r) and X_A = A_i^T (d_in x r):
+ *   R_B = R(X_B), R_A = R(X_A): the R factors of the thin QRs, upper triangular,
+ *         diag >= 0, computed by a batched tall-skinny QR over row tiles of every
+ *         module at once (leaf tiles folded into a running R, chunk results merged
+ *         in a fixed order);
+ *   M = R_B R_A^T (r x r) and its SVD M = U S V^T in fp64:
+ *   sigma (descending) are the singular values of dW = B A, Q_B U its left and
+ *   Q_A V its right singular vectors.
+ * Outputs (rs = lf_rank_stride):
+ *   R_B, R_A : n x rs x rs fp32, entries past r_i are zero.
+ *   sigma    : n x rs fp64, descending, zero past r_i.
+ *   U, V     : n x rs x rs fp64; column j of U[i] / V[i] pairs with sigma[i][j];
+ *              V columns with sigma = 0 are zero.
+ * Workspace: lf_tsqr_workspace_size(mods, n) bytes.  B_base and A_base are fp32. */
+size_t lf_tsqr_workspace_size(const lf_module* mods /*[host]*/, int32_t n);
+lf_status lf_tsqr_batched(const lf_module* mods /*[host]*/, int32_t n,
+                          const float* B_base, const float* A_base,
+                          float* R_B, float* R_A, double* sigma, double* U, double* V,
+                          void* ws, size_t ws_bytes, lf_stream_t stream);
+
+/* ---- Rank allocation alone (LoRAForge-U / -S) --------------------------------
+ * ranks[i] from sigma (n x rs fp64, rows descending) under `pol`; off_A / off_Bt
+ * are n+1 prefix sums of ranks[i]*d_in and ranks[i]*d_out (pool element offsets).
+ * Workspace: lf_select_workspace_size(mods, n). */
+size_t lf_select_workspace_size(const lf_module* mods /*[host]*/, int32_t n);
+lf_status lf_select_ranks(const lf_module* mods /*[host]*/, int32_t n, lf_policy pol,
+                          const double* sigma, int32_t* ranks, int64_t* off_A, int64_t* off_Bt,
+                          void* ws, size_t ws_bytes, lf_stream_t stream);
+
+/* ---- Truncation + export -----------------------------------------------------
+ * Allocates ranks as lf_select_ranks does.  For LoRAForge-S, modules with a
+ * candidate energy within a relative band of 1e-4 around their group's selection
+ * threshold get their spectrum recomputed in fp64 from B and A before the final
+ * choice, so ranks match an fp64 computation.  Then, per module with k = ranks[i]:
+ *   B'^T = (R_A^T V_k S_k^-1)^T B^T   (k x d_out, rows of the retained left
+ *                                      singular vectors of dW)
+ *   A'   = (U_k^T R_B) A               (k x d_in, = S_k V_k^T Q_A^T)
+ * so that B' A' is the rank-k truncated SVD of dW.  Directions with sigma = 0
+ * export as zero rows.  Pools are packed with no padding: module i occupies
+ * A_pool[off_A[i] .. off_A[i+1]) and Bt_pool[off_Bt[i] .. off_Bt[i+1]).
+ * pool_cap_A / pool_cap_Bt = pool capacities in elements; a larger total latches
+ * LF_ERR_WORKSPACE and writes nothing past the capacity (lf_export_pool_bound gives
+ * a safe capacity).  A_pool_bf16 / Bt_pool_bf16 (same offsets, at least the same
+ * capacities) may be NULL. */
+size_t lf_export_workspace_size(const lf_module* mods /*[host]*/, int32_t n);
+void lf_export_pool_bound(const lf_module* mods /*[host]*/, int32_t n, lf_policy pol,
+                          int64_t* cap_A /*[host]*/, int64_t* cap_Bt /*[host]*/);
+lf_status lf_truncate_export(const lf_module* mods /*[host]*/, int32_t n, lf_policy pol,
+                             const float* B_base, const float* A_base,
+                             const float* R_B, const float* R_A, const double* sigma,
+                             const double* U, const double* V,
+                             int32_t* ranks, int64_t* off_A, int64_t* off_Bt,
+                             float* A_pool, float* Bt_pool,
+                             void* A_pool_bf16, void* Bt_pool_bf16,
+                             int64_t pool_cap_A, int64_t pool_cap_Bt,
+                             void* ws, size_t ws_bytes, lf_stream_t stream);
+
+/* ---- Multi-LoRA shrink / expand (one projection) -----------------------------
+ * For every token t with a = ids[t] >= 0:
+ *   t_vec = A'_a x_t              (k_a values, fp32, never rounded)
+ *   y_t   = bf16( y_t + scale * B'_a t_vec )   (one rounding, RN-even)
+ * x: T x d_in bf16, y: T x d_out bf16 (in place), ids: T int32 (-1 = no adapter,
+ * row left bit-for-bit unchanged; an id >= n_adapters or < -1 latches
+ * LF_ERR_BAD_INDEX and leaves that token untouched).
+ * ranks / off_A / off_Bt: per adapter, this projection's retained rank and element
+ * offsets of its A' (k x d_in) and B'^T (k x d_out) inside the bf16 pools, which
+ * hold pool_elems_A / pool_elems_Bt elements; an adapter whose rows would reach
+ * past a pool (or whose offset is not a multiple of 8, or k > 64) latches an error
+ * on the device and its tokens are left untouched.
+ * Tokens are routed by a stable sort on the adapter id into segments (adapter,
+ * start, length) over a permutation of token indices.  If seg_out is not NULL it
+ * receives, as int32: [n_seg, n_valid, then 3*n_seg (adapter,start,len),
+ * then n_valid token indices]; it must hold 2 + 3*min(T,n_adapters) + T ints.
+ * Segments with many tokens run on tcgen05 tensor cores, the rest on a segmented
+ * GEMV; both read every adapter's k rows once per segment and never pad k.
+ * Workspace: lf_apply_workspace_size(T, n_adapters). */
+size_t lf_apply_workspace_size(int32_t T, int32_t n_adapters);
+lf_status lf_lora_shrink_expand(int32_t T, int32_t d_in, int32_t d_out,
+                                const void* x, void* y, const int32_t* ids,
+                                int32_t n_adapters, const int32_t* ranks,
+                                const int64_t* off_A, const int64_t* off_Bt,
+                                const void* A_pool, const void* Bt_pool,
+                                int64_t pool_elems_A, int64_t pool_elems_Bt, float scale,
+                                int32_t* seg_out, void* ws, size_t ws_bytes,
+                                lf_stream_t stream);
+
+/* ---- Status ------------------------------------------------------------------ */
+const char* lf_status_string(lf_status s);
+/* Synchronises `stream`, returns the first device-side error latched since the
+ * last call (LF_OK if none) and clears it; LF_ERR_CUDA if the stream reports a
+ * CUDA error. */
+lf_status lf_get_device_status(lf_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* LORAFORGE_H */

@@ -1,0 +1,108 @@
+"""Convenience layer over the C ABI: allocates outputs/workspaces as torch CUDA
+tensors and calls the binding.  No arithmetic of the method happens here."""
+from __future__ import annotations
+
+import dataclasses
+
+import numpy as np
+import torch
+
+from . import loraforge as lf
+
+
+def modules_from_layout(layout) -> np.ndarray:
+    """lf_module array from a synth.FleetLayout (or any object with the same fields)."""
+    m = np.zeros(layout.n, dtype=lf.MODULE_DTYPE)
+    m["d_out"], m["d_in"], m["r"], m["group"] = layout.d_out, layout.d_in, layout.r, layout.group
+    m["B_off"], m["A_off"] = layout.B_off, layout.A_off
+    return m
+
+
+@dataclasses.dataclass
+class Factors:
+    R_B: torch.Tensor
+    R_A: torch.Tensor
+    sigma: torch.Tensor
+    U: torch.Tensor
+    V: torch.Tensor
+    rs: int
+
+
+@dataclasses.dataclass
+class Export:
+    ranks: torch.Tensor
+    off_A: torch.Tensor
+    off_Bt: torch.Tensor
+    A_pool: torch.Tensor
+    Bt_pool: torch.Tensor
+    A_pool16: torch.Tensor | None
+    Bt_pool16: torch.Tensor | None
+
+
+def workspace(nbytes: int, device) -> torch.Tensor:
+    return torch.empty(max(int(nbytes), 1), dtype=torch.uint8, device=device)
+
+
+def alloc_factors(mods: np.ndarray, device) -> Factors:
+    n = mods.shape[0]
+    rs = lf.lf_rank_stride(mods)
+    f32 = dict(dtype=torch.float32, device=device)
+    f64 = dict(dtype=torch.float64, device=device)
+    return Factors(torch.empty((n, rs, rs), **f32), torch.empty((n, rs, rs), **f32),
+                   torch.empty((n, rs), **f64), torch.empty((n, rs, rs), **f64),
+                   torch.empty((n, rs, rs), **f64), rs)
+
+
+def tsqr(mods, B_base, A_base, out: Factors | None = None, ws=None, stream=None) -> Factors:
+    dev = B_base.device
+    out = out or alloc_factors(mods, dev)
+    ws = ws if ws is not None else workspace(lf.lf_tsqr_workspace_size(mods), dev)
+    lf.lf_tsqr_batched(mods, B_base, A_base, out.R_B, out.R_A, out.sigma, out.U, out.V, ws, stream)
+    return out
+
+
+def alloc_export(mods, pol, device, bf16: bool = True) -> Export:
+    n = mods.shape[0]
+    capA, capB = lf.lf_export_pool_bound(mods, pol)
+    i64 = dict(dtype=torch.int64, device=device)
+    return Export(torch.empty(n, dtype=torch.int32, device=device), torch.empty(n + 1, **i64),
+                  torch.empty(n + 1, **i64),
+                  torch.empty(max(capA, 8), dtype=torch.float32, device=device),
+                  torch.empty(max(capB, 8), dtype=torch.float32, device=device),
+                  torch.empty(max(capA, 8), dtype=torch.bfloat16, device=device) if bf16 else None,
+                  torch.empty(max(capB, 8), dtype=torch.bfloat16, device=device) if bf16 else None)
+
+
+def truncate_export(mods, pol, B_base, A_base, F: Factors, out: Export | None = None, ws=None,
+                    stream=None, bf16: bool = True) -> Export:
+    dev = B_base.device
+    out = out or alloc_export(mods, pol, dev, bf16)
+    ws = ws if ws is not None else workspace(lf.lf_export_workspace_size(mods), dev)
+    lf.lf_truncate_export(mods, pol, B_base, A_base, F.R_B, F.R_A, F.sigma, F.U, F.V, out.ranks,
+                          out.off_A, out.off_Bt, out.A_pool, out.Bt_pool, out.A_pool16, out.Bt_pool16,
+                          ws, stream)
+    return out
+
+
+def select_ranks(mods, pol, sigma, stream=None):
+    dev = sigma.device
+    n = mods.shape[0]
+    ranks = torch.empty(n, dtype=torch.int32, device=dev)
+    offA = torch.empty(n + 1, dtype=torch.int64, device=dev)
+    offB = torch.empty(n + 1, dtype=torch.int64, device=dev)
+    ws = workspace(lf.lf_select_workspace_size(mods), dev)
+    lf.lf_select_ranks(mods, pol, sigma, ranks, offA, offB, ws, stream)
+    return ranks, offA, offB
+
+
+def shrink_expand(x, y, ids, ranks, off_A, off_Bt, A_pool, Bt_pool, scale, ws=None, seg_out=None,
+                  stream=None):
+    n_adapters = ranks.numel()
+    ws = ws if ws is not None else workspace(lf.lf_apply_workspace_size(x.shape[0], n_adapters), x.device)
+    lf.lf_lora_shrink_expand(x, y, ids, n_adapters, ranks, off_A, off_Bt, A_pool, Bt_pool, scale, ws,
+                             seg_out, stream)
+    return y
+
+
+def device_status(stream=None) -> int:
+    return lf.lf_get_device_status(stream)

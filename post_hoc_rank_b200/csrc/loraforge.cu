@@ -1,0 +1,624 @@
+// libloraforge: host planner + C ABI (see include/loraforge.h for the contract).
+// One translation unit: the kernel headers are included here so the device error
+// word needs no relocatable device code.
+#include <algorithm>
+#include <climits>
+#include <cstring>
+#include <map>
+#include <vector>
+
+#include "common.cuh"
+#include "tsqr.cuh"
+#include "select_export.cuh"
+#include "apply.cuh"
+
+namespace lf {
+
+// ----------------------------------------------------------------- validation
+static lf_status check_mods(const lf_module* mods, int32_t n) {
+    if (n < 0) return LF_ERR_INVALID_ARG;
+    if (n > 0 && !mods) return LF_ERR_INVALID_ARG;
+    for (int32_t i = 0; i < n; ++i) {
+        const lf_module& m = mods[i];
+        if (m.d_out < 1 || m.d_in < 1 || m.r < 1 || m.r > kMaxRank || m.r > m.d_out || m.r > m.d_in)
+            return LF_ERR_SHAPE;
+        if (m.group < 0 || m.B_off < 0 || m.A_off < 0) return LF_ERR_INVALID_ARG;
+        if ((m.B_off & 3) || (m.A_off & 3)) return LF_ERR_ALIGNMENT;
+    }
+    return LF_OK;
+}
+
+static lf_status check_policy(const lf_module* mods, int32_t n, lf_policy p) {
+    if (p.kind != 0 && p.kind != 1) return LF_ERR_INVALID_ARG;
+    if (p.ratio_num < 0 || p.ratio_den <= 0 || p.floor < 1) return LF_ERR_INVALID_ARG;
+    for (int32_t i = 0; i < n; ++i)
+        if (p.floor > mods[i].r) return LF_ERR_SHAPE;
+    return LF_OK;
+}
+
+static int rank_stride(const lf_module* mods, int32_t n) {
+    int rs = 0;
+    for (int32_t i = 0; i < n; ++i) rs = std::max(rs, (int)mods[i].r);
+    return rs;
+}
+
+static int rt_bucket(int rs) { return rs <= 16 ? 16 : (rs <= 32 ? 32 : 64); }
+
+// Host staging: pieces laid out exactly as the Carver lays them out on the device,
+// so one cudaMemcpyAsync uploads all of them.
+struct Staging {
+    std::vector<char> buf;
+    size_t off = 0;
+    template <typename T>
+    size_t put(const T* src, size_t count) {
+        off = (size_t)align_up((int64_t)off, 256);
+        const size_t at = off;
+        off += count * sizeof(T);
+        if (buf.size() < off) buf.resize(off);
+        if (count) std::memcpy(buf.data() + at, src, count * sizeof(T));
+        return at;
+    }
+};
+
+// ------------------------------------------------------------------ TSQR plan
+struct TsqrPlan {
+    std::vector<TsqrWork> work;
+    std::vector<TsqrInfo> info;
+    int32_t slots = 0;
+    int rs = 0, RT = 16;
+};
+
+static void plan_tsqr(const lf_module* mods, int32_t n, TsqrPlan& p) {
+    p.rs = rank_stride(mods, n);
+    p.RT = rt_bucket(p.rs);
+    p.info.resize((size_t)2 * n);
+    p.work.clear();
+    for (int32_t i = 0; i < n; ++i)
+        for (int f = 0; f < 2; ++f) {
+            const int rows = f == 0 ? mods[i].d_out : mods[i].d_in;
+            const int nch = (int)cdiv(rows, kTsqrChunk);
+            const int mf = 2 * i + f;
+            p.info[mf] = TsqrInfo{nch, nch > 1 ? p.slots : -1};
+            for (int c = 0; c < nch; ++c)
+                p.work.push_back(TsqrWork{mf, c * kTsqrChunk, std::min(kTsqrChunk, rows - c * kTsqrChunk),
+                                          nch > 1 ? p.slots + c : -1});
+            if (nch > 1) p.slots += nch;
+        }
+}
+
+struct TsqrLayout {
+    size_t mods, work, nwork, info, n_dev, counters, partial, total;
+};
+
+static TsqrLayout tsqr_layout(int32_t n, const TsqrPlan& p) {
+    Carver c(nullptr);
+    TsqrLayout L;
+#define LF_TAKE(field, T, cnt)                          \
+    do {                                                \
+        c.take<T>(cnt);                                 \
+        L.field = c.off - (size_t)(cnt) * sizeof(T);    \
+    } while (0)
+    LF_TAKE(mods, lf_module, n);
+    LF_TAKE(work, TsqrWork, p.work.size());
+    LF_TAKE(nwork, int32_t, 1);
+    LF_TAKE(info, TsqrInfo, p.info.size());
+    LF_TAKE(n_dev, int32_t, 1);
+    LF_TAKE(counters, int32_t, (size_t)2 * n);
+    LF_TAKE(partial, float, (size_t)p.slots * p.RT * p.RT);
+#undef LF_TAKE
+    L.total = c.off + 256;
+    return L;
+}
+
+template <typename T, int RT>
+static cudaError_t launch_tsqr(const TsqrArgs<T>& a, int grid, cudaStream_t st) {
+    constexpr size_t smem = sizeof(TsqrSmem<T, RT, kTsqrTM>);
+    auto k = tsqr_kernel<T, RT, kTsqrTM, kTsqrThreads>;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    if (grid > 0) k<<<grid, kTsqrThreads, smem, st>>>(a);
+    return cudaGetLastError();
+}
+
+template <typename T>
+static cudaError_t launch_tsqr_rt(int RT, const TsqrArgs<T>& a, int grid, cudaStream_t st) {
+    if (RT == 16) return launch_tsqr<T, 16>(a, grid, st);
+    if (RT == 32) return launch_tsqr<T, 32>(a, grid, st);
+    return launch_tsqr<T, 64>(a, grid, st);
+}
+
+template <typename TIN, int RT>
+static cudaError_t launch_svd(const SvdArgs<TIN>& a, int grid, cudaStream_t st) {
+    constexpr size_t smem = sizeof(SvdSmem<RT>);
+    auto k = svd_kernel<TIN, RT>;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    if (grid > 0) k<<<grid, kSvdThreads, smem, st>>>(a);
+    return cudaGetLastError();
+}
+
+template <typename TIN>
+static cudaError_t launch_svd_rt(int RT, const SvdArgs<TIN>& a, int grid, cudaStream_t st) {
+    if (RT == 16) return launch_svd<TIN, 16>(a, grid, st);
+    if (RT == 32) return launch_svd<TIN, 32>(a, grid, st);
+    return launch_svd<TIN, 64>(a, grid, st);
+}
+
+// ------------------------------------------------------------ groups (S scope)
+static void build_groups(const lf_module* mods, int32_t n, std::vector<int32_t>& ptr, std::vector<int32_t>& gm) {
+    std::map<int32_t, std::vector<int32_t>> by;
+    for (int32_t i = 0; i < n; ++i) by[mods[i].group].push_back(i);
+    ptr.assign(1, 0);
+    gm.clear();
+    for (auto& kv : by) {
+        for (int32_t i : kv.second) gm.push_back(i);
+        ptr.push_back((int32_t)gm.size());
+    }
+}
+
+// ----------------------------------------------------------- export planning
+constexpr int kRefineChunk = 4096;
+constexpr int kExportItem = 2048;
+
+struct ExportPlan {
+    std::vector<int32_t> gptr, gmods;
+    std::vector<ExportWork> ework;
+    int rs = 0, RT = 16;
+    int32_t refine_cap = 0;
+    int32_t refine_max_work = 0;
+    int32_t refine_slots = 0;
+};
+
+static void plan_export(const lf_module* mods, int32_t n, ExportPlan& p) {
+    p.rs = rank_stride(mods, n);
+    p.RT = rt_bucket(p.rs);
+    build_groups(mods, n, p.gptr, p.gmods);
+    const int32_t ngroups = (int32_t)p.gptr.size() - 1;
+    p.ework.clear();
+    int maxd = 1;
+    for (int32_t i = 0; i < n; ++i) {
+        for (int s = 0; s < mods[i].d_out; s += kExportItem)
+            p.ework.push_back(ExportWork{i, 0, s, std::min(kExportItem, mods[i].d_out - s)});
+        for (int s = 0; s < mods[i].d_in; s += kExportItem)
+            p.ework.push_back(ExportWork{i, 1, s, std::min(kExportItem, mods[i].d_in - s)});
+        maxd = std::max(maxd, std::max(mods[i].d_out, mods[i].d_in));
+    }
+    p.refine_cap = std::min<int32_t>(n, 16 * ngroups + 64);
+    const int per = (int)cdiv(maxd, kRefineChunk);
+    p.refine_max_work = p.refine_cap * 2 * per;
+    p.refine_slots = p.refine_cap * 2 * (per > 1 ? per : 0);
+}
+
+struct ExportLayout {
+    size_t mods, gptr, gmods, ework, energy, sigref, flist, fcount, rwork, rnwork, rinfo, rcnt, rpart, rRB, rRA,
+        rsig, CA, CB, total;
+};
+
+static ExportLayout export_layout(int32_t n, const ExportPlan& p) {
+    Carver c(nullptr);
+    ExportLayout L;
+#define LF_TAKE(field, T, cnt)                          \
+    do {                                                \
+        c.take<T>(cnt);                                 \
+        L.field = c.off - (size_t)(cnt) * sizeof(T);    \
+    } while (0)
+    const size_t rs2 = (size_t)p.rs * p.rs;
+    LF_TAKE(mods, lf_module, n);
+    LF_TAKE(gptr, int32_t, p.gptr.size());
+    LF_TAKE(gmods, int32_t, p.gmods.size());
+    LF_TAKE(ework, ExportWork, p.ework.size());
+    LF_TAKE(energy, double, (size_t)n * p.rs);
+    LF_TAKE(sigref, double, (size_t)n * p.rs);
+    LF_TAKE(flist, int32_t, (size_t)n);
+    LF_TAKE(fcount, int32_t, 2);
+    LF_TAKE(rwork, TsqrWork, (size_t)p.refine_max_work);
+    LF_TAKE(rnwork, int32_t, 1);
+    LF_TAKE(rinfo, TsqrInfo, (size_t)2 * p.refine_cap);
+    LF_TAKE(rcnt, int32_t, (size_t)2 * p.refine_cap);
+    LF_TAKE(rpart, double, (size_t)p.refine_slots * p.RT * p.RT);
+    LF_TAKE(rRB, double, (size_t)p.refine_cap * rs2);
+    LF_TAKE(rRA, double, (size_t)p.refine_cap * rs2);
+    LF_TAKE(rsig, double, (size_t)p.refine_cap * p.rs);
+    LF_TAKE(CA, float, (size_t)n * rs2);
+    LF_TAKE(CB, float, (size_t)n * rs2);
+#undef LF_TAKE
+    L.total = c.off + 256;
+    return L;
+}
+
+// Caps the refinement list at `cap` and stores the capped count at count[1].
+__global__ void cap_flags_kernel(int32_t* count, int cap) {
+    if (threadIdx.x == 0 && blockIdx.x == 0) {
+        int c = count[0];
+        if (c > cap) {
+            latch_error(LF_ERR_WORKSPACE);
+            c = cap;
+        }
+        count[0] = c;
+        count[1] = c;
+    }
+}
+
+}  // namespace lf
+
+using namespace lf;
+
+extern "C" {
+
+int32_t lf_rank_stride(const lf_module* mods, int32_t n) { return mods && n > 0 ? rank_stride(mods, n) : 0; }
+
+size_t lf_tsqr_workspace_size(const lf_module* mods, int32_t n) {
+    if (check_mods(mods, n) != LF_OK) return 0;
+    TsqrPlan p;
+    plan_tsqr(mods, n, p);
+    return tsqr_layout(n, p).total;
+}
+
+lf_status lf_tsqr_batched(const lf_module* mods, int32_t n, const float* B_base, const float* A_base, float* R_B,
+                          float* R_A, double* sigma, double* U, double* V, void* ws, size_t ws_bytes,
+                          lf_stream_t stream) {
+    lf_status st = check_mods(mods, n);
+    if (st != LF_OK) return st;
+    if (n == 0) return LF_OK;
+    if (!B_base || !A_base || !R_B || !R_A || !sigma || !ws) return LF_ERR_INVALID_ARG;
+    if (!aligned16(B_base) || !aligned16(A_base)) return LF_ERR_ALIGNMENT;
+    TsqrPlan p;
+    plan_tsqr(mods, n, p);
+    const TsqrLayout L = tsqr_layout(n, p);
+    if (ws_bytes < L.total) return LF_ERR_WORKSPACE;
+    char* base = reinterpret_cast<char*>(align_up((int64_t)reinterpret_cast<uintptr_t>(ws), 256));
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+
+    Staging h;
+    const int32_t nwork = (int32_t)p.work.size();
+    h.put(mods, n);
+    h.put(p.work.data(), p.work.size());
+    h.put(&nwork, 1);
+    h.put(p.info.data(), p.info.size());
+    h.put(&n, 1);
+    LF_CUDA_TRY(cudaMemcpyAsync(base, h.buf.data(), h.off, cudaMemcpyHostToDevice, s));
+    LF_CUDA_TRY(cudaMemsetAsync(base + L.counters, 0, (size_t)2 * n * sizeof(int32_t), s));
+
+    TsqrArgs<float> ta;
+    ta.mods = reinterpret_cast<const lf_module*>(base + L.mods);
+    ta.mod_ids = nullptr;
+    ta.B_base = B_base;
+    ta.A_base = A_base;
+    ta.work = reinterpret_cast<const TsqrWork*>(base + L.work);
+    ta.n_work = reinterpret_cast<const int32_t*>(base + L.nwork);
+    ta.info = reinterpret_cast<const TsqrInfo*>(base + L.info);
+    ta.counters = reinterpret_cast<int32_t*>(base + L.counters);
+    ta.partial = reinterpret_cast<float*>(base + L.partial);
+    ta.R_B = R_B;
+    ta.R_A = R_A;
+    ta.rs = p.rs;
+    LF_CUDA_TRY(launch_tsqr_rt<float>(p.RT, ta, nwork, s));
+
+    SvdArgs<float> sa;
+    sa.mods = ta.mods;
+    sa.mod_ids = nullptr;
+    sa.n = reinterpret_cast<const int32_t*>(base + L.n_dev);
+    sa.R_B = R_B;
+    sa.R_A = R_A;
+    sa.sigma = sigma;
+    sa.U = U;
+    sa.V = V;
+    sa.rs = p.rs;
+    sa.max_sweeps = 30;
+    LF_CUDA_TRY(launch_svd_rt<float>(p.RT, sa, n, s));
+    return LF_OK;
+}
+
+size_t lf_select_workspace_size(const lf_module* mods, int32_t n) {
+    if (check_mods(mods, n) != LF_OK) return 0;
+    ExportPlan p;
+    plan_export(mods, n, p);
+    Carver c(nullptr);
+    c.take<lf_module>(n);
+    c.take<int32_t>(p.gptr.size());
+    c.take<int32_t>(p.gmods.size());
+    c.take<double>((size_t)n * p.rs);
+    return c.off + 256;
+}
+
+lf_status lf_select_ranks(const lf_module* mods, int32_t n, lf_policy pol, const double* sigma, int32_t* ranks,
+                          int64_t* off_A, int64_t* off_Bt, void* ws, size_t ws_bytes, lf_stream_t stream) {
+    lf_status st = check_mods(mods, n);
+    if (st != LF_OK) return st;
+    st = check_policy(mods, n, pol);
+    if (st != LF_OK) return st;
+    if (n == 0) return LF_OK;
+    if (!sigma || !ranks || !off_A || !off_Bt || !ws) return LF_ERR_INVALID_ARG;
+    if (ws_bytes < lf_select_workspace_size(mods, n)) return LF_ERR_WORKSPACE;
+    ExportPlan p;
+    plan_export(mods, n, p);
+    char* base = reinterpret_cast<char*>(align_up((int64_t)reinterpret_cast<uintptr_t>(ws), 256));
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    Staging h;
+    const size_t om = h.put(mods, n);
+    const size_t og = h.put(p.gptr.data(), p.gptr.size());
+    const size_t ogm = h.put(p.gmods.data(), p.gmods.size());
+    h.off = (size_t)align_up((int64_t)h.off, 256);
+    const size_t oe = h.off;
+    LF_CUDA_TRY(cudaMemcpyAsync(base, h.buf.data(), h.buf.size(), cudaMemcpyHostToDevice, s));
+    SelArgs a;
+    a.mods = reinterpret_cast<const lf_module*>(base + om);
+    a.grp_ptr = reinterpret_cast<const int32_t*>(base + og);
+    a.grp_mods = reinterpret_cast<const int32_t*>(base + ogm);
+    a.sigma = sigma;
+    a.energy = reinterpret_cast<double*>(base + oe);
+    a.rs = p.rs;
+    a.pol = pol;
+    a.ranks = ranks;
+    a.band = 0.0;
+    a.flag_list = nullptr;
+    a.flag_count = nullptr;
+    const int ng = (int)p.gptr.size() - 1;
+    select_kernel<<<ng, kSelThreads, 0, s>>>(a);
+    LF_CUDA_TRY(cudaGetLastError());
+    offsets_kernel<<<1, 1024, 0, s>>>(a.mods, n, ranks, off_A, off_Bt, INT64_MAX, INT64_MAX);
+    return launch_status();
+}
+
+size_t lf_export_workspace_size(const lf_module* mods, int32_t n) {
+    if (check_mods(mods, n) != LF_OK) return 0;
+    ExportPlan p;
+    plan_export(mods, n, p);
+    return export_layout(n, p).total;
+}
+
+void lf_export_pool_bound(const lf_module* mods, int32_t n, lf_policy pol, int64_t* cap_A, int64_t* cap_Bt) {
+    if (!cap_A || !cap_Bt) return;
+    *cap_A = *cap_Bt = 0;
+    if (check_mods(mods, n) != LF_OK || check_policy(mods, n, pol) != LF_OK) return;
+    if (pol.kind == 0) {
+        for (int32_t i = 0; i < n; ++i) {
+            const int r = mods[i].r;
+            const int k = std::min(r, std::max(pol.floor, (pol.ratio_num * r + pol.ratio_den / 2) / pol.ratio_den));
+            *cap_A += (int64_t)k * mods[i].d_in;
+            *cap_Bt += (int64_t)k * mods[i].d_out;
+        }
+        return;
+    }
+    // S: floors everywhere, plus the group's extra slots on its widest modules
+    std::map<int32_t, std::vector<int32_t>> by;
+    for (int32_t i = 0; i < n; ++i) by[mods[i].group].push_back(i);
+    for (auto& kv : by) {
+        int64_t rsum = 0;
+        for (int32_t i : kv.second) rsum += mods[i].r;
+        const int64_t K = (int64_t)pol.ratio_num * rsum / pol.ratio_den;
+        int64_t extra = K - (int64_t)pol.floor * (int64_t)kv.second.size();
+        std::vector<std::pair<int, int>> slotsA, slotsB;  // (d, free slots)
+        for (int32_t i : kv.second) {
+            *cap_A += (int64_t)pol.floor * mods[i].d_in;
+            *cap_Bt += (int64_t)pol.floor * mods[i].d_out;
+            slotsA.push_back({mods[i].d_in, mods[i].r - pol.floor});
+            slotsB.push_back({mods[i].d_out, mods[i].r - pol.floor});
+        }
+        auto fill = [&](std::vector<std::pair<int, int>>& v, int64_t* cap) {
+            std::sort(v.begin(), v.end(), [](auto& x, auto& y) { return x.first > y.first; });
+            int64_t left = extra;
+            for (auto& s : v) {
+                if (left <= 0) break;
+                const int64_t t = std::min<int64_t>(left, s.second);
+                *cap += t * s.first;
+                left -= t;
+            }
+        };
+        if (extra > 0) {
+            fill(slotsA, cap_A);
+            fill(slotsB, cap_Bt);
+        }
+    }
+}
+
+lf_status lf_truncate_export(const lf_module* mods, int32_t n, lf_policy pol, const float* B_base,
+                             const float* A_base, const float* R_B, const float* R_A, const double* sigma,
+                             const double* U, const double* V, int32_t* ranks, int64_t* off_A, int64_t* off_Bt,
+                             float* A_pool, float* Bt_pool, void* A_pool_bf16, void* Bt_pool_bf16,
+                             int64_t pool_cap_A, int64_t pool_cap_Bt, void* ws, size_t ws_bytes,
+                             lf_stream_t stream) {
+    lf_status st = check_mods(mods, n);
+    if (st != LF_OK) return st;
+    st = check_policy(mods, n, pol);
+    if (st != LF_OK) return st;
+    if (n == 0) return LF_OK;
+    if (!B_base || !A_base || !R_B || !R_A || !sigma || !U || !V || !ranks || !off_A || !off_Bt || !A_pool ||
+        !Bt_pool || !ws || pool_cap_A < 0 || pool_cap_Bt < 0)
+        return LF_ERR_INVALID_ARG;
+    if (!aligned16(B_base) || !aligned16(A_base)) return LF_ERR_ALIGNMENT;
+    ExportPlan p;
+    plan_export(mods, n, p);
+    const ExportLayout L = export_layout(n, p);
+    if (ws_bytes < L.total) return LF_ERR_WORKSPACE;
+    char* base = reinterpret_cast<char*>(align_up((int64_t)reinterpret_cast<uintptr_t>(ws), 256));
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+
+    Staging h;
+    h.put(mods, n);
+    h.put(p.gptr.data(), p.gptr.size());
+    h.put(p.gmods.data(), p.gmods.size());
+    h.put(p.ework.data(), p.ework.size());
+    LF_CUDA_TRY(cudaMemcpyAsync(base, h.buf.data(), h.off, cudaMemcpyHostToDevice, s));
+    const lf_module* dmods = reinterpret_cast<const lf_module*>(base + L.mods);
+    const int ng = (int)p.gptr.size() - 1;
+
+    SelArgs a;
+    a.mods = dmods;
+    a.grp_ptr = reinterpret_cast<const int32_t*>(base + L.gptr);
+    a.grp_mods = reinterpret_cast<const int32_t*>(base + L.gmods);
+    a.sigma = sigma;
+    a.energy = reinterpret_cast<double*>(base + L.energy);
+    a.rs = p.rs;
+    a.pol = pol;
+    a.ranks = ranks;
+    a.band = 1e-4;
+    a.flag_list = nullptr;
+    a.flag_count = nullptr;
+
+    if (pol.kind == 1) {
+        int32_t* flist = reinterpret_cast<int32_t*>(base + L.flist);
+        int32_t* fcount = reinterpret_cast<int32_t*>(base + L.fcount);
+        LF_CUDA_TRY(cudaMemsetAsync(fcount, 0, 2 * sizeof(int32_t), s));
+        a.flag_list = flist;
+        a.flag_count = fcount;
+        select_kernel<<<ng, kSelThreads, 0, s>>>(a);
+        LF_CUDA_TRY(cudaGetLastError());
+        cap_flags_kernel<<<1, 32, 0, s>>>(fcount, p.refine_cap);
+        LF_CUDA_TRY(cudaGetLastError());
+        TsqrWork* rwork = reinterpret_cast<TsqrWork*>(base + L.rwork);
+        int32_t* rnwork = reinterpret_cast<int32_t*>(base + L.rnwork);
+        TsqrInfo* rinfo = reinterpret_cast<TsqrInfo*>(base + L.rinfo);
+        refine_plan_kernel<<<1, 32, 0, s>>>(dmods, flist, fcount, rwork, rnwork, rinfo, kRefineChunk);
+        LF_CUDA_TRY(cudaGetLastError());
+        LF_CUDA_TRY(cudaMemsetAsync(base + L.rcnt, 0, (size_t)2 * p.refine_cap * sizeof(int32_t), s));
+        TsqrArgs<double> ta;
+        ta.mods = dmods;
+        ta.mod_ids = flist;
+        ta.B_base = B_base;
+        ta.A_base = A_base;
+        ta.work = rwork;
+        ta.n_work = rnwork;
+        ta.info = rinfo;
+        ta.counters = reinterpret_cast<int32_t*>(base + L.rcnt);
+        ta.partial = reinterpret_cast<double*>(base + L.rpart);
+        ta.R_B = reinterpret_cast<double*>(base + L.rRB);
+        ta.R_A = reinterpret_cast<double*>(base + L.rRA);
+        ta.rs = p.rs;
+        LF_CUDA_TRY(launch_tsqr_rt<double>(p.RT, ta, p.refine_max_work, s));
+        SvdArgs<double> sa;
+        sa.mods = dmods;
+        sa.mod_ids = flist;
+        sa.n = fcount + 1;
+        sa.R_B = ta.R_B;
+        sa.R_A = ta.R_A;
+        sa.sigma = reinterpret_cast<double*>(base + L.rsig);
+        sa.U = nullptr;
+        sa.V = nullptr;
+        sa.rs = p.rs;
+        sa.max_sweeps = 30;
+        LF_CUDA_TRY(launch_svd_rt<double>(p.RT, sa, p.refine_cap, s));
+        double* sigref = reinterpret_cast<double*>(base + L.sigref);
+        LF_CUDA_TRY(cudaMemcpyAsync(sigref, sigma, (size_t)n * p.rs * sizeof(double), cudaMemcpyDeviceToDevice, s));
+        scatter_sigma_kernel<<<p.refine_cap, 64, 0, s>>>(flist, fcount + 1, sa.sigma, sigref, p.rs);
+        LF_CUDA_TRY(cudaGetLastError());
+        a.sigma = sigref;
+        a.flag_list = nullptr;
+        a.flag_count = nullptr;
+    }
+    select_kernel<<<ng, kSelThreads, 0, s>>>(a);
+    LF_CUDA_TRY(cudaGetLastError());
+    offsets_kernel<<<1, 1024, 0, s>>>(dmods, n, ranks, off_A, off_Bt, pool_cap_A, pool_cap_Bt);
+    LF_CUDA_TRY(cudaGetLastError());
+    float* CA = reinterpret_cast<float*>(base + L.CA);
+    float* CB = reinterpret_cast<float*>(base + L.CB);
+    export_coef_kernel<<<n, 128, 0, s>>>(dmods, ranks, R_B, R_A, sigma, U, V, p.rs, CA, CB);
+    LF_CUDA_TRY(cudaGetLastError());
+    ExportArgs ea;
+    ea.mods = dmods;
+    ea.work = reinterpret_cast<const ExportWork*>(base + L.ework);
+    ea.B_base = B_base;
+    ea.A_base = A_base;
+    ea.ranks = ranks;
+    ea.off_A = off_A;
+    ea.off_Bt = off_Bt;
+    ea.C_A = CA;
+    ea.C_Bt = CB;
+    ea.rs = p.rs;
+    ea.A_pool = A_pool;
+    ea.Bt_pool = Bt_pool;
+    ea.A_pool16 = reinterpret_cast<__nv_bfloat16*>(A_pool_bf16);
+    ea.Bt_pool16 = reinterpret_cast<__nv_bfloat16*>(Bt_pool_bf16);
+    ea.cap_A = pool_cap_A;
+    ea.cap_Bt = pool_cap_Bt;
+    LF_CUDA_TRY(cudaFuncSetAttribute(export_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kExportSmem));
+    export_kernel<<<(int)p.ework.size(), kExpThreads, kExportSmem, s>>>(ea);
+    return launch_status();
+}
+
+size_t lf_apply_workspace_size(int32_t T, int32_t n_adapters) {
+    if (T < 0 || n_adapters < 1) return 0;
+    const int64_t mseg = std::min<int64_t>(T, n_adapters);
+    Carver c(nullptr);
+    c.take<int32_t>(4);
+    c.take<Seg>((size_t)std::max<int64_t>(mseg, 1));
+    c.take<int32_t>((size_t)std::max(T, 1));
+    c.take<GemvItem>((size_t)(T / kGemvTok + mseg + 1));
+    return c.off + 256;
+}
+
+lf_status lf_lora_shrink_expand(int32_t T, int32_t d_in, int32_t d_out, const void* x, void* y, const int32_t* ids,
+                                int32_t n_adapters, const int32_t* ranks, const int64_t* off_A,
+                                const int64_t* off_Bt, const void* A_pool, const void* Bt_pool,
+                                int64_t pool_elems_A, int64_t pool_elems_Bt, float scale, int32_t* seg_out,
+                                void* ws, size_t ws_bytes, lf_stream_t stream) {
+    if (T < 0 || d_in < 1 || d_out < 1 || n_adapters < 1 || n_adapters > 16384 || pool_elems_A < 0 ||
+        pool_elems_Bt < 0)
+        return LF_ERR_INVALID_ARG;
+    if (T == 0) return LF_OK;
+    if (!x || !y || !ids || !ranks || !off_A || !off_Bt || !A_pool || !Bt_pool || !ws) return LF_ERR_INVALID_ARG;
+    if ((d_in & 7) || (d_out & 7)) return LF_ERR_ALIGNMENT;
+    if (!aligned16(x) || !aligned16(y) || !aligned16(A_pool) || !aligned16(Bt_pool)) return LF_ERR_ALIGNMENT;
+    if (ws_bytes < lf_apply_workspace_size(T, n_adapters)) return LF_ERR_WORKSPACE;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const int64_t mseg = std::min<int64_t>(T, n_adapters);
+    char* wsa = reinterpret_cast<char*>(align_up((int64_t)reinterpret_cast<uintptr_t>(ws), 256));
+    Carver c(wsa);
+    RouteOut o;
+    o.counts = c.take<int32_t>(4);
+    o.segs = c.take<Seg>((size_t)std::max<int64_t>(mseg, 1));
+    o.perm = c.take<int32_t>((size_t)T);
+    o.items = c.take<GemvItem>((size_t)(T / kGemvTok + mseg + 1));
+    o.seg_out = seg_out;
+    const size_t rsmem = (size_t)n_adapters * sizeof(int32_t);
+    LF_CUDA_TRY(cudaFuncSetAttribute(route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rsmem));
+    route_kernel<<<1, kRouteThreads, rsmem, s>>>(ids, T, n_adapters, o);
+    LF_CUDA_TRY(cudaGetLastError());
+    GemvArgs g;
+    g.d_in = d_in;
+    g.d_out = d_out;
+    g.x = reinterpret_cast<const __nv_bfloat16*>(x);
+    g.y = reinterpret_cast<__nv_bfloat16*>(y);
+    g.ranks = ranks;
+    g.off_A = off_A;
+    g.off_Bt = off_Bt;
+    g.A_pool = reinterpret_cast<const __nv_bfloat16*>(A_pool);
+    g.Bt_pool = reinterpret_cast<const __nv_bfloat16*>(Bt_pool);
+    g.pool_A = pool_elems_A;
+    g.pool_Bt = pool_elems_Bt;
+    g.scale = scale;
+    g.counts = o.counts;
+    g.segs = o.segs;
+    g.perm = o.perm;
+    g.items = o.items;
+    dim3 grid((unsigned)(T / kGemvTok + mseg + 1), (unsigned)cdiv(d_out, kGemvCols));
+    gemv_kernel<<<grid, kGemvThreads, 0, s>>>(g);
+    return launch_status();
+}
+
+const char* lf_status_string(lf_status s) {
+    switch (s) {
+        case LF_OK: return "ok";
+        case LF_ERR_INVALID_ARG: return "invalid argument";
+        case LF_ERR_SHAPE: return "bad shape (rank out of range or larger than a dimension)";
+        case LF_ERR_BAD_INDEX: return "adapter id out of range";
+        case LF_ERR_WORKSPACE: return "workspace or output pool too small";
+        case LF_ERR_NUMERIC: return "non-finite value";
+        case LF_ERR_TIMEOUT: return "bounded wait ran out";
+        case LF_ERR_CUDA: return "CUDA runtime error";
+        case LF_ERR_ALIGNMENT: return "misaligned pointer, offset or leading dimension";
+    }
+    return "unknown status";
+}
+
+lf_status lf_get_device_status(lf_stream_t stream) {
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(s) != cudaSuccess) return LF_ERR_CUDA;
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_error, sizeof(int)) != cudaSuccess) return LF_ERR_CUDA;
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_error, &zero, sizeof(int)) != cudaSuccess) return LF_ERR_CUDA;
+    return (lf_status)v;
+}
+
+}  // extern "C"

@@ -1,0 +1,194 @@
+"""ctypes binding of libloraforge.so: the C ABI of include/loraforge.h, same names.
+
+Argument marshalling only: every step of the path runs in the library's CUDA
+kernels.  Tensors are torch tensors used as device allocations; their data
+pointers are passed through.  There is no fallback: if the shared library is
+missing or fails to load, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libloraforge.so")
+
+LF_OK = 0
+STATUS_NAMES = {0: "LF_OK", 1: "LF_ERR_INVALID_ARG", 2: "LF_ERR_SHAPE", 3: "LF_ERR_BAD_INDEX",
+                4: "LF_ERR_WORKSPACE", 5: "LF_ERR_NUMERIC", 6: "LF_ERR_TIMEOUT", 7: "LF_ERR_CUDA",
+                8: "LF_ERR_ALIGNMENT"}
+
+# lf_module: int32 d_out, d_in, r, group; int64 B_off, A_off  (32 bytes, natural alignment)
+MODULE_DTYPE = np.dtype([("d_out", "<i4"), ("d_in", "<i4"), ("r", "<i4"), ("group", "<i4"),
+                         ("B_off", "<i8"), ("A_off", "<i8")], align=True)
+assert MODULE_DTYPE.itemsize == 32
+
+
+class lf_policy(ctypes.Structure):
+    _fields_ = [("kind", ctypes.c_int32), ("ratio_num", ctypes.c_int32),
+                ("ratio_den", ctypes.c_int32), ("floor", ctypes.c_int32)]
+
+
+def policy_U(num: int, den: int, floor: int = 1) -> lf_policy:
+    return lf_policy(0, num, den, floor)
+
+
+def policy_S(num: int, den: int, floor: int = 1) -> lf_policy:
+    return lf_policy(1, num, den, floor)
+
+
+class LFError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)}")
+
+
+_lib = None
+_P = ctypes.c_void_p
+_I32 = ctypes.c_int32
+_I64 = ctypes.c_int64
+_SZ = ctypes.c_size_t
+
+
+def lib() -> ctypes.CDLL:
+    """Load libloraforge.so (raises OSError if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise OSError(f"libloraforge.so not built (expected at {LIB_PATH}); "
+                          "run python -m post_hoc_rank_b200.build")
+        L = ctypes.CDLL(LIB_PATH)
+        L.lf_rank_stride.argtypes = [_P, _I32]; L.lf_rank_stride.restype = _I32
+        L.lf_tsqr_workspace_size.argtypes = [_P, _I32]; L.lf_tsqr_workspace_size.restype = _SZ
+        L.lf_tsqr_batched.argtypes = [_P, _I32, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]
+        L.lf_tsqr_batched.restype = ctypes.c_int
+        L.lf_select_workspace_size.argtypes = [_P, _I32]; L.lf_select_workspace_size.restype = _SZ
+        L.lf_select_ranks.argtypes = [_P, _I32, lf_policy, _P, _P, _P, _P, _P, _SZ, _P]
+        L.lf_select_ranks.restype = ctypes.c_int
+        L.lf_export_workspace_size.argtypes = [_P, _I32]; L.lf_export_workspace_size.restype = _SZ
+        L.lf_export_pool_bound.argtypes = [_P, _I32, lf_policy, _P, _P]; L.lf_export_pool_bound.restype = None
+        L.lf_truncate_export.argtypes = [_P, _I32, lf_policy, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
+                                         _P, _P, _P, _P, _I64, _I64, _P, _SZ, _P]
+        L.lf_truncate_export.restype = ctypes.c_int
+        L.lf_apply_workspace_size.argtypes = [_I32, _I32]; L.lf_apply_workspace_size.restype = _SZ
+        L.lf_lora_shrink_expand.argtypes = [_I32, _I32, _I32, _P, _P, _P, _I32, _P, _P, _P, _P, _P,
+                                            _I64, _I64, ctypes.c_float, _P, _P, _SZ, _P]
+        L.lf_lora_shrink_expand.restype = ctypes.c_int
+        L.lf_status_string.argtypes = [ctypes.c_int]; L.lf_status_string.restype = ctypes.c_char_p
+        L.lf_get_device_status.argtypes = [_P]; L.lf_get_device_status.restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def exported_symbols() -> list[str]:
+    return ["lf_rank_stride", "lf_tsqr_workspace_size", "lf_tsqr_batched", "lf_select_workspace_size",
+            "lf_select_ranks", "lf_export_workspace_size", "lf_export_pool_bound", "lf_truncate_export",
+            "lf_apply_workspace_size", "lf_lora_shrink_expand", "lf_status_string", "lf_get_device_status"]
+
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    if isinstance(t, np.ndarray):
+        return t.ctypes.data
+    return t.data_ptr()
+
+
+def _mods_ptr(mods: np.ndarray):
+    assert mods.dtype == MODULE_DTYPE and mods.flags["C_CONTIGUOUS"]
+    return mods.ctypes.data, int(mods.shape[0])
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(st: int, where: str) -> int:
+    if st != LF_OK:
+        raise LFError(st, where)
+    return st
+
+
+def lf_rank_stride(mods: np.ndarray) -> int:
+    p, n = _mods_ptr(mods)
+    return lib().lf_rank_stride(p, n)
+
+
+def lf_tsqr_workspace_size(mods: np.ndarray) -> int:
+    p, n = _mods_ptr(mods)
+    return lib().lf_tsqr_workspace_size(p, n)
+
+
+def lf_tsqr_batched(mods, B_base, A_base, R_B, R_A, sigma, U, V, ws, stream=None, check=True) -> int:
+    p, n = _mods_ptr(mods)
+    st = lib().lf_tsqr_batched(p, n, _ptr(B_base), _ptr(A_base), _ptr(R_B), _ptr(R_A), _ptr(sigma),
+                               _ptr(U), _ptr(V), _ptr(ws), ws.numel() if ws is not None else 0, _stream(stream))
+    return _check(st, "lf_tsqr_batched") if check else st
+
+
+def lf_select_workspace_size(mods: np.ndarray) -> int:
+    p, n = _mods_ptr(mods)
+    return lib().lf_select_workspace_size(p, n)
+
+
+def lf_select_ranks(mods, pol: lf_policy, sigma, ranks, off_A, off_Bt, ws, stream=None, check=True) -> int:
+    p, n = _mods_ptr(mods)
+    st = lib().lf_select_ranks(p, n, pol, _ptr(sigma), _ptr(ranks), _ptr(off_A), _ptr(off_Bt), _ptr(ws),
+                               ws.numel() if ws is not None else 0, _stream(stream))
+    return _check(st, "lf_select_ranks") if check else st
+
+
+def lf_export_workspace_size(mods: np.ndarray) -> int:
+    p, n = _mods_ptr(mods)
+    return lib().lf_export_workspace_size(p, n)
+
+
+def lf_export_pool_bound(mods: np.ndarray, pol: lf_policy) -> tuple[int, int]:
+    p, n = _mods_ptr(mods)
+    a, b = ctypes.c_int64(0), ctypes.c_int64(0)
+    lib().lf_export_pool_bound(p, n, pol, ctypes.addressof(a), ctypes.addressof(b))
+    return a.value, b.value
+
+
+def lf_truncate_export(mods, pol, B_base, A_base, R_B, R_A, sigma, U, V, ranks, off_A, off_Bt,
+                       A_pool, Bt_pool, A_pool_bf16, Bt_pool_bf16, ws, stream=None, check=True) -> int:
+    p, n = _mods_ptr(mods)
+    st = lib().lf_truncate_export(p, n, pol, _ptr(B_base), _ptr(A_base), _ptr(R_B), _ptr(R_A), _ptr(sigma),
+                                  _ptr(U), _ptr(V), _ptr(ranks), _ptr(off_A), _ptr(off_Bt), _ptr(A_pool),
+                                  _ptr(Bt_pool), _ptr(A_pool_bf16), _ptr(Bt_pool_bf16), A_pool.numel(),
+                                  Bt_pool.numel(), _ptr(ws), ws.numel() if ws is not None else 0,
+                                  _stream(stream))
+    return _check(st, "lf_truncate_export") if check else st
+
+
+def lf_apply_workspace_size(T: int, n_adapters: int) -> int:
+    return lib().lf_apply_workspace_size(T, n_adapters)
+
+
+def lf_lora_shrink_expand(x, y, ids, n_adapters, ranks, off_A, off_Bt, A_pool, Bt_pool, scale, ws,
+                          seg_out=None, stream=None, check=True) -> int:
+    T, d_in = x.shape
+    d_out = y.shape[1]
+    st = lib().lf_lora_shrink_expand(T, d_in, d_out, _ptr(x), _ptr(y), _ptr(ids), n_adapters, _ptr(ranks),
+                                     _ptr(off_A), _ptr(off_Bt), _ptr(A_pool), _ptr(Bt_pool), A_pool.numel(),
+                                     Bt_pool.numel(), float(scale),
+                                     _ptr(seg_out), _ptr(ws), ws.numel() if ws is not None else 0,
+                                     _stream(stream))
+    return _check(st, "lf_lora_shrink_expand") if check else st
+
+
+def lf_status_string(st: int) -> str:
+    return lib().lf_status_string(st).decode()
+
+
+def lf_get_device_status(stream=None) -> int:
+    return lib().lf_get_device_status(_stream(stream))

@@ -1,0 +1,131 @@
+"""C ABI checks that need no GPU: the library loads, exports every symbol the
+header declares, sizes workspaces, and rejects bad arguments on the host
+before any CUDA call."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from post_hoc_rank_b200 import build, loraforge as lf, synth
+from post_hoc_rank_b200.api import modules_from_layout
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    build.build()
+
+
+def header_symbols():
+    txt = open(os.path.join(ROOT, "include", "loraforge.h")).read()
+    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+    return sorted(set(re.findall(r"\b(lf_[a-z0-9_]+)\s*\(", txt)))
+
+
+def test_exports_every_declared_symbol():
+    L = ctypes.CDLL(lf.LIB_PATH)
+    syms = header_symbols()
+    assert len(syms) >= 12
+    for s in syms:
+        assert hasattr(L, s), s
+    assert sorted(lf.exported_symbols()) == syms
+
+
+def test_status_strings():
+    for st in range(9):
+        assert lf.lf_status_string(st) != "unknown status"
+
+
+def tiny_mods():
+    lay = synth.fleet_layout(4, shapes=[("w", 256, 256)], r=16, n_layers=1)
+    return modules_from_layout(lay)
+
+
+def test_rank_stride_and_workspace_sizes():
+    m = tiny_mods()
+    assert lf.lf_rank_stride(m) == 16
+    assert lf.lf_tsqr_workspace_size(m) > 0
+    assert lf.lf_export_workspace_size(m) > 0
+    assert lf.lf_select_workspace_size(m) > 0
+    assert lf.lf_apply_workspace_size(64, 4) > 0
+    assert lf.lf_apply_workspace_size(-1, 4) == 0
+
+
+def test_pool_bound_uniform_exact_and_spectral_safe():
+    m = tiny_mods()
+    a, b = lf.lf_export_pool_bound(m, lf.policy_U(1, 4))
+    assert (a, b) == (4 * 4 * 256, 4 * 4 * 256)
+    # S: 4 groups of one module, r = 16, 1/12 -> K = 1 = floor: only floors
+    a, b = lf.lf_export_pool_bound(m, lf.policy_S(1, 12))
+    assert (a, b) == (4 * 256, 4 * 256)
+    m2 = modules_from_layout(synth.fleet_layout(1, shapes=[("a", 512, 64), ("b", 64, 1024)], r=16, n_layers=1))
+    a, b = lf.lf_export_pool_bound(m2, lf.policy_S(1, 2))   # K = 16, extra 14 -> widest module first
+    assert a == 1 * 64 + 1 * 1024 + 14 * 1024
+    assert b == 1 * 512 + 1 * 64 + 14 * 512
+
+
+def call_tsqr(m, ws_bytes=1 << 20, **over):
+    args = dict(B=16, A=16, RB=16, RA=16, S=16, U=16, V=16)
+    args.update(over)
+    p, n = m.ctypes.data, m.shape[0]
+    return lf.lib().lf_tsqr_batched(p, n, args["B"], args["A"], args["RB"], args["RA"], args["S"],
+                                    args["U"], args["V"], 16, ws_bytes, None)
+
+
+def test_tsqr_rejects_bad_shapes_on_host():
+    m = tiny_mods()
+    bad = m.copy(); bad["r"][1] = 65
+    assert call_tsqr(bad) == 2
+    bad = m.copy(); bad["r"][0] = 300
+    assert call_tsqr(bad) == 2
+    bad = m.copy(); bad["d_in"][2] = 0
+    assert call_tsqr(bad) == 2
+    bad = m.copy(); bad["A_off"][3] = 6
+    assert call_tsqr(bad) == 8
+    assert call_tsqr(m, B=0) == 1
+    assert call_tsqr(m, A=12) == 8                  # misaligned base pointer
+    assert call_tsqr(m, ws_bytes=16) == 4           # workspace too small
+    assert lf.lib().lf_tsqr_batched(m.ctypes.data, -1, 16, 16, 16, 16, 16, 16, 16, 16, 1 << 20, None) == 1
+    assert lf.lib().lf_tsqr_batched(m.ctypes.data, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, None) == 0
+
+
+def test_policy_validation_on_host():
+    m = tiny_mods()
+    p, n = m.ctypes.data, m.shape[0]
+    L = lf.lib()
+    bad_policies = [lf.lf_policy(2, 1, 4, 1), lf.lf_policy(0, 1, 0, 1), lf.lf_policy(1, 1, 4, 0)]
+    for pol in bad_policies:
+        assert L.lf_select_ranks(p, n, pol, 16, 16, 16, 16, 16, 1 << 20, None) == 1
+    assert L.lf_select_ranks(p, n, lf.lf_policy(1, 1, 4, 17), 16, 16, 16, 16, 16, 1 << 20, None) == 2
+
+
+def test_apply_validation_on_host():
+    L = lf.lib()
+    ok = dict(T=4, d_in=64, d_out=64, x=16, y=16, ids=16, n=2, ranks=16, oa=16, ob=16, A=16, B=16, ws=16,
+              wsb=1 << 20, pa=1024, pb=1024)
+
+    def call(**o):
+        a = dict(ok); a.update(o)
+        return L.lf_lora_shrink_expand(a["T"], a["d_in"], a["d_out"], a["x"], a["y"], a["ids"], a["n"],
+                                       a["ranks"], a["oa"], a["ob"], a["A"], a["B"], a["pa"], a["pb"], 1.0,
+                                       None, a["ws"],
+                                       a["wsb"], None)
+    assert call(T=0) == 0
+    assert call(T=-1) == 1
+    assert call(d_in=60) == 8
+    assert call(d_out=12) == 8
+    assert call(x=8) == 8
+    assert call(n=0) == 1
+    assert call(n=20000) == 1
+    assert call(wsb=8) == 4
+    assert call(ids=0) == 1
+    assert call(pa=-1) == 1
+
+
+def test_module_dtype_matches_c_struct():
+    assert lf.MODULE_DTYPE.itemsize == 32
+    assert [lf.MODULE_DTYPE.fields[f][1] for f in ("d_out", "d_in", "r", "group", "B_off", "A_off")] == \
+        [0, 4, 8, 12, 16, 24]

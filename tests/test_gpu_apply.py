@@ -1,0 +1,138 @@
+"""GPU parity of lf_lora_shrink_expand (routing + shrink/expand) against the fp64
+oracle on the same bf16 bytes."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import apply as OP
+from post_hoc_rank_b200 import api, build, synth
+from post_hoc_rank_b200 import loraforge as lf
+from tests import gpu_util as G
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    build.build()
+    assert torch.cuda.is_available()
+
+
+def make_pools(ranks, d_in, d_out, key, std_a=None, std_b=None):
+    """Packed bf16 pools (A' k x d_in, B'^T k x d_out per adapter), N(0, 1/d) entries."""
+    ranks = np.asarray(ranks, dtype=np.int64)
+    offA = np.concatenate([[0], np.cumsum(ranks * d_in)])
+    offB = np.concatenate([[0], np.cumsum(ranks * d_out)])
+    Ap = synth.normal_bf16((max(int(offA[-1]), 8),), key + (0,), std=std_a or d_in ** -0.5)
+    Bt = synth.normal_bf16((max(int(offB[-1]), 8),), key + (1,), std=std_b or d_out ** -0.5)
+    return offA, offB, Ap, Bt
+
+
+def run_apply(x, y0, ids, ranks, offA, offB, Ap, Bt, scale, seg=False):
+    dev = "cuda"
+    T = x.shape[0]
+    n = len(ranks)
+    y = y0.clone().to(dev)
+    seg_out = torch.full((2 + 3 * min(T, n) + T,), -7, dtype=torch.int32, device=dev) if seg else None
+    api.shrink_expand(x.to(dev), y, torch.from_numpy(np.asarray(ids, np.int32)).to(dev),
+                      torch.from_numpy(np.asarray(ranks, np.int32)).to(dev),
+                      torch.from_numpy(np.asarray(offA[:-1], np.int64)).to(dev),
+                      torch.from_numpy(np.asarray(offB[:-1], np.int64)).to(dev),
+                      Ap.to(dev), Bt.to(dev), scale, seg_out=seg_out)
+    st = lf.lf_get_device_status()
+    return y.cpu(), (seg_out.cpu().numpy() if seg else None), st
+
+
+def oracle_y(x, y0, ids, ranks, offA, offB, Ap, Bt, scale):
+    return OP.lora_apply(x.float().numpy(), y0.float().numpy(), ids, ranks, offA[:-1], offB[:-1],
+                         Ap.float().numpy(), Bt.float().numpy(), scale)
+
+
+def assert_close(y_gpu, y_orc):
+    d = np.abs(y_gpu.float().numpy().astype(np.float64) - y_orc).max()
+    assert d <= G.APPLY_TOL * max(np.abs(y_orc).max(), 1e-30), (d, np.abs(y_orc).max())
+
+
+def check_routing(seg, ids, n):
+    segs_o, perm_o = OP.route(ids, n)
+    nseg, nval = int(seg[0]), int(seg[1])
+    assert nseg == len(segs_o) and nval == len(perm_o)
+    assert seg[2:2 + 3 * nseg].reshape(-1, 3).tolist() == segs_o.tolist()
+    assert seg[2 + 3 * nseg:2 + 3 * nseg + nval].tolist() == perm_o.tolist()
+
+
+def test_tiny_apply_and_routing():
+    T, n, d, k = 64, 4, 256, 4
+    ids = synth.uniform_ids(T, n, (1, 0))
+    offA, offB, Ap, Bt = make_pools([k] * n, d, d, (1, 1))
+    x = synth.normal_bf16((T, d), (1, 2))
+    y0 = torch.zeros(T, d, dtype=torch.bfloat16)
+    y, seg, st = run_apply(x, y0, ids, [k] * n, offA, offB, Ap, Bt, 2.0, seg=True)
+    assert st == 0
+    assert_close(y, oracle_y(x, y0, ids, [k] * n, offA, offB, Ap, Bt, 2.0))
+    check_routing(seg, ids, n)
+
+
+@pytest.mark.parametrize("d_in,d_out", [(4096, 1024), (1024, 14336), (3584, 512)])
+def test_ragged_ranks_zipf_with_unrouted_tokens(d_in, d_out):
+    T, n = 300, 37
+    g = np.random.default_rng(5)
+    ranks = g.integers(1, 65, size=n)
+    ids = synth.zipf_ids(T, n, 1.0, (2, d_in))
+    ids[g.random(T) < 0.1] = -1
+    offA, offB, Ap, Bt = make_pools(ranks, d_in, d_out, (2, d_out))
+    x = synth.normal_bf16((T, d_in), (2, 3))
+    y0 = synth.normal_bf16((T, d_out), (2, 4))
+    y, seg, st = run_apply(x, y0, ids, ranks, offA, offB, Ap, Bt, 0.5, seg=True)
+    assert st == 0
+    check_routing(seg, ids, n)
+    # unrouted rows are untouched, bit for bit
+    assert torch.equal(y[torch.from_numpy(ids < 0)], y0[torch.from_numpy(ids < 0)])
+    # the LoRA delta itself against the oracle (y0 = 0 measures the delta alone)
+    yz, _, _ = run_apply(x, torch.zeros_like(y0), ids, ranks, offA, offB, Ap, Bt, 0.5)
+    assert_close(yz, oracle_y(x, torch.zeros_like(y0), ids, ranks, offA, offB, Ap, Bt, 0.5))
+
+
+def test_bad_index_latches_error_and_skips_token():
+    T, n, d = 16, 3, 256
+    ids = np.array([0, 1, 2, 5, -3] + [1] * 11, dtype=np.int32)
+    offA, offB, Ap, Bt = make_pools([2, 3, 4], d, d, (3, 0))
+    x = synth.normal_bf16((T, d), (3, 1))
+    y0 = synth.normal_bf16((T, d), (3, 2))
+    y, _, st = run_apply(x, y0, ids, [2, 3, 4], offA, offB, Ap, Bt, 1.0)
+    assert st == 3  # LF_ERR_BAD_INDEX
+    assert torch.equal(y[3], y0[3]) and torch.equal(y[4], y0[4])
+
+
+def test_scale_zero_leaves_y():
+    T, n, d = 40, 5, 512
+    ids = synth.uniform_ids(T, n, (4, 0))
+    offA, offB, Ap, Bt = make_pools([3] * n, d, d, (4, 1))
+    x = synth.normal_bf16((T, d), (4, 2))
+    y0 = synth.normal_bf16((T, d), (4, 3))
+    y, _, st = run_apply(x, y0, ids, [3] * n, offA, offB, Ap, Bt, 0.0)
+    assert st == 0 and torch.equal(y, y0)
+
+
+@pytest.mark.parametrize("k", [16, 64])
+def test_prefill_segments(k):
+    # 4 requests x 512 tokens, request i -> adapter i; Qwen-like widths
+    T, n, d_in, d_out = 2048, 4, 3584, 18944
+    ids = np.repeat(np.arange(n, dtype=np.int32), 512)
+    offA, offB, Ap, Bt = make_pools([k] * n, d_in, d_out, (5, k))
+    x = synth.normal_bf16((T, d_in), (5, 1))
+    y0 = torch.zeros(T, d_out, dtype=torch.bfloat16)
+    y, seg, st = run_apply(x, y0, ids, [k] * n, offA, offB, Ap, Bt, 2.0, seg=True)
+    assert st == 0
+    check_routing(seg, ids, n)
+    assert_close(y, oracle_y(x, y0, ids, [k] * n, offA, offB, Ap, Bt, 2.0))
+
+
+def test_empty_batch_and_all_unrouted():
+    d = 256
+    offA, offB, Ap, Bt = make_pools([2], d, d, (6, 0))
+    x = synth.normal_bf16((8, d), (6, 1)); y0 = synth.normal_bf16((8, d), (6, 2))
+    y, seg, st = run_apply(x, y0, [-1] * 8, [2], offA, offB, Ap, Bt, 1.0, seg=True)
+    assert st == 0 and torch.equal(y, y0) and seg[0] == 0 and seg[1] == 0
+    y, _, st = run_apply(x[:0], y0[:0], [], [2], offA, offB, Ap, Bt, 1.0)
+    assert st == 0 and y.shape == (0, d)
