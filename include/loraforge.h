@@ -107,6 +107,7 @@ lf_status lf_tsqr_batched(const lf_module* mods /*[host]*/, int32_t n,
 /* ---- Rank allocation alone (LoRAForge-U / -S) --------------------------------
  * ranks[i] from sigma (n x rs fp64, rows descending) under `pol`; off_A / off_Bt
  * are n+1 prefix sums of ranks[i]*d_in and ranks[i]*d_out (pool element offsets).
+ * A row that is not in descending order latches LF_ERR_INVALID_ARG on the device.
  * Workspace: lf_select_workspace_size(mods, n). */
 size_t lf_select_workspace_size(const lf_module* mods /*[host]*/, int32_t n);
 lf_status lf_select_ranks(const lf_module* mods /*[host]*/, int32_t n, lf_policy pol,
@@ -169,6 +170,23 @@ lf_status lf_lora_shrink_expand(int32_t T, int32_t d_in, int32_t d_out,
                                 int64_t pool_elems_A, int64_t pool_elems_Bt, float scale,
                                 int32_t* seg_out, void* ws, size_t ws_bytes,
                                 lf_stream_t stream);
+
+/* ---- Tracing (no counterpart on the pages: measurement support) --------------
+ * Every kernel launch of the library is counted.  With timing enabled, each
+ * launch is also bracketed by CUDA events recorded on its own stream and its
+ * device time is added to a named phase ("tsqr_leaf_merge", "svd_jacobi",
+ * "select", "export_stream", "shrink_expand_gemv", ...).  lf_profile_read waits
+ * for the pending events, then copies up to max_phases entries into `out`
+ * [host] and returns the number of phases.  Process-wide state, not thread-safe. */
+typedef struct {
+    char name[32];
+    double total_ms;
+    int64_t launches;
+} lf_phase_time;
+void lf_profile_enable(int on);
+void lf_profile_reset(void);
+int32_t lf_profile_read(lf_phase_time* out /*[host]*/, int32_t max_phases);
+int64_t lf_launch_count(void);
 
 /* ---- Status ------------------------------------------------------------------ */
 const char* lf_status_string(lf_status s);

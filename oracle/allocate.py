@@ -71,6 +71,8 @@ def spectral_ranks(sigma_rows, r, group, num: int, den: int, floor: int):
             ri = int(r[i])
             if floor > ri:
                 raise ValueError("floor exceeds module rank")
+            if np.any(np.diff(sigma_rows[i][:ri]) > 0):
+                raise ValueError("singular values must be listed in descending order")
             e = energies(sigma_rows[i], ri)
             for j in range(floor, ri):
                 if e[j] > 0.0:

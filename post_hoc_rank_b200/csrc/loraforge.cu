@@ -5,6 +5,7 @@
 #include <climits>
 #include <cstring>
 #include <map>
+#include <string>
 #include <vector>
 
 #include "common.cuh"
@@ -13,6 +14,69 @@
 #include "apply.cuh"
 
 namespace lf {
+
+// ------------------------------------------------------------- tracing/timing
+// Every kernel launch goes through LF_LAUNCH, which counts it and, when timing is
+// on, brackets it with CUDA events recorded on the launching stream.
+struct ProfState {
+    bool on = false;
+    int64_t launches = 0;
+    struct Rec {
+        int phase;
+        cudaEvent_t a, b;
+    };
+    std::vector<Rec> pending;
+    std::vector<cudaEvent_t> free_events;
+    std::vector<std::string> names;
+    std::vector<double> ms;
+    std::vector<int64_t> count;
+};
+static ProfState g_prof;
+
+static int phase_id(const char* name) {
+    for (size_t i = 0; i < g_prof.names.size(); ++i)
+        if (g_prof.names[i] == name) return (int)i;
+    g_prof.names.push_back(name);
+    g_prof.ms.push_back(0.0);
+    g_prof.count.push_back(0);
+    return (int)g_prof.names.size() - 1;
+}
+
+static cudaEvent_t take_event() {
+    if (!g_prof.free_events.empty()) {
+        cudaEvent_t e = g_prof.free_events.back();
+        g_prof.free_events.pop_back();
+        return e;
+    }
+    cudaEvent_t e = nullptr;
+    cudaEventCreate(&e);
+    return e;
+}
+
+struct PhaseScope {
+    int phase = -1;
+    cudaEvent_t a = nullptr;
+    cudaStream_t s;
+    PhaseScope(const char* name, cudaStream_t st) : s(st) {
+        ++g_prof.launches;
+        if (!g_prof.on) return;
+        phase = phase_id(name);
+        a = take_event();
+        cudaEventRecord(a, s);
+    }
+    ~PhaseScope() {
+        if (phase < 0) return;
+        cudaEvent_t b = take_event();
+        cudaEventRecord(b, s);
+        g_prof.pending.push_back(ProfState::Rec{phase, a, b});
+    }
+};
+
+#define LF_LAUNCH(name, kernel, grid, block, smem, stream, ...)            \
+    do {                                                                   \
+        PhaseScope ps_(name, stream);                                      \
+        kernel<<<grid, block, smem, stream>>>(__VA_ARGS__);                \
+    } while (0)
 
 // ----------------------------------------------------------------- validation
 static lf_status check_mods(const lf_module* mods, int32_t n) {
@@ -116,7 +180,7 @@ static cudaError_t launch_tsqr(const TsqrArgs<T>& a, int grid, cudaStream_t st) 
     auto k = tsqr_kernel<T, RT, kTsqrTM, kTsqrThreads>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    if (grid > 0) k<<<grid, kTsqrThreads, smem, st>>>(a);
+    if (grid > 0) LF_LAUNCH(sizeof(T) == 8 ? "tsqr_fp64_refine" : "tsqr_leaf_merge", k, grid, kTsqrThreads, smem, st, a);
     return cudaGetLastError();
 }
 
@@ -133,7 +197,7 @@ static cudaError_t launch_svd(const SvdArgs<TIN>& a, int grid, cudaStream_t st) 
     auto k = svd_kernel<TIN, RT>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    if (grid > 0) k<<<grid, kSvdThreads, smem, st>>>(a);
+    if (grid > 0) LF_LAUNCH(sizeof(TIN) == 8 ? "svd_fp64_refine" : "svd_jacobi", k, grid, kSvdThreads, smem, st, a);
     return cudaGetLastError();
 }
 
@@ -354,9 +418,9 @@ lf_status lf_select_ranks(const lf_module* mods, int32_t n, lf_policy pol, const
     a.flag_list = nullptr;
     a.flag_count = nullptr;
     const int ng = (int)p.gptr.size() - 1;
-    select_kernel<<<ng, kSelThreads, 0, s>>>(a);
+    LF_LAUNCH("select", select_kernel, ng, kSelThreads, 0, s, a);
     LF_CUDA_TRY(cudaGetLastError());
-    offsets_kernel<<<1, 1024, 0, s>>>(a.mods, n, ranks, off_A, off_Bt, INT64_MAX, INT64_MAX);
+    LF_LAUNCH("offsets", offsets_kernel, 1, 1024, 0, s, a.mods, n, ranks, off_A, off_Bt, INT64_MAX, INT64_MAX);
     return launch_status();
 }
 
@@ -462,14 +526,14 @@ lf_status lf_truncate_export(const lf_module* mods, int32_t n, lf_policy pol, co
         LF_CUDA_TRY(cudaMemsetAsync(fcount, 0, 2 * sizeof(int32_t), s));
         a.flag_list = flist;
         a.flag_count = fcount;
-        select_kernel<<<ng, kSelThreads, 0, s>>>(a);
+        LF_LAUNCH("select", select_kernel, ng, kSelThreads, 0, s, a);
         LF_CUDA_TRY(cudaGetLastError());
-        cap_flags_kernel<<<1, 32, 0, s>>>(fcount, p.refine_cap);
+        LF_LAUNCH("refine_plan", cap_flags_kernel, 1, 32, 0, s, fcount, p.refine_cap);
         LF_CUDA_TRY(cudaGetLastError());
         TsqrWork* rwork = reinterpret_cast<TsqrWork*>(base + L.rwork);
         int32_t* rnwork = reinterpret_cast<int32_t*>(base + L.rnwork);
         TsqrInfo* rinfo = reinterpret_cast<TsqrInfo*>(base + L.rinfo);
-        refine_plan_kernel<<<1, 32, 0, s>>>(dmods, flist, fcount, rwork, rnwork, rinfo, kRefineChunk);
+        LF_LAUNCH("refine_plan", refine_plan_kernel, 1, 32, 0, s, dmods, flist, fcount, rwork, rnwork, rinfo, kRefineChunk);
         LF_CUDA_TRY(cudaGetLastError());
         LF_CUDA_TRY(cudaMemsetAsync(base + L.rcnt, 0, (size_t)2 * p.refine_cap * sizeof(int32_t), s));
         TsqrArgs<double> ta;
@@ -500,19 +564,19 @@ lf_status lf_truncate_export(const lf_module* mods, int32_t n, lf_policy pol, co
         LF_CUDA_TRY(launch_svd_rt<double>(p.RT, sa, p.refine_cap, s));
         double* sigref = reinterpret_cast<double*>(base + L.sigref);
         LF_CUDA_TRY(cudaMemcpyAsync(sigref, sigma, (size_t)n * p.rs * sizeof(double), cudaMemcpyDeviceToDevice, s));
-        scatter_sigma_kernel<<<p.refine_cap, 64, 0, s>>>(flist, fcount + 1, sa.sigma, sigref, p.rs);
+        LF_LAUNCH("refine_plan", scatter_sigma_kernel, p.refine_cap, 64, 0, s, flist, fcount + 1, sa.sigma, sigref, p.rs);
         LF_CUDA_TRY(cudaGetLastError());
         a.sigma = sigref;
         a.flag_list = nullptr;
         a.flag_count = nullptr;
     }
-    select_kernel<<<ng, kSelThreads, 0, s>>>(a);
+    LF_LAUNCH("select", select_kernel, ng, kSelThreads, 0, s, a);
     LF_CUDA_TRY(cudaGetLastError());
-    offsets_kernel<<<1, 1024, 0, s>>>(dmods, n, ranks, off_A, off_Bt, pool_cap_A, pool_cap_Bt);
+    LF_LAUNCH("offsets", offsets_kernel, 1, 1024, 0, s, dmods, n, ranks, off_A, off_Bt, pool_cap_A, pool_cap_Bt);
     LF_CUDA_TRY(cudaGetLastError());
     float* CA = reinterpret_cast<float*>(base + L.CA);
     float* CB = reinterpret_cast<float*>(base + L.CB);
-    export_coef_kernel<<<n, 128, 0, s>>>(dmods, ranks, R_B, R_A, sigma, U, V, p.rs, CA, CB);
+    LF_LAUNCH("export_coef", export_coef_kernel, n, 128, 0, s, dmods, ranks, R_B, R_A, sigma, U, V, p.rs, CA, CB);
     LF_CUDA_TRY(cudaGetLastError());
     ExportArgs ea;
     ea.mods = dmods;
@@ -532,7 +596,7 @@ lf_status lf_truncate_export(const lf_module* mods, int32_t n, lf_policy pol, co
     ea.cap_A = pool_cap_A;
     ea.cap_Bt = pool_cap_Bt;
     LF_CUDA_TRY(cudaFuncSetAttribute(export_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kExportSmem));
-    export_kernel<<<(int)p.ework.size(), kExpThreads, kExportSmem, s>>>(ea);
+    LF_LAUNCH("export_stream", export_kernel, (int)p.ework.size(), kExpThreads, kExportSmem, s, ea);
     return launch_status();
 }
 
@@ -572,7 +636,7 @@ lf_status lf_lora_shrink_expand(int32_t T, int32_t d_in, int32_t d_out, const vo
     o.seg_out = seg_out;
     const size_t rsmem = (size_t)n_adapters * sizeof(int32_t);
     LF_CUDA_TRY(cudaFuncSetAttribute(route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rsmem));
-    route_kernel<<<1, kRouteThreads, rsmem, s>>>(ids, T, n_adapters, o);
+    LF_LAUNCH("route", route_kernel, 1, kRouteThreads, rsmem, s, ids, T, n_adapters, o);
     LF_CUDA_TRY(cudaGetLastError());
     GemvArgs g;
     g.d_in = d_in;
@@ -592,9 +656,44 @@ lf_status lf_lora_shrink_expand(int32_t T, int32_t d_in, int32_t d_out, const vo
     g.perm = o.perm;
     g.items = o.items;
     dim3 grid((unsigned)(T / kGemvTok + mseg + 1), (unsigned)cdiv(d_out, kGemvCols));
-    gemv_kernel<<<grid, kGemvThreads, 0, s>>>(g);
+    LF_LAUNCH("shrink_expand_gemv", gemv_kernel, grid, kGemvThreads, 0, s, g);
     return launch_status();
 }
+
+void lf_profile_enable(int on) { g_prof.on = on != 0; }
+
+void lf_profile_reset(void) {
+    for (auto& r : g_prof.pending) {
+        g_prof.free_events.push_back(r.a);
+        g_prof.free_events.push_back(r.b);
+    }
+    g_prof.pending.clear();
+    std::fill(g_prof.ms.begin(), g_prof.ms.end(), 0.0);
+    std::fill(g_prof.count.begin(), g_prof.count.end(), 0);
+}
+
+int32_t lf_profile_read(lf_phase_time* out, int32_t max_phases) {
+    for (auto& r : g_prof.pending) {
+        float t = 0.f;
+        if (cudaEventSynchronize(r.b) == cudaSuccess && cudaEventElapsedTime(&t, r.a, r.b) == cudaSuccess) {
+            g_prof.ms[r.phase] += t;
+            g_prof.count[r.phase] += 1;
+        }
+        g_prof.free_events.push_back(r.a);
+        g_prof.free_events.push_back(r.b);
+    }
+    g_prof.pending.clear();
+    const int32_t np = (int32_t)g_prof.names.size();
+    for (int32_t i = 0; i < np && out && i < max_phases; ++i) {
+        std::memset(out[i].name, 0, sizeof(out[i].name));
+        std::strncpy(out[i].name, g_prof.names[i].c_str(), sizeof(out[i].name) - 1);
+        out[i].total_ms = g_prof.ms[i];
+        out[i].launches = g_prof.count[i];
+    }
+    return np;
+}
+
+int64_t lf_launch_count(void) { return g_prof.launches; }
 
 const char* lf_status_string(lf_status s) {
     switch (s) {

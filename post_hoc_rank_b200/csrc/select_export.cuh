@@ -93,6 +93,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelArgs a) {
         for (int j = 0; j < r; ++j) {
             const double sq = sg[j] * sg[j];
             tot += sq;
+            if (j + 1 < r && sg[j + 1] > sg[j]) latch_error(LF_ERR_INVALID_ARG);  // rows must descend
         }
         if (!isfinite(tot)) latch_error(LF_ERR_NUMERIC);
         double* en = a.energy + (size_t)i * a.rs;

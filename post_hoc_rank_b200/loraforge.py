@@ -39,6 +39,10 @@ def policy_S(num: int, den: int, floor: int = 1) -> lf_policy:
     return lf_policy(1, num, den, floor)
 
 
+class lf_phase_time(ctypes.Structure):
+    _fields_ = [("name", ctypes.c_char * 32), ("total_ms", ctypes.c_double), ("launches", ctypes.c_int64)]
+
+
 class LFError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
@@ -78,6 +82,10 @@ def lib() -> ctypes.CDLL:
         L.lf_lora_shrink_expand.restype = ctypes.c_int
         L.lf_status_string.argtypes = [ctypes.c_int]; L.lf_status_string.restype = ctypes.c_char_p
         L.lf_get_device_status.argtypes = [_P]; L.lf_get_device_status.restype = ctypes.c_int
+        L.lf_profile_enable.argtypes = [ctypes.c_int]; L.lf_profile_enable.restype = None
+        L.lf_profile_reset.argtypes = []; L.lf_profile_reset.restype = None
+        L.lf_profile_read.argtypes = [_P, _I32]; L.lf_profile_read.restype = _I32
+        L.lf_launch_count.argtypes = []; L.lf_launch_count.restype = _I64
         _lib = L
     return _lib
 
@@ -85,7 +93,8 @@ def lib() -> ctypes.CDLL:
 def exported_symbols() -> list[str]:
     return ["lf_rank_stride", "lf_tsqr_workspace_size", "lf_tsqr_batched", "lf_select_workspace_size",
             "lf_select_ranks", "lf_export_workspace_size", "lf_export_pool_bound", "lf_truncate_export",
-            "lf_apply_workspace_size", "lf_lora_shrink_expand", "lf_status_string", "lf_get_device_status"]
+            "lf_apply_workspace_size", "lf_lora_shrink_expand", "lf_status_string", "lf_get_device_status",
+            "lf_profile_enable", "lf_profile_reset", "lf_profile_read", "lf_launch_count"]
 
 
 def _ptr(t) -> int | None:
@@ -192,3 +201,22 @@ def lf_status_string(st: int) -> str:
 
 def lf_get_device_status(stream=None) -> int:
     return lib().lf_get_device_status(_stream(stream))
+
+
+def lf_profile_enable(on: bool) -> None:
+    lib().lf_profile_enable(1 if on else 0)
+
+
+def lf_profile_reset() -> None:
+    lib().lf_profile_reset()
+
+
+def lf_profile_read() -> dict[str, tuple[float, int]]:
+    """{phase: (total device ms, launches)} accumulated since the last reset."""
+    buf = (lf_phase_time * 64)()
+    n = lib().lf_profile_read(ctypes.addressof(buf), 64)
+    return {buf[i].name.decode(): (buf[i].total_ms, buf[i].launches) for i in range(min(n, 64))}
+
+
+def lf_launch_count() -> int:
+    return lib().lf_launch_count()

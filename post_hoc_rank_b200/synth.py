@@ -203,14 +203,15 @@ def tiny_fleet(seed_cfg: int = 0):
 
 def sigma_tables(n_adapters: int, model: ModelShape, r: int, cfg_id: int) -> np.ndarray:
     """Synthetic fp64 singular-value tables, one row of r per module, laid out in
-    fleet_layout's (adapter, projection, layer) order, sigma_j = (j+1)^-1 e^{0.5 z}."""
+    fleet_layout's (adapter, projection, layer) order: the values
+    (j+1)^-1 e^{0.5 z_j}, listed in descending order as singular values are."""
     rows = []
     for a in range(n_adapters):
         rng = np.random.Generator(np.random.Philox(derive_seed(cfg_id, a, 99)))
         for _p in range(7):
             for _l in range(model.layers):
-                rows.append(sigma_profile(rng.standard_normal, r, True))
-    return np.stack(rows)
+                rows.append(np.sort(sigma_profile(rng.standard_normal, r, True))[::-1])
+    return np.ascontiguousarray(np.stack(rows))
 
 
 def zipf_ids(T: int, n: int, alpha: float, key: tuple[int, ...]) -> np.ndarray:

@@ -74,3 +74,8 @@ def test_prefix_closed_with_ties():
     for num in range(1, 6):
         ranks, _ = AL.spectral_ranks(sig, [5], [0], num, 5, 1)
         assert ranks[0] == max(1, num)
+
+
+def test_rejects_unsorted_sigma():
+    with pytest.raises(ValueError):
+        AL.spectral_ranks(np.array([[1.0, 2.0, 0.5]]), [3], [0], 1, 2, 1)
