@@ -171,6 +171,37 @@ lf_status lf_lora_shrink_expand(int32_t T, int32_t d_in, int32_t d_out,
                                 int32_t* seg_out, void* ws, size_t ws_bytes,
                                 lf_stream_t stream);
 
+/* ---- Shrink / expand with library-owned scratch -------------------------------
+ * This entry point has no counterpart in the paper; it exists for callers that
+ * cannot call cudaMalloc.  Examples: a serving loop that reserved all device memory
+ * when it started and may not allocate afterwards, or a latency-critical path where
+ * cudaMalloc's implicit synchronisation and unbounded cost are not acceptable.
+ * Such a caller still passes x, y, ids, the rank table and the pools, but no
+ * workspace: the routing scratch lives in a fixed array inside the library
+ * (a file-scope __device__ array sized for LF_NOALLOC_MAX_TOKENS tokens and
+ * LF_NOALLOC_MAX_ADAPTERS adapters, 213 504 bytes, held on every GPU that loads the
+ * library until the process exits).
+ *  - Same arguments, results and device-side errors as lf_lora_shrink_expand, minus
+ *    the workspace.  T > LF_NOALLOC_MAX_TOKENS or n_adapters > LF_NOALLOC_MAX_ADAPTERS
+ *    returns LF_ERR_WORKSPACE without launching anything.
+ *  - Runs on the device that is current when it is called; `stream` must belong
+ *    to that device.  The first call on each device looks up the array's device
+ *    address (cudaGetSymbolAddress); make that first call before any stream capture.
+ *  - Allocates nothing: no cudaMalloc, cudaFree or allocating library routine.
+ *  - All calls on one device share the one array and every call overwrites what it
+ *    reads before reading it (nothing in it has to start at zero).  Two calls whose
+ *    work overlaps on the GPU (for instance on two streams) race on the array and
+ *    give wrong results: serialise them, e.g. on one stream. */
+#define LF_NOALLOC_MAX_TOKENS 16384
+#define LF_NOALLOC_MAX_ADAPTERS 4096
+lf_status lf_lora_shrink_expand_noalloc(int32_t T, int32_t d_in, int32_t d_out,
+                                        const void* x, void* y, const int32_t* ids,
+                                        int32_t n_adapters, const int32_t* ranks,
+                                        const int64_t* off_A, const int64_t* off_Bt,
+                                        const void* A_pool, const void* Bt_pool,
+                                        int64_t pool_elems_A, int64_t pool_elems_Bt,
+                                        float scale, int32_t* seg_out, lf_stream_t stream);
+
 /* ---- Tracing (no counterpart on the pages: measurement support) --------------
  * Every kernel launch of the library is counted.  With timing enabled, each
  * launch is also bracketed by CUDA events recorded on its own stream and its

@@ -5,6 +5,7 @@
 #include <climits>
 #include <cstring>
 #include <map>
+#include <mutex>
 #include <string>
 #include <vector>
 
@@ -301,6 +302,37 @@ __global__ void cap_flags_kernel(int32_t* count, int cap) {
         count[0] = c;
         count[1] = c;
     }
+}
+
+// ------------------------------------------------- library-owned apply scratch
+// Routing scratch for lf_lora_shrink_expand_noalloc, laid out exactly as the
+// Carver lays out a caller workspace for (LF_NOALLOC_MAX_TOKENS, LF_NOALLOC_MAX_ADAPTERS).
+constexpr size_t al256(size_t x) { return (x + 255) / 256 * 256; }
+constexpr size_t kNoallocScratchBytes =
+    al256(4 * sizeof(int32_t)) + al256((size_t)LF_NOALLOC_MAX_ADAPTERS * sizeof(Seg)) +
+    al256((size_t)LF_NOALLOC_MAX_TOKENS * sizeof(int32_t)) +
+    al256(((size_t)LF_NOALLOC_MAX_TOKENS / kGemvTok + LF_NOALLOC_MAX_ADAPTERS + 1) * sizeof(GemvItem));
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocScratchBytes];
+
+// In host code g_noalloc_scratch is only a host-side stand-in for the device array;
+// its device address is looked up once per device (with that device current) and
+// cached here.
+constexpr int kMaxDevices = 64;
+static std::mutex g_noalloc_mu;
+static void* g_noalloc_addr[kMaxDevices] = {};
+
+static lf_status noalloc_scratch(void** out) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return LF_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return LF_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_addr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return LF_ERR_CUDA;
+        g_noalloc_addr[dev] = p;
+    }
+    *out = g_noalloc_addr[dev];
+    return LF_OK;
 }
 
 }  // namespace lf
@@ -634,6 +666,58 @@ lf_status lf_lora_shrink_expand(int32_t T, int32_t d_in, int32_t d_out, const vo
     o.perm = c.take<int32_t>((size_t)T);
     o.items = c.take<GemvItem>((size_t)(T / kGemvTok + mseg + 1));
     o.seg_out = seg_out;
+    const size_t rsmem = (size_t)n_adapters * sizeof(int32_t);
+    LF_CUDA_TRY(cudaFuncSetAttribute(route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rsmem));
+    LF_LAUNCH("route", route_kernel, 1, kRouteThreads, rsmem, s, ids, T, n_adapters, o);
+    LF_CUDA_TRY(cudaGetLastError());
+    GemvArgs g;
+    g.d_in = d_in;
+    g.d_out = d_out;
+    g.x = reinterpret_cast<const __nv_bfloat16*>(x);
+    g.y = reinterpret_cast<__nv_bfloat16*>(y);
+    g.ranks = ranks;
+    g.off_A = off_A;
+    g.off_Bt = off_Bt;
+    g.A_pool = reinterpret_cast<const __nv_bfloat16*>(A_pool);
+    g.Bt_pool = reinterpret_cast<const __nv_bfloat16*>(Bt_pool);
+    g.pool_A = pool_elems_A;
+    g.pool_Bt = pool_elems_Bt;
+    g.scale = scale;
+    g.counts = o.counts;
+    g.segs = o.segs;
+    g.perm = o.perm;
+    g.items = o.items;
+    dim3 grid((unsigned)(T / kGemvTok + mseg + 1), (unsigned)cdiv(d_out, kGemvCols));
+    LF_LAUNCH("shrink_expand_gemv", gemv_kernel, grid, kGemvThreads, 0, s, g);
+    return launch_status();
+}
+
+lf_status lf_lora_shrink_expand_noalloc(int32_t T, int32_t d_in, int32_t d_out, const void* x, void* y,
+                                        const int32_t* ids, int32_t n_adapters, const int32_t* ranks,
+                                        const int64_t* off_A, const int64_t* off_Bt, const void* A_pool,
+                                        const void* Bt_pool, int64_t pool_elems_A, int64_t pool_elems_Bt,
+                                        float scale, int32_t* seg_out, lf_stream_t stream) {
+    if (T < 0 || d_in < 1 || d_out < 1 || n_adapters < 1 || pool_elems_A < 0 || pool_elems_Bt < 0)
+        return LF_ERR_INVALID_ARG;
+    if (T > LF_NOALLOC_MAX_TOKENS || n_adapters > LF_NOALLOC_MAX_ADAPTERS) return LF_ERR_WORKSPACE;
+    if (T == 0) return LF_OK;
+    if (!x || !y || !ids || !ranks || !off_A || !off_Bt || !A_pool || !Bt_pool) return LF_ERR_INVALID_ARG;
+    if ((d_in & 7) || (d_out & 7)) return LF_ERR_ALIGNMENT;
+    if (!aligned16(x) || !aligned16(y) || !aligned16(A_pool) || !aligned16(Bt_pool)) return LF_ERR_ALIGNMENT;
+    void* scratch = nullptr;
+    lf_status st = noalloc_scratch(&scratch);
+    if (st != LF_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    // same carve as a caller workspace sized for the maxima (fits kNoallocScratchBytes)
+    Carver c(scratch);
+    RouteOut o;
+    o.counts = c.take<int32_t>(4);
+    o.segs = c.take<Seg>((size_t)LF_NOALLOC_MAX_ADAPTERS);
+    o.perm = c.take<int32_t>((size_t)LF_NOALLOC_MAX_TOKENS);
+    o.items = c.take<GemvItem>((size_t)LF_NOALLOC_MAX_TOKENS / kGemvTok + LF_NOALLOC_MAX_ADAPTERS + 1);
+    o.seg_out = seg_out;
+    if (c.off > kNoallocScratchBytes) return LF_ERR_WORKSPACE;
+    const int64_t mseg = std::min<int64_t>(T, n_adapters);
     const size_t rsmem = (size_t)n_adapters * sizeof(int32_t);
     LF_CUDA_TRY(cudaFuncSetAttribute(route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rsmem));
     LF_LAUNCH("route", route_kernel, 1, kRouteThreads, rsmem, s, ids, T, n_adapters, o);

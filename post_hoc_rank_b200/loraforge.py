@@ -80,6 +80,9 @@ def lib() -> ctypes.CDLL:
         L.lf_lora_shrink_expand.argtypes = [_I32, _I32, _I32, _P, _P, _P, _I32, _P, _P, _P, _P, _P,
                                             _I64, _I64, ctypes.c_float, _P, _P, _SZ, _P]
         L.lf_lora_shrink_expand.restype = ctypes.c_int
+        L.lf_lora_shrink_expand_noalloc.argtypes = [_I32, _I32, _I32, _P, _P, _P, _I32, _P, _P, _P, _P, _P,
+                                                    _I64, _I64, ctypes.c_float, _P, _P]
+        L.lf_lora_shrink_expand_noalloc.restype = ctypes.c_int
         L.lf_status_string.argtypes = [ctypes.c_int]; L.lf_status_string.restype = ctypes.c_char_p
         L.lf_get_device_status.argtypes = [_P]; L.lf_get_device_status.restype = ctypes.c_int
         L.lf_profile_enable.argtypes = [ctypes.c_int]; L.lf_profile_enable.restype = None
@@ -94,7 +97,12 @@ def exported_symbols() -> list[str]:
     return ["lf_rank_stride", "lf_tsqr_workspace_size", "lf_tsqr_batched", "lf_select_workspace_size",
             "lf_select_ranks", "lf_export_workspace_size", "lf_export_pool_bound", "lf_truncate_export",
             "lf_apply_workspace_size", "lf_lora_shrink_expand", "lf_status_string", "lf_get_device_status",
-            "lf_profile_enable", "lf_profile_reset", "lf_profile_read", "lf_launch_count"]
+            "lf_profile_enable", "lf_profile_reset", "lf_profile_read", "lf_launch_count",
+            "lf_lora_shrink_expand_noalloc"]
+
+# Limits of lf_lora_shrink_expand_noalloc (its scratch is a fixed array in the library).
+NOALLOC_MAX_TOKENS = 16384
+NOALLOC_MAX_ADAPTERS = 4096
 
 
 def _ptr(t) -> int | None:
@@ -193,6 +201,19 @@ def lf_lora_shrink_expand(x, y, ids, n_adapters, ranks, off_A, off_Bt, A_pool, B
                                      _ptr(seg_out), _ptr(ws), ws.numel() if ws is not None else 0,
                                      _stream(stream))
     return _check(st, "lf_lora_shrink_expand") if check else st
+
+
+def lf_lora_shrink_expand_noalloc(x, y, ids, n_adapters, ranks, off_A, off_Bt, A_pool, Bt_pool, scale,
+                                  seg_out=None, stream=None, check=True) -> int:
+    """lf_lora_shrink_expand without a workspace argument, for callers that cannot
+    allocate device memory; the library keeps the routing scratch itself."""
+    T, d_in = x.shape
+    d_out = y.shape[1]
+    st = lib().lf_lora_shrink_expand_noalloc(T, d_in, d_out, _ptr(x), _ptr(y), _ptr(ids), n_adapters,
+                                             _ptr(ranks), _ptr(off_A), _ptr(off_Bt), _ptr(A_pool), _ptr(Bt_pool),
+                                             A_pool.numel(), Bt_pool.numel(), float(scale), _ptr(seg_out),
+                                             _stream(stream))
+    return _check(st, "lf_lora_shrink_expand_noalloc") if check else st
 
 
 def lf_status_string(st: int) -> str:
