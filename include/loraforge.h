@@ -179,7 +179,7 @@ lf_status lf_lora_shrink_expand(int32_t T, int32_t d_in, int32_t d_out,
  * Such a caller still passes x, y, ids, the rank table and the pools, but no
  * workspace: the routing scratch lives in a fixed array inside the library
  * (a file-scope __device__ array sized for LF_NOALLOC_MAX_TOKENS tokens and
- * LF_NOALLOC_MAX_ADAPTERS adapters, 213 504 bytes, held on every GPU that loads the
+ * LF_NOALLOC_MAX_ADAPTERS adapters, 4 407 808 bytes, held on every GPU that loads the
  * library until the process exits).
  *  - Same arguments, results and device-side errors as lf_lora_shrink_expand, minus
  *    the workspace.  T > LF_NOALLOC_MAX_TOKENS or n_adapters > LF_NOALLOC_MAX_ADAPTERS

@@ -33,48 +33,89 @@ struct RouteOut {
     int32_t* seg_out;    // optional caller copy
 };
 
-// One CTA: counting sort of token ids (stable), segments and GEMV work items.
-// Shared memory: n_adapters ints (counts, then running positions).
+// Block-wide exclusive scan of one int per thread (blockDim.x == kRouteThreads).
+__device__ __forceinline__ int block_excl_scan(int v, int* wsum, int* total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) wsum[warp] = x;
+    __syncthreads();
+    if (warp == 0) {
+        int w = wsum[lane];
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, w, o);
+            if (lane >= o) w += y;
+        }
+        wsum[lane] = w;   // inclusive over warps
+    }
+    __syncthreads();
+    const int base = warp > 0 ? wsum[warp - 1] : 0;
+    const int tot = wsum[31];
+    __syncthreads();
+    if (total) *total = tot;
+    return base + x - v;
+}
+
+// One CTA: stable counting sort of token ids into segments (adapter, start, len),
+// the token permutation, and GEMV work items of <= kGemvTok tokens.
+// Shared memory: 2 * n_adapters ints.
 __global__ void __launch_bounds__(kRouteThreads) route_kernel(const int32_t* __restrict__ ids, int T,
                                                               int n_adapters, RouteOut o) {
     extern __shared__ int32_t rsm[];
-    int32_t* pos = rsm;                         // n_adapters
+    int32_t* cnt = rsm;                  // n_adapters: counts, then running positions
+    int32_t* segidx = rsm + n_adapters;  // n_adapters: segment index of each adapter
     __shared__ int32_t wbase[32][32];
-    __shared__ int32_t s_tot[3];
+    __shared__ int wsum[32];
+    __shared__ int s_carry[3];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    for (int a = tid; a < n_adapters; a += kRouteThreads) pos[a] = 0;
+    for (int a = tid; a < n_adapters; a += kRouteThreads) cnt[a] = 0;
     __syncthreads();
     for (int t = tid; t < T; t += kRouteThreads) {
         const int a = ids[t];
-        if (a < -1 || a >= n_adapters) {
-            latch_error(LF_ERR_BAD_INDEX);
-        } else if (a >= 0) {
-            atomicAdd(&pos[a], 1);
-        }
+        if (a < -1 || a >= n_adapters) latch_error(LF_ERR_BAD_INDEX);
+        else if (a >= 0) atomicAdd(&cnt[a], 1);
     }
+    if (tid == 0) s_carry[0] = s_carry[1] = s_carry[2] = 0;
     __syncthreads();
-    // serial scan over adapters by thread 0 (n_adapters is small); emits segments/items
-    if (tid == 0) {
-        int run = 0, nseg = 0, nitem = 0;
-        for (int a = 0; a < n_adapters; ++a) {
-            const int c = pos[a];
-            pos[a] = run;
+    // scans over adapters in chunks of kRouteThreads: token start, segment index, item index
+    for (int a0 = 0; a0 < n_adapters; a0 += kRouteThreads) {
+        const int a = a0 + tid;
+        const int c = a < n_adapters ? cnt[a] : 0;
+        const int ni = (c + kGemvTok - 1) / kGemvTok;
+        int tt, ts, ti;
+        const int start = block_excl_scan(c, wsum, &tt) + s_carry[0];
+        const int sidx = block_excl_scan(c > 0 ? 1 : 0, wsum, &ts) + s_carry[1];
+        const int iidx = block_excl_scan(ni, wsum, &ti) + s_carry[2];
+        if (a < n_adapters) {
+            cnt[a] = start;
+            segidx[a] = sidx;
             if (c > 0) {
-                o.segs[nseg] = Seg{a, run, c};
-                for (int q = 0; q < c; q += kGemvTok) o.items[nitem++] = GemvItem{nseg, q, min(kGemvTok, c - q), 0};
-                ++nseg;
+                o.segs[sidx] = Seg{a, start, c};
+                for (int q = 0; q < ni; ++q)
+                    o.items[iidx + q] = GemvItem{sidx, q * kGemvTok, min(kGemvTok, c - q * kGemvTok), 0};
             }
-            run += c;
         }
-        s_tot[0] = nseg;
-        s_tot[1] = run;
-        s_tot[2] = nitem;
-        o.counts[0] = nseg;
-        o.counts[1] = run;
-        o.counts[2] = nitem;
+        __syncthreads();
+        if (tid == 0) {
+            s_carry[0] += tt;
+            s_carry[1] += ts;
+            s_carry[2] += ti;
+        }
+        __syncthreads();
     }
-    __syncthreads();
+    const int nval = s_carry[0], nseg = s_carry[1];
+    if (tid == 0) {
+        o.counts[0] = nseg;
+        o.counts[1] = nval;
+        o.counts[2] = s_carry[2];
+    }
     // stable scatter, chunk by chunk; warps take their turn in token order
+    const int nwarps_live = min(kRouteThreads / 32, (T + 31) / 32);
     for (int base = 0; base < T; base += kRouteThreads) {
         const int t = base + tid;
         int a = t < T ? ids[t] : -1;
@@ -82,10 +123,10 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const int32_t* __r
         const unsigned peers = __match_any_sync(0xffffffffu, a);
         const int leader = __ffs(peers) - 1;
         const int rank = __popc(peers & ((1u << lane) - 1u));
-        for (int w = 0; w < kRouteThreads / 32; ++w) {
+        for (int w = 0; w < nwarps_live; ++w) {
             if (warp == w && a >= 0 && lane == leader) {
-                wbase[warp][lane] = pos[a];
-                pos[a] += __popc(peers);
+                wbase[warp][lane] = cnt[a];
+                cnt[a] += __popc(peers);
             }
             __syncthreads();
         }
@@ -93,8 +134,6 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const int32_t* __r
         __syncthreads();
     }
     if (o.seg_out) {
-        __syncthreads();
-        const int nseg = s_tot[0], nval = s_tot[1];
         if (tid == 0) {
             o.seg_out[0] = nseg;
             o.seg_out[1] = nval;
@@ -123,6 +162,7 @@ struct GemvArgs {
     const Seg* segs;
     const int32_t* perm;
     const GemvItem* items;
+    float* t_buf;          // T x kMaxRank fp32 intermediate, row = position in the permutation
 };
 
 __device__ __forceinline__ void bf16x8_to_f32(const uint4& u, float* f) {
@@ -135,65 +175,104 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4& u, float* f) {
     }
 }
 
-// grid: (max items, ceil(d_out / kGemvCols)).  Each CTA recomputes t for its
-// <= kGemvTok tokens (A' rows and x rows come from L2 after the first CTA), then
-// updates its d_out slice of y for those tokens.
-__global__ void __launch_bounds__(kGemvThreads) gemv_kernel(GemvArgs a) {
-    __shared__ float tsm[kGemvTok][kMaxRank];
+__device__ __forceinline__ bool item_ok(const GemvArgs& a, int it, GemvItem& item, Seg& sg, int& k, int64_t& oa,
+                                        int64_t& ob, bool report) {
+    if (it >= a.counts[2]) return false;
+    item = a.items[it];
+    sg = a.segs[item.seg];
+    k = a.ranks[sg.adapter];
+    if (k <= 0) return false;
+    oa = a.off_A[sg.adapter];
+    ob = a.off_Bt[sg.adapter];
+    int err = 0;
+    if (k > kMaxRank) err = LF_ERR_SHAPE;
+    else if ((oa & 7) || (ob & 7)) err = LF_ERR_ALIGNMENT;
+    else if (oa < 0 || ob < 0 || oa + (int64_t)k * a.d_in > a.pool_A || ob + (int64_t)k * a.d_out > a.pool_Bt)
+        err = LF_ERR_WORKSPACE;
+    if (err) {
+        if (report && threadIdx.x == 0) latch_error(err);
+        return false;
+    }
+    return true;
+}
+
+constexpr int kShrinkJ = 8;   // rows of A' per pass
+
+// Shrink: t[item][q][j] = A'_a[j] . x[tok_q] (fp32), one CTA per work item.  The
+// d_in range is split across all warps so each warp keeps many 16-byte loads in
+// flight; partial sums are reduced through shared memory in a fixed order.
+__global__ void __launch_bounds__(kGemvThreads) shrink_kernel(GemvArgs a) {
+    __shared__ float part[kGemvThreads / 32][kShrinkJ][kGemvTok];
     __shared__ int32_t toks[kGemvTok];
-    const int it = blockIdx.x;
-    if (it >= a.counts[2]) return;
-    const GemvItem item = a.items[it];
-    const Seg sg = a.segs[item.seg];
-    const int ad = sg.adapter;
-    const int k = a.ranks[ad];
-    if (k <= 0) return;
-    if (k > kMaxRank) {
-        latch_error(LF_ERR_SHAPE);
-        return;
-    }
-    const int64_t oa = a.off_A[ad], ob = a.off_Bt[ad];
-    if ((oa & 7) || (ob & 7)) {
-        latch_error(LF_ERR_ALIGNMENT);
-        return;
-    }
-    if (oa < 0 || ob < 0 || oa + (int64_t)k * a.d_in > a.pool_A || ob + (int64_t)k * a.d_out > a.pool_Bt) {
-        latch_error(LF_ERR_WORKSPACE);
-        return;
-    }
+    GemvItem item; Seg sg; int k; int64_t oa, ob;
+    if (!item_ok(a, blockIdx.x, item, sg, k, oa, ob, true)) return;
     const int nt = item.ntok;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     if (tid < nt) toks[tid] = a.perm[sg.start + item.tok0 + tid];
     __syncthreads();
-
-    // shrink: warp w computes rows j = w, w+8, ... of t
     const __nv_bfloat16* Ap = a.A_pool + oa;
-    for (int j = warp; j < k; j += kGemvThreads / 32) {
-        float acc[kGemvTok];
+    float* tout = a.t_buf + (size_t)(sg.start + item.tok0) * kMaxRank;
+    for (int j0 = 0; j0 < k; j0 += kShrinkJ) {
+        float acc[kShrinkJ][kGemvTok];
 #pragma unroll
-        for (int q = 0; q < kGemvTok; ++q) acc[q] = 0.f;
-        const __nv_bfloat16* arow = Ap + (int64_t)j * a.d_in;
-        for (int d0 = lane * 8; d0 < a.d_in; d0 += 256) {
-            float af[8], xf[8];
-            bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(arow + d0)), af);
+        for (int jj = 0; jj < kShrinkJ; ++jj)
 #pragma unroll
-            for (int q = 0; q < kGemvTok; ++q) {
-                if (q < nt) {
-                    bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(a.x + (int64_t)toks[q] * a.d_in + d0)), xf);
+            for (int q = 0; q < kGemvTok; ++q) acc[jj][q] = 0.f;
+        for (int d0 = tid * 8; d0 < a.d_in; d0 += kGemvThreads * 8) {
+            float xf[kGemvTok][8];
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) acc[q] = fmaf(af[e], xf[e], acc[q]);
+            for (int q = 0; q < kGemvTok; ++q)
+                if (q < nt) bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(a.x + (int64_t)toks[q] * a.d_in + d0)), xf[q]);
+#pragma unroll
+            for (int jj = 0; jj < kShrinkJ; ++jj) {
+                if (j0 + jj < k) {
+                    float af[8];
+                    bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(Ap + (int64_t)(j0 + jj) * a.d_in + d0)), af);
+#pragma unroll
+                    for (int q = 0; q < kGemvTok; ++q) {
+                        if (q < nt) {
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) acc[jj][q] = fmaf(af[e], xf[q][e], acc[jj][q]);
+                        }
+                    }
                 }
             }
         }
 #pragma unroll
-        for (int q = 0; q < kGemvTok; ++q) {
-            const float v = warp_sum(acc[q]);
-            if (lane == 0 && q < nt) tsm[q][j] = v;
+        for (int jj = 0; jj < kShrinkJ; ++jj)
+#pragma unroll
+            for (int q = 0; q < kGemvTok; ++q) {
+                const float v = warp_sum(acc[jj][q]);
+                if (lane == 0) part[warp][jj][q] = v;
+            }
+        __syncthreads();
+        if (tid < kShrinkJ * kGemvTok) {
+            const int jj = tid / kGemvTok, q = tid % kGemvTok;
+            float v = 0.f;
+#pragma unroll
+            for (int w = 0; w < kGemvThreads / 32; ++w) v += part[w][jj][q];
+            if (j0 + jj < k && q < nt) tout[q * kMaxRank + j0 + jj] = v;
         }
+        __syncthreads();
+    }
+}
+
+// Expand: y[tok_q][e..e+7] = bf16(y + s * sum_j t[q][j] B'^T[j][e..e+7]);
+// grid (items, ceil(d_out / kGemvCols)).
+__global__ void __launch_bounds__(kGemvThreads) expand_kernel(GemvArgs a) {
+    __shared__ float tsm[kGemvTok][kMaxRank];
+    __shared__ int32_t toks[kGemvTok];
+    GemvItem item; Seg sg; int k; int64_t oa, ob;
+    if (!item_ok(a, blockIdx.x, item, sg, k, oa, ob, false)) return;
+    const int nt = item.ntok;
+    const int tid = threadIdx.x;
+    if (tid < nt) toks[tid] = a.perm[sg.start + item.tok0 + tid];
+    const float* tin = a.t_buf + (size_t)(sg.start + item.tok0) * kMaxRank;
+    for (int e = tid; e < nt * kMaxRank; e += kGemvThreads) {
+        const int q = e / kMaxRank, j = e % kMaxRank;
+        tsm[q][j] = j < k ? tin[e] : 0.f;
     }
     __syncthreads();
-
-    // expand: 8 consecutive columns per thread
     const int e = blockIdx.y * kGemvCols + tid * 8;
     if (e >= a.d_out) return;
     float acc[kGemvTok][8];
@@ -202,6 +281,7 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(GemvArgs a) {
 #pragma unroll
         for (int c = 0; c < 8; ++c) acc[q][c] = 0.f;
     const __nv_bfloat16* Bt = a.Bt_pool + ob + e;
+#pragma unroll 4
     for (int j = 0; j < k; ++j) {
         float bf[8];
         bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(Bt + (int64_t)j * a.d_out)), bf);

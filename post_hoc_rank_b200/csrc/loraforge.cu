@@ -176,12 +176,11 @@ static TsqrLayout tsqr_layout(int32_t n, const TsqrPlan& p) {
 }
 
 template <typename T, int RT>
-static cudaError_t launch_tsqr(const TsqrArgs<T>& a, int grid, cudaStream_t st) {
-    constexpr size_t smem = sizeof(TsqrSmem<T, RT, kTsqrTM>);
-    auto k = tsqr_kernel<T, RT, kTsqrTM, kTsqrThreads>;
-    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    if (grid > 0) LF_LAUNCH(sizeof(T) == 8 ? "tsqr_fp64_refine" : "tsqr_leaf_merge", k, grid, kTsqrThreads, smem, st, a);
+static cudaError_t launch_tsqr(const TsqrArgs<T>& a, int n_items, cudaStream_t st) {
+    auto k = tsqr_kernel<T, RT>;
+    constexpr int W = tsqr_warps<T>();
+    const int grid = (n_items + W - 1) / W;
+    if (grid > 0) LF_LAUNCH(sizeof(T) == 8 ? "tsqr_fp64_refine" : "tsqr_leaf_merge", k, grid, 32 * W, 0, st, a);
     return cudaGetLastError();
 }
 
@@ -192,21 +191,23 @@ static cudaError_t launch_tsqr_rt(int RT, const TsqrArgs<T>& a, int grid, cudaSt
     return launch_tsqr<T, 64>(a, grid, st);
 }
 
-template <typename TIN, int RT>
-static cudaError_t launch_svd(const SvdArgs<TIN>& a, int grid, cudaStream_t st) {
-    constexpr size_t smem = sizeof(SvdSmem<RT>);
-    auto k = svd_kernel<TIN, RT>;
+template <typename TIN, typename T, int RT>
+static cudaError_t launch_svd(const SvdArgs<TIN, T>& a, int n_items, cudaStream_t st) {
+    constexpr int W = svd_warps<T>();
+    constexpr size_t smem = W * sizeof(SvdSmem<T, RT>);
+    auto k = svd_kernel<TIN, T, RT>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    if (grid > 0) LF_LAUNCH(sizeof(TIN) == 8 ? "svd_fp64_refine" : "svd_jacobi", k, grid, kSvdThreads, smem, st, a);
+    const int grid = (n_items + W - 1) / W;
+    if (grid > 0) LF_LAUNCH(sizeof(T) == 8 ? "svd_fp64_refine" : "svd_jacobi", k, grid, 32 * W, smem, st, a);
     return cudaGetLastError();
 }
 
-template <typename TIN>
-static cudaError_t launch_svd_rt(int RT, const SvdArgs<TIN>& a, int grid, cudaStream_t st) {
-    if (RT == 16) return launch_svd<TIN, 16>(a, grid, st);
-    if (RT == 32) return launch_svd<TIN, 32>(a, grid, st);
-    return launch_svd<TIN, 64>(a, grid, st);
+template <typename TIN, typename T>
+static cudaError_t launch_svd_rt(int RT, const SvdArgs<TIN, T>& a, int n_items, cudaStream_t st) {
+    if (RT == 16) return launch_svd<TIN, T, 16>(a, n_items, st);
+    if (RT == 32) return launch_svd<TIN, T, 32>(a, n_items, st);
+    return launch_svd<TIN, T, 64>(a, n_items, st);
 }
 
 // ------------------------------------------------------------ groups (S scope)
@@ -311,7 +312,8 @@ constexpr size_t al256(size_t x) { return (x + 255) / 256 * 256; }
 constexpr size_t kNoallocScratchBytes =
     al256(4 * sizeof(int32_t)) + al256((size_t)LF_NOALLOC_MAX_ADAPTERS * sizeof(Seg)) +
     al256((size_t)LF_NOALLOC_MAX_TOKENS * sizeof(int32_t)) +
-    al256(((size_t)LF_NOALLOC_MAX_TOKENS / kGemvTok + LF_NOALLOC_MAX_ADAPTERS + 1) * sizeof(GemvItem));
+    al256(((size_t)LF_NOALLOC_MAX_TOKENS / kGemvTok + LF_NOALLOC_MAX_ADAPTERS + 1) * sizeof(GemvItem)) +
+    al256((size_t)LF_NOALLOC_MAX_TOKENS * kMaxRank * sizeof(float));
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocScratchBytes];
 
 // In host code g_noalloc_scratch is only a host-side stand-in for the device array;
@@ -390,7 +392,7 @@ lf_status lf_tsqr_batched(const lf_module* mods, int32_t n, const float* B_base,
     ta.rs = p.rs;
     LF_CUDA_TRY(launch_tsqr_rt<float>(p.RT, ta, nwork, s));
 
-    SvdArgs<float> sa;
+    SvdArgs<float, float> sa;
     sa.mods = ta.mods;
     sa.mod_ids = nullptr;
     sa.n = reinterpret_cast<const int32_t*>(base + L.n_dev);
@@ -400,8 +402,8 @@ lf_status lf_tsqr_batched(const lf_module* mods, int32_t n, const float* B_base,
     sa.U = U;
     sa.V = V;
     sa.rs = p.rs;
-    sa.max_sweeps = 30;
-    LF_CUDA_TRY(launch_svd_rt<float>(p.RT, sa, n, s));
+    sa.max_sweeps = 20;
+    LF_CUDA_TRY(launch_svd_rt(p.RT, sa, n, s));
     return LF_OK;
 }
 
@@ -582,7 +584,7 @@ lf_status lf_truncate_export(const lf_module* mods, int32_t n, lf_policy pol, co
         ta.R_A = reinterpret_cast<double*>(base + L.rRA);
         ta.rs = p.rs;
         LF_CUDA_TRY(launch_tsqr_rt<double>(p.RT, ta, p.refine_max_work, s));
-        SvdArgs<double> sa;
+        SvdArgs<double, double> sa;
         sa.mods = dmods;
         sa.mod_ids = flist;
         sa.n = fcount + 1;
@@ -592,8 +594,8 @@ lf_status lf_truncate_export(const lf_module* mods, int32_t n, lf_policy pol, co
         sa.U = nullptr;
         sa.V = nullptr;
         sa.rs = p.rs;
-        sa.max_sweeps = 30;
-        LF_CUDA_TRY(launch_svd_rt<double>(p.RT, sa, p.refine_cap, s));
+        sa.max_sweeps = 20;
+        LF_CUDA_TRY(launch_svd_rt(p.RT, sa, p.refine_cap, s));
         double* sigref = reinterpret_cast<double*>(base + L.sigref);
         LF_CUDA_TRY(cudaMemcpyAsync(sigref, sigma, (size_t)n * p.rs * sizeof(double), cudaMemcpyDeviceToDevice, s));
         LF_LAUNCH("refine_plan", scatter_sigma_kernel, p.refine_cap, 64, 0, s, flist, fcount + 1, sa.sigma, sigref, p.rs);
@@ -627,8 +629,7 @@ lf_status lf_truncate_export(const lf_module* mods, int32_t n, lf_policy pol, co
     ea.Bt_pool16 = reinterpret_cast<__nv_bfloat16*>(Bt_pool_bf16);
     ea.cap_A = pool_cap_A;
     ea.cap_Bt = pool_cap_Bt;
-    LF_CUDA_TRY(cudaFuncSetAttribute(export_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kExportSmem));
-    LF_LAUNCH("export_stream", export_kernel, (int)p.ework.size(), kExpThreads, kExportSmem, s, ea);
+    LF_LAUNCH("export_stream", export_kernel, (int)p.ework.size(), kExpThreads, 0, s, ea);
     return launch_status();
 }
 
@@ -640,6 +641,7 @@ size_t lf_apply_workspace_size(int32_t T, int32_t n_adapters) {
     c.take<Seg>((size_t)std::max<int64_t>(mseg, 1));
     c.take<int32_t>((size_t)std::max(T, 1));
     c.take<GemvItem>((size_t)(T / kGemvTok + mseg + 1));
+    c.take<float>((size_t)std::max(T, 1) * kMaxRank);
     return c.off + 256;
 }
 
@@ -665,8 +667,9 @@ lf_status lf_lora_shrink_expand(int32_t T, int32_t d_in, int32_t d_out, const vo
     o.segs = c.take<Seg>((size_t)std::max<int64_t>(mseg, 1));
     o.perm = c.take<int32_t>((size_t)T);
     o.items = c.take<GemvItem>((size_t)(T / kGemvTok + mseg + 1));
+    float* t_buf = c.take<float>((size_t)T * kMaxRank);
     o.seg_out = seg_out;
-    const size_t rsmem = (size_t)n_adapters * sizeof(int32_t);
+    const size_t rsmem = 2 * (size_t)n_adapters * sizeof(int32_t);
     LF_CUDA_TRY(cudaFuncSetAttribute(route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rsmem));
     LF_LAUNCH("route", route_kernel, 1, kRouteThreads, rsmem, s, ids, T, n_adapters, o);
     LF_CUDA_TRY(cudaGetLastError());
@@ -687,8 +690,11 @@ lf_status lf_lora_shrink_expand(int32_t T, int32_t d_in, int32_t d_out, const vo
     g.segs = o.segs;
     g.perm = o.perm;
     g.items = o.items;
-    dim3 grid((unsigned)(T / kGemvTok + mseg + 1), (unsigned)cdiv(d_out, kGemvCols));
-    LF_LAUNCH("shrink_expand_gemv", gemv_kernel, grid, kGemvThreads, 0, s, g);
+    g.t_buf = t_buf;
+    const unsigned max_items = (unsigned)(T / kGemvTok + mseg + 1);
+    LF_LAUNCH("shrink_gemv", shrink_kernel, max_items, kGemvThreads, 0, s, g);
+    LF_CUDA_TRY(cudaGetLastError());
+    LF_LAUNCH("expand_gemv", expand_kernel, dim3(max_items, (unsigned)cdiv(d_out, kGemvCols)), kGemvThreads, 0, s, g);
     return launch_status();
 }
 
@@ -715,10 +721,11 @@ lf_status lf_lora_shrink_expand_noalloc(int32_t T, int32_t d_in, int32_t d_out, 
     o.segs = c.take<Seg>((size_t)LF_NOALLOC_MAX_ADAPTERS);
     o.perm = c.take<int32_t>((size_t)LF_NOALLOC_MAX_TOKENS);
     o.items = c.take<GemvItem>((size_t)LF_NOALLOC_MAX_TOKENS / kGemvTok + LF_NOALLOC_MAX_ADAPTERS + 1);
+    float* t_buf = c.take<float>((size_t)LF_NOALLOC_MAX_TOKENS * kMaxRank);
     o.seg_out = seg_out;
     if (c.off > kNoallocScratchBytes) return LF_ERR_WORKSPACE;
     const int64_t mseg = std::min<int64_t>(T, n_adapters);
-    const size_t rsmem = (size_t)n_adapters * sizeof(int32_t);
+    const size_t rsmem = 2 * (size_t)n_adapters * sizeof(int32_t);
     LF_CUDA_TRY(cudaFuncSetAttribute(route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rsmem));
     LF_LAUNCH("route", route_kernel, 1, kRouteThreads, rsmem, s, ids, T, n_adapters, o);
     LF_CUDA_TRY(cudaGetLastError());
@@ -739,8 +746,11 @@ lf_status lf_lora_shrink_expand_noalloc(int32_t T, int32_t d_in, int32_t d_out, 
     g.segs = o.segs;
     g.perm = o.perm;
     g.items = o.items;
-    dim3 grid((unsigned)(T / kGemvTok + mseg + 1), (unsigned)cdiv(d_out, kGemvCols));
-    LF_LAUNCH("shrink_expand_gemv", gemv_kernel, grid, kGemvThreads, 0, s, g);
+    g.t_buf = t_buf;
+    const unsigned max_items = (unsigned)(T / kGemvTok + mseg + 1);
+    LF_LAUNCH("shrink_gemv", shrink_kernel, max_items, kGemvThreads, 0, s, g);
+    LF_CUDA_TRY(cudaGetLastError());
+    LF_LAUNCH("expand_gemv", expand_kernel, dim3(max_items, (unsigned)cdiv(d_out, kGemvCols)), kGemvThreads, 0, s, g);
     return launch_status();
 }
 

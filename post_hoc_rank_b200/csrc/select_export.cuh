@@ -302,74 +302,111 @@ struct ExportArgs {
     int64_t cap_A, cap_Bt;
 };
 
-constexpr int kExpThreads = 128;
-constexpr int kExpRows = 128;   // rows of B staged per step
+constexpr int kExpThreads = 256;   // 8 warps
+constexpr int kExpJ = 16;          // retained directions per accumulator pass
 
-template <int KB>
-__device__ void export_b_rows(const ExportArgs& a, const lf_module& md, int k, float* sm, const float* cB,
-                              int64_t obt, int start, int len) {
+// B part: lane owns one row e of B (r fp32 = 16 float4 loads issued together) and
+// writes B'^T[j][e] = sum_l C_Bt[j][l] B[e][l] for j < k (coalesced across lanes).
+__device__ void export_b_rows(const ExportArgs& a, const lf_module& md, int k, const float* cB, int64_t obt,
+                              int start, int len) {
     const int r = md.r, tid = threadIdx.x;
     const float* B = a.B_base + md.B_off;
-    for (int e0 = start; e0 < start + len; e0 += kExpRows) {
-        const int nr = min(kExpRows, start + len - e0);
-        __syncthreads();
-        // stage rows e0..e0+nr of B (contiguous nr*r floats) transposed: sm[l][row]
-        for (int q = tid; q < nr * r; q += kExpThreads) {
-            const int row = q / r, l = q % r;
-            sm[l * (kExpRows + 1) + row] = __ldg(B + (int64_t)(e0 + row) * r + l);
-        }
-        __syncthreads();
-        if (tid < nr) {
-            float acc[KB];
+    for (int e0 = start; e0 < start + len; e0 += kExpThreads) {
+        const int e = e0 + tid;
+        if (e >= start + len) break;
+        float x[kMaxRank];
+        if (r == kMaxRank) {
+            const float4* src = reinterpret_cast<const float4*>(B + (int64_t)e * kMaxRank);
 #pragma unroll
-            for (int j = 0; j < KB; ++j) acc[j] = 0.f;
-            for (int l = 0; l < r; ++l) {
-                const float x = sm[l * (kExpRows + 1) + tid];
-#pragma unroll
-                for (int j = 0; j < KB; ++j)
-                    if (j < k) acc[j] = fmaf(cB[j * r + l], x, acc[j]);
+            for (int q = 0; q < kMaxRank / 4; ++q) {
+                const float4 v = __ldg(src + q);
+                x[4 * q] = v.x; x[4 * q + 1] = v.y; x[4 * q + 2] = v.z; x[4 * q + 3] = v.w;
             }
-            const int64_t e = e0 + tid;
+        } else {
 #pragma unroll
-            for (int j = 0; j < KB; ++j) {
-                if (j < k) {
-                    const int64_t o = obt + (int64_t)j * md.d_out + e;
-                    a.Bt_pool[o] = acc[j];
-                    if (a.Bt_pool16) a.Bt_pool16[o] = __float2bfloat16_rn(acc[j]);
+            for (int l = 0; l < kMaxRank; ++l) x[l] = l < r ? __ldg(B + (int64_t)e * r + l) : 0.f;
+        }
+        for (int j0 = 0; j0 < k; j0 += kExpJ) {
+            float acc[kExpJ];
+#pragma unroll
+            for (int jj = 0; jj < kExpJ; ++jj) {
+                float t = 0.f;
+                if (j0 + jj < k) {
+                    const float* cr = cB + (j0 + jj) * kMaxRank;
+#pragma unroll
+                    for (int l = 0; l < kMaxRank; ++l) t = fmaf(cr[l], x[l], t);
+                }
+                acc[jj] = t;
+            }
+#pragma unroll
+            for (int jj = 0; jj < kExpJ; ++jj) {
+                if (j0 + jj < k) {
+                    const int64_t o = obt + (int64_t)(j0 + jj) * md.d_out + e;
+                    a.Bt_pool[o] = acc[jj];
+                    if (a.Bt_pool16) a.Bt_pool16[o] = __float2bfloat16_rn(acc[jj]);
                 }
             }
         }
     }
 }
 
-template <int KB>
+// A part: thread owns 4 consecutive columns d..d+3 of A (r x d_in) and writes
+// A'[j][d..d+3] = sum_l C_A[j][l] A[l][d..d+3].
 __device__ void export_a_cols(const ExportArgs& a, const lf_module& md, int k, const float* cA, int64_t oa,
                               int start, int len) {
     const int r = md.r;
     const float* A = a.A_base + md.A_off;
-    for (int d = start + threadIdx.x; d < start + len; d += kExpThreads) {
-        float acc[KB];
+    const bool vec = (md.d_in % 4 == 0) && (start % 4 == 0);
+    for (int d = start + 4 * threadIdx.x; d < start + len; d += 4 * kExpThreads) {
+        const int nd = min(4, start + len - d);
+        for (int j0 = 0; j0 < k; j0 += kExpJ) {
+            float acc[kExpJ][4];
 #pragma unroll
-        for (int j = 0; j < KB; ++j) acc[j] = 0.f;
-        for (int l = 0; l < r; ++l) {
-            const float x = __ldg(A + (int64_t)l * md.d_in + d);
+            for (int jj = 0; jj < kExpJ; ++jj)
 #pragma unroll
-            for (int j = 0; j < KB; ++j)
-                if (j < k) acc[j] = fmaf(cA[j * r + l], x, acc[j]);
-        }
+                for (int c = 0; c < 4; ++c) acc[jj][c] = 0.f;
+#pragma unroll 8
+            for (int l = 0; l < r; ++l) {
+                float4 v;
+                const float* src = A + (int64_t)l * md.d_in + d;
+                if (vec && nd == 4) {
+                    v = __ldg(reinterpret_cast<const float4*>(src));
+                } else {
+                    v.x = __ldg(src);
+                    v.y = nd > 1 ? __ldg(src + 1) : 0.f;
+                    v.z = nd > 2 ? __ldg(src + 2) : 0.f;
+                    v.w = nd > 3 ? __ldg(src + 3) : 0.f;
+                }
 #pragma unroll
-        for (int j = 0; j < KB; ++j) {
-            if (j < k) {
-                const int64_t o = oa + (int64_t)j * md.d_in + d;
-                a.A_pool[o] = acc[j];
-                if (a.A_pool16) a.A_pool16[o] = __float2bfloat16_rn(acc[j]);
+                for (int jj = 0; jj < kExpJ; ++jj) {
+                    if (j0 + jj < k) {
+                        const float cj = cA[(j0 + jj) * kMaxRank + l];
+                        acc[jj][0] = fmaf(cj, v.x, acc[jj][0]);
+                        acc[jj][1] = fmaf(cj, v.y, acc[jj][1]);
+                        acc[jj][2] = fmaf(cj, v.z, acc[jj][2]);
+                        acc[jj][3] = fmaf(cj, v.w, acc[jj][3]);
+                    }
+                }
+            }
+#pragma unroll
+            for (int jj = 0; jj < kExpJ; ++jj) {
+                if (j0 + jj < k) {
+                    const int64_t o = oa + (int64_t)(j0 + jj) * md.d_in + d;
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        if (c < nd) {
+                            a.A_pool[o + c] = acc[jj][c];
+                            if (a.A_pool16) a.A_pool16[o + c] = __float2bfloat16_rn(acc[jj][c]);
+                        }
+                    }
+                }
             }
         }
     }
 }
 
 __global__ void __launch_bounds__(kExpThreads) export_kernel(ExportArgs a) {
-    extern __shared__ __align__(16) float esm[];
+    __shared__ __align__(16) float coef[kMaxRank * kMaxRank];   // k x r, row stride kMaxRank, zero past r
     const ExportWork w = a.work[blockIdx.x];
     const lf_module md = a.mods[w.mod];
     const int k = a.ranks[w.mod];
@@ -381,26 +418,14 @@ __global__ void __launch_bounds__(kExpThreads) export_kernel(ExportArgs a) {
     } else {
         if (oa + (int64_t)k * md.d_in > a.cap_A) return;
     }
-    // coefficients for this module into smem (k x r, row-major, stride r)
-    float* coef = esm;                         // kMaxRank * kMaxRank
-    float* stage = esm + kMaxRank * kMaxRank;  // kMaxRank * (kExpRows + 1)
     const float* C = (w.part == 0 ? a.C_Bt : a.C_A) + (size_t)w.mod * a.rs * a.rs;
-    for (int e = threadIdx.x; e < k * r; e += kExpThreads) coef[e] = C[(e / r) * a.rs + (e % r)];
-    __syncthreads();
-#define LF_EXPORT_CASE(KB)                                                       \
-    if (k <= KB) {                                                               \
-        if (w.part == 0) export_b_rows<KB>(a, md, k, stage, coef, obt, w.start, w.len); \
-        else export_a_cols<KB>(a, md, k, coef, oa, w.start, w.len);              \
-        return;                                                                  \
+    for (int e = threadIdx.x; e < k * kMaxRank; e += kExpThreads) {
+        const int j = e / kMaxRank, l = e % kMaxRank;
+        coef[e] = l < r ? C[j * a.rs + l] : 0.f;
     }
-    LF_EXPORT_CASE(4)
-    LF_EXPORT_CASE(8)
-    LF_EXPORT_CASE(16)
-    LF_EXPORT_CASE(32)
-    LF_EXPORT_CASE(64)
-#undef LF_EXPORT_CASE
+    __syncthreads();
+    if (w.part == 0) export_b_rows(a, md, k, coef, obt, w.start, w.len);
+    else export_a_cols(a, md, k, coef, oa, w.start, w.len);
 }
-
-constexpr size_t kExportSmem = sizeof(float) * (kMaxRank * kMaxRank + kMaxRank * (kExpRows + 1));
 
 }  // namespace lf

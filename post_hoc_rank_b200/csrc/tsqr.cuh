@@ -8,19 +8,24 @@
 // M = R_B R_A^T (dW = Q_B M Q_A^T).
 //
 // Work decomposition: every (module, factor) matrix X (B: d_out x r, or A^T:
-// d_in x r) is cut into chunks of at most kTsqrChunk rows; one CTA owns one chunk
-// and folds its row tiles into a running R by structured Householder reflections
-// of [R; tile].  Chunk results are merged by the last CTA of the matrix to finish
-// (atomic counter, no waiting), always in chunk order, so the result does not
-// depend on scheduling.
+// d_in x r) is cut into chunks of at most kTsqrChunk rows; one warp owns one chunk
+// and folds its 32-row register tiles into a running R by structured Householder
+// reflections of [R; tile].  Chunk results are merged by the last warp of the
+// matrix to finish (atomic counter, no waiting), always in chunk order, so the
+// result does not depend on scheduling.
 #pragma once
 #include "common.cuh"
 
+#include <type_traits>
+
 namespace lf {
 
-constexpr int kTsqrChunk = 2048;   // rows per work item
-constexpr int kTsqrTM = 128;       // rows per smem tile
-constexpr int kTsqrThreads = 256;
+constexpr int kTsqrChunk = 1024;   // rows per work item (one warp)
+constexpr int kTsqrTM = 32;        // rows per register tile
+// warps (independent work items) per CTA: the packed R of every warp lives in static
+// shared memory (fp32 RT=64: 8.3 KB per warp; fp64: 16.6 KB)
+template <typename T>
+__host__ __device__ constexpr int tsqr_warps() { return sizeof(T) == 8 ? 2 : 4; }
 
 struct TsqrWork {
     int32_t mf;      // 2 * local module index + factor (0 = B, 1 = A^T)
@@ -49,107 +54,138 @@ struct TsqrArgs {
     int32_t rs;
 };
 
-template <typename T, int RT, int TM>
-struct TsqrSmem {
-    T R[RT][RT + 1];
-    T tile[TM][RT + 1];
-    T v[TM];
-    T scal[2];
-    int flag;
+// Packed upper triangle of an RT x RT matrix, row-major: row j holds columns j..RT-1.
+template <int RT>
+__device__ __forceinline__ int tri_off(int j, int c) { return j * RT - (j * (j - 1)) / 2 + (c - j); }
+template <int RT>
+__host__ __device__ constexpr int tri_size() { return RT * (RT + 1) / 2; }
+
+// Column ownership inside a warp: RT = 64 -> lane l owns columns l and 63 - l
+// (keeps the shrinking trailing triangle spread over the most lanes); RT <= 32 ->
+// lane l owns column l.
+template <int RT>
+struct Cols {
+    static constexpr int NS = RT > 32 ? 2 : 1;
+    __device__ static int col(int lane, int s) { return s == 0 ? lane : RT - 1 - lane; }
+    __device__ static int owner(int j) { return (RT > 32 && j >= 32) ? RT - 1 - j : j; }
+    __device__ static int slot(int j) { return (RT > 32 && j >= 32) ? 1 : 0; }
 };
 
-// Structured Householder QR of the stacked [R (RT x RT upper); tile (TM x RT)],
-// columns 0..ncols-1; R is overwritten with the new triangle, the tile is consumed.
-// Reflector j touches row j of R and every tile row (LAPACK tpqrt-style).
-template <typename T, int RT, int TM, int NT>
-__device__ void absorb_tile(TsqrSmem<T, RT, TM>& s, int ncols) {
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    constexpr int NW = NT / 32;
-    for (int j = 0; j < ncols; ++j) {
-        if (warp == 0) {
-            T ss = 0;
-            for (int i = lane; i < TM; i += 32) {
-                T x = s.tile[i][j];
-                ss += x * x;
+// One warp folds a TM x RT tile (registers x[s][i] = X[i][col(lane, s)]) into the
+// running triangle Rp (packed, shared memory) by structured Householder reflections
+// of [R; tile]: reflector j involves row j of R and every tile row, so
+//   beta_j = -sign(R_jj) ||[R_jj; X_:j]||,  tau = (beta - R_jj) / beta,
+//   v = [1; X_:j / (R_jj - beta)],  w_c = tau (R_jc + v^T X_:c),
+//   R_jc -= w_c,  X_:c -= w_c v   for c > j.
+// All dot products are over the lane's own rows; the reflector column is published
+// once through shared memory.
+template <typename T>
+__device__ __forceinline__ T quick_div(T a, T b) { return a / b; }
+template <>
+__device__ __forceinline__ float quick_div<float>(float a, float b) { return __fdividef(a, b); }
+
+template <typename T, int RT>
+__device__ __forceinline__ void warp_absorb(T (&x)[Cols<RT>::NS][kTsqrTM], T* Rp, T* vbuf, int r) {
+    const int lane = threadIdx.x & 31;
+    using C = Cols<RT>;
+    constexpr int VW = 16 / sizeof(T);   // elements per 16-byte vector
+    using V = typename std::conditional<sizeof(T) == 4, float4, double2>::type;
+    for (int j = 0; j < r; ++j) {
+        const int own = C::owner(j), sl = C::slot(j);
+        if (lane == own) {   // publish column j (16-byte stores)
+            V* dst = reinterpret_cast<V*>(vbuf);
+            if (sl == 0) {
+#pragma unroll
+                for (int i = 0; i < kTsqrTM; i += VW) dst[i / VW] = *reinterpret_cast<const V*>(&x[0][i]);
+            } else {
+#pragma unroll
+                for (int i = 0; i < kTsqrTM; i += VW) dst[i / VW] = *reinterpret_cast<const V*>(&x[C::NS - 1][i]);
             }
-            ss = warp_sum(ss);
-            if (lane == 0) {
-                T x0 = s.R[j][j];
-                T tau = 0, scale = 0;
-                if (ss > T(0)) {
-                    T nrm = sqrt(x0 * x0 + ss);
-                    T beta = x0 >= T(0) ? -nrm : nrm;
-                    tau = (beta - x0) / beta;
-                    scale = T(1) / (x0 - beta);
-                    s.R[j][j] = beta;
-                }
-                s.scal[0] = tau;
-                s.scal[1] = scale;
+        }
+        __syncwarp();
+        T v[kTsqrTM];
+#pragma unroll
+        for (int i = 0; i < kTsqrTM; i += VW) *reinterpret_cast<V*>(&v[i]) = reinterpret_cast<const V*>(vbuf)[i / VW];
+        const T x0 = Rp[tri_off<RT>(j, j)];
+        __syncwarp();
+        T s4[4] = {0, 0, 0, 0};
+#pragma unroll
+        for (int i = 0; i < kTsqrTM; ++i) s4[i & 3] = fma(v[i], v[i], s4[i & 3]);
+        const T ss = (s4[0] + s4[1]) + (s4[2] + s4[3]);
+        if (ss == T(0)) continue;  // column already zero below R_jj: H = I (warp-uniform)
+        const T nrm = sqrt(fma(x0, x0, ss));
+        const T beta = x0 >= T(0) ? -nrm : nrm;
+        const T tau = quick_div(beta - x0, beta);
+        const T scale = quick_div(T(1), x0 - beta);
+        if (lane == 0) Rp[tri_off<RT>(j, j)] = beta;
+#pragma unroll
+        for (int s = 0; s < C::NS; ++s) {
+            const int c = C::col(lane, s);
+            if (c > j && c < r) {
+                T d4[4] = {0, 0, 0, 0};
+#pragma unroll
+                for (int i = 0; i < kTsqrTM; ++i) d4[i & 3] = fma(v[i], x[s][i], d4[i & 3]);
+                const T d = (d4[0] + d4[1]) + (d4[2] + d4[3]);
+                const int o = tri_off<RT>(j, c);
+                const T w = tau * fma(scale, d, Rp[o]);
+                Rp[o] -= w;
+                const T a = w * scale;
+#pragma unroll
+                for (int i = 0; i < kTsqrTM; ++i) x[s][i] = fma(-a, v[i], x[s][i]);
             }
         }
-        __syncthreads();
-        const T tau = s.scal[0];
-        const T scale = s.scal[1];
-        if (tau == T(0)) {
-            __syncthreads();
-            continue;
-        }
-        for (int i = tid; i < TM; i += NT) s.v[i] = s.tile[i][j] * scale;
-        __syncthreads();
-        for (int c = j + 1 + warp; c < ncols; c += NW) {
-            T d = 0;
-            for (int i = lane; i < TM; i += 32) d += s.v[i] * s.tile[i][c];
-            d = warp_sum(d);
-            const T w = (s.R[j][c] + d) * tau;
-            __syncwarp();
-            if (lane == 0) s.R[j][c] -= w;
-            for (int i = lane; i < TM; i += 32) s.tile[i][c] -= w * s.v[i];
-        }
-        __syncthreads();
+        __syncwarp();
     }
 }
 
-template <typename T, int RT, int TM, int NT>
-__device__ void load_tile(TsqrSmem<T, RT, TM>& s, const float* __restrict__ X, int factor,
-                          int64_t row_base, int nr, int r, int ld) {
-    // factor 0: X = B (row-major, ld = r);  factor 1: X = A^T, A row-major (ld = d_in)
-    if (factor == 0) {
-        for (int e = threadIdx.x; e < TM * RT; e += NT) {
-            const int i = e / RT, c = e % RT;
-            T v = 0;
-            if (i < nr && c < r) v = (T)__ldg(X + (row_base + i) * (int64_t)r + c);
-            s.tile[i][c] = v;
-        }
-    } else {
-        for (int e = threadIdx.x; e < TM * RT; e += NT) {
-            const int c = e / TM, i = e % TM;
-            T v = 0;
-            if (i < nr && c < r) v = (T)__ldg(X + (int64_t)c * ld + row_base + i);
-            s.tile[i][c] = v;
+template <typename T, int RT>
+__device__ __forceinline__ void load_rows(T (&x)[Cols<RT>::NS][kTsqrTM], const float* __restrict__ X, int factor,
+                                          int64_t row_base, int nr, int r, int ld) {
+    const int lane = threadIdx.x & 31;
+    using C = Cols<RT>;
+#pragma unroll
+    for (int s = 0; s < C::NS; ++s) {
+        const int c = C::col(lane, s);
+        const bool okc = c < r;
+        if (factor == 0) {  // X = B, row-major d_out x r: X[i][c] = B[(row_base+i)*r + c]
+            const float* p = X + row_base * (int64_t)r + c;
+#pragma unroll
+            for (int i = 0; i < kTsqrTM; ++i) x[s][i] = (okc && i < nr) ? (T)__ldg(p + (int64_t)i * r) : T(0);
+        } else {            // X = A^T, A row-major r x d_in: X[i][c] = A[c*ld + row_base + i]
+            const float* p = X + (int64_t)c * ld + row_base;
+#pragma unroll
+            for (int i = 0; i < kTsqrTM; ++i) x[s][i] = (okc && i < nr) ? (T)__ldg(p + i) : T(0);
         }
     }
 }
 
-template <typename T, int RT, int TM, int NT>
-__device__ void write_final(TsqrSmem<T, RT, TM>& s, T* out, int r, int rs) {
-    // canonical sign: diag(R) >= 0 (flip whole rows)
-    for (int e = threadIdx.x; e < rs * rs; e += NT) {
-        const int j = e / rs, c = e % rs;
-        T v = 0;
-        if (j < r && c < r && c >= j) {
-            v = s.R[j][c];
-            if (s.R[j][j] < T(0)) v = -v;
+template <typename T, int RT>
+__device__ __forceinline__ void load_tri_rows(T (&x)[Cols<RT>::NS][kTsqrTM], const T* P, int i0) {
+    // rows i0..i0+TM-1 of a dense RT x RT (upper-triangular) partial R
+    const int lane = threadIdx.x & 31;
+    using C = Cols<RT>;
+#pragma unroll
+    for (int s = 0; s < C::NS; ++s) {
+        const int c = C::col(lane, s);
+#pragma unroll
+        for (int i = 0; i < kTsqrTM; ++i) {
+            const int row = i0 + i;
+            x[s][i] = (c < RT && row < RT) ? __ldcg(P + row * RT + c) : T(0);
         }
-        out[e] = v;
     }
 }
 
-template <typename T, int RT, int TM, int NT>
-__global__ void __launch_bounds__(NT) tsqr_kernel(TsqrArgs<T> a) {
-    extern __shared__ __align__(16) unsigned char smem_raw[];
-    auto& s = *reinterpret_cast<TsqrSmem<T, RT, TM>*>(smem_raw);
-    const int wi = blockIdx.x;
-    if (wi >= *a.n_work) return;
+template <typename T, int RT>
+__global__ void __launch_bounds__(32 * tsqr_warps<T>(), sizeof(T) == 4 ? 4 : 1) tsqr_kernel(TsqrArgs<T> a) {
+    constexpr int W = tsqr_warps<T>();
+    __shared__ T s_R[W][tri_size<RT>()];
+    __shared__ __align__(16) T s_v[W][kTsqrTM];
+    __shared__ int s_last[W];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int wi = blockIdx.x * W + warp;
+    if (wi >= *a.n_work) return;   // warp-uniform; no block-level barriers below
+    T* Rp = s_R[warp];
+    T* vbuf = s_v[warp];
     const TsqrWork w = a.work[wi];
     const int local = w.mf >> 1, factor = w.mf & 1;
     const int gm = a.mod_ids ? a.mod_ids[local] : local;
@@ -158,59 +194,67 @@ __global__ void __launch_bounds__(NT) tsqr_kernel(TsqrArgs<T> a) {
     const float* X = factor == 0 ? a.B_base + md.B_off : a.A_base + md.A_off;
     const int ld = factor == 0 ? r : md.d_in;
 
-    for (int e = threadIdx.x; e < RT * (RT + 1); e += NT) (&s.R[0][0])[e] = T(0);
-    for (int t0 = 0; t0 < w.nrows; t0 += TM) {
-        const int nr = min(TM, w.nrows - t0);
-        __syncthreads();
-        load_tile<T, RT, TM, NT>(s, X, factor, (int64_t)w.row0 + t0, nr, r, ld);
-        __syncthreads();
-        absorb_tile<T, RT, TM, NT>(s, r);
+    for (int e = lane; e < tri_size<RT>(); e += 32) Rp[e] = T(0);
+    __syncwarp();
+    T x[Cols<RT>::NS][kTsqrTM];
+    for (int t0 = 0; t0 < w.nrows; t0 += kTsqrTM) {
+        load_rows<T, RT>(x, X, factor, (int64_t)w.row0 + t0, min(kTsqrTM, w.nrows - t0), r, ld);
+        warp_absorb<T, RT>(x, Rp, vbuf, r);
     }
-    __syncthreads();
 
     T* out = (factor == 0 ? a.R_B : a.R_A) + (size_t)local * a.rs * a.rs;
     const TsqrInfo inf = a.info[w.mf];
-    if (inf.nchunks == 1) {
-        write_final<T, RT, TM, NT>(s, out, r, a.rs);
-        return;
-    }
-    T* P = a.partial + (size_t)w.slot * RT * RT;
-    for (int e = threadIdx.x; e < RT * RT; e += NT) P[e] = s.R[e / RT][e % RT];
-    __threadfence();
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        const int prev = atomicAdd(&a.counters[w.mf], 1);
-        s.flag = (prev == inf.nchunks - 1);
-    }
-    __syncthreads();
-    if (!s.flag) return;
-    __threadfence();
-    // fold the chunk triangles in chunk order: R = R_0, then R <- R([R; R_c])
-    const T* P0 = a.partial + (size_t)inf.slot0 * RT * RT;
-    for (int e = threadIdx.x; e < RT * RT; e += NT) s.R[e / RT][e % RT] = __ldcg(P0 + e);
-    for (int c = 1; c < inf.nchunks; ++c) {
-        const T* Pc = a.partial + (size_t)(inf.slot0 + c) * RT * RT;
-        __syncthreads();
-        for (int e = threadIdx.x; e < TM * RT; e += NT) {
-            const int i = e / RT, col = e % RT;
-            s.tile[i][col] = i < RT ? __ldcg(Pc + i * RT + col) : T(0);
+    if (inf.nchunks > 1) {
+        T* P = a.partial + (size_t)w.slot * RT * RT;
+        for (int e = lane; e < RT * RT; e += 32) {
+            const int j = e / RT, c = e % RT;
+            P[e] = c >= j ? Rp[tri_off<RT>(j, c)] : T(0);
         }
-        __syncthreads();
-        absorb_tile<T, RT, TM, NT>(s, r);
+        __threadfence();
+        __syncwarp();
+        if (lane == 0) s_last[warp] = (atomicAdd(&a.counters[w.mf], 1) == inf.nchunks - 1);
+        __syncwarp();
+        if (!s_last[warp]) return;
+        __threadfence();
+        // fold the chunk triangles in chunk order: R = R_0, then R <- R([R; R_c])
+        const T* P0 = a.partial + (size_t)inf.slot0 * RT * RT;
+        for (int e = lane; e < RT * RT; e += 32) {
+            const int j = e / RT, c = e % RT;
+            if (c >= j) Rp[tri_off<RT>(j, c)] = __ldcg(P0 + e);
+        }
+        __syncwarp();
+        for (int c = 1; c < inf.nchunks; ++c) {
+            const T* Pc = a.partial + (size_t)(inf.slot0 + c) * RT * RT;
+            for (int i0 = 0; i0 < r; i0 += kTsqrTM) {
+                load_tri_rows<T, RT>(x, Pc, i0);
+                warp_absorb<T, RT>(x, Rp, vbuf, r);
+            }
+        }
     }
-    __syncthreads();
-    write_final<T, RT, TM, NT>(s, out, r, a.rs);
+    // canonical sign: diag(R) >= 0 (flip whole rows); zero past r
+    for (int e = lane; e < a.rs * a.rs; e += 32) {
+        const int j = e / a.rs, c = e % a.rs;
+        T v = 0;
+        if (j < r && c < r && c >= j) {
+            v = Rp[tri_off<RT>(j, c)];
+            if (Rp[tri_off<RT>(j, j)] < T(0)) v = -v;
+        }
+        out[e] = v;
+    }
 }
 
 // ----------------------------------------------------------------------------
-// Small SVD: M = R_B R_A^T (r x r, fp64), one-sided Jacobi on the rows of M.
-// Rotating rows p, q of M by the same plane rotation that is applied to columns
+// Small SVD: M = R_B R_A^T (r x r), one-sided Jacobi on the rows of M.
+// Rotating rows p, q of M by the plane rotation that is also applied to columns
 // p, q of U (U starts at I) keeps M = U M'; at convergence the rows of M' are
-// orthogonal, sigma_p = |m'_p|, and row p of M' is sigma_p v_p^T.
+// orthogonal, sigma_p = |m'_p| and row p of M' is sigma_p v_p^T.
+// One warp per module; in each round of the round-robin ordering every lane owns
+// one of the r/2 disjoint pairs and forms its three dot products alone, so a round
+// needs no reductions.  T = float for the main path (the retained directions and
+// the energies near the S boundary are accurate to ~1e-6), T = double for the
+// boundary refinement.
 // ----------------------------------------------------------------------------
-constexpr int kSvdThreads = 128;
-
-template <typename TIN>
+template <typename TIN, typename T>
 struct SvdArgs {
     const lf_module* mods;
     const int32_t* mod_ids;   // local -> global (nullptr = identity)
@@ -224,127 +268,146 @@ struct SvdArgs {
     int32_t max_sweeps;
 };
 
-template <int RT>
+template <typename T, int RT>
 struct SvdSmem {
-    double M[RT][RT + 1];
-    double Ut[RT][RT + 1];
-    double sig[RT];
+    T M[RT][RT + 1];
+    T Ut[RT][RT + 1];   // Ut[p] = column p of U
+    T sig[RT];
     int perm[RT];
-    int rot;
 };
 
-template <typename TIN, int RT>
-__global__ void __launch_bounds__(kSvdThreads) svd_kernel(SvdArgs<TIN> a) {
+template <typename T>
+__host__ __device__ constexpr int svd_warps() { return sizeof(T) == 8 ? 1 : 2; }
+// Rotation threshold |gamma| > tol * sqrt(alpha beta): r * eps of the working type
+// (a tighter threshold cannot be met by rotations computed in that type).
+template <typename T>
+__device__ __forceinline__ T svd_tol(int r) { return T(r) * (sizeof(T) == 8 ? T(2.220446049250313e-16) : T(1.1920929e-7)); }
+
+template <typename TIN, typename T, int RT>
+__global__ void __launch_bounds__(32 * svd_warps<T>()) svd_kernel(SvdArgs<TIN, T> a) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
-    auto& s = *reinterpret_cast<SvdSmem<RT>*>(smem_raw);
-    const int local = blockIdx.x;
-    if (local >= *a.n) return;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    auto& s = reinterpret_cast<SvdSmem<T, RT>*>(smem_raw)[warp];
+    const int local = blockIdx.x * svd_warps<T>() + warp;
+    if (local >= *a.n) return;   // warp-uniform; no block barriers below
     const int gm = a.mod_ids ? a.mod_ids[local] : local;
     const int r = a.mods[gm].r;
     const int rs = a.rs;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    constexpr int NW = kSvdThreads / 32;
     const TIN* RB = a.R_B + (size_t)local * rs * rs;
     const TIN* RA = a.R_A + (size_t)local * rs * rs;
 
-    // M[i][j] = sum_{l >= max(i,j)} R_B[i][l] R_A[j][l]
-    for (int e = tid; e < r * r; e += kSvdThreads) {
-        const int i = e / r, j = e % r;
-        double acc = 0.0;
-        for (int l = max(i, j); l < r; ++l) acc += (double)RB[i * rs + l] * (double)RA[j * rs + l];
-        s.M[i][j] = acc;
+    // stage R_A in Ut, then M[i][j] = sum_{l >= max(i,j)} R_B[i][l] R_A[j][l] (one row per lane)
+    for (int e = lane; e < r * r; e += 32) {
+        const int i = e / r, l = e % r;
+        s.Ut[i][l] = (T)RA[i * rs + l];
     }
-    for (int e = tid; e < r * r; e += kSvdThreads) {
-        const int i = e / r, j = e % r;
-        s.Ut[i][j] = i == j ? 1.0 : 0.0;
+    __syncwarp();
+    for (int i = lane; i < r; i += 32) {
+        const TIN* rb = RB + (size_t)i * rs;
+        for (int j0 = 0; j0 < r; j0 += 4) {   // four columns of M at a time (independent chains)
+            T acc[4] = {0, 0, 0, 0};
+            for (int l = i; l < r; ++l) {
+                const T b = (T)rb[l];
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    if (j0 + q < r && l >= j0 + q) acc[q] = fma(b, s.Ut[j0 + q][l], acc[q]);
+            }
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                if (j0 + q < r) s.M[i][j0 + q] = acc[q];
+        }
     }
-    __syncthreads();
+    __syncwarp();
+    for (int e = lane; e < r * r; e += 32) {
+        const int i = e / r, l = e % r;
+        s.Ut[i][l] = i == l ? T(1) : T(0);
+    }
+    __syncwarp();
 
     const int rp = (r + 1) & ~1;  // even number of players (index r is a bye when r is odd)
-    const double tol = 1e-15;
+    const T tol = svd_tol<T>(r);
     for (int sweep = 0; sweep < a.max_sweeps; ++sweep) {
-        if (tid == 0) s.rot = 0;
-        __syncthreads();
+        bool rot = false;
         for (int t = 0; t < rp - 1; ++t) {
-            for (int pi = warp; pi < rp / 2; pi += NW) {
+            if (lane < rp / 2) {
                 int p, q;
-                if (pi == 0) {
+                if (lane == 0) {
                     p = rp - 1;
                     q = t;
                 } else {
-                    p = (t + pi) % (rp - 1);
-                    q = (t - pi + rp - 1) % (rp - 1);
+                    p = (t + lane) % (rp - 1);
+                    q = (t - lane + rp - 1) % (rp - 1);
                 }
-                if (p >= r || q >= r) continue;
-                double al = 0, be = 0, ga = 0;
-                for (int l = lane; l < r; l += 32) {
-                    const double x = s.M[p][l], y = s.M[q][l];
-                    al += x * x;
-                    be += y * y;
-                    ga += x * y;
+                if (p < r && q < r) {
+                    T al0 = 0, al1 = 0, be0 = 0, be1 = 0, ga0 = 0, ga1 = 0;
+                    int l = 0;
+                    for (; l + 1 < r; l += 2) {
+                        const T x0 = s.M[p][l], y0 = s.M[q][l], x1 = s.M[p][l + 1], y1 = s.M[q][l + 1];
+                        al0 = fma(x0, x0, al0); be0 = fma(y0, y0, be0); ga0 = fma(x0, y0, ga0);
+                        al1 = fma(x1, x1, al1); be1 = fma(y1, y1, be1); ga1 = fma(x1, y1, ga1);
+                    }
+                    if (l < r) {
+                        const T x0 = s.M[p][l], y0 = s.M[q][l];
+                        al0 = fma(x0, x0, al0); be0 = fma(y0, y0, be0); ga0 = fma(x0, y0, ga0);
+                    }
+                    const T al = al0 + al1, be = be0 + be1, ga = ga0 + ga1;
+                    if (ga != T(0) && fabs(ga) > tol * sqrt(al * be)) {
+                        rot = true;
+                        const T zeta = (be - al) / (T(2) * ga);
+                        const T tt = (zeta >= T(0) ? T(1) : T(-1)) / (fabs(zeta) + sqrt(T(1) + zeta * zeta));
+                        const T c = T(1) / sqrt(T(1) + tt * tt);
+                        const T sn = c * tt;
+                        for (int k = 0; k < r; ++k) {
+                            const T x = s.M[p][k], y = s.M[q][k];
+                            s.M[p][k] = c * x - sn * y;
+                            s.M[q][k] = sn * x + c * y;
+                            const T u = s.Ut[p][k], v = s.Ut[q][k];
+                            s.Ut[p][k] = c * u - sn * v;
+                            s.Ut[q][k] = sn * u + c * v;
+                        }
+                    }
                 }
-                al = warp_sum(al);
-                be = warp_sum(be);
-                ga = warp_sum(ga);
-                if (ga == 0.0 || fabs(ga) <= tol * sqrt(al * be)) continue;
-                const double zeta = (be - al) / (2.0 * ga);
-                const double tt = (zeta >= 0 ? 1.0 : -1.0) / (fabs(zeta) + sqrt(1.0 + zeta * zeta));
-                const double c = 1.0 / sqrt(1.0 + tt * tt);
-                const double sn = c * tt;
-                for (int l = lane; l < r; l += 32) {
-                    const double x = s.M[p][l], y = s.M[q][l];
-                    s.M[p][l] = c * x - sn * y;
-                    s.M[q][l] = sn * x + c * y;
-                    const double u = s.Ut[p][l], v = s.Ut[q][l];
-                    s.Ut[p][l] = c * u - sn * v;
-                    s.Ut[q][l] = sn * u + c * v;
-                }
-                if (lane == 0) s.rot = 1;
             }
-            __syncthreads();
+            __syncwarp();
         }
-        const int any = s.rot;
-        __syncthreads();
-        if (!any) break;
+        if (!__any_sync(0xffffffffu, rot)) break;
     }
 
-    for (int p = warp; p < r; p += NW) {
-        double nn = 0;
-        for (int l = lane; l < r; l += 32) nn += s.M[p][l] * s.M[p][l];
-        nn = warp_sum(nn);
-        if (lane == 0) s.sig[p] = sqrt(nn);
+    for (int p = lane; p < r; p += 32) {
+        T nn = 0;
+        for (int l = 0; l < r; ++l) nn = fma(s.M[p][l], s.M[p][l], nn);
+        s.sig[p] = sqrt(nn);
     }
-    __syncthreads();
-    // descending order, ties by index
-    for (int p = tid; p < r; p += kSvdThreads) {
-        const double sp = s.sig[p];
+    __syncwarp();
+    for (int p = lane; p < r; p += 32) {  // descending, ties by index
+        const T sp = s.sig[p];
         int rank = 0;
         for (int q = 0; q < r; ++q) {
-            const double sq = s.sig[q];
+            const T sq = s.sig[q];
             rank += (sq > sp) || (sq == sp && q < p);
         }
         s.perm[rank] = p;
-        if (!isfinite(sp)) latch_error(LF_ERR_NUMERIC);
+        if (!isfinite((double)sp)) latch_error(LF_ERR_NUMERIC);
     }
-    __syncthreads();
+    __syncwarp();
     double* sg = a.sigma + (size_t)local * rs;
-    for (int j = tid; j < rs; j += kSvdThreads) sg[j] = j < r ? s.sig[s.perm[j]] : 0.0;
+    for (int j = lane; j < rs; j += 32) sg[j] = j < r ? (double)s.sig[s.perm[j]] : 0.0;
     if (a.U) {
         double* Uo = a.U + (size_t)local * rs * rs;
-        for (int e = tid; e < rs * rs; e += kSvdThreads) {
+        for (int e = lane; e < rs * rs; e += 32) {
             const int row = e / rs, j = e % rs;
-            Uo[e] = (row < r && j < r) ? s.Ut[s.perm[j]][row] : 0.0;
+            Uo[e] = (row < r && j < r) ? (double)s.Ut[s.perm[j]][row] : 0.0;
         }
     }
     if (a.V) {
         double* Vo = a.V + (size_t)local * rs * rs;
-        for (int e = tid; e < rs * rs; e += kSvdThreads) {
+        for (int e = lane; e < rs * rs; e += 32) {
             const int row = e / rs, j = e % rs;
             double v = 0.0;
             if (row < r && j < r) {
                 const int p = s.perm[j];
-                const double sp = s.sig[p];
-                v = sp > 0.0 ? s.M[p][row] / sp : 0.0;
+                const double sp = (double)s.sig[p];
+                v = sp > 0.0 ? (double)s.M[p][row] / sp : 0.0;
             }
             Vo[e] = v;
         }
