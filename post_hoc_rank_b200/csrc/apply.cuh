@@ -10,6 +10,7 @@
 // at their retained ranks, without padding.
 #pragma once
 #include "common.cuh"
+#include "prefill_tc.cuh"
 
 namespace lf {
 
@@ -21,8 +22,12 @@ constexpr int kGemvCols = kGemvThreads * 8;   // d_out columns per CTA
 struct Seg {
     int32_t adapter, start, len;
 };
+// Self-contained work item (64 bytes): everything a shrink/expand CTA needs, so it
+// starts its data loads after one dependent read.
 struct GemvItem {
-    int32_t seg, tok0, ntok, pad;
+    int32_t adapter, k, ntok, tok0;   // tok0: position of the first token in the permutation
+    int64_t oa, ob;                   // element offsets of A' and B'^T in the pools
+    int32_t tok[kGemvTok];            // token indices
 };
 
 struct RouteOut {
@@ -31,6 +36,14 @@ struct RouteOut {
     int32_t* perm;       // T
     GemvItem* items;     // T / kGemvTok + min(T, n_adapters)
     int32_t* seg_out;    // optional caller copy
+    // per-adapter rank table of this projection, used to fill and validate items
+    const int32_t* ranks;
+    const int64_t* off_A;
+    const int64_t* off_Bt;
+    int64_t pool_A, pool_Bt;
+    int32_t d_in, d_out;
+    TcItem* tc_items;    // T / kTcM + min(T, n_adapters) + 1
+    int32_t tc_enable;   // segments with >= kTcMin tokens become tensor-core items
 };
 
 // Block-wide exclusive scan of one int per thread (blockDim.x == kRouteThreads).
@@ -71,7 +84,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const int32_t* __r
     int32_t* segidx = rsm + n_adapters;  // n_adapters: segment index of each adapter
     __shared__ int32_t wbase[32][32];
     __shared__ int wsum[32];
-    __shared__ int s_carry[3];
+    __shared__ int s_carry[4];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     for (int a = tid; a < n_adapters; a += kRouteThreads) cnt[a] = 0;
     __syncthreads();
@@ -80,24 +93,57 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const int32_t* __r
         if (a < -1 || a >= n_adapters) latch_error(LF_ERR_BAD_INDEX);
         else if (a >= 0) atomicAdd(&cnt[a], 1);
     }
-    if (tid == 0) s_carry[0] = s_carry[1] = s_carry[2] = 0;
+    if (tid == 0) s_carry[0] = s_carry[1] = s_carry[2] = s_carry[3] = 0;
     __syncthreads();
     // scans over adapters in chunks of kRouteThreads: token start, segment index, item index
     for (int a0 = 0; a0 < n_adapters; a0 += kRouteThreads) {
         const int a = a0 + tid;
         const int c = a < n_adapters ? cnt[a] : 0;
-        const int ni = (c + kGemvTok - 1) / kGemvTok;
-        int tt, ts, ti;
+        const bool use_tc = o.tc_enable && c >= kTcMin;
+        const int ni = use_tc ? 0 : (c + kGemvTok - 1) / kGemvTok;
+        const int nti = use_tc ? (c + kTcM - 1) / kTcM : 0;
+        int tt, ts, ti, tq;
         const int start = block_excl_scan(c, wsum, &tt) + s_carry[0];
         const int sidx = block_excl_scan(c > 0 ? 1 : 0, wsum, &ts) + s_carry[1];
         const int iidx = block_excl_scan(ni, wsum, &ti) + s_carry[2];
+        const int qidx = block_excl_scan(nti, wsum, &tq) + s_carry[3];
         if (a < n_adapters) {
             cnt[a] = start;
             segidx[a] = sidx;
             if (c > 0) {
                 o.segs[sidx] = Seg{a, start, c};
-                for (int q = 0; q < ni; ++q)
-                    o.items[iidx + q] = GemvItem{sidx, q * kGemvTok, min(kGemvTok, c - q * kGemvTok), 0};
+                int k = o.ranks[a];
+                const int64_t oa = o.off_A[a], ob = o.off_Bt[a];
+                int err = 0;
+                if (k > kMaxRank) err = LF_ERR_SHAPE;
+                else if (k > 0 && ((oa & 7) || (ob & 7))) err = LF_ERR_ALIGNMENT;
+                else if (k > 0 && (oa < 0 || ob < 0 || oa + (int64_t)k * o.d_in > o.pool_A ||
+                                   ob + (int64_t)k * o.d_out > o.pool_Bt))
+                    err = LF_ERR_WORKSPACE;
+                if (err) {
+                    latch_error(err);
+                    k = 0;   // the adapter's tokens are left untouched
+                }
+                for (int q = 0; q < nti; ++q) {
+                    TcItem ti2;
+                    ti2.adapter = a;
+                    ti2.k = k < 0 ? 0 : k;
+                    ti2.ntok = min(kTcM, c - q * kTcM);
+                    ti2.tok0 = start + q * kTcM;
+                    ti2.oa = oa;
+                    ti2.ob = ob;
+                    o.tc_items[qidx + q] = ti2;
+                }
+                for (int q = 0; q < ni; ++q) {
+                    GemvItem it;
+                    it.adapter = a;
+                    it.k = k < 0 ? 0 : k;
+                    it.ntok = min(kGemvTok, c - q * kGemvTok);
+                    it.tok0 = start + q * kGemvTok;
+                    it.oa = oa;
+                    it.ob = ob;
+                    o.items[iidx + q] = it;
+                }
             }
         }
         __syncthreads();
@@ -105,6 +151,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const int32_t* __r
             s_carry[0] += tt;
             s_carry[1] += ts;
             s_carry[2] += ti;
+            s_carry[3] += tq;
         }
         __syncthreads();
     }
@@ -113,10 +160,28 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const int32_t* __r
         o.counts[0] = nseg;
         o.counts[1] = nval;
         o.counts[2] = s_carry[2];
+        o.counts[3] = s_carry[3];
+    }
+    if (T <= kRouteThreads) {
+        // small batch: rank = number of earlier tokens with the same id (ids staged in smem)
+        __shared__ int32_t s_ids[kRouteThreads];
+        int a = -1;
+        if (tid < T) {
+            a = ids[tid];
+            if (a < -1 || a >= n_adapters) a = -1;
+            s_ids[tid] = a;
+        }
+        __syncthreads();
+        if (a >= 0) {
+            int rank = 0;
+            for (int t2 = 0; t2 < tid; ++t2) rank += (s_ids[t2] == a);
+            o.perm[cnt[a] + rank] = tid;
+        }
+        __syncthreads();
     }
     // stable scatter, chunk by chunk; warps take their turn in token order
     const int nwarps_live = min(kRouteThreads / 32, (T + 31) / 32);
-    for (int base = 0; base < T; base += kRouteThreads) {
+    for (int base = 0; T > kRouteThreads && base < T; base += kRouteThreads) {
         const int t = base + tid;
         int a = t < T ? ids[t] : -1;
         if (a < -1 || a >= n_adapters) a = -1;
@@ -132,6 +197,13 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const int32_t* __r
         }
         if (a >= 0) o.perm[wbase[warp][leader] + rank] = t;
         __syncthreads();
+    }
+    __syncthreads();
+    for (int it = tid; it < s_carry[2]; it += kRouteThreads) {
+        GemvItem& g = o.items[it];
+        const int n = g.ntok, p0 = g.tok0;
+#pragma unroll
+        for (int q = 0; q < kGemvTok; ++q) g.tok[q] = q < n ? o.perm[p0 + q] : 0;
     }
     if (o.seg_out) {
         if (tid == 0) {
@@ -175,28 +247,14 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4& u, float* f) {
     }
 }
 
-__device__ __forceinline__ bool item_ok(const GemvArgs& a, int it, GemvItem& item, Seg& sg, int& k, int64_t& oa,
-                                        int64_t& ob, bool report) {
-    if (it >= a.counts[2]) return false;
+__device__ __forceinline__ bool item_ok(const GemvArgs& a, int it, GemvItem& item) {
+    const int n_items = a.counts[2];
+    if (it >= n_items) return false;
     item = a.items[it];
-    sg = a.segs[item.seg];
-    k = a.ranks[sg.adapter];
-    if (k <= 0) return false;
-    oa = a.off_A[sg.adapter];
-    ob = a.off_Bt[sg.adapter];
-    int err = 0;
-    if (k > kMaxRank) err = LF_ERR_SHAPE;
-    else if ((oa & 7) || (ob & 7)) err = LF_ERR_ALIGNMENT;
-    else if (oa < 0 || ob < 0 || oa + (int64_t)k * a.d_in > a.pool_A || ob + (int64_t)k * a.d_out > a.pool_Bt)
-        err = LF_ERR_WORKSPACE;
-    if (err) {
-        if (report && threadIdx.x == 0) latch_error(err);
-        return false;
-    }
-    return true;
+    return item.k > 0;
 }
 
-constexpr int kShrinkJ = 8;   // rows of A' per pass
+constexpr int kShrinkJ = 4;   // rows of A' per pass
 
 // Shrink: t[item][q][j] = A'_a[j] . x[tok_q] (fp32), one CTA per work item.  The
 // d_in range is split across all warps so each warp keeps many 16-byte loads in
@@ -204,14 +262,14 @@ constexpr int kShrinkJ = 8;   // rows of A' per pass
 __global__ void __launch_bounds__(kGemvThreads) shrink_kernel(GemvArgs a) {
     __shared__ float part[kGemvThreads / 32][kShrinkJ][kGemvTok];
     __shared__ int32_t toks[kGemvTok];
-    GemvItem item; Seg sg; int k; int64_t oa, ob;
-    if (!item_ok(a, blockIdx.x, item, sg, k, oa, ob, true)) return;
-    const int nt = item.ntok;
+    GemvItem item;
+    if (!item_ok(a, blockIdx.x, item)) return;
+    const int nt = item.ntok, k = item.k;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    if (tid < nt) toks[tid] = a.perm[sg.start + item.tok0 + tid];
+    if (tid < nt) toks[tid] = a.items[blockIdx.x].tok[tid];
     __syncthreads();
-    const __nv_bfloat16* Ap = a.A_pool + oa;
-    float* tout = a.t_buf + (size_t)(sg.start + item.tok0) * kMaxRank;
+    const __nv_bfloat16* Ap = a.A_pool + item.oa;
+    float* tout = a.t_buf + (size_t)item.tok0 * kMaxRank;
     for (int j0 = 0; j0 < k; j0 += kShrinkJ) {
         float acc[kShrinkJ][kGemvTok];
 #pragma unroll
@@ -238,12 +296,15 @@ __global__ void __launch_bounds__(kGemvThreads) shrink_kernel(GemvArgs a) {
                 }
             }
         }
+        const int nj = min(kShrinkJ, k - j0);   // block-uniform bounds: reduce live slots only
 #pragma unroll
         for (int jj = 0; jj < kShrinkJ; ++jj)
 #pragma unroll
             for (int q = 0; q < kGemvTok; ++q) {
-                const float v = warp_sum(acc[jj][q]);
-                if (lane == 0) part[warp][jj][q] = v;
+                if (jj < nj && q < nt) {
+                    const float v = warp_sum(acc[jj][q]);
+                    if (lane == 0) part[warp][jj][q] = v;
+                }
             }
         __syncthreads();
         if (tid < kShrinkJ * kGemvTok) {
@@ -262,17 +323,127 @@ __global__ void __launch_bounds__(kGemvThreads) shrink_kernel(GemvArgs a) {
 __global__ void __launch_bounds__(kGemvThreads) expand_kernel(GemvArgs a) {
     __shared__ float tsm[kGemvTok][kMaxRank];
     __shared__ int32_t toks[kGemvTok];
-    GemvItem item; Seg sg; int k; int64_t oa, ob;
-    if (!item_ok(a, blockIdx.x, item, sg, k, oa, ob, false)) return;
-    const int nt = item.ntok;
+    GemvItem item;
+    if (!item_ok(a, blockIdx.x, item)) return;
+    const int nt = item.ntok, k = item.k;
+    const int64_t ob = item.ob;
     const int tid = threadIdx.x;
-    if (tid < nt) toks[tid] = a.perm[sg.start + item.tok0 + tid];
-    const float* tin = a.t_buf + (size_t)(sg.start + item.tok0) * kMaxRank;
+    if (tid < nt) toks[tid] = a.items[blockIdx.x].tok[tid];
+    const float* tin = a.t_buf + (size_t)item.tok0 * kMaxRank;
     for (int e = tid; e < nt * kMaxRank; e += kGemvThreads) {
         const int q = e / kMaxRank, j = e % kMaxRank;
         tsm[q][j] = j < k ? tin[e] : 0.f;
     }
     __syncthreads();
+    const int e = blockIdx.y * kGemvCols + tid * 8;
+    if (e >= a.d_out) return;
+    float acc[kGemvTok][8];
+#pragma unroll
+    for (int q = 0; q < kGemvTok; ++q)
+#pragma unroll
+        for (int c = 0; c < 8; ++c) acc[q][c] = 0.f;
+    const __nv_bfloat16* Bt = a.Bt_pool + ob + e;
+#pragma unroll 4
+    for (int j = 0; j < k; ++j) {
+        float bf[8];
+        bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(Bt + (int64_t)j * a.d_out)), bf);
+#pragma unroll
+        for (int q = 0; q < kGemvTok; ++q) {
+            if (q < nt) {
+                const float tv = tsm[q][j];
+#pragma unroll
+                for (int c = 0; c < 8; ++c) acc[q][c] = fmaf(tv, bf[c], acc[q][c]);
+            }
+        }
+    }
+#pragma unroll
+    for (int q = 0; q < kGemvTok; ++q) {
+        if (q < nt) {
+            __nv_bfloat16* yp = a.y + (int64_t)toks[q] * a.d_out + e;
+            float yf[8];
+            uint4 u = *reinterpret_cast<const uint4*>(yp);
+            bf16x8_to_f32(u, yf);
+            __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&u);
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+                h[c] = __floats2bfloat162_rn(fmaf(a.scale, acc[q][2 * c], yf[2 * c]),
+                                             fmaf(a.scale, acc[q][2 * c + 1], yf[2 * c + 1]));
+            *reinterpret_cast<uint4*>(yp) = u;
+        }
+    }
+}
+
+
+// Decode regime (few tokens per adapter): one launch does shrink and expand.  CTA
+// (item, d_out chunk): all warps share the dot products of each A' row over d_in
+// (16-byte loads issued together), t is reduced in a fixed order in shared memory,
+// then the CTA updates its d_out slice of y.  CTAs of one item in different chunks
+// recompute the same t (identical arithmetic, A' and x served from L2).
+__global__ void __launch_bounds__(kGemvThreads) fused_gemv_kernel(GemvArgs a) {
+    __shared__ float part[kGemvThreads / 32][kShrinkJ][kGemvTok];
+    __shared__ float tsm[kGemvTok][kMaxRank];
+    __shared__ int32_t toks[kGemvTok];
+    GemvItem item;
+    if (!item_ok(a, blockIdx.x, item)) return;
+    const int nt = item.ntok, k = item.k;
+    const int64_t ob = item.ob;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    if (tid < nt) toks[tid] = a.items[blockIdx.x].tok[tid];
+    __syncthreads();
+    const __nv_bfloat16* Ap = a.A_pool + item.oa;
+    for (int j0 = 0; j0 < k; j0 += kShrinkJ) {
+        const int nj = min(kShrinkJ, k - j0);
+        float acc[kShrinkJ][kGemvTok];
+#pragma unroll
+        for (int jj = 0; jj < kShrinkJ; ++jj)
+#pragma unroll
+            for (int q = 0; q < kGemvTok; ++q) acc[jj][q] = 0.f;
+        for (int d0 = tid * 8; d0 < a.d_in; d0 += kGemvThreads * 8) {
+            uint4 xr[kGemvTok], ar[kShrinkJ];
+#pragma unroll
+            for (int q = 0; q < kGemvTok; ++q)
+                if (q < nt) xr[q] = __ldg(reinterpret_cast<const uint4*>(a.x + (int64_t)toks[q] * a.d_in + d0));
+#pragma unroll
+            for (int jj = 0; jj < kShrinkJ; ++jj)
+                if (jj < nj) ar[jj] = __ldg(reinterpret_cast<const uint4*>(Ap + (int64_t)(j0 + jj) * a.d_in + d0));
+#pragma unroll
+            for (int jj = 0; jj < kShrinkJ; ++jj) {
+                if (jj < nj) {
+                    float af[8];
+                    bf16x8_to_f32(ar[jj], af);
+#pragma unroll
+                    for (int q = 0; q < kGemvTok; ++q) {
+                        if (q < nt) {
+                            float xf[8];
+                            bf16x8_to_f32(xr[q], xf);
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) acc[jj][q] = fmaf(af[e], xf[e], acc[jj][q]);
+                        }
+                    }
+                }
+            }
+        }
+#pragma unroll
+        for (int jj = 0; jj < kShrinkJ; ++jj)
+#pragma unroll
+            for (int q = 0; q < kGemvTok; ++q) {
+                if (jj < nj && q < nt) {
+                    const float v = warp_sum(acc[jj][q]);
+                    if (lane == 0) part[warp][jj][q] = v;
+                }
+            }
+        __syncthreads();
+        if (tid < kShrinkJ * kGemvTok) {
+            const int jj = tid / kGemvTok, q = tid % kGemvTok;
+            if (jj < nj && q < nt) {
+                float v = 0.f;
+#pragma unroll
+                for (int w = 0; w < kGemvThreads / 32; ++w) v += part[w][jj][q];
+                tsm[q][j0 + jj] = v;
+            }
+        }
+        __syncthreads();
+    }
     const int e = blockIdx.y * kGemvCols + tid * 8;
     if (e >= a.d_out) return;
     float acc[kGemvTok][8];

@@ -26,6 +26,61 @@ __device__ __forceinline__ T warp_sum(T v) {
     return v;
 }
 
+// Packed fp32 FMA on sm_100 (two lanes of fp32 per instruction): d = a * b + c elementwise.
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+    unsigned long long d;
+    const unsigned long long A = *reinterpret_cast<const unsigned long long*>(&a);
+    const unsigned long long B = *reinterpret_cast<const unsigned long long*>(&b);
+    const unsigned long long C = *reinterpret_cast<const unsigned long long*>(&c);
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(A), "l"(B), "l"(C));
+    return *reinterpret_cast<const float2*>(&d);
+}
+
+// ---- shared-memory async copies (TMA bulk engine) and mbarriers -------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+// make mbarrier initialisation visible to the async (bulk copy) proxy
+__device__ __forceinline__ void fence_barrier_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+// 1-D bulk copy global -> shared, completion counted on `bar` (16-byte aligned, size % 16 == 0)
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar))
+                 : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// Bounded wait on an mbarrier phase: gives up after 2^25 polls or ~2e9 SM cycles
+// (about a second), latches LF_ERR_TIMEOUT and returns false.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const long long t0 = clock64();
+    for (int i = 0; i < (1 << 25); ++i) {
+        if (mbar_try_wait(bar, parity)) return true;
+        __nanosleep(32);
+        if ((i & 1023) == 1023 && clock64() - t0 > 2000000000ll) break;
+    }
+    latch_error(LF_ERR_TIMEOUT);
+    return false;
+}
+
 // Carves caller workspace into aligned sub-buffers; tracks the bytes needed.
 struct Carver {
     char* base;

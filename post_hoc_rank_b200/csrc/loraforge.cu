@@ -642,6 +642,8 @@ size_t lf_apply_workspace_size(int32_t T, int32_t n_adapters) {
     c.take<int32_t>((size_t)std::max(T, 1));
     c.take<GemvItem>((size_t)(T / kGemvTok + mseg + 1));
     c.take<float>((size_t)std::max(T, 1) * kMaxRank);
+    c.take<TcItem>((size_t)(T / kTcM + mseg + 1));
+    c.take<float>((size_t)kTcMaxSplit * std::max(T, 1) * kMaxRank);
     return c.off + 256;
 }
 
@@ -662,13 +664,24 @@ lf_status lf_lora_shrink_expand(int32_t T, int32_t d_in, int32_t d_out, const vo
     const int64_t mseg = std::min<int64_t>(T, n_adapters);
     char* wsa = reinterpret_cast<char*>(align_up((int64_t)reinterpret_cast<uintptr_t>(ws), 256));
     Carver c(wsa);
-    RouteOut o;
+    RouteOut o{};
     o.counts = c.take<int32_t>(4);
     o.segs = c.take<Seg>((size_t)std::max<int64_t>(mseg, 1));
     o.perm = c.take<int32_t>((size_t)T);
     o.items = c.take<GemvItem>((size_t)(T / kGemvTok + mseg + 1));
     float* t_buf = c.take<float>((size_t)T * kMaxRank);
+    o.tc_items = c.take<TcItem>((size_t)(T / kTcM + mseg + 1));
+    float* t_part = c.take<float>((size_t)kTcMaxSplit * T * kMaxRank);
     o.seg_out = seg_out;
+    o.ranks = ranks;
+    o.off_A = off_A;
+    o.off_Bt = off_Bt;
+    o.pool_A = pool_elems_A;
+    o.pool_Bt = pool_elems_Bt;
+    o.d_in = d_in;
+    o.d_out = d_out;
+    const bool decode_regime = (int64_t)T <= (int64_t)kGemvTok * n_adapters;
+    o.tc_enable = decode_regime ? 0 : 1;
     const size_t rsmem = 2 * (size_t)n_adapters * sizeof(int32_t);
     LF_CUDA_TRY(cudaFuncSetAttribute(route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rsmem));
     LF_LAUNCH("route", route_kernel, 1, kRouteThreads, rsmem, s, ids, T, n_adapters, o);
@@ -692,9 +705,38 @@ lf_status lf_lora_shrink_expand(int32_t T, int32_t d_in, int32_t d_out, const vo
     g.items = o.items;
     g.t_buf = t_buf;
     const unsigned max_items = (unsigned)(T / kGemvTok + mseg + 1);
+    const dim3 grid2(max_items, (unsigned)cdiv(d_out, kGemvCols));
+    if (decode_regime) {
+        // few tokens per adapter: shrink and expand in one launch
+        LF_LAUNCH("fused_gemv", fused_gemv_kernel, grid2, kGemvThreads, 0, s, g);
+        return launch_status();
+    }
     LF_LAUNCH("shrink_gemv", shrink_kernel, max_items, kGemvThreads, 0, s, g);
     LF_CUDA_TRY(cudaGetLastError());
-    LF_LAUNCH("expand_gemv", expand_kernel, dim3(max_items, (unsigned)cdiv(d_out, kGemvCols)), kGemvThreads, 0, s, g);
+    LF_LAUNCH("expand_gemv", expand_kernel, grid2, kGemvThreads, 0, s, g);
+    LF_CUDA_TRY(cudaGetLastError());
+    // segments with >= kTcMin tokens: tcgen05 shrink, then expand
+    TcArgs ta;
+    ta.d_in = d_in;
+    ta.d_out = d_out;
+    ta.x = g.x;
+    ta.y = g.y;
+    ta.A_pool = g.A_pool;
+    ta.Bt_pool = g.Bt_pool;
+    ta.scale = scale;
+    ta.counts = o.counts;
+    ta.items = o.tc_items;
+    ta.perm = o.perm;
+    ta.t_part = t_part;
+    ta.T = T;
+    const unsigned max_tc = (unsigned)(T / kTcM + mseg + 1);
+    const unsigned nsplit = (unsigned)cdiv(d_in, tc_split_len(d_in));
+    LF_CUDA_TRY(cudaFuncSetAttribute(shrink_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kShrinkTcSmem));
+    LF_CUDA_TRY(cudaFuncSetAttribute(expand_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kExpandTcSmem));
+    LF_LAUNCH("shrink_tc", shrink_tc_kernel, dim3(max_tc, nsplit), kTcThreads, kShrinkTcSmem, s, ta);
+    LF_CUDA_TRY(cudaGetLastError());
+    LF_LAUNCH("expand_tc", expand_tc_kernel, dim3(max_tc, (unsigned)cdiv(d_out, kTcCols)), kTcThreads, kExpandTcSmem, s,
+              ta);
     return launch_status();
 }
 
@@ -716,13 +758,22 @@ lf_status lf_lora_shrink_expand_noalloc(int32_t T, int32_t d_in, int32_t d_out, 
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     // same carve as a caller workspace sized for the maxima (fits kNoallocScratchBytes)
     Carver c(scratch);
-    RouteOut o;
+    RouteOut o{};
     o.counts = c.take<int32_t>(4);
     o.segs = c.take<Seg>((size_t)LF_NOALLOC_MAX_ADAPTERS);
     o.perm = c.take<int32_t>((size_t)LF_NOALLOC_MAX_TOKENS);
     o.items = c.take<GemvItem>((size_t)LF_NOALLOC_MAX_TOKENS / kGemvTok + LF_NOALLOC_MAX_ADAPTERS + 1);
     float* t_buf = c.take<float>((size_t)LF_NOALLOC_MAX_TOKENS * kMaxRank);
     o.seg_out = seg_out;
+    o.ranks = ranks;
+    o.off_A = off_A;
+    o.off_Bt = off_Bt;
+    o.pool_A = pool_elems_A;
+    o.pool_Bt = pool_elems_Bt;
+    o.d_in = d_in;
+    o.d_out = d_out;
+    o.tc_items = nullptr;
+    o.tc_enable = 0;   // this entry point keeps every segment on the GEMV kernels
     if (c.off > kNoallocScratchBytes) return LF_ERR_WORKSPACE;
     const int64_t mseg = std::min<int64_t>(T, n_adapters);
     const size_t rsmem = 2 * (size_t)n_adapters * sizeof(int32_t);
@@ -748,9 +799,15 @@ lf_status lf_lora_shrink_expand_noalloc(int32_t T, int32_t d_in, int32_t d_out, 
     g.items = o.items;
     g.t_buf = t_buf;
     const unsigned max_items = (unsigned)(T / kGemvTok + mseg + 1);
-    LF_LAUNCH("shrink_gemv", shrink_kernel, max_items, kGemvThreads, 0, s, g);
-    LF_CUDA_TRY(cudaGetLastError());
-    LF_LAUNCH("expand_gemv", expand_kernel, dim3(max_items, (unsigned)cdiv(d_out, kGemvCols)), kGemvThreads, 0, s, g);
+    const dim3 grid2(max_items, (unsigned)cdiv(d_out, kGemvCols));
+    if ((int64_t)T <= (int64_t)kGemvTok * n_adapters) {
+        // decode regime (few tokens per adapter): shrink and expand in one launch
+        LF_LAUNCH("fused_gemv", fused_gemv_kernel, grid2, kGemvThreads, 0, s, g);
+    } else {
+        LF_LAUNCH("shrink_gemv", shrink_kernel, max_items, kGemvThreads, 0, s, g);
+        LF_CUDA_TRY(cudaGetLastError());
+        LF_LAUNCH("expand_gemv", expand_kernel, grid2, kGemvThreads, 0, s, g);
+    }
     return launch_status();
 }
 

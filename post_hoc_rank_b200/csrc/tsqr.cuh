@@ -20,7 +20,7 @@
 
 namespace lf {
 
-constexpr int kTsqrChunk = 1024;   // rows per work item (one warp)
+constexpr int kTsqrChunk = 2048;   // rows per work item (one warp)
 constexpr int kTsqrTM = 32;        // rows per register tile
 // warps (independent work items) per CTA: the packed R of every warp lives in static
 // shared memory (fp32 RT=64: 8.3 KB per warp; fp64: 16.6 KB)
@@ -108,7 +108,7 @@ __device__ __forceinline__ void warp_absorb(T (&x)[Cols<RT>::NS][kTsqrTM], T* Rp
         for (int i = 0; i < kTsqrTM; i += VW) *reinterpret_cast<V*>(&v[i]) = reinterpret_cast<const V*>(vbuf)[i / VW];
         const T x0 = Rp[tri_off<RT>(j, j)];
         __syncwarp();
-        T s4[4] = {0, 0, 0, 0};
+        T s4[4] = {0, 0, 0, 0};   // every lane forms the column norm from its copy of v
 #pragma unroll
         for (int i = 0; i < kTsqrTM; ++i) s4[i & 3] = fma(v[i], v[i], s4[i & 3]);
         const T ss = (s4[0] + s4[1]) + (s4[2] + s4[3]);

@@ -74,8 +74,9 @@ def test_tiny_apply_and_routing():
 
 
 @pytest.mark.parametrize("d_in,d_out", [(4096, 1024), (1024, 14336), (3584, 512)])
-def test_ragged_ranks_zipf_with_unrouted_tokens(d_in, d_out):
-    T, n = 300, 37
+@pytest.mark.parametrize("n", [37, 64])   # 37: split shrink/expand path, 64: fused decode path
+def test_ragged_ranks_zipf_with_unrouted_tokens(d_in, d_out, n):
+    T = 300
     g = np.random.default_rng(5)
     ranks = g.integers(1, 65, size=n)
     ids = synth.zipf_ids(T, n, 1.0, (2, d_in))
