@@ -149,6 +149,9 @@ static void plan_tsqr(const lf_module* mods, int32_t n, TsqrPlan& p) {
                                           nch > 1 ? p.slots + c : -1});
             if (nch > 1) p.slots += nch;
         }
+    // longest chunks first: single-warp CTAs of similar length finish together
+    std::stable_sort(p.work.begin(), p.work.end(),
+                     [](const TsqrWork& a, const TsqrWork& b) { return a.nrows > b.nrows; });
 }
 
 struct TsqrLayout {

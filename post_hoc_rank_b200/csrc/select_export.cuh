@@ -365,7 +365,7 @@ __device__ void export_a_cols(const ExportArgs& a, const lf_module& md, int k, c
             for (int jj = 0; jj < kExpJ; ++jj)
 #pragma unroll
                 for (int c = 0; c < 4; ++c) acc[jj][c] = 0.f;
-#pragma unroll 8
+#pragma unroll 16
             for (int l = 0; l < r; ++l) {
                 float4 v;
                 const float* src = A + (int64_t)l * md.d_in + d;

@@ -23,9 +23,10 @@ namespace lf {
 constexpr int kTsqrChunk = 2048;   // rows per work item (one warp)
 constexpr int kTsqrTM = 32;        // rows per register tile
 // warps (independent work items) per CTA: the packed R of every warp lives in static
-// shared memory (fp32 RT=64: 8.3 KB per warp; fp64: 16.6 KB)
+// shared memory (fp32 RT=64: 8.3 KB per warp; fp64: 16.6 KB).  fp32 uses one warp
+// per CTA so a short chunk never holds a finished warp resident.
 template <typename T>
-__host__ __device__ constexpr int tsqr_warps() { return sizeof(T) == 8 ? 2 : 4; }
+__host__ __device__ constexpr int tsqr_warps() { return sizeof(T) == 8 ? 2 : 1; }
 
 struct TsqrWork {
     int32_t mf;      // 2 * local module index + factor (0 = B, 1 = A^T)
@@ -176,7 +177,7 @@ __device__ __forceinline__ void load_tri_rows(T (&x)[Cols<RT>::NS][kTsqrTM], con
 }
 
 template <typename T, int RT>
-__global__ void __launch_bounds__(32 * tsqr_warps<T>(), sizeof(T) == 4 ? 4 : 1) tsqr_kernel(TsqrArgs<T> a) {
+__global__ void __launch_bounds__(32 * tsqr_warps<T>(), sizeof(T) == 4 ? 16 : 1) tsqr_kernel(TsqrArgs<T> a) {
     constexpr int W = tsqr_warps<T>();
     __shared__ T s_R[W][tri_size<RT>()];
     __shared__ __align__(16) T s_v[W][kTsqrTM];
