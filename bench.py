@@ -127,6 +127,56 @@ def timed(fn, steps, sync_all, stream):
     return start.elapsed_time(end)
 
 
+
+# ------------------------------------------------------------- roofline
+# fp32 SIMT FMA peak from unit counts: 148 SMs x 128 fp32 lanes x 2 flop x SM clock.
+B200_SMS, FP32_LANES_PER_SM = 148, 128
+
+
+def alu_peak_tflops(sm_mhz):
+    return B200_SMS * FP32_LANES_PER_SM * 2 * (sm_mhz or 1965.0) * 1e6 / 1e12
+
+
+def kernel_traffic(kernel, units):
+    """DRAM bytes per launch from the committed ncu summary (profiles/traffic.json), scaled
+    by the units one launch processes; None when the kernel's source changed since."""
+    import hashlib
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    rec = json.load(open(p)).get(kernel)
+    if not rec:
+        return None
+    src = os.path.join(ROOT, rec["source"])
+    if not os.path.exists(src) or hashlib.sha256(open(src, "rb").read()).hexdigest() != rec["source_sha256"]:
+        return None
+    return int(rec["bytes_per_unit"] * units)
+
+
+def dominant_roofline(dom, per_launch_ms, fr, hbm, peak_kind, sm_mhz):
+    n = fr["n"]
+    if dom == "tsqr_leaf_merge":
+        # Householder QR of an m x r matrix: 2 m r^2 - 2 r^3 / 3 flop; both factors of every module
+        flops = fr["qr_flops"]
+        ach = flops / (per_launch_ms * 1e-3) / 1e12
+        peak = alu_peak_tflops(sm_mhz)
+        gbs = fr["bytes_in"] / (per_launch_ms * 1e-3) / 1e9
+        return {"kernel": dom, "bound": "alu", "achieved": round(ach, 2), "peak": round(peak, 1),
+                "unit": "TFLOP/s", "frac": round(ach / peak, 4), "traffic": kernel_traffic(dom, n),
+                "algo_flops": int(flops), "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 x SM clock",
+                "hbm": {"achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s", "frac": round(gbs / hbm, 4),
+                        "algo_bytes": int(fr["bytes_in"]), "peak_source": peak_kind}}
+    algo = {"export_stream": fr["bytes_in"] + fr["bytes_out"]}
+    b = algo.get(dom)
+    if b is None:
+        return {"kernel": dom, "bound": "alu", "achieved": None, "peak": None, "unit": None, "frac": None,
+                "traffic": None}
+    ach = b / (per_launch_ms * 1e-3) / 1e9
+    return {"kernel": dom, "bound": "hbm", "achieved": round(ach, 1), "peak": hbm, "unit": "GB/s",
+            "frac": round(ach / hbm, 4), "traffic": kernel_traffic(dom, n), "algo_bytes": int(b),
+            "peak_source": peak_kind}
+
+
 # ------------------------------------------------------------ factor path
 def factor_bench(args, rank, world, dev, sync_all, stream, hbm, peak_kind):
     import torch
@@ -164,7 +214,10 @@ def factor_bench(args, rank, world, dev, sync_all, stream, hbm, peak_kind):
     st = lf.lf_get_device_status(stream)
     ranks = E.ranks.cpu().numpy()
     inp, out, small = algo_bytes_factor(mods, ranks)
-    res = dict(ms=ms, launches=launches, phases=phases, clocks=clk.summary(), status=st, n=lay.n,
+    m_rows = (lay.d_out.astype(np.int64) + lay.d_in.astype(np.int64))
+    rr = lay.r.astype(np.int64)
+    qr_flops = float((2 * m_rows * rr * rr - 2 * (2 * rr ** 3) // 3).sum())
+    res = dict(ms=ms, launches=launches, phases=phases, clocks=clk.summary(), status=st, n=lay.n, qr_flops=qr_flops,
                bytes_in=inp, bytes_out=out, bytes_small=small, ranks_sum=int(ranks.sum()),
                params_frac=float((ranks.astype(np.int64) * (lay.d_in + lay.d_out)).sum() /
                                  (lay.r.astype(np.int64) * (lay.d_in + lay.d_out)).sum()))
@@ -430,17 +483,7 @@ def main():
     tot = {k: v[0] for k, v in ph.items()}
     dom = max(tot, key=tot.get)
     per_launch_ms = ph[dom][0] / max(ph[dom][1], 1)
-    algo = {"tsqr_leaf_merge": fr["bytes_in"] + fr["n"] * 2 * 4 * 64 * 64,
-            "export_stream": fr["bytes_in"] + fr["bytes_out"]}
-    dom_bytes = algo.get(dom)
-    roof = None
-    if dom_bytes is not None:
-        ach = dom_bytes / (per_launch_ms * 1e-3) / 1e9
-        roof = {"kernel": dom, "bound": "hbm", "achieved": round(ach, 1), "peak": hbm, "unit": "GB/s",
-                "frac": round(ach / hbm, 4), "traffic": None, "peak_source": peak_kind}
-    else:
-        roof = {"kernel": dom, "bound": "alu", "achieved": None, "peak": None, "unit": None, "frac": None,
-                "traffic": None}
+    roof = dominant_roofline(dom, per_launch_ms, fr, hbm, peak_kind, fr["clocks"].get("sm_mhz"))
     step_bytes_2touch = 2 * fr["bytes_in"] + fr["bytes_out"] + fr["bytes_small"]
     step_gbs = step_bytes_2touch / (ms_step * 1e-3) / 1e9
 

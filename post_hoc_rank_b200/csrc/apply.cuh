@@ -46,7 +46,7 @@ struct RouteOut {
     int32_t tc_enable;   // segments with >= kTcMin tokens become tensor-core items
 };
 
-// Block-wide exclusive scan of one int per thread (blockDim.x == kRouteThreads).
+// Block-wide exclusive scan of one int per thread (blockDim.x a multiple of 32, <= 1024).
 __device__ __forceinline__ int block_excl_scan(int v, int* wsum, int* total) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     int x = v;
@@ -58,7 +58,8 @@ __device__ __forceinline__ int block_excl_scan(int v, int* wsum, int* total) {
     if (lane == 31) wsum[warp] = x;
     __syncthreads();
     if (warp == 0) {
-        int w = wsum[lane];
+        const int nw = (int)(blockDim.x >> 5);
+        int w = lane < nw ? wsum[lane] : 0;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             const int y = __shfl_up_sync(0xffffffffu, w, o);
@@ -68,7 +69,7 @@ __device__ __forceinline__ int block_excl_scan(int v, int* wsum, int* total) {
     }
     __syncthreads();
     const int base = warp > 0 ? wsum[warp - 1] : 0;
-    const int tot = wsum[31];
+    const int tot = wsum[(blockDim.x >> 5) - 1];
     __syncthreads();
     if (total) *total = tot;
     return base + x - v;
@@ -86,9 +87,10 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const int32_t* __r
     __shared__ int wsum[32];
     __shared__ int s_carry[4];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    for (int a = tid; a < n_adapters; a += kRouteThreads) cnt[a] = 0;
+    const int nthr = (int)blockDim.x;
+    for (int a = tid; a < n_adapters; a += nthr) cnt[a] = 0;
     __syncthreads();
-    for (int t = tid; t < T; t += kRouteThreads) {
+    for (int t = tid; t < T; t += nthr) {
         const int a = ids[t];
         if (a < -1 || a >= n_adapters) latch_error(LF_ERR_BAD_INDEX);
         else if (a >= 0) atomicAdd(&cnt[a], 1);
@@ -96,7 +98,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const int32_t* __r
     if (tid == 0) s_carry[0] = s_carry[1] = s_carry[2] = s_carry[3] = 0;
     __syncthreads();
     // scans over adapters in chunks of kRouteThreads: token start, segment index, item index
-    for (int a0 = 0; a0 < n_adapters; a0 += kRouteThreads) {
+    for (int a0 = 0; a0 < n_adapters; a0 += nthr) {
         const int a = a0 + tid;
         const int c = a < n_adapters ? cnt[a] : 0;
         const bool use_tc = o.tc_enable && c >= kTcMin;
@@ -162,7 +164,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const int32_t* __r
         o.counts[2] = s_carry[2];
         o.counts[3] = s_carry[3];
     }
-    if (T <= kRouteThreads) {
+    if (T <= nthr) {
         // small batch: rank = number of earlier tokens with the same id (ids staged in smem)
         __shared__ int32_t s_ids[kRouteThreads];
         int a = -1;
@@ -180,8 +182,8 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const int32_t* __r
         __syncthreads();
     }
     // stable scatter, chunk by chunk; warps take their turn in token order
-    const int nwarps_live = min(kRouteThreads / 32, (T + 31) / 32);
-    for (int base = 0; T > kRouteThreads && base < T; base += kRouteThreads) {
+    const int nwarps_live = min(nthr / 32, (T + 31) / 32);
+    for (int base = 0; T > nthr && base < T; base += nthr) {
         const int t = base + tid;
         int a = t < T ? ids[t] : -1;
         if (a < -1 || a >= n_adapters) a = -1;
@@ -199,7 +201,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const int32_t* __r
         __syncthreads();
     }
     __syncthreads();
-    for (int it = tid; it < s_carry[2]; it += kRouteThreads) {
+    for (int it = tid; it < s_carry[2]; it += nthr) {
         GemvItem& g = o.items[it];
         const int n = g.ntok, p0 = g.tok0;
 #pragma unroll
@@ -210,12 +212,12 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const int32_t* __r
             o.seg_out[0] = nseg;
             o.seg_out[1] = nval;
         }
-        for (int s = tid; s < nseg; s += kRouteThreads) {
+        for (int s = tid; s < nseg; s += nthr) {
             o.seg_out[2 + 3 * s] = o.segs[s].adapter;
             o.seg_out[3 + 3 * s] = o.segs[s].start;
             o.seg_out[4 + 3 * s] = o.segs[s].len;
         }
-        for (int q = tid; q < nval; q += kRouteThreads) o.seg_out[2 + 3 * nseg + q] = o.perm[q];
+        for (int q = tid; q < nval; q += nthr) o.seg_out[2 + 3 * nseg + q] = o.perm[q];
     }
 }
 

@@ -213,6 +213,13 @@ static cudaError_t launch_svd_rt(int RT, const SvdArgs<TIN, T>& a, int n_items, 
     return launch_svd<TIN, T, 64>(a, n_items, st);
 }
 
+// Routing block size: enough threads for one pass over the batch and the adapters
+// (fewer warps make its block-wide barriers cheaper), at least 128, at most 1024.
+static int route_threads(int T, int n_adapters) {
+    const int need = std::max(T, n_adapters);
+    return need >= kRouteThreads ? kRouteThreads : std::max(128, (need + 31) / 32 * 32);
+}
+
 // ------------------------------------------------------------ groups (S scope)
 static void build_groups(const lf_module* mods, int32_t n, std::vector<int32_t>& ptr, std::vector<int32_t>& gm) {
     std::map<int32_t, std::vector<int32_t>> by;
@@ -226,7 +233,7 @@ static void build_groups(const lf_module* mods, int32_t n, std::vector<int32_t>&
 }
 
 // ----------------------------------------------------------- export planning
-constexpr int kRefineChunk = 4096;
+constexpr int kRefineChunk = 1024;
 constexpr int kExportItem = 2048;
 
 struct ExportPlan {
@@ -687,7 +694,7 @@ lf_status lf_lora_shrink_expand(int32_t T, int32_t d_in, int32_t d_out, const vo
     o.tc_enable = decode_regime ? 0 : 1;
     const size_t rsmem = 2 * (size_t)n_adapters * sizeof(int32_t);
     LF_CUDA_TRY(cudaFuncSetAttribute(route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rsmem));
-    LF_LAUNCH("route", route_kernel, 1, kRouteThreads, rsmem, s, ids, T, n_adapters, o);
+    LF_LAUNCH("route", route_kernel, 1, route_threads(T, n_adapters), rsmem, s, ids, T, n_adapters, o);
     LF_CUDA_TRY(cudaGetLastError());
     GemvArgs g;
     g.d_in = d_in;
@@ -781,7 +788,7 @@ lf_status lf_lora_shrink_expand_noalloc(int32_t T, int32_t d_in, int32_t d_out, 
     const int64_t mseg = std::min<int64_t>(T, n_adapters);
     const size_t rsmem = 2 * (size_t)n_adapters * sizeof(int32_t);
     LF_CUDA_TRY(cudaFuncSetAttribute(route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rsmem));
-    LF_LAUNCH("route", route_kernel, 1, kRouteThreads, rsmem, s, ids, T, n_adapters, o);
+    LF_LAUNCH("route", route_kernel, 1, route_threads(T, n_adapters), rsmem, s, ids, T, n_adapters, o);
     LF_CUDA_TRY(cudaGetLastError());
     GemvArgs g;
     g.d_in = d_in;

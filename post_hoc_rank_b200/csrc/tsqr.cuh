@@ -340,31 +340,59 @@ __global__ void __launch_bounds__(32 * svd_warps<T>()) svd_kernel(SvdArgs<TIN, T
                     q = (t - lane + rp - 1) % (rp - 1);
                 }
                 if (p < r && q < r) {
-                    T al0 = 0, al1 = 0, be0 = 0, be1 = 0, ga0 = 0, ga1 = 0;
+                    T al[4] = {0, 0, 0, 0}, be[4] = {0, 0, 0, 0}, ga[4] = {0, 0, 0, 0};
+                    const T* mp = s.M[p];
+                    const T* mq = s.M[q];
                     int l = 0;
-                    for (; l + 1 < r; l += 2) {
-                        const T x0 = s.M[p][l], y0 = s.M[q][l], x1 = s.M[p][l + 1], y1 = s.M[q][l + 1];
-                        al0 = fma(x0, x0, al0); be0 = fma(y0, y0, be0); ga0 = fma(x0, y0, ga0);
-                        al1 = fma(x1, x1, al1); be1 = fma(y1, y1, be1); ga1 = fma(x1, y1, ga1);
+                    for (; l + 3 < r; l += 4) {   // four independent chains per sum
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            const T x = mp[l + u], y = mq[l + u];
+                            al[u] = fma(x, x, al[u]);
+                            be[u] = fma(y, y, be[u]);
+                            ga[u] = fma(x, y, ga[u]);
+                        }
                     }
-                    if (l < r) {
-                        const T x0 = s.M[p][l], y0 = s.M[q][l];
-                        al0 = fma(x0, x0, al0); be0 = fma(y0, y0, be0); ga0 = fma(x0, y0, ga0);
+                    for (; l < r; ++l) {
+                        const T x = mp[l], y = mq[l];
+                        al[0] = fma(x, x, al[0]);
+                        be[0] = fma(y, y, be[0]);
+                        ga[0] = fma(x, y, ga[0]);
                     }
-                    const T al = al0 + al1, be = be0 + be1, ga = ga0 + ga1;
-                    if (ga != T(0) && fabs(ga) > tol * sqrt(al * be)) {
+                    const T alpha = (al[0] + al[1]) + (al[2] + al[3]);
+                    const T beta_ = (be[0] + be[1]) + (be[2] + be[3]);
+                    const T gamma = (ga[0] + ga[1]) + (ga[2] + ga[3]);
+                    if (gamma != T(0) && fabs(gamma) > tol * sqrt(alpha * beta_)) {
                         rot = true;
-                        const T zeta = (be - al) / (T(2) * ga);
+                        const T zeta = (beta_ - alpha) / (T(2) * gamma);
                         const T tt = (zeta >= T(0) ? T(1) : T(-1)) / (fabs(zeta) + sqrt(T(1) + zeta * zeta));
                         const T c = T(1) / sqrt(T(1) + tt * tt);
                         const T sn = c * tt;
-                        for (int k = 0; k < r; ++k) {
-                            const T x = s.M[p][k], y = s.M[q][k];
-                            s.M[p][k] = c * x - sn * y;
-                            s.M[q][k] = sn * x + c * y;
-                            const T u = s.Ut[p][k], v = s.Ut[q][k];
-                            s.Ut[p][k] = c * u - sn * v;
-                            s.Ut[q][k] = sn * u + c * v;
+                        T* Mp = s.M[p];
+                        T* Mq = s.M[q];
+                        T* Up = s.Ut[p];
+                        T* Uq = s.Ut[q];
+                        int k = 0;
+                        for (; k + 3 < r; k += 4) {   // loads of four columns issued together
+                            T x[4], y[4], u[4], v[4];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                x[e] = Mp[k + e]; y[e] = Mq[k + e]; u[e] = Up[k + e]; v[e] = Uq[k + e];
+                            }
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                Mp[k + e] = c * x[e] - sn * y[e];
+                                Mq[k + e] = sn * x[e] + c * y[e];
+                                Up[k + e] = c * u[e] - sn * v[e];
+                                Uq[k + e] = sn * u[e] + c * v[e];
+                            }
+                        }
+                        for (; k < r; ++k) {
+                            const T x = Mp[k], y = Mq[k], u = Up[k], v = Uq[k];
+                            Mp[k] = c * x - sn * y;
+                            Mq[k] = sn * x + c * y;
+                            Up[k] = c * u - sn * v;
+                            Uq[k] = sn * u + c * v;
                         }
                     }
                 }
