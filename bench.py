@@ -129,12 +129,17 @@ def timed(fn, steps, sync_all, stream):
 
 
 # ------------------------------------------------------------- roofline
-# fp32 SIMT FMA peak from unit counts: 148 SMs x 128 fp32 lanes x 2 flop x SM clock.
-B200_SMS, FP32_LANES_PER_SM = 148, 128
+# ALU peaks from unit counts x SM clock: fp32 SIMT 148 SMs x 128 lanes x 2 flop; fp64
+# (mma.m8n8k4.f64 and DFMA share the rate) 148 SMs x 64 FMA/clk x 2 flop = 37.2 TF at 1965 MHz.
+B200_SMS, FP32_LANES_PER_SM, FP64_FMA_PER_SM = 148, 128, 64
 
 
 def alu_peak_tflops(sm_mhz):
     return B200_SMS * FP32_LANES_PER_SM * 2 * (sm_mhz or 1965.0) * 1e6 / 1e12
+
+
+def fp64_peak_tflops(sm_mhz):
+    return B200_SMS * FP64_FMA_PER_SM * 2 * (sm_mhz or 1965.0) * 1e6 / 1e12
 
 
 def kernel_traffic(kernel, units):
@@ -155,7 +160,19 @@ def kernel_traffic(kernel, units):
 
 def dominant_roofline(dom, per_launch_ms, fr, hbm, peak_kind, sm_mhz):
     n = fr["n"]
-    if dom == "tsqr_leaf_merge":
+    if dom == "tsqr_gram_leaf":
+        # symmetric Gram X^T X of an m x r fp32 matrix in fp64: m r (r + 1) flop; both factors of every module
+        flops = fr["gram_flops"]
+        ach = flops / (per_launch_ms * 1e-3) / 1e12
+        peak = fp64_peak_tflops(sm_mhz)
+        gbs = fr["bytes_in"] / (per_launch_ms * 1e-3) / 1e9
+        return {"kernel": dom, "bound": "alu", "achieved": round(ach, 2), "peak": round(peak, 1),
+                "unit": "TFLOP/s", "frac": round(ach / peak, 4), "traffic": kernel_traffic(dom, n),
+                "algo_flops": int(flops), "dtype": "f64",
+                "peak_source": "derived: 148 SMs x 64 fp64 FMA/clk x 2 x SM clock",
+                "hbm": {"achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s", "frac": round(gbs / hbm, 4),
+                        "algo_bytes": int(fr["bytes_in"]), "peak_source": peak_kind}}
+    if dom == "tsqr_householder":
         # Householder QR of an m x r matrix: 2 m r^2 - 2 r^3 / 3 flop; both factors of every module
         flops = fr["qr_flops"]
         ach = flops / (per_launch_ms * 1e-3) / 1e12
@@ -217,7 +234,9 @@ def factor_bench(args, rank, world, dev, sync_all, stream, hbm, peak_kind):
     m_rows = (lay.d_out.astype(np.int64) + lay.d_in.astype(np.int64))
     rr = lay.r.astype(np.int64)
     qr_flops = float((2 * m_rows * rr * rr - 2 * (2 * rr ** 3) // 3).sum())
+    gram_flops = float((m_rows * rr * (rr + 1)).sum())
     res = dict(ms=ms, launches=launches, phases=phases, clocks=clk.summary(), status=st, n=lay.n, qr_flops=qr_flops,
+               gram_flops=gram_flops,
                bytes_in=inp, bytes_out=out, bytes_small=small, ranks_sum=int(ranks.sum()),
                params_frac=float((ranks.astype(np.int64) * (lay.d_in + lay.d_out)).sum() /
                                  (lay.r.astype(np.int64) * (lay.d_in + lay.d_out)).sum()))

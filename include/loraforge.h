@@ -87,9 +87,15 @@ int32_t lf_rank_stride(const lf_module* mods /*[host]*/, int32_t n);
  * For every module i, with X_B = B_i (d_out x r) and X_A = A_i^T (d_in x r):
  *   R_B = R(X_B), R_A = R(X_A): the R factors of the thin QRs, upper triangular,
  *         diag >= 0, computed by a batched tall-skinny QR over row tiles of every
- *         module at once (leaf tiles folded into a running R, chunk results merged
- *         in a fixed order);
- *   M = R_B R_A^T (r x r) and its SVD M = U S V^T in fp64:
+ *         module at once: each row tile contributes its Gram X_t^T X_t (fp32
+ *         products, exact in fp64, fp64 sums), tile Grams are summed in a fixed
+ *         order and R = chol(X^T X) in fp64 (R^T R = X^T X defines the same R as
+ *         the QR).  A matrix whose Cholesky pivot falls to <= 1e-9 of its Gram
+ *         diagonal (numerically rank-deficient, a zero column, non-finite input) is
+ *         factored instead by structured Householder reflections of [R; tile]
+ *         over the same row tiles, merged in chunk order;
+ *   M = R_B R_A^T (r x r) and its SVD M = U S V^T (one-sided Jacobi in fp32,
+ *   outputs stored as fp64):
  *   sigma (descending) are the singular values of dW = B A, Q_B U its left and
  *   Q_A V its right singular vectors.
  * Outputs (rs = lf_rank_stride):
@@ -205,7 +211,7 @@ lf_status lf_lora_shrink_expand_noalloc(int32_t T, int32_t d_in, int32_t d_out,
 /* ---- Tracing (no counterpart on the pages: measurement support) --------------
  * Every kernel launch of the library is counted.  With timing enabled, each
  * launch is also bracketed by CUDA events recorded on its own stream and its
- * device time is added to a named phase ("tsqr_leaf_merge", "svd_jacobi",
+ * device time is added to a named phase ("tsqr_gram_leaf", "svd_jacobi",
  * "select", "export_stream", "shrink_expand_gemv", ...).  lf_profile_read waits
  * for the pending events, then copies up to max_phases entries into `out`
  * [host] and returns the number of phases.  Process-wide state, not thread-safe. */

@@ -11,6 +11,7 @@
 
 #include "common.cuh"
 #include "tsqr.cuh"
+#include "gram.cuh"
 #include "select_export.cuh"
 #include "apply.cuh"
 
@@ -158,6 +159,12 @@ struct TsqrLayout {
     size_t mods, work, nwork, info, n_dev, counters, partial, total;
 };
 
+// Partial-slot bytes: the fp64 packed Gram of the leaf pass or the fp32 partial R of
+// the Householder pass, whichever is larger (the two passes run one after the other).
+static size_t tsqr_slot_bytes(int RT) {
+    return RT == 16 ? gram_slot_bytes<16>() : (RT == 32 ? gram_slot_bytes<32>() : gram_slot_bytes<64>());
+}
+
 static TsqrLayout tsqr_layout(int32_t n, const TsqrPlan& p) {
     Carver c(nullptr);
     TsqrLayout L;
@@ -171,8 +178,8 @@ static TsqrLayout tsqr_layout(int32_t n, const TsqrPlan& p) {
     LF_TAKE(nwork, int32_t, 1);
     LF_TAKE(info, TsqrInfo, p.info.size());
     LF_TAKE(n_dev, int32_t, 1);
-    LF_TAKE(counters, int32_t, (size_t)2 * n);
-    LF_TAKE(partial, float, (size_t)p.slots * p.RT * p.RT);
+    LF_TAKE(counters, int32_t, (size_t)6 * n);   // Gram counters, Householder counters, flags (2n each)
+    LF_TAKE(partial, char, (size_t)p.slots * tsqr_slot_bytes(p.RT));
 #undef LF_TAKE
     L.total = c.off + 256;
     return L;
@@ -183,8 +190,20 @@ static cudaError_t launch_tsqr(const TsqrArgs<T>& a, int n_items, cudaStream_t s
     auto k = tsqr_kernel<T, RT>;
     constexpr int W = tsqr_warps<T>();
     const int grid = (n_items + W - 1) / W;
-    if (grid > 0) LF_LAUNCH(sizeof(T) == 8 ? "tsqr_fp64_refine" : "tsqr_leaf_merge", k, grid, 32 * W, 0, st, a);
+    if (grid > 0) LF_LAUNCH(sizeof(T) == 8 ? "tsqr_fp64_refine" : "tsqr_householder", k, grid, 32 * W, 0, st, a);
     return cudaGetLastError();
+}
+
+template <int RT>
+static cudaError_t launch_gram(const GramArgs& a, int n_items, cudaStream_t st) {
+    if (n_items > 0) LF_LAUNCH("tsqr_gram_leaf", gram_kernel<RT>, n_items, 32, 0, st, a);
+    return cudaGetLastError();
+}
+
+static cudaError_t launch_gram_rt(int RT, const GramArgs& a, int n_items, cudaStream_t st) {
+    if (RT == 16) return launch_gram<16>(a, n_items, st);
+    if (RT == 32) return launch_gram<32>(a, n_items, st);
+    return launch_gram<64>(a, n_items, st);
 }
 
 template <typename T>
@@ -385,8 +404,28 @@ lf_status lf_tsqr_batched(const lf_module* mods, int32_t n, const float* B_base,
     h.put(p.info.data(), p.info.size());
     h.put(&n, 1);
     LF_CUDA_TRY(cudaMemcpyAsync(base, h.buf.data(), h.off, cudaMemcpyHostToDevice, s));
-    LF_CUDA_TRY(cudaMemsetAsync(base + L.counters, 0, (size_t)2 * n * sizeof(int32_t), s));
+    LF_CUDA_TRY(cudaMemsetAsync(base + L.counters, 0, (size_t)6 * n * sizeof(int32_t), s));
+    int32_t* gram_counters = reinterpret_cast<int32_t*>(base + L.counters);
+    int32_t* hh_counters = gram_counters + 2 * n;
+    int32_t* flags = gram_counters + 4 * n;
 
+    GramArgs ga;
+    ga.mods = reinterpret_cast<const lf_module*>(base + L.mods);
+    ga.B_base = B_base;
+    ga.A_base = A_base;
+    ga.work = reinterpret_cast<const TsqrWork*>(base + L.work);
+    ga.n_work = reinterpret_cast<const int32_t*>(base + L.nwork);
+    ga.info = reinterpret_cast<const TsqrInfo*>(base + L.info);
+    ga.counters = gram_counters;
+    ga.partial = reinterpret_cast<double*>(base + L.partial);
+    ga.slot_doubles = (int64_t)(tsqr_slot_bytes(p.RT) / sizeof(double));
+    ga.flags = flags;
+    ga.R_B = R_B;
+    ga.R_A = R_A;
+    ga.rs = p.rs;
+    LF_CUDA_TRY(launch_gram_rt(p.RT, ga, nwork, s));
+
+    // structured-Householder TSQR for the matrices whose Gram Cholesky was rejected
     TsqrArgs<float> ta;
     ta.mods = reinterpret_cast<const lf_module*>(base + L.mods);
     ta.mod_ids = nullptr;
@@ -395,11 +434,12 @@ lf_status lf_tsqr_batched(const lf_module* mods, int32_t n, const float* B_base,
     ta.work = reinterpret_cast<const TsqrWork*>(base + L.work);
     ta.n_work = reinterpret_cast<const int32_t*>(base + L.nwork);
     ta.info = reinterpret_cast<const TsqrInfo*>(base + L.info);
-    ta.counters = reinterpret_cast<int32_t*>(base + L.counters);
+    ta.counters = hh_counters;
     ta.partial = reinterpret_cast<float*>(base + L.partial);
     ta.R_B = R_B;
     ta.R_A = R_A;
     ta.rs = p.rs;
+    ta.only = flags;
     LF_CUDA_TRY(launch_tsqr_rt<float>(p.RT, ta, nwork, s));
 
     SvdArgs<float, float> sa;
@@ -593,6 +633,7 @@ lf_status lf_truncate_export(const lf_module* mods, int32_t n, lf_policy pol, co
         ta.R_B = reinterpret_cast<double*>(base + L.rRB);
         ta.R_A = reinterpret_cast<double*>(base + L.rRA);
         ta.rs = p.rs;
+        ta.only = nullptr;
         LF_CUDA_TRY(launch_tsqr_rt<double>(p.RT, ta, p.refine_max_work, s));
         SvdArgs<double, double> sa;
         sa.mods = dmods;

@@ -190,14 +190,15 @@ __global__ void __launch_bounds__(kTcThreads) shrink_tc_kernel(TcArgs a) {
 constexpr size_t kShrinkTcSmem = sizeof(ShrinkTcSmem) + 1024;
 
 // ---- expand ---------------------------------------------------------------
+constexpr int kTcStageLd = 68;   // 64 columns + 4: rows stay 16-byte aligned, 4-bank shift per row
 struct ExpandTcSmem {
     __nv_bfloat16 ahi[kTcM * kMaxRank];   // t_hi, K-major, 16 KB
     __nv_bfloat16 alo[kTcM * kMaxRank];   // t_lo
     __nv_bfloat16 b[kMaxRank * kTcN];     // B'^T tile, MN-major, 32 KB
+    float stage[kTcThreads / 32][32][kTcStageLd];   // per-warp accumulator transpose, 34 KB
     uint64_t bar;
     uint32_t tmem;
     int32_t toks[kTcM];
-    unsigned char pad[20 * 1024];          // keeps two CTAs per SM (2 x 256 TMEM columns)
 };
 
 __global__ void __launch_bounds__(kTcThreads) expand_tc_kernel(TcArgs a) {
@@ -250,8 +251,6 @@ __global__ void __launch_bounds__(kTcThreads) expand_tc_kernel(TcArgs a) {
     const uint32_t tmem = s.tmem;
     const uint32_t idesc = tc::idesc_bf16(kTcM, kTcN, 0, 1);
     const __nv_bfloat16* Bt = a.Bt_pool + it.ob;
-    const int m = warp * 32 + lane;
-    const int tok = s.toks[m];
     bool ok = true;
     int phase = 0;
     for (int e0 = e_begin; e0 < e_end && ok; e0 += kTcN, ++phase) {
@@ -280,35 +279,55 @@ __global__ void __launch_bounds__(kTcThreads) expand_tc_kernel(TcArgs a) {
             }
             tc::commit(&s.bar);
         }
-        // y row segment of this thread's token, loaded while the MMAs run
-        __nv_bfloat16* yrow = a.y + (int64_t)tok * a.d_out + e0;
-        const bool live = m < nt;
-        uint4 yv[kTcN / 8];
+        // y for this warp's 32 token rows, loaded while the MMAs run, in the coalesced
+        // mapping of the epilogue: iteration i covers rows 4*(i%8) + lane/8 of column
+        // block i/8, eight lanes per 128-byte row segment
+        const int cl = (lane & 7) * 8;   // column offset of this lane inside a 64-column block
+        uint4 yv[32];
 #pragma unroll
-        for (int h = 0; h < kTcN / 8; ++h)
-            yv[h] = (live && e0 + 8 * h < e_end) ? *reinterpret_cast<const uint4*>(yrow + 8 * h) : make_uint4(0, 0, 0, 0);
+        for (int i = 0; i < 32; ++i) {
+            const int rr = warp * 32 + 4 * (i & 7) + (lane >> 3);
+            const int e = e0 + 64 * (i >> 3) + cl;
+            yv[i] = (rr < nt && e < e_end)
+                        ? *reinterpret_cast<const uint4*>(a.y + (int64_t)s.toks[rr] * a.d_out + e)
+                        : make_uint4(0, 0, 0, 0);
+        }
         ok = mbar_wait(&s.bar, (uint32_t)(phase & 1));
         tc::fence_after_sync();
         if (ok) {
+            float (*st)[kTcStageLd] = s.stage[warp];
 #pragma unroll
-            for (int c0 = 0; c0 < kTcN; c0 += 16) {
-                float v[16];
-                tc::tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c0, v);
+            for (int blk = 0; blk < kTcN / 64; ++blk) {
+                // accumulator rows (one per lane) of this 64-column block -> shared memory
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    __nv_bfloat162* p2 = reinterpret_cast<__nv_bfloat162*>(&yv[c0 / 8 + h]);
+                for (int c16 = 0; c16 < 4; ++c16) {
+                    float v[16];
+                    tc::tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(blk * 64 + c16 * 16), v);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        *reinterpret_cast<float4*>(&st[lane][c16 * 16 + 4 * q]) =
+                            make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+                }
+                __syncwarp();
+#pragma unroll
+                for (int i8 = 0; i8 < 8; ++i8) {
+                    const int i = blk * 8 + i8;
+                    const int rl = 4 * i8 + (lane >> 3);   // row inside the warp's 32
+                    const int rr = warp * 32 + rl;
+                    const int e = e0 + 64 * blk + cl;
+                    const float4 p0 = *reinterpret_cast<const float4*>(&st[rl][cl]);
+                    const float4 p1 = *reinterpret_cast<const float4*>(&st[rl][cl + 4]);
+                    const float acc[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+                    __nv_bfloat162* p2 = reinterpret_cast<__nv_bfloat162*>(&yv[i]);
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
                         const float2 yf = __bfloat1622float2(p2[q]);
-                        p2[q] = __floats2bfloat162_rn(fmaf(a.scale, v[8 * h + 2 * q], yf.x),
-                                                      fmaf(a.scale, v[8 * h + 2 * q + 1], yf.y));
+                        p2[q] = __floats2bfloat162_rn(fmaf(a.scale, acc[2 * q], yf.x), fmaf(a.scale, acc[2 * q + 1], yf.y));
                     }
+                    if (rr < nt && e < e_end)
+                        *reinterpret_cast<uint4*>(a.y + (int64_t)s.toks[rr] * a.d_out + e) = yv[i];
                 }
-            }
-            if (live) {
-#pragma unroll
-                for (int h = 0; h < kTcN / 8; ++h)
-                    if (e0 + 8 * h < e_end) *reinterpret_cast<uint4*>(yrow + 8 * h) = yv[h];
+                __syncwarp();
             }
         }
         tc::fence_before_sync();

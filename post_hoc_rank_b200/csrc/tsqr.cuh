@@ -53,6 +53,7 @@ struct TsqrArgs {
     T* R_B;                     // per local module, rs x rs
     T* R_A;
     int32_t rs;
+    const int32_t* only;        // per local mf (nullable): nonzero = factor this matrix, zero = skip it
 };
 
 // Packed upper triangle of an RT x RT matrix, row-major: row j holds columns j..RT-1.
@@ -188,6 +189,7 @@ __global__ void __launch_bounds__(32 * tsqr_warps<T>(), sizeof(T) == 4 ? 16 : 1)
     T* Rp = s_R[warp];
     T* vbuf = s_v[warp];
     const TsqrWork w = a.work[wi];
+    if (a.only && a.only[w.mf] == 0) return;   // warp-uniform
     const int local = w.mf >> 1, factor = w.mf & 1;
     const int gm = a.mod_ids ? a.mod_ids[local] : local;
     const lf_module md = a.mods[gm];
