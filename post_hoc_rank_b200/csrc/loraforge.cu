@@ -680,7 +680,8 @@ lf_status lf_truncate_export(const lf_module* mods, int32_t n, lf_policy pol, co
     ea.Bt_pool16 = reinterpret_cast<__nv_bfloat16*>(Bt_pool_bf16);
     ea.cap_A = pool_cap_A;
     ea.cap_Bt = pool_cap_Bt;
-    LF_LAUNCH("export_stream", export_kernel, (int)p.ework.size(), kExpThreads, 0, s, ea);
+    LF_CUDA_TRY(cudaFuncSetAttribute(export_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kExportSmem));
+    LF_LAUNCH("export_stream", export_kernel, (int)p.ework.size(), kExpThreads, kExportSmem, s, ea);
     return launch_status();
 }
 

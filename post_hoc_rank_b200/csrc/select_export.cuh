@@ -15,6 +15,7 @@
 //   B'^T = (R_A^T V_k S_k^-1)^T B^T,   A' = (U_k^T R_B) A.
 #pragma once
 #include "common.cuh"
+#include "tc.cuh"
 
 namespace lf {
 
@@ -303,110 +304,135 @@ struct ExportArgs {
 };
 
 constexpr int kExpThreads = 256;   // 8 warps
-constexpr int kExpJ = 16;          // retained directions per accumulator pass
+constexpr int kExpRows = 64;       // B rows (or A columns) per pipeline stage
+constexpr int kExpStages = 3;
+constexpr int kExpLdB = 68;        // row stride (floats) of a B stage: 16-byte rows, 4-bank shift per row
+constexpr int kExpStageFloats = kExpRows * kExpLdB;
+constexpr size_t kExportSmem = (size_t)(kMaxRank * kMaxRank + kExpStages * kExpStageFloats) * sizeof(float);
 
-// B part: lane owns one row e of B (r fp32 = 16 float4 loads issued together) and
-// writes B'^T[j][e] = sum_l C_Bt[j][l] B[e][l] for j < k (coalesced across lanes).
-__device__ void export_b_rows(const ExportArgs& a, const lf_module& md, int k, const float* cB, int64_t obt,
-                              int start, int len) {
+__device__ __forceinline__ void exp_cp16(float* dst, const float* src, uint32_t n) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(n) : "memory");
+}
+__device__ __forceinline__ void exp_cp4(float* dst, const float* src, uint32_t n) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(n) : "memory");
+}
+
+// Stage t of a work item: B part = rows e0 .. e0+63 of B (row-major, stride kExpLdB);
+// A part = columns d0 .. d0+63 of all r rows of A (stage[l * 64 + c]).  Entries past
+// the item, past r or past the matrix are zero-filled.
+__device__ __forceinline__ void export_issue(float* st, const float* X, const lf_module& md, int part, int i0,
+                                             int nrem, bool vec) {
     const int r = md.r, tid = threadIdx.x;
-    const float* B = a.B_base + md.B_off;
-    for (int e0 = start; e0 < start + len; e0 += kExpThreads) {
-        const int e = e0 + tid;
-        if (e >= start + len) break;
-        float x[kMaxRank];
-        if (r == kMaxRank) {
-            const float4* src = reinterpret_cast<const float4*>(B + (int64_t)e * kMaxRank);
-#pragma unroll
-            for (int q = 0; q < kMaxRank / 4; ++q) {
-                const float4 v = __ldg(src + q);
-                x[4 * q] = v.x; x[4 * q + 1] = v.y; x[4 * q + 2] = v.z; x[4 * q + 3] = v.w;
+    if (part == 0) {
+        if (vec) {
+            for (int q = tid; q < kExpRows * 16; q += kExpThreads) {
+                const int row = q >> 4, c4 = q & 15;
+                const bool ok = row < nrem && 4 * c4 < r;
+                exp_cp16(st + row * kExpLdB + 4 * c4, ok ? X + (int64_t)(i0 + row) * r + 4 * c4 : X, ok ? 16u : 0u);
             }
         } else {
-#pragma unroll
-            for (int l = 0; l < kMaxRank; ++l) x[l] = l < r ? __ldg(B + (int64_t)e * r + l) : 0.f;
-        }
-        for (int j0 = 0; j0 < k; j0 += kExpJ) {
-            float acc[kExpJ];
-#pragma unroll
-            for (int jj = 0; jj < kExpJ; ++jj) {
-                float t = 0.f;
-                if (j0 + jj < k) {
-                    const float* cr = cB + (j0 + jj) * kMaxRank;
-#pragma unroll
-                    for (int l = 0; l < kMaxRank; ++l) t = fmaf(cr[l], x[l], t);
-                }
-                acc[jj] = t;
+            for (int q = tid; q < kExpRows * kMaxRank; q += kExpThreads) {
+                const int row = q >> 6, c = q & 63;
+                const bool ok = row < nrem && c < r;
+                exp_cp4(st + row * kExpLdB + c, ok ? X + (int64_t)(i0 + row) * r + c : X, ok ? 4u : 0u);
             }
-#pragma unroll
-            for (int jj = 0; jj < kExpJ; ++jj) {
-                if (j0 + jj < k) {
-                    const int64_t o = obt + (int64_t)(j0 + jj) * md.d_out + e;
-                    a.Bt_pool[o] = acc[jj];
-                    if (a.Bt_pool16) a.Bt_pool16[o] = __float2bfloat16_rn(acc[jj]);
-                }
+        }
+    } else {
+        if (vec) {
+            for (int q = tid; q < kMaxRank * 16; q += kExpThreads) {
+                const int l = q >> 4, c4 = q & 15;
+                const int nv = l < r ? min(4, max(0, nrem - 4 * c4)) : 0;
+                exp_cp16(st + l * kExpRows + 4 * c4, nv > 0 ? X + (int64_t)l * md.d_in + i0 + 4 * c4 : X,
+                         4u * (uint32_t)nv);
+            }
+        } else {
+            for (int q = tid; q < kMaxRank * kExpRows; q += kExpThreads) {
+                const int l = q >> 6, c = q & 63;
+                const bool ok = l < r && c < nrem;
+                exp_cp4(st + l * kExpRows + c, ok ? X + (int64_t)l * md.d_in + i0 + c : X, ok ? 4u : 0u);
             }
         }
     }
 }
 
-// A part: thread owns 4 consecutive columns d..d+3 of A (r x d_in) and writes
-// A'[j][d..d+3] = sum_l C_A[j][l] A[l][d..d+3].
-__device__ void export_a_cols(const ExportArgs& a, const lf_module& md, int k, const float* cA, int64_t oa,
-                              int start, int len) {
-    const int r = md.r;
-    const float* A = a.A_base + md.A_off;
-    const bool vec = (md.d_in % 4 == 0) && (start % 4 == 0);
-    for (int d = start + 4 * threadIdx.x; d < start + len; d += 4 * kExpThreads) {
-        const int nd = min(4, start + len - d);
-        for (int j0 = 0; j0 < k; j0 += kExpJ) {
-            float acc[kExpJ][4];
+// One stage: thread (item row / column `e` = tid % 64, output group g = tid / 64)
+// forms outputs j = jbase + g + 4q (q < NQ, j < k) as dot products of its 64 stage
+// values with coefficient rows j (shared memory, broadcast within the warp).
+template <int NQ>
+__device__ __forceinline__ void export_stage(const ExportArgs& a, const lf_module& md, int part, int k,
+                                             const float* coef, const float* st, int i0, int nrem, int64_t obase,
+                                             int jbase) {
+    const int tid = threadIdx.x, e = tid & (kExpRows - 1), g = tid >> 6;
+    float acc[NQ];
 #pragma unroll
-            for (int jj = 0; jj < kExpJ; ++jj)
+    for (int q = 0; q < NQ; ++q) acc[q] = 0.f;
+#pragma unroll 4
+    for (int l = 0; l < kMaxRank; l += 4) {
+        float4 x;
+        if (part == 0) {
+            x = *reinterpret_cast<const float4*>(st + e * kExpLdB + l);
+        } else {
+            x.x = st[l * kExpRows + e];
+            x.y = st[(l + 1) * kExpRows + e];
+            x.z = st[(l + 2) * kExpRows + e];
+            x.w = st[(l + 3) * kExpRows + e];
+        }
 #pragma unroll
-                for (int c = 0; c < 4; ++c) acc[jj][c] = 0.f;
-#pragma unroll 16
-            for (int l = 0; l < r; ++l) {
-                float4 v;
-                const float* src = A + (int64_t)l * md.d_in + d;
-                if (vec && nd == 4) {
-                    v = __ldg(reinterpret_cast<const float4*>(src));
-                } else {
-                    v.x = __ldg(src);
-                    v.y = nd > 1 ? __ldg(src + 1) : 0.f;
-                    v.z = nd > 2 ? __ldg(src + 2) : 0.f;
-                    v.w = nd > 3 ? __ldg(src + 3) : 0.f;
-                }
+        for (int q = 0; q < NQ; ++q) {
+            const float4 c = *reinterpret_cast<const float4*>(coef + (jbase + g + 4 * q) * kMaxRank + l);
+            acc[q] = fmaf(c.x, x.x, fmaf(c.y, x.y, fmaf(c.z, x.z, fmaf(c.w, x.w, acc[q]))));
+        }
+    }
+    if (e >= nrem) return;
+    const int64_t ld = part == 0 ? md.d_out : md.d_in;
+    float* pool = part == 0 ? a.Bt_pool : a.A_pool;
+    __nv_bfloat16* pool16 = part == 0 ? a.Bt_pool16 : a.A_pool16;
 #pragma unroll
-                for (int jj = 0; jj < kExpJ; ++jj) {
-                    if (j0 + jj < k) {
-                        const float cj = cA[(j0 + jj) * kMaxRank + l];
-                        acc[jj][0] = fmaf(cj, v.x, acc[jj][0]);
-                        acc[jj][1] = fmaf(cj, v.y, acc[jj][1]);
-                        acc[jj][2] = fmaf(cj, v.z, acc[jj][2]);
-                        acc[jj][3] = fmaf(cj, v.w, acc[jj][3]);
-                    }
-                }
-            }
-#pragma unroll
-            for (int jj = 0; jj < kExpJ; ++jj) {
-                if (j0 + jj < k) {
-                    const int64_t o = oa + (int64_t)(j0 + jj) * md.d_in + d;
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        if (c < nd) {
-                            a.A_pool[o + c] = acc[jj][c];
-                            if (a.A_pool16) a.A_pool16[o + c] = __float2bfloat16_rn(acc[jj][c]);
-                        }
-                    }
-                }
-            }
+    for (int q = 0; q < NQ; ++q) {
+        const int j = jbase + g + 4 * q;
+        if (j < k) {
+            const int64_t o = obase + (int64_t)j * ld + i0 + e;
+            pool[o] = acc[q];
+            if (pool16) pool16[o] = __float2bfloat16_rn(acc[q]);
         }
     }
 }
 
-__global__ void __launch_bounds__(kExpThreads) export_kernel(ExportArgs a) {
-    __shared__ __align__(16) float coef[kMaxRank * kMaxRank];   // k x r, row stride kMaxRank, zero past r
+template <int NQ>
+__device__ void export_item(const ExportArgs& a, const lf_module& md, int part, int k, const float* coef,
+                            float* stages, const float* X, int start, int len, int64_t obase, bool vec) {
+    const int nst = (len + kExpRows - 1) / kExpRows;
+#pragma unroll
+    for (int s = 0; s < kExpStages - 1; ++s) {
+        if (s < nst)
+            export_issue(stages + s * kExpStageFloats, X, md, part, start + s * kExpRows, len - s * kExpRows, vec);
+        tc::cp_async_commit();
+    }
+    for (int t = 0; t < nst; ++t) {
+        tc::cp_async_wait<kExpStages - 2>();
+        __syncthreads();   // stage t landed for every thread; stage t - 1 fully consumed
+        const int tn = t + kExpStages - 1;
+        if (tn < nst)
+            export_issue(stages + (tn % kExpStages) * kExpStageFloats, X, md, part, start + tn * kExpRows,
+                         len - tn * kExpRows, vec);
+        tc::cp_async_commit();
+        const float* st = stages + (t % kExpStages) * kExpStageFloats;
+        export_stage<NQ>(a, md, part, k, coef, st, start + t * kExpRows, len - t * kExpRows, obase, 0);
+        if (NQ == 8)   // k > 16: a second pass for j = 32 .. 63
+            export_stage<NQ>(a, md, part, k, coef, st, start + t * kExpRows, len - t * kExpRows, obase, 32);
+    }
+    tc::cp_async_wait<0>();
+}
+
+// One CTA per work item (a run of up to 2048 rows of B or columns of A of one
+// module): the item streams through a 3-stage cp.async ring of 64-row stages and
+// every output element is one 64-term dot product with a row of the coefficients
+//   B part: B'^T[j][e] = sum_l C_Bt[j][l] B[e][l]
+//   A part: A'[j][d]   = sum_l C_A[j][l]  A[l][d].
+__global__ void __launch_bounds__(kExpThreads, 3) export_kernel(ExportArgs a) {
+    extern __shared__ __align__(16) float exp_smem[];
+    float* coef = exp_smem;                             // k x 64, row stride 64, zero past r
+    float* stages = exp_smem + kMaxRank * kMaxRank;
     const ExportWork w = a.work[blockIdx.x];
     const lf_module md = a.mods[w.mod];
     const int k = a.ranks[w.mod];
@@ -419,13 +445,23 @@ __global__ void __launch_bounds__(kExpThreads) export_kernel(ExportArgs a) {
         if (oa + (int64_t)k * md.d_in > a.cap_A) return;
     }
     const float* C = (w.part == 0 ? a.C_Bt : a.C_A) + (size_t)w.mod * a.rs * a.rs;
-    for (int e = threadIdx.x; e < k * kMaxRank; e += kExpThreads) {
+    const int kfill = k <= 4 ? 4 : (k <= 8 ? 8 : (k <= 16 ? 16 : kMaxRank));   // rows export_stage reads
+    for (int e = threadIdx.x; e < kfill * kMaxRank; e += kExpThreads) {
         const int j = e / kMaxRank, l = e % kMaxRank;
-        coef[e] = l < r ? C[j * a.rs + l] : 0.f;
+        coef[e] = (j < k && l < r) ? C[j * a.rs + l] : 0.f;
     }
-    __syncthreads();
-    if (w.part == 0) export_b_rows(a, md, k, coef, obt, w.start, w.len);
-    else export_a_cols(a, md, k, coef, oa, w.start, w.len);
+    const float* X = w.part == 0 ? a.B_base + md.B_off : a.A_base + md.A_off;
+    const bool vec = w.part == 0 ? (r % 4 == 0) : (md.d_in % 4 == 0);
+    const int64_t obase = w.part == 0 ? obt : oa;
+    // coefficient rows are read after the first barrier inside export_item
+    if (k <= 4)
+        export_item<1>(a, md, w.part, k, coef, stages, X, w.start, w.len, obase, vec);
+    else if (k <= 8)
+        export_item<2>(a, md, w.part, k, coef, stages, X, w.start, w.len, obase, vec);
+    else if (k <= 16)
+        export_item<4>(a, md, w.part, k, coef, stages, X, w.start, w.len, obase, vec);
+    else
+        export_item<8>(a, md, w.part, k, coef, stages, X, w.start, w.len, obase, vec);
 }
 
 }  // namespace lf

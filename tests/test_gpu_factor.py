@@ -179,3 +179,64 @@ def test_pool_capacity_too_small_latches_workspace_error():
     api.truncate_export(mods, pol, B, A, F, out=E)
     assert lf.lf_get_device_status() == 4          # LF_ERR_WORKSPACE, latched on the device
     assert lf.lf_get_device_status() == 0          # and cleared by the read
+
+
+def _planted(d_out, r, sig, seed):
+    """B = G diag(sig) H with G (d_out x r) orthonormal and H (r x r) orthogonal: the
+    singular values of B are exactly sig (up to fp32 rounding of the stored bytes)."""
+    g = np.random.default_rng(seed)
+    Gq, _ = np.linalg.qr(g.standard_normal((d_out, r)))
+    H, _ = np.linalg.qr(g.standard_normal((r, r)))
+    return (Gq * sig) @ H
+
+
+def test_gram_leaf_accuracy_on_ill_conditioned_factor():
+    # cond(B) = 1e3: the fp64 Gram + Cholesky R carries ~1e-16 * cond^2 = 1e-10 relative
+    # error before the fp32 store, far inside what fp32 Householder (~u32 * cond) reaches
+    r, d_out, d_in = 16, 3000, 700
+    lay = synth.fleet_layout(1, shapes=[("m", d_out, d_in)], r=r, n_layers=1)
+    Bh = torch.zeros(lay.B_total); Ah = torch.zeros(lay.A_total)
+    synth.fill_fleet(lay, Bh, Ah, cfg_id=11)
+    b0 = int(lay.B_off[0])
+    Bh[b0:b0 + d_out * r] = torch.from_numpy(_planted(d_out, r, np.logspace(0, -3, r), 5).ravel()).float()
+    B, A = upload(Bh, Ah)
+    mods = api.modules_from_layout(lay)
+    F = api.tsqr(mods, B, A)
+    assert lf.lf_get_device_status() == 0
+    Bn, _ = G.module_np(lay, Bh, Ah, 0)
+    want = OF.qr_r(Bn)
+    got = F.R_B[0][:r, :r].double().cpu().numpy()
+    assert np.linalg.norm(got - want) / np.linalg.norm(want) <= 1e-6
+
+
+def test_rank_deficient_factors_take_householder_route():
+    # a duplicated column, a zero column and cond = 1e7: Cholesky pivots fall below
+    # 1e-9 of the Gram diagonal, so these matrices are factored by Householder TSQR;
+    # R is then not unique past the rank, but R^T R = X^T X and sigma(B A) are
+    r, d_out, d_in = 16, 2500, 2100
+    shapes = [("dup", d_out, d_in), ("zero_col", d_out, d_in), ("cond1e7", d_out, d_in), ("ok", d_out, d_in)]
+    lay = synth.fleet_layout(1, shapes=shapes, r=r, n_layers=1)
+    Bh = torch.zeros(lay.B_total); Ah = torch.zeros(lay.A_total)
+    synth.fill_fleet(lay, Bh, Ah, cfg_id=12)
+    for i in range(3):
+        b0 = int(lay.B_off[i])
+        Bm = Bh[b0:b0 + d_out * r].view(d_out, r)
+        if i == 0:
+            Bm[:, 5] = Bm[:, 2]
+        elif i == 1:
+            Bm[:, 7] = 0.0
+        else:
+            Bm[:] = torch.from_numpy(_planted(d_out, r, np.logspace(0, -7, r), 6)).float()
+    B, A = upload(Bh, Ah)
+    mods = api.modules_from_layout(lay)
+    F = api.tsqr(mods, B, A)
+    assert lf.lf_get_device_status() == 0
+    RB, S = F.R_B.double().cpu().numpy(), F.sigma.cpu().numpy()
+    for i in range(lay.n):
+        Bn, An = G.module_np(lay, Bh, Ah, i)
+        R = RB[i][:r, :r]
+        assert np.allclose(np.tril(R, -1), 0) and np.all(np.diag(R) >= 0)
+        gram = Bn.T @ Bn
+        assert np.linalg.norm(R.T @ R - gram) <= 1e-5 * np.linalg.norm(gram), i
+        s, *_ = OF.spectrum_factor(Bn, An)
+        assert np.max(np.abs(S[i][:r] - s)) <= G.SIGMA_TOL * s[0], i
