@@ -377,6 +377,9 @@ def _apply_run(args, calls, ids_d, n_ad, T, total_bytes, stream, hbm, meta):
         step(stream)
     torch.cuda.synchronize()
     assert lf.lf_get_device_status(stream) == 0
+    l0 = lf.lf_launch_count()
+    step(stream)
+    launches = lf.lf_launch_count() - l0
     # CUDA graph of one step (host launch cost out of the measurement)
     g = torch.cuda.CUDAGraph()
     cap = torch.cuda.Stream()
@@ -406,7 +409,7 @@ def _apply_run(args, calls, ids_d, n_ad, T, total_bytes, stream, hbm, meta):
     del g
     out = dict(meta)
     out.update(tokens_per_s=T / (ms * 1e-3), ms_per_step=ms, algo_bytes=int(total_bytes), achieved_gbs=gbs,
-               hbm_frac=gbs / hbm, launches_per_step=2 * len(calls),
+               hbm_frac=gbs / hbm, launches_per_step=launches,
                phases_ms={k: v[0] / 3 for k, v in ph.items()})
     return out
 

@@ -376,6 +376,125 @@ __global__ void __launch_bounds__(kGemvThreads) expand_kernel(GemvArgs a) {
 }
 
 
+// Decode regime, token-parallel (BGMV form: every token carries its adapter index,
+// no sorting).  CTA (token, 4096-column slice of d_out): t = A'_a x (k fp32 dot
+// products over d_in, reduced across the CTA in a fixed order), then
+// y[slice] += s * B'_a^T t with 16-byte loads of the k rows of B'^T.  Each slice
+// CTA recomputes the same t (identical arithmetic; x and A'_a come from L2), and
+// tokens of one adapter read its factors from L2 after the first touch, so HBM
+// sees every distinct factor row, x and y once.
+constexpr int kBgmvThreads = 256;
+constexpr int kBgmvVec = 2;                                  // 8-column vectors per thread in the expand
+constexpr int kBgmvCols = kBgmvThreads * 8 * kBgmvVec;       // d_out columns per CTA
+constexpr int kBgmvJ = 8;                                    // retained directions per shrink pass
+
+struct BgmvArgs {
+    int32_t n_adapters, d_in, d_out;
+    const __nv_bfloat16* x;
+    __nv_bfloat16* y;
+    const int32_t* ids;
+    const int32_t* ranks;
+    const int64_t* off_A;
+    const int64_t* off_Bt;
+    const __nv_bfloat16* A_pool;
+    const __nv_bfloat16* Bt_pool;
+    int64_t pool_A, pool_Bt;
+    float scale;
+};
+
+__global__ void __launch_bounds__(kBgmvThreads) bgmv_kernel(BgmvArgs a) {
+    __shared__ float red[kBgmvThreads / 32][kBgmvJ];
+    __shared__ float ts[kMaxRank];
+    const int tok = blockIdx.x;
+    const int ad = a.ids[tok];
+    if (ad == -1) return;
+    const bool lead = blockIdx.y == 0 && threadIdx.x == 0;   // one CTA per token reports errors
+    if (ad < -1 || ad >= a.n_adapters) {
+        if (lead) latch_error(LF_ERR_BAD_INDEX);
+        return;
+    }
+    const int k = a.ranks[ad];
+    const int64_t oa = a.off_A[ad], ob = a.off_Bt[ad];
+    int err = 0;
+    if (k > kMaxRank) err = LF_ERR_SHAPE;
+    else if (k > 0 && ((oa & 7) || (ob & 7))) err = LF_ERR_ALIGNMENT;
+    else if (k > 0 && (oa < 0 || ob < 0 || oa + (int64_t)k * a.d_in > a.pool_A || ob + (int64_t)k * a.d_out > a.pool_Bt))
+        err = LF_ERR_WORKSPACE;
+    if (err) {
+        if (lead) latch_error(err);
+        return;
+    }
+    if (k <= 0) return;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const __nv_bfloat16* xr = a.x + (int64_t)tok * a.d_in;
+    const __nv_bfloat16* Ap = a.A_pool + oa;
+    for (int j0 = 0; j0 < k; j0 += kBgmvJ) {
+        const int nj = min(kBgmvJ, k - j0);
+        float acc[kBgmvJ];
+#pragma unroll
+        for (int jj = 0; jj < kBgmvJ; ++jj) acc[jj] = 0.f;
+        for (int d0 = tid * 8; d0 < a.d_in; d0 += kBgmvThreads * 8) {
+            uint4 ar[kBgmvJ];
+            const uint4 xv = __ldg(reinterpret_cast<const uint4*>(xr + d0));
+#pragma unroll
+            for (int jj = 0; jj < kBgmvJ; ++jj)
+                if (jj < nj) ar[jj] = __ldg(reinterpret_cast<const uint4*>(Ap + (int64_t)(j0 + jj) * a.d_in + d0));
+            float xf[8];
+            bf16x8_to_f32(xv, xf);
+#pragma unroll
+            for (int jj = 0; jj < kBgmvJ; ++jj) {
+                if (jj < nj) {
+                    float af[8];
+                    bf16x8_to_f32(ar[jj], af);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) acc[jj] = fmaf(af[e], xf[e], acc[jj]);
+                }
+            }
+        }
+#pragma unroll
+        for (int jj = 0; jj < kBgmvJ; ++jj) {
+            if (jj < nj) {
+                const float v = warp_sum(acc[jj]);
+                if (lane == 0) red[warp][jj] = v;
+            }
+        }
+        __syncthreads();
+        if (tid < nj) {
+            float v = 0.f;
+#pragma unroll
+            for (int w = 0; w < kBgmvThreads / 32; ++w) v += red[w][tid];
+            ts[j0 + tid] = v;
+        }
+        __syncthreads();
+    }
+    const __nv_bfloat16* Bt = a.Bt_pool + ob;
+    __nv_bfloat16* yr = a.y + (int64_t)tok * a.d_out;
+#pragma unroll
+    for (int h = 0; h < kBgmvVec; ++h) {
+        const int e = blockIdx.y * kBgmvCols + h * (kBgmvThreads * 8) + tid * 8;
+        if (e >= a.d_out) break;
+        uint4 yv = *reinterpret_cast<const uint4*>(yr + e);   // issued before the k-row loads are consumed
+        float acc[8];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) acc[c] = 0.f;
+#pragma unroll 4
+        for (int j = 0; j < k; ++j) {
+            float bf[8];
+            bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(Bt + (int64_t)j * a.d_out + e)), bf);
+            const float tv = ts[j];
+#pragma unroll
+            for (int c = 0; c < 8; ++c) acc[c] = fmaf(tv, bf[c], acc[c]);
+        }
+        __nv_bfloat162* y2 = reinterpret_cast<__nv_bfloat162*>(&yv);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const float2 yf = __bfloat1622float2(y2[q]);
+            y2[q] = __floats2bfloat162_rn(fmaf(a.scale, acc[2 * q], yf.x), fmaf(a.scale, acc[2 * q + 1], yf.y));
+        }
+        *reinterpret_cast<uint4*>(yr + e) = yv;
+    }
+}
+
 // Decode regime (few tokens per adapter): one launch does shrink and expand.  CTA
 // (item, d_out chunk): all warps share the dot products of each A' row over d_in
 // (16-byte loads issued together), t is reduced in a fixed order in shared memory,

@@ -736,6 +736,31 @@ lf_status lf_lora_shrink_expand(int32_t T, int32_t d_in, int32_t d_out, const vo
     o.tc_enable = decode_regime ? 0 : 1;
     const size_t rsmem = 2 * (size_t)n_adapters * sizeof(int32_t);
     LF_CUDA_TRY(cudaFuncSetAttribute(route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rsmem));
+    if (decode_regime) {
+        // few tokens per adapter: token-parallel shrink + expand, no sort; the routing
+        // pass runs only when the caller asks for the segment table
+        if (seg_out) {
+            LF_LAUNCH("route", route_kernel, 1, route_threads(T, n_adapters), rsmem, s, ids, T, n_adapters, o);
+            LF_CUDA_TRY(cudaGetLastError());
+        }
+        BgmvArgs b;
+        b.n_adapters = n_adapters;
+        b.d_in = d_in;
+        b.d_out = d_out;
+        b.x = reinterpret_cast<const __nv_bfloat16*>(x);
+        b.y = reinterpret_cast<__nv_bfloat16*>(y);
+        b.ids = ids;
+        b.ranks = ranks;
+        b.off_A = off_A;
+        b.off_Bt = off_Bt;
+        b.A_pool = reinterpret_cast<const __nv_bfloat16*>(A_pool);
+        b.Bt_pool = reinterpret_cast<const __nv_bfloat16*>(Bt_pool);
+        b.pool_A = pool_elems_A;
+        b.pool_Bt = pool_elems_Bt;
+        b.scale = scale;
+        LF_LAUNCH("bgmv", bgmv_kernel, dim3((unsigned)T, (unsigned)cdiv(d_out, kBgmvCols)), kBgmvThreads, 0, s, b);
+        return launch_status();
+    }
     LF_LAUNCH("route", route_kernel, 1, route_threads(T, n_adapters), rsmem, s, ids, T, n_adapters, o);
     LF_CUDA_TRY(cudaGetLastError());
     GemvArgs g;
@@ -758,11 +783,6 @@ lf_status lf_lora_shrink_expand(int32_t T, int32_t d_in, int32_t d_out, const vo
     g.t_buf = t_buf;
     const unsigned max_items = (unsigned)(T / kGemvTok + mseg + 1);
     const dim3 grid2(max_items, (unsigned)cdiv(d_out, kGemvCols));
-    if (decode_regime) {
-        // few tokens per adapter: shrink and expand in one launch
-        LF_LAUNCH("fused_gemv", fused_gemv_kernel, grid2, kGemvThreads, 0, s, g);
-        return launch_status();
-    }
     LF_LAUNCH("shrink_gemv", shrink_kernel, max_items, kGemvThreads, 0, s, g);
     LF_CUDA_TRY(cudaGetLastError());
     LF_LAUNCH("expand_gemv", expand_kernel, grid2, kGemvThreads, 0, s, g);
