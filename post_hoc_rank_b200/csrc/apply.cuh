@@ -15,6 +15,7 @@
 namespace lf {
 
 constexpr int kRouteThreads = 1024;
+constexpr int kRouteChunk = 4096;  // tokens staged per pass of the run detection
 constexpr int kGemvTok = 8;        // tokens per GEMV work item
 constexpr int kGemvThreads = 256;
 constexpr int kGemvCols = kGemvThreads * 8;   // d_out columns per CTA
@@ -44,6 +45,11 @@ struct RouteOut {
     int32_t d_in, d_out;
     TcItem* tc_items;    // T / kTcM + min(T, n_adapters) + 1
     int32_t tc_enable;   // segments with >= kTcMin tokens become tensor-core items
+    // Run scratch (nullable, T ints each): with it the sort works on runs of equal
+    // consecutive ids (the histogram and the stable scatter touch runs, not tokens).
+    int32_t* run_start;  // first token of run i
+    int32_t* run_pos;    // position of run i's first token in the permutation
+    int32_t* tok_run;    // run index of every token
 };
 
 // Block-wide exclusive scan of one int per thread (blockDim.x a multiple of 32, <= 1024).
@@ -89,12 +95,57 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const int32_t* __r
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int nthr = (int)blockDim.x;
     for (int a = tid; a < n_adapters; a += nthr) cnt[a] = 0;
+    if (tid == 0) s_carry[0] = 0;
     __syncthreads();
-    for (int t = tid; t < T; t += nthr) {
+    const bool runs = o.run_start != nullptr;
+    auto valid_id = [&](int t) {
         const int a = ids[t];
-        if (a < -1 || a >= n_adapters) latch_error(LF_ERR_BAD_INDEX);
-        else if (a >= 0) atomicAdd(&cnt[a], 1);
+        return (a < -1 || a >= n_adapters) ? -1 : a;
+    };
+    int n_runs = 0;
+    if (runs) {
+        // runs of equal consecutive (valid) ids, in chunks of kRouteChunk tokens staged
+        // through shared memory (coalesced loads); each thread owns a contiguous slice
+        // of the chunk, counts its run starts, and one block scan numbers the runs
+        __shared__ int32_t s_idc[kRouteChunk + 1];
+        for (int base = 0; base < T; base += kRouteChunk) {
+            const int len = min(kRouteChunk, T - base);
+            for (int i = tid; i < len; i += nthr) {
+                const int raw = ids[base + i];
+                const bool bad = raw < -1 || raw >= n_adapters;
+                if (bad) latch_error(LF_ERR_BAD_INDEX);
+                s_idc[i + 1] = bad ? -1 : raw;
+            }
+            if (tid == 0) s_idc[0] = base > 0 ? valid_id(base - 1) : -2;
+            __syncthreads();
+            const int per = (len + nthr - 1) / nthr;
+            const int t0 = min(len, tid * per), t1 = min(len, t0 + per);
+            int nf = 0;
+            for (int i = t0; i < t1; ++i) nf += (s_idc[i + 1] != s_idc[i]);
+            int tot;
+            int ri = block_excl_scan(nf, wsum, &tot) + s_carry[0] - 1;
+            for (int i = t0; i < t1; ++i) {
+                if (s_idc[i + 1] != s_idc[i]) o.run_start[++ri] = base + i;
+                o.tok_run[base + i] = ri;
+            }
+            __syncthreads();
+            if (tid == 0) s_carry[0] += tot;
+            __syncthreads();
+        }
+        n_runs = s_carry[0];
+        for (int ri = tid; ri < n_runs; ri += nthr) {
+            const int t0 = o.run_start[ri];
+            const int a = valid_id(t0);
+            if (a >= 0) atomicAdd(&cnt[a], (ri + 1 < n_runs ? o.run_start[ri + 1] : T) - t0);
+        }
+    } else {
+        for (int t = tid; t < T; t += nthr) {
+            const int a = ids[t];
+            if (a < -1 || a >= n_adapters) latch_error(LF_ERR_BAD_INDEX);
+            else if (a >= 0) atomicAdd(&cnt[a], 1);
+        }
     }
+    __syncthreads();
     if (tid == 0) s_carry[0] = s_carry[1] = s_carry[2] = s_carry[3] = 0;
     __syncthreads();
     // scans over adapters in chunks of kRouteThreads: token start, segment index, item index
@@ -164,7 +215,44 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const int32_t* __r
         o.counts[2] = s_carry[2];
         o.counts[3] = s_carry[3];
     }
-    if (T <= nthr) {
+    if (runs) {
+        // stable scatter of runs (warp turns in run order), then every token in parallel
+        const int nwr = min(nthr / 32, (n_runs + 31) / 32);
+        for (int base = 0; base < n_runs; base += nthr) {
+            const int ri = base + tid;
+            int a = -1, len = 0;
+            if (ri < n_runs) {
+                const int t0 = o.run_start[ri];
+                a = valid_id(t0);
+                len = (ri + 1 < n_runs ? o.run_start[ri + 1] : T) - t0;
+            }
+            const unsigned peers = __match_any_sync(0xffffffffu, a);
+            const int leader = __ffs(peers) - 1;
+            int before = 0, total = 0;   // lengths of this warp's earlier / all runs of the same id
+            for (int l = 0; l < 32; ++l) {
+                const int v = __shfl_sync(0xffffffffu, len, l);
+                if ((peers >> l) & 1u) {
+                    total += v;
+                    if (l < lane) before += v;
+                }
+            }
+            for (int w = 0; w < nwr; ++w) {
+                if (warp == w && a >= 0 && lane == leader) {
+                    wbase[warp][lane] = cnt[a];
+                    cnt[a] += total;
+                }
+                __syncthreads();
+            }
+            if (a >= 0) o.run_pos[ri] = wbase[warp][leader] + before;
+            __syncthreads();
+        }
+        for (int t = tid; t < T; t += nthr) {
+            const int ri = o.tok_run[t];
+            if (valid_id(t) >= 0) o.perm[o.run_pos[ri] + t - o.run_start[ri]] = t;
+        }
+        __syncthreads();
+    }
+    if (!runs && T <= nthr) {
         // small batch: rank = number of earlier tokens with the same id (ids staged in smem)
         __shared__ int32_t s_ids[kRouteThreads];
         int a = -1;
@@ -183,7 +271,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const int32_t* __r
     }
     // stable scatter, chunk by chunk; warps take their turn in token order
     const int nwarps_live = min(nthr / 32, (T + 31) / 32);
-    for (int base = 0; T > nthr && base < T; base += nthr) {
+    for (int base = 0; !runs && T > nthr && base < T; base += nthr) {
         const int t = base + tid;
         int a = t < T ? ids[t] : -1;
         if (a < -1 || a >= n_adapters) a = -1;

@@ -10,7 +10,7 @@
 //   gathered through the token permutation with 16-byte cp.async into a 4-stage
 //   ring of K-major core matrices; one thread issues the MMAs and commits each
 //   stage to an mbarrier that frees the stage for the next copy.
-// Expand: D[128 x 256] = t_hi * B + t_lo * B with t = t_hi + t_lo split into two
+// Expand: D[128 x 128] = t_hi * B + t_lo * B with t = t_hi + t_lo split into two
 //   bf16 values (about 16 significant bits of the fp32 t); B = B'^T tile,
 //   MN-major; the epilogue reads D from tensor memory and updates y once.
 #pragma once
@@ -23,8 +23,7 @@ constexpr int kTcMin = 64;       // segments with at least this many tokens use 
 constexpr int kTcM = 128;        // tokens per tile (UMMA M)
 constexpr int kTcKB = 64;        // d_in elements per pipeline stage (128 bytes per row)
 constexpr int kTcStages = 4;
-constexpr int kTcThreads = 128;  // 4 warps: warp w owns tensor-memory lanes 32w .. 32w+31
-constexpr int kTcN = 256;        // expand tile width (UMMA N)
+constexpr int kTcThreads = 128;  // shrink: 4 warps, warp w owns tensor-memory lanes 32w .. 32w+31
 constexpr int kTcCols = 2048;    // d_out columns per expand CTA
 constexpr int kTcMaxSplit = 8;   // d_in is split over at most this many CTAs per token tile
 
@@ -55,10 +54,24 @@ struct TcArgs {
 };
 
 // ---- shrink ---------------------------------------------------------------
+// CTA (token tile of one segment, split of d_in), 4 warps in roles:
+//   warps 0, 2, 3, producers: gather the stage's 128 x rows (64 d_in elements,
+//     through the token permutation) and the k rows of A' into a kTcStages ring
+//     with 16-byte cp.async; kTcAhead stages stay in flight; once a stage's copies
+//     have landed (cp.async.wait_group) each lane fences them to the async proxy and
+//     arrives on the stage's `full` barrier; a stage is refilled after the
+//     tcgen05.commit of the MMAs that read it arrives on its `empty` barrier;
+//   warp 1 lane 0, MMA issuer: waits on `full`, issues four K = 16 MMAs into TMEM,
+//     commits to `empty`, and at the end to `done`;
+//   all warps: epilogue from TMEM (warp w reads lanes 32w ..) into t_part.
+constexpr int kTcAhead = 2;      // stages in flight before the producers signal the oldest
+constexpr int kTcProducers = 3;  // producer warps: 0, 2, 3 (warp 1 issues the MMAs)
 struct ShrinkTcSmem {
     __nv_bfloat16 a[kTcStages][kTcM * kTcKB];       // 16 KB per stage
     __nv_bfloat16 b[kTcStages][kMaxRank * kTcKB];   //  8 KB per stage
-    uint64_t bar[kTcStages];
+    uint64_t full[kTcStages];
+    uint64_t empty[kTcStages];
+    uint64_t done;
     uint32_t tmem;
     int32_t toks[kTcM];
 };
@@ -73,12 +86,19 @@ __device__ __forceinline__ void cp_async16_zfill(void* dst, const void* src, boo
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(n) : "memory");
 }
 
+__device__ __forceinline__ void mbar_arrive1(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
 __global__ void __launch_bounds__(kTcThreads) shrink_tc_kernel(TcArgs a) {
     extern __shared__ __align__(1024) unsigned char tc_raw[];
     auto& s = *reinterpret_cast<ShrinkTcSmem*>(tc_raw);
     if ((int)blockIdx.x >= a.counts[3]) return;
     const TcItem it = a.items[blockIdx.x];
     if (it.k <= 0) return;
+    const int split = blockIdx.y, slen = tc_split_len(a.d_in);
+    const int kbeg = split * slen;
+    if (kbeg >= a.d_in) return;   // uniform: this split has no columns
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int k = it.k, nt = it.ntok;
     const int npad = (k + 15) & ~15;
@@ -91,82 +111,84 @@ __global__ void __launch_bounds__(kTcThreads) shrink_tc_kernel(TcArgs a) {
     }
     if (warp == 0) tc::tmem_alloc(&s.tmem, 64);
     if (tid == 0) {
-        for (int i = 0; i < kTcStages; ++i) mbar_init(&s.bar[i], 1);
+        for (int i = 0; i < kTcStages; ++i) {
+            mbar_init(&s.full[i], 32 * kTcProducers);
+            mbar_init(&s.empty[i], 1);
+        }
+        mbar_init(&s.done, 1);
         fence_barrier_init();
     }
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
     const uint32_t tmem = s.tmem;
-    const int split = blockIdx.y, slen = tc_split_len(a.d_in);
-    const int kbeg = split * slen;
-    if (kbeg >= a.d_in) {   // uniform: this split has no columns (before any async work)
-        tc::fence_before_sync();
-        __syncthreads();
-        if (warp == 0) tc::tmem_dealloc(s.tmem, 64);
-        return;
-    }
     const int kend = min(a.d_in, kbeg + slen);
     const int nK = (kend - kbeg + kTcKB - 1) / kTcKB;
-    const __nv_bfloat16* Ap = a.A_pool + it.oa;
-    const uint32_t idesc = tc::idesc_bf16(kTcM, npad, 0, 0);
-
-    auto load_stage = [&](int kb, int st) {
-        char* abase = reinterpret_cast<char*>(s.a[st]);
-        char* bbase = reinterpret_cast<char*>(s.b[st]);
-        const int k0 = kbeg + kb * kTcKB;
-#pragma unroll
-        for (int i = 0; i < (kTcM * kTcKB / 8) / kTcThreads; ++i) {   // 8 chunks per thread
-            const int c = tid + i * kTcThreads;
-            const int m = c % kTcM, kc = c / kTcM;
-            const int kk = k0 + kc * 8;
-            const bool ok = m < nt && kk < kend;
-            const __nv_bfloat16* src = ok ? a.x + (int64_t)s.toks[m] * a.d_in + kk : a.x;
-            cp_async16_zfill(abase + kmaj64(m, kc * 8), src, ok);
-        }
-        for (int c = tid; c < k * (kTcKB / 8); c += kTcThreads) {
-            const int n = c / (kTcKB / 8), kc = c % (kTcKB / 8);
-            const int kk = k0 + kc * 8;
-            const bool ok = kk < kend;
-            const __nv_bfloat16* src = ok ? Ap + (int64_t)n * a.d_in + kk : Ap;
-            cp_async16_zfill(bbase + kmaj64(n, kc * 8), src, ok);
-        }
-    };
-
-    for (int p = 0; p < kTcStages - 1; ++p) {
-        if (p < nK) load_stage(p, p);
-        tc::cp_async_commit();
-    }
     bool ok = true;
-    for (int kb = 0; kb < nK && ok; ++kb) {
-        const int nxt = kb + kTcStages - 1;
-        if (nxt < nK) {
-            const int st = nxt % kTcStages;
-            if (nxt >= kTcStages) ok = mbar_wait(&s.bar[st], (uint32_t)((nxt / kTcStages - 1) & 1));
-            if (ok) load_stage(nxt, st);
-        }
-        tc::cp_async_commit();
-        tc::cp_async_wait<kTcStages - 1>();
-        tc::fence_proxy_async();
-        ok = __syncthreads_and(ok);   // block-uniform: a timed-out wait stops every thread
-        if (!ok) break;
-        if (tid == 0) {
-            tc::fence_after_sync();
+
+    const int pidx = warp == 0 ? 0 : warp - 1;   // producer index (warps 0, 2, 3)
+    if (warp != 1 && pidx < kTcProducers) {   // producers
+        const __nv_bfloat16* Ap = a.A_pool + it.oa;
+        for (int kb = 0; kb < nK && ok; ++kb) {
             const int st = kb % kTcStages;
+            if (kb >= kTcStages) ok = mbar_wait(&s.empty[st], (uint32_t)((kb / kTcStages - 1) & 1));
+            if (!ok) break;
+            char* abase = reinterpret_cast<char*>(s.a[st]);
+            char* bbase = reinterpret_cast<char*>(s.b[st]);
+            const int k0 = kbeg + kb * kTcKB;
+            // chunk mapping: a half-warp covers 8 rows x 32 contiguous bytes (full sectors);
+            // each quarter-warp writes 8 rows of one 16-byte column (distinct banks)
+            for (int i = pidx; i < (kTcM * kTcKB / 8) / 32; i += kTcProducers) {
+                const int u = 2 * i + (lane >> 4);
+                const int m = 8 * (u & 15) + (lane & 7);
+                const int kc = 2 * (u >> 4) + ((lane >> 3) & 1);
+                const int kk = k0 + kc * 8;
+                const bool v = m < nt && kk < kend;
+                cp_async16_zfill(abase + kmaj64(m, kc * 8), v ? a.x + (int64_t)s.toks[m] * a.d_in + kk : a.x, v);
+            }
+            const int nrb = (k + 7) >> 3;
+            for (int c = lane + 32 * pidx; c < nrb * 64; c += 32 * kTcProducers) {
+                const int u = c >> 4;
+                const int n = 8 * (u % nrb) + (c & 7);
+                const int kc = 2 * (u / nrb) + ((c >> 3) & 1);
+                const int kk = k0 + kc * 8;
+                if (n < k) {
+                    const bool v = kk < kend;
+                    cp_async16_zfill(bbase + kmaj64(n, kc * 8), v ? Ap + (int64_t)n * a.d_in + kk : Ap, v);
+                }
+            }
+            tc::cp_async_commit();
+            if (kb >= kTcAhead) {   // stage kb - kTcAhead has landed: hand it to the MMA issuer
+                tc::cp_async_wait<kTcAhead>();
+                tc::fence_proxy_async();
+                mbar_arrive1(&s.full[(kb - kTcAhead) % kTcStages]);
+            }
+        }
+        tc::cp_async_wait<0>();
+        tc::fence_proxy_async();
+        if (ok)
+            for (int kb = max(0, nK - kTcAhead); kb < nK; ++kb) mbar_arrive1(&s.full[kb % kTcStages]);
+    } else if (warp == 1 && lane == 0) {   // MMA issuer
+        const uint32_t idesc = tc::idesc_bf16(kTcM, npad, 0, 0);
+        for (int kb = 0; kb < nK && ok; ++kb) {
+            const int st = kb % kTcStages;
+            ok = mbar_wait(&s.full[st], (uint32_t)((kb / kTcStages) & 1));
+            if (!ok) break;
+            tc::fence_after_sync();
 #pragma unroll
             for (int ks = 0; ks < kTcKB / 16; ++ks) {
                 const uint64_t ad = tc::smem_desc(reinterpret_cast<char*>(s.a[st]) + ks * 256, 128, 1024);
                 const uint64_t bd = tc::smem_desc(reinterpret_cast<char*>(s.b[st]) + ks * 256, 128, 1024);
                 tc::mma_bf16(tmem, ad, bd, idesc, kb > 0 || ks > 0);
             }
-            tc::commit(&s.bar[st]);
+            tc::commit(&s.empty[st]);
         }
+        if (ok) tc::commit(&s.done);
     }
-    tc::cp_async_wait<0>();
-    if (ok) {
-        const int last = nK - 1;
-        ok = mbar_wait(&s.bar[last % kTcStages], (uint32_t)((last / kTcStages) & 1));
-    }
+    __syncwarp();
+    // epilogue: every thread waits for the final commit (a failed role above makes this
+    // wait run out as well; the error is latched either way)
+    ok = ok && mbar_wait(&s.done, 0);
     ok = __syncthreads_and(ok);
     tc::fence_after_sync();
     if (ok) {
@@ -190,18 +212,31 @@ __global__ void __launch_bounds__(kTcThreads) shrink_tc_kernel(TcArgs a) {
 constexpr size_t kShrinkTcSmem = sizeof(ShrinkTcSmem) + 1024;
 
 // ---- expand ---------------------------------------------------------------
-constexpr int kTcStageLd = 68;   // 64 columns + 4: rows stay 16-byte aligned, 4-bank shift per row
+// CTA (token tile of one segment, kTcCols columns of d_out), 256 threads.  The
+// column range is walked in kTcN2-wide steps through a software pipeline:
+//   y tiles (gathered rows of y through the permutation) stream into a 3-buffer
+//   shared-memory ring by cp.async, B'^T tiles into 2 buffers, so the loads of
+//   steps i+1 and i+2 are in flight while step i runs;
+//   one thread issues D = t_hi B + t_lo B (M = 128, N = kTcN2, fp32 in TMEM) and
+//   commits to an mbarrier;
+//   8 warps read D (warp w: lanes 32(w%4).., columns 64(w/4)..), add s*D to the
+//   staged y in shared memory with one bf16 rounding, then the tile is written
+//   back with coalesced 16-byte stores.
+constexpr int kTcN2 = 128;                  // expand step width (UMMA N)
+constexpr int kTcYBuf = 3;
+constexpr int kTcYLd = kTcN2 + 8;           // bf16 per staged y row: 272 bytes, conflict-free 16-byte rows
+constexpr int kTcExpThreads = 256;
 struct ExpandTcSmem {
-    __nv_bfloat16 ahi[kTcM * kMaxRank];   // t_hi, K-major, 16 KB
-    __nv_bfloat16 alo[kTcM * kMaxRank];   // t_lo
-    __nv_bfloat16 b[kMaxRank * kTcN];     // B'^T tile, MN-major, 32 KB
-    float stage[kTcThreads / 32][32][kTcStageLd];   // per-warp accumulator transpose, 34 KB
+    __nv_bfloat16 ahi[kTcM * kMaxRank];          // t_hi, K-major, 16 KB
+    __nv_bfloat16 alo[kTcM * kMaxRank];          // t_lo
+    __nv_bfloat16 b[2][kMaxRank * kTcN2];        // B'^T tiles, MN-major, 16 KB each
+    __nv_bfloat16 yt[kTcYBuf][kTcM * kTcYLd];    // staged y tiles, 34 KB each
     uint64_t bar;
     uint32_t tmem;
     int32_t toks[kTcM];
 };
 
-__global__ void __launch_bounds__(kTcThreads) expand_tc_kernel(TcArgs a) {
+__global__ void __launch_bounds__(kTcExpThreads, 1) expand_tc_kernel(TcArgs a) {
     extern __shared__ __align__(1024) unsigned char tc_raw[];
     auto& s = *reinterpret_cast<ExpandTcSmem*>(tc_raw);
     if ((int)blockIdx.x >= a.counts[3]) return;
@@ -210,17 +245,17 @@ __global__ void __launch_bounds__(kTcThreads) expand_tc_kernel(TcArgs a) {
     const int e_begin = blockIdx.y * kTcCols;
     if (e_begin >= a.d_out) return;
     const int e_end = min(a.d_out, e_begin + kTcCols);
+    const int nit = (e_end - e_begin + kTcN2 - 1) / kTcN2;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int k = it.k, nt = it.ntok;
     const int kpad = (k + 15) & ~15;
-    const uint32_t sbo_a = (uint32_t)(kpad / 8) * 128;   // 8-row groups of the K-major t tiles
-    const uint32_t sbo_b = (uint32_t)(kpad / 8) * 128;   // 8-column groups of the MN-major B tile
-    for (int m = tid; m < kTcM; m += kTcThreads) s.toks[m] = m < nt ? a.perm[it.tok0 + m] : 0;
-    // t tile -> (t_hi, t_lo) bf16, K-major: element (m, j) at (m/8)*sbo_a + (j/8)*128 + (m%8)*16 + (j%8)*2
-    for (int c = tid; c < kTcM * (kpad / 8); c += kTcThreads) {
+    const uint32_t sbo = (uint32_t)(kpad / 8) * 128;   // 8-row groups of t / 8-column groups of B
+    for (int m = tid; m < kTcM; m += kTcExpThreads) s.toks[m] = m < nt ? a.perm[it.tok0 + m] : 0;
+    // t tile -> (t_hi, t_lo) bf16, K-major: element (m, j) at (m/8)*sbo + (j/8)*128 + (m%8)*16 + (j%8)*2
+    const int nsplit = (a.d_in + tc_split_len(a.d_in) - 1) / tc_split_len(a.d_in);
+    for (int c = tid; c < kTcM * (kpad / 8); c += kTcExpThreads) {
         const int m = c % kTcM, jc = c / kTcM;
         float tv[8];
-        const int nsplit = (a.d_in + tc_split_len(a.d_in) - 1) / tc_split_len(a.d_in);
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
             const int j = jc * 8 + i;
@@ -236,104 +271,115 @@ __global__ void __launch_bounds__(kTcThreads) expand_tc_kernel(TcArgs a) {
             hi[i] = __float2bfloat16_rn(tv[i]);
             lo[i] = __float2bfloat16_rn(tv[i] - __bfloat162float(hi[i]));
         }
-        const uint32_t off = (uint32_t)(m >> 3) * sbo_a + (uint32_t)jc * 128 + (uint32_t)(m & 7) * 16;
+        const uint32_t off = (uint32_t)(m >> 3) * sbo + (uint32_t)jc * 128 + (uint32_t)(m & 7) * 16;
         *reinterpret_cast<uint4*>(reinterpret_cast<char*>(s.ahi) + off) = *reinterpret_cast<const uint4*>(hi);
         *reinterpret_cast<uint4*>(reinterpret_cast<char*>(s.alo) + off) = *reinterpret_cast<const uint4*>(lo);
     }
-    if (warp == 0) tc::tmem_alloc(&s.tmem, kTcN);
+    if (warp == 0) tc::tmem_alloc(&s.tmem, kTcN2);
     if (tid == 0) {
         mbar_init(&s.bar, 1);
         fence_barrier_init();
     }
+    __syncthreads();   // toks visible to the copies below
+
+    const __nv_bfloat16* Bt = a.Bt_pool + it.ob;
+    auto issue_y = [&](int i) {   // y rows of step i -> yt[i % 3]; rows past the tile / columns past the range zero-filled
+        const int e0 = e_begin + i * kTcN2;
+        __nv_bfloat16* dst = s.yt[i % kTcYBuf];
+        for (int c = tid; c < kTcM * (kTcN2 / 8); c += kTcExpThreads) {
+            const int row = c >> 4, ch = c & 15;
+            const int e = e0 + ch * 8;
+            const bool ok = row < nt && e < e_end;
+            cp_async16_zfill(dst + row * kTcYLd + ch * 8, ok ? a.y + (int64_t)s.toks[row] * a.d_out + e : a.y, ok);
+        }
+    };
+    auto issue_b = [&](int i) {   // B'^T rows 0..kpad-1 of step i -> b[i % 2], MN-major
+        const int e0 = e_begin + i * kTcN2;
+        char* dst = reinterpret_cast<char*>(s.b[i & 1]);
+        for (int c = tid; c < kpad * (kTcN2 / 8); c += kTcExpThreads) {
+            const int j = c / (kTcN2 / 8), nc = c % (kTcN2 / 8);
+            const int e = e0 + nc * 8;
+            const bool ok = j < k && e < e_end;
+            cp_async16_zfill(dst + (uint32_t)nc * sbo + (uint32_t)(j >> 3) * 128 + (uint32_t)(j & 7) * 16,
+                             ok ? Bt + (int64_t)j * a.d_out + e : Bt, ok);
+        }
+    };
+    issue_y(0);
+    issue_b(0);
+    tc::cp_async_commit();
+    if (nit > 1) {
+        issue_y(1);
+        issue_b(1);
+    }
+    tc::cp_async_commit();
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
     const uint32_t tmem = s.tmem;
-    const uint32_t idesc = tc::idesc_bf16(kTcM, kTcN, 0, 1);
-    const __nv_bfloat16* Bt = a.Bt_pool + it.ob;
+    const uint32_t idesc = tc::idesc_bf16(kTcM, kTcN2, 0, 1);
+    const int q = warp & 3, h = warp >> 2;   // TMEM lane quadrant, column half
+    const int m = 32 * q + lane;             // tile row of this thread in the epilogue
     bool ok = true;
-    int phase = 0;
-    for (int e0 = e_begin; e0 < e_end && ok; e0 += kTcN, ++phase) {
-        // B tile: element (j, n) = B'^T[j][e0 + n] at (n/8)*sbo_b + (j/8)*128 + (j%8)*16 + (n%8)*2
-        for (int c = tid; c < kpad * (kTcN / 8); c += kTcThreads) {
-            const int j = c / (kTcN / 8), nc = c % (kTcN / 8);
-            const int e = e0 + nc * 8;
-            const bool valid = j < k && e < e_end;
-            const __nv_bfloat16* src = valid ? Bt + (int64_t)j * a.d_out + e : Bt;
-            cp_async16_zfill(reinterpret_cast<char*>(s.b) + (uint32_t)nc * sbo_b + (uint32_t)(j >> 3) * 128 +
-                                 (uint32_t)(j & 7) * 16,
-                             src, valid);
-        }
-        tc::cp_async_commit();
-        tc::cp_async_wait<0>();
-        tc::fence_proxy_async();
+    for (int i = 0; i < nit && ok; ++i) {
+        tc::cp_async_wait<1>();              // step i's y and B tiles (this thread's copies)
+        tc::fence_proxy_async();             // B tile -> visible to the tensor core
         __syncthreads();
         if (tid == 0) {
             tc::fence_after_sync();
+            const char* bb = reinterpret_cast<const char*>(s.b[i & 1]);
             for (int ks = 0; ks < kpad / 16; ++ks) {
-                const uint64_t bd = tc::smem_desc(reinterpret_cast<char*>(s.b) + ks * 256, 128, sbo_b);
-                const uint64_t ah = tc::smem_desc(reinterpret_cast<char*>(s.ahi) + ks * 256, 128, sbo_a);
-                const uint64_t al = tc::smem_desc(reinterpret_cast<char*>(s.alo) + ks * 256, 128, sbo_a);
+                const uint64_t bd = tc::smem_desc(bb + ks * 256, 128, sbo);
+                const uint64_t ah = tc::smem_desc(reinterpret_cast<char*>(s.ahi) + ks * 256, 128, sbo);
+                const uint64_t al = tc::smem_desc(reinterpret_cast<char*>(s.alo) + ks * 256, 128, sbo);
                 tc::mma_bf16(tmem, ah, bd, idesc, ks > 0);
                 tc::mma_bf16(tmem, al, bd, idesc, true);
             }
             tc::commit(&s.bar);
         }
-        // y for this warp's 32 token rows, loaded while the MMAs run, in the coalesced
-        // mapping of the epilogue: iteration i covers rows 4*(i%8) + lane/8 of column
-        // block i/8, eight lanes per 128-byte row segment
-        const int cl = (lane & 7) * 8;   // column offset of this lane inside a 64-column block
-        uint4 yv[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            const int rr = warp * 32 + 4 * (i & 7) + (lane >> 3);
-            const int e = e0 + 64 * (i >> 3) + cl;
-            yv[i] = (rr < nt && e < e_end)
-                        ? *reinterpret_cast<const uint4*>(a.y + (int64_t)s.toks[rr] * a.d_out + e)
-                        : make_uint4(0, 0, 0, 0);
-        }
-        ok = mbar_wait(&s.bar, (uint32_t)(phase & 1));
+        if (i + 2 < nit) issue_y(i + 2);     // yt[(i+2) % 3] held step i-1, already written back
+        ok = mbar_wait(&s.bar, (uint32_t)(i & 1));
         tc::fence_after_sync();
+        if (i + 2 < nit) issue_b(i + 2);     // b[i % 2] is free once the MMAs of step i completed
+        tc::cp_async_commit();
+        __nv_bfloat16* yt = s.yt[i % kTcYBuf];
         if (ok) {
-            float (*st)[kTcStageLd] = s.stage[warp];
 #pragma unroll
-            for (int blk = 0; blk < kTcN / 64; ++blk) {
-                // accumulator rows (one per lane) of this 64-column block -> shared memory
+            for (int c16 = 0; c16 < 4; ++c16) {
+                float v[16];
+                tc::tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(64 * h + 16 * c16), v);
+                uint4* yp = reinterpret_cast<uint4*>(yt + m * kTcYLd + 64 * h + 16 * c16);
 #pragma unroll
-                for (int c16 = 0; c16 < 4; ++c16) {
-                    float v[16];
-                    tc::tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(blk * 64 + c16 * 16), v);
+                for (int half = 0; half < 2; ++half) {
+                    uint4 yv = yp[half];
+                    __nv_bfloat162* y2 = reinterpret_cast<__nv_bfloat162*>(&yv);
 #pragma unroll
-                    for (int q = 0; q < 4; ++q)
-                        *reinterpret_cast<float4*>(&st[lane][c16 * 16 + 4 * q]) =
-                            make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
-                }
-                __syncwarp();
-#pragma unroll
-                for (int i8 = 0; i8 < 8; ++i8) {
-                    const int i = blk * 8 + i8;
-                    const int rl = 4 * i8 + (lane >> 3);   // row inside the warp's 32
-                    const int rr = warp * 32 + rl;
-                    const int e = e0 + 64 * blk + cl;
-                    const float4 p0 = *reinterpret_cast<const float4*>(&st[rl][cl]);
-                    const float4 p1 = *reinterpret_cast<const float4*>(&st[rl][cl + 4]);
-                    const float acc[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
-                    __nv_bfloat162* p2 = reinterpret_cast<__nv_bfloat162*>(&yv[i]);
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const float2 yf = __bfloat1622float2(p2[q]);
-                        p2[q] = __floats2bfloat162_rn(fmaf(a.scale, acc[2 * q], yf.x), fmaf(a.scale, acc[2 * q + 1], yf.y));
+                    for (int p = 0; p < 4; ++p) {
+                        const float2 yf = __bfloat1622float2(y2[p]);
+                        y2[p] = __floats2bfloat162_rn(fmaf(a.scale, v[8 * half + 2 * p], yf.x),
+                                                      fmaf(a.scale, v[8 * half + 2 * p + 1], yf.y));
                     }
-                    if (rr < nt && e < e_end)
-                        *reinterpret_cast<uint4*>(a.y + (int64_t)s.toks[rr] * a.d_out + e) = yv[i];
+                    yp[half] = yv;
                 }
-                __syncwarp();
             }
         }
         tc::fence_before_sync();
-        ok = __syncthreads_and(ok);   // B tile and tensor memory free for the next tile; uniform ok
+        ok = __syncthreads_and(ok);          // staged tile complete; TMEM free for the next MMA
+        if (ok) {
+            const int e0 = e_begin + i * kTcN2;
+            for (int c = tid; c < kTcM * (kTcN2 / 8); c += kTcExpThreads) {
+                const int row = c >> 4, ch = c & 15;
+                const int e = e0 + ch * 8;
+                if (row < nt && e < e_end)
+                    *reinterpret_cast<uint4*>(a.y + (int64_t)s.toks[row] * a.d_out + e) =
+                        *reinterpret_cast<const uint4*>(yt + row * kTcYLd + ch * 8);
+            }
+        }
     }
-    if (warp == 0) tc::tmem_dealloc(tmem, kTcN);
+    tc::cp_async_wait<0>();
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    if (warp == 0) tc::tmem_dealloc(tmem, kTcN2);
 }
 
 constexpr size_t kExpandTcSmem = sizeof(ExpandTcSmem) + 1024;

@@ -137,3 +137,27 @@ def test_empty_batch_and_all_unrouted():
     assert st == 0 and torch.equal(y, y0) and seg[0] == 0 and seg[1] == 0
     y, _, st = run_apply(x[:0], y0[:0], [], [2], offA, offB, Ap, Bt, 1.0)
     assert st == 0 and y.shape == (0, d)
+
+
+def test_routing_of_long_mixed_batch():
+    # > 4 chunks of the routing block: long runs (prefill requests), single tokens
+    # (decode requests) and unrouted tokens interleaved; the segment table and the
+    # permutation must equal the stable argsort bit for bit
+    g = np.random.default_rng(17)
+    n, d = 100, 256
+    parts = []
+    while sum(len(p) for p in parts) < 5000:
+        if g.random() < 0.3:
+            parts.append(np.full(int(g.integers(20, 400)), int(g.integers(0, n)), dtype=np.int32))
+        else:
+            parts.append(g.integers(-1, n, size=int(g.integers(1, 40))).astype(np.int32))
+    ids = np.concatenate(parts)[:5000]
+    T = len(ids)
+    ranks = g.integers(1, 17, size=n)
+    offA, offB, Ap, Bt = make_pools(ranks, d, d, (7, 0))
+    x = synth.normal_bf16((T, d), (7, 1))
+    y0 = torch.zeros(T, d, dtype=torch.bfloat16)
+    y, seg, st = run_apply(x, y0, ids, ranks, offA, offB, Ap, Bt, 1.0, seg=True)
+    assert st == 0
+    check_routing(seg, ids, n)
+    assert_close(y, oracle_y(x, y0, ids, ranks, offA, offB, Ap, Bt, 1.0))
