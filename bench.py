@@ -9,11 +9,17 @@ TSQR + small SVD (lf_tsqr_batched) followed by allocation, fp64 boundary
 refinement and export of the ragged fp32+bf16 pools (lf_truncate_export).
 Metric: modules/s, plus the fraction of the HBM roofline.
 
-Also reported in the same line (``lora_path``): the rank-specialised side path
-y += s B'(A'x) on the decode workload (Llama-3-8B shapes, 32 layers x 7
-projections, 256 tokens over 128 adapters with Zipf(1) ids, ranks from the S
-allocation of synthetic spectra) and the prefill workload (Qwen2.5-7B layer,
-32 requests x 512 tokens, k = 16 and uncompressed r = 64), in tokens/s.
+Also reported in the same line:
+* ``lora_path``: the rank-specialised side path y += s B'(A'x) on the decode
+  workload (Llama-3-8B shapes, 32 layers x 7 projections, 256 tokens over 128
+  adapters with Zipf(1) ids, ranks from the S allocation of synthetic spectra),
+  with its padded-to-max and uncompressed rank-64 variants, and the prefill
+  workload (Qwen2.5-7B layer, 32 requests x 512 tokens, k = 16 and uncompressed
+  r = 64), in tokens/s;
+* ``large_fleet``: 1024 Llama-3-8B-shaped adapters compressed in chunks of 64,
+  then a mixed 4096-token batch through all 32 layers, ragged vs padded;
+* ``library_qr_context``: torch.linalg.qr (cuSOLVER) on one adapter's modules
+  next to this library's TSQR on the same bytes.
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl loraforge|reference]
 For N > 1 launch under torchrun; every rank compresses its own fleet (weak scaling).
@@ -297,8 +303,11 @@ def apply_bytes(T, d_in, d_out, ranks_used):
     return 2 * T * d_in + 4 * T * d_out + 4 * T + sum(2 * k * (d_in + d_out) for k in ranks_used)
 
 
-def decode_bench(args, dev, stream, hbm):
-    """Config 3: Llama-3-8B shapes, 32 layers x 7 projections, T=256, 128 adapters."""
+def decode_bench(args, dev, stream, hbm, variant="ragged"):
+    """Config 3: Llama-3-8B shapes, 32 layers x 7 projections, T=256, 128 adapters.
+    variant: "ragged" (retained ranks as allocated), "padded" (every adapter's factors
+    of a projection zero-padded to the largest retained rank over the 128 resident
+    adapters), "r64" (uncompressed rank-64 adapters)."""
     import torch
     from post_hoc_rank_b200 import api, synth
     from post_hoc_rank_b200 import loraforge as lf
@@ -320,20 +329,37 @@ def decode_bench(args, dev, stream, hbm):
         x_h = synth.normal_bf16((T, M.hidden), (3, 1, l), device=dev)
         x_f = synth.normal_bf16((T, M.ffn), (3, 2, l), device=dev)
         for p, (_, d_out, d_in) in enumerate(shapes):
-            rk = ranks_all[:, p, l].astype(np.int64)
+            rk_true = ranks_all[:, p, l].astype(np.int64)
+            if variant == "ragged":
+                rk = rk_true
+            elif variant == "padded":
+                rk = np.full(n_ad, int(rk_true.max()), dtype=np.int64)
+            else:
+                rk = np.full(n_ad, 64, dtype=np.int64)
             offA = np.concatenate([[0], np.cumsum(rk * d_in)]); offB = np.concatenate([[0], np.cumsum(rk * d_out)])
             Ap = synth.normal_bf16((int(offA[-1]),), (3, 3, l, p), std=d_in ** -0.5, device=dev)
             Bt = synth.normal_bf16((int(offB[-1]),), (3, 4, l, p), std=d_out ** -0.5, device=dev)
+            if variant == "padded":   # rows past each adapter's retained rank are zero
+                kmax = int(rk[0])
+                pad = torch.from_numpy(np.arange(kmax)[None, :] >= rk_true[:, None]).to(dev)
+                Ap.view(n_ad, kmax, d_in)[pad] = 0
+                Bt.view(n_ad, kmax, d_out)[pad] = 0
             y = synth.normal_bf16((T, d_out), (3, 5, l, p), device=dev)
             x = x_f if d_in == M.ffn else x_h
             ws = api.workspace(lf.lf_apply_workspace_size(T, n_ad), dev)
             calls.append((x, y, torch.from_numpy(rk.astype(np.int32)).to(dev),
                           torch.from_numpy(offA[:-1]).to(dev), torch.from_numpy(offB[:-1]).to(dev), Ap, Bt, ws))
             total_bytes += apply_bytes(T, d_in, d_out, [int(rk[a]) for a in distinct])
-    return _apply_run(args, calls, ids_d, n_ad, T, total_bytes, stream, hbm, dict(
+    names = {"ragged": "S 1/12 floor 1 ranks (ragged)",
+             "padded": "S 1/12 floor 1 ranks zero-padded to the per-projection max over resident adapters",
+             "r64": "uncompressed rank-64 adapters"}
+    out = _apply_run(args, calls, ids_d, n_ad, T, total_bytes, stream, hbm, dict(
         workload="decode: Llama-3-8B, 32 layers x 7 projections, 256 tokens, 128 adapters Zipf(1), "
-                 "S 1/12 floor 1 ranks", distinct_adapters=len(distinct),
+                 + names[variant], distinct_adapters=len(distinct),
         mean_rank=float(ranks_all.mean())))
+    del calls
+    torch.cuda.empty_cache()
+    return out
 
 
 def prefill_bench(args, dev, stream, hbm, k):
@@ -414,6 +440,208 @@ def _apply_run(args, calls, ids_d, n_ad, T, total_bytes, stream, hbm, meta):
     return out
 
 
+def large_fleet_bench(args, dev, stream, hbm):
+    """Config 5: 1024 Llama-3-8B-shaped adapters (224 modules each, r = 64), compressed
+    with LoRAForge-S 1/12 floor 1 in chunks of 64 adapters (each chunk generated in
+    HBM, then one lf_tsqr_batched + lf_truncate_export, device-timed), then a mixed
+    batch of 4096 tokens (64 prefill segments x 48 tokens + 1024 decode tokens, ids
+    Zipf(1.2) over the 1024 adapters) through all 32 layers x 7 projections with the
+    exported bf16 factors, ragged and padded to the per-projection max rank over the
+    adapters the batch references."""
+    import torch
+    from post_hoc_rank_b200 import api, synth
+    from post_hoc_rank_b200 import loraforge as lf
+
+    M = synth.LLAMA3_8B
+    n_total, chunk = args.large_adapters, 64
+    nchunks = (n_total + chunk - 1) // chunk
+    lay = synth.fleet_layout(chunk, M, r=64)
+    mods = api.modules_from_layout(lay)
+    B = torch.empty(lay.B_total, dtype=torch.float32, device=dev)
+    A = torch.empty(lay.A_total, dtype=torch.float32, device=dev)
+    pol = lf.lf_policy(*POLICY)
+    F = api.alloc_factors(mods, dev)
+    E = api.alloc_export(mods, pol, dev, bf16=True)
+    ws_t = api.workspace(lf.lf_tsqr_workspace_size(mods), dev)
+    ws_e = api.workspace(lf.lf_export_workspace_size(mods), dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    compress_ms, ranks_c, offA_c, offB_c, poolsA, poolsB = 0.0, [], [], [], [], []
+    for c in range(nchunks):
+        synth.fill_fleet(lay, B, A, cfg_id=5, adapter_base=c * chunk)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        api.tsqr(mods, B, A, out=F, ws=ws_t, stream=stream)
+        api.truncate_export(mods, pol, B, A, F, out=E, ws=ws_e, stream=stream)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        compress_ms += e0.elapsed_time(e1)
+        assert lf.lf_get_device_status(stream) == 0
+        oa, ob = E.off_A.cpu().numpy(), E.off_Bt.cpu().numpy()
+        ranks_c.append(E.ranks.cpu().numpy()); offA_c.append(oa); offB_c.append(ob)
+        poolsA.append(E.A_pool16[:int(oa[-1])].clone()); poolsB.append(E.Bt_pool16[:int(ob[-1])].clone())
+    n_mod = nchunks * lay.n
+    del B, A, F, E, ws_t, ws_e
+    torch.cuda.empty_cache()
+    baseA = np.concatenate([[0], np.cumsum([p.numel() for p in poolsA])]).astype(np.int64)
+    baseB = np.concatenate([[0], np.cumsum([p.numel() for p in poolsB])]).astype(np.int64)
+    poolA = torch.cat(poolsA); poolB = torch.cat(poolsB)
+    del poolsA, poolsB
+    torch.cuda.empty_cache()
+    # module index of (adapter, proj, layer) inside a chunk: (a_local * 7 + p) * layers + l
+    a_all = np.arange(nchunks * chunk)
+    cidx, aloc = a_all // chunk, a_all % chunk
+    T = 4096
+    seg_ids = synth.zipf_ids(64, n_total, 1.2, (5, 1))
+    dec_ids = synth.zipf_ids(1024, n_total, 1.2, (5, 2))
+    ids = np.concatenate([np.repeat(seg_ids, 48), dec_ids]).astype(np.int32)
+    ids_d = torch.from_numpy(ids).to(dev)
+    ref = np.unique(ids)
+    shapes = M.proj_shapes()
+    out = {"workload": f"large fleet: {n_total} adapters x Llama-3-8B (224 modules each, r=64), LoRAForge-S "
+                       "1/12 floor 1, compressed in chunks of 64 adapters; then 4096 tokens (64 prefill segments "
+                       "x 48 + 1024 decode tokens, Zipf(1.2) ids) through 32 layers x 7 projections",
+           "modules": int(n_mod), "compress_ms": round(compress_ms, 2),
+           "modules_per_s": round(n_mod / (compress_ms * 1e-3), 1), "distinct_adapters": int(len(ref))}
+    for variant in ("ragged", "padded"):
+        calls, total_bytes = [], 0
+        for l in range(M.layers):
+            x_h = synth.normal_bf16((T, M.hidden), (5, 3, l), device=dev)
+            x_f = synth.normal_bf16((T, M.ffn), (5, 4, l), device=dev)
+            for p, (_, d_out, d_in) in enumerate(shapes):
+                mi = (aloc * 7 + p) * M.layers + l
+                rk = np.array([ranks_c[c][m] for c, m in zip(cidx, mi)], dtype=np.int64)
+                oa = np.array([baseA[c] + offA_c[c][m] for c, m in zip(cidx, mi)], dtype=np.int64)
+                ob = np.array([baseB[c] + offB_c[c][m] for c, m in zip(cidx, mi)], dtype=np.int64)
+                y = synth.normal_bf16((T, d_out), (5, 5, l, p), device=dev)
+                x = x_f if d_in == M.ffn else x_h
+                if variant == "ragged":
+                    k_used = rk[ref]
+                    pa, pb, rk_d, oa_d, ob_d = poolA, poolB, rk, oa, ob
+                else:
+                    # padded pools for the referenced adapters: kmax rows each, rows past k zero
+                    kmax = int(rk[ref].max())
+                    jr = torch.arange(kmax, device=dev)
+                    live = (jr[None, :] < torch.from_numpy(rk[ref]).to(dev)[:, None])
+                    rows_a = torch.from_numpy(oa[ref]).to(dev)[:, None] + jr[None, :] * d_in
+                    rows_b = torch.from_numpy(ob[ref]).to(dev)[:, None] + jr[None, :] * d_out
+                    ia = (rows_a[:, :, None] + torch.arange(d_in, device=dev)[None, None, :]) * live[:, :, None]
+                    ib = (rows_b[:, :, None] + torch.arange(d_out, device=dev)[None, None, :]) * live[:, :, None]
+                    pa = (poolA[ia] * live[:, :, None]).reshape(-1).contiguous()
+                    pb = (poolB[ib] * live[:, :, None]).reshape(-1).contiguous()
+                    del ia, ib
+                    rk_d = np.zeros(n_total, dtype=np.int64); rk_d[ref] = kmax
+                    oa_d = np.zeros(n_total, dtype=np.int64); ob_d = np.zeros(n_total, dtype=np.int64)
+                    oa_d[ref] = np.arange(len(ref)) * kmax * d_in; ob_d[ref] = np.arange(len(ref)) * kmax * d_out
+                    k_used = np.full(len(ref), kmax)
+                ws = api.workspace(lf.lf_apply_workspace_size(T, n_total), dev)
+                calls.append((x, y, torch.from_numpy(rk_d.astype(np.int32)).to(dev), torch.from_numpy(oa_d).to(dev),
+                              torch.from_numpy(ob_d).to(dev), pa, pb, ws))
+                total_bytes += apply_bytes(T, d_in, d_out, [int(k) for k in k_used])
+        r = _apply_run(args, calls, ids_d, n_total, T, total_bytes, stream, hbm, {})
+        out[variant] = {k: r[k] for k in ("tokens_per_s", "ms_per_step", "algo_bytes", "achieved_gbs", "hbm_frac",
+                                          "launches_per_step", "phases_ms")}
+        del calls
+        torch.cuda.empty_cache()
+    del poolA, poolB
+    torch.cuda.empty_cache()
+    return out
+
+
+def library_qr_context(dev, stream):
+    """Matched library QR on the same modules: torch.linalg.qr (cuSOLVER geqrf, R only)
+    on one Qwen2.5-7B-shaped adapter (196 modules, r = 64), B and A^T of each projection
+    batched over the 28 layers, against this library's TSQR phases on the same bytes."""
+    import torch
+    from post_hoc_rank_b200 import api, synth
+    from post_hoc_rank_b200 import loraforge as lf
+
+    M = synth.QWEN25_7B
+    lay = synth.fleet_layout(1, M, r=64)
+    mods = api.modules_from_layout(lay)
+    B = torch.empty(lay.B_total, dtype=torch.float32, device=dev)
+    A = torch.empty(lay.A_total, dtype=torch.float32, device=dev)
+    synth.fill_fleet(lay, B, A, cfg_id=2, adapter_base=20_000)
+    groups = []
+    for p, (_, d_out, d_in) in enumerate(M.proj_shapes()):
+        i0 = p * M.layers
+        Bs = torch.stack([B[int(lay.B_off[i0 + l]):int(lay.B_off[i0 + l]) + d_out * 64].view(d_out, 64)
+                          for l in range(M.layers)])
+        As = torch.stack([A[int(lay.A_off[i0 + l]):int(lay.A_off[i0 + l]) + 64 * d_in].view(64, d_in)
+                          for l in range(M.layers)]).transpose(1, 2)
+        groups.append((Bs, As))
+
+    def lib_step():
+        for Bs, As in groups:
+            torch.linalg.qr(Bs, mode="r"); torch.linalg.qr(As, mode="r")
+
+    F = api.alloc_factors(mods, dev)
+    ws = api.workspace(lf.lf_tsqr_workspace_size(mods), dev)
+    for _ in range(2):
+        lib_step(); api.tsqr(mods, B, A, out=F, ws=ws, stream=stream)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    reps = 3
+    e0.record(stream)
+    for _ in range(reps):
+        lib_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    lib_ms = e0.elapsed_time(e1) / reps
+    lf.lf_profile_reset(); lf.lf_profile_enable(True)
+    for _ in range(reps):
+        api.tsqr(mods, B, A, out=F, ws=ws, stream=stream)
+    lf.lf_profile_enable(False)
+    ph = lf.lf_profile_read()
+    qr_ms = sum(ph[k][0] for k in ("tsqr_gram_leaf", "tsqr_householder") if k in ph) / reps
+    del B, A, F, ws, groups
+    torch.cuda.empty_cache()
+    return {"sample": "one Qwen2.5-7B-shaped adapter, 196 modules, B and A^T (R only)",
+            "library": "torch.linalg.qr (cuSOLVER), per projection batched over 28 layers",
+            "library_ms": round(lib_ms, 3), "tsqr_ms": round(qr_ms, 3),
+            "library_modules_per_s": round(lay.n / (lib_ms * 1e-3), 1),
+            "tsqr_modules_per_s": round(lay.n / (qr_ms * 1e-3), 1),
+            "speedup_vs_library": round(lib_ms / qr_ms, 2)}
+
+
+def cpu_apply_baseline():
+    """The oracle's brute-force fp64 apply on the host: layer 0 of the decode workload
+    (7 Llama-3-8B projections, 256 tokens, 128 adapters, S-policy ranks), scaled to the
+    32-layer step."""
+    import torch
+    from oracle import apply as OP
+    from post_hoc_rank_b200 import api, synth
+    from post_hoc_rank_b200 import loraforge as lf
+
+    M = synth.LLAMA3_8B
+    n_ad, T = 128, 256
+    sig = synth.sigma_tables(n_ad, M, 64, cfg_id=3)
+    lay = synth.fleet_layout(n_ad, M, r=64)
+    ranks = OA_spectral(sig, lay)
+    ranks = ranks.reshape(n_ad, 7, M.layers)
+    ids = synth.zipf_ids(T, n_ad, 1.0, (3, 0))
+    t_total = 0.0
+    for p, (_, d_out, d_in) in enumerate(M.proj_shapes()):
+        rk = ranks[:, p, 0].astype(np.int64)
+        offA = np.concatenate([[0], np.cumsum(rk * d_in)]); offB = np.concatenate([[0], np.cumsum(rk * d_out)])
+        Ap = synth.normal_bf16((int(offA[-1]),), (3, 3, 0, p), std=d_in ** -0.5).float().numpy()
+        Bt = synth.normal_bf16((int(offB[-1]),), (3, 4, 0, p), std=d_out ** -0.5).float().numpy()
+        x = synth.normal_bf16((T, d_in), (3, 1, 0)).float().numpy()
+        y = synth.normal_bf16((T, d_out), (3, 5, 0, p)).float().numpy()
+        t0 = time.perf_counter()
+        OP.lora_apply(x, y, ids, rk, offA[:-1], offB[:-1], Ap, Bt, 2.0)
+        t_total += time.perf_counter() - t0
+    step_s = t_total * M.layers
+    return {"value": round(T / step_s, 1), "unit": "tokens/s", "cores": torch.get_num_threads(), "kind": "oracle",
+            "sample": "layer 0 of the decode workload (7 projections, 256 tokens), fp64 brute force, "
+                      "time x 32 layers"}
+
+
+def OA_spectral(sig, lay):
+    from oracle import allocate as OA
+    ranks, _ = OA.spectral_ranks(sig, lay.r, lay.group, 1, 12, 1)
+    return np.asarray(ranks)
+
+
 # ----------------------------------------------------------- CPU baseline
 def cpu_oracle_adapter(cfg_id=2, adapter=0, model=None, n_layers=None):
     """The fp64 oracle's fleet route on one Qwen-shaped adapter (196 modules, or the
@@ -458,6 +686,8 @@ def main():
     ap.add_argument("--no-apply", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-large", action="store_true")
+    ap.add_argument("--large-adapters", type=int, default=1024)
     args = ap.parse_args()
 
     rank = int(os.environ.get("RANK", "0"))
@@ -510,13 +740,23 @@ def main():
     step_gbs = step_bytes_2touch / (ms_step * 1e-3) / 1e9
 
     lora = None
-    if not args.no_apply:
+    if not args.no_apply and rank == 0:   # per-GPU side-path figures: rank 0 only
         lora = {"decode": decode_bench(args, dev, stream, hbm),
+                "decode_padded_to_max": decode_bench(args, dev, stream, hbm, "padded"),
+                "decode_uncompressed_r64": decode_bench(args, dev, stream, hbm, "r64"),
                 "prefill_k16": prefill_bench(args, dev, stream, hbm, 16),
                 "prefill_r64": prefill_bench(args, dev, stream, hbm, 64)}
+        if rank == 0 and not args.no_cpu:
+            lora["decode"]["cpu_baseline"] = cpu_apply_baseline()
+    large = None if (args.no_large or rank != 0) else large_fleet_bench(args, dev, stream, hbm)
+    libqr = None if (args.no_apply or rank != 0) else library_qr_context(dev, stream)
     e2e = None
     if not args.no_e2e:
         e = factor_e2e(args, dev, stream)
+        if pg is not None:   # every rank compresses its own adapters: whole-job rate over the slowest rank
+            t = torch.tensor([e["modules"] / e["value"]], dtype=torch.float64, device=dev)
+            pg.all_reduce(t, op=pg.ReduceOp.MAX)
+            e["value"] = e["modules"] * world / float(t.item())
         e2e = {"value": round(e["value"], 1), "unit": "modules/s", "h2d_bytes_per_step": e["h2d"],
                "d2h_bytes_per_step": e["d2h"],
                "sample": f"{e['adapters']} adapters ({e['modules']} modules) from pinned host memory"}
@@ -543,6 +783,8 @@ def main():
         "clocks": fr["clocks"],
         "e2e": e2e,
         "lora_path": lora,
+        "large_fleet": large,
+        "library_qr_context": libqr,
         "cpu_baseline": cpu,
         "device_status": fr["status"],
     }
