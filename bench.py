@@ -200,6 +200,28 @@ def dominant_roofline(dom, per_launch_ms, fr, hbm, peak_kind, sm_mhz):
             "peak_source": peak_kind}
 
 
+# ------------------------------------------------------------ sharding
+def shard_adapter_base(rank: int, n_adapters_per_rank: int) -> int:
+    """Adapters are sharded across ranks with no exchange (the S budget is per adapter):
+    rank r compresses adapters [r * n, (r + 1) * n) of the fleet."""
+    return rank * n_adapters_per_rank
+
+
+def max_over_ranks(x: float, pg, dev) -> float:
+    """Max of a per-rank device time over all ranks (identity without a process group)."""
+    if pg is None:
+        return x
+    import torch
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_rank: int, world: int, max_ms: float) -> float:
+    """Units all ranks processed divided by the slowest rank's time (per second)."""
+    return units_per_rank * world / (max_ms * 1e-3)
+
+
 # ------------------------------------------------------------ factor path
 def factor_bench(args, rank, world, dev, sync_all, stream, hbm, peak_kind):
     import torch
@@ -211,7 +233,7 @@ def factor_bench(args, rank, world, dev, sync_all, stream, hbm, peak_kind):
     mods = api.modules_from_layout(lay)
     B = torch.empty(lay.B_total, dtype=torch.float32, device=dev)
     A = torch.empty(lay.A_total, dtype=torch.float32, device=dev)
-    synth.fill_fleet(lay, B, A, cfg_id=2, adapter_base=rank * n_ad)
+    synth.fill_fleet(lay, B, A, cfg_id=2, adapter_base=shard_adapter_base(rank, n_ad))
     pol = lf.lf_policy(*POLICY)
     F = api.alloc_factors(mods, dev)
     E = api.alloc_export(mods, pol, dev, bf16=True)
@@ -251,7 +273,7 @@ def factor_bench(args, rank, world, dev, sync_all, stream, hbm, peak_kind):
     return res
 
 
-def factor_e2e(args, dev, stream):
+def factor_e2e(args, dev, stream, rank=0):
     """Same step through the C ABI with the inputs in pinned HOST memory: the H2D copy of
     B and A and the D2H copy of the rank table, offsets and bf16 pools are timed."""
     import torch
@@ -265,7 +287,7 @@ def factor_e2e(args, dev, stream):
     Ah = torch.empty(lay.A_total, dtype=torch.float32, pin_memory=True)
     Bd = torch.empty(lay.B_total, dtype=torch.float32, device=dev)
     Ad = torch.empty(lay.A_total, dtype=torch.float32, device=dev)
-    synth.fill_fleet(lay, Bd, Ad, cfg_id=2, adapter_base=10_000)
+    synth.fill_fleet(lay, Bd, Ad, cfg_id=2, adapter_base=10_000 + shard_adapter_base(rank, n_ad))
     Bh.copy_(Bd); Ah.copy_(Ad)
     pol = lf.lf_policy(*POLICY)
     F = api.alloc_factors(mods, dev)
@@ -721,13 +743,8 @@ def main():
     stream = torch.cuda.current_stream()
     hbm, peak_kind = peaks()
     fr = factor_bench(args, rank, world, dev, sync_all, stream, hbm, peak_kind)
-    ms = fr["ms"]
-    if pg is not None:
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        ms = float(t.item())
-    total_modules = fr["n"] * args.steps * world
-    value = total_modules / (ms * 1e-3)
+    ms = max_over_ranks(fr["ms"], pg, dev)
+    value = whole_job_rate(fr["n"] * args.steps, world, ms)
     ms_step = ms / args.steps
 
     # dominant kernel roofline
@@ -752,11 +769,9 @@ def main():
     libqr = None if (args.no_apply or rank != 0) else library_qr_context(dev, stream)
     e2e = None
     if not args.no_e2e:
-        e = factor_e2e(args, dev, stream)
+        e = factor_e2e(args, dev, stream, rank)
         if pg is not None:   # every rank compresses its own adapters: whole-job rate over the slowest rank
-            t = torch.tensor([e["modules"] / e["value"]], dtype=torch.float64, device=dev)
-            pg.all_reduce(t, op=pg.ReduceOp.MAX)
-            e["value"] = e["modules"] * world / float(t.item())
+            e["value"] = whole_job_rate(e["modules"], world, max_over_ranks(1e3 * e["modules"] / e["value"], pg, dev))
         e2e = {"value": round(e["value"], 1), "unit": "modules/s", "h2d_bytes_per_step": e["h2d"],
                "d2h_bytes_per_step": e["d2h"],
                "sample": f"{e['adapters']} adapters ({e['modules']} modules) from pinned host memory"}
