@@ -49,7 +49,6 @@ struct RouteOut {
     // consecutive ids (the histogram and the stable scatter touch runs, not tokens).
     int32_t* run_start;  // first token of run i
     int32_t* run_pos;    // position of run i's first token in the permutation
-    int32_t* tok_run;    // run index of every token
 };
 
 // Block-wide exclusive scan of one int per thread (blockDim.x a multiple of 32, <= 1024).
@@ -124,10 +123,8 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const int32_t* __r
             for (int i = t0; i < t1; ++i) nf += (s_idc[i + 1] != s_idc[i]);
             int tot;
             int ri = block_excl_scan(nf, wsum, &tot) + s_carry[0] - 1;
-            for (int i = t0; i < t1; ++i) {
+            for (int i = t0; i < t1; ++i)
                 if (s_idc[i + 1] != s_idc[i]) o.run_start[++ri] = base + i;
-                o.tok_run[base + i] = ri;
-            }
             __syncthreads();
             if (tid == 0) s_carry[0] += tot;
             __syncthreads();
@@ -246,9 +243,13 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const int32_t* __r
             if (a >= 0) o.run_pos[ri] = wbase[warp][leader] + before;
             __syncthreads();
         }
-        for (int t = tid; t < T; t += nthr) {
-            const int ri = o.tok_run[t];
-            if (valid_id(t) >= 0) o.perm[o.run_pos[ri] + t - o.run_start[ri]] = t;
+        // permutation: one warp per run writes the run's consecutive token indices
+        for (int ri = warp; ri < n_runs; ri += nthr / 32) {
+            const int t0 = o.run_start[ri];
+            if (valid_id(t0) < 0) continue;
+            const int len = (ri + 1 < n_runs ? o.run_start[ri + 1] : T) - t0;
+            const int p0 = o.run_pos[ri];
+            for (int i = lane; i < len; i += 32) o.perm[p0 + i] = t0 + i;
         }
         __syncthreads();
     }
@@ -490,7 +491,7 @@ struct BgmvArgs {
     float scale;
 };
 
-__global__ void __launch_bounds__(kBgmvThreads) bgmv_kernel(BgmvArgs a) {
+__global__ void __launch_bounds__(kBgmvThreads, 4) bgmv_kernel(BgmvArgs a) {
     __shared__ float red[kBgmvThreads / 32][kBgmvJ];
     __shared__ float ts[kMaxRank];
     const int tok = blockIdx.x;

@@ -696,7 +696,7 @@ size_t lf_apply_workspace_size(int32_t T, int32_t n_adapters) {
     c.take<float>((size_t)std::max(T, 1) * kMaxRank);
     c.take<TcItem>((size_t)(T / kTcM + mseg + 1));
     c.take<float>((size_t)kTcMaxSplit * std::max(T, 1) * kMaxRank);
-    c.take<int32_t>((size_t)3 * std::max(T, 1));   // run scratch of the routing pass
+    c.take<int32_t>((size_t)2 * std::max(T, 1));   // run scratch of the routing pass
     return c.off + 256;
 }
 
@@ -725,10 +725,9 @@ lf_status lf_lora_shrink_expand(int32_t T, int32_t d_in, int32_t d_out, const vo
     float* t_buf = c.take<float>((size_t)T * kMaxRank);
     o.tc_items = c.take<TcItem>((size_t)(T / kTcM + mseg + 1));
     float* t_part = c.take<float>((size_t)kTcMaxSplit * T * kMaxRank);
-    int32_t* run_scratch = c.take<int32_t>((size_t)3 * T);
+    int32_t* run_scratch = c.take<int32_t>((size_t)2 * T);
     o.run_start = run_scratch;
     o.run_pos = run_scratch + T;
-    o.tok_run = run_scratch + 2 * T;
     o.seg_out = seg_out;
     o.ranks = ranks;
     o.off_A = off_A;
