@@ -272,15 +272,34 @@ struct SvdArgs {
 };
 
 template <typename T, int RT>
-struct SvdSmem {
-    T M[RT][RT + 1];
-    T Ut[RT][RT + 1];   // Ut[p] = column p of U
+struct alignas(16) SvdSmem {
+    static constexpr int LD = RT + 16 / (int)sizeof(T);   // 16-byte aligned rows, 4-bank shift per row
+    T M[RT][LD];
+    T Ut[RT][LD];   // Ut[p] = column p of U
     T sig[RT];
     int perm[RT];
 };
 
+// Four consecutive elements from / to a 16-byte aligned address in shared memory.
+__device__ __forceinline__ void ld4(const float* p, float (&v)[4]) {
+    const float4 f = *reinterpret_cast<const float4*>(p);
+    v[0] = f.x; v[1] = f.y; v[2] = f.z; v[3] = f.w;
+}
+__device__ __forceinline__ void ld4(const double* p, double (&v)[4]) {
+    const double2 a = reinterpret_cast<const double2*>(p)[0], b = reinterpret_cast<const double2*>(p)[1];
+    v[0] = a.x; v[1] = a.y; v[2] = b.x; v[3] = b.y;
+}
+__device__ __forceinline__ void st4(float* p, const float (&v)[4]) {
+    *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+}
+__device__ __forceinline__ void st4(double* p, const double (&v)[4]) {
+    reinterpret_cast<double2*>(p)[0] = make_double2(v[0], v[1]);
+    reinterpret_cast<double2*>(p)[1] = make_double2(v[2], v[3]);
+}
+
+// One warp (one module) per CTA: a finished module frees its shared memory at once.
 template <typename T>
-__host__ __device__ constexpr int svd_warps() { return sizeof(T) == 8 ? 1 : 2; }
+__host__ __device__ constexpr int svd_warps() { return 1; }
 // Rotation threshold |gamma| > tol * sqrt(alpha beta): r * eps of the working type
 // (a tighter threshold cannot be met by rotations computed in that type).
 template <typename T>
@@ -346,13 +365,16 @@ __global__ void __launch_bounds__(32 * svd_warps<T>()) svd_kernel(SvdArgs<TIN, T
                     const T* mp = s.M[p];
                     const T* mq = s.M[q];
                     int l = 0;
-                    for (; l + 3 < r; l += 4) {   // four independent chains per sum
+#pragma unroll 4
+                    for (; l + 3 < r; l += 4) {   // four independent chains per sum, 16-byte loads
+                        T xv[4], yv[4];
+                        ld4(mp + l, xv);
+                        ld4(mq + l, yv);
 #pragma unroll
                         for (int u = 0; u < 4; ++u) {
-                            const T x = mp[l + u], y = mq[l + u];
-                            al[u] = fma(x, x, al[u]);
-                            be[u] = fma(y, y, be[u]);
-                            ga[u] = fma(x, y, ga[u]);
+                            al[u] = fma(xv[u], xv[u], al[u]);
+                            be[u] = fma(yv[u], yv[u], be[u]);
+                            ga[u] = fma(xv[u], yv[u], ga[u]);
                         }
                     }
                     for (; l < r; ++l) {
@@ -375,19 +397,18 @@ __global__ void __launch_bounds__(32 * svd_warps<T>()) svd_kernel(SvdArgs<TIN, T
                         T* Up = s.Ut[p];
                         T* Uq = s.Ut[q];
                         int k = 0;
-                        for (; k + 3 < r; k += 4) {   // loads of four columns issued together
-                            T x[4], y[4], u[4], v[4];
+#pragma unroll 2
+                        for (; k + 3 < r; k += 4) {   // 16-byte loads and stores of four columns
+                            T x[4], y[4], u[4], v[4], x2[4], y2[4], u2[4], v2[4];
+                            ld4(Mp + k, x); ld4(Mq + k, y); ld4(Up + k, u); ld4(Uq + k, v);
 #pragma unroll
                             for (int e = 0; e < 4; ++e) {
-                                x[e] = Mp[k + e]; y[e] = Mq[k + e]; u[e] = Up[k + e]; v[e] = Uq[k + e];
+                                x2[e] = c * x[e] - sn * y[e];
+                                y2[e] = sn * x[e] + c * y[e];
+                                u2[e] = c * u[e] - sn * v[e];
+                                v2[e] = sn * u[e] + c * v[e];
                             }
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                Mp[k + e] = c * x[e] - sn * y[e];
-                                Mq[k + e] = sn * x[e] + c * y[e];
-                                Up[k + e] = c * u[e] - sn * v[e];
-                                Uq[k + e] = sn * u[e] + c * v[e];
-                            }
+                            st4(Mp + k, x2); st4(Mq + k, y2); st4(Up + k, u2); st4(Uq + k, v2);
                         }
                         for (; k < r; ++k) {
                             const T x = Mp[k], y = Mq[k], u = Up[k], v = Uq[k];
