@@ -304,11 +304,14 @@ struct ExportArgs {
 };
 
 constexpr int kExpThreads = 256;   // 8 warps
-constexpr int kExpRows = 64;       // B rows (or A columns) per pipeline stage
+constexpr int kExpRows = 64;       // B part: rows per pipeline stage
 constexpr int kExpStages = 3;
-constexpr int kExpLdB = 68;        // row stride (floats) of a B stage: 16-byte rows, 4-bank shift per row
-constexpr int kExpStageFloats = kExpRows * kExpLdB;
+constexpr int kExpStageFloats = kExpRows * kMaxRank;   // 16 KB per stage
+constexpr int kExpACols = 256;     // A part: columns per block (one per thread)
+constexpr int kExpALRows = 16;     // A part: rows of A per stage (4 stages per column block)
+constexpr int kExpAJ = 16;         // A part: retained directions per pass
 constexpr size_t kExportSmem = (size_t)(kMaxRank * kMaxRank + kExpStages * kExpStageFloats) * sizeof(float);
+static_assert(kExpACols * kExpALRows == kExpStageFloats, "A stage = B stage size");
 
 __device__ __forceinline__ void exp_cp16(float* dst, const float* src, uint32_t n) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(n) : "memory");
@@ -317,95 +320,88 @@ __device__ __forceinline__ void exp_cp4(float* dst, const float* src, uint32_t n
     asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(n) : "memory");
 }
 
-// Stage t of a work item: B part = rows e0 .. e0+63 of B (row-major, stride kExpLdB);
-// A part = columns d0 .. d0+63 of all r rows of A (stage[l * 64 + c]).  Entries past
-// the item, past r or past the matrix are zero-filled.
-__device__ __forceinline__ void export_issue(float* st, const float* X, const lf_module& md, int part, int i0,
-                                             int nrem, bool vec) {
-    const int r = md.r, tid = threadIdx.x;
-    if (part == 0) {
-        if (vec) {
-            for (int q = tid; q < kExpRows * 16; q += kExpThreads) {
-                const int row = q >> 4, c4 = q & 15;
-                const bool ok = row < nrem && 4 * c4 < r;
-                exp_cp16(st + row * kExpLdB + 4 * c4, ok ? X + (int64_t)(i0 + row) * r + 4 * c4 : X, ok ? 16u : 0u);
-            }
-        } else {
-            for (int q = tid; q < kExpRows * kMaxRank; q += kExpThreads) {
-                const int row = q >> 6, c = q & 63;
-                const bool ok = row < nrem && c < r;
-                exp_cp4(st + row * kExpLdB + c, ok ? X + (int64_t)(i0 + row) * r + c : X, ok ? 4u : 0u);
-            }
+// B stage: rows e0 .. e0+63 of B, 64 floats per row, 16-byte chunk c of row e stored at
+// chunk position c ^ (e & 7) (whole 128-byte lines for the copies, distinct banks for
+// the per-row reads).  Entries past the item or past r are zero-filled.
+__device__ __forceinline__ void export_issue_b(float* st, const float* X, int r, int i0, int nrem, bool vec) {
+    const int tid = threadIdx.x;
+    if (vec) {
+        for (int q = tid; q < kExpRows * 16; q += kExpThreads) {
+            const int row = q >> 4, c4 = q & 15;
+            const bool ok = row < nrem && 4 * c4 < r;
+            exp_cp16(st + row * kMaxRank + 4 * (c4 ^ (row & 7)), ok ? X + (int64_t)(i0 + row) * r + 4 * c4 : X,
+                     ok ? 16u : 0u);
         }
     } else {
-        if (vec) {
-            for (int q = tid; q < kMaxRank * 16; q += kExpThreads) {
-                const int l = q >> 4, c4 = q & 15;
-                const int nv = l < r ? min(4, max(0, nrem - 4 * c4)) : 0;
-                exp_cp16(st + l * kExpRows + 4 * c4, nv > 0 ? X + (int64_t)l * md.d_in + i0 + 4 * c4 : X,
-                         4u * (uint32_t)nv);
-            }
-        } else {
-            for (int q = tid; q < kMaxRank * kExpRows; q += kExpThreads) {
-                const int l = q >> 6, c = q & 63;
-                const bool ok = l < r && c < nrem;
-                exp_cp4(st + l * kExpRows + c, ok ? X + (int64_t)l * md.d_in + i0 + c : X, ok ? 4u : 0u);
-            }
+        for (int q = tid; q < kExpRows * kMaxRank; q += kExpThreads) {
+            const int row = q >> 6, c = q & 63;
+            const bool ok = row < nrem && c < r;
+            exp_cp4(st + row * kMaxRank + 4 * ((c >> 2) ^ (row & 7)) + (c & 3),
+                    ok ? X + (int64_t)(i0 + row) * r + c : X, ok ? 4u : 0u);
         }
     }
 }
 
-// One stage: thread (item row / column `e` = tid % 64, output group g = tid / 64)
-// forms outputs j = jbase + g + 4q (q < NQ, j < k) as dot products of its 64 stage
-// values with coefficient rows j (shared memory, broadcast within the warp).
+// A stage: rows l0 .. l0+15 of A, columns c0 .. c0+255 (row-major, 1 KB per row).
+// Rows past r and columns past the item are zero-filled.
+__device__ __forceinline__ void export_issue_a(float* st, const float* X, int r, int64_t d_in, int l0, int c0,
+                                               int ncols, bool vec) {
+    const int tid = threadIdx.x;
+    if (vec) {
+        for (int q = tid; q < kExpALRows * (kExpACols / 4); q += kExpThreads) {
+            const int l = q >> 6, c4 = q & 63;
+            const int nv = (l0 + l < r) ? min(4, max(0, ncols - 4 * c4)) : 0;
+            exp_cp16(st + l * kExpACols + 4 * c4, nv > 0 ? X + (int64_t)(l0 + l) * d_in + c0 + 4 * c4 : X,
+                     4u * (uint32_t)nv);
+        }
+    } else {
+        for (int q = tid; q < kExpALRows * kExpACols; q += kExpThreads) {
+            const int l = q >> 8, c = q & 255;
+            const bool ok = l0 + l < r && c < ncols;
+            exp_cp4(st + l * kExpACols + c, ok ? X + (int64_t)(l0 + l) * d_in + c0 + c : X, ok ? 4u : 0u);
+        }
+    }
+}
+
+// One B stage: thread (row e = tid % 64, output group g = tid / 64) forms outputs
+// j = g, g + 4, ... (< k) as dot products of its row with coefficient rows j (shared
+// memory, broadcast within the warp):  B'^T[j][e] = sum_l C_Bt[j][l] B[e][l].
 template <int NQ>
-__device__ __forceinline__ void export_stage(const ExportArgs& a, const lf_module& md, int part, int k,
-                                             const float* coef, const float* st, int i0, int nrem, int64_t obase,
-                                             int jbase) {
+__device__ __forceinline__ void export_stage_b(const ExportArgs& a, const lf_module& md, int k, const float* coef,
+                                               const float* st, int i0, int nrem, int64_t obase, int jbase) {
     const int tid = threadIdx.x, e = tid & (kExpRows - 1), g = tid >> 6;
     float acc[NQ];
 #pragma unroll
     for (int q = 0; q < NQ; ++q) acc[q] = 0.f;
+    const float* row = st + e * kMaxRank;
 #pragma unroll 4
-    for (int l = 0; l < kMaxRank; l += 4) {
-        float4 x;
-        if (part == 0) {
-            x = *reinterpret_cast<const float4*>(st + e * kExpLdB + l);
-        } else {
-            x.x = st[l * kExpRows + e];
-            x.y = st[(l + 1) * kExpRows + e];
-            x.z = st[(l + 2) * kExpRows + e];
-            x.w = st[(l + 3) * kExpRows + e];
-        }
+    for (int c = 0; c < 16; ++c) {
+        const float4 x = *reinterpret_cast<const float4*>(row + 4 * (c ^ (e & 7)));
 #pragma unroll
         for (int q = 0; q < NQ; ++q) {
-            const float4 c = *reinterpret_cast<const float4*>(coef + (jbase + g + 4 * q) * kMaxRank + l);
-            acc[q] = fmaf(c.x, x.x, fmaf(c.y, x.y, fmaf(c.z, x.z, fmaf(c.w, x.w, acc[q]))));
+            const float4 cf = *reinterpret_cast<const float4*>(coef + (jbase + g + 4 * q) * kMaxRank + 4 * c);
+            acc[q] = fmaf(cf.x, x.x, fmaf(cf.y, x.y, fmaf(cf.z, x.z, fmaf(cf.w, x.w, acc[q]))));
         }
     }
     if (e >= nrem) return;
-    const int64_t ld = part == 0 ? md.d_out : md.d_in;
-    float* pool = part == 0 ? a.Bt_pool : a.A_pool;
-    __nv_bfloat16* pool16 = part == 0 ? a.Bt_pool16 : a.A_pool16;
 #pragma unroll
     for (int q = 0; q < NQ; ++q) {
         const int j = jbase + g + 4 * q;
         if (j < k) {
-            const int64_t o = obase + (int64_t)j * ld + i0 + e;
-            pool[o] = acc[q];
-            if (pool16) pool16[o] = __float2bfloat16_rn(acc[q]);
+            const int64_t o = obase + (int64_t)j * md.d_out + i0 + e;
+            a.Bt_pool[o] = acc[q];
+            if (a.Bt_pool16) a.Bt_pool16[o] = __float2bfloat16_rn(acc[q]);
         }
     }
 }
 
 template <int NQ>
-__device__ void export_item(const ExportArgs& a, const lf_module& md, int part, int k, const float* coef,
-                            float* stages, const float* X, int start, int len, int64_t obase, bool vec) {
+__device__ void export_item_b(const ExportArgs& a, const lf_module& md, int k, const float* coef, float* stages,
+                              const float* X, int start, int len, int64_t obase, bool vec) {
     const int nst = (len + kExpRows - 1) / kExpRows;
 #pragma unroll
     for (int s = 0; s < kExpStages - 1; ++s) {
-        if (s < nst)
-            export_issue(stages + s * kExpStageFloats, X, md, part, start + s * kExpRows, len - s * kExpRows, vec);
+        if (s < nst) export_issue_b(stages + s * kExpStageFloats, X, md.r, start + s * kExpRows, len - s * kExpRows, vec);
         tc::cp_async_commit();
     }
     for (int t = 0; t < nst; ++t) {
@@ -413,25 +409,92 @@ __device__ void export_item(const ExportArgs& a, const lf_module& md, int part, 
         __syncthreads();   // stage t landed for every thread; stage t - 1 fully consumed
         const int tn = t + kExpStages - 1;
         if (tn < nst)
-            export_issue(stages + (tn % kExpStages) * kExpStageFloats, X, md, part, start + tn * kExpRows,
-                         len - tn * kExpRows, vec);
+            export_issue_b(stages + (tn % kExpStages) * kExpStageFloats, X, md.r, start + tn * kExpRows,
+                           len - tn * kExpRows, vec);
         tc::cp_async_commit();
         const float* st = stages + (t % kExpStages) * kExpStageFloats;
-        export_stage<NQ>(a, md, part, k, coef, st, start + t * kExpRows, len - t * kExpRows, obase, 0);
+        export_stage_b<NQ>(a, md, k, coef, st, start + t * kExpRows, len - t * kExpRows, obase, 0);
         if (NQ == 8)   // k > 16: a second pass for j = 32 .. 63
-            export_stage<NQ>(a, md, part, k, coef, st, start + t * kExpRows, len - t * kExpRows, obase, 32);
+            export_stage_b<NQ>(a, md, k, coef, st, start + t * kExpRows, len - t * kExpRows, obase, 32);
+    }
+    tc::cp_async_wait<0>();
+}
+
+// A part: the item's columns go in blocks of 256 (one column per thread); each block is
+// four stages of 16 rows of A, accumulated in registers for kExpAJ retained directions
+// at a time (further passes re-stream the block when k > kExpAJ):
+//   A'[j][d] = sum_l C_A[j][l] A[l][d].
+__device__ void export_item_a(const ExportArgs& a, const lf_module& md, int k, const float* coef, float* stages,
+                              const float* X, int start, int len, int64_t obase, bool vec) {
+    const int tid = threadIdx.x;
+    const int nblk = (len + kExpACols - 1) / kExpACols;
+    const int npass = (k + kExpAJ - 1) / kExpAJ;
+    const int nst = npass * nblk * 4;
+    auto issue = [&](int t) {
+        const int lq = t & 3, blk = (t >> 2) % nblk;
+        const int c0 = start + blk * kExpACols;
+        export_issue_a(stages + (t % kExpStages) * kExpStageFloats, X, md.r, md.d_in, kExpALRows * lq, c0,
+                       min(kExpACols, start + len - c0), vec);
+    };
+#pragma unroll
+    for (int s = 0; s < kExpStages - 1; ++s) {
+        if (s < nst) issue(s);
+        tc::cp_async_commit();
+    }
+    float acc[kExpAJ];
+    for (int t = 0; t < nst; ++t) {
+        tc::cp_async_wait<kExpStages - 2>();
+        __syncthreads();
+        const int tn = t + kExpStages - 1;
+        if (tn < nst) issue(tn);
+        tc::cp_async_commit();
+        const int lq = t & 3, blk = (t >> 2) % nblk, pass = t / (4 * nblk);
+        const int j0 = pass * kExpAJ;
+        if (lq == 0) {
+#pragma unroll
+            for (int jj = 0; jj < kExpAJ; ++jj) acc[jj] = 0.f;
+        }
+        const float* st = stages + (t % kExpStages) * kExpStageFloats;
+        float x[kExpALRows];
+#pragma unroll
+        for (int l = 0; l < kExpALRows; ++l) x[l] = st[l * kExpACols + tid];
+        const int nj = min(kExpAJ, k - j0);
+#pragma unroll
+        for (int jj = 0; jj < kExpAJ; ++jj) {
+            if (jj < nj) {
+                const float* cr = coef + (j0 + jj) * kMaxRank + kExpALRows * lq;
+                float t4 = acc[jj];
+#pragma unroll
+                for (int l4 = 0; l4 < kExpALRows / 4; ++l4) {
+                    const float4 cf = *reinterpret_cast<const float4*>(cr + 4 * l4);
+                    t4 = fmaf(cf.x, x[4 * l4], fmaf(cf.y, x[4 * l4 + 1], fmaf(cf.z, x[4 * l4 + 2], fmaf(cf.w, x[4 * l4 + 3], t4))));
+                }
+                acc[jj] = t4;
+            }
+        }
+        if (lq == 3) {
+            const int d = start + blk * kExpACols + tid;
+            if (d < start + len) {
+#pragma unroll
+                for (int jj = 0; jj < kExpAJ; ++jj) {
+                    if (jj < nj) {
+                        const int64_t o = obase + (int64_t)(j0 + jj) * md.d_in + d;
+                        a.A_pool[o] = acc[jj];
+                        if (a.A_pool16) a.A_pool16[o] = __float2bfloat16_rn(acc[jj]);
+                    }
+                }
+            }
+        }
     }
     tc::cp_async_wait<0>();
 }
 
 // One CTA per work item (a run of up to 2048 rows of B or columns of A of one
-// module): the item streams through a 3-stage cp.async ring of 64-row stages and
-// every output element is one 64-term dot product with a row of the coefficients
-//   B part: B'^T[j][e] = sum_l C_Bt[j][l] B[e][l]
-//   A part: A'[j][d]   = sum_l C_A[j][l]  A[l][d].
+// module), streamed through a kExpStages cp.async ring of 16 KB stages; every output
+// element is one 64-term dot product with a row of the coefficients.
 __global__ void __launch_bounds__(kExpThreads, 3) export_kernel(ExportArgs a) {
     extern __shared__ __align__(16) float exp_smem[];
-    float* coef = exp_smem;                             // k x 64, row stride 64, zero past r
+    float* coef = exp_smem;                             // k x 64, row stride 64, zero past r and past k
     float* stages = exp_smem + kMaxRank * kMaxRank;
     const ExportWork w = a.work[blockIdx.x];
     const lf_module md = a.mods[w.mod];
@@ -445,23 +508,27 @@ __global__ void __launch_bounds__(kExpThreads, 3) export_kernel(ExportArgs a) {
         if (oa + (int64_t)k * md.d_in > a.cap_A) return;
     }
     const float* C = (w.part == 0 ? a.C_Bt : a.C_A) + (size_t)w.mod * a.rs * a.rs;
-    const int kfill = k <= 4 ? 4 : (k <= 8 ? 8 : (k <= 16 ? 16 : kMaxRank));   // rows export_stage reads
+    const int kfill = w.part == 1 ? min(kMaxRank, ((k + kExpAJ - 1) / kExpAJ) * kExpAJ)
+                                  : (k <= 4 ? 4 : (k <= 8 ? 8 : (k <= 16 ? 16 : kMaxRank)));   // rows the stages read
     for (int e = threadIdx.x; e < kfill * kMaxRank; e += kExpThreads) {
         const int j = e / kMaxRank, l = e % kMaxRank;
         coef[e] = (j < k && l < r) ? C[j * a.rs + l] : 0.f;
     }
     const float* X = w.part == 0 ? a.B_base + md.B_off : a.A_base + md.A_off;
-    const bool vec = w.part == 0 ? (r % 4 == 0) : (md.d_in % 4 == 0);
-    const int64_t obase = w.part == 0 ? obt : oa;
-    // coefficient rows are read after the first barrier inside export_item
+    // coefficient rows are read after the first barrier inside export_item_*
+    if (w.part == 1) {
+        export_item_a(a, md, k, coef, stages, X, w.start, w.len, oa, md.d_in % 4 == 0);
+        return;
+    }
+    const bool vec = r % 4 == 0;
     if (k <= 4)
-        export_item<1>(a, md, w.part, k, coef, stages, X, w.start, w.len, obase, vec);
+        export_item_b<1>(a, md, k, coef, stages, X, w.start, w.len, obt, vec);
     else if (k <= 8)
-        export_item<2>(a, md, w.part, k, coef, stages, X, w.start, w.len, obase, vec);
+        export_item_b<2>(a, md, k, coef, stages, X, w.start, w.len, obt, vec);
     else if (k <= 16)
-        export_item<4>(a, md, w.part, k, coef, stages, X, w.start, w.len, obase, vec);
+        export_item_b<4>(a, md, k, coef, stages, X, w.start, w.len, obt, vec);
     else
-        export_item<8>(a, md, w.part, k, coef, stages, X, w.start, w.len, obase, vec);
+        export_item_b<8>(a, md, k, coef, stages, X, w.start, w.len, obt, vec);
 }
 
 }  // namespace lf
