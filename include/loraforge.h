@@ -160,13 +160,16 @@ lf_status lf_truncate_export(const lf_module* mods /*[host]*/, int32_t n, lf_pol
  * hold pool_elems_A / pool_elems_Bt elements; an adapter whose rows would reach
  * past a pool (or whose offset is not a multiple of 8, or k > 64) latches an error
  * on the device and its tokens are left untouched.
- * Tokens are routed by a stable sort on the adapter id into segments (adapter,
- * start, length) over a permutation of token indices.  If seg_out is not NULL it
- * receives, as int32: [n_seg, n_valid, then 3*n_seg (adapter,start,len),
- * then n_valid token indices]; it must hold 2 + 3*min(T,n_adapters) + T ints.
- * Segments with many tokens run on tcgen05 tensor cores, the rest on a segmented
- * GEMV; both read every adapter's k rows once per segment and never pad k.
- * Workspace: lf_apply_workspace_size(T, n_adapters). */
+ * With few tokens per adapter (T <= 8 * n_adapters) every token is applied with
+ * its own adapter index (no sort).  Otherwise tokens are routed by a stable sort
+ * on the adapter id into segments (adapter, start, length) over a permutation of
+ * token indices; segments with many tokens run on tcgen05 tensor cores, the rest
+ * on a segmented GEMV; both read every adapter's k rows once per segment and never
+ * pad k.  If seg_out is not NULL it receives the routing, as int32: [n_seg,
+ * n_valid, then 3*n_seg (adapter,start,len), then n_valid token indices]; it must
+ * hold 2 + 3*min(T,n_adapters) + T ints.
+ * Workspace: lf_apply_workspace_size(T, n_adapters).  The same as a one-slice
+ * lf_lora_shrink_expand_slices call with y_ld = d_out. */
 size_t lf_apply_workspace_size(int32_t T, int32_t n_adapters);
 lf_status lf_lora_shrink_expand(int32_t T, int32_t d_in, int32_t d_out,
                                 const void* x, void* y, const int32_t* ids,
@@ -176,6 +179,41 @@ lf_status lf_lora_shrink_expand(int32_t T, int32_t d_in, int32_t d_out,
                                 int64_t pool_elems_A, int64_t pool_elems_Bt, float scale,
                                 int32_t* seg_out, void* ws, size_t ws_bytes,
                                 lf_stream_t stream);
+
+/* ---- Multi-LoRA shrink / expand over output slices sharing x ------------------
+ * LoRAForge's serving side runs the projections that read the same input (q/k/v,
+ * gate/up) together: one call applies up to 4 output slices, each a projection
+ * with its own factor pools, ranks and place in y.  For every token t with
+ * a = ids[t] >= 0 and every slice s:
+ *   t_s    = A'_{s,a} x_t                                    (k_{s,a} fp32 values)
+ *   y_t[y_offset_s .. y_offset_s + d_out_s) =
+ *            bf16( y_t[...] + scale_a * B'_{s,a} t_s )       (one rounding)
+ * with scale_a = adapter_scale[a] when adapter_scale (device, n_adapters floats)
+ * is not NULL, else `scale`.  y has T rows of y_ld elements; slices must not
+ * overlap in y (overlapping slices race).  The routing is computed once for all
+ * slices, and on the tensor-core path x is read once: the shrink contracts x with
+ * the slices' A' rows concatenated (N = sum of ranks).  Argument rules as for
+ * lf_lora_shrink_expand, plus: 1 <= n_slices <= 4, d_out_s, y_offset_s and y_ld
+ * multiples of 8, y_offset_s + d_out_s <= y_ld; errors per (adapter, slice) leave
+ * that slice of the adapter's tokens untouched.
+ * Workspace: lf_apply_slices_workspace_size(T, n_adapters, n_slices). */
+typedef struct {
+    int32_t d_out;              /* output columns of the slice */
+    int32_t reserved;           /* 0 */
+    int64_t y_offset;           /* first column of the slice in each row of y */
+    const int32_t* ranks;       /* per adapter: retained rank of this slice's module */
+    const int64_t* off_A;       /* per adapter: element offset of A' (k x d_in) in A_pool */
+    const int64_t* off_Bt;      /* per adapter: element offset of B'^T (k x d_out) in Bt_pool */
+    const void* A_pool;         /* bf16 */
+    const void* Bt_pool;        /* bf16 */
+    int64_t pool_elems_A, pool_elems_Bt;
+} lf_slice;
+size_t lf_apply_slices_workspace_size(int32_t T, int32_t n_adapters, int32_t n_slices);
+lf_status lf_lora_shrink_expand_slices(int32_t T, int32_t d_in, const void* x, void* y, int64_t y_ld,
+                                       const int32_t* ids, int32_t n_adapters,
+                                       const lf_slice* slices /*[host]*/, int32_t n_slices,
+                                       float scale, const float* adapter_scale, int32_t* seg_out,
+                                       void* ws, size_t ws_bytes, lf_stream_t stream);
 
 /* ---- Shrink / expand with library-owned scratch -------------------------------
  * This entry point has no counterpart in the paper; it exists for callers that

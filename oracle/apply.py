@@ -92,3 +92,32 @@ def lora_apply_dense(x, y0, ids, ranks, off_A, off_Bt, A_pool, Bt_pool, scale: f
         Ap, Bt = adapter_factors(a, ranks, off_A, off_Bt, A_pool, Bt_pool, d_in, d_out)
         y[t] = y[t] + scale * ((Bt.T @ Ap) @ x[t])
     return y
+
+
+def lora_apply_slices(x, y0, ids, slices, scale: float, adapter_scale=None):
+    """Side path of several output slices that share x ("Compress then Serve" §13.4:
+    the LoRA buffer comes from x per token and is added to each projection's output).
+
+    slices: list of (d_out, y_offset, ranks, off_A, off_Bt, A_pool, Bt_pool); y0 is
+    T x y_ld and slice s occupies columns y_offset .. y_offset + d_out.  For every
+    token t with adapter a = ids[t] >= 0 and every slice:
+        y[t, slice] += scale_a * B'_{s,a} (A'_{s,a} x_t),
+    scale_a = adapter_scale[a] when given, else scale.  Columns outside the slices
+    keep y0.  Returns y in float64.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    y = np.array(y0, dtype=np.float64, copy=True)
+    ids = np.asarray(ids)
+    n_adapters = len(slices[0][2])
+    if np.any(ids < -1) or np.any(ids >= n_adapters):
+        raise ValueError("adapter id out of range")
+    d_in = x.shape[1]
+    for t in range(x.shape[0]):
+        a = int(ids[t])
+        if a < 0:
+            continue
+        sa = float(adapter_scale[a]) if adapter_scale is not None else scale
+        for d_out, y_off, ranks, off_A, off_Bt, A_pool, Bt_pool in slices:
+            Ap, Bt = adapter_factors(a, ranks, off_A, off_Bt, A_pool, Bt_pool, d_in, d_out)
+            y[t, y_off:y_off + d_out] += sa * (Bt.T @ (Ap @ x[t]))
+    return y

@@ -104,5 +104,17 @@ def shrink_expand(x, y, ids, ranks, off_A, off_Bt, A_pool, Bt_pool, scale, ws=No
     return y
 
 
+def shrink_expand_slices(x, y, ids, slices, scale, adapter_scale=None, ws=None, seg_out=None, stream=None):
+    """Side path of several output slices sharing x.  slices: list of tuples
+    (d_out, y_offset, ranks, off_A, off_Bt, A_pool, Bt_pool) with device tensors
+    (ranks int32 and offsets int64 per adapter, bf16 pools); y is T x y_ld."""
+    n_adapters = slices[0][2].numel()
+    ns = len(slices)
+    ws = ws if ws is not None else workspace(lf.lf_apply_slices_workspace_size(x.shape[0], n_adapters, ns), x.device)
+    sl = [lf.make_slice(*t) for t in slices]
+    lf.lf_lora_shrink_expand_slices(x, y, ids, n_adapters, sl, scale, ws, adapter_scale, seg_out, stream)
+    return y
+
+
 def device_status(stream=None) -> int:
     return lf.lf_get_device_status(stream)

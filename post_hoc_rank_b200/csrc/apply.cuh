@@ -16,33 +16,15 @@ namespace lf {
 
 constexpr int kRouteThreads = 1024;
 constexpr int kRouteChunk = 4096;  // tokens staged per pass of the run detection
-constexpr int kGemvTok = 8;        // tokens per GEMV work item
 constexpr int kGemvThreads = 256;
 constexpr int kGemvCols = kGemvThreads * 8;   // d_out columns per CTA
 
-struct Seg {
-    int32_t adapter, start, len;
-};
-// Self-contained work item (64 bytes): everything a shrink/expand CTA needs, so it
-// starts its data loads after one dependent read.
-struct GemvItem {
-    int32_t adapter, k, ntok, tok0;   // tok0: position of the first token in the permutation
-    int64_t oa, ob;                   // element offsets of A' and B'^T in the pools
-    int32_t tok[kGemvTok];            // token indices
-};
-
 struct RouteOut {
-    int32_t* counts;     // [0] n_seg, [1] n_valid, [2] n_items
+    int32_t* counts;     // [0] n_seg, [1] n_valid, [2] n_items, [3] n_tc_items
     Seg* segs;           // min(T, n_adapters)
     int32_t* perm;       // T
     GemvItem* items;     // T / kGemvTok + min(T, n_adapters)
     int32_t* seg_out;    // optional caller copy
-    // per-adapter rank table of this projection, used to fill and validate items
-    const int32_t* ranks;
-    const int64_t* off_A;
-    const int64_t* off_Bt;
-    int64_t pool_A, pool_Bt;
-    int32_t d_in, d_out;
     TcItem* tc_items;    // T / kTcM + min(T, n_adapters) + 1
     int32_t tc_enable;   // segments with >= kTcMin tokens become tensor-core items
     // Run scratch (nullable, T ints each): with it the sort works on runs of equal
@@ -81,7 +63,9 @@ __device__ __forceinline__ int block_excl_scan(int v, int* wsum, int* total) {
 }
 
 // One CTA: stable counting sort of token ids into segments (adapter, start, len),
-// the token permutation, and GEMV work items of <= kGemvTok tokens.
+// the token permutation, GEMV work items of <= kGemvTok tokens and tensor-core items
+// of <= 128 tokens.  Depends on the ids only (no factor tables), so one routing
+// serves every slice and projection of a batch.
 // Shared memory: 2 * n_adapters ints.
 __global__ void __launch_bounds__(kRouteThreads) route_kernel(const int32_t* __restrict__ ids, int T,
                                                               int n_adapters, RouteOut o) {
@@ -162,36 +146,19 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const int32_t* __r
             segidx[a] = sidx;
             if (c > 0) {
                 o.segs[sidx] = Seg{a, start, c};
-                int k = o.ranks[a];
-                const int64_t oa = o.off_A[a], ob = o.off_Bt[a];
-                int err = 0;
-                if (k > kMaxRank) err = LF_ERR_SHAPE;
-                else if (k > 0 && ((oa & 7) || (ob & 7))) err = LF_ERR_ALIGNMENT;
-                else if (k > 0 && (oa < 0 || ob < 0 || oa + (int64_t)k * o.d_in > o.pool_A ||
-                                   ob + (int64_t)k * o.d_out > o.pool_Bt))
-                    err = LF_ERR_WORKSPACE;
-                if (err) {
-                    latch_error(err);
-                    k = 0;   // the adapter's tokens are left untouched
-                }
                 for (int q = 0; q < nti; ++q) {
                     TcItem ti2;
                     ti2.adapter = a;
-                    ti2.k = k < 0 ? 0 : k;
                     ti2.ntok = min(kTcM, c - q * kTcM);
                     ti2.tok0 = start + q * kTcM;
-                    ti2.oa = oa;
-                    ti2.ob = ob;
+                    ti2.pad0 = 0;
                     o.tc_items[qidx + q] = ti2;
                 }
                 for (int q = 0; q < ni; ++q) {
-                    GemvItem it;
+                    GemvItem it{};
                     it.adapter = a;
-                    it.k = k < 0 ? 0 : k;
                     it.ntok = min(kGemvTok, c - q * kGemvTok);
                     it.tok0 = start + q * kGemvTok;
-                    it.oa = oa;
-                    it.ob = ob;
                     o.items[iidx + q] = it;
                 }
             }
@@ -310,57 +277,44 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const int32_t* __r
     }
 }
 
-struct GemvArgs {
-    int32_t d_in, d_out;
-    const __nv_bfloat16* x;
-    __nv_bfloat16* y;
-    const int32_t* ranks;
-    const int64_t* off_A;
-    const int64_t* off_Bt;
-    const __nv_bfloat16* A_pool;
-    const __nv_bfloat16* Bt_pool;
-    int64_t pool_A, pool_Bt;
-    float scale;
-    const int32_t* counts;
-    const Seg* segs;
-    const int32_t* perm;
-    const GemvItem* items;
-    float* t_buf;          // T x kMaxRank fp32 intermediate, row = position in the permutation
-};
-
-__device__ __forceinline__ void bf16x8_to_f32(const uint4& u, float* f) {
-    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const float2 v = __bfloat1622float2(h[i]);
-        f[2 * i] = v.x;
-        f[2 * i + 1] = v.y;
-    }
+__device__ __forceinline__ bool item_ok(const ApplyArgs& a, int it, GemvItem& item) {
+    if (it >= a.counts[2]) return false;
+    item = a.items[it];
+    return true;
 }
 
-__device__ __forceinline__ bool item_ok(const GemvArgs& a, int it, GemvItem& item) {
-    const int n_items = a.counts[2];
-    if (it >= n_items) return false;
-    item = a.items[it];
-    return item.k > 0;
+// y[tok][e .. e+7] = bf16(y + scale * acc) for one 16-byte vector of y.
+__device__ __forceinline__ void y_update8(__nv_bfloat16* yp, const float (&acc)[8], float scale) {
+    uint4 u = *reinterpret_cast<const uint4*>(yp);
+    float yf[8];
+    bf16x8_to_f32(u, yf);
+    __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&u);
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
+        h[c] = __floats2bfloat162_rn(fmaf(scale, acc[2 * c], yf[2 * c]), fmaf(scale, acc[2 * c + 1], yf[2 * c + 1]));
+    *reinterpret_cast<uint4*>(yp) = u;
 }
 
 constexpr int kShrinkJ = 4;   // rows of A' per pass
 
-// Shrink: t[item][q][j] = A'_a[j] . x[tok_q] (fp32), one CTA per work item.  The
+// Shrink: t[item][q][j] = A'_a[j] . x[tok_q] (fp32); grid (work items, slices).  The
 // d_in range is split across all warps so each warp keeps many 16-byte loads in
 // flight; partial sums are reduced through shared memory in a fixed order.
-__global__ void __launch_bounds__(kGemvThreads) shrink_kernel(GemvArgs a) {
+__global__ void __launch_bounds__(kGemvThreads) shrink_kernel(ApplyArgs a) {
     __shared__ float part[kGemvThreads / 32][kShrinkJ][kGemvTok];
     __shared__ int32_t toks[kGemvTok];
     GemvItem item;
     if (!item_ok(a, blockIdx.x, item)) return;
-    const int nt = item.ntok, k = item.k;
+    const int sl = blockIdx.y;
+    int k;
+    int64_t oa, ob;
+    if (!slice_factors(a, sl, item.adapter, true, k, oa, ob)) return;
+    const int nt = item.ntok;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     if (tid < nt) toks[tid] = a.items[blockIdx.x].tok[tid];
     __syncthreads();
-    const __nv_bfloat16* Ap = a.A_pool + item.oa;
-    float* tout = a.t_buf + (size_t)item.tok0 * kMaxRank;
+    const __nv_bfloat16* Ap = a.sl[sl].A_pool + oa;
+    float* tout = a.t_buf + (size_t)item.tok0 * a.ldt + a.sl[sl].t_col;
     for (int j0 = 0; j0 < k; j0 += kShrinkJ) {
         float acc[kShrinkJ][kGemvTok];
 #pragma unroll
@@ -403,41 +357,45 @@ __global__ void __launch_bounds__(kGemvThreads) shrink_kernel(GemvArgs a) {
             float v = 0.f;
 #pragma unroll
             for (int w = 0; w < kGemvThreads / 32; ++w) v += part[w][jj][q];
-            if (j0 + jj < k && q < nt) tout[q * kMaxRank + j0 + jj] = v;
+            if (j0 + jj < k && q < nt) tout[q * a.ldt + j0 + jj] = v;
         }
         __syncthreads();
     }
 }
 
-// Expand: y[tok_q][e..e+7] = bf16(y + s * sum_j t[q][j] B'^T[j][e..e+7]);
-// grid (items, ceil(d_out / kGemvCols)).
-__global__ void __launch_bounds__(kGemvThreads) expand_kernel(GemvArgs a) {
+// Expand: y[tok_q][e..e+7] = bf16(y + s * sum_j t[q][j] B'^T[j][e..e+7]); grid (work
+// items, column chunks of kGemvCols over all slices).
+__global__ void __launch_bounds__(kGemvThreads) expand_kernel(ApplyArgs a) {
     __shared__ float tsm[kGemvTok][kMaxRank];
     __shared__ int32_t toks[kGemvTok];
     GemvItem item;
     if (!item_ok(a, blockIdx.x, item)) return;
-    const int nt = item.ntok, k = item.k;
-    const int64_t ob = item.ob;
+    const int sl = slice_of_chunk(a, blockIdx.y);
+    const SliceTab& S = a.sl[sl];
+    int k;
+    int64_t oa, ob;
+    if (!slice_factors(a, sl, item.adapter, false, k, oa, ob)) return;   // reported by the shrink
+    const int nt = item.ntok;
     const int tid = threadIdx.x;
     if (tid < nt) toks[tid] = a.items[blockIdx.x].tok[tid];
-    const float* tin = a.t_buf + (size_t)item.tok0 * kMaxRank;
+    const float* tin = a.t_buf + (size_t)item.tok0 * a.ldt + S.t_col;
     for (int e = tid; e < nt * kMaxRank; e += kGemvThreads) {
         const int q = e / kMaxRank, j = e % kMaxRank;
-        tsm[q][j] = j < k ? tin[e] : 0.f;
+        tsm[q][j] = j < k ? tin[q * a.ldt + j] : 0.f;
     }
     __syncthreads();
-    const int e = blockIdx.y * kGemvCols + tid * 8;
-    if (e >= a.d_out) return;
+    const int e = ((int)blockIdx.y - S.chunk0) * kGemvCols + tid * 8;
+    if (e >= S.d_out) return;
     float acc[kGemvTok][8];
 #pragma unroll
     for (int q = 0; q < kGemvTok; ++q)
 #pragma unroll
         for (int c = 0; c < 8; ++c) acc[q][c] = 0.f;
-    const __nv_bfloat16* Bt = a.Bt_pool + ob + e;
+    const __nv_bfloat16* Bt = S.Bt_pool + ob + e;
 #pragma unroll 4
     for (int j = 0; j < k; ++j) {
         float bf[8];
-        bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(Bt + (int64_t)j * a.d_out)), bf);
+        bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(Bt + (int64_t)j * S.d_out)), bf);
 #pragma unroll
         for (int q = 0; q < kGemvTok; ++q) {
             if (q < nt) {
@@ -447,76 +405,44 @@ __global__ void __launch_bounds__(kGemvThreads) expand_kernel(GemvArgs a) {
             }
         }
     }
+    const float scale = adapter_scale(a, item.adapter);
 #pragma unroll
-    for (int q = 0; q < kGemvTok; ++q) {
-        if (q < nt) {
-            __nv_bfloat16* yp = a.y + (int64_t)toks[q] * a.d_out + e;
-            float yf[8];
-            uint4 u = *reinterpret_cast<const uint4*>(yp);
-            bf16x8_to_f32(u, yf);
-            __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&u);
-#pragma unroll
-            for (int c = 0; c < 4; ++c)
-                h[c] = __floats2bfloat162_rn(fmaf(a.scale, acc[q][2 * c], yf[2 * c]),
-                                             fmaf(a.scale, acc[q][2 * c + 1], yf[2 * c + 1]));
-            *reinterpret_cast<uint4*>(yp) = u;
-        }
-    }
+    for (int q = 0; q < kGemvTok; ++q)
+        if (q < nt) y_update8(a.y + (int64_t)toks[q] * a.y_ld + S.y_off + e, acc[q], scale);
 }
 
 
 // Decode regime, token-parallel (BGMV form: every token carries its adapter index,
-// no sorting).  CTA (token, 4096-column slice of d_out): t = A'_a x (k fp32 dot
+// no sorting).  CTA (token, 4096-column chunk of one slice): t = A' x (k fp32 dot
 // products over d_in, reduced across the CTA in a fixed order), then
-// y[slice] += s * B'_a^T t with 16-byte loads of the k rows of B'^T.  Each slice
-// CTA recomputes the same t (identical arithmetic; x and A'_a come from L2), and
-// tokens of one adapter read its factors from L2 after the first touch, so HBM
-// sees every distinct factor row, x and y once.
+// y[chunk] += s * B'^T t with 16-byte loads of the k rows of B'^T.  Each chunk CTA
+// recomputes the same t (identical arithmetic; x and A' come from L2), and tokens
+// of one adapter read its factors from L2 after the first touch, so HBM sees every
+// distinct factor row, x and y once.
 constexpr int kBgmvThreads = 256;
 constexpr int kBgmvVec = 2;                                  // 8-column vectors per thread in the expand
 constexpr int kBgmvCols = kBgmvThreads * 8 * kBgmvVec;       // d_out columns per CTA
 constexpr int kBgmvJ = 8;                                    // retained directions per shrink pass
 
-struct BgmvArgs {
-    int32_t n_adapters, d_in, d_out;
-    const __nv_bfloat16* x;
-    __nv_bfloat16* y;
-    const int32_t* ids;
-    const int32_t* ranks;
-    const int64_t* off_A;
-    const int64_t* off_Bt;
-    const __nv_bfloat16* A_pool;
-    const __nv_bfloat16* Bt_pool;
-    int64_t pool_A, pool_Bt;
-    float scale;
-};
-
-__global__ void __launch_bounds__(kBgmvThreads, 4) bgmv_kernel(BgmvArgs a) {
+__global__ void __launch_bounds__(kBgmvThreads, 4) bgmv_kernel(ApplyArgs a) {
     __shared__ float red[kBgmvThreads / 32][kBgmvJ];
     __shared__ float ts[kMaxRank];
     const int tok = blockIdx.x;
     const int ad = a.ids[tok];
     if (ad == -1) return;
-    const bool lead = blockIdx.y == 0 && threadIdx.x == 0;   // one CTA per token reports errors
+    const int sl = slice_of_chunk(a, blockIdx.y);
+    const SliceTab& S = a.sl[sl];
+    const bool lead = (int)blockIdx.y == S.chunk0 && threadIdx.x == 0;   // one CTA per (token, slice) reports
     if (ad < -1 || ad >= a.n_adapters) {
-        if (lead) latch_error(LF_ERR_BAD_INDEX);
+        if (lead && sl == 0) latch_error(LF_ERR_BAD_INDEX);
         return;
     }
-    const int k = a.ranks[ad];
-    const int64_t oa = a.off_A[ad], ob = a.off_Bt[ad];
-    int err = 0;
-    if (k > kMaxRank) err = LF_ERR_SHAPE;
-    else if (k > 0 && ((oa & 7) || (ob & 7))) err = LF_ERR_ALIGNMENT;
-    else if (k > 0 && (oa < 0 || ob < 0 || oa + (int64_t)k * a.d_in > a.pool_A || ob + (int64_t)k * a.d_out > a.pool_Bt))
-        err = LF_ERR_WORKSPACE;
-    if (err) {
-        if (lead) latch_error(err);
-        return;
-    }
-    if (k <= 0) return;
+    int k;
+    int64_t oa, ob;
+    if (!slice_factors(a, sl, ad, lead, k, oa, ob)) return;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const __nv_bfloat16* xr = a.x + (int64_t)tok * a.d_in;
-    const __nv_bfloat16* Ap = a.A_pool + oa;
+    const __nv_bfloat16* Ap = S.A_pool + oa;
     for (int j0 = 0; j0 < k; j0 += kBgmvJ) {
         const int nj = min(kBgmvJ, k - j0);
         float acc[kBgmvJ];
@@ -556,12 +482,14 @@ __global__ void __launch_bounds__(kBgmvThreads, 4) bgmv_kernel(BgmvArgs a) {
         }
         __syncthreads();
     }
-    const __nv_bfloat16* Bt = a.Bt_pool + ob;
-    __nv_bfloat16* yr = a.y + (int64_t)tok * a.d_out;
+    const __nv_bfloat16* Bt = S.Bt_pool + ob;
+    __nv_bfloat16* yr = a.y + (int64_t)tok * a.y_ld + S.y_off;
+    const float scale = adapter_scale(a, ad);
+    const int cbase = ((int)blockIdx.y - S.chunk0) * kBgmvCols;
 #pragma unroll
     for (int h = 0; h < kBgmvVec; ++h) {
-        const int e = blockIdx.y * kBgmvCols + h * (kBgmvThreads * 8) + tid * 8;
-        if (e >= a.d_out) break;
+        const int e = cbase + h * (kBgmvThreads * 8) + tid * 8;
+        if (e >= S.d_out) break;
         uint4 yv = *reinterpret_cast<const uint4*>(yr + e);   // issued before the k-row loads are consumed
         float acc[8];
 #pragma unroll
@@ -569,7 +497,7 @@ __global__ void __launch_bounds__(kBgmvThreads, 4) bgmv_kernel(BgmvArgs a) {
 #pragma unroll 4
         for (int j = 0; j < k; ++j) {
             float bf[8];
-            bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(Bt + (int64_t)j * a.d_out + e)), bf);
+            bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(Bt + (int64_t)j * S.d_out + e)), bf);
             const float tv = ts[j];
 #pragma unroll
             for (int c = 0; c < 8; ++c) acc[c] = fmaf(tv, bf[c], acc[c]);
@@ -578,29 +506,32 @@ __global__ void __launch_bounds__(kBgmvThreads, 4) bgmv_kernel(BgmvArgs a) {
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
             const float2 yf = __bfloat1622float2(y2[q]);
-            y2[q] = __floats2bfloat162_rn(fmaf(a.scale, acc[2 * q], yf.x), fmaf(a.scale, acc[2 * q + 1], yf.y));
+            y2[q] = __floats2bfloat162_rn(fmaf(scale, acc[2 * q], yf.x), fmaf(scale, acc[2 * q + 1], yf.y));
         }
         *reinterpret_cast<uint4*>(yr + e) = yv;
     }
 }
 
-// Decode regime (few tokens per adapter): one launch does shrink and expand.  CTA
+// Decode regime of the no-allocation entry point (one slice, sorted items): CTA
 // (item, d_out chunk): all warps share the dot products of each A' row over d_in
 // (16-byte loads issued together), t is reduced in a fixed order in shared memory,
-// then the CTA updates its d_out slice of y.  CTAs of one item in different chunks
+// then the CTA updates its d_out chunk of y.  CTAs of one item in different chunks
 // recompute the same t (identical arithmetic, A' and x served from L2).
-__global__ void __launch_bounds__(kGemvThreads) fused_gemv_kernel(GemvArgs a) {
+__global__ void __launch_bounds__(kGemvThreads) fused_gemv_kernel(ApplyArgs a) {
     __shared__ float part[kGemvThreads / 32][kShrinkJ][kGemvTok];
     __shared__ float tsm[kGemvTok][kMaxRank];
     __shared__ int32_t toks[kGemvTok];
     GemvItem item;
     if (!item_ok(a, blockIdx.x, item)) return;
-    const int nt = item.ntok, k = item.k;
-    const int64_t ob = item.ob;
+    const SliceTab& S = a.sl[0];
+    int k;
+    int64_t oa, ob;
+    if (!slice_factors(a, 0, item.adapter, blockIdx.y == 0, k, oa, ob)) return;
+    const int nt = item.ntok;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     if (tid < nt) toks[tid] = a.items[blockIdx.x].tok[tid];
     __syncthreads();
-    const __nv_bfloat16* Ap = a.A_pool + item.oa;
+    const __nv_bfloat16* Ap = S.A_pool + oa;
     for (int j0 = 0; j0 < k; j0 += kShrinkJ) {
         const int nj = min(kShrinkJ, k - j0);
         float acc[kShrinkJ][kGemvTok];
@@ -655,17 +586,17 @@ __global__ void __launch_bounds__(kGemvThreads) fused_gemv_kernel(GemvArgs a) {
         __syncthreads();
     }
     const int e = blockIdx.y * kGemvCols + tid * 8;
-    if (e >= a.d_out) return;
+    if (e >= S.d_out) return;
     float acc[kGemvTok][8];
 #pragma unroll
     for (int q = 0; q < kGemvTok; ++q)
 #pragma unroll
         for (int c = 0; c < 8; ++c) acc[q][c] = 0.f;
-    const __nv_bfloat16* Bt = a.Bt_pool + ob + e;
+    const __nv_bfloat16* Bt = S.Bt_pool + ob + e;
 #pragma unroll 4
     for (int j = 0; j < k; ++j) {
         float bf[8];
-        bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(Bt + (int64_t)j * a.d_out)), bf);
+        bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(Bt + (int64_t)j * S.d_out)), bf);
 #pragma unroll
         for (int q = 0; q < kGemvTok; ++q) {
             if (q < nt) {
@@ -675,21 +606,10 @@ __global__ void __launch_bounds__(kGemvThreads) fused_gemv_kernel(GemvArgs a) {
             }
         }
     }
+    const float scale = adapter_scale(a, item.adapter);
 #pragma unroll
-    for (int q = 0; q < kGemvTok; ++q) {
-        if (q < nt) {
-            __nv_bfloat16* yp = a.y + (int64_t)toks[q] * a.d_out + e;
-            float yf[8];
-            uint4 u = *reinterpret_cast<const uint4*>(yp);
-            bf16x8_to_f32(u, yf);
-            __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&u);
-#pragma unroll
-            for (int c = 0; c < 4; ++c)
-                h[c] = __floats2bfloat162_rn(fmaf(a.scale, acc[q][2 * c], yf[2 * c]),
-                                             fmaf(a.scale, acc[q][2 * c + 1], yf[2 * c + 1]));
-            *reinterpret_cast<uint4*>(yp) = u;
-        }
-    }
+    for (int q = 0; q < kGemvTok; ++q)
+        if (q < nt) y_update8(a.y + (int64_t)toks[q] * a.y_ld + S.y_off + e, acc[q], scale);
 }
 
 }  // namespace lf

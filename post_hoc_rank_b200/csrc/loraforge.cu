@@ -334,6 +334,153 @@ __global__ void cap_flags_kernel(int32_t* count, int cap) {
     }
 }
 
+// ------------------------------------------------------------ apply workspace
+struct ApplyWs {
+    int32_t* counts;
+    Seg* segs;
+    int32_t* perm;
+    GemvItem* items;
+    float* t_buf;
+    TcItem* tc_items;
+    float* t_part;
+    int32_t* runs;
+};
+
+// Carves (or, with base == nullptr, sizes) the side-path workspace for T tokens,
+// n adapters and ns slices.
+static size_t carve_apply(void* base, int64_t T, int64_t n, int ns, ApplyWs* w) {
+    Carver c(base);
+    const int64_t mseg = std::min<int64_t>(T, n);
+    const int64_t T1 = std::max<int64_t>(T, 1);
+    w->counts = c.take<int32_t>(4);
+    w->segs = c.take<Seg>((size_t)std::max<int64_t>(mseg, 1));
+    w->perm = c.take<int32_t>((size_t)T1);
+    w->items = c.take<GemvItem>((size_t)(T / kGemvTok + mseg + 1));
+    w->t_buf = c.take<float>((size_t)T1 * kMaxRank * ns);
+    w->tc_items = c.take<TcItem>((size_t)(T / kTcM + mseg + 1));
+    w->t_part = c.take<float>((size_t)kTcMaxSplit * T1 * kMaxRank * ns);
+    w->runs = c.take<int32_t>((size_t)2 * T1);   // run scratch of the routing pass
+    return c.off + 256;
+}
+
+// Grid column chunks of width W over the slices (expand launches).
+static void set_chunks(ApplyArgs& a, int W) {
+    int c = 0;
+    for (int q = 0; q < a.n_slices; ++q) {
+        a.sl[q].chunk0 = c;
+        c += (int)cdiv(a.sl[q].d_out, W);
+    }
+    a.n_chunks = c;
+}
+
+static lf_status apply_impl(int32_t T, int32_t d_in, const void* x, void* y, int64_t y_ld, const int32_t* ids,
+                            int32_t n_adapters, const lf_slice* sl, int32_t ns, float scale, const float* scales,
+                            int32_t* seg_out, void* ws, size_t ws_bytes, cudaStream_t s) {
+    if (T < 0 || d_in < 1 || n_adapters < 1 || n_adapters > 16384 || ns < 1 || ns > kMaxSlices || !sl)
+        return LF_ERR_INVALID_ARG;
+    if (T == 0) return LF_OK;
+    if (!x || !y || !ids || !ws) return LF_ERR_INVALID_ARG;
+    if ((d_in & 7) || (y_ld & 7)) return LF_ERR_ALIGNMENT;
+    if (!aligned16(x) || !aligned16(y)) return LF_ERR_ALIGNMENT;
+    for (int q = 0; q < ns; ++q) {
+        const lf_slice& t = sl[q];
+        if (t.d_out < 1 || t.pool_elems_A < 0 || t.pool_elems_Bt < 0 || t.y_offset < 0 || t.y_offset + t.d_out > y_ld)
+            return LF_ERR_INVALID_ARG;
+        if (!t.ranks || !t.off_A || !t.off_Bt || !t.A_pool || !t.Bt_pool) return LF_ERR_INVALID_ARG;
+        if ((t.d_out & 7) || (t.y_offset & 7)) return LF_ERR_ALIGNMENT;
+        if (!aligned16(t.A_pool) || !aligned16(t.Bt_pool)) return LF_ERR_ALIGNMENT;
+    }
+    ApplyWs w;
+    if (ws_bytes < carve_apply(nullptr, T, n_adapters, ns, &w)) return LF_ERR_WORKSPACE;
+    carve_apply(reinterpret_cast<char*>(align_up((int64_t)reinterpret_cast<uintptr_t>(ws), 256)), T, n_adapters,
+                ns, &w);
+    ApplyArgs A{};
+    A.T = T;
+    A.d_in = d_in;
+    A.n_adapters = n_adapters;
+    A.n_slices = ns;
+    A.y_ld = y_ld;
+    A.ldt = kMaxRank * ns;
+    A.x = reinterpret_cast<const __nv_bfloat16*>(x);
+    A.y = reinterpret_cast<__nv_bfloat16*>(y);
+    A.ids = ids;
+    A.scale = scale;
+    A.scales = scales;
+    for (int q = 0; q < ns; ++q) {
+        SliceTab& t = A.sl[q];
+        t.d_out = sl[q].d_out;
+        t.t_col = kMaxRank * q;
+        t.y_off = sl[q].y_offset;
+        t.ranks = sl[q].ranks;
+        t.off_A = sl[q].off_A;
+        t.off_Bt = sl[q].off_Bt;
+        t.A_pool = reinterpret_cast<const __nv_bfloat16*>(sl[q].A_pool);
+        t.Bt_pool = reinterpret_cast<const __nv_bfloat16*>(sl[q].Bt_pool);
+        t.pool_A = sl[q].pool_elems_A;
+        t.pool_Bt = sl[q].pool_elems_Bt;
+    }
+    A.counts = w.counts;
+    A.segs = w.segs;
+    A.perm = w.perm;
+    A.items = w.items;
+    A.tc_items = w.tc_items;
+    A.t_buf = w.t_buf;
+    A.t_part = w.t_part;
+
+    RouteOut o{};
+    o.counts = w.counts;
+    o.segs = w.segs;
+    o.perm = w.perm;
+    o.items = w.items;
+    o.tc_items = w.tc_items;
+    o.run_start = w.runs;
+    o.run_pos = w.runs + T;
+    o.seg_out = seg_out;
+    const bool decode_regime = (int64_t)T <= (int64_t)kGemvTok * n_adapters;
+    o.tc_enable = decode_regime ? 0 : 1;
+    const size_t rsmem = 2 * (size_t)n_adapters * sizeof(int32_t);
+    LF_CUDA_TRY(cudaFuncSetAttribute(route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rsmem));
+    if (decode_regime) {
+        // few tokens per adapter: token-parallel shrink + expand, no sort; the routing
+        // pass runs only when the caller asks for the segment table
+        if (seg_out) {
+            LF_LAUNCH("route", route_kernel, 1, route_threads(T, n_adapters), rsmem, s, ids, T, n_adapters, o);
+            LF_CUDA_TRY(cudaGetLastError());
+        }
+        set_chunks(A, kBgmvCols);
+        LF_LAUNCH("bgmv", bgmv_kernel, dim3((unsigned)T, (unsigned)A.n_chunks), kBgmvThreads, 0, s, A);
+        return launch_status();
+    }
+    LF_LAUNCH("route", route_kernel, 1, route_threads(T, n_adapters), rsmem, s, ids, T, n_adapters, o);
+    LF_CUDA_TRY(cudaGetLastError());
+    const int64_t mseg = std::min<int64_t>(T, n_adapters);
+    // segments under kTcMin tokens: GEMV shrink (per slice), then expand
+    const unsigned max_items = (unsigned)(T / kGemvTok + mseg + 1);
+    set_chunks(A, kGemvCols);
+    LF_LAUNCH("shrink_gemv", shrink_kernel, dim3(max_items, (unsigned)ns), kGemvThreads, 0, s, A);
+    LF_CUDA_TRY(cudaGetLastError());
+    LF_LAUNCH("expand_gemv", expand_kernel, dim3(max_items, (unsigned)A.n_chunks), kGemvThreads, 0, s, A);
+    LF_CUDA_TRY(cudaGetLastError());
+    // segments with >= kTcMin tokens: one tcgen05 shrink over all slices, then expand
+    const unsigned max_tc = (unsigned)(T / kTcM + mseg + 1);
+    const unsigned nsplit = (unsigned)cdiv(d_in, tc_split_len(d_in));
+    set_chunks(A, kTcCols);
+    if (ns == 1) {
+        constexpr size_t sm = shrink_tc_smem<kMaxRank>();
+        LF_CUDA_TRY(cudaFuncSetAttribute(shrink_tc_kernel<kMaxRank>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm));
+        LF_LAUNCH("shrink_tc", shrink_tc_kernel<kMaxRank>, dim3(max_tc, nsplit), kTcThreads, sm, s, A);
+    } else {
+        constexpr size_t sm = shrink_tc_smem<kMaxSlices * kMaxRank>();
+        LF_CUDA_TRY(cudaFuncSetAttribute(shrink_tc_kernel<kMaxSlices * kMaxRank>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm));
+        LF_LAUNCH("shrink_tc", shrink_tc_kernel<kMaxSlices * kMaxRank>, dim3(max_tc, nsplit), kTcThreads, sm, s, A);
+    }
+    LF_CUDA_TRY(cudaGetLastError());
+    LF_CUDA_TRY(cudaFuncSetAttribute(expand_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kExpandTcSmem));
+    LF_LAUNCH("expand_tc", expand_tc_kernel, dim3(max_tc, (unsigned)A.n_chunks), kTcExpThreads, kExpandTcSmem, s, A);
+    return launch_status();
+}
+
 // ------------------------------------------------- library-owned apply scratch
 // Routing scratch for lf_lora_shrink_expand_noalloc, laid out exactly as the
 // Carver lays out a caller workspace for (LF_NOALLOC_MAX_TOKENS, LF_NOALLOC_MAX_ADAPTERS).
@@ -685,135 +832,41 @@ lf_status lf_truncate_export(const lf_module* mods, int32_t n, lf_policy pol, co
     return launch_status();
 }
 
-size_t lf_apply_workspace_size(int32_t T, int32_t n_adapters) {
-    if (T < 0 || n_adapters < 1) return 0;
-    const int64_t mseg = std::min<int64_t>(T, n_adapters);
-    Carver c(nullptr);
-    c.take<int32_t>(4);
-    c.take<Seg>((size_t)std::max<int64_t>(mseg, 1));
-    c.take<int32_t>((size_t)std::max(T, 1));
-    c.take<GemvItem>((size_t)(T / kGemvTok + mseg + 1));
-    c.take<float>((size_t)std::max(T, 1) * kMaxRank);
-    c.take<TcItem>((size_t)(T / kTcM + mseg + 1));
-    c.take<float>((size_t)kTcMaxSplit * std::max(T, 1) * kMaxRank);
-    c.take<int32_t>((size_t)2 * std::max(T, 1));   // run scratch of the routing pass
-    return c.off + 256;
+size_t lf_apply_slices_workspace_size(int32_t T, int32_t n_adapters, int32_t n_slices) {
+    if (T < 0 || n_adapters < 1 || n_slices < 1 || n_slices > kMaxSlices) return 0;
+    ApplyWs w;
+    return carve_apply(nullptr, T, n_adapters, n_slices, &w);
 }
+
+size_t lf_apply_workspace_size(int32_t T, int32_t n_adapters) { return lf_apply_slices_workspace_size(T, n_adapters, 1); }
 
 lf_status lf_lora_shrink_expand(int32_t T, int32_t d_in, int32_t d_out, const void* x, void* y, const int32_t* ids,
                                 int32_t n_adapters, const int32_t* ranks, const int64_t* off_A,
                                 const int64_t* off_Bt, const void* A_pool, const void* Bt_pool,
                                 int64_t pool_elems_A, int64_t pool_elems_Bt, float scale, int32_t* seg_out,
                                 void* ws, size_t ws_bytes, lf_stream_t stream) {
-    if (T < 0 || d_in < 1 || d_out < 1 || n_adapters < 1 || n_adapters > 16384 || pool_elems_A < 0 ||
-        pool_elems_Bt < 0)
-        return LF_ERR_INVALID_ARG;
-    if (T == 0) return LF_OK;
-    if (!x || !y || !ids || !ranks || !off_A || !off_Bt || !A_pool || !Bt_pool || !ws) return LF_ERR_INVALID_ARG;
-    if ((d_in & 7) || (d_out & 7)) return LF_ERR_ALIGNMENT;
-    if (!aligned16(x) || !aligned16(y) || !aligned16(A_pool) || !aligned16(Bt_pool)) return LF_ERR_ALIGNMENT;
-    if (ws_bytes < lf_apply_workspace_size(T, n_adapters)) return LF_ERR_WORKSPACE;
-    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    const int64_t mseg = std::min<int64_t>(T, n_adapters);
-    char* wsa = reinterpret_cast<char*>(align_up((int64_t)reinterpret_cast<uintptr_t>(ws), 256));
-    Carver c(wsa);
-    RouteOut o{};
-    o.counts = c.take<int32_t>(4);
-    o.segs = c.take<Seg>((size_t)std::max<int64_t>(mseg, 1));
-    o.perm = c.take<int32_t>((size_t)T);
-    o.items = c.take<GemvItem>((size_t)(T / kGemvTok + mseg + 1));
-    float* t_buf = c.take<float>((size_t)T * kMaxRank);
-    o.tc_items = c.take<TcItem>((size_t)(T / kTcM + mseg + 1));
-    float* t_part = c.take<float>((size_t)kTcMaxSplit * T * kMaxRank);
-    int32_t* run_scratch = c.take<int32_t>((size_t)2 * T);
-    o.run_start = run_scratch;
-    o.run_pos = run_scratch + T;
-    o.seg_out = seg_out;
-    o.ranks = ranks;
-    o.off_A = off_A;
-    o.off_Bt = off_Bt;
-    o.pool_A = pool_elems_A;
-    o.pool_Bt = pool_elems_Bt;
-    o.d_in = d_in;
-    o.d_out = d_out;
-    const bool decode_regime = (int64_t)T <= (int64_t)kGemvTok * n_adapters;
-    o.tc_enable = decode_regime ? 0 : 1;
-    const size_t rsmem = 2 * (size_t)n_adapters * sizeof(int32_t);
-    LF_CUDA_TRY(cudaFuncSetAttribute(route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rsmem));
-    if (decode_regime) {
-        // few tokens per adapter: token-parallel shrink + expand, no sort; the routing
-        // pass runs only when the caller asks for the segment table
-        if (seg_out) {
-            LF_LAUNCH("route", route_kernel, 1, route_threads(T, n_adapters), rsmem, s, ids, T, n_adapters, o);
-            LF_CUDA_TRY(cudaGetLastError());
-        }
-        BgmvArgs b;
-        b.n_adapters = n_adapters;
-        b.d_in = d_in;
-        b.d_out = d_out;
-        b.x = reinterpret_cast<const __nv_bfloat16*>(x);
-        b.y = reinterpret_cast<__nv_bfloat16*>(y);
-        b.ids = ids;
-        b.ranks = ranks;
-        b.off_A = off_A;
-        b.off_Bt = off_Bt;
-        b.A_pool = reinterpret_cast<const __nv_bfloat16*>(A_pool);
-        b.Bt_pool = reinterpret_cast<const __nv_bfloat16*>(Bt_pool);
-        b.pool_A = pool_elems_A;
-        b.pool_Bt = pool_elems_Bt;
-        b.scale = scale;
-        LF_LAUNCH("bgmv", bgmv_kernel, dim3((unsigned)T, (unsigned)cdiv(d_out, kBgmvCols)), kBgmvThreads, 0, s, b);
-        return launch_status();
-    }
-    LF_LAUNCH("route", route_kernel, 1, route_threads(T, n_adapters), rsmem, s, ids, T, n_adapters, o);
-    LF_CUDA_TRY(cudaGetLastError());
-    GemvArgs g;
-    g.d_in = d_in;
-    g.d_out = d_out;
-    g.x = reinterpret_cast<const __nv_bfloat16*>(x);
-    g.y = reinterpret_cast<__nv_bfloat16*>(y);
-    g.ranks = ranks;
-    g.off_A = off_A;
-    g.off_Bt = off_Bt;
-    g.A_pool = reinterpret_cast<const __nv_bfloat16*>(A_pool);
-    g.Bt_pool = reinterpret_cast<const __nv_bfloat16*>(Bt_pool);
-    g.pool_A = pool_elems_A;
-    g.pool_Bt = pool_elems_Bt;
-    g.scale = scale;
-    g.counts = o.counts;
-    g.segs = o.segs;
-    g.perm = o.perm;
-    g.items = o.items;
-    g.t_buf = t_buf;
-    const unsigned max_items = (unsigned)(T / kGemvTok + mseg + 1);
-    const dim3 grid2(max_items, (unsigned)cdiv(d_out, kGemvCols));
-    LF_LAUNCH("shrink_gemv", shrink_kernel, max_items, kGemvThreads, 0, s, g);
-    LF_CUDA_TRY(cudaGetLastError());
-    LF_LAUNCH("expand_gemv", expand_kernel, grid2, kGemvThreads, 0, s, g);
-    LF_CUDA_TRY(cudaGetLastError());
-    // segments with >= kTcMin tokens: tcgen05 shrink, then expand
-    TcArgs ta;
-    ta.d_in = d_in;
-    ta.d_out = d_out;
-    ta.x = g.x;
-    ta.y = g.y;
-    ta.A_pool = g.A_pool;
-    ta.Bt_pool = g.Bt_pool;
-    ta.scale = scale;
-    ta.counts = o.counts;
-    ta.items = o.tc_items;
-    ta.perm = o.perm;
-    ta.t_part = t_part;
-    ta.T = T;
-    const unsigned max_tc = (unsigned)(T / kTcM + mseg + 1);
-    const unsigned nsplit = (unsigned)cdiv(d_in, tc_split_len(d_in));
-    LF_CUDA_TRY(cudaFuncSetAttribute(shrink_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kShrinkTcSmem));
-    LF_CUDA_TRY(cudaFuncSetAttribute(expand_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kExpandTcSmem));
-    LF_LAUNCH("shrink_tc", shrink_tc_kernel, dim3(max_tc, nsplit), kTcThreads, kShrinkTcSmem, s, ta);
-    LF_CUDA_TRY(cudaGetLastError());
-    LF_LAUNCH("expand_tc", expand_tc_kernel, dim3(max_tc, (unsigned)cdiv(d_out, kTcCols)), kTcExpThreads, kExpandTcSmem, s,
-              ta);
-    return launch_status();
+    if (d_out < 1) return LF_ERR_INVALID_ARG;
+    if (T > 0 && (!ranks || !off_A || !off_Bt || !A_pool || !Bt_pool)) return LF_ERR_INVALID_ARG;
+    lf_slice one{};
+    one.d_out = d_out;
+    one.y_offset = 0;
+    one.ranks = ranks;
+    one.off_A = off_A;
+    one.off_Bt = off_Bt;
+    one.A_pool = A_pool;
+    one.Bt_pool = Bt_pool;
+    one.pool_elems_A = pool_elems_A;
+    one.pool_elems_Bt = pool_elems_Bt;
+    return apply_impl(T, d_in, x, y, d_out, ids, n_adapters, &one, 1, scale, nullptr, seg_out, ws, ws_bytes,
+                      reinterpret_cast<cudaStream_t>(stream));
+}
+
+lf_status lf_lora_shrink_expand_slices(int32_t T, int32_t d_in, const void* x, void* y, int64_t y_ld,
+                                       const int32_t* ids, int32_t n_adapters, const lf_slice* slices,
+                                       int32_t n_slices, float scale, const float* adapter_scale, int32_t* seg_out,
+                                       void* ws, size_t ws_bytes, lf_stream_t stream) {
+    return apply_impl(T, d_in, x, y, y_ld, ids, n_adapters, slices, n_slices, scale, adapter_scale, seg_out, ws,
+                      ws_bytes, reinterpret_cast<cudaStream_t>(stream));
 }
 
 lf_status lf_lora_shrink_expand_noalloc(int32_t T, int32_t d_in, int32_t d_out, const void* x, void* y,
@@ -841,13 +894,6 @@ lf_status lf_lora_shrink_expand_noalloc(int32_t T, int32_t d_in, int32_t d_out, 
     o.items = c.take<GemvItem>((size_t)LF_NOALLOC_MAX_TOKENS / kGemvTok + LF_NOALLOC_MAX_ADAPTERS + 1);
     float* t_buf = c.take<float>((size_t)LF_NOALLOC_MAX_TOKENS * kMaxRank);
     o.seg_out = seg_out;
-    o.ranks = ranks;
-    o.off_A = off_A;
-    o.off_Bt = off_Bt;
-    o.pool_A = pool_elems_A;
-    o.pool_Bt = pool_elems_Bt;
-    o.d_in = d_in;
-    o.d_out = d_out;
     o.tc_items = nullptr;
     o.tc_enable = 0;   // this entry point keeps every segment on the GEMV kernels
     if (c.off > kNoallocScratchBytes) return LF_ERR_WORKSPACE;
@@ -856,33 +902,44 @@ lf_status lf_lora_shrink_expand_noalloc(int32_t T, int32_t d_in, int32_t d_out, 
     LF_CUDA_TRY(cudaFuncSetAttribute(route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rsmem));
     LF_LAUNCH("route", route_kernel, 1, route_threads(T, n_adapters), rsmem, s, ids, T, n_adapters, o);
     LF_CUDA_TRY(cudaGetLastError());
-    GemvArgs g;
-    g.d_in = d_in;
-    g.d_out = d_out;
-    g.x = reinterpret_cast<const __nv_bfloat16*>(x);
-    g.y = reinterpret_cast<__nv_bfloat16*>(y);
-    g.ranks = ranks;
-    g.off_A = off_A;
-    g.off_Bt = off_Bt;
-    g.A_pool = reinterpret_cast<const __nv_bfloat16*>(A_pool);
-    g.Bt_pool = reinterpret_cast<const __nv_bfloat16*>(Bt_pool);
-    g.pool_A = pool_elems_A;
-    g.pool_Bt = pool_elems_Bt;
-    g.scale = scale;
-    g.counts = o.counts;
-    g.segs = o.segs;
-    g.perm = o.perm;
-    g.items = o.items;
-    g.t_buf = t_buf;
+    ApplyArgs A{};
+    A.T = T;
+    A.d_in = d_in;
+    A.n_adapters = n_adapters;
+    A.n_slices = 1;
+    A.y_ld = d_out;
+    A.ldt = kMaxRank;
+    A.x = reinterpret_cast<const __nv_bfloat16*>(x);
+    A.y = reinterpret_cast<__nv_bfloat16*>(y);
+    A.ids = ids;
+    A.scale = scale;
+    A.scales = nullptr;
+    SliceTab& t = A.sl[0];
+    t.d_out = d_out;
+    t.t_col = 0;
+    t.y_off = 0;
+    t.ranks = ranks;
+    t.off_A = off_A;
+    t.off_Bt = off_Bt;
+    t.A_pool = reinterpret_cast<const __nv_bfloat16*>(A_pool);
+    t.Bt_pool = reinterpret_cast<const __nv_bfloat16*>(Bt_pool);
+    t.pool_A = pool_elems_A;
+    t.pool_Bt = pool_elems_Bt;
+    A.counts = o.counts;
+    A.segs = o.segs;
+    A.perm = o.perm;
+    A.items = o.items;
+    A.t_buf = t_buf;
+    set_chunks(A, kGemvCols);
     const unsigned max_items = (unsigned)(T / kGemvTok + mseg + 1);
-    const dim3 grid2(max_items, (unsigned)cdiv(d_out, kGemvCols));
+    const dim3 grid2(max_items, (unsigned)A.n_chunks);
     if ((int64_t)T <= (int64_t)kGemvTok * n_adapters) {
         // decode regime (few tokens per adapter): shrink and expand in one launch
-        LF_LAUNCH("fused_gemv", fused_gemv_kernel, grid2, kGemvThreads, 0, s, g);
+        LF_LAUNCH("fused_gemv", fused_gemv_kernel, grid2, kGemvThreads, 0, s, A);
     } else {
-        LF_LAUNCH("shrink_gemv", shrink_kernel, max_items, kGemvThreads, 0, s, g);
+        LF_LAUNCH("shrink_gemv", shrink_kernel, dim3(max_items, 1u), kGemvThreads, 0, s, A);
         LF_CUDA_TRY(cudaGetLastError());
-        LF_LAUNCH("expand_gemv", expand_kernel, grid2, kGemvThreads, 0, s, g);
+        LF_LAUNCH("expand_gemv", expand_kernel, grid2, kGemvThreads, 0, s, A);
     }
     return launch_status();
 }

@@ -5,16 +5,17 @@
 // then the scaled B step into y).  Only the prefill-shaped case is a real dense
 // contraction (M = tokens of one adapter), so only it uses the tensor cores.
 //
-// Shrink: D[128 tokens x N] = X[128 x d_in] * A'^T[d_in x N], bf16 in, fp32 in TMEM,
-//   N = k rounded up to 16 (padding lives in shared memory only).  X rows are
+// Shrink: D[128 tokens x N] = X[128 x d_in] * [A'_1; A'_2; ...]^T, bf16 in, fp32 in
+//   TMEM, N = the sum of the slices' ranks rounded up to 16 (padding lives in shared
+//   memory only): x is read once for every slice that shares it.  X rows are
 //   gathered through the token permutation with 16-byte cp.async into a 4-stage
 //   ring of K-major core matrices; one thread issues the MMAs and commits each
 //   stage to an mbarrier that frees the stage for the next copy.
-// Expand: D[128 x 128] = t_hi * B + t_lo * B with t = t_hi + t_lo split into two
-//   bf16 values (about 16 significant bits of the fp32 t); B = B'^T tile,
+// Expand (per slice): D[128 x 128] = t_hi * B + t_lo * B with t = t_hi + t_lo split
+//   into two bf16 values (about 16 significant bits of the fp32 t); B = B'^T tile,
 //   MN-major; the epilogue reads D from tensor memory and updates y once.
 #pragma once
-#include "common.cuh"
+#include "apply_common.cuh"
 #include "tc.cuh"
 
 namespace lf {
@@ -34,25 +35,6 @@ __host__ __device__ inline int tc_split_len(int d_in) {
     return len < 1024 ? 1024 : len;
 }
 
-struct TcItem {
-    int32_t adapter, k, ntok, tok0;   // tok0: position of the first token in the permutation
-    int64_t oa, ob;
-};
-
-struct TcArgs {
-    int32_t d_in, d_out;
-    const __nv_bfloat16* x;
-    __nv_bfloat16* y;
-    const __nv_bfloat16* A_pool;
-    const __nv_bfloat16* Bt_pool;
-    float scale;
-    const int32_t* counts;   // [3] = number of tensor-core items
-    const TcItem* items;
-    const int32_t* perm;
-    float* t_part;           // kTcMaxSplit x T x kMaxRank fp32 partial sums, row = permutation position
-    int32_t T;
-};
-
 // ---- shrink ---------------------------------------------------------------
 // CTA (token tile of one segment, split of d_in), 4 warps in roles:
 //   warps 0, 2, 3, producers: gather the stage's 128 x rows (64 d_in elements,
@@ -66,14 +48,18 @@ struct TcArgs {
 //   all warps: epilogue from TMEM (warp w reads lanes 32w ..) into t_part.
 constexpr int kTcAhead = 2;      // stages in flight before the producers signal the oldest
 constexpr int kTcProducers = 3;  // producer warps: 0, 2, 3 (warp 1 issues the MMAs)
+// MAXN = most B rows (summed ranks) a CTA can take: 64 for one slice, 256 for up to 4.
+template <int MAXN>
 struct ShrinkTcSmem {
-    __nv_bfloat16 a[kTcStages][kTcM * kTcKB];       // 16 KB per stage
-    __nv_bfloat16 b[kTcStages][kMaxRank * kTcKB];   //  8 KB per stage
+    __nv_bfloat16 a[kTcStages][kTcM * kTcKB];    // 16 KB per stage
+    __nv_bfloat16 b[kTcStages][MAXN * kTcKB];    //  8 KB (MAXN 64) or 32 KB (MAXN 256) per stage
     uint64_t full[kTcStages];
     uint64_t empty[kTcStages];
     uint64_t done;
     uint32_t tmem;
     int32_t toks[kTcM];
+    int32_t kcum[kMaxSlices + 1];   // B rows of slice s: kcum[s] .. kcum[s+1]-1
+    int64_t oa[kMaxSlices];
 };
 
 // byte offset of element (row, kk) of a K-major operand tile with 64 K-elements per row
@@ -90,26 +76,41 @@ __device__ __forceinline__ void mbar_arrive1(uint64_t* bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
-__global__ void __launch_bounds__(kTcThreads) shrink_tc_kernel(TcArgs a) {
+template <int MAXN>
+__global__ void __launch_bounds__(kTcThreads) shrink_tc_kernel(ApplyArgs a) {
     extern __shared__ __align__(1024) unsigned char tc_raw[];
-    auto& s = *reinterpret_cast<ShrinkTcSmem*>(tc_raw);
+    auto& s = *reinterpret_cast<ShrinkTcSmem<MAXN>*>(tc_raw);
     if ((int)blockIdx.x >= a.counts[3]) return;
-    const TcItem it = a.items[blockIdx.x];
-    if (it.k <= 0) return;
+    const TcItem it = a.tc_items[blockIdx.x];
     const int split = blockIdx.y, slen = tc_split_len(a.d_in);
     const int kbeg = split * slen;
     if (kbeg >= a.d_in) return;   // uniform: this split has no columns
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int k = it.k, nt = it.ntok;
-    const int npad = (k + 15) & ~15;
+    if (tid == 0) {   // rows of every slice in the concatenated B operand
+        int kc = 0;
+        for (int q = 0; q < a.n_slices; ++q) {
+            int k;
+            int64_t oa, ob;
+            slice_factors(a, q, it.adapter, split == 0, k, oa, ob);
+            s.kcum[q] = kc;
+            s.oa[q] = oa;
+            kc += k;
+        }
+        s.kcum[a.n_slices] = kc;
+    }
+    __syncthreads();
+    const int ktot = s.kcum[a.n_slices];
+    if (ktot <= 0) return;   // uniform
+    const int nt = it.ntok;
+    const int npad = (ktot + 15) & ~15;
     for (int m = tid; m < kTcM; m += kTcThreads) s.toks[m] = m < nt ? a.perm[it.tok0 + m] : 0;
-    // rows k..npad-1 of every B stage stay zero (never written by the copies)
-    for (int e = tid; e < kTcStages * (npad - k) * kTcKB; e += kTcThreads) {
-        const int st = e / ((npad - k) * kTcKB), r2 = e % ((npad - k) * kTcKB);
-        const int n = k + r2 / kTcKB, kk = r2 % kTcKB;
+    // rows ktot..npad-1 of every B stage stay zero (never written by the copies)
+    for (int e = tid; e < kTcStages * (npad - ktot) * kTcKB; e += kTcThreads) {
+        const int st = e / ((npad - ktot) * kTcKB), r2 = e % ((npad - ktot) * kTcKB);
+        const int n = ktot + r2 / kTcKB, kk = r2 % kTcKB;
         *reinterpret_cast<__nv_bfloat16*>(reinterpret_cast<char*>(s.b[st]) + kmaj64(n, kk)) = __float2bfloat16(0.f);
     }
-    if (warp == 0) tc::tmem_alloc(&s.tmem, 64);
+    if (warp == 0) tc::tmem_alloc(&s.tmem, MAXN);
     if (tid == 0) {
         for (int i = 0; i < kTcStages; ++i) {
             mbar_init(&s.full[i], 32 * kTcProducers);
@@ -128,7 +129,6 @@ __global__ void __launch_bounds__(kTcThreads) shrink_tc_kernel(TcArgs a) {
 
     const int pidx = warp == 0 ? 0 : warp - 1;   // producer index (warps 0, 2, 3)
     if (warp != 1 && pidx < kTcProducers) {   // producers
-        const __nv_bfloat16* Ap = a.A_pool + it.oa;
         for (int kb = 0; kb < nK && ok; ++kb) {
             const int st = kb % kTcStages;
             if (kb >= kTcStages) ok = mbar_wait(&s.empty[st], (uint32_t)((kb / kTcStages - 1) & 1));
@@ -146,15 +146,19 @@ __global__ void __launch_bounds__(kTcThreads) shrink_tc_kernel(TcArgs a) {
                 const bool v = m < nt && kk < kend;
                 cp_async16_zfill(abase + kmaj64(m, kc * 8), v ? a.x + (int64_t)s.toks[m] * a.d_in + kk : a.x, v);
             }
-            const int nrb = (k + 7) >> 3;
+            const int nrb = (ktot + 7) >> 3;
             for (int c = lane + 32 * pidx; c < nrb * 64; c += 32 * kTcProducers) {
                 const int u = c >> 4;
                 const int n = 8 * (u % nrb) + (c & 7);
                 const int kc = 2 * (u / nrb) + ((c >> 3) & 1);
                 const int kk = k0 + kc * 8;
-                if (n < k) {
+                if (n < ktot) {
+                    int q = 0;
+                    while (q + 1 < a.n_slices && n >= s.kcum[q + 1]) ++q;
+                    const __nv_bfloat16* Ap = a.sl[q].A_pool + s.oa[q];
                     const bool v = kk < kend;
-                    cp_async16_zfill(bbase + kmaj64(n, kc * 8), v ? Ap + (int64_t)n * a.d_in + kk : Ap, v);
+                    cp_async16_zfill(bbase + kmaj64(n, kc * 8),
+                                     v ? Ap + (int64_t)(n - s.kcum[q]) * a.d_in + kk : Ap, v);
                 }
             }
             tc::cp_async_commit();
@@ -193,23 +197,30 @@ __global__ void __launch_bounds__(kTcThreads) shrink_tc_kernel(TcArgs a) {
     tc::fence_after_sync();
     if (ok) {
         const int m = warp * 32 + lane;
-        float* trow = a.t_part + ((size_t)split * a.T + it.tok0 + m) * kMaxRank;
+        float* trow = a.t_part + ((size_t)split * a.T + it.tok0 + m) * a.ldt;
+        int q = 0;
         for (int c0 = 0; c0 < npad; c0 += 16) {
             float v[16];
             tc::tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c0, v);
             if (m < nt) {
 #pragma unroll
-                for (int i = 0; i < 16; ++i)
-                    if (c0 + i < k) trow[c0 + i] = v[i];
+                for (int i = 0; i < 16; ++i) {
+                    const int c = c0 + i;
+                    if (c < ktot) {
+                        while (q + 1 < a.n_slices && c >= s.kcum[q + 1]) ++q;
+                        trow[a.sl[q].t_col + c - s.kcum[q]] = v[i];
+                    }
+                }
             }
         }
     }
     tc::fence_before_sync();
     __syncthreads();
-    if (warp == 0) tc::tmem_dealloc(tmem, 64);
+    if (warp == 0) tc::tmem_dealloc(tmem, MAXN);
 }
 
-constexpr size_t kShrinkTcSmem = sizeof(ShrinkTcSmem) + 1024;
+template <int MAXN>
+constexpr size_t shrink_tc_smem() { return sizeof(ShrinkTcSmem<MAXN>) + 1024; }
 
 // ---- expand ---------------------------------------------------------------
 // CTA (token tile of one segment, kTcCols columns of d_out), 256 threads.  The
@@ -236,18 +247,24 @@ struct ExpandTcSmem {
     int32_t toks[kTcM];
 };
 
-__global__ void __launch_bounds__(kTcExpThreads, 1) expand_tc_kernel(TcArgs a) {
+__global__ void __launch_bounds__(kTcExpThreads, 1) expand_tc_kernel(ApplyArgs a) {
     extern __shared__ __align__(1024) unsigned char tc_raw[];
     auto& s = *reinterpret_cast<ExpandTcSmem*>(tc_raw);
     if ((int)blockIdx.x >= a.counts[3]) return;
-    const TcItem it = a.items[blockIdx.x];
-    if (it.k <= 0) return;
-    const int e_begin = blockIdx.y * kTcCols;
-    if (e_begin >= a.d_out) return;
-    const int e_end = min(a.d_out, e_begin + kTcCols);
+    const TcItem it = a.tc_items[blockIdx.x];
+    const int sl = slice_of_chunk(a, blockIdx.y);
+    const SliceTab& S = a.sl[sl];
+    int k;
+    int64_t oa, ob;
+    if (!slice_factors(a, sl, it.adapter, false, k, oa, ob)) return;   // reported by the shrink
+    const int e_begin = ((int)blockIdx.y - S.chunk0) * kTcCols;
+    if (e_begin >= S.d_out) return;
+    const int e_end = min(S.d_out, e_begin + kTcCols);
     const int nit = (e_end - e_begin + kTcN2 - 1) / kTcN2;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int k = it.k, nt = it.ntok;
+    const int nt = it.ntok;
+    const float scale = adapter_scale(a, it.adapter);
+    __nv_bfloat16* ybase = a.y + S.y_off;
     const int kpad = (k + 15) & ~15;
     const uint32_t sbo = (uint32_t)(kpad / 8) * 128;   // 8-row groups of t / 8-column groups of B
     for (int m = tid; m < kTcM; m += kTcExpThreads) s.toks[m] = m < nt ? a.perm[it.tok0 + m] : 0;
@@ -262,7 +279,7 @@ __global__ void __launch_bounds__(kTcExpThreads, 1) expand_tc_kernel(TcArgs a) {
             float acc = 0.f;
             if (m < nt && j < k)
                 for (int sp = 0; sp < nsplit; ++sp)   // fixed order: bitwise reproducible
-                    acc += a.t_part[((size_t)sp * a.T + it.tok0 + m) * kMaxRank + j];
+                    acc += a.t_part[((size_t)sp * a.T + it.tok0 + m) * a.ldt + S.t_col + j];
             tv[i] = acc;
         }
         __align__(16) __nv_bfloat16 hi[8], lo[8];
@@ -282,7 +299,7 @@ __global__ void __launch_bounds__(kTcExpThreads, 1) expand_tc_kernel(TcArgs a) {
     }
     __syncthreads();   // toks visible to the copies below
 
-    const __nv_bfloat16* Bt = a.Bt_pool + it.ob;
+    const __nv_bfloat16* Bt = S.Bt_pool + ob;
     auto issue_y = [&](int i) {   // y rows of step i -> yt[i % 3]; rows past the tile / columns past the range zero-filled
         const int e0 = e_begin + i * kTcN2;
         __nv_bfloat16* dst = s.yt[i % kTcYBuf];
@@ -290,7 +307,7 @@ __global__ void __launch_bounds__(kTcExpThreads, 1) expand_tc_kernel(TcArgs a) {
             const int row = c >> 4, ch = c & 15;
             const int e = e0 + ch * 8;
             const bool ok = row < nt && e < e_end;
-            cp_async16_zfill(dst + row * kTcYLd + ch * 8, ok ? a.y + (int64_t)s.toks[row] * a.d_out + e : a.y, ok);
+            cp_async16_zfill(dst + row * kTcYLd + ch * 8, ok ? ybase + (int64_t)s.toks[row] * a.y_ld + e : ybase, ok);
         }
     };
     auto issue_b = [&](int i) {   // B'^T rows 0..kpad-1 of step i -> b[i % 2], MN-major
@@ -301,7 +318,7 @@ __global__ void __launch_bounds__(kTcExpThreads, 1) expand_tc_kernel(TcArgs a) {
             const int e = e0 + nc * 8;
             const bool ok = j < k && e < e_end;
             cp_async16_zfill(dst + (uint32_t)nc * sbo + (uint32_t)(j >> 3) * 128 + (uint32_t)(j & 7) * 16,
-                             ok ? Bt + (int64_t)j * a.d_out + e : Bt, ok);
+                             ok ? Bt + (int64_t)j * S.d_out + e : Bt, ok);
         }
     };
     issue_y(0);
@@ -355,8 +372,8 @@ __global__ void __launch_bounds__(kTcExpThreads, 1) expand_tc_kernel(TcArgs a) {
 #pragma unroll
                     for (int p = 0; p < 4; ++p) {
                         const float2 yf = __bfloat1622float2(y2[p]);
-                        y2[p] = __floats2bfloat162_rn(fmaf(a.scale, v[8 * half + 2 * p], yf.x),
-                                                      fmaf(a.scale, v[8 * half + 2 * p + 1], yf.y));
+                        y2[p] = __floats2bfloat162_rn(fmaf(scale, v[8 * half + 2 * p], yf.x),
+                                                      fmaf(scale, v[8 * half + 2 * p + 1], yf.y));
                     }
                     yp[half] = yv;
                 }
@@ -370,7 +387,7 @@ __global__ void __launch_bounds__(kTcExpThreads, 1) expand_tc_kernel(TcArgs a) {
                 const int row = c >> 4, ch = c & 15;
                 const int e = e0 + ch * 8;
                 if (row < nt && e < e_end)
-                    *reinterpret_cast<uint4*>(a.y + (int64_t)s.toks[row] * a.d_out + e) =
+                    *reinterpret_cast<uint4*>(ybase + (int64_t)s.toks[row] * a.y_ld + e) =
                         *reinterpret_cast<const uint4*>(yt + row * kTcYLd + ch * 8);
             }
         }

@@ -43,6 +43,14 @@ class lf_phase_time(ctypes.Structure):
     _fields_ = [("name", ctypes.c_char * 32), ("total_ms", ctypes.c_double), ("launches", ctypes.c_int64)]
 
 
+class lf_slice(ctypes.Structure):
+    """One output slice of lf_lora_shrink_expand_slices (mirrors the C struct)."""
+    _fields_ = [("d_out", ctypes.c_int32), ("reserved", ctypes.c_int32), ("y_offset", ctypes.c_int64),
+                ("ranks", ctypes.c_void_p), ("off_A", ctypes.c_void_p), ("off_Bt", ctypes.c_void_p),
+                ("A_pool", ctypes.c_void_p), ("Bt_pool", ctypes.c_void_p),
+                ("pool_elems_A", ctypes.c_int64), ("pool_elems_Bt", ctypes.c_int64)]
+
+
 class LFError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
@@ -80,6 +88,11 @@ def lib() -> ctypes.CDLL:
         L.lf_lora_shrink_expand.argtypes = [_I32, _I32, _I32, _P, _P, _P, _I32, _P, _P, _P, _P, _P,
                                             _I64, _I64, ctypes.c_float, _P, _P, _SZ, _P]
         L.lf_lora_shrink_expand.restype = ctypes.c_int
+        L.lf_apply_slices_workspace_size.argtypes = [_I32, _I32, _I32]
+        L.lf_apply_slices_workspace_size.restype = _SZ
+        L.lf_lora_shrink_expand_slices.argtypes = [_I32, _I32, _P, _P, _I64, _P, _I32, _P, _I32,
+                                                   ctypes.c_float, _P, _P, _P, _SZ, _P]
+        L.lf_lora_shrink_expand_slices.restype = ctypes.c_int
         L.lf_lora_shrink_expand_noalloc.argtypes = [_I32, _I32, _I32, _P, _P, _P, _I32, _P, _P, _P, _P, _P,
                                                     _I64, _I64, ctypes.c_float, _P, _P]
         L.lf_lora_shrink_expand_noalloc.restype = ctypes.c_int
@@ -98,7 +111,7 @@ def exported_symbols() -> list[str]:
             "lf_select_ranks", "lf_export_workspace_size", "lf_export_pool_bound", "lf_truncate_export",
             "lf_apply_workspace_size", "lf_lora_shrink_expand", "lf_status_string", "lf_get_device_status",
             "lf_profile_enable", "lf_profile_reset", "lf_profile_read", "lf_launch_count",
-            "lf_lora_shrink_expand_noalloc"]
+            "lf_lora_shrink_expand_noalloc", "lf_apply_slices_workspace_size", "lf_lora_shrink_expand_slices"]
 
 # Limits of lf_lora_shrink_expand_noalloc (its scratch is a fixed array in the library).
 NOALLOC_MAX_TOKENS = 16384
@@ -201,6 +214,27 @@ def lf_lora_shrink_expand(x, y, ids, n_adapters, ranks, off_A, off_Bt, A_pool, B
                                      _ptr(seg_out), _ptr(ws), ws.numel() if ws is not None else 0,
                                      _stream(stream))
     return _check(st, "lf_lora_shrink_expand") if check else st
+
+
+def lf_apply_slices_workspace_size(T: int, n_adapters: int, n_slices: int) -> int:
+    return lib().lf_apply_slices_workspace_size(T, n_adapters, n_slices)
+
+
+def make_slice(d_out, y_offset, ranks, off_A, off_Bt, A_pool, Bt_pool) -> lf_slice:
+    """lf_slice from device tensors (ranks int32, offsets int64, pools bf16)."""
+    return lf_slice(int(d_out), 0, int(y_offset), _ptr(ranks), _ptr(off_A), _ptr(off_Bt), _ptr(A_pool),
+                    _ptr(Bt_pool), A_pool.numel(), Bt_pool.numel())
+
+
+def lf_lora_shrink_expand_slices(x, y, ids, n_adapters, slices, scale, ws, adapter_scale=None, seg_out=None,
+                                 stream=None, check=True) -> int:
+    """slices: list of lf_slice (make_slice); y: T x y_ld bf16 holding every slice."""
+    T, d_in = x.shape
+    arr = (lf_slice * len(slices))(*slices)
+    st = lib().lf_lora_shrink_expand_slices(T, d_in, _ptr(x), _ptr(y), y.shape[1], _ptr(ids), n_adapters, arr,
+                                            len(slices), float(scale), _ptr(adapter_scale), _ptr(seg_out), _ptr(ws),
+                                            ws.numel() if ws is not None else 0, _stream(stream))
+    return _check(st, "lf_lora_shrink_expand_slices") if check else st
 
 
 def lf_lora_shrink_expand_noalloc(x, y, ids, n_adapters, ranks, off_A, off_Bt, A_pool, Bt_pool, scale,

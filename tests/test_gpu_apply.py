@@ -161,3 +161,95 @@ def test_routing_of_long_mixed_batch():
     assert st == 0
     check_routing(seg, ids, n)
     assert_close(y, oracle_y(x, y0, ids, ranks, offA, offB, Ap, Bt, 1.0))
+
+
+def make_slices(widths, n, d_in, key, rank_hi=65):
+    """Per-slice pools with ragged ranks; slices laid out in y with an 8-column gap each."""
+    g = np.random.default_rng(key[-1])
+    out, y_off = [], 0
+    for s, d_out in enumerate(widths):
+        ranks = g.integers(1, rank_hi, size=n)
+        offA, offB, Ap, Bt = make_pools(ranks, d_in, d_out, key + (s,))
+        out.append(dict(d_out=d_out, y_off=y_off, ranks=ranks, offA=offA, offB=offB, Ap=Ap, Bt=Bt))
+        y_off += d_out + 8
+    return out, y_off
+
+
+def run_slices(x, y0, ids, sl, scale, adapter_scale=None, seg=False):
+    dev = "cuda"
+    T = x.shape[0]
+    n = len(sl[0]["ranks"])
+    y = y0.clone().to(dev)
+    keep = []
+    tup = []
+    for s in sl:
+        t = (s["d_out"], s["y_off"], torch.from_numpy(np.asarray(s["ranks"], np.int32)).to(dev),
+             torch.from_numpy(np.asarray(s["offA"][:-1], np.int64)).to(dev),
+             torch.from_numpy(np.asarray(s["offB"][:-1], np.int64)).to(dev), s["Ap"].to(dev), s["Bt"].to(dev))
+        keep.append(t)
+        tup.append(t)
+    seg_out = torch.full((2 + 3 * min(T, n) + T,), -7, dtype=torch.int32, device=dev) if seg else None
+    asc = torch.from_numpy(np.asarray(adapter_scale, np.float32)).to(dev) if adapter_scale is not None else None
+    api.shrink_expand_slices(x.to(dev), y, torch.from_numpy(np.asarray(ids, np.int32)).to(dev), tup, scale,
+                             adapter_scale=asc, seg_out=seg_out)
+    st = lf.lf_get_device_status()
+    return y.cpu(), (seg_out.cpu().numpy() if seg else None), st
+
+
+def oracle_slices(x, y0, ids, sl, scale, adapter_scale=None):
+    tup = [(s["d_out"], s["y_off"], s["ranks"], s["offA"][:-1], s["offB"][:-1], s["Ap"].float().numpy(),
+            s["Bt"].float().numpy()) for s in sl]
+    return OP.lora_apply_slices(x.float().numpy(), y0.float().numpy(), ids, tup, scale, adapter_scale)
+
+
+def check_slices(y, y0, want, sl, ids):
+    yv = y.float().numpy().astype(np.float64)
+    covered = np.zeros(y.shape[1], dtype=bool)
+    for s in sl:
+        c = slice(s["y_off"], s["y_off"] + s["d_out"])
+        d = np.abs(yv[:, c] - want[:, c]).max()
+        delta = np.abs(want[:, c] - y0.float().numpy()[:, c]).max()
+        assert d <= G.APPLY_TOL * max(delta, 1e-30), (s["d_out"], d, delta)
+        covered[c] = True
+    assert torch.equal(y[:, torch.from_numpy(~covered)], y0[:, torch.from_numpy(~covered)])   # gaps untouched
+    assert torch.equal(y[torch.from_numpy(ids < 0)], y0[torch.from_numpy(ids < 0)])           # unrouted rows
+
+
+@pytest.mark.parametrize("regime", ["decode", "gemv", "tensor_core"])
+def test_slices_match_oracle(regime):
+    # q/k/v-like slices sharing x; per-adapter scales; the three execution regimes:
+    # token-parallel (T <= 8n), sorted GEMV items (short segments), tcgen05 tiles
+    d_in = 512
+    if regime == "decode":
+        T, n = 96, 32
+        ids = synth.zipf_ids(T, n, 1.0, (8, 0))
+    elif regime == "gemv":
+        T, n = 300, 37
+        ids = synth.zipf_ids(T, n, 1.0, (8, 1))
+    else:
+        T, n = 1024, 4
+        ids = np.repeat(np.arange(n, dtype=np.int32), 256)
+    ids = ids.copy()
+    ids[np.random.default_rng(3).random(T) < 0.05] = -1
+    sl, y_ld = make_slices([512, 128, 256], n, d_in, (8, 2, T))
+    x = synth.normal_bf16((T, d_in), (8, 3, T))
+    y0 = synth.normal_bf16((T, y_ld), (8, 4, T))
+    asc = 0.5 + np.arange(n) / n
+    y, seg, st = run_slices(x, y0, ids, sl, 1.0, adapter_scale=asc, seg=True)
+    assert st == 0
+    check_routing(seg, ids, n)
+    check_slices(y, y0, oracle_slices(x, y0, ids, sl, 1.0, asc), sl, ids)
+
+
+def test_one_slice_call_equals_projection_call():
+    # lf_lora_shrink_expand is the one-slice case of the slice entry point: same bits
+    T, n, d_in, d_out = 2048, 4, 1024, 512
+    ids = np.repeat(np.arange(n, dtype=np.int32), 512)
+    offA, offB, Ap, Bt = make_pools([16, 24, 8, 64], d_in, d_out, (9, 0))
+    x = synth.normal_bf16((T, d_in), (9, 1))
+    y0 = synth.normal_bf16((T, d_out), (9, 2))
+    y1, _, st1 = run_apply(x, y0, ids, [16, 24, 8, 64], offA, offB, Ap, Bt, 0.75)
+    sl = [dict(d_out=d_out, y_off=0, ranks=np.array([16, 24, 8, 64]), offA=offA, offB=offB, Ap=Ap, Bt=Bt)]
+    y2, _, st2 = run_slices(x, y0, ids, sl, 0.75)
+    assert st1 == 0 and st2 == 0
+    assert torch.equal(y1, y2)

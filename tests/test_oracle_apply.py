@@ -87,3 +87,48 @@ def test_apply_matches_dense_delta_w(seed):
 def test_empty_batch():
     y = AP.lora_apply(np.zeros((0, 4)), np.zeros((0, 6)), [], [1], [0], [0], np.ones(4), np.ones(6), 2.0)
     assert y.shape == (0, 6)
+
+
+def _slice_case(seed):
+    g = np.random.default_rng(seed)
+    T, n, d_in = 23, 5, 16
+    widths = [24, 8, 16]
+    slices, y_off = [], 0
+    for d_out in widths:
+        ranks = g.integers(0, 5, size=n)
+        offA = np.concatenate([[0], np.cumsum(ranks * d_in)])
+        offB = np.concatenate([[0], np.cumsum(ranks * d_out)])
+        slices.append((d_out, y_off, ranks, offA[:-1], offB[:-1], g.standard_normal(int(offA[-1])),
+                       g.standard_normal(int(offB[-1]))))
+        y_off += d_out + 8            # gaps between slices stay untouched
+    ids = g.integers(-1, n, size=T)
+    x = g.standard_normal((T, d_in))
+    y0 = g.standard_normal((T, y_off))
+    return ids, x, y0, slices
+
+
+@pytest.mark.parametrize("seed", [0, 1])
+def test_slices_equal_per_projection_apply(seed):
+    # each slice is one projection's side path: the multi-slice definition must equal
+    # lora_apply on every slice's columns and leave the gaps between slices alone
+    ids, x, y0, slices = _slice_case(seed)
+    y = AP.lora_apply_slices(x, y0, ids, slices, 1.5)
+    covered = np.zeros(y0.shape[1], dtype=bool)
+    for d_out, y_off, ranks, offA, offB, Ap, Bt in slices:
+        want = AP.lora_apply(x, y0[:, y_off:y_off + d_out], ids, ranks, offA, offB, Ap, Bt, 1.5)
+        np.testing.assert_allclose(y[:, y_off:y_off + d_out], want, rtol=1e-13, atol=1e-13)
+        covered[y_off:y_off + d_out] = True
+    assert np.array_equal(y[:, ~covered], y0[:, ~covered])
+
+
+def test_slices_per_adapter_scale():
+    # a per-adapter scale scales each token's delta by its own adapter's value only
+    ids, x, y0, slices = _slice_case(3)
+    n = len(slices[0][2])
+    sc = np.arange(1, n + 1, dtype=np.float64)
+    y = AP.lora_apply_slices(x, y0, ids, slices, 0.0, adapter_scale=sc)
+    for a in range(n):
+        one = AP.lora_apply_slices(x, y0, np.where(ids == a, a, -1), slices, 1.0)
+        rows = ids == a
+        np.testing.assert_allclose(y[rows] - y0[rows], sc[a] * (one[rows] - y0[rows]), rtol=1e-12, atol=1e-12)
+    assert np.array_equal(y[ids < 0], y0[ids < 0])
