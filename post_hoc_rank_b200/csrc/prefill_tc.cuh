@@ -86,24 +86,24 @@ __global__ void __launch_bounds__(kTcThreads) shrink_tc_kernel(ApplyArgs a) {
     const int kbeg = split * slen;
     if (kbeg >= a.d_in) return;   // uniform: this split has no columns
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    if (tid == 0) {   // rows of every slice in the concatenated B operand
-        int kc = 0;
-        for (int q = 0; q < a.n_slices; ++q) {
-            int k;
-            int64_t oa, ob;
-            slice_factors(a, q, it.adapter, split == 0, k, oa, ob);
-            s.kcum[q] = kc;
-            s.oa[q] = oa;
-            kc += k;
-        }
-        s.kcum[a.n_slices] = kc;
+    const int nt = it.ntok;
+    if (tid < a.n_slices) {   // each slice's rank and A' offset, looked up in parallel
+        int k;
+        int64_t oa, ob;
+        slice_factors(a, tid, it.adapter, split == 0, k, oa, ob);
+        s.kcum[tid + 1] = k;
+        s.oa[tid] = oa;
+    }
+    for (int m = tid; m < kTcM; m += kTcThreads) s.toks[m] = m < nt ? a.perm[it.tok0 + m] : 0;
+    __syncthreads();
+    if (tid == 0) {   // prefix sums: B rows of slice q are kcum[q] .. kcum[q+1]-1
+        s.kcum[0] = 0;
+        for (int q = 1; q <= a.n_slices; ++q) s.kcum[q] += s.kcum[q - 1];
     }
     __syncthreads();
     const int ktot = s.kcum[a.n_slices];
     if (ktot <= 0) return;   // uniform
-    const int nt = it.ntok;
     const int npad = (ktot + 15) & ~15;
-    for (int m = tid; m < kTcM; m += kTcThreads) s.toks[m] = m < nt ? a.perm[it.tok0 + m] : 0;
     // rows ktot..npad-1 of every B stage stay zero (never written by the copies)
     for (int e = tid; e < kTcStages * (npad - ktot) * kTcKB; e += kTcThreads) {
         const int st = e / ((npad - ktot) * kTcKB), r2 = e % ((npad - ktot) * kTcKB);
@@ -129,6 +129,7 @@ __global__ void __launch_bounds__(kTcThreads) shrink_tc_kernel(ApplyArgs a) {
 
     const int pidx = warp == 0 ? 0 : warp - 1;   // producer index (warps 0, 2, 3)
     if (warp != 1 && pidx < kTcProducers) {   // producers
+        const __nv_bfloat16* A0 = a.sl[0].A_pool + s.oa[0];   // the only slice when MAXN == 64
         for (int kb = 0; kb < nK && ok; ++kb) {
             const int st = kb % kTcStages;
             if (kb >= kTcStages) ok = mbar_wait(&s.empty[st], (uint32_t)((kb / kTcStages - 1) & 1));
@@ -154,8 +155,9 @@ __global__ void __launch_bounds__(kTcThreads) shrink_tc_kernel(ApplyArgs a) {
                 const int kk = k0 + kc * 8;
                 if (n < ktot) {
                     int q = 0;
-                    while (q + 1 < a.n_slices && n >= s.kcum[q + 1]) ++q;
-                    const __nv_bfloat16* Ap = a.sl[q].A_pool + s.oa[q];
+                    if (MAXN > kMaxRank)
+                        while (q + 1 < a.n_slices && n >= s.kcum[q + 1]) ++q;
+                    const __nv_bfloat16* Ap = (MAXN > kMaxRank ? a.sl[q].A_pool + s.oa[q] : A0);
                     const bool v = kk < kend;
                     cp_async16_zfill(bbase + kmaj64(n, kc * 8),
                                      v ? Ap + (int64_t)(n - s.kcum[q]) * a.d_in + kk : Ap, v);
@@ -207,8 +209,12 @@ __global__ void __launch_bounds__(kTcThreads) shrink_tc_kernel(ApplyArgs a) {
                 for (int i = 0; i < 16; ++i) {
                     const int c = c0 + i;
                     if (c < ktot) {
-                        while (q + 1 < a.n_slices && c >= s.kcum[q + 1]) ++q;
-                        trow[a.sl[q].t_col + c - s.kcum[q]] = v[i];
+                        if (MAXN > kMaxRank) {
+                            while (q + 1 < a.n_slices && c >= s.kcum[q + 1]) ++q;
+                            trow[a.sl[q].t_col + c - s.kcum[q]] = v[i];
+                        } else {
+                            trow[c] = v[i];   // one slice, t columns 0 .. k-1
+                        }
                     }
                 }
             }
