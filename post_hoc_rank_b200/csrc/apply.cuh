@@ -297,118 +297,127 @@ __device__ __forceinline__ void y_update8(__nv_bfloat16* yp, const float (&acc)[
 
 constexpr int kShrinkJ = 4;   // rows of A' per pass
 
-// Shrink: t[item][q][j] = A'_a[j] . x[tok_q] (fp32); grid (work items, slices).  The
-// d_in range is split across all warps so each warp keeps many 16-byte loads in
-// flight; partial sums are reduced through shared memory in a fixed order.
+// Shrink: t[item][q][j] = A'_a[j] . x[tok_q] (fp32) for every (work item, slice); a
+// bounded grid strides over the items the routing produced.  The d_in range is
+// split across all warps so each warp keeps many 16-byte loads in flight; partial
+// sums are reduced through shared memory in a fixed order.
 __global__ void __launch_bounds__(kGemvThreads) shrink_kernel(ApplyArgs a) {
     __shared__ float part[kGemvThreads / 32][kShrinkJ][kGemvTok];
     __shared__ int32_t toks[kGemvTok];
-    GemvItem item;
-    if (!item_ok(a, blockIdx.x, item)) return;
-    const int sl = blockIdx.y;
-    int k;
-    int64_t oa, ob;
-    if (!slice_factors(a, sl, item.adapter, true, k, oa, ob)) return;
-    const int nt = item.ntok;
+    const int n_units = a.counts[2] * a.n_slices;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    if (tid < nt) toks[tid] = a.items[blockIdx.x].tok[tid];
-    __syncthreads();
-    const __nv_bfloat16* Ap = a.sl[sl].A_pool + oa;
-    float* tout = a.t_buf + (size_t)item.tok0 * a.ldt + a.sl[sl].t_col;
-    for (int j0 = 0; j0 < k; j0 += kShrinkJ) {
-        float acc[kShrinkJ][kGemvTok];
+    for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
+        const int itx = u / a.n_slices, sl = u - itx * a.n_slices;
+        const GemvItem& item = a.items[itx];
+        int k;
+        int64_t oa, ob;
+        if (!slice_factors(a, sl, item.adapter, true, k, oa, ob)) continue;   // uniform
+        const int nt = item.ntok;
+        if (tid < nt) toks[tid] = item.tok[tid];
+        __syncthreads();
+        const __nv_bfloat16* Ap = a.sl[sl].A_pool + oa;
+        float* tout = a.t_buf + (size_t)item.tok0 * a.ldt + a.sl[sl].t_col;
+        for (int j0 = 0; j0 < k; j0 += kShrinkJ) {
+            float acc[kShrinkJ][kGemvTok];
 #pragma unroll
-        for (int jj = 0; jj < kShrinkJ; ++jj)
+            for (int jj = 0; jj < kShrinkJ; ++jj)
 #pragma unroll
-            for (int q = 0; q < kGemvTok; ++q) acc[jj][q] = 0.f;
-        for (int d0 = tid * 8; d0 < a.d_in; d0 += kGemvThreads * 8) {
-            float xf[kGemvTok][8];
+                for (int q = 0; q < kGemvTok; ++q) acc[jj][q] = 0.f;
+            for (int d0 = tid * 8; d0 < a.d_in; d0 += kGemvThreads * 8) {
+                float xf[kGemvTok][8];
 #pragma unroll
-            for (int q = 0; q < kGemvTok; ++q)
-                if (q < nt) bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(a.x + (int64_t)toks[q] * a.d_in + d0)), xf[q]);
+                for (int q = 0; q < kGemvTok; ++q)
+                    if (q < nt)
+                        bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(a.x + (int64_t)toks[q] * a.d_in + d0)), xf[q]);
 #pragma unroll
-            for (int jj = 0; jj < kShrinkJ; ++jj) {
-                if (j0 + jj < k) {
-                    float af[8];
-                    bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(Ap + (int64_t)(j0 + jj) * a.d_in + d0)), af);
+                for (int jj = 0; jj < kShrinkJ; ++jj) {
+                    if (j0 + jj < k) {
+                        float af[8];
+                        bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(Ap + (int64_t)(j0 + jj) * a.d_in + d0)), af);
 #pragma unroll
-                    for (int q = 0; q < kGemvTok; ++q) {
-                        if (q < nt) {
+                        for (int q = 0; q < kGemvTok; ++q) {
+                            if (q < nt) {
 #pragma unroll
-                            for (int e = 0; e < 8; ++e) acc[jj][q] = fmaf(af[e], xf[q][e], acc[jj][q]);
+                                for (int e = 0; e < 8; ++e) acc[jj][q] = fmaf(af[e], xf[q][e], acc[jj][q]);
+                            }
                         }
                     }
                 }
             }
-        }
-        const int nj = min(kShrinkJ, k - j0);   // block-uniform bounds: reduce live slots only
+            const int nj = min(kShrinkJ, k - j0);   // block-uniform bounds: reduce live slots only
 #pragma unroll
-        for (int jj = 0; jj < kShrinkJ; ++jj)
+            for (int jj = 0; jj < kShrinkJ; ++jj)
 #pragma unroll
-            for (int q = 0; q < kGemvTok; ++q) {
-                if (jj < nj && q < nt) {
-                    const float v = warp_sum(acc[jj][q]);
-                    if (lane == 0) part[warp][jj][q] = v;
+                for (int q = 0; q < kGemvTok; ++q) {
+                    if (jj < nj && q < nt) {
+                        const float v = warp_sum(acc[jj][q]);
+                        if (lane == 0) part[warp][jj][q] = v;
+                    }
                 }
-            }
-        __syncthreads();
-        if (tid < kShrinkJ * kGemvTok) {
-            const int jj = tid / kGemvTok, q = tid % kGemvTok;
-            float v = 0.f;
+            __syncthreads();
+            if (tid < kShrinkJ * kGemvTok) {
+                const int jj = tid / kGemvTok, q = tid % kGemvTok;
+                float v = 0.f;
 #pragma unroll
-            for (int w = 0; w < kGemvThreads / 32; ++w) v += part[w][jj][q];
-            if (j0 + jj < k && q < nt) tout[q * a.ldt + j0 + jj] = v;
+                for (int w = 0; w < kGemvThreads / 32; ++w) v += part[w][jj][q];
+                if (j0 + jj < k && q < nt) tout[q * a.ldt + j0 + jj] = v;
+            }
+            __syncthreads();
         }
-        __syncthreads();
     }
 }
 
-// Expand: y[tok_q][e..e+7] = bf16(y + s * sum_j t[q][j] B'^T[j][e..e+7]); grid (work
-// items, column chunks of kGemvCols over all slices).
+// Expand: y[tok_q][e..e+7] = bf16(y + s * sum_j t[q][j] B'^T[j][e..e+7]) for every
+// (work item, column chunk of kGemvCols over all slices); bounded grid, strided.
 __global__ void __launch_bounds__(kGemvThreads) expand_kernel(ApplyArgs a) {
     __shared__ float tsm[kGemvTok][kMaxRank];
     __shared__ int32_t toks[kGemvTok];
-    GemvItem item;
-    if (!item_ok(a, blockIdx.x, item)) return;
-    const int sl = slice_of_chunk(a, blockIdx.y);
-    const SliceTab& S = a.sl[sl];
-    int k;
-    int64_t oa, ob;
-    if (!slice_factors(a, sl, item.adapter, false, k, oa, ob)) return;   // reported by the shrink
-    const int nt = item.ntok;
+    const int n_units = a.counts[2] * a.n_chunks;
     const int tid = threadIdx.x;
-    if (tid < nt) toks[tid] = a.items[blockIdx.x].tok[tid];
-    const float* tin = a.t_buf + (size_t)item.tok0 * a.ldt + S.t_col;
-    for (int e = tid; e < nt * kMaxRank; e += kGemvThreads) {
-        const int q = e / kMaxRank, j = e % kMaxRank;
-        tsm[q][j] = j < k ? tin[q * a.ldt + j] : 0.f;
-    }
-    __syncthreads();
-    const int e = ((int)blockIdx.y - S.chunk0) * kGemvCols + tid * 8;
-    if (e >= S.d_out) return;
-    float acc[kGemvTok][8];
-#pragma unroll
-    for (int q = 0; q < kGemvTok; ++q)
-#pragma unroll
-        for (int c = 0; c < 8; ++c) acc[q][c] = 0.f;
-    const __nv_bfloat16* Bt = S.Bt_pool + ob + e;
-#pragma unroll 4
-    for (int j = 0; j < k; ++j) {
-        float bf[8];
-        bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(Bt + (int64_t)j * S.d_out)), bf);
-#pragma unroll
-        for (int q = 0; q < kGemvTok; ++q) {
-            if (q < nt) {
-                const float tv = tsm[q][j];
-#pragma unroll
-                for (int c = 0; c < 8; ++c) acc[q][c] = fmaf(tv, bf[c], acc[q][c]);
-            }
+    for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
+        const int itx = u / a.n_chunks, chunk = u - itx * a.n_chunks;
+        const GemvItem& item = a.items[itx];
+        const int sl = slice_of_chunk(a, chunk);
+        const SliceTab& S = a.sl[sl];
+        int k;
+        int64_t oa, ob;
+        if (!slice_factors(a, sl, item.adapter, false, k, oa, ob)) continue;   // reported by the shrink; uniform
+        const int nt = item.ntok;
+        if (tid < nt) toks[tid] = item.tok[tid];
+        const float* tin = a.t_buf + (size_t)item.tok0 * a.ldt + S.t_col;
+        for (int e = tid; e < nt * kMaxRank; e += kGemvThreads) {
+            const int q = e / kMaxRank, j = e % kMaxRank;
+            tsm[q][j] = j < k ? tin[q * a.ldt + j] : 0.f;
         }
-    }
-    const float scale = adapter_scale(a, item.adapter);
+        __syncthreads();
+        const int e = (chunk - S.chunk0) * kGemvCols + tid * 8;
+        if (e < S.d_out) {
+            float acc[kGemvTok][8];
 #pragma unroll
-    for (int q = 0; q < kGemvTok; ++q)
-        if (q < nt) y_update8(a.y + (int64_t)toks[q] * a.y_ld + S.y_off + e, acc[q], scale);
+            for (int q = 0; q < kGemvTok; ++q)
+#pragma unroll
+                for (int c = 0; c < 8; ++c) acc[q][c] = 0.f;
+            const __nv_bfloat16* Bt = S.Bt_pool + ob + e;
+#pragma unroll 4
+            for (int j = 0; j < k; ++j) {
+                float bf[8];
+                bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(Bt + (int64_t)j * S.d_out)), bf);
+#pragma unroll
+                for (int q = 0; q < kGemvTok; ++q) {
+                    if (q < nt) {
+                        const float tv = tsm[q][j];
+#pragma unroll
+                        for (int c = 0; c < 8; ++c) acc[q][c] = fmaf(tv, bf[c], acc[q][c]);
+                    }
+                }
+            }
+            const float scale = adapter_scale(a, item.adapter);
+#pragma unroll
+            for (int q = 0; q < kGemvTok; ++q)
+                if (q < nt) y_update8(a.y + (int64_t)toks[q] * a.y_ld + S.y_off + e, acc[q], scale);
+        }
+        __syncthreads();   // tsm / toks are rewritten by the next unit
+    }
 }
 
 

@@ -363,6 +363,12 @@ static size_t carve_apply(void* base, int64_t T, int64_t n, int ns, ApplyWs* w) 
     return c.off + 256;
 }
 
+// Bounded grid of the grid-stride GEMV kernels: enough CTAs to fill the GPU (8 per
+// SM of 148), never more than the largest possible number of work units.
+static unsigned gemv_grid(int64_t max_units) {
+    return (unsigned)std::max<int64_t>(1, std::min<int64_t>(max_units, 8 * 148));
+}
+
 // Grid column chunks of width W over the slices (expand launches).
 static void set_chunks(ApplyArgs& a, int W) {
     int c = 0;
@@ -457,9 +463,9 @@ static lf_status apply_impl(int32_t T, int32_t d_in, const void* x, void* y, int
     // segments under kTcMin tokens: GEMV shrink (per slice), then expand
     const unsigned max_items = (unsigned)(T / kGemvTok + mseg + 1);
     set_chunks(A, kGemvCols);
-    LF_LAUNCH("shrink_gemv", shrink_kernel, dim3(max_items, (unsigned)ns), kGemvThreads, 0, s, A);
+    LF_LAUNCH("shrink_gemv", shrink_kernel, gemv_grid((int64_t)max_items * ns), kGemvThreads, 0, s, A);
     LF_CUDA_TRY(cudaGetLastError());
-    LF_LAUNCH("expand_gemv", expand_kernel, dim3(max_items, (unsigned)A.n_chunks), kGemvThreads, 0, s, A);
+    LF_LAUNCH("expand_gemv", expand_kernel, gemv_grid((int64_t)max_items * A.n_chunks), kGemvThreads, 0, s, A);
     LF_CUDA_TRY(cudaGetLastError());
     // segments with >= kTcMin tokens: one tcgen05 shrink over all slices, then expand
     const unsigned max_tc = (unsigned)(T / kTcM + mseg + 1);
@@ -937,9 +943,9 @@ lf_status lf_lora_shrink_expand_noalloc(int32_t T, int32_t d_in, int32_t d_out, 
         // decode regime (few tokens per adapter): shrink and expand in one launch
         LF_LAUNCH("fused_gemv", fused_gemv_kernel, grid2, kGemvThreads, 0, s, A);
     } else {
-        LF_LAUNCH("shrink_gemv", shrink_kernel, dim3(max_items, 1u), kGemvThreads, 0, s, A);
+        LF_LAUNCH("shrink_gemv", shrink_kernel, gemv_grid(max_items), kGemvThreads, 0, s, A);
         LF_CUDA_TRY(cudaGetLastError());
-        LF_LAUNCH("expand_gemv", expand_kernel, grid2, kGemvThreads, 0, s, A);
+        LF_LAUNCH("expand_gemv", expand_kernel, gemv_grid((int64_t)max_items * A.n_chunks), kGemvThreads, 0, s, A);
     }
     return launch_status();
 }
