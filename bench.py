@@ -325,11 +325,12 @@ def apply_bytes(T, d_in, d_out, ranks_used):
     return 2 * T * d_in + 4 * T * d_out + 4 * T + sum(2 * k * (d_in + d_out) for k in ranks_used)
 
 
-def decode_bench(args, dev, stream, hbm, variant="ragged"):
+def decode_bench(args, dev, stream, hbm, variant="ragged", fused=False):
     """Config 3: Llama-3-8B shapes, 32 layers x 7 projections, T=256, 128 adapters.
     variant: "ragged" (retained ranks as allocated), "padded" (every adapter's factors
     of a projection zero-padded to the largest retained rank over the 128 resident
-    adapters), "r64" (uncompressed rank-64 adapters)."""
+    adapters), "r64" (uncompressed rank-64 adapters).  fused: q/k/v and gate/up as
+    one multi-slice call each (4 calls per layer instead of 7)."""
     import torch
     from post_hoc_rank_b200 import api, synth
     from post_hoc_rank_b200 import loraforge as lf
@@ -350,6 +351,7 @@ def decode_bench(args, dev, stream, hbm, variant="ragged"):
     for l in range(M.layers):
         x_h = synth.normal_bf16((T, M.hidden), (3, 1, l), device=dev)
         x_f = synth.normal_bf16((T, M.ffn), (3, 2, l), device=dev)
+        groups = []
         for p, (_, d_out, d_in) in enumerate(shapes):
             rk_true = ranks_all[:, p, l].astype(np.int64)
             if variant == "ragged":
@@ -366,26 +368,27 @@ def decode_bench(args, dev, stream, hbm, variant="ragged"):
                 pad = torch.from_numpy(np.arange(kmax)[None, :] >= rk_true[:, None]).to(dev)
                 Ap.view(n_ad, kmax, d_in)[pad] = 0
                 Bt.view(n_ad, kmax, d_out)[pad] = 0
-            y = synth.normal_bf16((T, d_out), (3, 5, l, p), device=dev)
-            x = x_f if d_in == M.ffn else x_h
-            ws = api.workspace(lf.lf_apply_workspace_size(T, n_ad), dev)
-            calls.append((x, y, torch.from_numpy(rk.astype(np.int32)).to(dev),
-                          torch.from_numpy(offA[:-1]).to(dev), torch.from_numpy(offB[:-1]).to(dev), Ap, Bt, ws))
+            groups.append((d_in, d_out, rk, offA, offB, Ap, Bt))
             total_bytes += apply_bytes(T, d_in, d_out, [int(rk[a]) for a in distinct])
+        lc, sets = _layer_calls(groups, lambda d: x_f if d == M.ffn else x_h, ids_d, n_ad, T, dev, (3, 5, l), fused)
+        calls += lc
+        if fused:   # x is read once per call, not once per projection
+            total_bytes -= sum(2 * T * groups[ps[0]][0] * (len(ps) - 1) for ps in sets)
     names = {"ragged": "S 1/12 floor 1 ranks (ragged)",
              "padded": "S 1/12 floor 1 ranks zero-padded to the per-projection max over resident adapters",
              "r64": "uncompressed rank-64 adapters"}
     out = _apply_run(args, calls, ids_d, n_ad, T, total_bytes, stream, hbm, dict(
         workload="decode: Llama-3-8B, 32 layers x 7 projections, 256 tokens, 128 adapters Zipf(1), "
-                 + names[variant], distinct_adapters=len(distinct),
-        mean_rank=float(ranks_all.mean())))
+                 + names[variant] + ("; q/k/v and gate/up as one slice call each" if fused else ""),
+        distinct_adapters=len(distinct), mean_rank=float(ranks_all.mean())))
     del calls
     torch.cuda.empty_cache()
     return out
 
 
-def prefill_bench(args, dev, stream, hbm, k):
-    """Config 4: Qwen2.5-7B layer, 7 projections, 32 requests x 512 tokens, request i -> adapter i."""
+def prefill_bench(args, dev, stream, hbm, k, fused=False):
+    """Config 4: Qwen2.5-7B layer, 7 projections, 32 requests x 512 tokens, request i -> adapter i.
+    fused: q/k/v and gate/up as one multi-slice call each."""
     import torch
     from post_hoc_rank_b200 import api, synth
     from post_hoc_rank_b200 import loraforge as lf
@@ -396,20 +399,71 @@ def prefill_bench(args, dev, stream, hbm, k):
     ids_d = torch.from_numpy(ids).to(dev)
     x_h = synth.normal_bf16((T, M.hidden), (4, 1), device=dev)
     x_f = synth.normal_bf16((T, M.ffn), (4, 2), device=dev)
-    calls, total_bytes = [], 0
+    groups, total_bytes = [], 0
     for p, (_, d_out, d_in) in enumerate(M.proj_shapes()):
         rk = np.full(n_ad, k, dtype=np.int64)
         offA = np.concatenate([[0], np.cumsum(rk * d_in)]); offB = np.concatenate([[0], np.cumsum(rk * d_out)])
         Ap = synth.normal_bf16((int(offA[-1]),), (4, 3, p, k), std=d_in ** -0.5, device=dev)
         Bt = synth.normal_bf16((int(offB[-1]),), (4, 4, p, k), std=d_out ** -0.5, device=dev)
-        y = synth.normal_bf16((T, d_out), (4, 5, p), device=dev)
-        x = x_f if d_in == M.ffn else x_h
-        ws = api.workspace(lf.lf_apply_workspace_size(T, n_ad), dev)
-        calls.append((x, y, torch.from_numpy(rk.astype(np.int32)).to(dev), torch.from_numpy(offA[:-1]).to(dev),
-                      torch.from_numpy(offB[:-1]).to(dev), Ap, Bt, ws))
+        groups.append((d_in, d_out, rk, offA, offB, Ap, Bt))
         total_bytes += apply_bytes(T, d_in, d_out, [k] * n_ad)
+    calls, sets = _layer_calls(groups, lambda d: x_f if d == M.ffn else x_h, ids_d, n_ad, T, dev, (4, 5), fused)
+    if fused:
+        total_bytes -= sum(2 * T * groups[ps[0]][0] * (len(ps) - 1) for ps in sets)
     return _apply_run(args, calls, ids_d, n_ad, T, total_bytes, stream, hbm, dict(
-        workload=f"prefill: Qwen2.5-7B layer x 7 projections, 32 requests x 512 tokens, k={k}"))
+        workload=f"prefill: Qwen2.5-7B layer x 7 projections, 32 requests x 512 tokens, k={k}"
+                 + ("; q/k/v and gate/up as one slice call each" if fused else "")))
+
+
+def _proj_call(x, y, ids_d, n_ad, rk, oa, ob, Ap, Bt, ws, scale=2.0):
+    """One projection through lf_lora_shrink_expand."""
+    from post_hoc_rank_b200 import loraforge as lf
+
+    def run(st=None):
+        lf.lf_lora_shrink_expand(x, y, ids_d, n_ad, rk, oa, ob, Ap, Bt, scale, ws, stream=st)
+    return run
+
+
+def _slices_call(x, y, ids_d, n_ad, slices, ws, scale=2.0):
+    """Projections sharing x through one lf_lora_shrink_expand_slices call; slices:
+    (d_out, y_offset, ranks, off_A, off_Bt, A_pool, Bt_pool) device tensors."""
+    from post_hoc_rank_b200 import loraforge as lf
+    sl = [lf.make_slice(*t) for t in slices]
+
+    def run(st=None, _keep=slices):
+        lf.lf_lora_shrink_expand_slices(x, y, ids_d, n_ad, sl, scale, ws, stream=st)
+    return run
+
+
+def _layer_calls(groups, x_of, ids_d, n_ad, T, dev, key, fused):
+    """Calls of one layer.  groups: per projection (d_in, d_out, rk int64 array, offA,
+    offB, Ap, Bt); fused: q/k/v and gate/up (projections reading the same x) go as
+    one slice call each.  Returns (callables, algorithmic bytes given the adapters used)."""
+    import torch
+    from post_hoc_rank_b200 import api, synth
+    from post_hoc_rank_b200 import loraforge as lf
+    sets = [[0, 1, 2], [3], [4, 5], [6]] if fused else [[p] for p in range(len(groups))]
+    calls = []
+    for gi, ps in enumerate(sets):
+        d_in = groups[ps[0]][0]
+        x = x_of(d_in)
+        widths = [groups[p][1] for p in ps]
+        y = synth.normal_bf16((T, sum(widths)), key + (gi,), device=dev)
+        tens = []
+        y_off = 0
+        for p in ps:
+            _, d_out, rk, offA, offB, Ap, Bt = groups[p]
+            tens.append((d_out, y_off, torch.from_numpy(rk.astype(np.int32)).to(dev),
+                         torch.from_numpy(offA[:-1]).to(dev), torch.from_numpy(offB[:-1]).to(dev), Ap, Bt))
+            y_off += d_out
+        if len(ps) == 1:
+            ws = api.workspace(lf.lf_apply_workspace_size(T, n_ad), dev)
+            d_out, _, rk_d, oa_d, ob_d, Ap, Bt = tens[0]
+            calls.append(_proj_call(x, y, ids_d, n_ad, rk_d, oa_d, ob_d, Ap, Bt, ws))
+        else:
+            ws = api.workspace(lf.lf_apply_slices_workspace_size(T, n_ad, len(ps)), dev)
+            calls.append(_slices_call(x, y, ids_d, n_ad, tens, ws))
+    return calls, sets
 
 
 def _apply_run(args, calls, ids_d, n_ad, T, total_bytes, stream, hbm, meta):
@@ -418,8 +472,8 @@ def _apply_run(args, calls, ids_d, n_ad, T, total_bytes, stream, hbm, meta):
 
     def step(st=None):
         # st=None: torch's current stream (the capture stream inside torch.cuda.graph)
-        for (x, y, rk, oa, ob, Ap, Bt, ws) in calls:
-            lf.lf_lora_shrink_expand(x, y, ids_d, n_ad, rk, oa, ob, Ap, Bt, 2.0, ws, stream=st)
+        for c in calls:
+            c(st)
 
     for _ in range(max(args.warmup, 3)):
         step(stream)
@@ -556,8 +610,8 @@ def large_fleet_bench(args, dev, stream, hbm):
                     oa_d[ref] = np.arange(len(ref)) * kmax * d_in; ob_d[ref] = np.arange(len(ref)) * kmax * d_out
                     k_used = np.full(len(ref), kmax)
                 ws = api.workspace(lf.lf_apply_workspace_size(T, n_total), dev)
-                calls.append((x, y, torch.from_numpy(rk_d.astype(np.int32)).to(dev), torch.from_numpy(oa_d).to(dev),
-                              torch.from_numpy(ob_d).to(dev), pa, pb, ws))
+                calls.append(_proj_call(x, y, ids_d, n_total, torch.from_numpy(rk_d.astype(np.int32)).to(dev),
+                                        torch.from_numpy(oa_d).to(dev), torch.from_numpy(ob_d).to(dev), pa, pb, ws))
                 total_bytes += apply_bytes(T, d_in, d_out, [int(k) for k in k_used])
         r = _apply_run(args, calls, ids_d, n_total, T, total_bytes, stream, hbm, {})
         out[variant] = {k: r[k] for k in ("tokens_per_s", "ms_per_step", "algo_bytes", "achieved_gbs", "hbm_frac",
@@ -761,7 +815,9 @@ def main():
         lora = {"decode": decode_bench(args, dev, stream, hbm),
                 "decode_padded_to_max": decode_bench(args, dev, stream, hbm, "padded"),
                 "decode_uncompressed_r64": decode_bench(args, dev, stream, hbm, "r64"),
+                "decode_fused_slices": decode_bench(args, dev, stream, hbm, fused=True),
                 "prefill_k16": prefill_bench(args, dev, stream, hbm, 16),
+                "prefill_k16_fused_slices": prefill_bench(args, dev, stream, hbm, 16, fused=True),
                 "prefill_r64": prefill_bench(args, dev, stream, hbm, 64)}
         if rank == 0 and not args.no_cpu:
             lora["decode"]["cpu_baseline"] = cpu_apply_baseline()
