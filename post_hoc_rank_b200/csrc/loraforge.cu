@@ -189,7 +189,9 @@ template <typename T, int RT>
 static cudaError_t launch_tsqr(const TsqrArgs<T>& a, int n_items, cudaStream_t st) {
     auto k = tsqr_kernel<T, RT>;
     constexpr int W = tsqr_warps<T>();
-    const int grid = (n_items + W - 1) / W;
+    // the kernel strides over the device-side item count: a bounded grid (16 CTAs per
+    // SM for fp32, 8 for fp64) covers any number of items
+    const int grid = std::min((n_items + W - 1) / W, 148 * (sizeof(T) == 4 ? 16 : 8));
     if (grid > 0) LF_LAUNCH(sizeof(T) == 8 ? "tsqr_fp64_refine" : "tsqr_householder", k, grid, 32 * W, 0, st, a);
     return cudaGetLastError();
 }

@@ -178,16 +178,7 @@ __device__ __forceinline__ void load_tri_rows(T (&x)[Cols<RT>::NS][kTsqrTM], con
 }
 
 template <typename T, int RT>
-__global__ void __launch_bounds__(32 * tsqr_warps<T>(), sizeof(T) == 4 ? 16 : 1) tsqr_kernel(TsqrArgs<T> a) {
-    constexpr int W = tsqr_warps<T>();
-    __shared__ T s_R[W][tri_size<RT>()];
-    __shared__ __align__(16) T s_v[W][kTsqrTM];
-    __shared__ int s_last[W];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int wi = blockIdx.x * W + warp;
-    if (wi >= *a.n_work) return;   // warp-uniform; no block-level barriers below
-    T* Rp = s_R[warp];
-    T* vbuf = s_v[warp];
+__device__ __forceinline__ void tsqr_item(const TsqrArgs<T>& a, int wi, T* Rp, T* vbuf, int* s_last, int lane) {
     const TsqrWork w = a.work[wi];
     if (a.only && a.only[w.mf] == 0) return;   // warp-uniform
     const int local = w.mf >> 1, factor = w.mf & 1;
@@ -215,9 +206,9 @@ __global__ void __launch_bounds__(32 * tsqr_warps<T>(), sizeof(T) == 4 ? 16 : 1)
         }
         __threadfence();
         __syncwarp();
-        if (lane == 0) s_last[warp] = (atomicAdd(&a.counters[w.mf], 1) == inf.nchunks - 1);
+        if (lane == 0) *s_last = (atomicAdd(&a.counters[w.mf], 1) == inf.nchunks - 1);
         __syncwarp();
-        if (!s_last[warp]) return;
+        if (!*s_last) return;
         __threadfence();
         // fold the chunk triangles in chunk order: R = R_0, then R <- R([R; R_c])
         const T* P0 = a.partial + (size_t)inf.slot0 * RT * RT;
@@ -243,6 +234,21 @@ __global__ void __launch_bounds__(32 * tsqr_warps<T>(), sizeof(T) == 4 ? 16 : 1)
             if (Rp[tri_off<RT>(j, j)] < T(0)) v = -v;
         }
         out[e] = v;
+    }
+}
+
+// One warp per work item; a bounded grid strides over the device-side item count
+// (warps are independent: no block-level barriers).
+template <typename T, int RT>
+__global__ void __launch_bounds__(32 * tsqr_warps<T>(), sizeof(T) == 4 ? 16 : 1) tsqr_kernel(TsqrArgs<T> a) {
+    constexpr int W = tsqr_warps<T>();
+    __shared__ T s_R[W][tri_size<RT>()];
+    __shared__ __align__(16) T s_v[W][kTsqrTM];
+    __shared__ int s_last[W];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int wi = blockIdx.x * W + warp; wi < *a.n_work; wi += gridDim.x * W) {
+        tsqr_item<T, RT>(a, wi, s_R[warp], s_v[warp], &s_last[warp], lane);
+        __syncwarp();
     }
 }
 
