@@ -69,13 +69,18 @@ typedef struct {
     int64_t B_off, A_off;
 } lf_module;
 
-/* Allocation policy.  kind 0 = LoRAForge-U, kind 1 = LoRAForge-S.
+/* Allocation policy.  kind 0 = LoRAForge-U, kind 1 = LoRAForge-S, kind 2 =
+ * spectral budget on absolute energies (variant of S).
  * ratio = ratio_num / ratio_den (exact integers, e.g. 1/4, 1/12); floor >= 1.
  *  U: k = clamp(floor(ratio_num*r/ratio_den + 1/2), floor, r).
  *  S: per group, K = floor(ratio_num * sum r / ratio_den); every module gets
  *     `floor`; the remaining K - floor*M slots go to the largest normalised
  *     energies e_ij = sigma_ij^2 / sum_j sigma_ij^2 (j >= floor, e_ij > 0),
- *     ties to the lower module index, then lower j. */
+ *     ties to the lower module index, then lower j.
+ *  kind 2: as S with e_ij = sigma_ij^2 (the choice that minimises the group's
+ *     summed squared Frobenius error sum_i ||dW_i - B'_i A'_i||^2 under the budget).
+ * The budget scope is the module `group`: one group per adapter gives per-adapter
+ * budgets, one group over all modules a fleet-wide budget. */
 typedef struct {
     int32_t kind, ratio_num, ratio_den, floor;
 } lf_policy;

@@ -38,18 +38,23 @@ def uniform_rank(r: int, num: int, den: int, floor: int) -> int:
     return min(r, max(floor, k))
 
 
-def energies(sigma, r: int) -> np.ndarray:
-    """Normalised spectral energies e_j = sigma_j^2 / sum sigma^2 (zeros for a zero module)."""
+def energies(sigma, r: int, absolute: bool = False) -> np.ndarray:
+    """Normalised spectral energies e_j = sigma_j^2 / sum sigma^2 (zeros for a zero
+    module); with absolute=True the energies sigma_j^2 themselves."""
     s = np.asarray(sigma, dtype=np.float64)[:r]
     sq = s * s
+    if absolute:
+        return sq
     tot = math.fsum(sq.tolist())
     if tot == 0.0:
         return np.zeros(r)
     return sq / tot
 
 
-def spectral_ranks(sigma_rows, r, group, num: int, den: int, floor: int):
-    """LoRAForge-S ranks for every module.
+def spectral_ranks(sigma_rows, r, group, num: int, den: int, floor: int, absolute: bool = False):
+    """LoRAForge-S ranks for every module (absolute=True: the variant that ranks the
+    candidates by sigma_ij^2, which minimises the group's summed squared Frobenius
+    truncation error under the same budget).
 
     sigma_rows: n x r_max array, row i holds module i's singular values in
     descending order (entries past r_i ignored).
@@ -73,7 +78,7 @@ def spectral_ranks(sigma_rows, r, group, num: int, den: int, floor: int):
                 raise ValueError("floor exceeds module rank")
             if np.any(np.diff(sigma_rows[i][:ri]) > 0):
                 raise ValueError("singular values must be listed in descending order")
-            e = energies(sigma_rows[i], ri)
+            e = energies(sigma_rows[i], ri, absolute)
             for j in range(floor, ri):
                 if e[j] > 0.0:
                     cands.append((-e[j], i, j))
@@ -93,7 +98,7 @@ def spectral_ranks(sigma_rows, r, group, num: int, den: int, floor: int):
     return ranks, info
 
 
-def brute_force_ranks(sigma_rows, r, num: int, den: int, floor: int):
+def brute_force_ranks(sigma_rows, r, num: int, den: int, floor: int, absolute: bool = False):
     """Exhaustive search for one group (tiny cases only): every rank vector with
     floor <= k_i <= r_i and sum k_i <= K; returns (best objective, list of optimal
     rank tuples) for the objective sum_i sum_{j<k_i} e_ij."""
@@ -101,14 +106,15 @@ def brute_force_ranks(sigma_rows, r, num: int, den: int, floor: int):
     sigma_rows = np.asarray(sigma_rows, dtype=np.float64)
     r = [int(x) for x in r]
     K = (num * sum(r)) // den
-    E = [energies(sigma_rows[i], r[i]) for i in range(len(r))]
+    E = [energies(sigma_rows[i], r[i], absolute) for i in range(len(r))]
     best, arg = -1.0, []
     for ks in itertools.product(*[range(floor, ri + 1) for ri in r]):
         if sum(ks) > max(K, floor * len(r)):
             continue
         val = math.fsum(math.fsum(E[i][:ks[i]].tolist()) for i in range(len(r)))
-        if val > best + 1e-15:
+        tol = 1e-15 * max(abs(best), 1.0)
+        if val > best + tol:
             best, arg = val, [ks]
-        elif abs(val - best) <= 1e-15:
+        elif abs(val - best) <= tol:
             arg.append(ks)
     return best, arg

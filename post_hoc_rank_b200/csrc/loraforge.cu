@@ -95,7 +95,7 @@ static lf_status check_mods(const lf_module* mods, int32_t n) {
 }
 
 static lf_status check_policy(const lf_module* mods, int32_t n, lf_policy p) {
-    if (p.kind != 0 && p.kind != 1) return LF_ERR_INVALID_ARG;
+    if (p.kind < 0 || p.kind > 2) return LF_ERR_INVALID_ARG;
     if (p.ratio_num < 0 || p.ratio_den <= 0 || p.floor < 1) return LF_ERR_INVALID_ARG;
     for (int32_t i = 0; i < n; ++i)
         if (p.floor > mods[i].r) return LF_ERR_SHAPE;
@@ -759,7 +759,7 @@ lf_status lf_truncate_export(const lf_module* mods, int32_t n, lf_policy pol, co
     a.flag_list = nullptr;
     a.flag_count = nullptr;
 
-    if (pol.kind == 1) {
+    if (pol.kind >= 1) {   // spectral policies: refine the modules near the boundary
         int32_t* flist = reinterpret_cast<int32_t*>(base + L.flist);
         int32_t* fcount = reinterpret_cast<int32_t*>(base + L.fcount);
         LF_CUDA_TRY(cudaMemsetAsync(fcount, 0, 2 * sizeof(int32_t), s));

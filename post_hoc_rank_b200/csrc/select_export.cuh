@@ -26,7 +26,7 @@ struct SelArgs {
     const int32_t* grp_ptr;    // n_groups + 1
     const int32_t* grp_mods;   // module indices, ascending inside each group
     const double* sigma;       // n x rs
-    double* energy;            // n x rs scratch (normalised energies)
+    double* energy;            // n x rs scratch (energies: normalised, or absolute for kind 2)
     int32_t rs;
     lf_policy pol;
     int32_t* ranks;            // n
@@ -102,7 +102,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelArgs a) {
             double e = 0.0;
             if (j < r && tot > 0.0) {
                 const double sq = sg[j] * sg[j];
-                e = __ddiv_rn(sq, tot);
+                e = a.pol.kind == 2 ? sq : __ddiv_rn(sq, tot);   // kind 2: absolute energy
             }
             en[j] = e;
         }

@@ -35,8 +35,10 @@ def policy_U(num: int, den: int, floor: int = 1) -> lf_policy:
     return lf_policy(0, num, den, floor)
 
 
-def policy_S(num: int, den: int, floor: int = 1) -> lf_policy:
-    return lf_policy(1, num, den, floor)
+def policy_S(num: int, den: int, floor: int = 1, absolute: bool = False) -> lf_policy:
+    """LoRAForge-S (normalised energies), or with absolute=True the variant that ranks
+    candidates by sigma^2 (kind 2)."""
+    return lf_policy(2 if absolute else 1, num, den, floor)
 
 
 class lf_phase_time(ctypes.Structure):

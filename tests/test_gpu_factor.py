@@ -240,3 +240,29 @@ def test_rank_deficient_factors_take_householder_route():
         assert np.linalg.norm(R.T @ R - gram) <= 1e-5 * np.linalg.norm(gram), i
         s, *_ = OF.spectrum_factor(Bn, An)
         assert np.max(np.abs(S[i][:r] - s)) <= G.SIGMA_TOL * s[0], i
+
+
+@pytest.mark.parametrize("variant", ["absolute_energy", "fleet_global_budget"])
+def test_allocation_variants_ranks_bit_exact(variant):
+    # allocation variants of the spectral policy: ranking candidates by sigma^2
+    # (kind 2), and one budget over every module of the fleet (a single group)
+    shapes = [("q", 896, 896), ("k", 128, 896), ("v", 128, 896), ("o", 896, 896),
+              ("gate", 4736, 896), ("up", 4736, 896), ("down", 896, 4736)]
+    lay = synth.fleet_layout(3, shapes=shapes, r=64, n_layers=2)
+    Bh = torch.zeros(lay.B_total); Ah = torch.zeros(lay.A_total)
+    synth.fill_fleet(lay, Bh, Ah, cfg_id=13)
+    if variant == "fleet_global_budget":
+        lay.group[:] = 0
+    B, A = upload(Bh, Ah)
+    absolute = variant == "absolute_energy"
+    pol = lf.policy_S(1, 12, 1, absolute=absolute)
+    mods, F, E, st = G.run_factor_path(lay, B, A, pol)
+    assert st == 0
+    sig = G.oracle_sigma_rows(lay, Bh, Ah, range(lay.n))
+    ranks_o, info = OA.spectral_ranks(sig, lay.r, lay.group, 1, 12, 1, absolute=absolute)
+    ranks_g = E.ranks.cpu().numpy()
+    assert G.compare_ranks(ranks_g, ranks_o, info), (ranks_g, ranks_o)
+    for g in set(lay.group.tolist()):
+        assert ranks_g[lay.group == g].sum() <= (64 * int((lay.group == g).sum())) // 12
+    for eg, eo in G.recon_errors(lay, Bh, Ah, E, sig, range(lay.n)):
+        assert abs(eg - eo) <= G.RECON_TOL

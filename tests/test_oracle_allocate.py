@@ -79,3 +79,50 @@ def test_prefix_closed_with_ties():
 def test_rejects_unsorted_sigma():
     with pytest.raises(ValueError):
         AL.spectral_ranks(np.array([[1.0, 2.0, 0.5]]), [3], [0], 1, 2, 1)
+
+
+def test_absolute_energy_variant_hand_case():
+    # module 0: sigma (10, 1), module 1: sigma (1, 0.9); K = floor(3 * 4 / 4) = 3,
+    # floor 1 -> one extra slot.  Normalised energies of the second directions:
+    # 1/101 = 0.0099 vs 0.81/1.81 = 0.4475 -> module 1 gets it.  Absolute energies:
+    # 1.0 vs 0.81 -> module 0 gets it.
+    sig = np.array([[10.0, 1.0], [1.0, 0.9]])
+    rk_norm, _ = AL.spectral_ranks(sig, [2, 2], [0, 0], 3, 4, 1)
+    rk_abs, _ = AL.spectral_ranks(sig, [2, 2], [0, 0], 3, 4, 1, absolute=True)
+    assert rk_norm.tolist() == [1, 2]
+    assert rk_abs.tolist() == [2, 1]
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_absolute_energy_variant_minimises_dense_truncation_error(seed):
+    # the definition: among all rank vectors within the budget, the variant's ranks
+    # minimise sum_i ||dW_i - best rank-k_i approximation||_F^2, evaluated here from
+    # dense SVDs of dW_i = B_i A_i (no energies involved)
+    g = np.random.default_rng(seed)
+    mods = []
+    for _ in range(3):
+        B = g.standard_normal((9, 4)) * np.exp(g.standard_normal(4))
+        A = g.standard_normal((4, 7))
+        mods.append(B @ A)
+    sig = np.stack([np.linalg.svd(W, compute_uv=False)[:4] for W in mods])
+    rk, _ = AL.spectral_ranks(sig, [4] * 3, [0] * 3, 1, 2, 1, absolute=True)
+
+    def err(ks):
+        tot = 0.0
+        for W, k in zip(mods, ks):
+            U, s, Vt = np.linalg.svd(W, full_matrices=False)
+            tot += np.linalg.norm(W - (U[:, :k] * s[:k]) @ Vt[:k]) ** 2
+        return tot
+    import itertools
+    K = (1 * 12) // 2
+    best = min(err(ks) for ks in itertools.product(range(1, 5), repeat=3) if sum(ks) <= K)
+    assert err(rk) <= best * (1 + 1e-12) + 1e-12
+    assert int(rk.sum()) <= K
+
+
+def test_absolute_energy_brute_force_agrees():
+    g = np.random.default_rng(7)
+    sig = np.sort(np.exp(g.standard_normal((4, 4))), axis=1)[:, ::-1]
+    rk, _ = AL.spectral_ranks(sig, [4] * 4, [0] * 4, 1, 2, 1, absolute=True)
+    best, args = AL.brute_force_ranks(sig, [4] * 4, 1, 2, 1, absolute=True)
+    assert tuple(rk.tolist()) in [tuple(a) for a in args]
