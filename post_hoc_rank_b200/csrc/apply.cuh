@@ -422,14 +422,14 @@ __global__ void __launch_bounds__(kGemvThreads) expand_kernel(ApplyArgs a) {
 
 
 // Decode regime, token-parallel (BGMV form: every token carries its adapter index,
-// no sorting).  CTA (token, 4096-column chunk of one slice): t = A' x (k fp32 dot
+// no sorting).  CTA (token, 8192-column chunk of one slice): t = A' x (k fp32 dot
 // products over d_in, reduced across the CTA in a fixed order), then
 // y[chunk] += s * B'^T t with 16-byte loads of the k rows of B'^T.  Each chunk CTA
 // recomputes the same t (identical arithmetic; x and A' come from L2), and tokens
 // of one adapter read its factors from L2 after the first touch, so HBM sees every
 // distinct factor row, x and y once.
 constexpr int kBgmvThreads = 256;
-constexpr int kBgmvVec = 2;                                  // 8-column vectors per thread in the expand
+constexpr int kBgmvVec = 4;                                  // 8-column vectors per thread in the expand
 constexpr int kBgmvCols = kBgmvThreads * 8 * kBgmvVec;       // d_out columns per CTA
 constexpr int kBgmvJ = 8;                                    // retained directions per shrink pass
 
