@@ -220,6 +220,22 @@ lf_status lf_lora_shrink_expand_slices(int32_t T, int32_t d_in, const void* x, v
                                        float scale, const float* adapter_scale, int32_t* seg_out,
                                        void* ws, size_t ws_bytes, lf_stream_t stream);
 
+/* ---- Sigma-sandwich serving (jointly compressed adapters) ---------------------
+ * "Compress then Serve" (academ.us/article/2407.00066), sections 3.1 and 11: the
+ * adapters of one module share U (d_out x rank) and V (d_in x rank) and keep a
+ * small Sigma_a each, B_a A_a ~ U Sigma_a V^T; serving applies, for every token t
+ * with a = ids[t] >= 0,
+ *   y_t = bf16( y_t + scale * U (Sigma_a (V^T x_t)) )     (fp32 intermediates, one rounding)
+ * Vt = V^T (rank x d_in bf16), Ut = U^T (rank x d_out bf16), both shared by all
+ * adapters; sigma (device fp32): sigma_diag = 1 -> n_adapters x rank (diagonal
+ * Sigma_a), sigma_diag = 0 -> n_adapters x rank x rank row-major (full Sigma_a).
+ * Same routing, regimes, id rules and workspace as lf_lora_shrink_expand
+ * (lf_apply_workspace_size(T, n_adapters)); 1 <= rank <= 64. */
+lf_status lf_lora_sigma_sandwich(int32_t T, int32_t d_in, int32_t d_out, const void* x, void* y,
+                                 const int32_t* ids, int32_t n_adapters, int32_t rank,
+                                 const void* Vt, const void* Ut, const float* sigma, int32_t sigma_diag,
+                                 float scale, void* ws, size_t ws_bytes, lf_stream_t stream);
+
 /* ---- Shrink / expand with library-owned scratch -------------------------------
  * This entry point has no counterpart in the paper; it exists for callers that
  * cannot call cudaMalloc.  Examples: a serving loop that reserved all device memory

@@ -121,3 +121,29 @@ def lora_apply_slices(x, y0, ids, slices, scale: float, adapter_scale=None):
             Ap, Bt = adapter_factors(a, ranks, off_A, off_Bt, A_pool, Bt_pool, d_in, d_out)
             y[t, y_off:y_off + d_out] += sa * (Bt.T @ (Ap @ x[t]))
     return y
+
+
+def sigma_sandwich_apply(x, y0, ids, Vt, Ut, sigma, diagonal: bool, scale: float):
+    """Serving of jointly compressed adapters ("Compress then Serve" §3.1, §11):
+    B_a A_a ~ U Sigma_a V^T with U, V shared by all adapters and a small Sigma_a each;
+    for every token t with a = ids[t] >= 0,  y_t += scale * U (Sigma_a (V^T x_t)).
+
+    Vt = V^T (rank x d_in), Ut = U^T (rank x d_out); sigma: n_adapters x rank
+    (diagonal Sigma_a) or n_adapters x rank x rank (full).  Returns y in float64.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    y = np.array(y0, dtype=np.float64, copy=True)
+    Vt = np.asarray(Vt, dtype=np.float64); Ut = np.asarray(Ut, dtype=np.float64)
+    sig = np.asarray(sigma, dtype=np.float64)
+    ids = np.asarray(ids)
+    n = sig.shape[0]
+    if np.any(ids < -1) or np.any(ids >= n):
+        raise ValueError("adapter id out of range")
+    for t in range(x.shape[0]):
+        a = int(ids[t])
+        if a < 0:
+            continue
+        z = Vt @ x[t]                                   # V^T x
+        w = sig[a] * z if diagonal else sig[a] @ z      # Sigma_a (V^T x)
+        y[t] += scale * (Ut.T @ w)                      # U (...)
+    return y

@@ -371,6 +371,7 @@ __global__ void __launch_bounds__(kGemvThreads) shrink_kernel(ApplyArgs a) {
 // (work item, column chunk of kGemvCols over all slices); bounded grid, strided.
 __global__ void __launch_bounds__(kGemvThreads) expand_kernel(ApplyArgs a) {
     __shared__ float tsm[kGemvTok][kMaxRank];
+    __shared__ float tsw[kGemvTok][kMaxRank];
     __shared__ int32_t toks[kGemvTok];
     const int n_units = a.counts[2] * a.n_chunks;
     const int tid = threadIdx.x;
@@ -390,6 +391,16 @@ __global__ void __launch_bounds__(kGemvThreads) expand_kernel(ApplyArgs a) {
             tsm[q][j] = j < k ? tin[q * a.ldt + j] : 0.f;
         }
         __syncthreads();
+        if (a.sigma_mode) {   // Sigma-sandwich: every token's t <- Sigma_a t (one adapter per item)
+            const int q = tid / 32;   // 8 warps, one token each
+            if (q < nt) sigma_apply(a, item.adapter, k, tsm[q], tsw[q], tid & 31, 32);
+            __syncthreads();
+            for (int e = tid; e < nt * kMaxRank; e += kGemvThreads) {
+                const int q2 = e / kMaxRank, j = e % kMaxRank;
+                tsm[q2][j] = j < k ? tsw[q2][j] : 0.f;
+            }
+            __syncthreads();
+        }
         const int e = (chunk - S.chunk0) * kGemvCols + tid * 8;
         if (e < S.d_out) {
             float acc[kGemvTok][8];
@@ -436,6 +447,7 @@ constexpr int kBgmvJ = 8;                                    // retained directi
 __global__ void __launch_bounds__(kBgmvThreads, 4) bgmv_kernel(ApplyArgs a) {
     __shared__ float red[kBgmvThreads / 32][kBgmvJ];
     __shared__ float ts[kMaxRank];
+    __shared__ float tw[kMaxRank];
     const int tok = blockIdx.x;
     const int ad = a.ids[tok];
     if (ad == -1) return;
@@ -491,6 +503,12 @@ __global__ void __launch_bounds__(kBgmvThreads, 4) bgmv_kernel(ApplyArgs a) {
         }
         __syncthreads();
     }
+    const float* tv = ts;
+    if (a.sigma_mode) {   // Sigma-sandwich: t <- Sigma_a t
+        sigma_apply(a, ad, k, ts, tw, tid, kBgmvThreads);
+        __syncthreads();
+        tv = tw;
+    }
     const __nv_bfloat16* Bt = S.Bt_pool + ob;
     __nv_bfloat16* yr = a.y + (int64_t)tok * a.y_ld + S.y_off;
     const float scale = adapter_scale(a, ad);
@@ -507,9 +525,9 @@ __global__ void __launch_bounds__(kBgmvThreads, 4) bgmv_kernel(ApplyArgs a) {
         for (int j = 0; j < k; ++j) {
             float bf[8];
             bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(Bt + (int64_t)j * S.d_out + e)), bf);
-            const float tv = ts[j];
+            const float tj = tv[j];
 #pragma unroll
-            for (int c = 0; c < 8; ++c) acc[c] = fmaf(tv, bf[c], acc[c]);
+            for (int c = 0; c < 8; ++c) acc[c] = fmaf(tj, bf[c], acc[c]);
         }
         __nv_bfloat162* y2 = reinterpret_cast<__nv_bfloat162*>(&yv);
 #pragma unroll

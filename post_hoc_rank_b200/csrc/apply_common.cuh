@@ -34,7 +34,7 @@ struct SliceTab {
     int32_t d_out;      // output columns of the slice
     int32_t t_col;      // first column of the slice's t in the t buffers
     int32_t chunk0;     // first grid column chunk of the slice (set per expand launch)
-    int32_t pad0;
+    int32_t k_shared;   // ranks == nullptr: every adapter uses the slice's shared factors (rank k_shared, offset 0)
     int64_t y_off;      // first column of the slice in y
     const int32_t* ranks;
     const int64_t* off_A;
@@ -54,6 +54,10 @@ struct ApplyArgs {
     const int32_t* ids;        // T
     float scale;
     const float* scales;       // per adapter (nullable): replaces `scale`
+    // Sigma-sandwich serving: t <- Sigma_a t before the expand (0 = none, 1 = diagonal
+    // Sigma, n_adapters x k fp32, 2 = full Sigma, n_adapters x k x k fp32 row-major)
+    int32_t sigma_mode;
+    const float* sigma;
     SliceTab sl[kMaxSlices];
     // routing (sorted path)
     const int32_t* counts;     // [0] segments, [1] routed tokens, [2] GEMV items, [3] tensor-core items
@@ -91,9 +95,15 @@ __device__ __forceinline__ int slice_of_chunk(const ApplyArgs& a, int c) {
 __device__ __forceinline__ bool slice_factors(const ApplyArgs& a, int s, int ad, bool report, int& k, int64_t& oa,
                                               int64_t& ob) {
     const SliceTab& t = a.sl[s];
-    k = t.ranks[ad];
-    oa = t.off_A[ad];
-    ob = t.off_Bt[ad];
+    if (t.ranks) {
+        k = t.ranks[ad];
+        oa = t.off_A[ad];
+        ob = t.off_Bt[ad];
+    } else {   // shared factors
+        k = t.k_shared;
+        oa = 0;
+        ob = 0;
+    }
     int err = 0;
     if (k > kMaxRank) err = LF_ERR_SHAPE;
     else if (k > 0 && ((oa & 7) || (ob & 7))) err = LF_ERR_ALIGNMENT;
@@ -111,6 +121,24 @@ __device__ __forceinline__ bool slice_factors(const ApplyArgs& a, int s, int ad,
 
 __device__ __forceinline__ float adapter_scale(const ApplyArgs& a, int ad) {
     return a.scales ? a.scales[ad] : a.scale;
+}
+
+// Sigma-sandwich step on one token's t (k values, fp32, in `t`): w = Sigma_ad t, written to
+// `w` (may not alias `t`).  Called by `nthreads` threads with thread index `ti`; each
+// output i is formed by one thread in a fixed order.
+__device__ __forceinline__ void sigma_apply(const ApplyArgs& a, int ad, int k, const float* t, float* w, int ti,
+                                            int nthreads) {
+    if (a.sigma_mode == 1) {
+        const float* d = a.sigma + (size_t)ad * k;
+        for (int i = ti; i < k; i += nthreads) w[i] = d[i] * t[i];
+    } else {
+        const float* S = a.sigma + (size_t)ad * k * k;
+        for (int i = ti; i < k; i += nthreads) {
+            float acc = 0.f;
+            for (int j = 0; j < k; ++j) acc = fmaf(S[i * k + j], t[j], acc);
+            w[i] = acc;
+        }
+    }
 }
 
 }  // namespace lf

@@ -381,9 +381,18 @@ static void set_chunks(ApplyArgs& a, int W) {
     a.n_chunks = c;
 }
 
+// Shared-factor slice for Sigma-sandwich serving (every adapter uses rank k_shared and
+// the pools at offset 0).
+struct SharedSlice {
+    int32_t k = 0;
+    const float* sigma = nullptr;
+    int32_t mode = 0;
+};
+
 static lf_status apply_impl(int32_t T, int32_t d_in, const void* x, void* y, int64_t y_ld, const int32_t* ids,
                             int32_t n_adapters, const lf_slice* sl, int32_t ns, float scale, const float* scales,
-                            int32_t* seg_out, void* ws, size_t ws_bytes, cudaStream_t s) {
+                            int32_t* seg_out, void* ws, size_t ws_bytes, cudaStream_t s,
+                            const SharedSlice* shared = nullptr) {
     if (T < 0 || d_in < 1 || n_adapters < 1 || n_adapters > 16384 || ns < 1 || ns > kMaxSlices || !sl)
         return LF_ERR_INVALID_ARG;
     if (T == 0) return LF_OK;
@@ -394,7 +403,8 @@ static lf_status apply_impl(int32_t T, int32_t d_in, const void* x, void* y, int
         const lf_slice& t = sl[q];
         if (t.d_out < 1 || t.pool_elems_A < 0 || t.pool_elems_Bt < 0 || t.y_offset < 0 || t.y_offset + t.d_out > y_ld)
             return LF_ERR_INVALID_ARG;
-        if (!t.ranks || !t.off_A || !t.off_Bt || !t.A_pool || !t.Bt_pool) return LF_ERR_INVALID_ARG;
+        if (!shared && (!t.ranks || !t.off_A || !t.off_Bt)) return LF_ERR_INVALID_ARG;
+        if (!t.A_pool || !t.Bt_pool) return LF_ERR_INVALID_ARG;
         if ((t.d_out & 7) || (t.y_offset & 7)) return LF_ERR_ALIGNMENT;
         if (!aligned16(t.A_pool) || !aligned16(t.Bt_pool)) return LF_ERR_ALIGNMENT;
     }
@@ -414,10 +424,15 @@ static lf_status apply_impl(int32_t T, int32_t d_in, const void* x, void* y, int
     A.ids = ids;
     A.scale = scale;
     A.scales = scales;
+    if (shared) {
+        A.sigma_mode = shared->mode;
+        A.sigma = shared->sigma;
+    }
     for (int q = 0; q < ns; ++q) {
         SliceTab& t = A.sl[q];
         t.d_out = sl[q].d_out;
         t.t_col = kMaxRank * q;
+        t.k_shared = shared ? shared->k : 0;
         t.y_off = sl[q].y_offset;
         t.ranks = sl[q].ranks;
         t.off_A = sl[q].off_A;
@@ -847,6 +862,26 @@ size_t lf_apply_slices_workspace_size(int32_t T, int32_t n_adapters, int32_t n_s
 }
 
 size_t lf_apply_workspace_size(int32_t T, int32_t n_adapters) { return lf_apply_slices_workspace_size(T, n_adapters, 1); }
+
+lf_status lf_lora_sigma_sandwich(int32_t T, int32_t d_in, int32_t d_out, const void* x, void* y, const int32_t* ids,
+                                 int32_t n_adapters, int32_t rank, const void* Vt, const void* Ut, const float* sigma,
+                                 int32_t sigma_diag, float scale, void* ws, size_t ws_bytes, lf_stream_t stream) {
+    if (rank < 1 || rank > kMaxRank || d_out < 1 || (sigma_diag != 0 && sigma_diag != 1)) return LF_ERR_INVALID_ARG;
+    if (T > 0 && (!Vt || !Ut || !sigma)) return LF_ERR_INVALID_ARG;
+    lf_slice one{};
+    one.d_out = d_out;
+    one.y_offset = 0;
+    one.A_pool = Vt;
+    one.Bt_pool = Ut;
+    one.pool_elems_A = (int64_t)rank * d_in;
+    one.pool_elems_Bt = (int64_t)rank * d_out;
+    SharedSlice sh;
+    sh.k = rank;
+    sh.sigma = sigma;
+    sh.mode = sigma_diag ? 1 : 2;
+    return apply_impl(T, d_in, x, y, d_out, ids, n_adapters, &one, 1, scale, nullptr, nullptr, ws, ws_bytes,
+                      reinterpret_cast<cudaStream_t>(stream), &sh);
+}
 
 lf_status lf_lora_shrink_expand(int32_t T, int32_t d_in, int32_t d_out, const void* x, void* y, const int32_t* ids,
                                 int32_t n_adapters, const int32_t* ranks, const int64_t* off_A,

@@ -248,6 +248,7 @@ struct ExpandTcSmem {
     __nv_bfloat16 alo[kTcM * kMaxRank];          // t_lo
     __nv_bfloat16 b[2][kMaxRank * kTcN2];        // B'^T tiles, MN-major, 16 KB each
     __nv_bfloat16 yt[kTcYBuf][kTcM * kTcYLd];    // staged y tiles, 34 KB each
+    float tw[kTcM][kMaxRank + 1];                // summed t rows (Sigma-sandwich only), 33 KB
     uint64_t bar;
     uint32_t tmem;
     int32_t toks[kTcM];
@@ -276,17 +277,41 @@ __global__ void __launch_bounds__(kTcExpThreads, 1) expand_tc_kernel(ApplyArgs a
     for (int m = tid; m < kTcM; m += kTcExpThreads) s.toks[m] = m < nt ? a.perm[it.tok0 + m] : 0;
     // t tile -> (t_hi, t_lo) bf16, K-major: element (m, j) at (m/8)*sbo + (j/8)*128 + (m%8)*16 + (j%8)*2
     const int nsplit = (a.d_in + tc_split_len(a.d_in) - 1) / tc_split_len(a.d_in);
+    auto t_of = [&](int m, int j) {   // t = sum of the split-K partials, fixed order: bitwise reproducible
+        float acc = 0.f;
+        if (m < nt && j < k)
+            for (int sp = 0; sp < nsplit; ++sp) acc += a.t_part[((size_t)sp * a.T + it.tok0 + m) * a.ldt + S.t_col + j];
+        return acc;
+    };
+    if (a.sigma_mode) {   // Sigma-sandwich: stage t rows, then t <- Sigma_a t per row
+        for (int c = tid; c < kTcM * k; c += kTcExpThreads) {
+            const int m = c / k, j = c % k;
+            s.tw[m][j] = t_of(m, j);
+        }
+        __syncthreads();
+    }
     for (int c = tid; c < kTcM * (kpad / 8); c += kTcExpThreads) {
         const int m = c % kTcM, jc = c / kTcM;
         float tv[8];
+        if (a.sigma_mode) {
+            const float* row = s.tw[m];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const int j = jc * 8 + i;
-            float acc = 0.f;
-            if (m < nt && j < k)
-                for (int sp = 0; sp < nsplit; ++sp)   // fixed order: bitwise reproducible
-                    acc += a.t_part[((size_t)sp * a.T + it.tok0 + m) * a.ldt + S.t_col + j];
-            tv[i] = acc;
+            for (int i = 0; i < 8; ++i) {
+                const int j = jc * 8 + i;
+                float acc = 0.f;
+                if (m < nt && j < k) {
+                    if (a.sigma_mode == 1) {
+                        acc = a.sigma[(size_t)it.adapter * k + j] * row[j];
+                    } else {
+                        const float* Sr = a.sigma + ((size_t)it.adapter * k + j) * k;
+                        for (int l = 0; l < k; ++l) acc = fmaf(Sr[l], row[l], acc);
+                    }
+                }
+                tv[i] = acc;
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) tv[i] = t_of(m, jc * 8 + i);
         }
         __align__(16) __nv_bfloat16 hi[8], lo[8];
 #pragma unroll

@@ -95,6 +95,9 @@ def lib() -> ctypes.CDLL:
         L.lf_lora_shrink_expand_slices.argtypes = [_I32, _I32, _P, _P, _I64, _P, _I32, _P, _I32,
                                                    ctypes.c_float, _P, _P, _P, _SZ, _P]
         L.lf_lora_shrink_expand_slices.restype = ctypes.c_int
+        L.lf_lora_sigma_sandwich.argtypes = [_I32, _I32, _I32, _P, _P, _P, _I32, _I32, _P, _P, _P, _I32,
+                                             ctypes.c_float, _P, _SZ, _P]
+        L.lf_lora_sigma_sandwich.restype = ctypes.c_int
         L.lf_lora_shrink_expand_noalloc.argtypes = [_I32, _I32, _I32, _P, _P, _P, _I32, _P, _P, _P, _P, _P,
                                                     _I64, _I64, ctypes.c_float, _P, _P]
         L.lf_lora_shrink_expand_noalloc.restype = ctypes.c_int
@@ -113,7 +116,8 @@ def exported_symbols() -> list[str]:
             "lf_select_ranks", "lf_export_workspace_size", "lf_export_pool_bound", "lf_truncate_export",
             "lf_apply_workspace_size", "lf_lora_shrink_expand", "lf_status_string", "lf_get_device_status",
             "lf_profile_enable", "lf_profile_reset", "lf_profile_read", "lf_launch_count",
-            "lf_lora_shrink_expand_noalloc", "lf_apply_slices_workspace_size", "lf_lora_shrink_expand_slices"]
+            "lf_lora_shrink_expand_noalloc", "lf_apply_slices_workspace_size", "lf_lora_shrink_expand_slices",
+            "lf_lora_sigma_sandwich"]
 
 # Limits of lf_lora_shrink_expand_noalloc (its scratch is a fixed array in the library).
 NOALLOC_MAX_TOKENS = 16384
@@ -237,6 +241,18 @@ def lf_lora_shrink_expand_slices(x, y, ids, n_adapters, slices, scale, ws, adapt
                                             len(slices), float(scale), _ptr(adapter_scale), _ptr(seg_out), _ptr(ws),
                                             ws.numel() if ws is not None else 0, _stream(stream))
     return _check(st, "lf_lora_shrink_expand_slices") if check else st
+
+
+def lf_lora_sigma_sandwich(x, y, ids, n_adapters, Vt, Ut, sigma, diagonal, scale, ws, stream=None,
+                           check=True) -> int:
+    """Sigma-sandwich serving: y += scale * U (Sigma_a (V^T x)); Vt rank x d_in, Ut rank x d_out
+    (bf16), sigma n_adapters x rank (diagonal) or n_adapters x rank x rank (fp32)."""
+    T, d_in = x.shape
+    d_out = y.shape[1]
+    st = lib().lf_lora_sigma_sandwich(T, d_in, d_out, _ptr(x), _ptr(y), _ptr(ids), n_adapters, Vt.shape[0],
+                                      _ptr(Vt), _ptr(Ut), _ptr(sigma), 1 if diagonal else 0, float(scale), _ptr(ws),
+                                      ws.numel() if ws is not None else 0, _stream(stream))
+    return _check(st, "lf_lora_sigma_sandwich") if check else st
 
 
 def lf_lora_shrink_expand_noalloc(x, y, ids, n_adapters, ranks, off_A, off_Bt, A_pool, Bt_pool, scale,

@@ -253,3 +253,37 @@ def test_one_slice_call_equals_projection_call():
     y2, _, st2 = run_slices(x, y0, ids, sl, 0.75)
     assert st1 == 0 and st2 == 0
     assert torch.equal(y1, y2)
+
+
+@pytest.mark.parametrize("regime", ["decode", "gemv", "tensor_core"])
+@pytest.mark.parametrize("diagonal", [True, False])
+def test_sigma_sandwich_matches_oracle(regime, diagonal):
+    # jointly compressed adapters: shared V^T, U^T and a Sigma_a per adapter
+    d_in, d_out, r = 512, 1024, 24
+    if regime == "decode":
+        T, n = 96, 32
+        ids = synth.zipf_ids(T, n, 1.0, (10, 0))
+    elif regime == "gemv":
+        T, n = 300, 37
+        ids = synth.zipf_ids(T, n, 1.0, (10, 1))
+    else:
+        T, n = 1024, 4
+        ids = np.repeat(np.arange(n, dtype=np.int32), 256)
+    ids = ids.copy()
+    ids[np.random.default_rng(11).random(T) < 0.05] = -1
+    Vt = synth.normal_bf16((r, d_in), (10, 2), std=d_in ** -0.5)
+    Ut = synth.normal_bf16((r, d_out), (10, 3), std=d_out ** -0.5)
+    g = np.random.default_rng(12)
+    sig = (g.standard_normal((n, r)) if diagonal else g.standard_normal((n, r, r)) / np.sqrt(r)).astype(np.float32)
+    x = synth.normal_bf16((T, d_in), (10, 4))
+    y0 = torch.zeros(T, d_out, dtype=torch.bfloat16)
+    dev = "cuda"
+    y = y0.clone().to(dev)
+    ws = api.workspace(lf.lf_apply_workspace_size(T, n), dev)
+    lf.lf_lora_sigma_sandwich(x.to(dev), y, torch.from_numpy(ids).to(dev), n, Vt.to(dev), Ut.to(dev),
+                              torch.from_numpy(sig).to(dev), diagonal, 1.5, ws)
+    assert lf.lf_get_device_status() == 0
+    want = OP.sigma_sandwich_apply(x.float().numpy(), y0.float().numpy(), ids, Vt.float().numpy(),
+                                   Ut.float().numpy(), sig.astype(np.float64), diagonal, 1.5)
+    assert_close(y.cpu(), want)
+    assert torch.equal(y.cpu()[torch.from_numpy(ids < 0)], y0[torch.from_numpy(ids < 0)])

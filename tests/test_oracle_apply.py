@@ -132,3 +132,42 @@ def test_slices_per_adapter_scale():
         rows = ids == a
         np.testing.assert_allclose(y[rows] - y0[rows], sc[a] * (one[rows] - y0[rows]), rtol=1e-12, atol=1e-12)
     assert np.array_equal(y[ids < 0], y0[ids < 0])
+
+
+def _sandwich_case(seed, n=4, T=19, d_in=12, d_out=10, r=3):
+    g = np.random.default_rng(seed)
+    return (g.integers(-1, n, size=T), g.standard_normal((T, d_in)), g.standard_normal((T, d_out)),
+            g.standard_normal((r, d_in)), g.standard_normal((r, d_out)))
+
+
+@pytest.mark.parametrize("diagonal", [True, False])
+def test_sigma_sandwich_equals_dense_adapter_matrices(diagonal):
+    # brute force: materialise each adapter's dW_a = U Sigma_a V^T and apply it densely
+    ids, x, y0, Vt, Ut = _sandwich_case(1)
+    g = np.random.default_rng(2)
+    sig = g.standard_normal((4, 3)) if diagonal else g.standard_normal((4, 3, 3))
+    y = AP.sigma_sandwich_apply(x, y0, ids, Vt, Ut, sig, diagonal, 0.7)
+    for t in range(len(ids)):
+        a = int(ids[t])
+        if a < 0:
+            assert np.array_equal(y[t], y0[t])
+            continue
+        S = np.diag(sig[a]) if diagonal else sig[a]
+        dW = Ut.T @ S @ Vt
+        np.testing.assert_allclose(y[t], y0[t] + 0.7 * dW @ x[t], rtol=1e-12, atol=1e-12)
+
+
+def test_sigma_sandwich_identity_sigma_is_a_shared_lora():
+    # Sigma_a = I for every adapter: every adapter is the same LoRA (A' = V^T, B'^T = U^T),
+    # so the result equals lora_apply with shared factors
+    ids, x, y0, Vt, Ut = _sandwich_case(3)
+    n, r = 4, 3
+    y = AP.sigma_sandwich_apply(x, y0, ids, Vt, Ut, np.tile(np.eye(r), (n, 1, 1)), False, 1.3)
+    ranks = np.full(n, r)
+    y_ref = AP.lora_apply(x, y0, ids, ranks, np.zeros(n, np.int64), np.zeros(n, np.int64), Vt.ravel(), Ut.ravel(), 1.3)
+    np.testing.assert_allclose(y, y_ref, rtol=1e-12, atol=1e-12)
+    # and a diagonal Sigma equals the full form with that diagonal
+    d = np.random.default_rng(4).standard_normal((n, r))
+    np.testing.assert_allclose(AP.sigma_sandwich_apply(x, y0, ids, Vt, Ut, d, True, 0.5),
+                               AP.sigma_sandwich_apply(x, y0, ids, Vt, Ut, np.stack([np.diag(v) for v in d]), False, 0.5),
+                               rtol=1e-12, atol=1e-12)
