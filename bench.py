@@ -386,6 +386,47 @@ def decode_bench(args, dev, stream, hbm, variant="ragged", fused=False):
     return out
 
 
+def sandwich_bench(args, dev, stream, hbm, rank=16, diagonal=True):
+    """Sigma-sandwich serving of jointly compressed adapters on the decode workload:
+    Llama-3-8B shapes, 32 layers x 7 projections, 256 tokens over 128 adapters (Zipf(1));
+    per projection a shared V^T (rank x d_in), U^T (rank x d_out) and a Sigma_a per adapter
+    (diagonal or full rank x rank)."""
+    import torch
+    from post_hoc_rank_b200 import api, synth
+    from post_hoc_rank_b200 import loraforge as lf
+
+    M = synth.LLAMA3_8B
+    n_ad, T = 128, 256
+    ids = synth.zipf_ids(T, n_ad, 1.0, (3, 0))
+    ids_d = torch.from_numpy(ids).to(dev)
+    n_dist = len(set(ids.tolist()))
+    calls, total_bytes = [], 0
+    g = np.random.default_rng(6)
+    for l in range(M.layers):
+        x_h = synth.normal_bf16((T, M.hidden), (6, 1, l), device=dev)
+        x_f = synth.normal_bf16((T, M.ffn), (6, 2, l), device=dev)
+        for p, (_, d_out, d_in) in enumerate(M.proj_shapes()):
+            Vt = synth.normal_bf16((rank, d_in), (6, 3, l, p), std=d_in ** -0.5, device=dev)
+            Ut = synth.normal_bf16((rank, d_out), (6, 4, l, p), std=d_out ** -0.5, device=dev)
+            shape = (n_ad, rank) if diagonal else (n_ad, rank, rank)
+            sig = torch.from_numpy(g.standard_normal(shape).astype(np.float32)).to(dev)
+            y = synth.normal_bf16((T, d_out), (6, 5, l, p), device=dev)
+            x = x_f if d_in == M.ffn else x_h
+            ws = api.workspace(lf.lf_apply_workspace_size(T, n_ad), dev)
+
+            def run(st=None, x=x, y=y, Vt=Vt, Ut=Ut, sig=sig, ws=ws):
+                lf.lf_lora_sigma_sandwich(x, y, ids_d, n_ad, Vt, Ut, sig, diagonal, 2.0, ws, stream=st)
+            calls.append(run)
+            total_bytes += 2 * T * d_in + 4 * T * d_out + 4 * T + 2 * rank * (d_in + d_out) \
+                + 4 * n_dist * (rank if diagonal else rank * rank)
+    out = _apply_run(args, calls, ids_d, n_ad, T, total_bytes, stream, hbm, dict(
+        workload=f"Sigma-sandwich decode: Llama-3-8B, 32 layers x 7 projections, 256 tokens, 128 adapters "
+                 f"Zipf(1), shared U, V of rank {rank}, {'diagonal' if diagonal else 'full'} Sigma per adapter"))
+    del calls
+    torch.cuda.empty_cache()
+    return out
+
+
 def prefill_bench(args, dev, stream, hbm, k, fused=False):
     """Config 4: Qwen2.5-7B layer, 7 projections, 32 requests x 512 tokens, request i -> adapter i.
     fused: q/k/v and gate/up as one multi-slice call each."""
@@ -816,6 +857,8 @@ def main():
                 "decode_padded_to_max": decode_bench(args, dev, stream, hbm, "padded"),
                 "decode_uncompressed_r64": decode_bench(args, dev, stream, hbm, "r64"),
                 "decode_fused_slices": decode_bench(args, dev, stream, hbm, fused=True),
+                "decode_sigma_sandwich_r16_diag": sandwich_bench(args, dev, stream, hbm, 16, True),
+                "decode_sigma_sandwich_r16_full": sandwich_bench(args, dev, stream, hbm, 16, False),
                 "prefill_k16": prefill_bench(args, dev, stream, hbm, 16),
                 "prefill_k16_fused_slices": prefill_bench(args, dev, stream, hbm, 16, fused=True),
                 "prefill_r64": prefill_bench(args, dev, stream, hbm, 64)}
