@@ -16,6 +16,8 @@ written for a reader to check against the pages by eye:
                   energy budget with a per-module floor) rank allocation.
 * ``apply``    -- adapter routing and the multi-LoRA side path
                   y += s * B' (A' x) by brute force.
+* ``jd``       -- joint diagonalization (JD-Full) of a LoRA collection by
+                  eigenvalue iteration with a QR orthogonalize.
 
 Every function names the passage it follows by page title and section.
 Readings of passages the pages leave open are stated beside the code.
@@ -23,4 +25,4 @@ Pins: every function here is pinned by ``tests/test_oracle_*.py`` against
 closed forms, library special cases, brute force or hand-worked fixtures
 (``tests/golden``); none is "parity unpinned".
 """
-from . import factor, allocate, apply  # noqa: F401
+from . import factor, allocate, apply, jd  # noqa: F401
