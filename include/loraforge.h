@@ -236,6 +236,53 @@ lf_status lf_lora_sigma_sandwich(int32_t T, int32_t d_in, int32_t d_out, const v
                                  const void* Vt, const void* Ut, const float* sigma, int32_t sigma_diag,
                                  float scale, void* ws, size_t ws_bytes, lf_stream_t stream);
 
+/* ---- Joint diagonalization (JD-Full) by eigenvalue iteration ------------------
+ * "Compress then Serve" (academ.us/article/2407.00066), section 3.1 eq. 1 and
+ * Appendix 8.1 (case 1, eqs. 6-7) / 8.2.  A problem is one module position shared
+ * by `count` LoRAs (modules mods[members[first + j]], all of the problem's d_out x
+ * d_in, ranks r_i <= 64): find U (d_out x rank) and V (d_in x rank) with
+ * orthonormal columns and one full rank x rank Sigma_i per LoRA such that
+ * B_i A_i ~ U Sigma_i V^T.  Each of `iters` steps updates both bases from the
+ * previous iterate, with P_i = A_i V and Q_i = B_i^T U:
+ *     U <- orthogonalize(sum_i w_i B_i (P_i (P_i^T Q_i))),
+ *     V <- orthogonalize(sum_i w_i A_i^T (Q_i (Q_i^T P_i))),
+ * orthogonalize = the Q of the thin QR with positive diag(R) (the factor-
+ * construction TSQR gives R, then Q = X R^-1, done twice).  Afterwards, if
+ * `sigma` is not null, Sigma_i = U^T B_i A_i V (eq. 6) at the final U, V.
+ * Contractions run on the fp64 tensor-core path (fp32 inputs, exact products,
+ * fp64 sums); U, V and Sigma are stored fp32.
+ * State: U of problem p at U_base + U_off (d_out x rank fp32, row-major), V^T at
+ * Vt_base + Vt_off (rank x d_in fp32, row-major): the layout of a rank-`rank`
+ * LoRA module (B = U, A = V^T) and of lf_lora_sigma_sandwich's V^T.  On entry
+ * they hold the starting bases (used as given; they need not be orthonormal),
+ * on return the bases after `iters` steps (unchanged when iters = 0).
+ * Sigma_i of the problem's j-th LoRA: rank x rank fp32 row-major at
+ * sigma + sigma_off + j * rank * rank (the layout of lf_lora_sigma_sandwich's
+ * full Sigma).  weights (nullable = all 1): fp64, one per entry of `members`;
+ * the pages' unit-Frobenius normalisation is w_i = 1 / ||B_i A_i||_F^2 (the sum
+ * of sigma^2 from lf_tsqr_batched).
+ * Errors: LF_ERR_INVALID_ARG (null pointers, iters < 0, member index out of
+ * range, count < 1), LF_ERR_SHAPE (rank outside 1..min(64, d_out, d_in), a
+ * member whose d_out / d_in differ from the problem's, r_i outside 1..64),
+ * LF_ERR_ALIGNMENT (a base pointer not 16-byte aligned), LF_ERR_WORKSPACE.
+ * Device-side: LF_ERR_NUMERIC when an update is numerically rank deficient
+ * (orthogonalize meets R_jj <= 0; the columns from there on are zeroed). */
+typedef struct {
+    int32_t d_out, d_in, rank;
+    int32_t first, count;      /* members[first .. first + count): module indices */
+    int64_t U_off, Vt_off;     /* element offsets of U and V^T */
+    int64_t sigma_off;         /* element offset of the problem's Sigma block */
+} lf_jd_problem;
+size_t lf_jd_workspace_size(const lf_module* mods /*[host]*/, int32_t n_mods,
+                            const int32_t* members /*[host]*/, int32_t n_members,
+                            const lf_jd_problem* probs /*[host]*/, int32_t n_probs);
+lf_status lf_jd_full(const lf_module* mods /*[host]*/, int32_t n_mods,
+                     const int32_t* members /*[host]*/, int32_t n_members,
+                     const lf_jd_problem* probs /*[host]*/, int32_t n_probs,
+                     const float* B_base, const float* A_base, const double* weights,
+                     int32_t iters, float* U_base, float* Vt_base, float* sigma,
+                     void* ws, size_t ws_bytes, lf_stream_t stream);
+
 /* ---- Shrink / expand with library-owned scratch -------------------------------
  * This entry point has no counterpart in the paper; it exists for callers that
  * cannot call cudaMalloc.  Examples: a serving loop that reserved all device memory

@@ -116,5 +116,43 @@ def shrink_expand_slices(x, y, ids, slices, scale, adapter_scale=None, ws=None, 
     return y
 
 
+@dataclasses.dataclass
+class JdTables:
+    members: np.ndarray    # int32 module indices, problem by problem
+    probs: np.ndarray      # lf_jd_problem records
+    U_total: int           # fp32 elements of the U buffer
+    Vt_total: int          # fp32 elements of the V^T buffer
+    sigma_total: int       # fp32 elements of the Sigma buffer
+
+
+def jd_tables(mods: np.ndarray, positions, rank: int) -> JdTables:
+    """Problem table for JD-Full over module positions.  positions: one list of module
+    indices per problem (the LoRAs sharing that position, all of one shape).  U, V^T and
+    Sigma of consecutive problems are laid out back to back (offsets multiples of 4)."""
+    members, rows = [], []
+    u = v = sg = 0
+    for pos in positions:
+        pos = [int(m) for m in pos]
+        d_out, d_in = int(mods["d_out"][pos[0]]), int(mods["d_in"][pos[0]])
+        rows.append((d_out, d_in, rank, len(members), len(pos), u, v, sg))
+        members += pos
+        u += (d_out * rank + 3) // 4 * 4
+        v += (rank * d_in + 3) // 4 * 4
+        sg += len(pos) * rank * rank
+    probs = np.zeros(len(rows), dtype=lf.JD_PROBLEM_DTYPE)
+    for i, r in enumerate(rows):
+        probs[i] = r
+    return JdTables(np.asarray(members, dtype=np.int32), probs, u, v, sg)
+
+
+def jd_full(mods, tabs: JdTables, B_base, A_base, U, Vt, iters: int, weights=None, sigma=None, ws=None,
+            stream=None):
+    """JD-Full eigenvalue iteration in place on U / Vt (fp32 device buffers laid out by
+    jd_tables); writes Sigma_i into `sigma` when given."""
+    ws = ws if ws is not None else workspace(lf.lf_jd_workspace_size(mods, tabs.members, tabs.probs), U.device)
+    lf.lf_jd_full(mods, tabs.members, tabs.probs, B_base, A_base, weights, iters, U, Vt, sigma, ws, stream)
+    return U, Vt, sigma
+
+
 def device_status(stream=None) -> int:
     return lf.lf_get_device_status(stream)

@@ -14,6 +14,7 @@
 #include "gram.cuh"
 #include "select_export.cuh"
 #include "apply.cuh"
+#include "jd.cuh"
 
 namespace lf {
 
@@ -536,6 +537,169 @@ static lf_status noalloc_scratch(void** out) {
     return LF_OK;
 }
 
+// ------------------------------------------------------------ JD-Full plan
+struct JdPlan {
+    std::vector<JdMember> members;
+    std::vector<JdProbDev> probs;
+    std::vector<lf_module> basis_user, basis_ws;
+    std::vector<TsqrWork> pwork;
+    std::vector<TsqrInfo> pinfo;
+    int32_t pslots = 0;
+    std::vector<JdTile> tiles;
+    TsqrPlan orth;
+    int RX = 16, RY = 16;
+    int64_t ws_U = 0, ws_Vt = 0;   // floats of the workspace copies of the state
+};
+
+static lf_status check_jd(const lf_module* mods, int32_t n_mods, const int32_t* members, int32_t n_members,
+                          const lf_jd_problem* probs, int32_t n_probs) {
+    lf_status st = check_mods(mods, n_mods);
+    if (st != LF_OK) return st;
+    if (n_members < 0 || n_probs < 0 || (n_members > 0 && !members) || (n_probs > 0 && !probs))
+        return LF_ERR_INVALID_ARG;
+    for (int32_t p = 0; p < n_probs; ++p) {
+        const lf_jd_problem& q = probs[p];
+        if (q.count < 1 || q.first < 0 || (int64_t)q.first + q.count > n_members) return LF_ERR_INVALID_ARG;
+        if (q.d_out < 1 || q.d_in < 1 || q.rank < 1 || q.rank > kMaxRank || q.rank > q.d_out || q.rank > q.d_in)
+            return LF_ERR_SHAPE;
+        if (q.U_off < 0 || q.Vt_off < 0 || q.sigma_off < 0) return LF_ERR_INVALID_ARG;
+        if ((q.U_off & 3) || (q.Vt_off & 3)) return LF_ERR_ALIGNMENT;
+        for (int32_t j = 0; j < q.count; ++j) {
+            const int32_t m = members[q.first + j];
+            if (m < 0 || m >= n_mods) return LF_ERR_INVALID_ARG;
+            if (mods[m].d_out != q.d_out || mods[m].d_in != q.d_in) return LF_ERR_SHAPE;
+        }
+    }
+    return LF_OK;
+}
+
+static void plan_jd(const lf_module* mods, const int32_t* members, const lf_jd_problem* probs, int32_t n_probs,
+                    JdPlan& P) {
+    int rx = 1, ry = 1;
+    for (int32_t p = 0; p < n_probs; ++p) {
+        const lf_jd_problem& q = probs[p];
+        P.probs.push_back(JdProbDev{(int32_t)P.members.size(), q.count, q.sigma_off});
+        for (int32_t j = 0; j < q.count; ++j) {
+            const int32_t m = members[q.first + j];
+            P.members.push_back(JdMember{m, p, j, 0});
+            rx = std::max(rx, (int)mods[m].r);
+        }
+        ry = std::max(ry, (int)q.rank);
+        P.basis_user.push_back(lf_module{q.d_out, q.d_in, q.rank, 0, q.U_off, q.Vt_off});
+        P.basis_ws.push_back(lf_module{q.d_out, q.d_in, q.rank, 0, P.ws_U, P.ws_Vt});
+        P.ws_U += align_up((int64_t)q.d_out * q.rank, 4);
+        P.ws_Vt += align_up((int64_t)q.rank * q.d_in, 4);
+        for (int f = 0; f < 2; ++f) {
+            const int rows = f == 0 ? q.d_out : q.d_in;
+            for (int r0 = 0; r0 < rows; r0 += kJdTR) P.tiles.push_back(JdTile{p, f, r0, std::min(kJdTR, rows - r0)});
+        }
+    }
+    P.RX = rt_bucket(rx);
+    P.RY = rt_bucket(ry);
+    const int32_t ng = (int32_t)P.members.size();
+    P.pinfo.resize((size_t)2 * ng);
+    for (int32_t g = 0; g < ng; ++g) {
+        const lf_module& md = mods[P.members[g].mod];
+        for (int f = 0; f < 2; ++f) {
+            const int rows = f == 0 ? md.d_out : md.d_in;
+            const int nch = (int)cdiv(rows, kJdChunk);
+            P.pinfo[2 * g + f] = TsqrInfo{nch, nch > 1 ? P.pslots : -1};
+            for (int c = 0; c < nch; ++c)
+                P.pwork.push_back(TsqrWork{2 * g + f, c * kJdChunk, std::min(kJdChunk, rows - c * kJdChunk),
+                                           nch > 1 ? P.pslots + c : -1});
+            if (nch > 1) P.pslots += nch;
+        }
+    }
+    std::stable_sort(P.pwork.begin(), P.pwork.end(),
+                     [](const TsqrWork& a, const TsqrWork& b) { return a.nrows > b.nrows; });
+    plan_tsqr(P.basis_ws.data(), n_probs, P.orth);
+}
+
+struct JdLayout {
+    size_t mods, members, probs, basis_user, basis_ws, pwork, pinfo, tiles, owork, onwork, oinfo;
+    size_t pcounters, ocounters, ppartial, opartial, QP, WZ, wsU, wsVt, RB, RA, total;
+};
+
+static JdLayout jd_layout(int32_t n_mods, int32_t n_probs, const JdPlan& P) {
+    Carver c(nullptr);
+    JdLayout L;
+    const size_t ng = P.members.size();
+    const size_t blk = (size_t)P.RX * P.RY;
+    const size_t rs2 = (size_t)P.orth.rs * P.orth.rs;
+#define LF_TAKE(field, T, cnt)                          \
+    do {                                                \
+        c.take<T>(cnt);                                 \
+        L.field = c.off - (size_t)(cnt) * sizeof(T);    \
+    } while (0)
+    LF_TAKE(mods, lf_module, n_mods);
+    LF_TAKE(members, JdMember, ng);
+    LF_TAKE(probs, JdProbDev, n_probs);
+    LF_TAKE(basis_user, lf_module, n_probs);
+    LF_TAKE(basis_ws, lf_module, n_probs);
+    LF_TAKE(pwork, TsqrWork, P.pwork.size());
+    LF_TAKE(pinfo, TsqrInfo, P.pinfo.size());
+    LF_TAKE(tiles, JdTile, P.tiles.size());
+    LF_TAKE(owork, TsqrWork, P.orth.work.size());
+    LF_TAKE(onwork, int32_t, 1);
+    LF_TAKE(oinfo, TsqrInfo, P.orth.info.size());
+    LF_TAKE(pcounters, int32_t, 2 * ng);
+    LF_TAKE(ocounters, int32_t, (size_t)12 * n_probs);   // two orthogonalize rounds x (Gram, Householder, flags)
+    LF_TAKE(ppartial, double, (size_t)P.pslots * blk);
+    LF_TAKE(opartial, char, (size_t)P.orth.slots * tsqr_slot_bytes(P.orth.RT));
+    LF_TAKE(QP, double, 2 * ng * blk);
+    LF_TAKE(WZ, float, 2 * ng * blk);
+    LF_TAKE(wsU, float, (size_t)P.ws_U);
+    LF_TAKE(wsVt, float, (size_t)P.ws_Vt);
+    LF_TAKE(RB, float, (size_t)n_probs * rs2);
+    LF_TAKE(RA, float, (size_t)n_probs * rs2);
+#undef LF_TAKE
+    L.total = c.off + 256;
+    return L;
+}
+
+template <int RX, int RY>
+static cudaError_t launch_jd_rxry(int which, const void* args, int grid, cudaStream_t st) {
+    if (grid <= 0) return cudaSuccess;
+    if (which == 0) {
+        LF_LAUNCH("jd_project", (jd_project_kernel<RX, RY>), grid, 32 * jd_project_warps<RY>(), 0, st,
+                  *static_cast<const JdProjArgs*>(args));
+    } else if (which == 1) {
+        auto k = jd_core_kernel<RX, RY>;
+        constexpr size_t smem = jd_core_smem<RX, RY>();
+        cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        LF_LAUNCH("jd_core", k, grid, 256, smem, st, *static_cast<const JdCoreArgs*>(args));
+    } else {
+        auto k = jd_update_kernel<RX, RY>;
+        constexpr size_t smem = jd_update_smem<RX, RY>();
+        cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        LF_LAUNCH("jd_update", k, grid, 128, smem, st, *static_cast<const JdUpdArgs*>(args));
+    }
+    return cudaGetLastError();
+}
+
+template <int RX>
+static cudaError_t launch_jd_rx(int RY, int which, const void* args, int grid, cudaStream_t st) {
+    if (RY == 16) return launch_jd_rxry<RX, 16>(which, args, grid, st);
+    if (RY == 32) return launch_jd_rxry<RX, 32>(which, args, grid, st);
+    return launch_jd_rxry<RX, 64>(which, args, grid, st);
+}
+
+static cudaError_t launch_jd(int RX, int RY, int which, const void* args, int grid, cudaStream_t st) {
+    if (RX == 16) return launch_jd_rx<16>(RY, which, args, grid, st);
+    if (RX == 32) return launch_jd_rx<32>(RY, which, args, grid, st);
+    return launch_jd_rx<64>(RY, which, args, grid, st);
+}
+
+static cudaError_t launch_jd_qform(int RT, const JdQArgs& a, int grid, cudaStream_t st) {
+    if (grid <= 0) return cudaSuccess;
+    if (RT == 16) LF_LAUNCH("jd_qform", jd_qform_kernel<16>, grid, kJdTR, 0, st, a);
+    else if (RT == 32) LF_LAUNCH("jd_qform", jd_qform_kernel<32>, grid, kJdTR, 0, st, a);
+    else LF_LAUNCH("jd_qform", jd_qform_kernel<64>, grid, kJdTR, 0, st, a);
+    return cudaGetLastError();
+}
+
 }  // namespace lf
 
 using namespace lf;
@@ -985,6 +1149,164 @@ lf_status lf_lora_shrink_expand_noalloc(int32_t T, int32_t d_in, int32_t d_out, 
         LF_LAUNCH("expand_gemv", expand_kernel, gemv_grid((int64_t)max_items * A.n_chunks), kGemvThreads, 0, s, A);
     }
     return launch_status();
+}
+
+size_t lf_jd_workspace_size(const lf_module* mods, int32_t n_mods, const int32_t* members, int32_t n_members,
+                            const lf_jd_problem* probs, int32_t n_probs) {
+    if (check_jd(mods, n_mods, members, n_members, probs, n_probs) != LF_OK) return 0;
+    JdPlan P;
+    plan_jd(mods, members, probs, n_probs, P);
+    return jd_layout(n_mods, n_probs, P).total;
+}
+
+lf_status lf_jd_full(const lf_module* mods, int32_t n_mods, const int32_t* members, int32_t n_members,
+                     const lf_jd_problem* probs, int32_t n_probs, const float* B_base, const float* A_base,
+                     const double* weights, int32_t iters, float* U_base, float* Vt_base, float* sigma, void* ws,
+                     size_t ws_bytes, lf_stream_t stream) {
+    lf_status st = check_jd(mods, n_mods, members, n_members, probs, n_probs);
+    if (st != LF_OK) return st;
+    if (iters < 0) return LF_ERR_INVALID_ARG;
+    if (n_probs == 0) return LF_OK;
+    if (!B_base || !A_base || !U_base || !Vt_base || !ws) return LF_ERR_INVALID_ARG;
+    if (!aligned16(B_base) || !aligned16(A_base) || !aligned16(U_base) || !aligned16(Vt_base))
+        return LF_ERR_ALIGNMENT;
+    JdPlan P;
+    plan_jd(mods, members, probs, n_probs, P);
+    const JdLayout L = jd_layout(n_mods, n_probs, P);
+    if (ws_bytes < L.total) return LF_ERR_WORKSPACE;
+    char* base = reinterpret_cast<char*>(align_up((int64_t)reinterpret_cast<uintptr_t>(ws), 256));
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const int32_t ng = (int32_t)P.members.size();
+
+    Staging h;
+    const int32_t onwork = (int32_t)P.orth.work.size();
+    h.put(mods, n_mods);
+    h.put(P.members.data(), P.members.size());
+    h.put(P.probs.data(), P.probs.size());
+    h.put(P.basis_user.data(), P.basis_user.size());
+    h.put(P.basis_ws.data(), P.basis_ws.size());
+    h.put(P.pwork.data(), P.pwork.size());
+    h.put(P.pinfo.data(), P.pinfo.size());
+    h.put(P.tiles.data(), P.tiles.size());
+    h.put(P.orth.work.data(), P.orth.work.size());
+    h.put(&onwork, 1);
+    h.put(P.orth.info.data(), P.orth.info.size());
+    LF_CUDA_TRY(cudaMemcpyAsync(base, h.buf.data(), h.off, cudaMemcpyHostToDevice, s));
+    LF_CUDA_TRY(cudaMemsetAsync(base + L.pcounters, 0, (size_t)2 * ng * sizeof(int32_t), s));
+
+    auto at = [&](size_t off) { return base + off; };
+    const lf_module* d_mods = reinterpret_cast<const lf_module*>(at(L.mods));
+    const JdMember* d_members = reinterpret_cast<const JdMember*>(at(L.members));
+    const JdProbDev* d_probs = reinterpret_cast<const JdProbDev*>(at(L.probs));
+    const lf_module* d_bu = reinterpret_cast<const lf_module*>(at(L.basis_user));
+    const lf_module* d_bw = reinterpret_cast<const lf_module*>(at(L.basis_ws));
+    float* wsU = reinterpret_cast<float*>(at(L.wsU));
+    float* wsVt = reinterpret_cast<float*>(at(L.wsVt));
+    float* RB = reinterpret_cast<float*>(at(L.RB));
+    float* RA = reinterpret_cast<float*>(at(L.RA));
+    const int npw = (int)P.pwork.size(), ntile = (int)P.tiles.size();
+
+    JdProjArgs pa;
+    pa.mods = d_mods;
+    pa.members = d_members;
+    pa.basis = d_bu;
+    pa.B_base = B_base;
+    pa.A_base = A_base;
+    pa.U_base = U_base;
+    pa.Vt_base = Vt_base;
+    pa.work = reinterpret_cast<const TsqrWork*>(at(L.pwork));
+    pa.info = reinterpret_cast<const TsqrInfo*>(at(L.pinfo));
+    pa.counters = reinterpret_cast<int32_t*>(at(L.pcounters));
+    pa.partial = reinterpret_cast<double*>(at(L.ppartial));
+    pa.QP = reinterpret_cast<double*>(at(L.QP));
+
+    JdCoreArgs ca;
+    ca.members = d_members;
+    ca.mods = d_mods;
+    ca.basis = d_bu;
+    ca.probs = d_probs;
+    ca.QP = pa.QP;
+    ca.weights = weights;
+    ca.WZ = reinterpret_cast<float*>(at(L.WZ));
+    ca.sigma = nullptr;
+    ca.write_wz = 1;
+
+    JdUpdArgs ua;
+    ua.mods = d_mods;
+    ua.members = d_members;
+    ua.probs = d_probs;
+    ua.basis_ws = d_bw;
+    ua.B_base = B_base;
+    ua.A_base = A_base;
+    ua.WZ = ca.WZ;
+    ua.tiles = reinterpret_cast<const JdTile*>(at(L.tiles));
+    ua.U_ws = wsU;
+    ua.Vt_ws = wsVt;
+
+    // orthogonalize round: TSQR R of the workspace state, then Q = X R^-1 into dst
+    auto orth_round = [&](int round, const lf_module* dst_tab, float* dst_U, float* dst_Vt) -> cudaError_t {
+        int32_t* cnt = reinterpret_cast<int32_t*>(at(L.ocounters)) + (size_t)6 * n_probs * round;
+        GramArgs ga;
+        ga.mods = d_bw;
+        ga.B_base = wsU;
+        ga.A_base = wsVt;
+        ga.work = reinterpret_cast<const TsqrWork*>(at(L.owork));
+        ga.n_work = reinterpret_cast<const int32_t*>(at(L.onwork));
+        ga.info = reinterpret_cast<const TsqrInfo*>(at(L.oinfo));
+        ga.counters = cnt;
+        ga.partial = reinterpret_cast<double*>(at(L.opartial));
+        ga.slot_doubles = (int64_t)(tsqr_slot_bytes(P.orth.RT) / sizeof(double));
+        ga.flags = cnt + 4 * n_probs;
+        ga.R_B = RB;
+        ga.R_A = RA;
+        ga.rs = P.orth.rs;
+        cudaError_t e = launch_gram_rt(P.orth.RT, ga, onwork, s);
+        if (e != cudaSuccess) return e;
+        TsqrArgs<float> ta;
+        ta.mods = d_bw;
+        ta.mod_ids = nullptr;
+        ta.B_base = wsU;
+        ta.A_base = wsVt;
+        ta.work = ga.work;
+        ta.n_work = ga.n_work;
+        ta.info = ga.info;
+        ta.counters = cnt + 2 * n_probs;
+        ta.partial = reinterpret_cast<float*>(at(L.opartial));
+        ta.R_B = RB;
+        ta.R_A = RA;
+        ta.rs = P.orth.rs;
+        ta.only = ga.flags;
+        e = launch_tsqr_rt<float>(P.orth.RT, ta, onwork, s);
+        if (e != cudaSuccess) return e;
+        JdQArgs qa;
+        qa.src = d_bw;
+        qa.dst = dst_tab;
+        qa.src_U = wsU;
+        qa.src_Vt = wsVt;
+        qa.dst_U = dst_U;
+        qa.dst_Vt = dst_Vt;
+        qa.R_B = RB;
+        qa.R_A = RA;
+        qa.rs = P.orth.rs;
+        qa.tiles = ua.tiles;
+        return launch_jd_qform(P.orth.RT, qa, ntile, s);
+    };
+
+    for (int32_t it = 0; it < iters; ++it) {
+        LF_CUDA_TRY(launch_jd(P.RX, P.RY, 0, &pa, npw, s));
+        LF_CUDA_TRY(launch_jd(P.RX, P.RY, 1, &ca, ng, s));
+        LF_CUDA_TRY(launch_jd(P.RX, P.RY, 2, &ua, ntile, s));
+        LF_CUDA_TRY(cudaMemsetAsync(at(L.ocounters), 0, (size_t)12 * n_probs * sizeof(int32_t), s));
+        LF_CUDA_TRY(orth_round(0, d_bw, wsU, wsVt));
+        LF_CUDA_TRY(orth_round(1, d_bu, U_base, Vt_base));
+    }
+    if (sigma) {
+        LF_CUDA_TRY(launch_jd(P.RX, P.RY, 0, &pa, npw, s));
+        ca.sigma = sigma;
+        ca.write_wz = 0;
+        LF_CUDA_TRY(launch_jd(P.RX, P.RY, 1, &ca, ng, s));
+    }
+    return LF_OK;
 }
 
 void lf_profile_enable(int on) { g_prof.on = on != 0; }

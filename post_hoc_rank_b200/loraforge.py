@@ -26,6 +26,13 @@ MODULE_DTYPE = np.dtype([("d_out", "<i4"), ("d_in", "<i4"), ("r", "<i4"), ("grou
 assert MODULE_DTYPE.itemsize == 32
 
 
+# lf_jd_problem: int32 d_out, d_in, rank, first, count; int64 U_off, Vt_off, sigma_off (48 bytes)
+JD_PROBLEM_DTYPE = np.dtype([("d_out", "<i4"), ("d_in", "<i4"), ("rank", "<i4"), ("first", "<i4"),
+                             ("count", "<i4"), ("U_off", "<i8"), ("Vt_off", "<i8"), ("sigma_off", "<i8")],
+                            align=True)
+assert JD_PROBLEM_DTYPE.itemsize == 48
+
+
 class lf_policy(ctypes.Structure):
     _fields_ = [("kind", ctypes.c_int32), ("ratio_num", ctypes.c_int32),
                 ("ratio_den", ctypes.c_int32), ("floor", ctypes.c_int32)]
@@ -98,6 +105,9 @@ def lib() -> ctypes.CDLL:
         L.lf_lora_sigma_sandwich.argtypes = [_I32, _I32, _I32, _P, _P, _P, _I32, _I32, _P, _P, _P, _I32,
                                              ctypes.c_float, _P, _SZ, _P]
         L.lf_lora_sigma_sandwich.restype = ctypes.c_int
+        L.lf_jd_workspace_size.argtypes = [_P, _I32, _P, _I32, _P, _I32]; L.lf_jd_workspace_size.restype = _SZ
+        L.lf_jd_full.argtypes = [_P, _I32, _P, _I32, _P, _I32, _P, _P, _P, _I32, _P, _P, _P, _P, _SZ, _P]
+        L.lf_jd_full.restype = ctypes.c_int
         L.lf_lora_shrink_expand_noalloc.argtypes = [_I32, _I32, _I32, _P, _P, _P, _I32, _P, _P, _P, _P, _P,
                                                     _I64, _I64, ctypes.c_float, _P, _P]
         L.lf_lora_shrink_expand_noalloc.restype = ctypes.c_int
@@ -117,7 +127,7 @@ def exported_symbols() -> list[str]:
             "lf_apply_workspace_size", "lf_lora_shrink_expand", "lf_status_string", "lf_get_device_status",
             "lf_profile_enable", "lf_profile_reset", "lf_profile_read", "lf_launch_count",
             "lf_lora_shrink_expand_noalloc", "lf_apply_slices_workspace_size", "lf_lora_shrink_expand_slices",
-            "lf_lora_sigma_sandwich"]
+            "lf_lora_sigma_sandwich", "lf_jd_workspace_size", "lf_jd_full"]
 
 # Limits of lf_lora_shrink_expand_noalloc (its scratch is a fixed array in the library).
 NOALLOC_MAX_TOKENS = 16384
@@ -253,6 +263,27 @@ def lf_lora_sigma_sandwich(x, y, ids, n_adapters, Vt, Ut, sigma, diagonal, scale
                                       _ptr(Vt), _ptr(Ut), _ptr(sigma), 1 if diagonal else 0, float(scale), _ptr(ws),
                                       ws.numel() if ws is not None else 0, _stream(stream))
     return _check(st, "lf_lora_sigma_sandwich") if check else st
+
+
+def _jd_tables(mods, members, probs):
+    pm, nm = _mods_ptr(mods)
+    assert members.dtype == np.int32 and members.flags["C_CONTIGUOUS"]
+    assert probs.dtype == JD_PROBLEM_DTYPE and probs.flags["C_CONTIGUOUS"]
+    return pm, nm, members.ctypes.data, int(members.shape[0]), probs.ctypes.data, int(probs.shape[0])
+
+
+def lf_jd_workspace_size(mods: np.ndarray, members: np.ndarray, probs: np.ndarray) -> int:
+    return lib().lf_jd_workspace_size(*_jd_tables(mods, members, probs))
+
+
+def lf_jd_full(mods, members, probs, B_base, A_base, weights, iters, U_base, Vt_base, sigma, ws, stream=None,
+               check=True) -> int:
+    """JD-Full eigenvalue iteration: U_base / Vt_base hold the starting bases on entry and the
+    bases after `iters` steps on return; sigma (nullable) receives Sigma_i = U^T B_i A_i V."""
+    st = lib().lf_jd_full(*_jd_tables(mods, members, probs), _ptr(B_base), _ptr(A_base), _ptr(weights),
+                          int(iters), _ptr(U_base), _ptr(Vt_base), _ptr(sigma), _ptr(ws),
+                          ws.numel() if ws is not None else 0, _stream(stream))
+    return _check(st, "lf_jd_full") if check else st
 
 
 def lf_lora_shrink_expand_noalloc(x, y, ids, n_adapters, ranks, off_A, off_Bt, A_pool, Bt_pool, scale,

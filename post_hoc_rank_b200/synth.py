@@ -214,6 +214,51 @@ def sigma_tables(n_adapters: int, model: ModelShape, r: int, cfg_id: int) -> np.
     return np.ascontiguousarray(np.stack(rows))
 
 
+def collection_layout(d_out: int, d_in: int, ranks) -> FleetLayout:
+    """One module position shared by len(ranks) LoRAs of the given ranks (one group each)."""
+    rows = []
+    b_off = a_off = 0
+    for a, r in enumerate(ranks):
+        rows.append((d_out, d_in, int(r), a, b_off, a_off, 0, 0))
+        b_off += _align4(d_out * int(r))
+        a_off += _align4(int(r) * d_in)
+    arr = np.array(rows, dtype=np.int64).reshape(-1, 8)
+    return FleetLayout(
+        d_out=arr[:, 0].astype(np.int32), d_in=arr[:, 1].astype(np.int32),
+        r=arr[:, 2].astype(np.int32), group=arr[:, 3].astype(np.int32),
+        B_off=arr[:, 4].copy(), A_off=arr[:, 5].copy(), B_total=b_off, A_total=a_off,
+        proj=arr[:, 6].astype(np.int32), layer=arr[:, 7].astype(np.int32))
+
+
+def fill_collection(layout: FleetLayout, key: tuple[int, ...]):
+    """CPU fp32 torch buffers for a collection_layout: B = column-normalised Gaussian
+    times sigma_j = (j+1)^-1 e^{0.5 z_j}, A ~ N(0, 1/d_in), seeded per LoRA."""
+    import torch
+    B = torch.zeros(layout.B_total, dtype=torch.float32)
+    A = torch.zeros(layout.A_total, dtype=torch.float32)
+    for i in range(layout.n):
+        d_out, d_in, r = int(layout.d_out[i]), int(layout.d_in[i]), int(layout.r[i])
+        g = torch.Generator()
+        g.manual_seed(derive_seed(*key, i, 0))
+        Bi = torch.randn((d_out, r), generator=g, dtype=torch.float32)
+        Bi /= torch.linalg.vector_norm(Bi, dim=0, keepdim=True)
+        rng = np.random.Generator(np.random.Philox(derive_seed(*key, i, 1)))
+        Bi *= torch.from_numpy(sigma_profile(rng.standard_normal, r, True).astype(np.float32))[None, :]
+        Ai = torch.randn((r, d_in), generator=g, dtype=torch.float32) * (1.0 / math.sqrt(d_in))
+        b0, a0 = int(layout.B_off[i]), int(layout.A_off[i])
+        B[b0:b0 + d_out * r] = Bi.reshape(-1)
+        A[a0:a0 + r * d_in] = Ai.reshape(-1)
+    return B, A
+
+
+def normal_f32(shape, key: tuple[int, ...], device="cpu"):
+    """fp32 tensor of N(0, 1) draws (torch, seeded)."""
+    import torch
+    g = torch.Generator(device=device)
+    g.manual_seed(derive_seed(*key))
+    return torch.randn(shape, generator=g, device=device, dtype=torch.float32)
+
+
 def zipf_ids(T: int, n: int, alpha: float, key: tuple[int, ...]) -> np.ndarray:
     """T adapter ids drawn from P(i) ~ (i+1)^-alpha on 0..n-1 (finite support), shuffled."""
     rng = np.random.Generator(np.random.Philox(derive_seed(*key)))

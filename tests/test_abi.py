@@ -129,3 +129,45 @@ def test_module_dtype_matches_c_struct():
     assert lf.MODULE_DTYPE.itemsize == 32
     assert [lf.MODULE_DTYPE.fields[f][1] for f in ("d_out", "d_in", "r", "group", "B_off", "A_off")] == \
         [0, 4, 8, 12, 16, 24]
+
+
+def test_jd_problem_dtype_matches_c_struct():
+    assert lf.JD_PROBLEM_DTYPE.itemsize == 48
+    assert [lf.JD_PROBLEM_DTYPE.fields[f][1] for f in
+            ("d_out", "d_in", "rank", "first", "count", "U_off", "Vt_off", "sigma_off")] == \
+        [0, 4, 8, 12, 16, 24, 32, 40]
+
+
+def test_jd_validation_on_host():
+    """lf_jd_full rejects bad problem tables before any CUDA call."""
+    from post_hoc_rank_b200 import api
+    lay = synth.collection_layout(40, 36, [4, 4, 3])
+    mods = modules_from_layout(lay)
+    tabs = api.jd_tables(mods, [[0, 1, 2]], 4)
+    assert lf.lf_jd_workspace_size(mods, tabs.members, tabs.probs) > 0
+
+    def call(members=None, probs=None, iters=1, ptr=16, ws=16, wsb=1 << 24):
+        members = tabs.members if members is None else members
+        probs = tabs.probs.copy() if probs is None else probs
+        return lf.lib().lf_jd_full(
+            mods.ctypes.data, len(mods), members.ctypes.data, len(members), probs.ctypes.data, len(probs),
+            ptr, ptr, None, iters, ptr, ptr, None, ws, wsb, None)
+
+    def with_prob(**kv):
+        p = tabs.probs.copy()
+        for k, v in kv.items():
+            p[0][k] = v
+        return p
+    assert call(iters=-1) == 1
+    assert call(probs=with_prob(rank=0)) == 2
+    assert call(probs=with_prob(rank=65)) == 2
+    assert call(probs=with_prob(rank=37)) == 2            # > d_in
+    assert call(probs=with_prob(count=0)) == 1
+    assert call(probs=with_prob(count=4)) == 1            # past the member list
+    assert call(probs=with_prob(d_out=41)) == 2           # members of another shape
+    assert call(probs=with_prob(U_off=2)) == 8
+    assert call(members=np.array([0, 1, 7], dtype=np.int32)) == 1
+    assert call(ptr=0) == 1
+    assert call(ptr=8) == 8
+    assert call(wsb=64) == 4
+    assert call(probs=tabs.probs[:0]) == 0                # nothing to do
