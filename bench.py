@@ -664,6 +664,109 @@ def large_fleet_bench(args, dev, stream, hbm):
     return out
 
 
+def jd_bench(dev, stream, hbm, sm_mhz, n_lora=64, r=16, rank=64, iters=10, with_cpu=True):
+    """JD-Full eigenvalue iteration ("Compress then Serve", Appendix 8.2): n_lora
+    Llama-3-8B-shaped LoRAs of rank r at each of one layer's 7 module positions (7 problems
+    in one call), shared rank `rank`, `iters` steps, Sigma_i at the final bases."""
+    import torch
+    from post_hoc_rank_b200 import api, synth
+    from post_hoc_rank_b200 import loraforge as lf
+
+    M = synth.LLAMA3_8B
+    lay = synth.fleet_layout(n_lora, M, r=r, n_layers=1)
+    mods = api.modules_from_layout(lay)
+    B = torch.empty(lay.B_total, dtype=torch.float32, device=dev)
+    A = torch.empty(lay.A_total, dtype=torch.float32, device=dev)
+    synth.fill_fleet(lay, B, A, cfg_id=7)
+    positions = [[i for i in range(lay.n) if int(lay.proj[i]) == p] for p in range(7)]
+    tabs = api.jd_tables(mods, positions, rank)
+    U0 = torch.empty(tabs.U_total, dtype=torch.float32, device=dev)
+    Vt0 = torch.empty(tabs.Vt_total, dtype=torch.float32, device=dev)
+    for p, pr in enumerate(tabs.probs):
+        d_out, d_in, uo, vo = int(pr["d_out"]), int(pr["d_in"]), int(pr["U_off"]), int(pr["Vt_off"])
+        U0[uo:uo + d_out * rank] = synth.normal_f32((d_out * rank,), (7, 1, p), device=dev)
+        Vt0[vo:vo + rank * d_in] = synth.normal_f32((rank * d_in,), (7, 2, p), device=dev)
+    U, Vt = U0.clone(), Vt0.clone()
+    sig = torch.empty(tabs.sigma_total, dtype=torch.float32, device=dev)
+    ws = api.workspace(lf.lf_jd_workspace_size(mods, tabs.members, tabs.probs), dev)
+
+    def solve():
+        U.copy_(U0); Vt.copy_(Vt0)
+        lf.lf_jd_full(mods, tabs.members, tabs.probs, B, A, None, iters, U, Vt, sig, ws, stream)
+
+    for _ in range(2):
+        solve()
+    torch.cuda.synchronize()
+    reps = 3
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        solve()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / reps
+    lf.lf_profile_reset(); lf.lf_profile_enable(True)
+    l0 = lf.lf_launch_count()
+    solve()
+    launches = lf.lf_launch_count() - l0
+    lf.lf_profile_enable(False)
+    ph = lf.lf_profile_read()
+    st = lf.lf_get_device_status(stream)
+    # algorithmic work: each pass reads every factor once (fp32) and does 2 (d_out + d_in) r r~ flops per LoRA
+    passes = 2 * iters + 1
+    fac_bytes = 4 * int(((lay.d_out + lay.d_in).astype(np.int64) * lay.r).sum())
+    pass_flops = 2.0 * float(((lay.d_out + lay.d_in).astype(np.int64) * lay.r).sum()) * rank
+    state_bytes = 4 * int(((tabs.probs["d_out"] + tabs.probs["d_in"]).astype(np.int64)).sum()) * rank
+    algo_bytes = passes * fac_bytes + (3 * passes + 6 * iters) * state_bytes
+    algo_flops = passes * pass_flops
+    dom = max(("jd_project", "jd_update"), key=lambda k: ph.get(k, (0.0, 1))[0])
+    dom_ms, dom_n = ph[dom]
+    dom_flops = (iters + 1 if dom == "jd_project" else iters) * pass_flops
+    fp64 = fp64_peak_tflops(sm_mhz)
+    ach = dom_flops / (dom_ms * 1e-3) / 1e12
+    out = {
+        "workload": f"JD-Full eigenvalue iteration: {n_lora} Llama-3-8B-shaped LoRAs (rank {r}) at each of the 7 "
+                    f"module positions of one layer, shared rank {rank}, {iters} steps + Sigma",
+        "ms_per_solve": round(ms, 3), "positions_per_s": round(7 / (ms * 1e-3), 2),
+        "ms_per_step": round(ms / iters, 3),
+        "algo_bytes": int(algo_bytes), "algo_gbs": round(algo_bytes / (ms * 1e-3) / 1e9, 1),
+        "hbm_frac": round(algo_bytes / (ms * 1e-3) / 1e9 / hbm, 4),
+        "algo_tflops": round(algo_flops / (ms * 1e-3) / 1e12, 2),
+        "roofline": {"kernel": dom, "bound": "fp64_tensor", "achieved": round(ach, 2),
+                     "peak": round(fp64, 1), "unit": "TFLOP/s", "frac": round(ach / fp64, 4),
+                     "peak_source": "derived: 148 SMs x 64 fp64 FMA/clk x 2 x median SM clock"},
+        "phases_ms": {k: round(v[0], 3) for k, v in ph.items()},
+        "gpu_launches": int(launches), "device_status": st,
+    }
+    if with_cpu:
+        out["cpu_baseline"] = cpu_jd_baseline(B, A, lay, tabs, U0, Vt0, rank, iters)
+    del B, A, U, Vt, U0, Vt0, sig, ws
+    torch.cuda.empty_cache()
+    return out
+
+
+def cpu_jd_baseline(B, A, lay, tabs, U0, Vt0, rank, iters):
+    """The fp64 oracle's JD-Full on one module position of the same workload (q, 64 LoRAs),
+    same start and step count; positions/s on the host cores."""
+    import torch
+    from oracle import jd as OJ
+    pr = tabs.probs[0]
+    m = tabs.members[int(pr["first"]):int(pr["first"]) + int(pr["count"])]
+    Bh, Ah = B.cpu(), A.cpu()
+    Bs = [Bh[int(lay.B_off[i]):int(lay.B_off[i]) + int(lay.d_out[i]) * int(lay.r[i])].double().numpy()
+          .reshape(int(lay.d_out[i]), int(lay.r[i])) for i in m]
+    As = [Ah[int(lay.A_off[i]):int(lay.A_off[i]) + int(lay.r[i]) * int(lay.d_in[i])].double().numpy()
+          .reshape(int(lay.r[i]), int(lay.d_in[i])) for i in m]
+    d_out, d_in = int(pr["d_out"]), int(pr["d_in"])
+    Us = U0[:d_out * rank].cpu().double().numpy().reshape(d_out, rank)
+    Vs = Vt0[:rank * d_in].cpu().double().numpy().reshape(rank, d_in).T
+    t0 = time.perf_counter()
+    OJ.jd_full(Bs, As, Us, Vs, iters)
+    dt = time.perf_counter() - t0
+    return {"kind": "oracle", "value": round(1.0 / dt, 4), "unit": "positions/s", "cores": torch.get_num_threads(),
+            "sample": f"one position (q, 4096 x 4096) x {len(m)} LoRAs, {iters} steps + Sigma"}
+
+
 def library_qr_context(dev, stream):
     """Matched library QR on the same modules: torch.linalg.qr (cuSOLVER geqrf, R only)
     on one Qwen2.5-7B-shaped adapter (196 modules, r = 64), B and A^T of each projection
@@ -804,6 +907,7 @@ def main():
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-large", action="store_true")
+    ap.add_argument("--no-jd", action="store_true")
     ap.add_argument("--large-adapters", type=int, default=1024)
     args = ap.parse_args()
 
@@ -866,6 +970,8 @@ def main():
             lora["decode"]["cpu_baseline"] = cpu_apply_baseline()
     large = None if (args.no_large or rank != 0) else large_fleet_bench(args, dev, stream, hbm)
     libqr = None if (args.no_apply or rank != 0) else library_qr_context(dev, stream)
+    jd = None if (args.no_jd or rank != 0) else jd_bench(dev, stream, hbm, fr["clocks"].get("sm_mhz"),
+                                                         with_cpu=not args.no_cpu)
     e2e = None
     if not args.no_e2e:
         e = factor_e2e(args, dev, stream, rank)
@@ -899,6 +1005,7 @@ def main():
         "lora_path": lora,
         "large_fleet": large,
         "library_qr_context": libqr,
+        "jd_full": jd,
         "cpu_baseline": cpu,
         "device_status": fr["status"],
     }

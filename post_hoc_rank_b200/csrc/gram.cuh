@@ -63,6 +63,8 @@ struct GramArgs {
     float* R_B;                // per module, rs x rs
     float* R_A;
     int32_t rs;
+    const int32_t* only;       // per mf (nullable): zero = skip this matrix
+    double* R64;               // nullable: per mf, rs x rs fp64 copy of R (mf = 2 * module + factor)
 };
 
 // D (8x8, two entries per lane) += A (8x4) * B (4x8), fp64, one warp.
@@ -161,6 +163,39 @@ __device__ __forceinline__ void gram_chunk(double (&acc)[(RT / 8) * (RT / 8 + 1)
     __syncwarp();
 }
 
+// Right-looking Cholesky of the packed Gram G (r x r used) in place by one warp: row
+// j of R overwrites row j of G.  Returns false (warp-uniform: every lane reads the same
+// values) when a pivot falls to <= kGramPivotTol times its Gram diagonal.
+template <int RT>
+__device__ __forceinline__ bool gram_cholesky(double* G, double* s_diag, int r, int lane) {
+    using C = Cols<RT>;
+    for (int j = lane; j < r; j += 32) s_diag[j] = G[tri_off<RT>(j, j)];
+    __syncwarp();
+    for (int j = 0; j < r; ++j) {
+        const double d = G[tri_off<RT>(j, j)];
+        if (!(d > kGramPivotTol * s_diag[j])) return false;
+        const double rjj = sqrt(d);
+        __syncwarp();
+#pragma unroll
+        for (int s = 0; s < C::NS; ++s) {
+            const int c = C::col(lane, s);
+            if (c > j && c < r) G[tri_off<RT>(j, c)] /= rjj;
+        }
+        if (lane == 0) G[tri_off<RT>(j, j)] = rjj;
+        __syncwarp();
+#pragma unroll
+        for (int s = 0; s < C::NS; ++s) {
+            const int c = C::col(lane, s);
+            if (c > j && c < r) {
+                const double gjc = G[tri_off<RT>(j, c)];
+                for (int k = j + 1; k <= c; ++k) G[tri_off<RT>(k, c)] -= G[tri_off<RT>(j, k)] * gjc;
+            }
+        }
+        __syncwarp();
+    }
+    return true;
+}
+
 template <int RT>
 __global__ void __launch_bounds__(32, 8) gram_kernel(GramArgs a) {
     constexpr int NB = RT / 8;
@@ -174,6 +209,7 @@ __global__ void __launch_bounds__(32, 8) gram_kernel(GramArgs a) {
     if ((int)blockIdx.x >= *a.n_work) return;
     const TsqrWork w = a.work[blockIdx.x];
     const int mf = w.mf, factor = mf & 1;
+    if (a.only && a.only[mf] == 0) return;
     const lf_module md = a.mods[mf >> 1];
     const int r = md.r;
     const float* X = factor == 0 ? a.B_base + md.B_off : a.A_base + md.A_off;
@@ -225,39 +261,21 @@ __global__ void __launch_bounds__(32, 8) gram_kernel(GramArgs a) {
     }
     __syncwarp();
 
-    // right-looking Cholesky of the packed G in place: row j of R overwrites row j of G
-    using C = Cols<RT>;
-    for (int j = lane; j < r; j += 32) s_diag[j] = G[tri_off<RT>(j, j)];
-    __syncwarp();
-    for (int j = 0; j < r; ++j) {
-        const double d = G[tri_off<RT>(j, j)];
-        if (!(d > kGramPivotTol * s_diag[j])) {   // warp-uniform: every lane read the same values
-            if (lane == 0) a.flags[mf] = 1;
-            return;
-        }
-        const double rjj = sqrt(d);
-        __syncwarp();
-#pragma unroll
-        for (int s = 0; s < C::NS; ++s) {
-            const int c = C::col(lane, s);
-            if (c > j && c < r) G[tri_off<RT>(j, c)] /= rjj;
-        }
-        if (lane == 0) G[tri_off<RT>(j, j)] = rjj;
-        __syncwarp();
-#pragma unroll
-        for (int s = 0; s < C::NS; ++s) {
-            const int c = C::col(lane, s);
-            if (c > j && c < r) {
-                const double gjc = G[tri_off<RT>(j, c)];
-                for (int k = j + 1; k <= c; ++k) G[tri_off<RT>(k, c)] -= G[tri_off<RT>(j, k)] * gjc;
-            }
-        }
-        __syncwarp();
+    if (!gram_cholesky<RT>(G, s_diag, r, lane)) {
+        if (lane == 0) a.flags[mf] = 1;
+        return;
     }
     float* out = (factor == 0 ? a.R_B : a.R_A) + (size_t)(mf >> 1) * a.rs * a.rs;
     for (int e = lane; e < a.rs * a.rs; e += 32) {
         const int j = e / a.rs, c = e % a.rs;
         out[e] = (j < r && c < r && c >= j) ? (float)G[tri_off<RT>(j, c)] : 0.f;
+    }
+    if (a.R64) {
+        double* o64 = a.R64 + (size_t)mf * a.rs * a.rs;
+        for (int e = lane; e < a.rs * a.rs; e += 32) {
+            const int j = e / a.rs, c = e % a.rs;
+            o64[e] = (j < r && c < r && c >= j) ? G[tri_off<RT>(j, c)] : 0.0;
+        }
     }
 }
 

@@ -9,10 +9,13 @@
 // and Sigma_i = U^T B_i A_i V = Q_i^T P_i = S_i^T (eq. 6) at the final U, V.
 //
 // The state (U, V^T) of a problem has the layout of a LoRA module of rank r~ (U
-// d_out x r~ row-major like B, V^T r~ x d_in row-major like A), so orthogonalize
-// runs the factor-construction TSQR (Gram leaf, Householder fallback) on it and
-// forms Q = X R^-1 here; two rounds (CholeskyQR2) make Q orthonormal to fp32
-// rounding for any numerically full-rank X.
+// d_out x r~ row-major like B, V^T r~ x d_in row-major like A), so orthogonalize is
+// the factor-construction TSQR on it followed by Q = X R^-1: the update kernel's
+// epilogue forms the Gram of each finished 128-row tile (the TSQR leaf), the tiles are
+// merged in order and the fp64 Cholesky is taken (the root), and Q = X R^-1 uses that
+// fp64 R (orthonormal to ~kappa^2 u_64 + u_32).  A matrix whose pivot is rejected
+// gets its R from the Householder TSQR kernel instead and a second round (Gram leaf +
+// Cholesky on Q_1, then Q = Q_1 R_2^-1: CholeskyQR2) restores orthonormality.
 //
 // Kernels of one step, all fp64 on the tensor-core path (mma.m8n8k4.f64: every
 // product of two fp32 values is exact, sums are fp64):
@@ -22,8 +25,11 @@
 //   jd_core_kernel     per member: S, W = w P S, Z = w Q S^T (and Sigma = S^T).
 //   jd_update_kernel   per (problem, factor, 128-row tile): sum over members of
 //                      X_tile W_i (or A_i^T Z_i) -> U_0 rows (or V_0^T columns).
-//   jd_qform_kernel    per (problem, factor, 128-row tile): Q = X R^-1 by forward
-//                      substitution in fp64, one row per thread.
+//                      Its epilogue writes the tile's Gram.
+//   jd_gram_sum_kernel per (problem, factor, slice of the Gram): tile Grams summed in order.
+//   jd_chol_kernel     per (problem, factor): fp64 Cholesky of the summed Gram.
+//   jd_rinv_kernel     per (problem, factor): R^-1 in fp64.
+//   jd_qform_kernel    per (problem, factor, 128-row tile): Q = X R^-1 (fp64 tensor cores).
 #pragma once
 #include "common.cuh"
 #include "tc.cuh"
@@ -254,7 +260,8 @@ __global__ void __launch_bounds__(256) jd_core_kernel(JdCoreArgs a) {
     extern __shared__ __align__(16) double js[];
     double* P = js;                  // RX x RY
     double* Q = P + RX * RY;
-    double* S = Q + RX * RY;         // RY x RY (jd_core_smem)
+    double* S = Q + RX * RY;         // RY x (RY + 1): the padded stride keeps S[j][m] reads over j conflict-free
+    constexpr int LS = RY + 1;
     const int g = blockIdx.x, tid = threadIdx.x;
     const JdMember mb = a.members[g];
     const int r = a.mods[mb.mod].r, rt = a.basis[mb.prob].r;
@@ -268,8 +275,9 @@ __global__ void __launch_bounds__(256) jd_core_kernel(JdCoreArgs a) {
     for (int e = tid; e < rt * rt; e += 256) {
         const int i = e / rt, j = e - i * rt;
         double s = 0.0;
+#pragma unroll 4
         for (int l = 0; l < r; ++l) s = fma(P[l * RY + i], Q[l * RY + j], s);
-        S[i * RY + j] = s;
+        S[i * LS + j] = s;
     }
     __syncthreads();
     if (a.sigma) {
@@ -277,7 +285,7 @@ __global__ void __launch_bounds__(256) jd_core_kernel(JdCoreArgs a) {
         float* out = a.sigma + pd.sigma_off + (int64_t)mb.local * rt * rt;
         for (int e = tid; e < rt * rt; e += 256) {
             const int i = e / rt, j = e - i * rt;
-            out[e] = (float)S[j * RY + i];
+            out[e] = (float)S[j * LS + i];
         }
     }
     if (!a.write_wz) return;
@@ -288,9 +296,10 @@ __global__ void __launch_bounds__(256) jd_core_kernel(JdCoreArgs a) {
         const int l = e / RY, j = e - l * RY;
         double sw = 0.0, sz = 0.0;
         if (l < r && j < rt) {
+#pragma unroll 4
             for (int m = 0; m < rt; ++m) {
-                sw = fma(P[l * RY + m], S[m * RY + j], sw);
-                sz = fma(Q[l * RY + m], S[j * RY + m], sz);
+                sw = fma(P[l * RY + m], S[m * LS + j], sw);
+                sz = fma(Q[l * RY + m], S[j * LS + m], sz);
             }
         }
         W[e] = (float)(w * sw);
@@ -300,7 +309,7 @@ __global__ void __launch_bounds__(256) jd_core_kernel(JdCoreArgs a) {
 
 template <int RX, int RY>
 __host__ __device__ constexpr size_t jd_core_smem() {
-    return (size_t)(2 * RX * RY + RY * RY) * sizeof(double);
+    return (size_t)(2 * RX * RY + RY * (RY + 1)) * sizeof(double);
 }
 
 template <int RX, int RY>
@@ -311,9 +320,16 @@ template <int RX, int RY>
 __host__ __device__ constexpr int jd_update_stage_floats() {
     return jd_update_x_floats<RX, RY>() + RX * (RY + 8);
 }
+// Epilogue buffers: the finished tile (fp32, [kJdTR][RY + 8]) and the packed Gram sum.
+template <int RY>
+__host__ __device__ constexpr size_t jd_epilogue_bytes() {
+    return (size_t)kJdTR * (RY + 8) * sizeof(float) + (size_t)tri_size<RY>() * sizeof(double);
+}
 template <int RX, int RY>
 __host__ __device__ constexpr size_t jd_update_smem() {
-    return 2 * (size_t)jd_update_stage_floats<RX, RY>() * sizeof(float);
+    return 2 * (size_t)jd_update_stage_floats<RX, RY>() * sizeof(float) > jd_epilogue_bytes<RY>()
+               ? 2 * (size_t)jd_update_stage_floats<RX, RY>() * sizeof(float)
+               : jd_epilogue_bytes<RY>();
 }
 
 struct JdUpdArgs {
@@ -327,6 +343,7 @@ struct JdUpdArgs {
     const JdTile* tiles;
     float* U_ws;
     float* Vt_ws;
+    double* gram;                // per tile: packed upper Gram of the finished (fp32) tile, tri_size<RY>()
 };
 
 // Stage the member's rows of X (kJdTR rows) and its W (or Z) (r x RY) into one buffer.
@@ -447,10 +464,314 @@ __global__ void __launch_bounds__(128) jd_update_kernel(JdUpdArgs a) {
         __syncthreads();   // the buffer is refilled by the next iteration's issue
     }
     tc::cp_async_wait<0>();
+    __syncthreads();
+    // epilogue: round the tile to fp32 in shared memory, store it, and form its Gram
+    // (the first, row-tile level of the orthogonalize TSQR) from the stored values
+    constexpr int LT = RY + 8;
+    float* tile = us;
     const int rt = bw.r;
 #pragma unroll
     for (int bm = 0; bm < 4; ++bm) {
         const int row = 32 * warp + 8 * bm + (lane >> 2);
+#pragma unroll
+        for (int bn = 0; bn < NBN; ++bn)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const int c = 8 * bn + 2 * (lane & 3) + e;
+                tile[row * LT + c] = (row < tl.nrows && c < rt) ? (float)acc[bm][bn][e] : 0.f;
+            }
+    }
+    __syncthreads();
+    if (tl.f == 0) {
+        float* out = a.U_ws + bw.B_off + (int64_t)tl.row0 * rt;
+        for (int i = tid; i < tl.nrows * rt; i += 128) {
+            const int row = i / rt, c = i - row * rt;
+            out[i] = tile[row * LT + c];
+        }
+    } else {
+        for (int i = tid; i < rt * tl.nrows; i += 128) {
+            const int c = i / tl.nrows, row = i - c * tl.nrows;
+            a.Vt_ws[bw.A_off + (int64_t)c * bw.d_in + tl.row0 + row] = tile[row * LT + c];
+        }
+    }
+    constexpr int NB = RY / 8, NP = NB * (NB + 1) / 2;
+    double g[NP][2];
+#pragma unroll
+    for (int q = 0; q < NP; ++q) g[q][0] = g[q][1] = 0.0;
+    const float* fb = tile + (32 * warp + (lane & 3)) * LT + (lane >> 2);
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+        double f[NB];
+#pragma unroll
+        for (int b = 0; b < NB; ++b) f[b] = (double)fb[ks * 4 * LT + 8 * b];
+        int q = 0;
+#pragma unroll
+        for (int bi = 0; bi < NB; ++bi)
+#pragma unroll
+            for (int bj = bi; bj < NB; ++bj) dmma_8x8x4(g[q++], f[bi], f[bj]);
+    }
+    double* red = reinterpret_cast<double*>(tile + kJdTR * LT);
+    for (int w = 0; w < 4; ++w) {   // the four warps' row blocks, summed in order
+        if (warp == w) {
+            const int m = lane >> 2, n2 = 2 * (lane & 3);
+            int q = 0;
+#pragma unroll
+            for (int bi = 0; bi < NB; ++bi)
+#pragma unroll
+                for (int bj = bi; bj < NB; ++bj, ++q)
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const int row = 8 * bi + m, col = 8 * bj + n2 + e;
+                        if (col >= row) {
+                            const int o = tri_off<RY>(row, col);
+                            red[o] = (w == 0 ? 0.0 : red[o]) + g[q][e];
+                        }
+                    }
+        }
+        __syncthreads();
+    }
+    double* slot = a.gram + (int64_t)blockIdx.x * tri_size<RY>();
+    for (int e = tid; e < tri_size<RY>(); e += 128) slot[e] = red[e];
+}
+
+// Per (problem, factor): the tile Grams summed in tile order (one thread per packed
+// entry, CTAs over slices of the triangle).
+struct JdGramSumArgs {
+    const int32_t* tile0;    // per mf: first tile (tiles of one mf are consecutive)
+    const int32_t* ntiles;   // per mf
+    const double* gram;      // per tile
+    double* G;               // per mf: packed Gram
+};
+
+template <int RT>
+__global__ void __launch_bounds__(128) jd_gram_sum_kernel(JdGramSumArgs a) {
+    constexpr int TRI = tri_size<RT>();
+    const int mf = blockIdx.x, e = blockIdx.y * 128 + threadIdx.x;
+    if (e >= TRI) return;
+    const int nt = a.ntiles[mf];
+    const double* src = a.gram + (int64_t)a.tile0[mf] * TRI + e;
+    double s = 0.0;
+#pragma unroll 8
+    for (int t = 0; t < nt; ++t) s += src[(int64_t)t * TRI];
+    a.G[(int64_t)mf * TRI + e] = s;
+}
+
+// Upper-triangular inverse of the r x r R held in the upper triangle of `A` (dense,
+// stride RT + 1), by rows from the last: row i of R^-1 needs only rows > i.  Entry
+// (l, j), l < j, is written to A[j][l] (the unused lower triangle), the diagonal to
+// `dinv`.  Called by all `nt` threads of the block; columns j >= bad are zero.
+// Four threads share each entry's dot product (strided terms, combined by shuffles in a
+// fixed order); nt must be a multiple of 128.
+template <int RT>
+__device__ __forceinline__ void jd_upper_inverse(double (*A)[RT + 1], double* dinv, int r, int bad, int tid, int nt) {
+    const int part = tid & 3;
+    for (int i = r - 1; i >= 0; --i) {
+        for (int j0 = i; j0 < i + RT; j0 += nt / 4) {   // uniform trip count: shuffles stay converged
+            const int j = j0 + (tid >> 2);
+            const bool live = j < r;
+            double v = 0.0;
+            if (live && j > i && j < bad) {
+                if (part == 0) v = A[i][j] * dinv[j];   // l = j term
+                for (int l = i + 1 + part; l < j; l += 4) v = fma(A[i][l], A[j][l], v);
+            }
+            v += __shfl_xor_sync(0xffffffffu, v, 1);
+            v += __shfl_xor_sync(0xffffffffu, v, 2);
+            if (live && part == 0) {
+                if (j >= bad) {
+                    if (j == i) dinv[i] = 0.0;
+                    else A[j][i] = 0.0;
+                } else if (j == i) {
+                    dinv[i] = 1.0 / A[i][i];
+                } else {
+                    A[j][i] = -v / A[i][i];
+                }
+            }
+        }
+        __syncthreads();
+    }
+}
+
+template <int RT>
+__device__ __forceinline__ void jd_store_inverse(const double (*A)[RT + 1], const double* dinv, int r, double* out,
+                                                 int rs, int tid, int nt) {
+    for (int e = tid; e < rs * rs; e += nt) {
+        const int l = e / rs, j = e - l * rs;
+        out[e] = (l < r && j < r && j >= l) ? (j == l ? dinv[l] : A[j][l]) : 0.0;
+    }
+}
+
+// Per (problem, factor), 256 threads: G = R^T R by fp64 Cholesky (the TSQR root; the
+// same pivot rule as the Gram leaf), then R^-1.  A rejected pivot marks the matrix in
+// `flags`; its R then comes from the Householder TSQR and jd_rinv_kernel inverts it.
+struct JdCholArgs {
+    const lf_module* basis;
+    const double* G;         // per mf: packed Gram
+    double* Rinv;            // per mf: rs x rs
+    int32_t* flags;          // per mf, zero on entry
+    int32_t rs;
+};
+
+template <int RT>
+__global__ void __launch_bounds__(256) jd_chol_kernel(JdCholArgs a) {
+    __shared__ double A[RT][RT + 1];
+    __shared__ double s_diag[RT];
+    __shared__ double dinv[RT];
+    __shared__ int s_fail;
+    const int mf = blockIdx.x, tid = threadIdx.x;
+    const int r = a.basis[mf >> 1].r;
+    const double* Gp = a.G + (int64_t)mf * tri_size<RT>();
+    for (int e = tid; e < RT * RT; e += 256) {
+        const int j = e / RT, c = e - j * RT;
+        if (c >= j) A[j][c] = Gp[tri_off<RT>(j, c)];
+    }
+    if (tid < RT) s_diag[tid] = Gp[tri_off<RT>(tid, tid)];
+    if (tid == 0) s_fail = 0;
+    __syncthreads();
+    for (int j = 0; j < r; ++j) {
+        if (tid == 0) {
+            const double d = A[j][j];
+            if (!(d > kGramPivotTol * s_diag[j])) s_fail = 1;
+            else A[j][j] = sqrt(d);
+        }
+        __syncthreads();
+        if (s_fail) {
+            if (tid == 0) a.flags[mf] = 1;
+            return;
+        }
+        const double rjj = A[j][j];
+        for (int c = j + 1 + tid; c < r; c += 256) A[j][c] /= rjj;
+        __syncthreads();
+        // trailing update of rows k > j: 8 warps over rows, lanes over columns
+        for (int k = j + 1 + (tid >> 5); k < r; k += 8) {
+            const double gjk = A[j][k];
+            for (int c = k + (tid & 31); c < r; c += 32) A[k][c] -= gjk * A[j][c];
+        }
+        __syncthreads();
+    }
+    jd_upper_inverse<RT>(A, dinv, r, r, tid, 256);
+    jd_store_inverse<RT>(A, dinv, r, a.Rinv + (int64_t)mf * a.rs * a.rs, a.rs, tid, 256);
+}
+
+// Per (problem, factor) whose R comes from elsewhere: R^-1 of the Householder TSQR's
+// fp32 R (use32[mf] set) or of an fp64 R.  A diagonal entry that is not positive and
+// finite (the update is numerically rank deficient) latches LF_ERR_NUMERIC; the columns
+// from there on are zero.
+struct JdRinvArgs {
+    const lf_module* basis;
+    const int32_t* only;     // per mf (nullable): zero = skip
+    const int32_t* use32;    // per mf
+    const double* R64;       // per mf, rs x rs
+    const float* R_B;        // per problem, rs x rs
+    const float* R_A;
+    double* Rinv;            // per mf, rs x rs
+    int32_t rs;
+};
+
+template <int RT>
+__global__ void __launch_bounds__(128) jd_rinv_kernel(JdRinvArgs a) {
+    __shared__ double A[RT][RT + 1];
+    __shared__ double dinv[RT];
+    const int mf = blockIdx.x, tid = threadIdx.x;
+    if (a.only && a.only[mf] == 0) return;
+    const int r = a.basis[mf >> 1].r;
+    for (int e = tid; e < r * r; e += 128) {
+        const int j = e / r, c = e - j * r;
+        if (c >= j)
+            A[j][c] = a.use32[mf] ? (double)((mf & 1) == 0 ? a.R_B : a.R_A)[(int64_t)(mf >> 1) * a.rs * a.rs + j * a.rs + c]
+                                  : a.R64[(int64_t)mf * a.rs * a.rs + j * a.rs + c];
+    }
+    __syncthreads();
+    int bad = r;
+    for (int j = 0; j < r; ++j)
+        if (!(A[j][j] > 0.0) || !isfinite(A[j][j])) {
+            bad = j;
+            break;
+        }
+    if (bad < r && tid == 0) latch_error(LF_ERR_NUMERIC);
+    jd_upper_inverse<RT>(A, dinv, r, bad, tid, 128);
+    jd_store_inverse<RT>(A, dinv, r, a.Rinv + (int64_t)mf * a.rs * a.rs, a.rs, tid, 128);
+}
+
+struct JdQArgs {
+    const lf_module* src;    // per problem: B_off / A_off of X in src_U / src_Vt
+    const float* src_U;
+    const float* src_Vt;
+    const lf_module* dst;    // per problem: where Q goes
+    float* dst_U;
+    float* dst_Vt;
+    const lf_module* alt;    // per problem: where Q goes when route[mf] != 0
+    float* alt_U;
+    float* alt_Vt;
+    const int32_t* route;    // per mf (nullable)
+    const int32_t* only;     // per mf (nullable): zero = leave this matrix alone
+    const double* Rinv;      // per mf, rs x rs
+    int32_t rs;
+    const JdTile* tiles;
+};
+
+template <int RT>
+__host__ __device__ constexpr size_t jd_qform_smem() {
+    return (size_t)kJdTR * (RT + 4) * sizeof(float) + (size_t)RT * (RT + 8) * sizeof(double);
+}
+
+// Q = X R^-1 on one 128-row tile: a fp64 tensor-core product of the staged fp32 tile
+// with the fp64 R^-1, 4 warps of 32 rows.
+template <int RT>
+__global__ void __launch_bounds__(kJdTR) jd_qform_kernel(JdQArgs a) {
+    extern __shared__ __align__(16) double qs[];
+    constexpr int LX = RT + 4, LR = RT + 8, NBN = RT / 8;
+    double* sRi = qs;                                           // RT x LR
+    float* sx = reinterpret_cast<float*>(qs + RT * LR);         // kJdTR x LX
+    const JdTile tl = a.tiles[blockIdx.x];
+    const int mf = 2 * tl.p + tl.f;
+    if (a.only && a.only[mf] == 0) return;
+    const lf_module s = a.src[tl.p];
+    const bool to_alt = a.route && a.route[mf] != 0;
+    const lf_module d = to_alt ? a.alt[tl.p] : a.dst[tl.p];
+    float* dU = to_alt ? a.alt_U : a.dst_U;
+    float* dVt = to_alt ? a.alt_Vt : a.dst_Vt;
+    const int rt = s.r, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const double* Ri = a.Rinv + (int64_t)mf * a.rs * a.rs;
+    for (int e = tid; e < RT * RT; e += kJdTR) {
+        const int i = e / RT, j = e - i * RT;
+        sRi[i * LR + j] = (i < rt && j < rt) ? Ri[i * a.rs + j] : 0.0;
+    }
+    if (tl.f == 0) {
+        const float* x = a.src_U + s.B_off + (int64_t)tl.row0 * rt;
+        for (int e = tid; e < kJdTR * RT; e += kJdTR) {
+            const int i = e / RT, c = e - i * RT;
+            sx[i * LX + c] = (i < tl.nrows && c < rt) ? x[i * rt + c] : 0.f;
+        }
+    } else {
+        const float* x = a.src_Vt + s.A_off + tl.row0;
+        for (int e = tid; e < kJdTR * RT; e += kJdTR) {
+            const int c = e / kJdTR, i = e - c * kJdTR;
+            sx[i * LX + c] = (i < tl.nrows && c < rt) ? x[(int64_t)c * s.d_in + i] : 0.f;
+        }
+    }
+    __syncthreads();
+    double acc[4][NBN][2];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < NBN; ++j) acc[i][j][0] = acc[i][j][1] = 0.0;
+    const int rl = 32 * warp + (lane >> 2);
+#pragma unroll
+    for (int ks = 0; ks < RT / 4; ++ks) {
+        const int l = 4 * ks + (lane & 3);
+        double xa[4], rb[NBN];
+#pragma unroll
+        for (int bm = 0; bm < 4; ++bm) xa[bm] = (double)sx[(rl + 8 * bm) * LX + l];
+#pragma unroll
+        for (int bn = 0; bn < NBN; ++bn) rb[bn] = sRi[l * LR + 8 * bn + (lane >> 2)];
+#pragma unroll
+        for (int bm = 0; bm < 4; ++bm)
+#pragma unroll
+            for (int bn = 0; bn < NBN; ++bn) dmma_8x8x4(acc[bm][bn], xa[bm], rb[bn]);
+    }
+#pragma unroll
+    for (int bm = 0; bm < 4; ++bm) {
+        const int row = rl + 8 * bm;
         if (row >= tl.nrows) continue;
         const int64_t grow = tl.row0 + row;
 #pragma unroll
@@ -460,82 +781,10 @@ __global__ void __launch_bounds__(128) jd_update_kernel(JdUpdArgs a) {
                 const int c = 8 * bn + 2 * (lane & 3) + e;
                 if (c >= rt) continue;
                 if (tl.f == 0)
-                    a.U_ws[bw.B_off + grow * rt + c] = (float)acc[bm][bn][e];
+                    dU[d.B_off + grow * rt + c] = (float)acc[bm][bn][e];
                 else
-                    a.Vt_ws[bw.A_off + (int64_t)c * bw.d_in + grow] = (float)acc[bm][bn][e];
+                    dVt[d.A_off + (int64_t)c * d.d_in + grow] = (float)acc[bm][bn][e];
             }
-    }
-}
-
-struct JdQArgs {
-    const lf_module* src;    // per problem: B_off / A_off of X in src_U / src_Vt
-    const lf_module* dst;    // per problem: B_off / A_off of Q in dst_U / dst_Vt
-    const float* src_U;
-    const float* src_Vt;
-    float* dst_U;
-    float* dst_Vt;
-    const float* R_B;        // per problem, rs x rs upper-triangular
-    const float* R_A;
-    int32_t rs;
-    const JdTile* tiles;
-};
-
-// Q = X R^-1, one row of X per thread (forward substitution in fp64).  A diagonal
-// entry of R that is not positive and finite (X numerically rank deficient) latches
-// LF_ERR_NUMERIC and zeroes the columns from there on.
-template <int RT>
-__global__ void __launch_bounds__(kJdTR) jd_qform_kernel(JdQArgs a) {
-    __shared__ double sR[RT][RT + 1];
-    __shared__ double sInv[RT];
-    const JdTile tl = a.tiles[blockIdx.x];
-    const lf_module s = a.src[tl.p], d = a.dst[tl.p];
-    const int rt = s.r, tid = threadIdx.x;
-    const float* R = (tl.f == 0 ? a.R_B : a.R_A) + (int64_t)tl.p * a.rs * a.rs;
-    for (int e = tid; e < rt * rt; e += kJdTR) {
-        const int i = e / rt, j = e - i * rt;
-        sR[i][j] = (double)R[i * a.rs + j];
-    }
-    __syncthreads();
-    int bad = rt;
-    for (int j = 0; j < rt; ++j)
-        if (!(sR[j][j] > 0.0) || !isfinite(sR[j][j])) {
-            bad = j;
-            break;
-        }
-    if (tid < rt) sInv[tid] = tid < bad ? 1.0 / sR[tid][tid] : 0.0;
-    if (bad < rt && tid == 0 && blockIdx.x == 0) latch_error(LF_ERR_NUMERIC);
-    __syncthreads();
-    const int row = tl.row0 + tid;
-    if (tid >= tl.nrows) return;
-    double q[RT];
-    if (tl.f == 0) {
-        const float* x = a.src_U + s.B_off + (int64_t)row * rt;
-#pragma unroll
-        for (int c = 0; c < RT; ++c) q[c] = c < rt ? (double)x[c] : 0.0;
-    } else {
-        const float* x = a.src_Vt + s.A_off + row;
-#pragma unroll
-        for (int c = 0; c < RT; ++c) q[c] = c < rt ? (double)x[(int64_t)c * s.d_in] : 0.0;
-    }
-#pragma unroll
-    for (int j = 0; j < RT; ++j) {
-        if (j < rt) {
-            double v = q[j];
-#pragma unroll
-            for (int l = 0; l < j; ++l) v = fma(-q[l], sR[l][j], v);
-            q[j] = j < bad ? v * sInv[j] : 0.0;
-        }
-    }
-    if (tl.f == 0) {
-        float* y = a.dst_U + d.B_off + (int64_t)row * rt;
-#pragma unroll
-        for (int c = 0; c < RT; ++c)
-            if (c < rt) y[c] = (float)q[c];
-    } else {
-        float* y = a.dst_Vt + d.A_off + row;
-#pragma unroll
-        for (int c = 0; c < RT; ++c)
-            if (c < rt) y[(int64_t)c * d.d_in] = (float)q[c];
     }
 }
 

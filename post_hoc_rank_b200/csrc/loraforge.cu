@@ -546,6 +546,7 @@ struct JdPlan {
     std::vector<TsqrInfo> pinfo;
     int32_t pslots = 0;
     std::vector<JdTile> tiles;
+    std::vector<int32_t> tile0, ntiles;   // per mf = 2 * problem + factor
     TsqrPlan orth;
     int RX = 16, RY = 16;
     int64_t ws_U = 0, ws_Vt = 0;   // floats of the workspace copies of the state
@@ -591,6 +592,8 @@ static void plan_jd(const lf_module* mods, const int32_t* members, const lf_jd_p
         P.ws_Vt += align_up((int64_t)q.rank * q.d_in, 4);
         for (int f = 0; f < 2; ++f) {
             const int rows = f == 0 ? q.d_out : q.d_in;
+            P.tile0.push_back((int32_t)P.tiles.size());
+            P.ntiles.push_back((int32_t)cdiv(rows, kJdTR));
             for (int r0 = 0; r0 < rows; r0 += kJdTR) P.tiles.push_back(JdTile{p, f, r0, std::min(kJdTR, rows - r0)});
         }
     }
@@ -616,8 +619,8 @@ static void plan_jd(const lf_module* mods, const int32_t* members, const lf_jd_p
 }
 
 struct JdLayout {
-    size_t mods, members, probs, basis_user, basis_ws, pwork, pinfo, tiles, owork, onwork, oinfo;
-    size_t pcounters, ocounters, ppartial, opartial, QP, WZ, wsU, wsVt, RB, RA, total;
+    size_t mods, members, probs, basis_user, basis_ws, pwork, pinfo, tiles, tile0, ntiles, owork, onwork, oinfo;
+    size_t pcounters, ocounters, ppartial, opartial, tgram, gsum, QP, WZ, wsU, wsVt, RB, RA, R64, Rinv, total;
 };
 
 static JdLayout jd_layout(int32_t n_mods, int32_t n_probs, const JdPlan& P) {
@@ -639,19 +642,27 @@ static JdLayout jd_layout(int32_t n_mods, int32_t n_probs, const JdPlan& P) {
     LF_TAKE(pwork, TsqrWork, P.pwork.size());
     LF_TAKE(pinfo, TsqrInfo, P.pinfo.size());
     LF_TAKE(tiles, JdTile, P.tiles.size());
+    LF_TAKE(tile0, int32_t, P.tile0.size());
+    LF_TAKE(ntiles, int32_t, P.ntiles.size());
     LF_TAKE(owork, TsqrWork, P.orth.work.size());
     LF_TAKE(onwork, int32_t, 1);
     LF_TAKE(oinfo, TsqrInfo, P.orth.info.size());
     LF_TAKE(pcounters, int32_t, 2 * ng);
-    LF_TAKE(ocounters, int32_t, (size_t)12 * n_probs);   // two orthogonalize rounds x (Gram, Householder, flags)
+    // orthogonalize: flags of round 1, Gram counters of round 2, Householder counters of
+    // both rounds, flags of round 2 (2 per problem each), zeroed every step
+    LF_TAKE(ocounters, int32_t, (size_t)10 * n_probs);
     LF_TAKE(ppartial, double, (size_t)P.pslots * blk);
     LF_TAKE(opartial, char, (size_t)P.orth.slots * tsqr_slot_bytes(P.orth.RT));
+    LF_TAKE(tgram, double, P.tiles.size() * (size_t)(P.RY * (P.RY + 1) / 2));
+    LF_TAKE(gsum, double, (size_t)2 * n_probs * (P.RY * (P.RY + 1) / 2));
     LF_TAKE(QP, double, 2 * ng * blk);
     LF_TAKE(WZ, float, 2 * ng * blk);
     LF_TAKE(wsU, float, (size_t)P.ws_U);
     LF_TAKE(wsVt, float, (size_t)P.ws_Vt);
     LF_TAKE(RB, float, (size_t)n_probs * rs2);
     LF_TAKE(RA, float, (size_t)n_probs * rs2);
+    LF_TAKE(R64, double, (size_t)4 * n_probs * rs2);   // two rounds x two factors
+    LF_TAKE(Rinv, double, (size_t)2 * n_probs * rs2);
 #undef LF_TAKE
     L.total = c.off + 256;
     return L;
@@ -692,11 +703,45 @@ static cudaError_t launch_jd(int RX, int RY, int which, const void* args, int gr
     return launch_jd_rx<64>(RY, which, args, grid, st);
 }
 
+template <int RT>
+static cudaError_t launch_jd_qform_rt(const JdQArgs& a, int grid, cudaStream_t st) {
+    auto k = jd_qform_kernel<RT>;
+    constexpr size_t smem = jd_qform_smem<RT>();
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    LF_LAUNCH("jd_qform", k, grid, kJdTR, smem, st, a);
+    return cudaGetLastError();
+}
+
 static cudaError_t launch_jd_qform(int RT, const JdQArgs& a, int grid, cudaStream_t st) {
     if (grid <= 0) return cudaSuccess;
-    if (RT == 16) LF_LAUNCH("jd_qform", jd_qform_kernel<16>, grid, kJdTR, 0, st, a);
-    else if (RT == 32) LF_LAUNCH("jd_qform", jd_qform_kernel<32>, grid, kJdTR, 0, st, a);
-    else LF_LAUNCH("jd_qform", jd_qform_kernel<64>, grid, kJdTR, 0, st, a);
+    if (RT == 16) return launch_jd_qform_rt<16>(a, grid, st);
+    if (RT == 32) return launch_jd_qform_rt<32>(a, grid, st);
+    return launch_jd_qform_rt<64>(a, grid, st);
+}
+
+static cudaError_t launch_jd_gram_sum(int RT, const JdGramSumArgs& a, int n_mf, cudaStream_t st) {
+    if (n_mf <= 0) return cudaSuccess;
+    const dim3 grid(n_mf, (unsigned)cdiv(RT * (RT + 1) / 2, 128));
+    if (RT == 16) LF_LAUNCH("jd_gram_sum", jd_gram_sum_kernel<16>, grid, 128, 0, st, a);
+    else if (RT == 32) LF_LAUNCH("jd_gram_sum", jd_gram_sum_kernel<32>, grid, 128, 0, st, a);
+    else LF_LAUNCH("jd_gram_sum", jd_gram_sum_kernel<64>, grid, 128, 0, st, a);
+    return cudaGetLastError();
+}
+
+static cudaError_t launch_jd_rinv(int RT, const JdRinvArgs& a, int grid, cudaStream_t st) {
+    if (grid <= 0) return cudaSuccess;
+    if (RT == 16) LF_LAUNCH("jd_rinv", jd_rinv_kernel<16>, grid, 128, 0, st, a);
+    else if (RT == 32) LF_LAUNCH("jd_rinv", jd_rinv_kernel<32>, grid, 128, 0, st, a);
+    else LF_LAUNCH("jd_rinv", jd_rinv_kernel<64>, grid, 128, 0, st, a);
+    return cudaGetLastError();
+}
+
+static cudaError_t launch_jd_chol(int RT, const JdCholArgs& a, int grid, cudaStream_t st) {
+    if (grid <= 0) return cudaSuccess;
+    if (RT == 16) LF_LAUNCH("jd_chol", jd_chol_kernel<16>, grid, 256, 0, st, a);
+    else if (RT == 32) LF_LAUNCH("jd_chol", jd_chol_kernel<32>, grid, 256, 0, st, a);
+    else LF_LAUNCH("jd_chol", jd_chol_kernel<64>, grid, 256, 0, st, a);
     return cudaGetLastError();
 }
 
@@ -757,6 +802,8 @@ lf_status lf_tsqr_batched(const lf_module* mods, int32_t n, const float* B_base,
     ga.R_B = R_B;
     ga.R_A = R_A;
     ga.rs = p.rs;
+    ga.only = nullptr;
+    ga.R64 = nullptr;
     LF_CUDA_TRY(launch_gram_rt(p.RT, ga, nwork, s));
 
     // structured-Householder TSQR for the matrices whose Gram Cholesky was rejected
@@ -1188,6 +1235,8 @@ lf_status lf_jd_full(const lf_module* mods, int32_t n_mods, const int32_t* membe
     h.put(P.pwork.data(), P.pwork.size());
     h.put(P.pinfo.data(), P.pinfo.size());
     h.put(P.tiles.data(), P.tiles.size());
+    h.put(P.tile0.data(), P.tile0.size());
+    h.put(P.ntiles.data(), P.ntiles.size());
     h.put(P.orth.work.data(), P.orth.work.size());
     h.put(&onwork, 1);
     h.put(P.orth.info.data(), P.orth.info.size());
@@ -1242,63 +1291,120 @@ lf_status lf_jd_full(const lf_module* mods, int32_t n_mods, const int32_t* membe
     ua.tiles = reinterpret_cast<const JdTile*>(at(L.tiles));
     ua.U_ws = wsU;
     ua.Vt_ws = wsVt;
+    ua.gram = reinterpret_cast<double*>(at(L.tgram));
 
-    // orthogonalize round: TSQR R of the workspace state, then Q = X R^-1 into dst
-    auto orth_round = [&](int round, const lf_module* dst_tab, float* dst_U, float* dst_Vt) -> cudaError_t {
-        int32_t* cnt = reinterpret_cast<int32_t*>(at(L.ocounters)) + (size_t)6 * n_probs * round;
-        GramArgs ga;
-        ga.mods = d_bw;
-        ga.B_base = wsU;
-        ga.A_base = wsVt;
-        ga.work = reinterpret_cast<const TsqrWork*>(at(L.owork));
-        ga.n_work = reinterpret_cast<const int32_t*>(at(L.onwork));
-        ga.info = reinterpret_cast<const TsqrInfo*>(at(L.oinfo));
-        ga.counters = cnt;
-        ga.partial = reinterpret_cast<double*>(at(L.opartial));
-        ga.slot_doubles = (int64_t)(tsqr_slot_bytes(P.orth.RT) / sizeof(double));
-        ga.flags = cnt + 4 * n_probs;
-        ga.R_B = RB;
-        ga.R_A = RA;
-        ga.rs = P.orth.rs;
-        cudaError_t e = launch_gram_rt(P.orth.RT, ga, onwork, s);
-        if (e != cudaSuccess) return e;
+    // orthogonalize (the state in the workspace -> the caller's U, V^T).  Round 1: tile
+    // Grams (update epilogue) -> jd_chol -> Householder TSQR for rejected matrices ->
+    // Q = X R^-1, written to the caller's state, or back into the workspace for the
+    // rejected ones, which round 2 (Gram leaf + Cholesky on Q_1, Householder if
+    // rejected again, Q = Q_1 R_2^-1) finishes.  Round-2 kernels skip every other matrix.
+    const size_t rs2 = (size_t)P.orth.rs * P.orth.rs;
+    int32_t* oc = reinterpret_cast<int32_t*>(at(L.ocounters));
+    int32_t* flags1 = oc;
+    int32_t* gram2_cnt = oc + 2 * n_probs;
+    int32_t* hh1_cnt = oc + 4 * n_probs;
+    int32_t* hh2_cnt = oc + 6 * n_probs;
+    int32_t* flags2 = oc + 8 * n_probs;
+    double* R64_1 = reinterpret_cast<double*>(at(L.R64));
+    double* R64_2 = R64_1 + 2 * n_probs * rs2;
+    const TsqrWork* owork = reinterpret_cast<const TsqrWork*>(at(L.owork));
+    const int32_t* onw = reinterpret_cast<const int32_t*>(at(L.onwork));
+    const TsqrInfo* oinfo = reinterpret_cast<const TsqrInfo*>(at(L.oinfo));
+
+    JdGramSumArgs gsa;
+    gsa.tile0 = reinterpret_cast<const int32_t*>(at(L.tile0));
+    gsa.ntiles = reinterpret_cast<const int32_t*>(at(L.ntiles));
+    gsa.gram = ua.gram;
+    gsa.G = reinterpret_cast<double*>(at(L.gsum));
+    double* Rinv = reinterpret_cast<double*>(at(L.Rinv));
+    JdCholArgs cha;
+    cha.basis = d_bw;
+    cha.G = gsa.G;
+    cha.Rinv = Rinv;
+    cha.flags = flags1;
+    cha.rs = P.orth.rs;
+    JdRinvArgs ra1;   // round 1: only the matrices the Cholesky rejected (Householder R)
+    ra1.basis = d_bw;
+    ra1.only = flags1;
+    ra1.use32 = flags1;
+    ra1.R64 = R64_1;
+    ra1.R_B = RB;
+    ra1.R_A = RA;
+    ra1.Rinv = Rinv;
+    ra1.rs = P.orth.rs;
+    JdRinvArgs ra2 = ra1;
+    ra2.only = flags1;
+    ra2.use32 = flags2;
+    ra2.R64 = R64_2;
+
+    auto householder = [&](const int32_t* only, int32_t* counters) -> cudaError_t {
         TsqrArgs<float> ta;
         ta.mods = d_bw;
         ta.mod_ids = nullptr;
         ta.B_base = wsU;
         ta.A_base = wsVt;
-        ta.work = ga.work;
-        ta.n_work = ga.n_work;
-        ta.info = ga.info;
-        ta.counters = cnt + 2 * n_probs;
+        ta.work = owork;
+        ta.n_work = onw;
+        ta.info = oinfo;
+        ta.counters = counters;
         ta.partial = reinterpret_cast<float*>(at(L.opartial));
         ta.R_B = RB;
         ta.R_A = RA;
         ta.rs = P.orth.rs;
-        ta.only = ga.flags;
-        e = launch_tsqr_rt<float>(P.orth.RT, ta, onwork, s);
-        if (e != cudaSuccess) return e;
-        JdQArgs qa;
-        qa.src = d_bw;
-        qa.dst = dst_tab;
-        qa.src_U = wsU;
-        qa.src_Vt = wsVt;
-        qa.dst_U = dst_U;
-        qa.dst_Vt = dst_Vt;
-        qa.R_B = RB;
-        qa.R_A = RA;
-        qa.rs = P.orth.rs;
-        qa.tiles = ua.tiles;
-        return launch_jd_qform(P.orth.RT, qa, ntile, s);
+        ta.only = only;
+        return launch_tsqr_rt<float>(P.orth.RT, ta, onwork, s);
     };
 
+    GramArgs ga;
+    ga.mods = d_bw;
+    ga.B_base = wsU;
+    ga.A_base = wsVt;
+    ga.work = owork;
+    ga.n_work = onw;
+    ga.info = oinfo;
+    ga.counters = gram2_cnt;
+    ga.partial = reinterpret_cast<double*>(at(L.opartial));
+    ga.slot_doubles = (int64_t)(tsqr_slot_bytes(P.orth.RT) / sizeof(double));
+    ga.flags = flags2;
+    ga.R_B = RB;
+    ga.R_A = RA;
+    ga.rs = P.orth.rs;
+    ga.only = flags1;
+    ga.R64 = R64_2;
+
+    JdQArgs q1;
+    q1.src = d_bw;
+    q1.src_U = wsU;
+    q1.src_Vt = wsVt;
+    q1.dst = d_bu;
+    q1.dst_U = U_base;
+    q1.dst_Vt = Vt_base;
+    q1.alt = d_bw;
+    q1.alt_U = wsU;
+    q1.alt_Vt = wsVt;
+    q1.route = flags1;
+    q1.only = nullptr;
+    q1.Rinv = Rinv;
+    q1.rs = P.orth.rs;
+    q1.tiles = ua.tiles;
+    JdQArgs q2 = q1;
+    q2.route = nullptr;
+    q2.only = flags1;
+
     for (int32_t it = 0; it < iters; ++it) {
+        LF_CUDA_TRY(cudaMemsetAsync(oc, 0, (size_t)10 * n_probs * sizeof(int32_t), s));
         LF_CUDA_TRY(launch_jd(P.RX, P.RY, 0, &pa, npw, s));
         LF_CUDA_TRY(launch_jd(P.RX, P.RY, 1, &ca, ng, s));
         LF_CUDA_TRY(launch_jd(P.RX, P.RY, 2, &ua, ntile, s));
-        LF_CUDA_TRY(cudaMemsetAsync(at(L.ocounters), 0, (size_t)12 * n_probs * sizeof(int32_t), s));
-        LF_CUDA_TRY(orth_round(0, d_bw, wsU, wsVt));
-        LF_CUDA_TRY(orth_round(1, d_bu, U_base, Vt_base));
+        LF_CUDA_TRY(launch_jd_gram_sum(P.RY, gsa, 2 * n_probs, s));
+        LF_CUDA_TRY(launch_jd_chol(P.RY, cha, 2 * n_probs, s));
+        LF_CUDA_TRY(householder(flags1, hh1_cnt));
+        LF_CUDA_TRY(launch_jd_rinv(P.RY, ra1, 2 * n_probs, s));
+        LF_CUDA_TRY(launch_jd_qform(P.RY, q1, ntile, s));
+        LF_CUDA_TRY(launch_gram_rt(P.orth.RT, ga, onwork, s));
+        LF_CUDA_TRY(householder(flags2, hh2_cnt));
+        LF_CUDA_TRY(launch_jd_rinv(P.RY, ra2, 2 * n_probs, s));
+        LF_CUDA_TRY(launch_jd_qform(P.RY, q2, ntile, s));
     }
     if (sigma) {
         LF_CUDA_TRY(launch_jd(P.RX, P.RY, 0, &pa, npw, s));
