@@ -908,6 +908,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-large", action="store_true")
     ap.add_argument("--no-jd", action="store_true")
+    ap.add_argument("--jd-only", action="store_true", help="run only the JD-Full workload and print its record")
     ap.add_argument("--large-adapters", type=int, default=1024)
     args = ap.parse_args()
 
@@ -917,6 +918,15 @@ def main():
 
     if args.impl == "reference":
         return reference_arm(args, rank, world)
+    if args.jd_only:
+        import torch
+        from post_hoc_rank_b200 import build as B
+        B.build()
+        dev = torch.device("cuda", local)
+        torch.cuda.set_device(dev)
+        hbm, _ = peaks()
+        print(json.dumps(jd_bench(dev, torch.cuda.current_stream(), hbm, None, with_cpu=not args.no_cpu)))
+        return
 
     import torch
     from post_hoc_rank_b200 import build as B
