@@ -72,9 +72,6 @@ __device__ __forceinline__ void cp_async16_zfill(void* dst, const void* src, boo
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(n) : "memory");
 }
 
-__device__ __forceinline__ void mbar_arrive1(uint64_t* bar) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
 
 template <int MAXN>
 __global__ void __launch_bounds__(kTcThreads) shrink_tc_kernel(ApplyArgs a) {
