@@ -244,8 +244,10 @@ struct ExpandTcSmem {
     __nv_bfloat16 ahi[kTcM * kMaxRank];          // t_hi, K-major, 16 KB
     __nv_bfloat16 alo[kTcM * kMaxRank];          // t_lo
     __nv_bfloat16 b[2][kMaxRank * kTcN2];        // B'^T tiles, MN-major, 16 KB each
-    __nv_bfloat16 yt[kTcYBuf][kTcM * kTcYLd];    // staged y tiles, 34 KB each
-    float tw[kTcM][kMaxRank + 1];                // summed t rows (Sigma-sandwich only), 33 KB
+    union {
+        __nv_bfloat16 yt[kTcYBuf][kTcM * kTcYLd];    // staged y tiles, 34 KB each
+        float tw[kTcM][kMaxRank + 1];                // summed t rows (Sigma-sandwich only, prologue), 33 KB
+    };
     uint64_t bar;
     uint32_t tmem;
     int32_t toks[kTcM];
