@@ -107,7 +107,11 @@ int32_t lf_rank_stride(const lf_module* mods /*[host]*/, int32_t n);
  *   R_B, R_A : n x rs x rs fp32, entries past r_i are zero.
  *   sigma    : n x rs fp64, descending, zero past r_i.
  *   U, V     : n x rs x rs fp64; column j of U[i] / V[i] pairs with sigma[i][j];
- *              V columns with sigma = 0 are zero.
+ *              U and V columns with sigma = 0 are zero.  The Jacobi sweeps rotate
+ *              the rows of M only (rows end as sigma_j v_j^T); column j of U is
+ *              M v_j / sigma_j, accurate to about 1e-7 sigma_1 / sigma_j, so the
+ *              leading (retained) directions are the accurate ones.  U may be null;
+ *              when it is not, its block also serves as scratch during the call.
  * Workspace: lf_tsqr_workspace_size(mods, n) bytes.  B_base and A_base are fp32. */
 size_t lf_tsqr_workspace_size(const lf_module* mods /*[host]*/, int32_t n);
 lf_status lf_tsqr_batched(const lf_module* mods /*[host]*/, int32_t n,

@@ -281,7 +281,9 @@ template <typename T, int RT>
 struct alignas(16) SvdSmem {
     static constexpr int LD = RT + 16 / (int)sizeof(T);   // 16-byte aligned rows, 4-bank shift per row
     T M[RT][LD];
-    T Ut[RT][LD];   // Ut[p] = column p of U
+    // Ut[p] = column p of U, accumulated by the fp64 refinement only (the fp32 path forms
+    // U at the end and stages R_A here during setup only when it has room: see svd_kernel)
+    T Ut[sizeof(T) == 8 ? RT : 1][LD];
     T sig[RT];
     int perm[RT];
 };
@@ -311,6 +313,113 @@ __host__ __device__ constexpr int svd_warps() { return 1; }
 template <typename T>
 __device__ __forceinline__ T svd_tol(int r) { return T(r) * (sizeof(T) == 8 ? T(2.220446049250313e-16) : T(1.1920929e-7)); }
 
+// One Jacobi rotation of rows p, q of M and of columns p, q of U (fp64 refinement):
+// returns whether the pair was rotated.
+template <typename T, int RT>
+__device__ __forceinline__ bool svd_rotate_acc(SvdSmem<T, RT>& s, int p, int q, int r, T tol) {
+    T al[4] = {0, 0, 0, 0}, be[4] = {0, 0, 0, 0}, ga[4] = {0, 0, 0, 0};
+    const T* mp = s.M[p];
+    const T* mq = s.M[q];
+    int l = 0;
+#pragma unroll 4
+    for (; l + 3 < r; l += 4) {   // four independent chains per sum, 16-byte loads
+        T xv[4], yv[4];
+        ld4(mp + l, xv);
+        ld4(mq + l, yv);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            al[u] = fma(xv[u], xv[u], al[u]);
+            be[u] = fma(yv[u], yv[u], be[u]);
+            ga[u] = fma(xv[u], yv[u], ga[u]);
+        }
+    }
+    for (; l < r; ++l) {
+        const T x = mp[l], y = mq[l];
+        al[0] = fma(x, x, al[0]);
+        be[0] = fma(y, y, be[0]);
+        ga[0] = fma(x, y, ga[0]);
+    }
+    const T alpha = (al[0] + al[1]) + (al[2] + al[3]);
+    const T beta_ = (be[0] + be[1]) + (be[2] + be[3]);
+    const T gamma = (ga[0] + ga[1]) + (ga[2] + ga[3]);
+    if (!(gamma != T(0) && fabs(gamma) > tol * sqrt(alpha * beta_))) return false;
+    const T zeta = (beta_ - alpha) / (T(2) * gamma);
+    const T tt = (zeta >= T(0) ? T(1) : T(-1)) / (fabs(zeta) + sqrt(T(1) + zeta * zeta));
+    const T c = T(1) / sqrt(T(1) + tt * tt);
+    const T sn = c * tt;
+    T* Mp = s.M[p];
+    T* Mq = s.M[q];
+    T* Up = s.Ut[p];
+    T* Uq = s.Ut[q];
+    int k = 0;
+#pragma unroll 2
+    for (; k + 3 < r; k += 4) {   // 16-byte loads and stores of four columns
+        T x[4], y[4], u[4], v[4], x2[4], y2[4], u2[4], v2[4];
+        ld4(Mp + k, x); ld4(Mq + k, y); ld4(Up + k, u); ld4(Uq + k, v);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            x2[e] = c * x[e] - sn * y[e];
+            y2[e] = sn * x[e] + c * y[e];
+            u2[e] = c * u[e] - sn * v[e];
+            v2[e] = sn * u[e] + c * v[e];
+        }
+        st4(Mp + k, x2); st4(Mq + k, y2); st4(Up + k, u2); st4(Uq + k, v2);
+    }
+    for (; k < r; ++k) {
+        const T x = Mp[k], y = Mq[k], u = Up[k], v = Uq[k];
+        Mp[k] = c * x - sn * y;
+        Mq[k] = sn * x + c * y;
+        Up[k] = c * u - sn * v;
+        Uq[k] = sn * u + c * v;
+    }
+    return true;
+}
+
+// One Jacobi rotation of rows p, q of M only (fp32 main path): both rows are read once
+// into registers (16-byte chunks; the row padding past r is zero), the three dot
+// products and the rotation run there, and the rows are written back once.
+template <typename T, int RT>
+__device__ __forceinline__ bool svd_rotate_rows(SvdSmem<T, RT>& s, int p, int q, int r, T tol) {
+    static_assert(sizeof(T) == 4, "register path is fp32");
+    constexpr int NC = RT / 4;
+    float4 x[NC], y[NC];
+    float al[4] = {0.f, 0.f, 0.f, 0.f}, be[4] = {0.f, 0.f, 0.f, 0.f}, ga[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int c = 0; c < NC; ++c) {
+        if (4 * c < r) {
+            x[c] = *reinterpret_cast<const float4*>(&s.M[p][4 * c]);
+            y[c] = *reinterpret_cast<const float4*>(&s.M[q][4 * c]);
+        } else {
+            x[c] = y[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        al[0] = fmaf(x[c].x, x[c].x, al[0]); al[1] = fmaf(x[c].y, x[c].y, al[1]);
+        al[2] = fmaf(x[c].z, x[c].z, al[2]); al[3] = fmaf(x[c].w, x[c].w, al[3]);
+        be[0] = fmaf(y[c].x, y[c].x, be[0]); be[1] = fmaf(y[c].y, y[c].y, be[1]);
+        be[2] = fmaf(y[c].z, y[c].z, be[2]); be[3] = fmaf(y[c].w, y[c].w, be[3]);
+        ga[0] = fmaf(x[c].x, y[c].x, ga[0]); ga[1] = fmaf(x[c].y, y[c].y, ga[1]);
+        ga[2] = fmaf(x[c].z, y[c].z, ga[2]); ga[3] = fmaf(x[c].w, y[c].w, ga[3]);
+    }
+    const float alpha = (al[0] + al[1]) + (al[2] + al[3]);
+    const float beta_ = (be[0] + be[1]) + (be[2] + be[3]);
+    const float gamma = (ga[0] + ga[1]) + (ga[2] + ga[3]);
+    if (!(gamma != 0.f && fabsf(gamma) > tol * sqrtf(alpha * beta_))) return false;
+    const float zeta = (beta_ - alpha) / (2.f * gamma);
+    const float tt = (zeta >= 0.f ? 1.f : -1.f) / (fabsf(zeta) + sqrtf(1.f + zeta * zeta));
+    const float cs = 1.f / sqrtf(1.f + tt * tt);
+    const float sn = cs * tt;
+#pragma unroll
+    for (int c = 0; c < NC; ++c) {
+        if (4 * c < r) {
+            const float4 a = x[c], b = y[c];
+            *reinterpret_cast<float4*>(&s.M[p][4 * c]) =
+                make_float4(cs * a.x - sn * b.x, cs * a.y - sn * b.y, cs * a.z - sn * b.z, cs * a.w - sn * b.w);
+            *reinterpret_cast<float4*>(&s.M[q][4 * c]) =
+                make_float4(sn * a.x + cs * b.x, sn * a.y + cs * b.y, sn * a.z + cs * b.z, sn * a.w + cs * b.w);
+        }
+    }
+    return true;
+}
+
 template <typename TIN, typename T, int RT>
 __global__ void __launch_bounds__(32 * svd_warps<T>()) svd_kernel(SvdArgs<TIN, T> a) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -324,31 +433,91 @@ __global__ void __launch_bounds__(32 * svd_warps<T>()) svd_kernel(SvdArgs<TIN, T
     const TIN* RB = a.R_B + (size_t)local * rs * rs;
     const TIN* RA = a.R_A + (size_t)local * rs * rs;
 
-    // stage R_A in Ut, then M[i][j] = sum_{l >= max(i,j)} R_B[i][l] R_A[j][l] (one row per lane)
-    for (int e = lane; e < r * r; e += 32) {
-        const int i = e / r, l = e % r;
-        s.Ut[i][l] = (T)RA[i * rs + l];
-    }
-    __syncwarp();
-    for (int i = lane; i < r; i += 32) {
-        const TIN* rb = RB + (size_t)i * rs;
-        for (int j0 = 0; j0 < r; j0 += 4) {   // four columns of M at a time (independent chains)
-            T acc[4] = {0, 0, 0, 0};
-            for (int l = i; l < r; ++l) {
-                const T b = (T)rb[l];
+    // fp64 (refinement): U accumulates the rotations.  fp32 (main path): rows of M only
+    // are rotated, and U = M_0 M'^T Sigma^-2 is formed at the end from M_0, which is
+    // parked in the module's U output block meanwhile.
+    constexpr bool kAccU = sizeof(T) == 8;
+    if constexpr (kAccU) {
+        // stage R_A in Ut, then M[i][j] = sum_{l >= max(i,j)} R_B[i][l] R_A[j][l] (one row per lane)
+        for (int e = lane; e < r * r; e += 32) {
+            const int i = e / r, l = e % r;
+            s.Ut[i][l] = (T)RA[i * rs + l];
+        }
+        __syncwarp();
+        for (int i = lane; i < r; i += 32) {
+            const TIN* rb = RB + (size_t)i * rs;
+            for (int j0 = 0; j0 < r; j0 += 4) {   // four columns of M at a time (independent chains)
+                T acc[4] = {0, 0, 0, 0};
+                for (int l = i; l < r; ++l) {
+                    const T b = (T)rb[l];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        if (j0 + q < r && l >= j0 + q) acc[q] = fma(b, s.Ut[j0 + q][l], acc[q]);
+                }
 #pragma unroll
                 for (int q = 0; q < 4; ++q)
-                    if (j0 + q < r && l >= j0 + q) acc[q] = fma(b, s.Ut[j0 + q][l], acc[q]);
+                    if (j0 + q < r) s.M[i][j0 + q] = acc[q];
+            }
+        }
+        __syncwarp();
+        for (int e = lane; e < RT * SvdSmem<T, RT>::LD; e += 32) {
+            const int i = e / SvdSmem<T, RT>::LD, l = e % SvdSmem<T, RT>::LD;
+            if (i < r && l >= r) s.M[i][l] = T(0);
+            s.Ut[i][l] = (i == l && i < r) ? T(1) : T(0);
+        }
+    } else {
+        // M[i][j] = R_B[i] . R_A[j] (both R are zero below the diagonal and past r): lane j
+        // holds rows j and j + 32 of R_A, row i of R_B is broadcast to the warp
+        constexpr int NC = RT / 4;
+        // 16-byte loads when every row starts on a 16-byte boundary (rs % 4 == 0: a chunk
+        // that starts below r then ends inside the row); element loads otherwise
+        const bool vec = (rs & 3) == 0 && ((reinterpret_cast<uintptr_t>(RA) | reinterpret_cast<uintptr_t>(RB)) & 15) == 0;
+        auto ld_chunk = [&](const float* row, int c) -> float4 {
+            if (4 * c >= r) return make_float4(0.f, 0.f, 0.f, 0.f);
+            if (vec) return *reinterpret_cast<const float4*>(row + 4 * c);
+            float v[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) v[u] = 4 * c + u < r ? row[4 * c + u] : 0.f;
+            return make_float4(v[0], v[1], v[2], v[3]);
+        };
+        float4 ra[2][NC];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int j = lane + 32 * h;
+#pragma unroll
+            for (int c = 0; c < NC; ++c)
+                ra[h][c] = j < r ? ld_chunk(RA + (size_t)j * rs, c) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        double* M0 = a.U ? a.U + (size_t)local * rs * rs : nullptr;
+        for (int i = 0; i < r; ++i) {
+            float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+            for (int c = 0; c < NC; ++c) {
+                if (4 * c < r) {
+                    const float4 b = ld_chunk(RB + (size_t)i * rs, c);
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        acc[h][0] = fmaf(b.x, ra[h][c].x, acc[h][0]);
+                        acc[h][1] = fmaf(b.y, ra[h][c].y, acc[h][1]);
+                        acc[h][2] = fmaf(b.z, ra[h][c].z, acc[h][2]);
+                        acc[h][3] = fmaf(b.w, ra[h][c].w, acc[h][3]);
+                    }
+                }
             }
 #pragma unroll
-            for (int q = 0; q < 4; ++q)
-                if (j0 + q < r) s.M[i][j0 + q] = acc[q];
+            for (int h = 0; h < 2; ++h) {
+                const int j = lane + 32 * h;
+                if (j < r) {
+                    const float m = (acc[h][0] + acc[h][1]) + (acc[h][2] + acc[h][3]);
+                    s.M[i][j] = m;
+                    if (M0) M0[(size_t)i * rs + j] = (double)m;
+                }
+            }
         }
-    }
-    __syncwarp();
-    for (int e = lane; e < r * r; e += 32) {
-        const int i = e / r, l = e % r;
-        s.Ut[i][l] = i == l ? T(1) : T(0);
+        for (int e = lane; e < RT * SvdSmem<T, RT>::LD; e += 32) {
+            const int i = e / SvdSmem<T, RT>::LD, l = e % SvdSmem<T, RT>::LD;
+            if (i < r && l >= r) s.M[i][l] = T(0);   // zero padding: whole 16-byte chunks are read
+        }
     }
     __syncwarp();
 
@@ -367,62 +536,10 @@ __global__ void __launch_bounds__(32 * svd_warps<T>()) svd_kernel(SvdArgs<TIN, T
                     q = (t - lane + rp - 1) % (rp - 1);
                 }
                 if (p < r && q < r) {
-                    T al[4] = {0, 0, 0, 0}, be[4] = {0, 0, 0, 0}, ga[4] = {0, 0, 0, 0};
-                    const T* mp = s.M[p];
-                    const T* mq = s.M[q];
-                    int l = 0;
-#pragma unroll 4
-                    for (; l + 3 < r; l += 4) {   // four independent chains per sum, 16-byte loads
-                        T xv[4], yv[4];
-                        ld4(mp + l, xv);
-                        ld4(mq + l, yv);
-#pragma unroll
-                        for (int u = 0; u < 4; ++u) {
-                            al[u] = fma(xv[u], xv[u], al[u]);
-                            be[u] = fma(yv[u], yv[u], be[u]);
-                            ga[u] = fma(xv[u], yv[u], ga[u]);
-                        }
-                    }
-                    for (; l < r; ++l) {
-                        const T x = mp[l], y = mq[l];
-                        al[0] = fma(x, x, al[0]);
-                        be[0] = fma(y, y, be[0]);
-                        ga[0] = fma(x, y, ga[0]);
-                    }
-                    const T alpha = (al[0] + al[1]) + (al[2] + al[3]);
-                    const T beta_ = (be[0] + be[1]) + (be[2] + be[3]);
-                    const T gamma = (ga[0] + ga[1]) + (ga[2] + ga[3]);
-                    if (gamma != T(0) && fabs(gamma) > tol * sqrt(alpha * beta_)) {
-                        rot = true;
-                        const T zeta = (beta_ - alpha) / (T(2) * gamma);
-                        const T tt = (zeta >= T(0) ? T(1) : T(-1)) / (fabs(zeta) + sqrt(T(1) + zeta * zeta));
-                        const T c = T(1) / sqrt(T(1) + tt * tt);
-                        const T sn = c * tt;
-                        T* Mp = s.M[p];
-                        T* Mq = s.M[q];
-                        T* Up = s.Ut[p];
-                        T* Uq = s.Ut[q];
-                        int k = 0;
-#pragma unroll 2
-                        for (; k + 3 < r; k += 4) {   // 16-byte loads and stores of four columns
-                            T x[4], y[4], u[4], v[4], x2[4], y2[4], u2[4], v2[4];
-                            ld4(Mp + k, x); ld4(Mq + k, y); ld4(Up + k, u); ld4(Uq + k, v);
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                x2[e] = c * x[e] - sn * y[e];
-                                y2[e] = sn * x[e] + c * y[e];
-                                u2[e] = c * u[e] - sn * v[e];
-                                v2[e] = sn * u[e] + c * v[e];
-                            }
-                            st4(Mp + k, x2); st4(Mq + k, y2); st4(Up + k, u2); st4(Uq + k, v2);
-                        }
-                        for (; k < r; ++k) {
-                            const T x = Mp[k], y = Mq[k], u = Up[k], v = Uq[k];
-                            Mp[k] = c * x - sn * y;
-                            Mq[k] = sn * x + c * y;
-                            Up[k] = c * u - sn * v;
-                            Uq[k] = sn * u + c * v;
-                        }
+                    if constexpr (kAccU) {
+                        rot |= svd_rotate_acc<T, RT>(s, p, q, r, tol);
+                    } else {
+                        rot |= svd_rotate_rows<T, RT>(s, p, q, r, tol);
                     }
                 }
             }
@@ -452,9 +569,38 @@ __global__ void __launch_bounds__(32 * svd_warps<T>()) svd_kernel(SvdArgs<TIN, T
     for (int j = lane; j < rs; j += 32) sg[j] = j < r ? (double)s.sig[s.perm[j]] : 0.0;
     if (a.U) {
         double* Uo = a.U + (size_t)local * rs * rs;
-        for (int e = lane; e < rs * rs; e += 32) {
-            const int row = e / rs, j = e % rs;
-            Uo[e] = (row < r && j < r) ? (double)s.Ut[s.perm[j]][row] : 0.0;
+        if constexpr (kAccU) {
+            for (int e = lane; e < rs * rs; e += 32) {
+                const int row = e / rs, j = e % rs;
+                Uo[e] = (row < r && j < r) ? (double)s.Ut[s.perm[j]][row] : 0.0;
+            }
+        } else {   // column j of U = M_0 m'_p / sigma_p^2 (p = perm[j]); zero where sigma_p = 0
+            for (int row = lane; row < rs; row += 32) {
+                float m0[RT];
+#pragma unroll
+                for (int l = 0; l < RT; ++l) m0[l] = (row < r && l < r) ? (float)Uo[(size_t)row * rs + l] : 0.f;
+                for (int j = 0; j < rs; ++j) {
+                    double u = 0.0;
+                    if (row < r && j < r) {
+                        const int pj = s.perm[j];
+                        const T sp = s.sig[pj];
+                        float d0 = 0.f, d1 = 0.f, d2 = 0.f, d3 = 0.f;
+#pragma unroll
+                        for (int c = 0; c < RT / 4; ++c) {
+                            if (4 * c < r) {
+                                const float4 mp = *reinterpret_cast<const float4*>(&s.M[pj][4 * c]);
+                                d0 = fmaf(m0[4 * c], mp.x, d0);
+                                d1 = fmaf(m0[4 * c + 1], mp.y, d1);
+                                d2 = fmaf(m0[4 * c + 2], mp.z, d2);
+                                d3 = fmaf(m0[4 * c + 3], mp.w, d3);
+                            }
+                        }
+                        const double dot = (double)((d0 + d1) + (d2 + d3));
+                        u = sp > T(0) ? dot / ((double)sp * (double)sp) : 0.0;
+                    }
+                    Uo[(size_t)row * rs + j] = u;   // row `row` of M_0 is in registers already
+                }
+            }
         }
     }
     if (a.V) {
