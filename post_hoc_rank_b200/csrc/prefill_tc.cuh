@@ -28,11 +28,13 @@ constexpr int kTcThreads = 128;  // shrink: 4 warps, warp w owns tensor-memory l
 constexpr int kTcCols = 2048;    // d_out columns per expand CTA
 constexpr int kTcMaxSplit = 8;   // d_in is split over at most this many CTAs per token tile
 
-// d_in elements per split: a multiple of the stage width, at least 1024, at most kTcMaxSplit splits
+// d_in elements per split: a multiple of the stage width, at least 2048, at most kTcMaxSplit splits
+// (swept 512 / 1024 / 2048 / 3072 / 4096 on the prefill layers: 2048 fills one wave of
+// CTAs for the hidden-width projections and keeps the expand's sum over partials short)
 __host__ __device__ inline int tc_split_len(int d_in) {
     int len = (d_in + kTcMaxSplit - 1) / kTcMaxSplit;
     len = ((len + kTcKB - 1) / kTcKB) * kTcKB;
-    return len < 1024 ? 1024 : len;
+    return len < 2048 ? 2048 : len;
 }
 
 // ---- shrink ---------------------------------------------------------------
