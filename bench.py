@@ -427,9 +427,11 @@ def sandwich_bench(args, dev, stream, hbm, rank=16, diagonal=True):
     return out
 
 
-def prefill_bench(args, dev, stream, hbm, k, fused=False):
+def prefill_bench(args, dev, stream, hbm, k, fused=False, route_once=True):
     """Config 4: Qwen2.5-7B layer, 7 projections, 32 requests x 512 tokens, request i -> adapter i.
-    fused: q/k/v and gate/up as one multi-slice call each."""
+    fused: q/k/v and gate/up as one multi-slice call each.  route_once: the batch is routed
+    once per step (lf_route_tokens) and every projection call reuses the tables; otherwise
+    every call routes the batch again."""
     import torch
     from post_hoc_rank_b200 import api, synth
     from post_hoc_rank_b200 import loraforge as lf
@@ -448,12 +450,15 @@ def prefill_bench(args, dev, stream, hbm, k, fused=False):
         Bt = synth.normal_bf16((int(offB[-1]),), (4, 4, p, k), std=d_out ** -0.5, device=dev)
         groups.append((d_in, d_out, rk, offA, offB, Ap, Bt))
         total_bytes += apply_bytes(T, d_in, d_out, [k] * n_ad)
-    calls, sets = _layer_calls(groups, lambda d: x_f if d == M.ffn else x_h, ids_d, n_ad, T, dev, (4, 5), fused)
+    calls, sets = _layer_calls(groups, lambda d: x_f if d == M.ffn else x_h, ids_d, n_ad, T, dev, (4, 5), fused,
+                               route_once)
     if fused:
         total_bytes -= sum(2 * T * groups[ps[0]][0] * (len(ps) - 1) for ps in sets)
     return _apply_run(args, calls, ids_d, n_ad, T, total_bytes, stream, hbm, dict(
         workload=f"prefill: Qwen2.5-7B layer x 7 projections, 32 requests x 512 tokens, k={k}"
-                 + ("; q/k/v and gate/up as one slice call each" if fused else "")))
+                 + ("; q/k/v and gate/up as one slice call each" if fused else "")
+                 + ("; routed once per step, projections reuse the tables" if route_once
+                    else "; every call routes the batch")))
 
 
 def _proj_call(x, y, ids_d, n_ad, rk, oa, ob, Ap, Bt, ws, scale=2.0):
@@ -476,15 +481,33 @@ def _slices_call(x, y, ids_d, n_ad, slices, ws, scale=2.0):
     return run
 
 
-def _layer_calls(groups, x_of, ids_d, n_ad, T, dev, key, fused):
+def _routed_call(x, y, ids_d, n_ad, slices, ws, scale=2.0):
+    """Projections through lf_lora_shrink_expand_slices_routed (tables already in ws)."""
+    from post_hoc_rank_b200 import loraforge as lf
+    sl = [lf.make_slice(*t) for t in slices]
+
+    def run(st=None, _keep=slices):
+        lf.lf_lora_shrink_expand_slices_routed(x, y, ids_d, n_ad, sl, scale, ws, stream=st)
+    return run
+
+
+def _layer_calls(groups, x_of, ids_d, n_ad, T, dev, key, fused, route_once=False):
     """Calls of one layer.  groups: per projection (d_in, d_out, rk int64 array, offA,
     offB, Ap, Bt); fused: q/k/v and gate/up (projections reading the same x) go as
-    one slice call each.  Returns (callables, algorithmic bytes given the adapters used)."""
+    one slice call each; route_once: one lf_route_tokens call, then routed projection
+    calls on the same workspace.  Returns (callables, the projection sets)."""
     import torch
     from post_hoc_rank_b200 import api, synth
     from post_hoc_rank_b200 import loraforge as lf
     sets = [[0, 1, 2], [3], [4, 5], [6]] if fused else [[p] for p in range(len(groups))]
     calls = []
+    rws = None
+    if route_once:
+        rws = api.workspace(lf.lf_apply_slices_workspace_size(T, n_ad, max(len(ps) for ps in sets)), dev)
+
+        def route(st=None):
+            lf.lf_route_tokens(ids_d, n_ad, rws, stream=st)
+        calls.append(route)
     for gi, ps in enumerate(sets):
         d_in = groups[ps[0]][0]
         x = x_of(d_in)
@@ -497,7 +520,9 @@ def _layer_calls(groups, x_of, ids_d, n_ad, T, dev, key, fused):
             tens.append((d_out, y_off, torch.from_numpy(rk.astype(np.int32)).to(dev),
                          torch.from_numpy(offA[:-1]).to(dev), torch.from_numpy(offB[:-1]).to(dev), Ap, Bt))
             y_off += d_out
-        if len(ps) == 1:
+        if route_once:
+            calls.append(_routed_call(x, y, ids_d, n_ad, tens, rws))
+        elif len(ps) == 1:
             ws = api.workspace(lf.lf_apply_workspace_size(T, n_ad), dev)
             d_out, _, rk_d, oa_d, ob_d, Ap, Bt = tens[0]
             calls.append(_proj_call(x, y, ids_d, n_ad, rk_d, oa_d, ob_d, Ap, Bt, ws))
@@ -974,6 +999,7 @@ def main():
                 "decode_sigma_sandwich_r16_diag": sandwich_bench(args, dev, stream, hbm, 16, True),
                 "decode_sigma_sandwich_r16_full": sandwich_bench(args, dev, stream, hbm, 16, False),
                 "prefill_k16": prefill_bench(args, dev, stream, hbm, 16),
+                "prefill_k16_route_per_call": prefill_bench(args, dev, stream, hbm, 16, route_once=False),
                 "prefill_k16_fused_slices": prefill_bench(args, dev, stream, hbm, 16, fused=True),
                 "prefill_r64": prefill_bench(args, dev, stream, hbm, 64)}
         if rank == 0 and not args.no_cpu:

@@ -224,6 +224,27 @@ lf_status lf_lora_shrink_expand_slices(int32_t T, int32_t d_in, const void* x, v
                                        float scale, const float* adapter_scale, int32_t* seg_out,
                                        void* ws, size_t ws_bytes, lf_stream_t stream);
 
+/* ---- Routing once per batch ---------------------------------------------------
+ * Every projection of a forward pass sees the same token ids, so the routing (the
+ * stable sort of tokens by adapter, the segment table and the work items) can be
+ * computed once: lf_route_tokens writes it into `ws`, and
+ * lf_lora_shrink_expand_slices_routed then applies any projection of the batch
+ * (same T, ids and n_adapters, any n_slices) from those tables without a routing
+ * pass.  ws must be sized for the largest n_slices used with it
+ * (lf_apply_slices_workspace_size); the tables in ws are those of the most recent
+ * routing pass on it (lf_route_tokens or any unrouted apply call).  A routed call on
+ * a workspace whose tables were written for another T or n_adapters (or never)
+ * applies nothing and latches LF_ERR_INVALID_ARG.  In the decode regime
+ * (T <= 8 n_adapters) the side path reads ids directly and the tables are not used.
+ * Host errors as for lf_lora_shrink_expand_slices. */
+lf_status lf_route_tokens(int32_t T, const int32_t* ids, int32_t n_adapters, void* ws, size_t ws_bytes,
+                          lf_stream_t stream);
+lf_status lf_lora_shrink_expand_slices_routed(int32_t T, int32_t d_in, const void* x, void* y, int64_t y_ld,
+                                              const int32_t* ids, int32_t n_adapters,
+                                              const lf_slice* slices /*[host]*/, int32_t n_slices,
+                                              float scale, const float* adapter_scale,
+                                              void* ws, size_t ws_bytes, lf_stream_t stream);
+
 /* ---- Sigma-sandwich serving (jointly compressed adapters) ---------------------
  * "Compress then Serve" (academ.us/article/2407.00066), sections 3.1 and 11: the
  * adapters of one module share U (d_out x rank) and V (d_in x rank) and keep a

@@ -31,7 +31,12 @@ struct RouteOut {
     // consecutive ids (the histogram and the stable scatter touch runs, not tokens).
     int32_t* run_start;  // first token of run i
     int32_t* run_pos;    // position of run i's first token in the permutation
+    int32_t* tag;        // nullable: {kRouteTagMagic, T, n_adapters, tc_enable} once the tables are complete
 };
+
+// Tag of a workspace whose routing tables were written for a batch of T tokens over
+// n_adapters (checked by route_check_kernel before a routed call reuses them).
+constexpr int32_t kRouteTagMagic = 0x52545447;
 
 // Block-wide exclusive scan of one int per thread (blockDim.x a multiple of 32, <= 1024).
 __device__ __forceinline__ int block_excl_scan(int v, int* wsum, int* total) {
@@ -178,6 +183,12 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const int32_t* __r
         o.counts[1] = nval;
         o.counts[2] = s_carry[2];
         o.counts[3] = s_carry[3];
+        if (o.tag) {
+            o.tag[0] = kRouteTagMagic;
+            o.tag[1] = T;
+            o.tag[2] = n_adapters;
+            o.tag[3] = o.tc_enable;
+        }
     }
     if (runs) {
         // stable scatter of runs (warp turns in run order), then every token in parallel
@@ -431,6 +442,18 @@ __global__ void __launch_bounds__(kGemvThreads) expand_kernel(ApplyArgs a) {
     }
 }
 
+
+// Routed calls reuse the routing tables already in the workspace.  If the tag does not
+// name this batch shape (no routing pass on this workspace, or one for another T or
+// adapter count), every work count is cleared, so no kernel of the call reads the tables,
+// and LF_ERR_INVALID_ARG is latched.
+__global__ void route_check_kernel(int32_t* tag, int32_t* counts, int T, int n_adapters, int tc_enable) {
+    if (threadIdx.x != 0) return;
+    if (!(tag[0] == kRouteTagMagic && tag[1] == T && tag[2] == n_adapters && tag[3] == tc_enable)) {
+        counts[0] = counts[1] = counts[2] = counts[3] = 0;
+        latch_error(LF_ERR_INVALID_ARG);
+    }
+}
 
 // Decode regime, token-parallel (BGMV form: every token carries its adapter index,
 // no sorting).  CTA (token, 8192-column chunk of one slice): t = A' x (k fp32 dot

@@ -339,6 +339,7 @@ __global__ void cap_flags_kernel(int32_t* count, int cap) {
 
 // ------------------------------------------------------------ apply workspace
 struct ApplyWs {
+    int32_t* tag;
     int32_t* counts;
     Seg* segs;
     int32_t* perm;
@@ -355,14 +356,17 @@ static size_t carve_apply(void* base, int64_t T, int64_t n, int ns, ApplyWs* w) 
     Carver c(base);
     const int64_t mseg = std::min<int64_t>(T, n);
     const int64_t T1 = std::max<int64_t>(T, 1);
+    // routing tables first: their offsets depend on (T, n) only, so a routing pass on
+    // this workspace serves calls with any number of slices
+    w->tag = c.take<int32_t>(4);
     w->counts = c.take<int32_t>(4);
     w->segs = c.take<Seg>((size_t)std::max<int64_t>(mseg, 1));
     w->perm = c.take<int32_t>((size_t)T1);
     w->items = c.take<GemvItem>((size_t)(T / kGemvTok + mseg + 1));
-    w->t_buf = c.take<float>((size_t)T1 * kMaxRank * ns);
     w->tc_items = c.take<TcItem>((size_t)(T / kTcM + mseg + 1));
-    w->t_part = c.take<float>((size_t)kTcMaxSplit * T1 * kMaxRank * ns);
     w->runs = c.take<int32_t>((size_t)2 * T1);   // run scratch of the routing pass
+    w->t_buf = c.take<float>((size_t)T1 * kMaxRank * ns);
+    w->t_part = c.take<float>((size_t)kTcMaxSplit * T1 * kMaxRank * ns);
     return c.off + 256;
 }
 
@@ -393,7 +397,7 @@ struct SharedSlice {
 static lf_status apply_impl(int32_t T, int32_t d_in, const void* x, void* y, int64_t y_ld, const int32_t* ids,
                             int32_t n_adapters, const lf_slice* sl, int32_t ns, float scale, const float* scales,
                             int32_t* seg_out, void* ws, size_t ws_bytes, cudaStream_t s,
-                            const SharedSlice* shared = nullptr) {
+                            const SharedSlice* shared = nullptr, bool routed = false) {
     if (T < 0 || d_in < 1 || n_adapters < 1 || n_adapters > 16384 || ns < 1 || ns > kMaxSlices || !sl)
         return LF_ERR_INVALID_ARG;
     if (T == 0) return LF_OK;
@@ -460,6 +464,7 @@ static lf_status apply_impl(int32_t T, int32_t d_in, const void* x, void* y, int
     o.run_start = w.runs;
     o.run_pos = w.runs + T;
     o.seg_out = seg_out;
+    o.tag = w.tag;
     const bool decode_regime = (int64_t)T <= (int64_t)kGemvTok * n_adapters;
     o.tc_enable = decode_regime ? 0 : 1;
     const size_t rsmem = 2 * (size_t)n_adapters * sizeof(int32_t);
@@ -475,7 +480,10 @@ static lf_status apply_impl(int32_t T, int32_t d_in, const void* x, void* y, int
         LF_LAUNCH("bgmv", bgmv_kernel, dim3((unsigned)T, (unsigned)A.n_chunks), kBgmvThreads, 0, s, A);
         return launch_status();
     }
-    LF_LAUNCH("route", route_kernel, 1, route_threads(T, n_adapters), rsmem, s, ids, T, n_adapters, o);
+    if (routed)   // tables from an earlier routing pass on this workspace
+        LF_LAUNCH("route_check", route_check_kernel, 1, 32, 0, s, w.tag, w.counts, T, n_adapters, 1);
+    else
+        LF_LAUNCH("route", route_kernel, 1, route_threads(T, n_adapters), rsmem, s, ids, T, n_adapters, o);
     LF_CUDA_TRY(cudaGetLastError());
     const int64_t mseg = std::min<int64_t>(T, n_adapters);
     // segments under kTcMin tokens: GEMV shrink (per slice), then expand
@@ -1121,6 +1129,41 @@ lf_status lf_lora_shrink_expand_slices(int32_t T, int32_t d_in, const void* x, v
                                        void* ws, size_t ws_bytes, lf_stream_t stream) {
     return apply_impl(T, d_in, x, y, y_ld, ids, n_adapters, slices, n_slices, scale, adapter_scale, seg_out, ws,
                       ws_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+lf_status lf_route_tokens(int32_t T, const int32_t* ids, int32_t n_adapters, void* ws, size_t ws_bytes,
+                          lf_stream_t stream) {
+    if (T < 0 || n_adapters < 1 || n_adapters > 16384) return LF_ERR_INVALID_ARG;
+    if (T == 0) return LF_OK;
+    if (!ids || !ws) return LF_ERR_INVALID_ARG;
+    ApplyWs w;
+    if (ws_bytes < carve_apply(nullptr, T, n_adapters, 1, &w)) return LF_ERR_WORKSPACE;
+    carve_apply(reinterpret_cast<char*>(align_up((int64_t)reinterpret_cast<uintptr_t>(ws), 256)), T, n_adapters, 1,
+                &w);
+    RouteOut o{};
+    o.counts = w.counts;
+    o.segs = w.segs;
+    o.perm = w.perm;
+    o.items = w.items;
+    o.tc_items = w.tc_items;
+    o.run_start = w.runs;
+    o.run_pos = w.runs + T;
+    o.seg_out = nullptr;
+    o.tag = w.tag;
+    o.tc_enable = (int64_t)T <= (int64_t)kGemvTok * n_adapters ? 0 : 1;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const size_t rsmem = 2 * (size_t)n_adapters * sizeof(int32_t);
+    LF_CUDA_TRY(cudaFuncSetAttribute(route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rsmem));
+    LF_LAUNCH("route", route_kernel, 1, route_threads(T, n_adapters), rsmem, s, ids, T, n_adapters, o);
+    return launch_status();
+}
+
+lf_status lf_lora_shrink_expand_slices_routed(int32_t T, int32_t d_in, const void* x, void* y, int64_t y_ld,
+                                              const int32_t* ids, int32_t n_adapters, const lf_slice* slices,
+                                              int32_t n_slices, float scale, const float* adapter_scale, void* ws,
+                                              size_t ws_bytes, lf_stream_t stream) {
+    return apply_impl(T, d_in, x, y, y_ld, ids, n_adapters, slices, n_slices, scale, adapter_scale, nullptr, ws,
+                      ws_bytes, reinterpret_cast<cudaStream_t>(stream), nullptr, true);
 }
 
 lf_status lf_lora_shrink_expand_noalloc(int32_t T, int32_t d_in, int32_t d_out, const void* x, void* y,

@@ -105,6 +105,10 @@ def lib() -> ctypes.CDLL:
         L.lf_lora_sigma_sandwich.argtypes = [_I32, _I32, _I32, _P, _P, _P, _I32, _I32, _P, _P, _P, _I32,
                                              ctypes.c_float, _P, _SZ, _P]
         L.lf_lora_sigma_sandwich.restype = ctypes.c_int
+        L.lf_route_tokens.argtypes = [_I32, _P, _I32, _P, _SZ, _P]; L.lf_route_tokens.restype = ctypes.c_int
+        L.lf_lora_shrink_expand_slices_routed.argtypes = [_I32, _I32, _P, _P, _I64, _P, _I32, _P, _I32,
+                                                          ctypes.c_float, _P, _P, _SZ, _P]
+        L.lf_lora_shrink_expand_slices_routed.restype = ctypes.c_int
         L.lf_jd_workspace_size.argtypes = [_P, _I32, _P, _I32, _P, _I32]; L.lf_jd_workspace_size.restype = _SZ
         L.lf_jd_full.argtypes = [_P, _I32, _P, _I32, _P, _I32, _P, _P, _P, _I32, _P, _P, _P, _P, _SZ, _P]
         L.lf_jd_full.restype = ctypes.c_int
@@ -127,7 +131,8 @@ def exported_symbols() -> list[str]:
             "lf_apply_workspace_size", "lf_lora_shrink_expand", "lf_status_string", "lf_get_device_status",
             "lf_profile_enable", "lf_profile_reset", "lf_profile_read", "lf_launch_count",
             "lf_lora_shrink_expand_noalloc", "lf_apply_slices_workspace_size", "lf_lora_shrink_expand_slices",
-            "lf_lora_sigma_sandwich", "lf_jd_workspace_size", "lf_jd_full"]
+            "lf_lora_sigma_sandwich", "lf_jd_workspace_size", "lf_jd_full", "lf_route_tokens",
+            "lf_lora_shrink_expand_slices_routed"]
 
 # Limits of lf_lora_shrink_expand_noalloc (its scratch is a fixed array in the library).
 NOALLOC_MAX_TOKENS = 16384
@@ -251,6 +256,24 @@ def lf_lora_shrink_expand_slices(x, y, ids, n_adapters, slices, scale, ws, adapt
                                             len(slices), float(scale), _ptr(adapter_scale), _ptr(seg_out), _ptr(ws),
                                             ws.numel() if ws is not None else 0, _stream(stream))
     return _check(st, "lf_lora_shrink_expand_slices") if check else st
+
+
+def lf_route_tokens(ids, n_adapters, ws, stream=None, check=True) -> int:
+    """Routing of a token batch into `ws`, for routed calls on the same batch."""
+    st = lib().lf_route_tokens(int(ids.numel()), _ptr(ids), n_adapters, _ptr(ws), ws.numel() if ws is not None else 0,
+                               _stream(stream))
+    return _check(st, "lf_route_tokens") if check else st
+
+
+def lf_lora_shrink_expand_slices_routed(x, y, ids, n_adapters, slices, scale, ws, adapter_scale=None, stream=None,
+                                        check=True) -> int:
+    """lf_lora_shrink_expand_slices on a workspace that already holds this batch's routing."""
+    T, d_in = x.shape
+    arr = (lf_slice * len(slices))(*slices)
+    st = lib().lf_lora_shrink_expand_slices_routed(T, d_in, _ptr(x), _ptr(y), y.shape[1], _ptr(ids), n_adapters, arr,
+                                                   len(slices), float(scale), _ptr(adapter_scale), _ptr(ws),
+                                                   ws.numel() if ws is not None else 0, _stream(stream))
+    return _check(st, "lf_lora_shrink_expand_slices_routed") if check else st
 
 
 def lf_lora_sigma_sandwich(x, y, ids, n_adapters, Vt, Ut, sigma, diagonal, scale, ws, stream=None,

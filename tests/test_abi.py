@@ -171,3 +171,12 @@ def test_jd_validation_on_host():
     assert call(ptr=8) == 8
     assert call(wsb=64) == 4
     assert call(probs=tabs.probs[:0]) == 0                # nothing to do
+
+
+def test_route_tokens_validation_on_host():
+    L = lf.lib()
+    assert L.lf_route_tokens(0, None, 4, None, 0, None) == 0          # empty batch: nothing to do
+    assert L.lf_route_tokens(-1, 16, 4, 16, 1 << 20, None) == 1
+    assert L.lf_route_tokens(8, 16, 0, 16, 1 << 20, None) == 1
+    assert L.lf_route_tokens(8, None, 4, 16, 1 << 20, None) == 1
+    assert L.lf_route_tokens(1000, 16, 4, 16, 64, None) == 4          # workspace too small

@@ -287,3 +287,58 @@ def test_sigma_sandwich_matches_oracle(regime, diagonal):
                                    Ut.float().numpy(), sig.astype(np.float64), diagonal, 1.5)
     assert_close(y.cpu(), want)
     assert torch.equal(y.cpu()[torch.from_numpy(ids < 0)], y0[torch.from_numpy(ids < 0)])
+
+
+def _slice_tensors(sl, dev="cuda"):
+    """lf_slice records and the device tensors they point into (keep both alive)."""
+    tens = [(s["d_out"], s["y_off"], torch.from_numpy(np.asarray(s["ranks"], np.int32)).to(dev),
+             torch.from_numpy(np.asarray(s["offA"][:-1], np.int64)).to(dev),
+             torch.from_numpy(np.asarray(s["offB"][:-1], np.int64)).to(dev), s["Ap"].to(dev), s["Bt"].to(dev))
+            for s in sl]
+    return [lf.make_slice(*t) for t in tens], tens
+
+
+def test_routing_once_serves_every_projection():
+    """lf_route_tokens + routed calls give the same bits as unrouted calls, for projections
+    with different slice counts on one workspace (segments for both GEMV and tensor-core items)."""
+    T, n, d_in = 1500, 6, 256
+    ids = np.concatenate([np.repeat(np.arange(4, dtype=np.int32), 300), synth.zipf_ids(300, n, 1.0, (12, 0))])
+    ids[np.random.default_rng(12).random(T) < 0.03] = -1
+    ids_d = torch.from_numpy(ids).cuda()
+    x = synth.normal_bf16((T, d_in), (12, 1)).cuda()
+    projs = [make_slices([256], n, d_in, (12, 2)), make_slices([128, 64, 64], n, d_in, (12, 3))]
+    ws = api.workspace(lf.lf_apply_slices_workspace_size(T, n, 3), "cuda")
+    lf.lf_route_tokens(ids_d, n, ws)
+    for p, (sl, y_ld) in enumerate(projs):
+        y0 = synth.normal_bf16((T, y_ld), (12, 4, p)).cuda()
+        keep, _alive = _slice_tensors(sl)
+        y_ref = y0.clone()
+        ws_ref = api.workspace(lf.lf_apply_slices_workspace_size(T, n, len(sl)), "cuda")
+        lf.lf_lora_shrink_expand_slices(x, y_ref, ids_d, n, keep, 1.25, ws_ref)
+        y = y0.clone()
+        lf.lf_lora_shrink_expand_slices_routed(x, y, ids_d, n, keep, 1.25, ws)
+        assert lf.lf_get_device_status() == 0
+        assert torch.equal(y, y_ref), p
+        check_slices(y.cpu(), y0.cpu(), oracle_slices(x.cpu(), y0.cpu(), ids, sl, 1.25), sl, ids)
+
+
+def test_routed_call_without_matching_routing_applies_nothing():
+    T, n, d_in = 600, 3, 128
+    ids = np.repeat(np.arange(n, dtype=np.int32), 200)
+    ids_d = torch.from_numpy(ids).cuda()
+    x = synth.normal_bf16((T, d_in), (13, 1)).cuda()
+    sl, y_ld = make_slices([128], n, d_in, (13, 2))
+    keep, _alive = _slice_tensors(sl)
+    y0 = synth.normal_bf16((T, y_ld), (13, 3)).cuda()
+    # a fresh (zeroed) workspace: no routing pass ever ran on it
+    ws = torch.zeros(lf.lf_apply_slices_workspace_size(T, n, 1), dtype=torch.uint8, device="cuda")
+    y = y0.clone()
+    lf.lf_lora_shrink_expand_slices_routed(x, y, ids_d, n, keep, 1.0, ws)
+    assert lf.lf_get_device_status() == 1   # LF_ERR_INVALID_ARG, latched on the device
+    assert torch.equal(y, y0)
+    # routing written for another batch shape (fewer tokens) is not reused either
+    lf.lf_route_tokens(ids_d[:300], n, ws)
+    assert lf.lf_get_device_status() == 0
+    lf.lf_lora_shrink_expand_slices_routed(x, y, ids_d, n, keep, 1.0, ws)
+    assert lf.lf_get_device_status() == 1
+    assert torch.equal(y, y0)
