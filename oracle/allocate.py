@@ -12,6 +12,10 @@ Sources
   energy accumulation curve, where spectral energy is the sum of squared
   singular values and each direction carries sigma_j^2 of it.
 
+* LoRASpace (the arXiv listing's abstract, "LoRASpace: A Pool-Wide Shared Substrate
+  for Static and Dynamic Multi-LoRA Composition"): the minimal subspace that keeps a
+  fraction (99 %) of the factor energy, found by SVD.
+
 Readings (the pages give no formula):
 * U: k = round-half-up(num * r / den), clamped to [floor, r].
 * S: budget in rank units per adapter (module ``group``):
@@ -24,6 +28,10 @@ Readings (the pages give no formula):
   with j, the chosen set is a prefix of every module, and the greedy choice
   maximises sum_i (retained energy fraction of module i) under sum_i k_i <= K.
   If K < floor * M every module keeps ``floor`` (budget exceeded, reported).
+* Energy fraction (LoRASpace's rule read per module): k is the smallest rank in
+  [floor, r] whose leading directions hold at least num/den of the module's
+  spectral energy, den * sum_{j<k} sigma_j^2 >= num * sum_j sigma_j^2 (both sums
+  taken in j order, ties keep the smaller k); a zero module keeps ``floor``.
 """
 from __future__ import annotations
 
@@ -118,3 +126,42 @@ def brute_force_ranks(sigma_rows, r, num: int, den: int, floor: int, absolute: b
         elif abs(val - best) <= tol:
             arg.append(ks)
     return best, arg
+
+
+def energy_fraction_rank(sigma, r: int, num: int, den: int, floor: int):
+    """Smallest k in [floor, r] with den * sum_{j<k} sigma_j^2 >= num * sum_j sigma_j^2.
+
+    Returns (k, gap_rel): gap_rel = the smallest |den * cum_k - num * tot| / (num * tot)
+    over k in [floor, r] (how far the module is from a tie at the threshold; inf for a
+    zero module or num = 0)."""
+    if floor > r:
+        raise ValueError("floor exceeds module rank")
+    s = np.asarray(sigma, dtype=np.float64)[:r]
+    if np.any(np.diff(s) > 0):
+        raise ValueError("singular values must be listed in descending order")
+    sq = s * s
+    tot = 0.0
+    for v in sq:
+        tot += float(v)
+    if tot == 0.0:
+        return floor, math.inf
+    rhs = num * tot
+    cum, k, gap = 0.0, None, math.inf
+    for j in range(r):
+        cum += float(sq[j])
+        kk = j + 1
+        if kk < floor:
+            continue
+        lhs = den * cum
+        if rhs > 0.0:
+            gap = min(gap, abs(lhs - rhs) / rhs)
+        if k is None and lhs >= rhs:
+            k = kk
+    return (r if k is None else k), gap
+
+
+def energy_fraction_ranks(sigma_rows, r, num: int, den: int, floor: int):
+    """energy_fraction_rank for every module: (ranks int32[n], gaps float64[n])."""
+    sigma_rows = np.asarray(sigma_rows, dtype=np.float64)
+    out = [energy_fraction_rank(sigma_rows[i], int(r[i]), num, den, floor) for i in range(len(r))]
+    return np.array([k for k, _ in out], dtype=np.int32), np.array([g for _, g in out])

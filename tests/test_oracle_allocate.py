@@ -1,5 +1,6 @@
 """Pins for oracle.allocate: hand-worked fixtures, brute force, invariants."""
 import json
+import math
 import os
 
 import numpy as np
@@ -126,3 +127,45 @@ def test_absolute_energy_brute_force_agrees():
     rk, _ = AL.spectral_ranks(sig, [4] * 4, [0] * 4, 1, 2, 1, absolute=True)
     best, args = AL.brute_force_ranks(sig, [4] * 4, 1, 2, 1, absolute=True)
     assert tuple(rk.tolist()) in [tuple(a) for a in args]
+
+
+# ---- energy fraction (LoRASpace's minimal subspace keeping a fraction of the energy) ----
+
+def test_energy_fraction_hand_case():
+    # sigma = 3, 2, 1: energies 9, 4, 1 of 14
+    s = [3.0, 2.0, 1.0]
+    assert AL.energy_fraction_rank(s, 3, 1, 2, 1)[0] == 1        # 9 >= 7
+    assert AL.energy_fraction_rank(s, 3, 9, 10, 1)[0] == 2       # 13 >= 12.6 > 9
+    assert AL.energy_fraction_rank(s, 3, 19, 20, 1)[0] == 3      # 13 < 13.3
+    assert AL.energy_fraction_rank(s, 3, 13, 14, 1)[0] == 2      # exactly 13/14: the tie keeps k = 2
+    assert AL.energy_fraction_rank(s, 3, 1, 100, 2)[0] == 2      # the floor
+    assert AL.energy_fraction_rank([2.0, 1.0, 0.0, 0.0], 4, 1, 1, 1)[0] == 2   # all of it: last nonzero
+    assert AL.energy_fraction_rank([0.0, 0.0], 2, 99, 100, 1)[0] == 1          # zero module: floor
+
+
+def test_energy_fraction_geometric_closed_form():
+    # sigma_j^2 = q^j (j = 0..r-1): the leading-k fraction is (1 - q^k) / (1 - q^r), so the
+    # smallest k reaching rho is ceil(log(1 - rho (1 - q^r)) / log q)
+    for q, r, num, den in [(0.5, 20, 99, 100), (0.8, 32, 9, 10), (0.9, 64, 99, 100), (0.7, 16, 1, 3)]:
+        s = np.sqrt(q ** np.arange(r))
+        rho = num / den
+        want = math.ceil(math.log(1 - rho * (1 - q ** r)) / math.log(q) - 1e-12)
+        assert AL.energy_fraction_rank(s, r, num, den, 1)[0] == max(1, want), (q, r, num, den)
+
+
+def test_energy_fraction_is_monotone_and_keeps_the_fraction():
+    g = np.random.default_rng(21)
+    for _ in range(50):
+        r = int(g.integers(1, 40))
+        s = np.sort(np.abs(g.standard_normal(r)) * np.exp(g.standard_normal(r)))[::-1]
+        fl = int(g.integers(1, r + 1))
+        prev = 0
+        for num in range(0, 101, 5):
+            k, _ = AL.energy_fraction_rank(s, r, num, 100, fl)
+            assert fl <= k <= r and k >= prev
+            prev = k
+            e = s * s
+            kept = e[:k].sum() / e.sum()
+            assert kept >= num / 100 - 1e-12
+            if k > fl:   # one direction fewer would not reach the fraction
+                assert e[:k - 1].sum() / e.sum() < num / 100 + 1e-12
