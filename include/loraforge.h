@@ -70,7 +70,7 @@ typedef struct {
 } lf_module;
 
 /* Allocation policy.  kind 0 = LoRAForge-U, kind 1 = LoRAForge-S, kind 2 =
- * spectral budget on absolute energies (variant of S).
+ * spectral budget on absolute energies (variant of S), kind 3 = energy fraction.
  * ratio = ratio_num / ratio_den (exact integers, e.g. 1/4, 1/12); floor >= 1.
  *  U: k = clamp(floor(ratio_num*r/ratio_den + 1/2), floor, r).
  *  S: per group, K = floor(ratio_num * sum r / ratio_den); every module gets
@@ -79,6 +79,12 @@ typedef struct {
  *     ties to the lower module index, then lower j.
  *  kind 2: as S with e_ij = sigma_ij^2 (the choice that minimises the group's
  *     summed squared Frobenius error sum_i ||dW_i - B'_i A'_i||^2 under the budget).
+ *  kind 3: per module, the smallest k in [floor, r] whose leading directions keep
+ *     ratio_num / ratio_den (<= 1) of its spectral energy,
+ *     ratio_den * sum_{j<k} sigma_j^2 >= ratio_num * sum_j sigma_j^2 (LoRASpace's
+ *     minimal subspace keeping 99 % of the energy, read per module); no group budget.
+ *  Spectral kinds (1-3) recompute in fp64 the modules whose decision lies within a
+ *  1e-4 relative band of the threshold, so ranks match an fp64 reference.
  * The budget scope is the module `group`: one group per adapter gives per-adapter
  * budgets, one group over all modules a fleet-wide budget. */
 typedef struct {

@@ -96,8 +96,9 @@ static lf_status check_mods(const lf_module* mods, int32_t n) {
 }
 
 static lf_status check_policy(const lf_module* mods, int32_t n, lf_policy p) {
-    if (p.kind < 0 || p.kind > 2) return LF_ERR_INVALID_ARG;
+    if (p.kind < 0 || p.kind > 3) return LF_ERR_INVALID_ARG;
     if (p.ratio_num < 0 || p.ratio_den <= 0 || p.floor < 1) return LF_ERR_INVALID_ARG;
+    if (p.kind == 3 && p.ratio_num > p.ratio_den) return LF_ERR_INVALID_ARG;   // a fraction of the energy
     for (int32_t i = 0; i < n; ++i)
         if (p.floor > mods[i].r) return LF_ERR_SHAPE;
     return LF_OK;
@@ -908,10 +909,11 @@ void lf_export_pool_bound(const lf_module* mods, int32_t n, lf_policy pol, int64
     if (!cap_A || !cap_Bt) return;
     *cap_A = *cap_Bt = 0;
     if (check_mods(mods, n) != LF_OK || check_policy(mods, n, pol) != LF_OK) return;
-    if (pol.kind == 0) {
+    if (pol.kind == 0 || pol.kind == 3) {   // kind 3 may keep every direction: bound by r
         for (int32_t i = 0; i < n; ++i) {
             const int r = mods[i].r;
-            const int k = std::min(r, std::max(pol.floor, (pol.ratio_num * r + pol.ratio_den / 2) / pol.ratio_den));
+            const int k = pol.kind == 3 ? r
+                                        : std::min(r, std::max(pol.floor, (pol.ratio_num * r + pol.ratio_den / 2) / pol.ratio_den));
             *cap_A += (int64_t)k * mods[i].d_in;
             *cap_Bt += (int64_t)k * mods[i].d_out;
         }

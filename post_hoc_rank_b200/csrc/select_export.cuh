@@ -83,6 +83,40 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelArgs a) {
         }
         return;
     }
+    if (a.pol.kind == 3) {  // energy fraction: smallest k >= floor with den * sum_{j<k} s_j^2 >= num * sum_j s_j^2
+        for (int mi = threadIdx.x; mi < M; mi += blockDim.x) {
+            const int i = a.grp_mods[m0 + mi];
+            const int r = a.mods[i].r;
+            const double* sg = a.sigma + (size_t)i * a.rs;
+            double tot = 0.0;
+            for (int j = 0; j < r; ++j) {
+                tot += sg[j] * sg[j];
+                if (j + 1 < r && sg[j + 1] > sg[j]) latch_error(LF_ERR_INVALID_ARG);  // rows must descend
+            }
+            if (!isfinite(tot)) latch_error(LF_ERR_NUMERIC);
+            int k = fl;
+            bool near = false;
+            if (tot > 0.0) {
+                const double rhs = (double)a.pol.ratio_num * tot;
+                double cum = 0.0;
+                int found = 0;
+                for (int j = 0; j < r; ++j) {
+                    cum += sg[j] * sg[j];
+                    if (j + 1 < fl) continue;
+                    const double lhs = (double)a.pol.ratio_den * cum;
+                    if (!found && lhs >= rhs) found = j + 1;
+                    if (rhs > 0.0 && fabs(lhs - rhs) <= a.band * rhs) near = true;   // within the fp32 SVD's reach
+                }
+                k = found ? found : r;
+            }
+            a.ranks[i] = min(r, max(fl, k));
+            if (a.flag_list && near) {
+                const int slot = atomicAdd(a.flag_count, 1);
+                a.flag_list[slot] = i;
+            }
+        }
+        return;
+    }
     // energies, one module per thread, summed in j order
     int64_t rsum = 0;
     for (int mi = threadIdx.x; mi < M; mi += blockDim.x) {

@@ -48,6 +48,12 @@ def policy_S(num: int, den: int, floor: int = 1, absolute: bool = False) -> lf_p
     return lf_policy(2 if absolute else 1, num, den, floor)
 
 
+def policy_E(num: int, den: int, floor: int = 1) -> lf_policy:
+    """Energy fraction (kind 3): the smallest rank >= floor keeping num/den of each
+    module's spectral energy."""
+    return lf_policy(3, num, den, floor)
+
+
 class lf_phase_time(ctypes.Structure):
     _fields_ = [("name", ctypes.c_char * 32), ("total_ms", ctypes.c_double), ("launches", ctypes.c_int64)]
 

@@ -96,7 +96,8 @@ def test_policy_validation_on_host():
     m = tiny_mods()
     p, n = m.ctypes.data, m.shape[0]
     L = lf.lib()
-    bad_policies = [lf.lf_policy(3, 1, 4, 1), lf.lf_policy(-1, 1, 4, 1), lf.lf_policy(0, 1, 0, 1), lf.lf_policy(1, 1, 4, 0)]
+    bad_policies = [lf.lf_policy(4, 1, 4, 1), lf.lf_policy(-1, 1, 4, 1), lf.lf_policy(0, 1, 0, 1), lf.lf_policy(1, 1, 4, 0),
+                    lf.lf_policy(3, 101, 100, 1)]   # kind 3 takes a fraction of the energy (num <= den)
     for pol in bad_policies:
         assert L.lf_select_ranks(p, n, pol, 16, 16, 16, 16, 16, 1 << 20, None) == 1
     assert L.lf_select_ranks(p, n, lf.lf_policy(1, 1, 4, 17), 16, 16, 16, 16, 16, 1 << 20, None) == 2

@@ -266,3 +266,24 @@ def test_allocation_variants_ranks_bit_exact(variant):
         assert ranks_g[lay.group == g].sum() <= (64 * int((lay.group == g).sum())) // 12
     for eg, eo in G.recon_errors(lay, Bh, Ah, E, sig, range(lay.n)):
         assert abs(eg - eo) <= G.RECON_TOL
+
+
+@pytest.mark.parametrize("num,den", [(99, 100), (9, 10), (1, 2)])
+def test_energy_fraction_ranks_bit_exact(num, den):
+    # kind 3: the smallest rank keeping num/den of each module's spectral energy (the
+    # minimal subspace rule of LoRASpace, per module); modules near the threshold are
+    # refined in fp64 like the spectral budget's boundary
+    shapes = [("q", 896, 896), ("k", 128, 896), ("gate", 4736, 896), ("down", 896, 4736)]
+    lay = synth.fleet_layout(3, shapes=shapes, r=64, n_layers=2)
+    Bh = torch.zeros(lay.B_total); Ah = torch.zeros(lay.A_total)
+    synth.fill_fleet(lay, Bh, Ah, cfg_id=14)
+    B, A = upload(Bh, Ah)
+    mods, F, E, st = G.run_factor_path(lay, B, A, lf.policy_E(num, den, 1))
+    assert st == 0
+    sig = G.oracle_sigma_rows(lay, Bh, Ah, range(lay.n))
+    ranks_o, gaps = OA.energy_fraction_ranks(sig, lay.r, num, den, 1)
+    ranks_g = E.ranks.cpu().numpy()
+    diff = ranks_g != ranks_o
+    assert not np.any(diff & (gaps > 1e-12)), (ranks_g[diff], ranks_o[diff], gaps[diff])
+    for eg, eo in G.recon_errors(lay, Bh, Ah, E, sig, range(lay.n)):
+        assert abs(eg - eo) <= G.RECON_TOL
