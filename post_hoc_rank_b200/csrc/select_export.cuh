@@ -404,6 +404,10 @@ template <int NQ>
 __device__ __forceinline__ void export_stage_b(const ExportArgs& a, const lf_module& md, int k, const float* coef,
                                                const float* st, int i0, int nrem, int64_t obase, int jbase) {
     const int tid = threadIdx.x, e = tid & (kExpRows - 1), g = tid >> 6;
+    // outputs j = jbase + g + 4q of this thread; g is uniform over a warp, so the
+    // directions past k are skipped without divergence (NQ covers the largest k)
+    const int nq = min(NQ, max(0, (k - jbase - g + 3) / 4));
+    if (nq == 0) return;
     float acc[NQ];
 #pragma unroll
     for (int q = 0; q < NQ; ++q) acc[q] = 0.f;
@@ -413,8 +417,10 @@ __device__ __forceinline__ void export_stage_b(const ExportArgs& a, const lf_mod
         const float4 x = *reinterpret_cast<const float4*>(row + 4 * (c ^ (e & 7)));
 #pragma unroll
         for (int q = 0; q < NQ; ++q) {
-            const float4 cf = *reinterpret_cast<const float4*>(coef + (jbase + g + 4 * q) * kMaxRank + 4 * c);
-            acc[q] = fmaf(cf.x, x.x, fmaf(cf.y, x.y, fmaf(cf.z, x.z, fmaf(cf.w, x.w, acc[q]))));
+            if (q < nq) {
+                const float4 cf = *reinterpret_cast<const float4*>(coef + (jbase + g + 4 * q) * kMaxRank + 4 * c);
+                acc[q] = fmaf(cf.x, x.x, fmaf(cf.y, x.y, fmaf(cf.z, x.z, fmaf(cf.w, x.w, acc[q]))));
+            }
         }
     }
     if (e >= nrem) return;
