@@ -277,9 +277,10 @@ lf_status lf_lora_sigma_sandwich(int32_t T, int32_t d_in, int32_t d_out, const v
  * previous iterate, with P_i = A_i V and Q_i = B_i^T U:
  *     U <- orthogonalize(sum_i w_i B_i (P_i (P_i^T Q_i))),
  *     V <- orthogonalize(sum_i w_i A_i^T (Q_i (Q_i^T P_i))),
- * orthogonalize = the Q of the thin QR with positive diag(R) (the factor-
- * construction TSQR gives R, then Q = X R^-1, done twice).  Afterwards, if
- * `sigma` is not null, Sigma_i = U^T B_i A_i V (eq. 6) at the final U, V.
+ * orthogonalize = the Q of the thin QR with positive diag(R): the factor-
+ * construction TSQR's Gram leaf and fp64 Cholesky give R, then Q = X R^-1; a matrix
+ * whose pivot is rejected takes the Householder TSQR and a second round on Q.
+ * Afterwards, if `sigma` is not null, Sigma_i = U^T B_i A_i V (eq. 6) at the final U, V.
  * Contractions run on the fp64 tensor-core path (fp32 inputs, exact products,
  * fp64 sums); U, V and Sigma are stored fp32.
  * State: U of problem p at U_base + U_off (d_out x rank fp32, row-major), V^T at

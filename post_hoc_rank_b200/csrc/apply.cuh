@@ -456,18 +456,21 @@ __global__ void route_check_kernel(int32_t* tag, int32_t* counts, int T, int n_a
 }
 
 // Decode regime, token-parallel (BGMV form: every token carries its adapter index,
-// no sorting).  CTA (token, 8192-column chunk of one slice): t = A' x (k fp32 dot
+// no sorting).  CTA (token, 16384-column chunk of one slice): t = A' x (k fp32 dot
 // products over d_in, reduced across the CTA in a fixed order), then
-// y[chunk] += s * B'^T t with 16-byte loads of the k rows of B'^T.  Each chunk CTA
-// recomputes the same t (identical arithmetic; x and A' come from L2), and tokens
+// y[chunk] += s * B'^T t with 16-byte loads of the k rows of B'^T.  A chunk covers a
+// whole projection up to 16384 columns, so t is formed once per (token, slice); wider
+// slices recompute it per chunk (identical arithmetic; x and A' come from L2).  Tokens
 // of one adapter read its factors from L2 after the first touch, so HBM sees every
-// distinct factor row, x and y once.
-constexpr int kBgmvThreads = 256;
+// distinct factor row, x and y once.  512 threads: a 4096-wide x row is one 16-byte
+// load per thread, so the shrink's loads go out in one round (swept 256 / 512 / 1024
+// threads and 8192 / 12288 / 16384 columns on the decode workload).
+constexpr int kBgmvThreads = 512;
 constexpr int kBgmvVec = 4;                                  // 8-column vectors per thread in the expand
 constexpr int kBgmvCols = kBgmvThreads * 8 * kBgmvVec;       // d_out columns per CTA
 constexpr int kBgmvJ = 8;                                    // retained directions per shrink pass
 
-__global__ void __launch_bounds__(kBgmvThreads, 4) bgmv_kernel(ApplyArgs a) {
+__global__ void __launch_bounds__(kBgmvThreads, 2) bgmv_kernel(ApplyArgs a) {
     __shared__ float red[kBgmvThreads / 32][kBgmvJ];
     __shared__ float ts[kMaxRank];
     __shared__ float tw[kMaxRank];

@@ -670,7 +670,7 @@ static JdLayout jd_layout(int32_t n_mods, int32_t n_probs, const JdPlan& P) {
     LF_TAKE(wsVt, float, (size_t)P.ws_Vt);
     LF_TAKE(RB, float, (size_t)n_probs * rs2);
     LF_TAKE(RA, float, (size_t)n_probs * rs2);
-    LF_TAKE(R64, double, (size_t)4 * n_probs * rs2);   // two rounds x two factors
+    LF_TAKE(R64, double, (size_t)2 * n_probs * rs2);   // round 2, two factors per problem
     LF_TAKE(Rinv, double, (size_t)2 * n_probs * rs2);
 #undef LF_TAKE
     L.total = c.off + 256;
@@ -1350,8 +1350,7 @@ lf_status lf_jd_full(const lf_module* mods, int32_t n_mods, const int32_t* membe
     int32_t* hh1_cnt = oc + 4 * n_probs;
     int32_t* hh2_cnt = oc + 6 * n_probs;
     int32_t* flags2 = oc + 8 * n_probs;
-    double* R64_1 = reinterpret_cast<double*>(at(L.R64));
-    double* R64_2 = R64_1 + 2 * n_probs * rs2;
+    double* R64_2 = reinterpret_cast<double*>(at(L.R64));   // round 2's fp64 R (round 1 inverts in jd_chol)
     const TsqrWork* owork = reinterpret_cast<const TsqrWork*>(at(L.owork));
     const int32_t* onw = reinterpret_cast<const int32_t*>(at(L.onwork));
     const TsqrInfo* oinfo = reinterpret_cast<const TsqrInfo*>(at(L.oinfo));
@@ -1372,7 +1371,7 @@ lf_status lf_jd_full(const lf_module* mods, int32_t n_mods, const int32_t* membe
     ra1.basis = d_bw;
     ra1.only = flags1;
     ra1.use32 = flags1;
-    ra1.R64 = R64_1;
+    ra1.R64 = nullptr;   // round 1 inverts only Householder R (use32 set for every matrix it takes)
     ra1.R_B = RB;
     ra1.R_A = RA;
     ra1.Rinv = Rinv;
