@@ -336,7 +336,7 @@ __global__ void __launch_bounds__(kTcExpThreads, 1) expand_tc_kernel(ApplyArgs a
         const int e0 = e_begin + i * kTcN2;
         __nv_bfloat16* dst = s.yt[i % kTcYBuf];
         for (int c = tid; c < kTcM * (kTcN2 / 8); c += kTcExpThreads) {
-            const int row = c >> 4, ch = c & 15;
+            const int row = c / (kTcN2 / 8), ch = c % (kTcN2 / 8);
             const int e = e0 + ch * 8;
             const bool ok = row < nt && e < e_end;
             cp_async16_zfill(dst + row * kTcYLd + ch * 8, ok ? ybase + (int64_t)s.toks[row] * a.y_ld + e : ybase, ok);
@@ -393,10 +393,10 @@ __global__ void __launch_bounds__(kTcExpThreads, 1) expand_tc_kernel(ApplyArgs a
         __nv_bfloat16* yt = s.yt[i % kTcYBuf];
         if (ok) {
 #pragma unroll
-            for (int c16 = 0; c16 < 4; ++c16) {
+            for (int c16 = 0; c16 < kTcN2 / 32; ++c16) {
                 float v[16];
-                tc::tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(64 * h + 16 * c16), v);
-                uint4* yp = reinterpret_cast<uint4*>(yt + m * kTcYLd + 64 * h + 16 * c16);
+                tc::tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)((kTcN2 / 2) * h + 16 * c16), v);
+                uint4* yp = reinterpret_cast<uint4*>(yt + m * kTcYLd + (kTcN2 / 2) * h + 16 * c16);
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
                     uint4 yv = yp[half];
@@ -416,7 +416,7 @@ __global__ void __launch_bounds__(kTcExpThreads, 1) expand_tc_kernel(ApplyArgs a
         if (ok) {
             const int e0 = e_begin + i * kTcN2;
             for (int c = tid; c < kTcM * (kTcN2 / 8); c += kTcExpThreads) {
-                const int row = c >> 4, ch = c & 15;
+                const int row = c / (kTcN2 / 8), ch = c % (kTcN2 / 8);
                 const int e = e0 + ch * 8;
                 if (row < nt && e < e_end)
                     *reinterpret_cast<uint4*>(ybase + (int64_t)s.toks[row] * a.y_ld + e) =
