@@ -279,7 +279,7 @@ lf_status lf_lora_sigma_sandwich(int32_t T, int32_t d_in, int32_t d_out, const v
  *     V <- orthogonalize(sum_i w_i A_i^T (Q_i (Q_i^T P_i))),
  * orthogonalize = the Q of the thin QR with positive diag(R): the factor-
  * construction TSQR's Gram leaf and fp64 Cholesky give R, then Q = X R^-1; a matrix
- * whose pivot is rejected takes the Householder TSQR and a second round on Q.
+ * whose pivot is rejected takes the Householder TSQR and a second pass on Q.
  * Afterwards, if `sigma` is not null, Sigma_i = U^T B_i A_i V (eq. 6) at the final U, V.
  * Contractions run on the fp64 tensor-core path (fp32 inputs, exact products,
  * fp64 sums); U, V and Sigma are stored fp32.

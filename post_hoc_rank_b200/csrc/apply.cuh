@@ -463,7 +463,7 @@ __global__ void route_check_kernel(int32_t* tag, int32_t* counts, int T, int n_a
 // slices recompute it per chunk (identical arithmetic; x and A' come from L2).  Tokens
 // of one adapter read its factors from L2 after the first touch, so HBM sees every
 // distinct factor row, x and y once.  512 threads: a 4096-wide x row is one 16-byte
-// load per thread, so the shrink's loads go out in one round (swept 256 / 512 / 1024
+// load per thread, so the shrink's loads are all in flight together (swept 256 / 512 / 1024
 // threads and 8192 / 12288 / 16384 columns on the decode workload).
 constexpr int kBgmvThreads = 512;
 constexpr int kBgmvVec = 4;                                  // 8-column vectors per thread in the expand

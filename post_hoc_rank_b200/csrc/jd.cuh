@@ -14,7 +14,7 @@
 // epilogue forms the Gram of each finished 128-row tile (the TSQR leaf), the tiles are
 // merged in order and the fp64 Cholesky is taken (the root), and Q = X R^-1 uses that
 // fp64 R (orthonormal to ~kappa^2 u_64 + u_32).  A matrix whose pivot is rejected
-// gets its R from the Householder TSQR kernel instead and a second round (Gram leaf +
+// gets its R from the Householder TSQR kernel instead and a second pass (Gram leaf +
 // Cholesky on Q_1, then Q = Q_1 R_2^-1: CholeskyQR2) restores orthonormality.
 //
 // Kernels of one step, all fp64 on the tensor-core path (mma.m8n8k4.f64: every

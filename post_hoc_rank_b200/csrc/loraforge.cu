@@ -657,8 +657,8 @@ static JdLayout jd_layout(int32_t n_mods, int32_t n_probs, const JdPlan& P) {
     LF_TAKE(onwork, int32_t, 1);
     LF_TAKE(oinfo, TsqrInfo, P.orth.info.size());
     LF_TAKE(pcounters, int32_t, 2 * ng);
-    // orthogonalize: flags of round 1, Gram counters of round 2, Householder counters of
-    // both rounds, flags of round 2 (2 per problem each), zeroed every step
+    // orthogonalize: flags of pass 1, Gram counters of pass 2, Householder counters of
+    // both passes, flags of pass 2 (2 per problem each), zeroed every step
     LF_TAKE(ocounters, int32_t, (size_t)10 * n_probs);
     LF_TAKE(ppartial, double, (size_t)P.pslots * blk);
     LF_TAKE(opartial, char, (size_t)P.orth.slots * tsqr_slot_bytes(P.orth.RT));
@@ -670,7 +670,7 @@ static JdLayout jd_layout(int32_t n_mods, int32_t n_probs, const JdPlan& P) {
     LF_TAKE(wsVt, float, (size_t)P.ws_Vt);
     LF_TAKE(RB, float, (size_t)n_probs * rs2);
     LF_TAKE(RA, float, (size_t)n_probs * rs2);
-    LF_TAKE(R64, double, (size_t)2 * n_probs * rs2);   // round 2, two factors per problem
+    LF_TAKE(R64, double, (size_t)2 * n_probs * rs2);   // pass 2, two factors per problem
     LF_TAKE(Rinv, double, (size_t)2 * n_probs * rs2);
 #undef LF_TAKE
     L.total = c.off + 256;
@@ -1338,11 +1338,11 @@ lf_status lf_jd_full(const lf_module* mods, int32_t n_mods, const int32_t* membe
     ua.Vt_ws = wsVt;
     ua.gram = reinterpret_cast<double*>(at(L.tgram));
 
-    // orthogonalize (the state in the workspace -> the caller's U, V^T).  Round 1: tile
+    // orthogonalize (the state in the workspace -> the caller's U, V^T).  Pass 1: tile
     // Grams (update epilogue) -> jd_chol -> Householder TSQR for rejected matrices ->
     // Q = X R^-1, written to the caller's state, or back into the workspace for the
-    // rejected ones, which round 2 (Gram leaf + Cholesky on Q_1, Householder if
-    // rejected again, Q = Q_1 R_2^-1) finishes.  Round-2 kernels skip every other matrix.
+    // rejected ones, which pass 2 (Gram leaf + Cholesky on Q_1, Householder if
+    // rejected again, Q = Q_1 R_2^-1) finishes.  Pass-2 kernels skip every other matrix.
     const size_t rs2 = (size_t)P.orth.rs * P.orth.rs;
     int32_t* oc = reinterpret_cast<int32_t*>(at(L.ocounters));
     int32_t* flags1 = oc;
@@ -1350,7 +1350,7 @@ lf_status lf_jd_full(const lf_module* mods, int32_t n_mods, const int32_t* membe
     int32_t* hh1_cnt = oc + 4 * n_probs;
     int32_t* hh2_cnt = oc + 6 * n_probs;
     int32_t* flags2 = oc + 8 * n_probs;
-    double* R64_2 = reinterpret_cast<double*>(at(L.R64));   // round 2's fp64 R (round 1 inverts in jd_chol)
+    double* R64_2 = reinterpret_cast<double*>(at(L.R64));   // pass 2's fp64 R (pass 1 inverts in jd_chol)
     const TsqrWork* owork = reinterpret_cast<const TsqrWork*>(at(L.owork));
     const int32_t* onw = reinterpret_cast<const int32_t*>(at(L.onwork));
     const TsqrInfo* oinfo = reinterpret_cast<const TsqrInfo*>(at(L.oinfo));
@@ -1367,11 +1367,11 @@ lf_status lf_jd_full(const lf_module* mods, int32_t n_mods, const int32_t* membe
     cha.Rinv = Rinv;
     cha.flags = flags1;
     cha.rs = P.orth.rs;
-    JdRinvArgs ra1;   // round 1: only the matrices the Cholesky rejected (Householder R)
+    JdRinvArgs ra1;   // pass 1: only the matrices the Cholesky rejected (Householder R)
     ra1.basis = d_bw;
     ra1.only = flags1;
     ra1.use32 = flags1;
-    ra1.R64 = nullptr;   // round 1 inverts only Householder R (use32 set for every matrix it takes)
+    ra1.R64 = nullptr;   // pass 1 inverts only Householder R (use32 set for every matrix it takes)
     ra1.R_B = RB;
     ra1.R_A = RA;
     ra1.Rinv = Rinv;
