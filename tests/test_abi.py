@@ -181,3 +181,20 @@ def test_route_tokens_validation_on_host():
     assert L.lf_route_tokens(8, 16, 0, 16, 1 << 20, None) == 1
     assert L.lf_route_tokens(8, None, 4, 16, 1 << 20, None) == 1
     assert L.lf_route_tokens(1000, 16, 4, 16, 64, None) == 4          # workspace too small
+
+
+def test_routed_apply_validation_on_host():
+    """The routed entry point applies the same host checks as the unrouted one."""
+    L = lf.lib()
+    sl = (lf.lf_slice * 1)(lf.lf_slice(64, 0, 0, 16, 16, 16, 16, 16, 1024, 1024))
+
+    def call(T=4, d_in=64, ns=1, x=16, ws=16, wsb=1 << 20, y_ld=64):
+        return L.lf_lora_shrink_expand_slices_routed(T, d_in, x, 16, y_ld, 16, 2, sl, ns, 1.0, None, ws, wsb, None)
+    assert call(T=0) == 0
+    assert call(T=-1) == 1
+    assert call(ns=0) == 1
+    assert call(ns=5) == 1
+    assert call(d_in=60) == 8
+    assert call(x=8) == 8
+    assert call(wsb=8) == 4
+    assert call(ws=None) == 1

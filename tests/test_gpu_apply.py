@@ -342,3 +342,24 @@ def test_routed_call_without_matching_routing_applies_nothing():
     lf.lf_lora_shrink_expand_slices_routed(x, y, ids_d, n, keep, 1.0, ws)
     assert lf.lf_get_device_status() == 1
     assert torch.equal(y, y0)
+
+
+def test_routed_call_in_decode_regime_reads_ids():
+    """T <= 8 n: the token-parallel kernel indexes adapters per token, so a routed call
+    gives the unrouted result whatever the routing tables hold."""
+    T, n, d_in = 96, 32, 256
+    ids = synth.zipf_ids(T, n, 1.0, (14, 0))
+    ids_d = torch.from_numpy(ids).cuda()
+    x = synth.normal_bf16((T, d_in), (14, 1)).cuda()
+    sl, y_ld = make_slices([256, 128], n, d_in, (14, 2))
+    keep, _alive = _slice_tensors(sl)
+    y0 = synth.normal_bf16((T, y_ld), (14, 3)).cuda()
+    ws = api.workspace(lf.lf_apply_slices_workspace_size(T, n, 2), "cuda")
+    lf.lf_route_tokens(ids_d, n, ws)
+    y = y0.clone()
+    lf.lf_lora_shrink_expand_slices_routed(x, y, ids_d, n, keep, 0.5, ws)
+    y_ref = y0.clone()
+    lf.lf_lora_shrink_expand_slices(x, y_ref, ids_d, n, keep, 0.5,
+                                    api.workspace(lf.lf_apply_slices_workspace_size(T, n, 2), "cuda"))
+    assert lf.lf_get_device_status() == 0
+    assert torch.equal(y, y_ref)
