@@ -371,6 +371,40 @@ static size_t carve_apply(void* base, int64_t T, int64_t n, int ns, ApplyWs* w) 
     return c.off + 256;
 }
 
+// Tensor map of x (T rows of d_in bf16) for the tensor-core shrink's TMA stages: box of
+// 64 elements (128 bytes) x 128 rows, 128-byte swizzle, out-of-range reads as zeros.
+// cuTensorMapEncodeTiled is looked up once through the runtime's driver entry point.
+// Returns false (the shrink then gathers x with cp.async) when the lookup or the
+// encoding fails or the shape is below one box.
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+static EncodeTiledFn encode_tiled_fn() {
+    static std::once_flag once;
+    static EncodeTiledFn fn = nullptr;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q{};
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+static bool encode_x_map(CUtensorMap* map, const void* x, int32_t T, int32_t d_in) {
+    if (T < kTcM || d_in < kTcKB || (d_in & 7) || !aligned16(x)) return false;
+    const EncodeTiledFn fn = encode_tiled_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)d_in, (cuuint64_t)T};
+    const cuuint64_t strides[1] = {(cuuint64_t)d_in * 2};
+    const cuuint32_t box[2] = {(cuuint32_t)kTcKB, (cuuint32_t)kTcM};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(x), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Bounded grid of the grid-stride GEMV kernels: enough CTAs to fill the GPU (8 per
 // SM of 148), never more than the largest possible number of work units.
 static unsigned gemv_grid(int64_t max_units) {
@@ -498,15 +532,19 @@ static lf_status apply_impl(int32_t T, int32_t d_in, const void* x, void* y, int
     const unsigned max_tc = (unsigned)(T / kTcM + mseg + 1);
     const unsigned nsplit = (unsigned)cdiv(d_in, tc_split_len(d_in));
     set_chunks(A, kTcCols);
+    alignas(64) CUtensorMap xmap;
+    std::memset(&xmap, 0, sizeof(xmap));
+    const int x_tma = encode_x_map(&xmap, x, T, d_in) ? 1 : 0;
     if (ns == 1) {
         constexpr size_t sm = shrink_tc_smem<kMaxRank>();
         LF_CUDA_TRY(cudaFuncSetAttribute(shrink_tc_kernel<kMaxRank>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm));
-        LF_LAUNCH("shrink_tc", shrink_tc_kernel<kMaxRank>, dim3(max_tc, nsplit), kTcThreads, sm, s, A);
+        LF_LAUNCH("shrink_tc", shrink_tc_kernel<kMaxRank>, dim3(max_tc, nsplit), kTcThreads, sm, s, A, xmap, x_tma);
     } else {
         constexpr size_t sm = shrink_tc_smem<kMaxSlices * kMaxRank>();
         LF_CUDA_TRY(cudaFuncSetAttribute(shrink_tc_kernel<kMaxSlices * kMaxRank>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm));
-        LF_LAUNCH("shrink_tc", shrink_tc_kernel<kMaxSlices * kMaxRank>, dim3(max_tc, nsplit), kTcThreads, sm, s, A);
+        LF_LAUNCH("shrink_tc", shrink_tc_kernel<kMaxSlices * kMaxRank>, dim3(max_tc, nsplit), kTcThreads, sm, s, A,
+                  xmap, x_tma);
     }
     LF_CUDA_TRY(cudaGetLastError());
     LF_CUDA_TRY(cudaFuncSetAttribute(expand_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kExpandTcSmem));
@@ -1343,7 +1381,6 @@ lf_status lf_jd_full(const lf_module* mods, int32_t n_mods, const int32_t* membe
     // Q = X R^-1, written to the caller's state, or back into the workspace for the
     // rejected ones, which pass 2 (Gram leaf + Cholesky on Q_1, Householder if
     // rejected again, Q = Q_1 R_2^-1) finishes.  Pass-2 kernels skip every other matrix.
-    const size_t rs2 = (size_t)P.orth.rs * P.orth.rs;
     int32_t* oc = reinterpret_cast<int32_t*>(at(L.ocounters));
     int32_t* flags1 = oc;
     int32_t* gram2_cnt = oc + 2 * n_probs;

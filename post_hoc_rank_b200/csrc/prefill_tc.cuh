@@ -9,12 +9,16 @@
 //   TMEM, N = the sum of the slices' ranks rounded up to 16 (padding lives in shared
 //   memory only): x is read once for every slice that shares it.  X rows are
 //   gathered through the token permutation with 16-byte cp.async into a 4-stage
-//   ring of K-major core matrices; one thread issues the MMAs and commits each
-//   stage to an mbarrier that frees the stage for the next copy.
+//   ring of K-major core matrices, or, when the tile's tokens are consecutive rows
+//   of x (a prefill request), loaded by one 2-D TMA copy per stage; one thread
+//   issues the MMAs and commits each stage to an mbarrier that frees the stage for
+//   the next copy.
 // Expand (per slice): D[128 x 128] = t_hi * B + t_lo * B with t = t_hi + t_lo split
 //   into two bf16 values (about 16 significant bits of the fp32 t); B = B'^T tile,
 //   MN-major; the epilogue reads D from tensor memory and updates y once.
 #pragma once
+#include <cuda.h>   // CUtensorMap (type only)
+
 #include "apply_common.cuh"
 #include "tc.cuh"
 
@@ -44,9 +48,13 @@ __host__ __device__ inline int tc_split_len(int d_in) {
 //     with 16-byte cp.async; kTcAhead stages stay in flight; once a stage's copies
 //     have landed (cp.async.wait_group) each lane fences them to the async proxy and
 //     arrives on the stage's `full` barrier; a stage is refilled after the
-//     tcgen05.commit of the MMAs that read it arrives on its `empty` barrier;
-//   warp 1 lane 0, MMA issuer: waits on `full`, issues four K = 16 MMAs into TMEM,
-//     commits to `empty`, and at the end to `done`;
+//     tcgen05.commit of the MMAs that read it arrives on its `empty` barrier.
+//     When the tile's tokens are consecutive rows of x and the caller encoded a
+//     tensor map of x (box 64 x 128, 128-byte swizzle), warp 0 lane 0 loads the x
+//     stage with one TMA copy counted on the stage's `xfull` barrier instead, and
+//     before leaving waits for every copy it issued;
+//   warp 1 lane 0, MMA issuer: waits on `full` (and `xfull`), issues four K = 16
+//     MMAs into TMEM, commits to `empty`, and at the end to `done`;
 //   all warps: epilogue from TMEM (warp w reads lanes 32w ..) into t_part.
 constexpr int kTcAhead = 2;      // stages in flight before the producers signal the oldest
 constexpr int kTcProducers = 3;  // producer warps: 0, 2, 3 (warp 1 issues the MMAs)
@@ -57,6 +65,7 @@ struct ShrinkTcSmem {
     __nv_bfloat16 b[kTcStages][MAXN * kTcKB];    //  8 KB (MAXN 64) or 32 KB (MAXN 256) per stage
     uint64_t full[kTcStages];
     uint64_t empty[kTcStages];
+    uint64_t xfull[kTcStages];   // TMA x stages (tx bytes)
     uint64_t done;
     uint32_t tmem;
     int32_t toks[kTcM];
@@ -75,8 +84,12 @@ __device__ __forceinline__ void cp_async16_zfill(void* dst, const void* src, boo
 }
 
 
+constexpr uint32_t kTcXStageBytes = kTcM * kTcKB * 2;   // one TMA box of x
+
+// x_tma: the caller encoded `xmap` (x as d_in x T bf16, box 64 x 128, 128-byte swizzle).
 template <int MAXN>
-__global__ void __launch_bounds__(kTcThreads) shrink_tc_kernel(ApplyArgs a) {
+__global__ void __launch_bounds__(kTcThreads) shrink_tc_kernel(ApplyArgs a, const __grid_constant__ CUtensorMap xmap,
+                                                               int x_tma) {
     extern __shared__ __align__(1024) unsigned char tc_raw[];
     auto& s = *reinterpret_cast<ShrinkTcSmem<MAXN>*>(tc_raw);
     if ((int)blockIdx.x >= a.counts[3]) return;
@@ -99,7 +112,10 @@ __global__ void __launch_bounds__(kTcThreads) shrink_tc_kernel(ApplyArgs a) {
         s.kcum[0] = 0;
         for (int q = 1; q <= a.n_slices; ++q) s.kcum[q] += s.kcum[q - 1];
     }
-    __syncthreads();
+    bool consecutive = true;
+    for (int m = tid; m < nt; m += kTcThreads) consecutive = consecutive && s.toks[m] == s.toks[0] + m;
+    // uniform: x stages by TMA (rows toks[0] .. +127; rows past nt are never stored)
+    const bool tma = __syncthreads_and(consecutive) && x_tma != 0 && (smem_u32(s.a[0]) & 1023u) == 0;
     const int ktot = s.kcum[a.n_slices];
     if (ktot <= 0) return;   // uniform
     const int npad = (ktot + 15) & ~15;
@@ -114,6 +130,7 @@ __global__ void __launch_bounds__(kTcThreads) shrink_tc_kernel(ApplyArgs a) {
         for (int i = 0; i < kTcStages; ++i) {
             mbar_init(&s.full[i], 32 * kTcProducers);
             mbar_init(&s.empty[i], 1);
+            mbar_init(&s.xfull[i], 1);
         }
         mbar_init(&s.done, 1);
         fence_barrier_init();
@@ -129,16 +146,23 @@ __global__ void __launch_bounds__(kTcThreads) shrink_tc_kernel(ApplyArgs a) {
     const int pidx = warp == 0 ? 0 : warp - 1;   // producer index (warps 0, 2, 3)
     if (warp != 1 && pidx < kTcProducers) {   // producers
         const __nv_bfloat16* A0 = a.sl[0].A_pool + s.oa[0];   // the only slice when MAXN == 64
+        const bool x_issuer = tma && warp == 0 && lane == 0;
+        int x_issued = 0;   // TMA x stages issued by this thread
         for (int kb = 0; kb < nK && ok; ++kb) {
             const int st = kb % kTcStages;
             if (kb >= kTcStages) ok = mbar_wait(&s.empty[st], (uint32_t)((kb / kTcStages - 1) & 1));
             if (!ok) break;
             char* abase = reinterpret_cast<char*>(s.a[st]);
             char* bbase = reinterpret_cast<char*>(s.b[st]);
-            const int k0 = kbeg + kb * kTcKB;
+            const int k0 = kbeg + kb * kTcKB;   // a multiple of 64 elements (128 bytes)
+            if (x_issuer) {
+                mbar_arrive_expect_tx(&s.xfull[st], kTcXStageBytes);
+                tc::tma_load_2d(abase, &xmap, k0, s.toks[0], &s.xfull[st]);
+                ++x_issued;
+            }
             // chunk mapping: a half-warp covers 8 rows x 32 contiguous bytes (full sectors);
             // each quarter-warp writes 8 rows of one 16-byte column (distinct banks)
-            for (int i = pidx; i < (kTcM * kTcKB / 8) / 32; i += kTcProducers) {
+            for (int i = pidx; !tma && i < (kTcM * kTcKB / 8) / 32; i += kTcProducers) {
                 const int u = 2 * i + (lane >> 4);
                 const int m = 8 * (u & 15) + (lane & 7);
                 const int kc = 2 * (u >> 4) + ((lane >> 3) & 1);
@@ -173,16 +197,22 @@ __global__ void __launch_bounds__(kTcThreads) shrink_tc_kernel(ApplyArgs a) {
         tc::fence_proxy_async();
         if (ok)
             for (int kb = max(0, nK - kTcAhead); kb < nK; ++kb) mbar_arrive1(&s.full[kb % kTcStages]);
+        // no TMA copy of this thread is still in flight when the CTA leaves (on the
+        // normal path these phases completed before the MMAs that read them)
+        for (int kb = max(0, x_issued - kTcStages); kb < x_issued; ++kb)
+            if (!mbar_wait(&s.xfull[kb % kTcStages], (uint32_t)((kb / kTcStages) & 1))) ok = false;
     } else if (warp == 1 && lane == 0) {   // MMA issuer
         const uint32_t idesc = tc::idesc_bf16(kTcM, npad, 0, 0);
         for (int kb = 0; kb < nK && ok; ++kb) {
             const int st = kb % kTcStages;
             ok = mbar_wait(&s.full[st], (uint32_t)((kb / kTcStages) & 1));
+            if (ok && tma) ok = mbar_wait(&s.xfull[st], (uint32_t)((kb / kTcStages) & 1));
             if (!ok) break;
             tc::fence_after_sync();
 #pragma unroll
             for (int ks = 0; ks < kTcKB / 16; ++ks) {
-                const uint64_t ad = tc::smem_desc(reinterpret_cast<char*>(s.a[st]) + ks * 256, 128, 1024);
+                const uint64_t ad = tma ? tc::smem_desc_sw128(reinterpret_cast<char*>(s.a[st]) + ks * 32)
+                                        : tc::smem_desc(reinterpret_cast<char*>(s.a[st]) + ks * 256, 128, 1024);
                 const uint64_t bd = tc::smem_desc(reinterpret_cast<char*>(s.b[st]) + ks * 256, 128, 1024);
                 tc::mma_bf16(tmem, ad, bd, idesc, kb > 0 || ks > 0);
             }

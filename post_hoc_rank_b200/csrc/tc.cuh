@@ -1,7 +1,8 @@
-// Thin wrappers over the sm_100a tensor-core (tcgen05) and tensor-memory
+// Thin wrappers over the sm_100a tensor-core (tcgen05), tensor-memory and TMA
 // instructions used by the prefill kernels.  Layouts follow the PTX ISA's
-// canonical shared-memory matrix descriptors (no swizzle): a "core matrix" is
-// 8 rows x 16 bytes stored contiguously (128 bytes).
+// canonical shared-memory matrix descriptors: without swizzle a "core matrix" is
+// 8 rows x 16 bytes stored contiguously (128 bytes); the 128-byte swizzle layout is
+// the one a TMA tile load writes.
 #pragma once
 #include "common.cuh"
 
@@ -21,6 +22,34 @@ __device__ __forceinline__ uint64_t smem_desc(const void* p, uint32_t lbo_bytes,
     d |= 1ull << 46;   // descriptor version for sm_100
     // base offset 0, LBO mode 0, layout type 0 = SWIZZLE_NONE
     return d;
+}
+
+// Shared-memory matrix descriptor of a K-major bf16 operand in the 128-byte swizzle
+// layout, as a 2-D TMA load with CU_TENSOR_MAP_SWIZZLE_128B and a 64-element inner box
+// writes it: row r at r * 128 bytes with its 16-byte chunks XOR-permuted by r % 8, atoms
+// of 8 rows (1024 bytes, the SBO).  The tile must start 1024-byte aligned; `p` is the
+// tile plus 32 bytes per K = 16 step (the swizzle is applied to the full address).
+// Layout type 2 (bits 61-63) = 128-byte swizzle; LBO is unused for this layout (1).
+__device__ __forceinline__ uint64_t smem_desc_sw128(const void* p) {
+    const uint64_t addr = smem_u32(p);
+    uint64_t d = 0;
+    d |= (addr >> 4) & 0x3FFFull;
+    d |= 1ull << 16;                        // LBO (unused)
+    d |= (uint64_t)(1024 >> 4) << 32;       // SBO: 8-row atoms
+    d |= 1ull << 46;                        // descriptor version for sm_100
+    d |= 2ull << 61;                        // layout type: 128-byte swizzle
+    return d;
+}
+
+// 2-D tiled TMA load (no multicast) of the tensor map's box at coordinates (c0 =
+// innermost, c1) into this CTA's shared memory; completion is counted in bytes on
+// `bar`.  c0 * element size must be a multiple of 16 bytes; rows or columns outside the
+// tensor read as zeros.
+__device__ __forceinline__ void tma_load_2d(void* dst, const void* tmap, int c0, int c1, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+        ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(tmap)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
+        : "memory");
 }
 
 // Instruction descriptor, kind::f16 with bf16 inputs and fp32 accumulation.
