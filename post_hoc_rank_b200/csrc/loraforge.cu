@@ -371,11 +371,11 @@ static size_t carve_apply(void* base, int64_t T, int64_t n, int ns, ApplyWs* w) 
     return c.off + 256;
 }
 
-// Tensor map of x (T rows of d_in bf16) for the tensor-core shrink's TMA stages: box of
-// 64 elements (128 bytes) x 128 rows, 128-byte swizzle, out-of-range reads as zeros.
-// cuTensorMapEncodeTiled is looked up once through the runtime's driver entry point.
-// Returns false (the shrink then gathers x with cp.async) when the lookup or the
-// encoding fails or the shape is below one box.
+// Tensor maps for the tensor-core kernels' TMA stages: box of 64 elements (128 bytes)
+// x 128 rows, 128-byte swizzle, out-of-range reads as zeros (and are not written by
+// stores).  cuTensorMapEncodeTiled is looked up once through the runtime's driver
+// entry point.  encode_rows_map returns false (the kernels then gather rows with
+// cp.async) when the lookup or the encoding fails or the shape is below one box.
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                    const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                    CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
@@ -392,15 +392,18 @@ static EncodeTiledFn encode_tiled_fn() {
     return fn;
 }
 
-static bool encode_x_map(CUtensorMap* map, const void* x, int32_t T, int32_t d_in) {
-    if (T < kTcM || d_in < kTcKB || (d_in & 7) || !aligned16(x)) return false;
+// Tensor map of a row-major bf16 matrix of `rows` rows of `cols` elements (row stride
+// `cols`), box 64 x 128, for the tensor-core kernels' TMA stages (x for the shrink,
+// y for the expand).
+static bool encode_rows_map(CUtensorMap* map, const void* base, int32_t rows, int64_t cols) {
+    if (rows < kTcM || cols < kTcKB || (cols & 7) || !aligned16(base)) return false;
     const EncodeTiledFn fn = encode_tiled_fn();
     if (!fn) return false;
-    const cuuint64_t dims[2] = {(cuuint64_t)d_in, (cuuint64_t)T};
-    const cuuint64_t strides[1] = {(cuuint64_t)d_in * 2};
+    const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
     const cuuint32_t box[2] = {(cuuint32_t)kTcKB, (cuuint32_t)kTcM};
     const cuuint32_t estr[2] = {1, 1};
-    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(x), dims, strides, box, estr,
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -532,9 +535,11 @@ static lf_status apply_impl(int32_t T, int32_t d_in, const void* x, void* y, int
     const unsigned max_tc = (unsigned)(T / kTcM + mseg + 1);
     const unsigned nsplit = (unsigned)cdiv(d_in, tc_split_len(d_in));
     set_chunks(A, kTcCols);
-    alignas(64) CUtensorMap xmap;
+    alignas(64) CUtensorMap xmap, ymap;
     std::memset(&xmap, 0, sizeof(xmap));
-    const int x_tma = encode_x_map(&xmap, x, T, d_in) ? 1 : 0;
+    std::memset(&ymap, 0, sizeof(ymap));
+    const int x_tma = encode_rows_map(&xmap, x, T, d_in) ? 1 : 0;
+    const int y_tma = encode_rows_map(&ymap, y, T, y_ld) ? 1 : 0;
     if (ns == 1) {
         constexpr size_t sm = shrink_tc_smem<kMaxRank>();
         LF_CUDA_TRY(cudaFuncSetAttribute(shrink_tc_kernel<kMaxRank>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm));
@@ -548,7 +553,8 @@ static lf_status apply_impl(int32_t T, int32_t d_in, const void* x, void* y, int
     }
     LF_CUDA_TRY(cudaGetLastError());
     LF_CUDA_TRY(cudaFuncSetAttribute(expand_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kExpandTcSmem));
-    LF_LAUNCH("expand_tc", expand_tc_kernel, dim3(max_tc, (unsigned)A.n_chunks), kTcExpThreads, kExpandTcSmem, s, A);
+    LF_LAUNCH("expand_tc", expand_tc_kernel, dim3(max_tc, (unsigned)A.n_chunks), kTcExpThreads, kExpandTcSmem, s, A,
+              ymap, y_tma);
     return launch_status();
 }
 

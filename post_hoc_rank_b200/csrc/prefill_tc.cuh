@@ -260,32 +260,49 @@ constexpr size_t shrink_tc_smem() { return sizeof(ShrinkTcSmem<MAXN>) + 1024; }
 // ---- expand ---------------------------------------------------------------
 // CTA (token tile of one segment, kTcCols columns of d_out), 256 threads.  The
 // column range is walked in kTcN2-wide steps through a software pipeline:
-//   y tiles (gathered rows of y through the permutation) stream into a 3-buffer
-//   shared-memory ring by cp.async, B'^T tiles into 2 buffers, so the loads of
-//   steps i+1 and i+2 are in flight while step i runs;
+//   y tiles stream into a 3-buffer shared-memory ring, B'^T tiles into 2 buffers
+//   (cp.async), so the loads of steps i+1 and i+2 are in flight while step i runs.
+//   A y tile is gathered row by row through the permutation with cp.async or, when
+//   the tile's tokens are consecutive rows of y and the caller encoded a tensor map
+//   of y (box 64 x 128, 128-byte swizzle), loaded by thread 0 with two TMA copies;
+//   either way it is held as two 64-column halves in the 128-byte swizzle layout;
 //   one thread issues D = t_hi B + t_lo B (M = 128, N = kTcN2, fp32 in TMEM) and
 //   commits to an mbarrier;
 //   8 warps read D (warp w: lanes 32(w%4).., columns 64(w/4)..), add s*D to the
 //   staged y in shared memory with one bf16 rounding, then the tile is written
-//   back with coalesced 16-byte stores.
+//   back: by two TMA stores when it is a full TMA tile (128 tokens, 128 columns
+//   inside the CTA's range), else with 16-byte stores of its rows < ntok and columns
+//   in range (rows past the tile belong to other CTAs and are never written).
 constexpr int kTcN2 = 128;                  // expand step width (UMMA N)
 constexpr int kTcYBuf = 3;
-constexpr int kTcYLd = kTcN2 + 8;           // bf16 per staged y row: 272 bytes, conflict-free 16-byte rows
 constexpr int kTcExpThreads = 256;
+constexpr uint32_t kTcYHalf = kTcM * 128;   // bytes of one 64-column half of a staged y tile
 struct ExpandTcSmem {
     __nv_bfloat16 ahi[kTcM * kMaxRank];          // t_hi, K-major, 16 KB
     __nv_bfloat16 alo[kTcM * kMaxRank];          // t_lo
     __nv_bfloat16 b[2][kMaxRank * kTcN2];        // B'^T tiles, MN-major, 16 KB each
     union {
-        __nv_bfloat16 yt[kTcYBuf][kTcM * kTcYLd];    // staged y tiles, 34 KB each
+        __nv_bfloat16 yt[kTcYBuf][kTcM * kTcN2];     // staged y tiles, 32 KB each (1024-byte aligned)
         float tw[kTcM][kMaxRank + 1];                // summed t rows (Sigma-sandwich only, prologue), 33 KB
     };
     uint64_t bar;
+    uint64_t ybar[kTcYBuf];   // TMA y tiles (tx bytes)
     uint32_t tmem;
     int32_t toks[kTcM];
 };
 
-__global__ void __launch_bounds__(kTcExpThreads, 1) expand_tc_kernel(ApplyArgs a) {
+// Byte offset of (row, col) in a staged y tile: 64-column halves of 128 rows x 128
+// bytes, the 16-byte chunk c of row r stored at chunk c ^ (r % 8) (the layout a TMA
+// copy with 128-byte swizzle writes; 16-byte row accesses of 8 consecutive rows hit
+// distinct banks).
+__device__ __forceinline__ uint32_t ytile_off(int row, int col) {
+    return (uint32_t)(col >> 6) * kTcYHalf + (uint32_t)row * 128 +
+           ((uint32_t)(((col >> 3) & 7) ^ (row & 7)) << 4) + (uint32_t)(col & 7) * 2;
+}
+
+// y_tma: the caller encoded `ymap` (y as y_ld x T bf16, box 64 x 128, 128-byte swizzle).
+__global__ void __launch_bounds__(kTcExpThreads, 1) expand_tc_kernel(ApplyArgs a, const __grid_constant__ CUtensorMap ymap,
+                                                                     int y_tma) {
     extern __shared__ __align__(1024) unsigned char tc_raw[];
     auto& s = *reinterpret_cast<ExpandTcSmem*>(tc_raw);
     if ((int)blockIdx.x >= a.counts[3]) return;
@@ -357,19 +374,37 @@ __global__ void __launch_bounds__(kTcExpThreads, 1) expand_tc_kernel(ApplyArgs a
     if (warp == 0) tc::tmem_alloc(&s.tmem, kTcN2);
     if (tid == 0) {
         mbar_init(&s.bar, 1);
+        for (int b2 = 0; b2 < kTcYBuf; ++b2) mbar_init(&s.ybar[b2], 1);
         fence_barrier_init();
     }
     __syncthreads();   // toks visible to the copies below
+    bool consecutive = true;
+    for (int m = tid; m < nt; m += kTcExpThreads) consecutive = consecutive && s.toks[m] == s.toks[0] + m;
+    // uniform: y tiles by TMA
+    const bool ytma = __syncthreads_and(consecutive) && y_tma != 0 && (smem_u32(s.yt[0]) & 1023u) == 0;
+    int y_issued = 0;   // TMA y tiles issued by thread 0
 
     const __nv_bfloat16* Bt = S.Bt_pool + ob;
-    auto issue_y = [&](int i) {   // y rows of step i -> yt[i % 3]; rows past the tile / columns past the range zero-filled
+    auto issue_y = [&](int i) {   // y rows of step i -> yt[i % 3]
         const int e0 = e_begin + i * kTcN2;
-        __nv_bfloat16* dst = s.yt[i % kTcYBuf];
+        char* dst = reinterpret_cast<char*>(s.yt[i % kTcYBuf]);
+        if (ytma) {   // rows toks[0] .. +127, columns y_off + e0 .. +127 (a multiple of 8 elements)
+            if (tid == 0) {
+                tc::bulk_wait_read0();   // the TMA store of the tile this buffer held has read it
+                uint64_t* bar = &s.ybar[i % kTcYBuf];
+                mbar_arrive_expect_tx(bar, 2 * kTcYHalf);
+                tc::tma_load_2d(dst, &ymap, (int)S.y_off + e0, s.toks[0], bar);
+                tc::tma_load_2d(dst + kTcYHalf, &ymap, (int)S.y_off + e0 + 64, s.toks[0], bar);
+                ++y_issued;
+            }
+            return;
+        }
+        // rows past the tile / columns past the range zero-filled
         for (int c = tid; c < kTcM * (kTcN2 / 8); c += kTcExpThreads) {
             const int row = c / (kTcN2 / 8), ch = c % (kTcN2 / 8);
             const int e = e0 + ch * 8;
             const bool ok = row < nt && e < e_end;
-            cp_async16_zfill(dst + row * kTcYLd + ch * 8, ok ? ybase + (int64_t)s.toks[row] * a.y_ld + e : ybase, ok);
+            cp_async16_zfill(dst + ytile_off(row, ch * 8), ok ? ybase + (int64_t)s.toks[row] * a.y_ld + e : ybase, ok);
         }
     };
     auto issue_b = [&](int i) {   // B'^T rows 0..kpad-1 of step i -> b[i % 2], MN-major
@@ -402,7 +437,9 @@ __global__ void __launch_bounds__(kTcExpThreads, 1) expand_tc_kernel(ApplyArgs a
     for (int i = 0; i < nit && ok; ++i) {
         tc::cp_async_wait<1>();              // step i's y and B tiles (this thread's copies)
         tc::fence_proxy_async();             // B tile -> visible to the tensor core
-        __syncthreads();
+        if (ytma) ok = mbar_wait(&s.ybar[i % kTcYBuf], (uint32_t)((i / kTcYBuf) & 1));
+        ok = __syncthreads_and(ok);
+        if (!ok) break;
         if (tid == 0) {
             tc::fence_after_sync();
             const char* bb = reinterpret_cast<const char*>(s.b[i & 1]);
@@ -426,10 +463,11 @@ __global__ void __launch_bounds__(kTcExpThreads, 1) expand_tc_kernel(ApplyArgs a
             for (int c16 = 0; c16 < kTcN2 / 32; ++c16) {
                 float v[16];
                 tc::tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)((kTcN2 / 2) * h + 16 * c16), v);
-                uint4* yp = reinterpret_cast<uint4*>(yt + m * kTcYLd + (kTcN2 / 2) * h + 16 * c16);
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
-                    uint4 yv = yp[half];
+                    uint4* yp = reinterpret_cast<uint4*>(reinterpret_cast<char*>(yt) +
+                                                         ytile_off(m, (kTcN2 / 2) * h + 16 * c16 + 8 * half));
+                    uint4 yv = *yp;
                     __nv_bfloat162* y2 = reinterpret_cast<__nv_bfloat162*>(&yv);
 #pragma unroll
                     for (int p = 0; p < 4; ++p) {
@@ -437,22 +475,38 @@ __global__ void __launch_bounds__(kTcExpThreads, 1) expand_tc_kernel(ApplyArgs a
                         y2[p] = __floats2bfloat162_rn(fmaf(scale, v[8 * half + 2 * p], yf.x),
                                                       fmaf(scale, v[8 * half + 2 * p + 1], yf.y));
                     }
-                    yp[half] = yv;
+                    *yp = yv;
                 }
             }
         }
+        tc::fence_proxy_async();             // staged tile -> visible to a TMA store / next TMA load
         tc::fence_before_sync();
         ok = __syncthreads_and(ok);          // staged tile complete; TMEM free for the next MMA
         if (ok) {
             const int e0 = e_begin + i * kTcN2;
-            for (int c = tid; c < kTcM * (kTcN2 / 8); c += kTcExpThreads) {
-                const int row = c / (kTcN2 / 8), ch = c % (kTcN2 / 8);
-                const int e = e0 + ch * 8;
-                if (row < nt && e < e_end)
-                    *reinterpret_cast<uint4*>(ybase + (int64_t)s.toks[row] * a.y_ld + e) =
-                        *reinterpret_cast<const uint4*>(yt + row * kTcYLd + ch * 8);
+            if (ytma && nt == kTcM && e0 + kTcN2 <= e_end) {   // the whole box is this CTA's
+                if (tid == 0) {
+                    const char* src = reinterpret_cast<const char*>(yt);
+                    tc::tma_store_2d(&ymap, (int)S.y_off + e0, s.toks[0], src);
+                    tc::tma_store_2d(&ymap, (int)S.y_off + e0 + 64, s.toks[0], src + kTcYHalf);
+                    tc::bulk_commit();
+                }
+            } else {
+                for (int c = tid; c < kTcM * (kTcN2 / 8); c += kTcExpThreads) {
+                    const int row = c / (kTcN2 / 8), ch = c % (kTcN2 / 8);
+                    const int e = e0 + ch * 8;
+                    if (row < nt && e < e_end)
+                        *reinterpret_cast<uint4*>(ybase + (int64_t)s.toks[row] * a.y_ld + e) =
+                            *reinterpret_cast<const uint4*>(reinterpret_cast<const char*>(yt) + ytile_off(row, ch * 8));
+                }
+                tc::fence_proxy_async();     // reads of the buffer before a later TMA copy refills it
             }
         }
+    }
+    if (tid == 0 && ytma) {   // nothing of this CTA's TMA traffic is in flight when it leaves
+        tc::bulk_wait0();
+        for (int j = max(0, y_issued - kTcYBuf); j < y_issued; ++j)
+            mbar_wait(&s.ybar[j % kTcYBuf], (uint32_t)((j / kTcYBuf) & 1));
     }
     tc::cp_async_wait<0>();
     tc::fence_before_sync();

@@ -52,6 +52,22 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const void* tmap, int c0,
         : "memory");
 }
 
+// 2-D tiled TMA store of a shared-memory box to the tensor map's coordinates (c0 =
+// innermost, c1); rows or columns outside the tensor are not written.  Tracked in
+// this thread's bulk async-group (commit with bulk_commit).  Shared-memory writes the
+// store reads must be fenced to the async proxy (fence_proxy_async) by their writers
+// before a barrier that precedes the store.
+__device__ __forceinline__ void tma_store_2d(const void* tmap, int c0, int c1, const void* src) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group [%0, {%1, %2}], [%3];"
+                 ::"l"(reinterpret_cast<uint64_t>(tmap)), "r"(c0), "r"(c1), "r"(smem_u32(src))
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// wait until this thread's committed bulk stores have finished reading shared memory
+__device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// wait until this thread's committed bulk stores have completed
+__device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 // Instruction descriptor, kind::f16 with bf16 inputs and fp32 accumulation.
 // a_mn / b_mn: 1 = MN-major operand, 0 = K-major.
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int a_mn, int b_mn) {
