@@ -282,7 +282,8 @@ struct ExpandTcSmem {
     __nv_bfloat16 alo[kTcM * kMaxRank];          // t_lo
     __nv_bfloat16 b[2][kMaxRank * kTcN2];        // B'^T tiles, MN-major, 16 KB each
     union {
-        __nv_bfloat16 yt[kTcYBuf][kTcM * kTcN2];     // staged y tiles, 32 KB each (1024-byte aligned)
+        __nv_bfloat16 yt[kTcYBuf][kTcM * kTcN2];     // staged y tiles, 32 KB each (64 KB into the block:
+                                                     // 1024-byte aligned when the block is; checked before TMA)
         float tw[kTcM][kMaxRank + 1];                // summed t rows (Sigma-sandwich only, prologue), 33 KB
     };
     uint64_t bar;
