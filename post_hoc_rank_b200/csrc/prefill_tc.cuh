@@ -32,13 +32,15 @@ constexpr int kTcThreads = 128;  // shrink: 4 warps, warp w owns tensor-memory l
 constexpr int kTcCols = 2048;    // d_out columns per expand CTA
 constexpr int kTcMaxSplit = 8;   // d_in is split over at most this many CTAs per token tile
 
-// d_in elements per split: a multiple of the stage width, at least 2048, at most kTcMaxSplit splits
-// (swept 512 / 1024 / 2048 / 3072 / 4096 on the prefill layers: 2048 fills one wave of
-// CTAs for the hidden-width projections and keeps the expand's sum over partials short)
+// d_in elements per split: d_in is cut into min(kTcMaxSplit, ceil(d_in / kTcSplitTarget))
+// splits of equal length rounded up to the stage width (3584 -> 2 x 1792, 18944 -> 8 x
+// 2368), so the CTAs of one token tile carry the same work.
+constexpr int kTcSplitTarget = 2048;
 __host__ __device__ inline int tc_split_len(int d_in) {
-    int len = (d_in + kTcMaxSplit - 1) / kTcMaxSplit;
-    len = ((len + kTcKB - 1) / kTcKB) * kTcKB;
-    return len < 2048 ? 2048 : len;
+    int n = (d_in + kTcSplitTarget - 1) / kTcSplitTarget;
+    n = n < 1 ? 1 : (n > kTcMaxSplit ? kTcMaxSplit : n);
+    const int len = (d_in + n - 1) / n;
+    return ((len + kTcKB - 1) / kTcKB) * kTcKB;
 }
 
 // ---- shrink ---------------------------------------------------------------
