@@ -180,7 +180,9 @@ lf_status lf_truncate_export(const lf_module* mods /*[host]*/, int32_t n, lf_pol
  * on the adapter id into segments (adapter, start, length) over a permutation of
  * token indices; segments with many tokens run on tcgen05 tensor cores, the rest
  * on a segmented GEMV; both read every adapter's k rows once per segment and never
- * pad k.  If seg_out is not NULL it receives the routing, as int32: [n_seg,
+ * pad k.  On the tensor-core path a 128-token tile whose tokens are consecutive rows
+ * of x and y (a prefill request) moves x and y by TMA tiles; a tile of scattered
+ * tokens gathers its rows one by one (same results, bit for bit).  If seg_out is not NULL it receives the routing, as int32: [n_seg,
  * n_valid, then 3*n_seg (adapter,start,len), then n_valid token indices]; it must
  * hold 2 + 3*min(T,n_adapters) + T ints.
  * Workspace: lf_apply_workspace_size(T, n_adapters).  The same as a one-slice
