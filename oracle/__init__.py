@@ -18,6 +18,8 @@ written for a reader to check against the pages by eye:
                   y += s * B' (A' x) by brute force.
 * ``jd``       -- joint diagonalization (JD-Full) of a LoRA collection by
                   eigenvalue iteration with a QR orthogonalize.
+* ``pool``     -- the pool-wide shared subspace of stacked LoRA factors that keeps
+                  a fraction (99 %) of their energy (LoRASpace).
 
 Every function names the passage it follows by page title and section.
 Readings of passages the pages leave open are stated beside the code.
@@ -25,4 +27,4 @@ Pins: every function here is pinned by ``tests/test_oracle_*.py`` against
 closed forms, library special cases, brute force or hand-worked fixtures
 (``tests/golden``); none is "parity unpinned".
 """
-from . import factor, allocate, apply, jd  # noqa: F401
+from . import factor, allocate, apply, jd, pool  # noqa: F401
