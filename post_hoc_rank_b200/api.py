@@ -95,6 +95,40 @@ def select_ranks(mods, pol, sigma, stream=None):
     return ranks, offA, offB
 
 
+def pool_module(A_offs, ranks, d_in: int) -> np.ndarray:
+    """lf_module of a pool's stacked row factors (LoRASpace's pool-wide subspace, the
+    arXiv listing abstract): the A_i (r_i x d_in) of one module position stored back to
+    back from element A_offs[0] of a pool form one contiguous (sum r_i) x d_in matrix,
+    entered as the A factor of one module whose B factor is the identity of order
+    sum r_i, so the module's singular values are those of the stack.  Host checks only:
+    sum r_i <= 64 (the kernels' rank limit) and <= d_in, and the factors contiguous."""
+    A_offs = [int(o) for o in A_offs]
+    ranks = [int(r) for r in ranks]
+    if not ranks or len(A_offs) != len(ranks) or min(ranks) < 1:
+        raise ValueError("one offset and a positive rank per LoRA")
+    R = sum(ranks)
+    if R > 64 or R > d_in:
+        raise ValueError("the stacked rank must be at most 64 and at most d_in")
+    for i in range(len(ranks) - 1):
+        if A_offs[i + 1] != A_offs[i] + ranks[i] * d_in:
+            raise ValueError("the pool's row factors must be stored back to back")
+    m = np.zeros(1, dtype=lf.MODULE_DTYPE)
+    m["d_out"], m["d_in"], m["r"], m["group"], m["B_off"], m["A_off"] = R, d_in, R, 0, 0, A_offs[0]
+    return m
+
+
+def pool_subspace_rows(A_base, A_offs, ranks, d_in: int, num: int = 99, den: int = 100, stream=None):
+    """Pool-wide subspace of stacked row factors on the GPU: lf_tsqr_batched on
+    pool_module (singular values of the stack), then lf_select_ranks with the
+    energy-fraction policy (floor 1).  Returns (k, sigma[sum r_i] fp64, Factors)."""
+    mods = pool_module(A_offs, ranks, d_in)
+    R = int(mods["r"][0])
+    eye = torch.eye(R, dtype=torch.float32, device=A_base.device)
+    F = tsqr(mods, eye.reshape(-1), A_base, stream=stream)
+    k, _, _ = select_ranks(mods, lf.policy_E(num, den, 1), F.sigma, stream=stream)
+    return int(k[0].item()), F.sigma[0, :R], F
+
+
 def shrink_expand(x, y, ids, ranks, off_A, off_Bt, A_pool, Bt_pool, scale, ws=None, seg_out=None,
                   stream=None):
     n_adapters = ranks.numel()

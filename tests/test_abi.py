@@ -198,3 +198,16 @@ def test_routed_apply_validation_on_host():
     assert call(x=8) == 8
     assert call(wsb=8) == 4
     assert call(ws=None) == 1
+
+
+def test_pool_module_host_checks():
+    """The stacked-row module of a pool (LoRASpace pool subspace): one module whose A is
+    the back-to-back stack and whose B is the identity of the summed rank; rejected on
+    the host when the factors are not contiguous or the summed rank exceeds 64 or d_in."""
+    from post_hoc_rank_b200 import api
+    m = api.pool_module([100, 100 + 16 * 256, 100 + 24 * 256], [16, 8, 12], 256)
+    assert m.shape == (1,)
+    assert (int(m["d_out"][0]), int(m["d_in"][0]), int(m["r"][0]), int(m["A_off"][0]), int(m["B_off"][0])) == (36, 256, 36, 100, 0)
+    for bad in [([0, 5], [4, 4], 256), ([0, 40 * 256], [40, 40], 256), ([0], [300], 1024), ([0], [8], 4), ([0, 8], [4], 2), ([], [], 8)]:
+        with pytest.raises(ValueError):
+            api.pool_module(*bad)
