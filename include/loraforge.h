@@ -175,14 +175,16 @@ lf_status lf_truncate_export(const lf_module* mods /*[host]*/, int32_t n, lf_pol
  * hold pool_elems_A / pool_elems_Bt elements; an adapter whose rows would reach
  * past a pool (or whose offset is not a multiple of 8, or k > 64) latches an error
  * on the device and its tokens are left untouched.
- * With few tokens per adapter (T <= 8 * n_adapters) every token is applied with
- * its own adapter index (no sort).  Otherwise tokens are routed by a stable sort
+ * A small batch with few tokens per adapter (T < 512 and T <= 8 * n_adapters) is
+ * applied token by token with each token's own adapter index (no sort).  Every
+ * other batch is routed, whatever the number of resident adapters, by a stable sort
  * on the adapter id into segments (adapter, start, length) over a permutation of
  * token indices; segments with many tokens run on tcgen05 tensor cores, the rest
  * on a segmented GEMV; both read every adapter's k rows once per segment and never
  * pad k.  On the tensor-core path a 128-token tile whose tokens are consecutive rows
  * of x and y (a prefill request) moves x and y by TMA tiles; a tile of scattered
- * tokens gathers its rows one by one (same results, bit for bit).  If seg_out is not NULL it receives the routing, as int32: [n_seg,
+ * tokens gathers its rows one by one (same results, bit for bit).  If seg_out is
+ * not NULL it receives the routing, as int32: [n_seg,
  * n_valid, then 3*n_seg (adapter,start,len), then n_valid token indices]; it must
  * hold 2 + 3*min(T,n_adapters) + T ints.
  * Workspace: lf_apply_workspace_size(T, n_adapters).  The same as a one-slice
@@ -243,7 +245,8 @@ lf_status lf_lora_shrink_expand_slices(int32_t T, int32_t d_in, const void* x, v
  * routing pass on it (lf_route_tokens or any unrouted apply call).  A routed call on
  * a workspace whose tables were written for another T or n_adapters (or never)
  * applies nothing and latches LF_ERR_INVALID_ARG.  In the decode regime
- * (T <= 8 n_adapters) the side path reads ids directly and the tables are not used.
+ * (T < 512 and T <= 8 n_adapters) the side path reads ids directly and the tables
+ * are not used.
  * Host errors as for lf_lora_shrink_expand_slices. */
 lf_status lf_route_tokens(int32_t T, const int32_t* ids, int32_t n_adapters, void* ws, size_t ws_bytes,
                           lf_stream_t stream);
@@ -327,12 +330,17 @@ lf_status lf_jd_full(const lf_module* mods /*[host]*/, int32_t n_mods,
  * (a file-scope __device__ array sized for LF_NOALLOC_MAX_TOKENS tokens and
  * LF_NOALLOC_MAX_ADAPTERS adapters, 4 407 808 bytes, held on every GPU that loads the
  * library until the process exits).
- *  - Same arguments, results and device-side errors as lf_lora_shrink_expand, minus
- *    the workspace.  T > LF_NOALLOC_MAX_TOKENS or n_adapters > LF_NOALLOC_MAX_ADAPTERS
- *    returns LF_ERR_WORKSPACE without launching anything.
+ *  - Same arguments and device-side errors as lf_lora_shrink_expand, minus the
+ *    workspace; the results agree with it within the apply tolerance (it always
+ *    runs the GEMV kernels, so the bf16 rounding of y may differ).
+ *    T > LF_NOALLOC_MAX_TOKENS or n_adapters > LF_NOALLOC_MAX_ADAPTERS returns
+ *    LF_ERR_WORKSPACE without launching anything.
  *  - Runs on the device that is current when it is called; `stream` must belong
  *    to that device.  The first call on each device looks up the array's device
- *    address (cudaGetSymbolAddress); make that first call before any stream capture.
+ *    address (cudaGetSymbolAddress) and keeps it until the process exits; make that
+ *    first call before any stream capture.  Resetting a device (cudaDeviceReset)
+ *    while the library is loaded is not supported: the array may come back at
+ *    another address.
  *  - Allocates nothing: no cudaMalloc, cudaFree or allocating library routine.
  *  - All calls on one device share the one array and every call overwrites what it
  *    reads before reading it (nothing in it has to start at zero).  Two calls whose
@@ -364,6 +372,15 @@ void lf_profile_enable(int on);
 void lf_profile_reset(void);
 int32_t lf_profile_read(lf_phase_time* out /*[host]*/, int32_t max_phases);
 int64_t lf_launch_count(void);
+
+/* ---- Failure detection check (no counterpart on the pages) --------------------
+ * Launches one thread that waits, through the same bounded mbarrier wait every
+ * pipeline of the library uses, on a barrier nothing arrives at, giving up after
+ * `polls` polls (0 .. 2^20).  The wait runs out, LF_ERR_TIMEOUT is latched and the
+ * kernel returns, so the context stays usable: lf_get_device_status then reports
+ * LF_ERR_TIMEOUT.  Nothing else is in flight in that kernel (no copy, no MMA).
+ * Returns LF_ERR_INVALID_ARG for polls outside the range. */
+lf_status lf_check_bounded_wait(int32_t polls, lf_stream_t stream);
 
 /* ---- Status ------------------------------------------------------------------ */
 const char* lf_status_string(lf_status s);

@@ -70,18 +70,23 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
-// Bounded wait on an mbarrier phase: gives up after 2^25 polls or ~2e9 SM cycles
-// (about a second), latches LF_ERR_TIMEOUT and returns false.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+// Bounded wait on an mbarrier phase: gives up after `max_polls` polls or ~2e9 SM
+// cycles (about a second), whichever comes first, latches LF_ERR_TIMEOUT and returns
+// false.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, int max_polls) {
     if (mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
-    for (int i = 0; i < (1 << 25); ++i) {
+    for (int i = 0; i < max_polls; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
         __nanosleep(32);
         if ((i & 1023) == 1023 && clock64() - t0 > 2000000000ll) break;
     }
     latch_error(LF_ERR_TIMEOUT);
     return false;
+}
+// The library's waits: at most 2^25 polls or about a second.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+    return mbar_wait_bounded(bar, parity, 1 << 25);
 }
 
 // Carves caller workspace into aligned sub-buffers; tracks the bytes needed.

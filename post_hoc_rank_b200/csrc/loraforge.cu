@@ -432,6 +432,16 @@ struct SharedSlice {
     int32_t mode = 0;
 };
 
+// Decode regime (token-parallel kernel, no routing pass) for small batches with few
+// tokens per adapter on average: T < kDecodeMaxTokens and T <= kGemvTok * n_adapters.
+// Every larger batch is routed, so its long segments (a prefill request of hundreds of
+// tokens) reach the GEMV items or the tensor-core tiles however many adapters are
+// resident.  The rule reads only T and the adapter count, so it costs no device pass.
+constexpr int64_t kDecodeMaxTokens = 512;
+static bool decode_regime(int64_t T, int64_t n_adapters) {
+    return T < kDecodeMaxTokens && T <= (int64_t)kGemvTok * n_adapters;
+}
+
 static lf_status apply_impl(int32_t T, int32_t d_in, const void* x, void* y, int64_t y_ld, const int32_t* ids,
                             int32_t n_adapters, const lf_slice* sl, int32_t ns, float scale, const float* scales,
                             int32_t* seg_out, void* ws, size_t ws_bytes, cudaStream_t s,
@@ -503,11 +513,11 @@ static lf_status apply_impl(int32_t T, int32_t d_in, const void* x, void* y, int
     o.run_pos = w.runs + T;
     o.seg_out = seg_out;
     o.tag = w.tag;
-    const bool decode_regime = (int64_t)T <= (int64_t)kGemvTok * n_adapters;
-    o.tc_enable = decode_regime ? 0 : 1;
+    const bool token_parallel = decode_regime(T, n_adapters);
+    o.tc_enable = token_parallel ? 0 : 1;
     const size_t rsmem = 2 * (size_t)n_adapters * sizeof(int32_t);
     LF_CUDA_TRY(cudaFuncSetAttribute(route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rsmem));
-    if (decode_regime) {
+    if (token_parallel) {
         // few tokens per adapter: token-parallel shrink + expand, no sort; the routing
         // pass runs only when the caller asks for the segment table
         if (seg_out) {
@@ -588,6 +598,18 @@ static lf_status noalloc_scratch(void** out) {
     }
     *out = g_noalloc_addr[dev];
     return LF_OK;
+}
+
+// ------------------------------------------------------- bounded-wait check
+// One thread waits on an mbarrier that nothing arrives at (no copy or MMA is in
+// flight), so the wait runs out after `polls` polls and latches LF_ERR_TIMEOUT: the
+// same exit every pipeline wait of the library takes when a producer never arrives.
+__global__ void wait_selftest_kernel(int polls) {
+    __shared__ __align__(8) uint64_t bar;
+    if (threadIdx.x != 0) return;
+    mbar_init(&bar, 1);
+    fence_barrier_init();
+    mbar_wait_bounded(&bar, 0, polls);
 }
 
 // ------------------------------------------------------------ JD-Full plan
@@ -1196,7 +1218,7 @@ lf_status lf_route_tokens(int32_t T, const int32_t* ids, int32_t n_adapters, voi
     o.run_pos = w.runs + T;
     o.seg_out = nullptr;
     o.tag = w.tag;
-    o.tc_enable = (int64_t)T <= (int64_t)kGemvTok * n_adapters ? 0 : 1;
+    o.tc_enable = decode_regime(T, n_adapters) ? 0 : 1;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const size_t rsmem = 2 * (size_t)n_adapters * sizeof(int32_t);
     LF_CUDA_TRY(cudaFuncSetAttribute(route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rsmem));
@@ -1550,6 +1572,12 @@ const char* lf_status_string(lf_status s) {
         case LF_ERR_ALIGNMENT: return "misaligned pointer, offset or leading dimension";
     }
     return "unknown status";
+}
+
+lf_status lf_check_bounded_wait(int32_t polls, lf_stream_t stream) {
+    if (polls < 0 || polls > (1 << 20)) return LF_ERR_INVALID_ARG;
+    LF_LAUNCH("wait_selftest", wait_selftest_kernel, 1, 32, 0, reinterpret_cast<cudaStream_t>(stream), polls);
+    return launch_status();
 }
 
 lf_status lf_get_device_status(lf_stream_t stream) {

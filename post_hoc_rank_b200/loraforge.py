@@ -121,6 +121,7 @@ def lib() -> ctypes.CDLL:
         L.lf_lora_shrink_expand_noalloc.argtypes = [_I32, _I32, _I32, _P, _P, _P, _I32, _P, _P, _P, _P, _P,
                                                     _I64, _I64, ctypes.c_float, _P, _P]
         L.lf_lora_shrink_expand_noalloc.restype = ctypes.c_int
+        L.lf_check_bounded_wait.argtypes = [_I32, _P]; L.lf_check_bounded_wait.restype = ctypes.c_int
         L.lf_status_string.argtypes = [ctypes.c_int]; L.lf_status_string.restype = ctypes.c_char_p
         L.lf_get_device_status.argtypes = [_P]; L.lf_get_device_status.restype = ctypes.c_int
         L.lf_profile_enable.argtypes = [ctypes.c_int]; L.lf_profile_enable.restype = None
@@ -138,7 +139,7 @@ def exported_symbols() -> list[str]:
             "lf_profile_enable", "lf_profile_reset", "lf_profile_read", "lf_launch_count",
             "lf_lora_shrink_expand_noalloc", "lf_apply_slices_workspace_size", "lf_lora_shrink_expand_slices",
             "lf_lora_sigma_sandwich", "lf_jd_workspace_size", "lf_jd_full", "lf_route_tokens",
-            "lf_lora_shrink_expand_slices_routed"]
+            "lf_lora_shrink_expand_slices_routed", "lf_check_bounded_wait"]
 
 # Limits of lf_lora_shrink_expand_noalloc (its scratch is a fixed array in the library).
 NOALLOC_MAX_TOKENS = 16384

@@ -211,3 +211,9 @@ def test_pool_module_host_checks():
     for bad in [([0, 5], [4, 4], 256), ([0, 40 * 256], [40, 40], 256), ([0], [300], 1024), ([0], [8], 4), ([0, 8], [4], 2), ([], [], 8)]:
         with pytest.raises(ValueError):
             api.pool_module(*bad)
+
+
+def test_bounded_wait_check_rejects_bad_poll_counts():
+    L = lf.lib()
+    assert L.lf_check_bounded_wait(-1, None) == 1          # LF_ERR_INVALID_ARG, nothing launched
+    assert L.lf_check_bounded_wait((1 << 20) + 1, None) == 1

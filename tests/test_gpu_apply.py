@@ -415,3 +415,33 @@ def test_routed_call_in_decode_regime(d_in, widths):
     assert lf.lf_get_device_status() == 0
     assert torch.equal(y, y_ref)
     check_slices(y.cpu(), y0, oracle_slices(x, y0, ids, sl, 1.0, asc.cpu().numpy()), sl, ids)
+
+
+def test_mixed_batch_with_many_resident_adapters_reaches_tensor_cores():
+    """A batch is routed per segment whatever the number of resident adapters: with
+    1024 adapters, two 512-token prefill requests go to the tensor-core tiles, a
+    48-token request and the decode tokens to the GEMV items, in one call; the result
+    matches the oracle and the routing equals the stable argsort."""
+    n, d_in, d_out = 1024, 1024, 2048
+    g = np.random.default_rng(18)
+    ranks = g.integers(1, 17, size=n)
+    dec = synth.zipf_ids(1024, n, 1.2, (18, 0))
+    ids = np.concatenate([np.full(512, 5, np.int32), dec[:600], np.full(48, 33, np.int32),
+                          np.full(512, 700, np.int32), dec[600:]]).astype(np.int32)
+    ids[g.random(len(ids)) < 0.02] = -1
+    T = len(ids)
+    assert T <= 8 * n                      # the old per-call rule sent all of this token by token
+    offA, offB, Ap, Bt = make_pools(ranks, d_in, d_out, (18, 1))
+    x = synth.normal_bf16((T, d_in), (18, 2))
+    y0 = torch.zeros(T, d_out, dtype=torch.bfloat16)
+    lf.lf_profile_reset(); lf.lf_profile_enable(True)
+    y, seg, st = run_apply(x, y0, ids, ranks, offA, offB, Ap, Bt, 2.0, seg=True)
+    lf.lf_profile_enable(False)
+    ph = lf.lf_profile_read()
+    assert st == 0
+    for name in ("route", "shrink_tc", "expand_tc", "shrink_gemv", "expand_gemv"):
+        assert name in ph and ph[name][1] > 0, (name, ph)
+    assert "bgmv" not in ph
+    check_routing(seg, ids, n)
+    assert_close(y, oracle_y(x, y0, ids, ranks, offA, offB, Ap, Bt, 2.0))
+    assert torch.equal(y[torch.from_numpy(ids < 0)], y0[torch.from_numpy(ids < 0)])

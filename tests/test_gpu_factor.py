@@ -106,7 +106,7 @@ def test_spectral_policy_ranks_bit_exact_and_errors():
     sig = G.oracle_sigma_rows(lay, Bh, Ah, range(lay.n))
     ranks_o, info = OA.spectral_ranks(sig, lay.r, lay.group, 1, 12, 1)
     ranks_g = E.ranks.cpu().numpy()
-    assert G.compare_ranks(ranks_g, ranks_o, info), (ranks_g, ranks_o)
+    assert G.compare_ranks(ranks_g, ranks_o, info, sig, lay.r, lay.group, 1), (ranks_g, ranks_o)
     for g in range(2):
         assert ranks_g[lay.group == g].sum() <= (64 * 28) // 12
     offA = E.off_A.cpu().numpy()
@@ -123,7 +123,7 @@ def test_select_ranks_alone_matches_oracle():
         ranks, offA, offB = api.select_ranks(mods, pol, torch.from_numpy(sig).cuda())
         assert lf.lf_get_device_status() == 0
         ranks_o, info = OA.spectral_ranks(sig, lay.r, lay.group, num, den, fl)
-        assert G.compare_ranks(ranks.cpu().numpy(), ranks_o, info)
+        assert G.compare_ranks(ranks.cpu().numpy(), ranks_o, info, sig, lay.r, lay.group, fl)
         ro = ranks_o.astype(np.int64)
         assert offA.cpu().numpy().tolist() == [0] + np.cumsum(ro * lay.d_in).tolist()
         assert offB.cpu().numpy().tolist() == [0] + np.cumsum(ro * lay.d_out).tolist()
@@ -261,7 +261,7 @@ def test_allocation_variants_ranks_bit_exact(variant):
     sig = G.oracle_sigma_rows(lay, Bh, Ah, range(lay.n))
     ranks_o, info = OA.spectral_ranks(sig, lay.r, lay.group, 1, 12, 1, absolute=absolute)
     ranks_g = E.ranks.cpu().numpy()
-    assert G.compare_ranks(ranks_g, ranks_o, info), (ranks_g, ranks_o)
+    assert G.compare_ranks(ranks_g, ranks_o, info, sig, lay.r, lay.group, 1, absolute=absolute), (ranks_g, ranks_o)
     for g in set(lay.group.tolist()):
         assert ranks_g[lay.group == g].sum() <= (64 * int((lay.group == g).sum())) // 12
     for eg, eo in G.recon_errors(lay, Bh, Ah, E, sig, range(lay.n)):

@@ -5,8 +5,9 @@
   (the S budget's scope) must equal the oracle's; sampled modules of every shape are
   checked for R, sigma and reconstruction error.
 * Decode apply (Llama-3-8B shapes, T = 256, 128 adapters, Zipf(1) ids) and prefill
-  apply (Qwen2.5-7B shapes, 32 x 512 tokens, k = 16 and 64): sampled tokens of every
-  projection against the oracle on the same bf16 bytes.
+  apply (Qwen2.5-7B shapes, 32 x 512 tokens, k = 16 and 64): every token of some
+  projections at y0 = 0 (the whole LoRA delta against the oracle) and sampled tokens of
+  every projection at the timed y0 ~ N(0, 1), on the same bf16 bytes.
 * Large fleet: adapters of the 1024-adapter Llama-3-8B fleet compressed in chunks, then
   the mixed batch (64 prefill segments of 48 tokens + 1024 decode tokens, Zipf(1.2) ids)
   applied through the exported pools; whole-adapter ranks and sampled tokens checked.
@@ -49,7 +50,8 @@ def check_adapter_ranks(lay, B, A, E, adapter, num, den, floor):
         sig[q, :len(s)] = s
     ranks_o, info = OA.spectral_ranks(sig, lay.r[idx], np.zeros(len(idx), int), num, den, floor)
     ranks_g = E.ranks.cpu().numpy()[idx]
-    assert G.compare_ranks(ranks_g, ranks_o, info), (adapter, np.nonzero(ranks_g != ranks_o))
+    assert G.compare_ranks(ranks_g, ranks_o, info, sig, lay.r[idx], np.zeros(len(idx), int), floor), \
+        (adapter, np.nonzero(ranks_g != ranks_o))
     return idx, sig
 
 
@@ -91,18 +93,32 @@ def test_factor_fleet_full_size():
     torch.cuda.empty_cache()
 
 
-def sampled_apply_check(x, y0, y, ids, ranks, offA, offB, Ap, Bt, scale, tokens):
-    """Oracle on the sampled tokens only (same bf16 bytes)."""
+def bf16_half_ulp(v):
+    """Half a bf16 ulp at |v| (8 significant bits): the error of the one rounding of y."""
+    e = np.floor(np.log2(np.maximum(np.abs(v), 2.0 ** -126)))
+    return 2.0 ** (e - 8)
+
+
+def apply_check(x, y0, y, ids, ranks, offA, offB, Ap, Bt, scale, tokens=None):
+    """Oracle on the given tokens (all tokens when None), on the same bf16 bytes.
+
+    Element by element, |y - y_oracle| may exceed half a bf16 ulp of y_oracle (the one
+    rounding of y = y0 + s B't) by at most APPLY_TOL times the largest LoRA delta
+    max|y_oracle - y0| of the checked rows; rows with id -1 must equal y0 bit for bit."""
+    ids = np.asarray(ids)
+    if tokens is None:
+        tokens = np.arange(len(ids))
     xs = x[tokens].float().cpu().numpy()
     ys0 = y0[tokens].float().cpu().numpy()
-    ref = OP.lora_apply(xs, ys0, np.asarray(ids)[tokens], ranks, offA, offB, Ap.float().cpu().numpy(),
+    ref = OP.lora_apply(xs, ys0, ids[tokens], ranks, offA, offB, Ap.float().cpu().numpy(),
                         Bt.float().cpu().numpy(), scale)
-    got = y[tokens].float().cpu().numpy()
-    delta_ref = ref - ys0
-    err = np.abs(got - ref).max()
-    # the LoRA delta is what the kernel computes; y0 only adds its own rounding
-    bound = G.APPLY_TOL * max(np.abs(delta_ref).max(), 1e-30) + np.abs(ref).max() * 2.0 ** -8
-    assert err <= bound, (err, bound)
+    got = y[tokens].float().cpu().numpy().astype(np.float64)
+    err = np.maximum(np.abs(got - ref) - bf16_half_ulp(ref), 0.0).max()
+    delta = np.abs(ref - ys0).max()
+    assert delta > 0.0
+    assert err <= G.APPLY_TOL * delta, (err, delta)
+    unrouted = torch.from_numpy(ids < 0)
+    assert torch.equal(y[unrouted.to(y.device)], y0[unrouted.to(y.device)])
 
 
 def make_pools_dev(ranks, d_in, d_out, key, dev):
@@ -137,11 +153,17 @@ def test_decode_full_size_layer():
         rk = ranks_all[:, p, 0]
         offA, offB, Ap, Bt = make_pools_dev(rk, d_in, d_out, (30, p), dev)
         x = synth.normal_bf16((T, d_in), (31, p), device=dev)
+        # every token at y0 = 0 (the check then measures the LoRA delta alone)
+        y0 = torch.zeros((T, d_out), dtype=torch.bfloat16, device=dev)
+        y = y0.clone()
+        run_projection(x, y, ids_d, rk, offA, offB, Ap, Bt, 2.0, dev)
+        apply_check(x, y0, y, ids, rk, offA[:-1], offB[:-1], Ap, Bt, 2.0)
+        # the timed configuration's y0 ~ N(0, 1), sampled tokens
         y0 = synth.normal_bf16((T, d_out), (32, p), device=dev)
         y = y0.clone()
         run_projection(x, y, ids_d, rk, offA, offB, Ap, Bt, 2.0, dev)
         toks = np.sort(g.choice(T, size=48, replace=False))
-        sampled_apply_check(x, y0, y, ids, rk, offA[:-1], offB[:-1], Ap, Bt, 2.0, toks)
+        apply_check(x, y0, y, ids, rk, offA[:-1], offB[:-1], Ap, Bt, 2.0, toks)
 
 
 @pytest.mark.parametrize("k", [16, 64])
@@ -156,11 +178,17 @@ def test_prefill_full_size_layer(k):
         rk = [k] * n_ad
         offA, offB, Ap, Bt = make_pools_dev(rk, d_in, d_out, (40, p, k), dev)
         x = synth.normal_bf16((T, d_in), (41, p), device=dev)
+        if p in (0, 6):
+            # q (3584 -> 3584) and down (18944 -> 3584): every token at y0 = 0
+            y0 = torch.zeros((T, d_out), dtype=torch.bfloat16, device=dev)
+            y = y0.clone()
+            run_projection(x, y, ids_d, rk, offA, offB, Ap, Bt, 2.0, dev)
+            apply_check(x, y0, y, ids, rk, offA[:-1], offB[:-1], Ap, Bt, 2.0)
         y0 = synth.normal_bf16((T, d_out), (42, p), device=dev)
         y = y0.clone()
         run_projection(x, y, ids_d, rk, offA, offB, Ap, Bt, 2.0, dev)
         toks = np.sort(g.choice(T, size=24, replace=False))
-        sampled_apply_check(x, y0, y, ids, rk, offA[:-1], offB[:-1], Ap, Bt, 2.0, toks)
+        apply_check(x, y0, y, ids, rk, offA[:-1], offB[:-1], Ap, Bt, 2.0, toks)
 
 
 def test_large_fleet_chunked_end_to_end():
@@ -210,8 +238,15 @@ def test_large_fleet_chunked_end_to_end():
                 baseA += k * d_in; baseB += k * d_out
         Ap = torch.cat(pools_A); Bt = torch.cat(pools_B)
         x = synth.normal_bf16((T, d_in), (51, p), device=dev)
+        offs = (np.array(offA + [baseA]), np.array(offB + [baseB]))
+        if p == 0:
+            # every token of the q projection at y0 = 0
+            y0 = torch.zeros((T, d_out), dtype=torch.bfloat16, device=dev)
+            y = y0.clone()
+            run_projection(x, y, ids_d, rk, offs[0], offs[1], Ap, Bt, 2.0, dev)
+            apply_check(x, y0, y, ids, rk, np.array(offA), np.array(offB), Ap, Bt, 2.0)
         y0 = synth.normal_bf16((T, d_out), (52, p), device=dev)
         y = y0.clone()
-        run_projection(x, y, ids_d, rk, np.array(offA + [baseA]), np.array(offB + [baseB]), Ap, Bt, 2.0, dev)
+        run_projection(x, y, ids_d, rk, offs[0], offs[1], Ap, Bt, 2.0, dev)
         toks = np.sort(np.concatenate([g.choice(T_pre, 16, replace=False), T_pre + g.choice(T_dec, 16, replace=False)]))
-        sampled_apply_check(x, y0, y, ids, rk, np.array(offA), np.array(offB), Ap, Bt, 2.0, toks)
+        apply_check(x, y0, y, ids, rk, np.array(offA), np.array(offB), Ap, Bt, 2.0, toks)

@@ -4,9 +4,11 @@ memory at start-up, or a latency-critical path that cannot afford cudaMalloc's
 implicit synchronisation).  It takes no workspace; the library keeps the routing
 scratch in a fixed device array.
 
-Checked here through the C ABI against the workspace entry point, on two calls in
-a row (the second with a different batch, so stale scratch contents from the first
-call would show), with the tolerance the apply parity tests use.  The file name
+Checked here through the C ABI against the workspace entry point, on calls in a row
+that alternate between batch shapes (a few tokens per adapter, which takes the fused
+single-launch GEMV kernel, and many tokens per adapter, which takes the separate
+shrink and expand kernels), so stale scratch contents from an earlier call would show,
+with the tolerance the apply parity tests use.  The file name
 sorts last so a run that stops at the first failure has run every other test."""
 import ctypes
 
@@ -68,9 +70,13 @@ def without_workspace(b, scale):
 
 
 def test_noalloc_matches_workspace_entry_point_on_two_calls():
-    first = batch(300, 37, 4096, 1024, seed=1)
-    second = batch(77, 5, 1024, 2048, seed=2)
-    for b, scale in ((first, 0.5), (second, 2.0)):
+    many = batch(300, 37, 4096, 1024, seed=1)     # > 8 tokens per adapter: shrink + expand kernels
+    few = batch(64, 37, 4096, 1024, seed=3)       # <= 8 tokens per adapter: fused GEMV kernel
+    many2 = batch(77, 5, 1024, 2048, seed=2)
+    few2 = batch(32, 16, 1024, 2048, seed=4)
+    assert few["x"].shape[0] <= 8 * few["n"] and few2["x"].shape[0] <= 8 * few2["n"]
+    assert many["x"].shape[0] > 8 * many["n"] and many2["x"].shape[0] > 8 * many2["n"]
+    for b, scale in ((many, 0.5), (few, 1.5), (many2, 2.0), (few2, 0.75)):
         ref = with_workspace(b, scale)
         got = without_workspace(b, scale)
         delta_ref = (ref.float() - b["y0"].float()).abs().max().item()
