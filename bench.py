@@ -641,17 +641,11 @@ def large_fleet_bench(args, dev, stream, hbm):
     shapes = M.proj_shapes()
     out = {"workload": f"large fleet: {n_total} adapters x Llama-3-8B (224 modules each, r=64), LoRAForge-S "
                        "1/12 floor 1, compressed in chunks of 64 adapters; then 4096 tokens (64 prefill segments "
-                       "x 48 + 1024 decode tokens, Zipf(1.2) ids) through 32 layers x 7 projections, routed once "
-                       "per step",
+                       "x 48 + 1024 decode tokens, Zipf(1.2) ids) through 32 layers x 7 projections",
            "modules": int(n_mod), "compress_ms": round(compress_ms, 2),
            "modules_per_s": round(n_mod / (compress_ms * 1e-3), 1), "distinct_adapters": int(len(ref))}
     for variant in ("ragged", "padded"):
-        # the batch is routed once per step; every projection call reuses the tables
-        rws = api.workspace(lf.lf_apply_slices_workspace_size(T, n_total, 1), dev)
-
-        def route(st=None, rws=rws):
-            lf.lf_route_tokens(ids_d, n_total, rws, stream=st)
-        calls, total_bytes = [route], 0
+        calls, total_bytes = [], 0
         for l in range(M.layers):
             x_h = synth.normal_bf16((T, M.hidden), (5, 3, l), device=dev)
             x_f = synth.normal_bf16((T, M.ffn), (5, 4, l), device=dev)
@@ -681,10 +675,9 @@ def large_fleet_bench(args, dev, stream, hbm):
                     oa_d = np.zeros(n_total, dtype=np.int64); ob_d = np.zeros(n_total, dtype=np.int64)
                     oa_d[ref] = np.arange(len(ref)) * kmax * d_in; ob_d[ref] = np.arange(len(ref)) * kmax * d_out
                     k_used = np.full(len(ref), kmax)
-                calls.append(_routed_call(x, y, ids_d, n_total,
-                                          [(d_out, 0, torch.from_numpy(rk_d.astype(np.int32)).to(dev),
-                                            torch.from_numpy(oa_d).to(dev), torch.from_numpy(ob_d).to(dev), pa, pb)],
-                                          rws))
+                ws = api.workspace(lf.lf_apply_workspace_size(T, n_total), dev)
+                calls.append(_proj_call(x, y, ids_d, n_total, torch.from_numpy(rk_d.astype(np.int32)).to(dev),
+                                        torch.from_numpy(oa_d).to(dev), torch.from_numpy(ob_d).to(dev), pa, pb, ws))
                 total_bytes += apply_bytes(T, d_in, d_out, [int(k) for k in k_used])
         r = _apply_run(args, calls, ids_d, n_total, T, total_bytes, stream, hbm, {})
         out[variant] = {k: r[k] for k in ("tokens_per_s", "ms_per_step", "algo_bytes", "achieved_gbs", "hbm_frac",
@@ -895,35 +888,165 @@ def OA_spectral(sig, lay):
 
 
 # ----------------------------------------------------------- CPU baseline
-def cpu_oracle_adapter(cfg_id=2, adapter=0, model=None, n_layers=None):
-    """The fp64 oracle's fleet route on one Qwen-shaped adapter (196 modules, or the
-    first n_layers layers of it): spectrum (QR of B and A^T, SVD of R_B R_A^T),
-    LoRAForge-S allocation, export."""
+def host_info():
+    """The host the CPU baseline ran on: logical CPUs, the ones this process may use,
+    the CPU model and whether SMT (more than one thread per core) is on."""
+    info = {"os_cpu_count": os.cpu_count(), "usable_cpus": len(os.sched_getaffinity(0))}
+    try:
+        out = subprocess.run(["lscpu"], capture_output=True, text=True, timeout=10).stdout
+        for line in out.splitlines():
+            k, _, v = line.partition(":")
+            k, v = k.strip(), v.strip()
+            if k == "Model name":
+                info["model"] = v
+            elif k == "Thread(s) per core":
+                info["threads_per_core"] = int(v)
+            elif k == "Socket(s)":
+                info["sockets"] = int(v)
+            elif k == "Core(s) per socket":
+                info["cores_per_socket"] = int(v)
+    except Exception:
+        pass
+    info["smt"] = info.get("threads_per_core", 1) > 1
+    return info
+
+
+# Worker side of the oracle's process pool (spawned processes, one BLAS thread each).
+# A task names a module of the adapter held in a shared-memory block: its B (d_out x r)
+# and A (r x d_in) element offsets.
+_SHM = {}
+
+
+def _pool_init():
+    from threadpoolctl import threadpool_limits
+    threadpool_limits(1)
+
+
+def _module_arrays(task):
+    from multiprocessing import shared_memory
+    name, nb, na, b0, a0, d_out, d_in, r = task[:8]
+    if name not in _SHM:
+        _SHM.clear()
+        _SHM[name] = shared_memory.SharedMemory(name=name)
+    buf = _SHM[name].buf
+    Bf = np.frombuffer(buf, dtype=np.float32, count=nb)
+    Af = np.frombuffer(buf, dtype=np.float32, count=na, offset=4 * nb)
+    return Bf[b0:b0 + d_out * r].reshape(d_out, r), Af[a0:a0 + r * d_in].reshape(r, d_in)
+
+
+def _cpu_spectrum(task):
+    from oracle import factor as OF
+    B, A = _module_arrays(task)
+    return OF.spectrum_factor(B, A)[0]
+
+
+def _cpu_export(task):
+    from oracle import factor as OF
+    B, A = _module_arrays(task)
+    Bp, Ap = OF.export_factor(B, A, int(task[8]))
+    return float(Bp[0, 0])
+
+
+class OraclePool:
+    """The fp64 oracle's fleet route (QR of B and A^T, SVD of R_B R_A^T per module; the
+    LoRAForge-S allocation over the adapter; export per module) run by a pool of spawned
+    worker processes with one BLAS thread each, on adapters of the same fleet recipe
+    generated into shared memory."""
+
+    def __init__(self, workers: int, model=None, n_layers=None):
+        import multiprocessing as mp
+        from multiprocessing import shared_memory
+        import torch
+        from post_hoc_rank_b200 import synth
+        self.model = model or synth.QWEN25_7B
+        self.lay = synth.fleet_layout(1, self.model, r=64, n_layers=n_layers)
+        nb, na = int(self.lay.B_total), int(self.lay.A_total)
+        self.shm = shared_memory.SharedMemory(create=True, size=4 * (nb + na))
+        arr = np.ndarray(nb + na, dtype=np.float32, buffer=self.shm.buf)
+        self.Bh = torch.from_numpy(arr[:nb])
+        self.Ah = torch.from_numpy(arr[nb:])
+        self.nb, self.na = nb, na
+        self.workers = workers
+        self.pool = mp.get_context("spawn").Pool(workers, initializer=_pool_init)
+
+    def tasks(self, idx):
+        L = self.lay
+        return [(self.shm.name, self.nb, self.na, int(L.B_off[i]), int(L.A_off[i]), int(L.d_out[i]),
+                 int(L.d_in[i]), int(L.r[i])) for i in idx]
+
+    def fill(self, adapter, cfg_id=2):
+        from post_hoc_rank_b200 import synth
+        synth.fill_fleet(self.lay, self.Bh, self.Ah, cfg_id=cfg_id, adapter_base=adapter)
+
+    def run(self, idx=None):
+        """Spectrum, S allocation over the modules idx (the whole adapter by default) and
+        export; returns (modules, seconds)."""
+        from oracle import allocate as OA
+        L = self.lay
+        idx = list(range(L.n)) if idx is None else list(idx)
+        t = self.tasks(idx)
+        t0 = time.perf_counter()
+        sig = np.stack(self.pool.map(_cpu_spectrum, t, chunksize=1))
+        ranks, _ = OA.spectral_ranks(sig, L.r[idx], np.zeros(len(idx), int), 1, 12, 1)
+        self.pool.map(_cpu_export, [tt + (int(k),) for tt, k in zip(t, ranks)], chunksize=1)
+        return len(idx), time.perf_counter() - t0
+
+    def close(self):
+        self.pool.close()
+        self.pool.join()
+        del self.Bh, self.Ah
+        self.shm.close()
+        self.shm.unlink()
+
+
+def cpu_definition_route(n_repeat=1):
+    """The plain definition on the seven sample modules (layer 0 of adapter 0, one per
+    projection): dense Delta W = B A and its SVD (numpy, the host's BLAS threads)."""
     import torch
     from post_hoc_rank_b200 import synth
-    from oracle import allocate as OA
     from oracle import factor as OF
-
-    model = model or synth.QWEN25_7B
-    lay = synth.fleet_layout(1, model, r=64, n_layers=n_layers)
+    lay = synth.fleet_layout(1, synth.QWEN25_7B, r=64, n_layers=1)
     Bh = torch.empty(lay.B_total); Ah = torch.empty(lay.A_total)
-    synth.fill_fleet(lay, Bh, Ah, cfg_id=cfg_id, adapter_base=adapter)
+    synth.fill_fleet(lay, Bh, Ah, cfg_id=2)
     mats = [tuple(t.numpy() for t in synth.module_view(lay, Bh, Ah, i)) for i in range(lay.n)]
     t0 = time.perf_counter()
-    sig = np.stack([OF.spectrum_factor(Bm, Am)[0] for Bm, Am in mats])
-    ranks, _ = OA.spectral_ranks(sig, lay.r, lay.group, 1, 12, 1)
-    for i, (Bm, Am) in enumerate(mats):
-        OF.export_factor(Bm, Am, int(ranks[i]))
-    dt = time.perf_counter() - t0
-    return lay.n, dt
+    for _ in range(n_repeat):
+        for Bm, Am in mats:
+            OF.spectrum_dense(Bm, Am)
+    dt = (time.perf_counter() - t0) / n_repeat
+    return {"modules": lay.n, "seconds": round(dt, 2), "modules_per_s": round(lay.n / dt, 3),
+            "sample": "layer 0 of adapter 0: q, k, v, o, gate, up, down (dense Delta W = B A, numpy SVD)"}
 
 
 def cpu_baseline():
-    import torch
-    n, dt = cpu_oracle_adapter()
-    return {"value": n / dt, "unit": "modules/s", "cores": torch.get_num_threads(), "kind": "oracle",
-            "sample": f"one Qwen2.5-7B-shaped adapter of the same fleet recipe ({n} modules, r=64, S 1/12): "
-                      "fp64 QR of B and A^T, SVD of R_B R_A^T, allocation, export; BLAS threads as listed"}
+    """The oracle on the host cores: a process pool over all usable CPUs on one whole
+    adapter (196 modules, the S budget's scope), one worker on a 14-module sample, and
+    the dense definition route on the seven sample modules."""
+    info = host_info()
+    workers = max(1, info["usable_cpus"])
+    P = OraclePool(workers)
+    try:
+        P.fill(0)
+        P.run(range(min(P.lay.n, 2 * workers)))         # warm the workers (imports, first BLAS calls)
+        n, dt = P.run()
+    finally:
+        P.close()
+    P1 = OraclePool(1)
+    try:
+        P1.fill(0)
+        sample = [p * 28 + l for p in range(7) for l in (0, 1)]
+        P1.run(sample[:1])
+        n1, dt1 = P1.run(sample)
+    finally:
+        P1.close()
+    return {"value": round(n / dt, 2), "unit": "modules/s", "cores": workers, "kind": "oracle",
+            "sample": f"one Qwen2.5-7B-shaped adapter of the same fleet recipe ({n} modules, r=64, S 1/12 over "
+                      "the adapter): fp64 QR of B and A^T, SVD of R_B R_A^T, allocation, export; a spawned "
+                      f"process pool of {workers} workers with one BLAS thread each",
+            "one_core": {"value": round(n1 / dt1, 3), "unit": "modules/s",
+                         "sample": "layers 0 and 1 of every projection (14 modules), one worker"},
+            "definition_route": cpu_definition_route(),
+            "host": info}
 
 
 # -------------------------------------------------------------------- main
@@ -1058,27 +1181,35 @@ def main():
 
 
 def reference_arm(args, rank, world):
-    """The fp64 oracle, as it stands, on the host cores: each step is one adapter of the
-    same fleet recipe (a bounded sample of the headline workload)."""
+    """The fp64 oracle, as it stands, on the host cores: each step is one whole adapter of
+    the same fleet recipe (196 modules, the scope of the S budget), run by a process pool
+    over all usable CPUs with one BLAS thread per worker."""
     if rank != 0:
         return
-    import torch
+    info = host_info()
+    workers = max(1, info["usable_cpus"])
+    P = OraclePool(workers)
     steps = []
-    for s in range(args.warmup + args.steps):
-        n, dt = cpu_oracle_adapter(adapter=s, n_layers=7)
-        if s >= args.warmup:
-            steps.append((n, dt))
+    try:
+        for s in range(args.warmup + args.steps):
+            P.fill(s)
+            n, dt = P.run()
+            if s >= args.warmup:
+                steps.append((n, dt))
+    finally:
+        P.close()
     n = sum(a for a, _ in steps); t = sum(b for _, b in steps)
     v = n / t
     line = {"impl": "reference", "metric": METRIC, "value": round(v, 2), "unit": "modules/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * t / len(steps), 1),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic",
-            "config": {"workload": "factor construction fleet: Qwen2.5-7B-shaped adapters, r=64, LoRAForge-S 1/12 "
-                                   "floor 1; per step 7 of the 28 layers of one adapter (49 modules)"},
-            "cpu_baseline": {"kind": "oracle", "cores": torch.get_num_threads(), "value": round(v, 2),
-                             "unit": "modules/s", "sample": "7 layers x 7 projections of one adapter "
-                                                            "(49 modules) per step, allocation over those"},
+            "config": {"workload": "factor construction fleet: Qwen2.5-7B-shaped adapters (196 modules each), "
+                                   "r=64, LoRAForge-S 1/12 floor 1; per step one whole adapter"},
+            "cpu_baseline": {"kind": "oracle", "cores": workers, "value": round(v, 2), "unit": "modules/s",
+                             "sample": "one whole adapter (196 modules, allocation over the adapter) per step; "
+                                       f"spawned process pool of {workers} workers, one BLAS thread each",
+                             "host": info},
             "e2e": {"value": round(v, 2), "unit": "modules/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line))
 

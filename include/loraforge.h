@@ -175,13 +175,12 @@ lf_status lf_truncate_export(const lf_module* mods /*[host]*/, int32_t n, lf_pol
  * hold pool_elems_A / pool_elems_Bt elements; an adapter whose rows would reach
  * past a pool (or whose offset is not a multiple of 8, or k > 64) latches an error
  * on the device and its tokens are left untouched.
- * A small batch with few tokens per adapter (T < 512 and T <= 8 * n_adapters) is
- * applied token by token with each token's own adapter index (no sort).  Every
- * other batch is routed, whatever the number of resident adapters, by a stable sort
- * on the adapter id into segments (adapter, start, length) over a permutation of
- * token indices; segments with many tokens run on tcgen05 tensor cores, the rest
- * on a segmented GEMV; both read every adapter's k rows once per segment and never
- * pad k.  On the tensor-core path a 128-token tile whose tokens are consecutive rows
+ * A batch with few tokens per resident adapter (T <= 8 * n_adapters) is applied
+ * token by token with each token's own adapter index (no sort).  Other batches are
+ * routed by a stable sort on the adapter id into segments (adapter, start, length)
+ * over a permutation of token indices; segments of 64 or more tokens run on tcgen05
+ * tensor cores (every adapter's k rows read once per 128-token tile), the other
+ * tokens on the token-parallel kernel in routing order; k is never padded.  On the tensor-core path a 128-token tile whose tokens are consecutive rows
  * of x and y (a prefill request) moves x and y by TMA tiles; a tile of scattered
  * tokens gathers its rows one by one (same results, bit for bit).  If seg_out is
  * not NULL it receives the routing, as int32: [n_seg,
@@ -245,8 +244,7 @@ lf_status lf_lora_shrink_expand_slices(int32_t T, int32_t d_in, const void* x, v
  * routing pass on it (lf_route_tokens or any unrouted apply call).  A routed call on
  * a workspace whose tables were written for another T or n_adapters (or never)
  * applies nothing and latches LF_ERR_INVALID_ARG.  In the decode regime
- * (T < 512 and T <= 8 n_adapters) the side path reads ids directly and the tables
- * are not used.
+ * (T <= 8 n_adapters) the side path reads ids directly and the tables are not used.
  * Host errors as for lf_lora_shrink_expand_slices. */
 lf_status lf_route_tokens(int32_t T, const int32_t* ids, int32_t n_adapters, void* ws, size_t ws_bytes,
                           lf_stream_t stream);
@@ -319,6 +317,41 @@ lf_status lf_jd_full(const lf_module* mods /*[host]*/, int32_t n_mods,
                      const float* B_base, const float* A_base, const double* weights,
                      int32_t iters, float* U_base, float* Vt_base, float* sigma,
                      void* ws, size_t ws_bytes, lf_stream_t stream);
+
+/* ---- Pool-wide shared subspace (LoRASpace) ------------------------------------
+ * LoRASpace (the arXiv listing's abstract, "LoRASpace: A Pool-Wide Shared Substrate
+ * for Static and Dynamic Multi-LoRA Composition"): the stacked factors of a LoRA pool
+ * need far fewer directions than their summed ranks; the SVD of the stack gives the
+ * minimal subspace that keeps 99 % of the factor energy.
+ * side 0: the row factors A_i (r_i x d, row-major, element offset offs[i] of base) are
+ *   stacked as rows, S = [A_1; A_2; ...] (R x d);
+ * side 1: the column factors B_i (d x r_i, row-major, element offset offs[i]) are put
+ *   side by side, S = [B_1 B_2 ...] (d x R).
+ * R = sum r_i, at most LF_POOL_MAX_RANK and at most d.  "Stack vector" a is row a of S
+ * (side 0) or column a (side 1), in the order of the factors.
+ * Outputs (device): k (1 int): the smallest k >= 1 whose leading directions hold
+ *   num/den of the energy sum_j sigma_j^2 (sums in order); sigma (R doubles): the
+ *   singular values of S, descending; basis (R x d fp32, row-major): row j = direction j
+ *   (orthonormal; the right singular vectors of the stacked rows, or the left ones of
+ *   the side-by-side columns); a direction with sigma_j <= 1e-6 sigma_1, which the
+ *   fp64 Gram does not resolve, has a zero row; coef (R x R fp32):
+ *   coef[a][j] = (stack vector a) . (direction j), so factor i is approximated by its
+ *   rows' first k coefficients times the first k directions; resid (1 double): the
+ *   energy outside the subspace, sum_a sum_{j >= k} coef[a][j]^2.
+ * Computed as the eigen-decomposition of the fp64 Gram S S^T (S^T S for side 1) by a
+ * one-sided Jacobi iteration across the GPU (cooperative launch).  All memory is the
+ * caller's; workspace: lf_pool_workspace_size (0 for invalid arguments).
+ * Errors: LF_ERR_INVALID_ARG (side, counts, ranks < 1, negative offsets, num/den not a
+ * fraction, null pointers), LF_ERR_SHAPE (R > LF_POOL_MAX_RANK or R > d),
+ * LF_ERR_WORKSPACE.  Device-side: LF_ERR_NUMERIC for a non-finite input (read as 0),
+ * LF_ERR_TIMEOUT when a grid barrier does not complete. */
+#define LF_POOL_MAX_RANK 512
+size_t lf_pool_workspace_size(int32_t side, int32_t n_lora, const int32_t* ranks /*[host]*/,
+                              const int64_t* offs /*[host]*/, int32_t d);
+lf_status lf_pool_subspace(int32_t side, int32_t n_lora, const int32_t* ranks /*[host]*/,
+                           const int64_t* offs /*[host]*/, int32_t d, const float* base,
+                           int32_t num, int32_t den, int32_t* k, double* sigma, float* basis,
+                           float* coef, double* resid, void* ws, size_t ws_bytes, lf_stream_t stream);
 
 /* ---- Shrink / expand with library-owned scratch -------------------------------
  * This entry point has no counterpart in the paper; it exists for callers that

@@ -129,6 +129,33 @@ def pool_subspace_rows(A_base, A_offs, ranks, d_in: int, num: int = 99, den: int
     return int(k[0].item()), F.sigma[0, :R], F
 
 
+@dataclasses.dataclass
+class PoolSubspace:
+    k: torch.Tensor        # int32 [1]
+    sigma: torch.Tensor    # fp64 [R], descending
+    basis: torch.Tensor    # fp32 [R, d], row j = direction j
+    coef: torch.Tensor     # fp32 [R, R], coef[a, j] = stack vector a . direction j
+    resid: torch.Tensor    # fp64 [1]
+
+
+def pool_subspace(base, offs, ranks, d: int, side: str = "row", num: int = 99, den: int = 100, stream=None):
+    """LoRASpace's pool-wide subspace of a pool's stacked factors on the GPU
+    (lf_pool_subspace): side "row" stacks the A_i (r_i x d) stored at element offsets
+    offs of `base`, side "col" puts the B_i (d x r_i) side by side.  Allocates the
+    outputs and the workspace as torch tensors."""
+    sd = {"row": 0, "col": 1}[side]
+    R = int(sum(int(r) for r in ranks))
+    dev = base.device
+    ws = workspace(lf.lf_pool_workspace_size(sd, ranks, offs, d), dev)
+    out = PoolSubspace(torch.zeros(1, dtype=torch.int32, device=dev), torch.zeros(R, dtype=torch.float64, device=dev),
+                       torch.zeros(R, d, dtype=torch.float32, device=dev),
+                       torch.zeros(R, R, dtype=torch.float32, device=dev),
+                       torch.zeros(1, dtype=torch.float64, device=dev))
+    lf.lf_pool_subspace(sd, ranks, offs, d, base, num, den, out.k, out.sigma, out.basis, out.coef, out.resid, ws,
+                        stream)
+    return out
+
+
 def shrink_expand(x, y, ids, ranks, off_A, off_Bt, A_pool, Bt_pool, scale, ws=None, seg_out=None,
                   stream=None):
     n_adapters = ranks.numel()

@@ -20,7 +20,7 @@ constexpr int kGemvThreads = 256;
 constexpr int kGemvCols = kGemvThreads * 8;   // d_out columns per CTA
 
 struct RouteOut {
-    int32_t* counts;     // [0] n_seg, [1] n_valid, [2] n_items, [3] n_tc_items
+    int32_t* counts;     // [0] n_seg, [1] n_valid, [2] n_items, [3] n_tc_items, [4] n_tok (with tok_list)
     Seg* segs;           // min(T, n_adapters)
     int32_t* perm;       // T
     GemvItem* items;     // T / kGemvTok + min(T, n_adapters)
@@ -32,6 +32,9 @@ struct RouteOut {
     int32_t* run_start;  // first token of run i
     int32_t* run_pos;    // position of run i's first token in the permutation
     int32_t* tag;        // nullable: {kRouteTagMagic, T, n_adapters, tc_enable} once the tables are complete
+    // nullable, T ints: the tokens of every segment that is not a tensor-core segment,
+    // in routing order (adapter by adapter), for the token-parallel kernel
+    int32_t* tok_list;
 };
 
 // Tag of a workspace whose routing tables were written for a batch of T tokens over
@@ -76,10 +79,10 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const int32_t* __r
                                                               int n_adapters, RouteOut o) {
     extern __shared__ int32_t rsm[];
     int32_t* cnt = rsm;                  // n_adapters: counts, then running positions
-    int32_t* segidx = rsm + n_adapters;  // n_adapters: segment index of each adapter
+    int32_t* tokoff = rsm + n_adapters;  // n_adapters: first tok_list position of each adapter
     __shared__ int32_t wbase[32][32];
     __shared__ int wsum[32];
-    __shared__ int s_carry[4];
+    __shared__ int s_carry[5];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int nthr = (int)blockDim.x;
     for (int a = tid; a < n_adapters; a += nthr) cnt[a] = 0;
@@ -132,23 +135,25 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const int32_t* __r
         }
     }
     __syncthreads();
-    if (tid == 0) s_carry[0] = s_carry[1] = s_carry[2] = s_carry[3] = 0;
+    if (tid == 0) s_carry[0] = s_carry[1] = s_carry[2] = s_carry[3] = s_carry[4] = 0;
     __syncthreads();
-    // scans over adapters in chunks of kRouteThreads: token start, segment index, item index
+    // scans over adapters in chunks of kRouteThreads: token start, segment index, item
+    // index, tensor-core item index, token-list position
     for (int a0 = 0; a0 < n_adapters; a0 += nthr) {
         const int a = a0 + tid;
         const int c = a < n_adapters ? cnt[a] : 0;
         const bool use_tc = o.tc_enable && c >= kTcMin;
         const int ni = use_tc ? 0 : (c + kGemvTok - 1) / kGemvTok;
         const int nti = use_tc ? (c + kTcM - 1) / kTcM : 0;
-        int tt, ts, ti, tq;
+        int tt, ts, ti, tq, tb;
         const int start = block_excl_scan(c, wsum, &tt) + s_carry[0];
         const int sidx = block_excl_scan(c > 0 ? 1 : 0, wsum, &ts) + s_carry[1];
         const int iidx = block_excl_scan(ni, wsum, &ti) + s_carry[2];
         const int qidx = block_excl_scan(nti, wsum, &tq) + s_carry[3];
+        const int bidx = block_excl_scan(use_tc ? 0 : c, wsum, &tb) + s_carry[4];
         if (a < n_adapters) {
             cnt[a] = start;
-            segidx[a] = sidx;
+            tokoff[a] = use_tc ? -1 : bidx;
             if (c > 0) {
                 o.segs[sidx] = Seg{a, start, c};
                 for (int q = 0; q < nti; ++q) {
@@ -174,6 +179,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const int32_t* __r
             s_carry[1] += ts;
             s_carry[2] += ti;
             s_carry[3] += tq;
+            s_carry[4] += tb;
         }
         __syncthreads();
     }
@@ -183,6 +189,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const int32_t* __r
         o.counts[1] = nval;
         o.counts[2] = s_carry[2];
         o.counts[3] = s_carry[3];
+        if (o.tok_list) o.counts[4] = s_carry[4];
         if (o.tag) {
             o.tag[0] = kRouteTagMagic;
             o.tag[1] = T;
@@ -273,6 +280,16 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const int32_t* __r
         const int n = g.ntok, p0 = g.tok0;
 #pragma unroll
         for (int q = 0; q < kGemvTok; ++q) g.tok[q] = q < n ? o.perm[p0 + q] : 0;
+    }
+    if (o.tok_list) {
+        // tokens of the segments left to the token-parallel kernel, segment by segment
+        // (one warp per segment; the permutation is complete after the barrier above)
+        for (int sg = warp; sg < nseg; sg += nthr / 32) {
+            const Seg sgm = o.segs[sg];
+            const int off = tokoff[sgm.adapter];
+            if (off < 0) continue;
+            for (int q = lane; q < sgm.len; q += 32) o.tok_list[off + q] = o.perm[sgm.start + q];
+        }
     }
     if (o.seg_out) {
         if (tid == 0) {
@@ -450,7 +467,7 @@ __global__ void __launch_bounds__(kGemvThreads) expand_kernel(ApplyArgs a) {
 __global__ void route_check_kernel(int32_t* tag, int32_t* counts, int T, int n_adapters, int tc_enable) {
     if (threadIdx.x != 0) return;
     if (!(tag[0] == kRouteTagMagic && tag[1] == T && tag[2] == n_adapters && tag[3] == tc_enable)) {
-        counts[0] = counts[1] = counts[2] = counts[3] = 0;
+        counts[0] = counts[1] = counts[2] = counts[3] = counts[4] = 0;
         latch_error(LF_ERR_INVALID_ARG);
     }
 }
@@ -470,11 +487,9 @@ constexpr int kBgmvVec = 4;                                  // 8-column vectors
 constexpr int kBgmvCols = kBgmvThreads * 8 * kBgmvVec;       // d_out columns per CTA
 constexpr int kBgmvJ = 8;                                    // retained directions per shrink pass
 
-__global__ void __launch_bounds__(kBgmvThreads, 2) bgmv_kernel(ApplyArgs a) {
-    __shared__ float red[kBgmvThreads / 32][kBgmvJ];
-    __shared__ float ts[kMaxRank];
-    __shared__ float tw[kMaxRank];
-    const int tok = blockIdx.x;
+// One (token, column chunk) of the token-parallel side path; CTA-uniform control flow.
+__device__ __forceinline__ void bgmv_token(const ApplyArgs& a, int tok, float (&red)[kBgmvThreads / 32][kBgmvJ],
+                                           float* ts, float* tw) {
     const int ad = a.ids[tok];
     if (ad == -1) return;
     const int sl = slice_of_chunk(a, blockIdx.y);
@@ -562,6 +577,26 @@ __global__ void __launch_bounds__(kBgmvThreads, 2) bgmv_kernel(ApplyArgs a) {
             y2[q] = __floats2bfloat162_rn(fmaf(scale, acc[2 * q], yf.x), fmaf(scale, acc[2 * q + 1], yf.y));
         }
         *reinterpret_cast<uint4*>(yr + e) = yv;
+    }
+}
+
+// LIST = false: CTA blockIdx.x applies token blockIdx.x (decode regime, no routing pass).
+// LIST = true: grid.x strides over the routing's list of tokens outside the tensor-core
+// segments (tok_list, counts[4] of them, adapter by adapter, so consecutive CTAs read the
+// same factors from L2).
+template <bool LIST>
+__global__ void __launch_bounds__(kBgmvThreads, 2) bgmv_kernel(ApplyArgs a) {
+    __shared__ float red[kBgmvThreads / 32][kBgmvJ];
+    __shared__ float ts[kMaxRank];
+    __shared__ float tw[kMaxRank];
+    if (!LIST) {
+        bgmv_token(a, blockIdx.x, red, ts, tw);
+        return;
+    }
+    const int n_tok = a.counts[4];
+    for (int u = blockIdx.x; u < n_tok; u += gridDim.x) {
+        bgmv_token(a, __ldg(a.tok_list + u), red, ts, tw);
+        __syncthreads();   // red / ts / tw are rewritten by the next token
     }
 }
 

@@ -60,11 +60,13 @@ struct ApplyArgs {
     const float* sigma;
     SliceTab sl[kMaxSlices];
     // routing (sorted path)
-    const int32_t* counts;     // [0] segments, [1] routed tokens, [2] GEMV items, [3] tensor-core items
+    const int32_t* counts;     // [0] segments, [1] routed tokens, [2] GEMV items, [3] tensor-core items,
+                               // [4] tokens in tok_list
     const Seg* segs;
     const int32_t* perm;
     const GemvItem* items;
     const TcItem* tc_items;
+    const int32_t* tok_list;   // nullable: tokens for the token-parallel kernel (counts[4] of them)
     float* t_buf;              // T x ldt fp32, row = permutation position
     float* t_part;             // kTcMaxSplit x T x ldt fp32 split-K partials
 };

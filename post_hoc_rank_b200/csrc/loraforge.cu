@@ -12,9 +12,11 @@
 #include "common.cuh"
 #include "tsqr.cuh"
 #include "gram.cuh"
+#include "gram_i8.cuh"
 #include "select_export.cuh"
 #include "apply.cuh"
 #include "jd.cuh"
+#include "pool.cuh"
 
 namespace lf {
 
@@ -157,8 +159,48 @@ static void plan_tsqr(const lf_module* mods, int32_t n, TsqrPlan& p) {
                      [](const TsqrWork& a, const TsqrWork& b) { return a.nrows > b.nrows; });
 }
 
+// Work list of the integer-Gram leaf: every matrix whose rows the bulk copies can
+// address (16-byte aligned rows and offsets) in items of at most kI8MaxRows rows,
+// longest first; fb (per matrix) starts at 1 for the others, which the fp64 leaf takes.
+struct I8Plan {
+    std::vector<TsqrWork> work;
+    std::vector<TsqrInfo> info;
+    std::vector<int32_t> fb;
+    int32_t slots = 0;
+};
+
+static bool i8_eligible(const lf_module& m, int factor) {
+    return factor == 0 ? ((m.r & 3) == 0 && (m.B_off & 3) == 0) : ((m.d_in & 3) == 0 && (m.A_off & 3) == 0);
+}
+
+static void plan_i8(const lf_module* mods, int32_t n, I8Plan& p) {
+    p.work.clear();
+    p.info.assign((size_t)2 * n, TsqrInfo{0, -1});
+    p.fb.assign((size_t)2 * n, 1);
+    p.slots = 0;
+    for (int32_t i = 0; i < n; ++i)
+        for (int f = 0; f < 2; ++f) {
+            if (!i8_eligible(mods[i], f)) continue;
+            const int rows = f == 0 ? mods[i].d_out : mods[i].d_in;
+            const int nch = (int)cdiv(rows, kI8MaxRows);
+            const int mf = 2 * i + f;
+            p.info[mf] = TsqrInfo{nch, nch > 1 ? p.slots : -1};
+            p.fb[mf] = 0;
+            for (int c = 0; c < nch; ++c)
+                p.work.push_back(TsqrWork{mf, c * kI8MaxRows, std::min(kI8MaxRows, rows - c * kI8MaxRows),
+                                          nch > 1 ? p.slots + c : -1});
+            if (nch > 1) p.slots += nch;
+        }
+    std::stable_sort(p.work.begin(), p.work.end(),
+                     [](const TsqrWork& a, const TsqrWork& b) { return a.nrows > b.nrows; });
+}
+
+static size_t i8_slot_bytes(int RT) {
+    return sizeof(double) * (size_t)(RT == 16 ? tri_size<16>() : (RT == 32 ? tri_size<32>() : tri_size<64>()));
+}
+
 struct TsqrLayout {
-    size_t mods, work, nwork, info, n_dev, counters, partial, total;
+    size_t mods, work, nwork, info, n_dev, counters, partial, i8work, i8info, fb, i8partial, total;
 };
 
 // Partial-slot bytes: the fp64 packed Gram of the leaf pass or the fp32 partial R of
@@ -167,7 +209,7 @@ static size_t tsqr_slot_bytes(int RT) {
     return RT == 16 ? gram_slot_bytes<16>() : (RT == 32 ? gram_slot_bytes<32>() : gram_slot_bytes<64>());
 }
 
-static TsqrLayout tsqr_layout(int32_t n, const TsqrPlan& p) {
+static TsqrLayout tsqr_layout(int32_t n, const TsqrPlan& p, const I8Plan& q) {
     Carver c(nullptr);
     TsqrLayout L;
 #define LF_TAKE(field, T, cnt)                          \
@@ -180,8 +222,13 @@ static TsqrLayout tsqr_layout(int32_t n, const TsqrPlan& p) {
     LF_TAKE(nwork, int32_t, 1);
     LF_TAKE(info, TsqrInfo, p.info.size());
     LF_TAKE(n_dev, int32_t, 1);
-    LF_TAKE(counters, int32_t, (size_t)6 * n);   // Gram counters, Householder counters, flags (2n each)
+    // Gram counters, Householder counters, flags, integer-Gram counters (2n each)
+    LF_TAKE(counters, int32_t, (size_t)8 * n);
     LF_TAKE(partial, char, (size_t)p.slots * tsqr_slot_bytes(p.RT));
+    LF_TAKE(i8work, TsqrWork, q.work.size());
+    LF_TAKE(i8info, TsqrInfo, q.info.size());
+    LF_TAKE(fb, int32_t, q.fb.size());
+    LF_TAKE(i8partial, char, (size_t)q.slots * i8_slot_bytes(p.RT));
 #undef LF_TAKE
     L.total = c.off + 256;
     return L;
@@ -196,6 +243,27 @@ static cudaError_t launch_tsqr(const TsqrArgs<T>& a, int n_items, cudaStream_t s
     const int grid = std::min((n_items + W - 1) / W, 148 * (sizeof(T) == 4 ? 16 : 8));
     if (grid > 0) LF_LAUNCH(sizeof(T) == 8 ? "tsqr_fp64_refine" : "tsqr_householder", k, grid, 32 * W, 0, st, a);
     return cudaGetLastError();
+}
+
+template <int RT>
+static cudaError_t launch_gram_i8(const GramI8Args& a, cudaStream_t st) {
+    if (a.n_work <= 0) return cudaSuccess;
+    int dev = 0, sms = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(gram_i8_kernel<RT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gram_i8_smem());
+    if (e != cudaSuccess) return e;
+    // one persistent CTA per SM (all of its tensor memory), static round-robin over the items
+    const int grid = std::min(a.n_work, std::max(sms, 1));
+    LF_LAUNCH("tsqr_gram_i8", gram_i8_kernel<RT>, grid, kI8Threads, gram_i8_smem(), st, a);
+    return cudaGetLastError();
+}
+
+static cudaError_t launch_gram_i8_rt(int RT, const GramI8Args& a, cudaStream_t st) {
+    if (RT == 16) return launch_gram_i8<16>(a, st);
+    if (RT == 32) return launch_gram_i8<32>(a, st);
+    return launch_gram_i8<64>(a, st);
 }
 
 template <int RT>
@@ -349,6 +417,7 @@ struct ApplyWs {
     TcItem* tc_items;
     float* t_part;
     int32_t* runs;
+    int32_t* tok_list;
 };
 
 // Carves (or, with base == nullptr, sizes) the side-path workspace for T tokens,
@@ -360,12 +429,13 @@ static size_t carve_apply(void* base, int64_t T, int64_t n, int ns, ApplyWs* w) 
     // routing tables first: their offsets depend on (T, n) only, so a routing pass on
     // this workspace serves calls with any number of slices
     w->tag = c.take<int32_t>(4);
-    w->counts = c.take<int32_t>(4);
+    w->counts = c.take<int32_t>(8);
     w->segs = c.take<Seg>((size_t)std::max<int64_t>(mseg, 1));
     w->perm = c.take<int32_t>((size_t)T1);
     w->items = c.take<GemvItem>((size_t)(T / kGemvTok + mseg + 1));
     w->tc_items = c.take<TcItem>((size_t)(T / kTcM + mseg + 1));
     w->runs = c.take<int32_t>((size_t)2 * T1);   // run scratch of the routing pass
+    w->tok_list = c.take<int32_t>((size_t)T1);   // tokens outside the tensor-core segments
     w->t_buf = c.take<float>((size_t)T1 * kMaxRank * ns);
     w->t_part = c.take<float>((size_t)kTcMaxSplit * T1 * kMaxRank * ns);
     return c.off + 256;
@@ -432,15 +502,13 @@ struct SharedSlice {
     int32_t mode = 0;
 };
 
-// Decode regime (token-parallel kernel, no routing pass) for small batches with few
-// tokens per adapter on average: T < kDecodeMaxTokens and T <= kGemvTok * n_adapters.
-// Every larger batch is routed, so its long segments (a prefill request of hundreds of
-// tokens) reach the GEMV items or the tensor-core tiles however many adapters are
-// resident.  The rule reads only T and the adapter count, so it costs no device pass.
-constexpr int64_t kDecodeMaxTokens = 512;
-static bool decode_regime(int64_t T, int64_t n_adapters) {
-    return T < kDecodeMaxTokens && T <= (int64_t)kGemvTok * n_adapters;
-}
+// Decode regime (token-parallel kernel, no routing pass): few tokens per resident adapter,
+// T <= kGemvTok * n_adapters.  Other batches are routed: tensor-core tiles for segments of
+// kTcMin or more tokens, the token-parallel kernel over the routing's list for the rest.
+// Measured on the mixed batch of the large fleet (4096 tokens: 64 requests of 48 tokens and
+// 1024 decode tokens over 1024 resident adapters), routing it anyway was 1.9x slower: its
+// adapters of 64+ tokens gather scattered rows into tensor-core tiles.
+static bool decode_regime(int64_t T, int64_t n_adapters) { return T <= (int64_t)kGemvTok * n_adapters; }
 
 static lf_status apply_impl(int32_t T, int32_t d_in, const void* x, void* y, int64_t y_ld, const int32_t* ids,
                             int32_t n_adapters, const lf_slice* sl, int32_t ns, float scale, const float* scales,
@@ -502,6 +570,7 @@ static lf_status apply_impl(int32_t T, int32_t d_in, const void* x, void* y, int
     A.tc_items = w.tc_items;
     A.t_buf = w.t_buf;
     A.t_part = w.t_part;
+    A.tok_list = nullptr;
 
     RouteOut o{};
     o.counts = w.counts;
@@ -513,6 +582,7 @@ static lf_status apply_impl(int32_t T, int32_t d_in, const void* x, void* y, int
     o.run_pos = w.runs + T;
     o.seg_out = seg_out;
     o.tag = w.tag;
+    o.tok_list = w.tok_list;
     const bool token_parallel = decode_regime(T, n_adapters);
     o.tc_enable = token_parallel ? 0 : 1;
     const size_t rsmem = 2 * (size_t)n_adapters * sizeof(int32_t);
@@ -525,7 +595,7 @@ static lf_status apply_impl(int32_t T, int32_t d_in, const void* x, void* y, int
             LF_CUDA_TRY(cudaGetLastError());
         }
         set_chunks(A, kBgmvCols);
-        LF_LAUNCH("bgmv", bgmv_kernel, dim3((unsigned)T, (unsigned)A.n_chunks), kBgmvThreads, 0, s, A);
+        LF_LAUNCH("bgmv", bgmv_kernel<false>, dim3((unsigned)T, (unsigned)A.n_chunks), kBgmvThreads, 0, s, A);
         return launch_status();
     }
     if (routed)   // tables from an earlier routing pass on this workspace
@@ -533,16 +603,17 @@ static lf_status apply_impl(int32_t T, int32_t d_in, const void* x, void* y, int
     else
         LF_LAUNCH("route", route_kernel, 1, route_threads(T, n_adapters), rsmem, s, ids, T, n_adapters, o);
     LF_CUDA_TRY(cudaGetLastError());
-    const int64_t mseg = std::min<int64_t>(T, n_adapters);
-    // segments under kTcMin tokens: GEMV shrink (per slice), then expand
-    const unsigned max_items = (unsigned)(T / kGemvTok + mseg + 1);
-    set_chunks(A, kGemvCols);
-    LF_LAUNCH("shrink_gemv", shrink_kernel, gemv_grid((int64_t)max_items * ns), kGemvThreads, 0, s, A);
-    LF_CUDA_TRY(cudaGetLastError());
-    LF_LAUNCH("expand_gemv", expand_kernel, gemv_grid((int64_t)max_items * A.n_chunks), kGemvThreads, 0, s, A);
+    // segments under kTcMin tokens: the token-parallel kernel over the routing's token
+    // list (adapter by adapter); the grid strides over the device-side count
+    A.tok_list = w.tok_list;
+    set_chunks(A, kBgmvCols);
+    LF_LAUNCH("bgmv", bgmv_kernel<true>, dim3(gemv_grid(T), (unsigned)A.n_chunks), kBgmvThreads, 0, s, A);
     LF_CUDA_TRY(cudaGetLastError());
     // segments with >= kTcMin tokens: one tcgen05 shrink over all slices, then expand
-    const unsigned max_tc = (unsigned)(T / kTcM + mseg + 1);
+    // tensor-core items: a segment of c >= kTcMin tokens gives ceil(c / kTcM) of them, so
+    // there are at most T / kTcM + (segments of kTcMin or more tokens) + 1
+    const int64_t mseg = std::min<int64_t>(T, n_adapters);
+    const unsigned max_tc = (unsigned)(T / kTcM + std::min<int64_t>(mseg, T / kTcMin) + 1);
     const unsigned nsplit = (unsigned)cdiv(d_in, tc_split_len(d_in));
     set_chunks(A, kTcCols);
     alignas(64) CUtensorMap xmap, ymap;
@@ -820,6 +891,36 @@ static cudaError_t launch_jd_chol(int RT, const JdCholArgs& a, int grid, cudaStr
     return cudaGetLastError();
 }
 
+// ------------------------------------------------------- pool-wide subspace
+static size_t pool_layout(int32_t R, int32_t d, size_t* off /* 10 entries or nullptr */) {
+    Carver c(nullptr);
+    size_t o[10];
+    c.take<int64_t>((size_t)R); o[0] = c.off - (size_t)R * 8;          // row_off
+    c.take<int32_t>((size_t)R); o[1] = c.off - (size_t)R * 4;          // row_step
+    c.take<float>((size_t)R * d); o[2] = c.off - (size_t)R * d * 4;    // Sv
+    c.take<double>((size_t)R * R); o[3] = c.off - (size_t)R * R * 8;   // X
+    c.take<double>((size_t)R * R); o[4] = c.off - (size_t)R * R * 8;   // V
+    c.take<double>((size_t)R); o[5] = c.off - (size_t)R * 8;           // lam
+    c.take<int32_t>((size_t)R); o[6] = c.off - (size_t)R * 4;          // order
+    c.take<uint32_t>(8); o[7] = c.off - 32;                            // barrier words
+    c.take<double>((size_t)R); o[8] = c.off - (size_t)R * 8;           // resid parts
+    o[9] = 0;
+    if (off) std::memcpy(off, o, sizeof(o));
+    return c.off + 256;
+}
+
+static lf_status check_pool(int32_t side, int32_t n_lora, const int32_t* ranks, const int64_t* offs, int32_t d,
+                            int32_t* R_out) {
+    if ((side != 0 && side != 1) || n_lora < 1 || !ranks || !offs || d < 1) return LF_ERR_INVALID_ARG;
+    int64_t R = 0;
+    for (int32_t i = 0; i < n_lora; ++i) {
+        if (ranks[i] < 1 || offs[i] < 0) return LF_ERR_INVALID_ARG;
+        R += ranks[i];
+    }
+    if (R > kPoolMaxRank || R > d) return LF_ERR_SHAPE;
+    *R_out = (int32_t)R;
+    return LF_OK;
+}
 }  // namespace lf
 
 using namespace lf;
@@ -832,7 +933,9 @@ size_t lf_tsqr_workspace_size(const lf_module* mods, int32_t n) {
     if (check_mods(mods, n) != LF_OK) return 0;
     TsqrPlan p;
     plan_tsqr(mods, n, p);
-    return tsqr_layout(n, p).total;
+    I8Plan q;
+    plan_i8(mods, n, q);
+    return tsqr_layout(n, p, q).total;
 }
 
 lf_status lf_tsqr_batched(const lf_module* mods, int32_t n, const float* B_base, const float* A_base, float* R_B,
@@ -845,7 +948,9 @@ lf_status lf_tsqr_batched(const lf_module* mods, int32_t n, const float* B_base,
     if (!aligned16(B_base) || !aligned16(A_base)) return LF_ERR_ALIGNMENT;
     TsqrPlan p;
     plan_tsqr(mods, n, p);
-    const TsqrLayout L = tsqr_layout(n, p);
+    I8Plan q;
+    plan_i8(mods, n, q);
+    const TsqrLayout L = tsqr_layout(n, p, q);
     if (ws_bytes < L.total) return LF_ERR_WORKSPACE;
     char* base = reinterpret_cast<char*>(align_up((int64_t)reinterpret_cast<uintptr_t>(ws), 256));
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -858,10 +963,36 @@ lf_status lf_tsqr_batched(const lf_module* mods, int32_t n, const float* B_base,
     h.put(p.info.data(), p.info.size());
     h.put(&n, 1);
     LF_CUDA_TRY(cudaMemcpyAsync(base, h.buf.data(), h.off, cudaMemcpyHostToDevice, s));
-    LF_CUDA_TRY(cudaMemsetAsync(base + L.counters, 0, (size_t)6 * n * sizeof(int32_t), s));
+    LF_CUDA_TRY(cudaMemsetAsync(base + L.counters, 0, (size_t)8 * n * sizeof(int32_t), s));
+    Staging h8;   // the integer-Gram tables sit after the partial slots
+    h8.put(q.work.data(), q.work.size());
+    h8.put(q.info.data(), q.info.size());
+    h8.put(q.fb.data(), q.fb.size());
+    LF_CUDA_TRY(cudaMemcpyAsync(base + L.i8work, h8.buf.data(), h8.off, cudaMemcpyHostToDevice, s));
     int32_t* gram_counters = reinterpret_cast<int32_t*>(base + L.counters);
     int32_t* hh_counters = gram_counters + 2 * n;
     int32_t* flags = gram_counters + 4 * n;
+    int32_t* i8_counters = gram_counters + 6 * n;
+    int32_t* fb = reinterpret_cast<int32_t*>(base + L.fb);
+
+    // integer Gram on the tensor cores for every addressable matrix; a matrix it leaves
+    // (unaddressable rows, a value past its column scale, a non-finite value) is marked
+    // in fb and factored by the fp64 Gram leaf below
+    GramI8Args ia;
+    ia.mods = reinterpret_cast<const lf_module*>(base + L.mods);
+    ia.B_base = B_base;
+    ia.A_base = A_base;
+    ia.work = reinterpret_cast<const TsqrWork*>(base + L.i8work);
+    ia.n_work = (int32_t)q.work.size();
+    ia.info = reinterpret_cast<const TsqrInfo*>(base + L.i8info);
+    ia.counters = i8_counters;
+    ia.partial = reinterpret_cast<double*>(base + L.i8partial);
+    ia.fb = fb;
+    ia.flags = flags;
+    ia.R_B = R_B;
+    ia.R_A = R_A;
+    ia.rs = p.rs;
+    LF_CUDA_TRY(launch_gram_i8_rt(p.RT, ia, s));
 
     GramArgs ga;
     ga.mods = reinterpret_cast<const lf_module*>(base + L.mods);
@@ -877,7 +1008,7 @@ lf_status lf_tsqr_batched(const lf_module* mods, int32_t n, const float* B_base,
     ga.R_B = R_B;
     ga.R_A = R_A;
     ga.rs = p.rs;
-    ga.only = nullptr;
+    ga.only = fb;
     ga.R64 = nullptr;
     LF_CUDA_TRY(launch_gram_rt(p.RT, ga, nwork, s));
 
@@ -1218,6 +1349,7 @@ lf_status lf_route_tokens(int32_t T, const int32_t* ids, int32_t n_adapters, voi
     o.run_pos = w.runs + T;
     o.seg_out = nullptr;
     o.tag = w.tag;
+    o.tok_list = w.tok_list;
     o.tc_enable = decode_regime(T, n_adapters) ? 0 : 1;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const size_t rsmem = 2 * (size_t)n_adapters * sizeof(int32_t);
@@ -1522,6 +1654,82 @@ lf_status lf_jd_full(const lf_module* mods, int32_t n_mods, const int32_t* membe
         LF_CUDA_TRY(launch_jd(P.RX, P.RY, 1, &ca, ng, s));
     }
     return LF_OK;
+}
+
+size_t lf_pool_workspace_size(int32_t side, int32_t n_lora, const int32_t* ranks, const int64_t* offs, int32_t d) {
+    int32_t R = 0;
+    if (check_pool(side, n_lora, ranks, offs, d, &R) != LF_OK) return 0;
+    return pool_layout(R, d, nullptr);
+}
+
+lf_status lf_pool_subspace(int32_t side, int32_t n_lora, const int32_t* ranks, const int64_t* offs, int32_t d,
+                           const float* base, int32_t num, int32_t den, int32_t* k, double* sigma, float* basis,
+                           float* coef, double* resid, void* ws, size_t ws_bytes, lf_stream_t stream) {
+    int32_t R = 0;
+    lf_status st = check_pool(side, n_lora, ranks, offs, d, &R);
+    if (st != LF_OK) return st;
+    if (num < 0 || den <= 0 || num > den) return LF_ERR_INVALID_ARG;
+    if (!base || !k || !sigma || !basis || !coef || !resid || !ws) return LF_ERR_INVALID_ARG;
+    size_t off[10];
+    if (ws_bytes < pool_layout(R, d, off)) return LF_ERR_WORKSPACE;
+    char* w = reinterpret_cast<char*>(align_up((int64_t)reinterpret_cast<uintptr_t>(ws), 256));
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    // where each stack vector starts and its step: a row of A_i (r_i x d row-major, step 1)
+    // or a column of B_i (d x r_i row-major, step r_i)
+    std::vector<int64_t> row_off((size_t)R);
+    std::vector<int32_t> row_step((size_t)R);
+    for (int32_t i = 0, a = 0; i < n_lora; ++i)
+        for (int32_t c = 0; c < ranks[i]; ++c, ++a) {
+            row_off[a] = side == 0 ? offs[i] + (int64_t)c * d : offs[i] + c;
+            row_step[a] = side == 0 ? 1 : ranks[i];
+        }
+    Staging h;
+    h.put(row_off.data(), row_off.size());
+    h.put(row_step.data(), row_step.size());
+    LF_CUDA_TRY(cudaMemcpyAsync(w, h.buf.data(), h.off, cudaMemcpyHostToDevice, s));
+    LF_CUDA_TRY(cudaMemsetAsync(w + off[7], 0, 32, s));
+    PoolArgs a;
+    a.R = R;
+    a.d = d;
+    a.num = num;
+    a.den = den;
+    a.base = base;
+    a.row_off = reinterpret_cast<const int64_t*>(w + off[0]);
+    a.row_step = reinterpret_cast<const int32_t*>(w + off[1]);
+    a.Sv = reinterpret_cast<float*>(w + off[2]);
+    a.X = reinterpret_cast<double*>(w + off[3]);
+    a.V = reinterpret_cast<double*>(w + off[4]);
+    a.lam = reinterpret_cast<double*>(w + off[5]);
+    a.order = reinterpret_cast<int32_t*>(w + off[6]);
+    a.bar = reinterpret_cast<uint32_t*>(w + off[7]);
+    a.k_out = k;
+    a.sigma = sigma;
+    a.basis = basis;
+    a.coef = coef;
+    a.resid_part = reinterpret_cast<double*>(w + off[8]);
+    a.resid = resid;
+    const unsigned tiles = (unsigned)cdiv(R, kPoolTile);
+    const unsigned xblocks = (unsigned)std::min<int64_t>(cdiv(d, kPoolThreads), 64);
+    LF_LAUNCH("pool_gather", pool_gather_kernel, dim3(xblocks, (unsigned)R), kPoolThreads, 0, s, a);
+    LF_LAUNCH("pool_gram", pool_gram_kernel, dim3(tiles, tiles), kPoolThreads, 0, s, a);
+    // cooperative launch: every CTA resident (one per SM at most), so the grid barrier completes
+    int dev = 0, sms = 0, per_sm = 0;
+    LF_CUDA_TRY(cudaGetDevice(&dev));
+    LF_CUDA_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+    LF_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, pool_jacobi_kernel, kPoolThreads, 0));
+    const int pairs = (R + 1) / 2;
+    const int grid = std::max(1, std::min({sms * std::max(per_sm, 1), sms, (int)cdiv(pairs, kPoolThreads / 32)}));
+    {
+        PhaseScope ps_("pool_jacobi", s);
+        void* args[] = {&a};
+        LF_CUDA_TRY(cudaLaunchCooperativeKernel((const void*)pool_jacobi_kernel, dim3(grid), dim3(kPoolThreads), args,
+                                                0, s));
+    }
+    LF_LAUNCH("pool_order", pool_order_kernel, 1, kPoolMaxRank, 0, s, a);
+    LF_LAUNCH("pool_basis", pool_basis_kernel, dim3((unsigned)cdiv(d, kPoolThreads), tiles), kPoolThreads, 0, s, a);
+    LF_LAUNCH("pool_coef", pool_coef_kernel, dim3(tiles, tiles), kPoolThreads, 0, s, a);
+    LF_LAUNCH("pool_resid", pool_resid_kernel, 1, kPoolMaxRank, 0, s, a);
+    return launch_status();
 }
 
 void lf_profile_enable(int on) { g_prof.on = on != 0; }

@@ -122,6 +122,9 @@ def lib() -> ctypes.CDLL:
                                                     _I64, _I64, ctypes.c_float, _P, _P]
         L.lf_lora_shrink_expand_noalloc.restype = ctypes.c_int
         L.lf_check_bounded_wait.argtypes = [_I32, _P]; L.lf_check_bounded_wait.restype = ctypes.c_int
+        L.lf_pool_workspace_size.argtypes = [_I32, _I32, _P, _P, _I32]; L.lf_pool_workspace_size.restype = _SZ
+        L.lf_pool_subspace.argtypes = [_I32, _I32, _P, _P, _I32, _P, _I32, _I32, _P, _P, _P, _P, _P, _P, _SZ, _P]
+        L.lf_pool_subspace.restype = ctypes.c_int
         L.lf_status_string.argtypes = [ctypes.c_int]; L.lf_status_string.restype = ctypes.c_char_p
         L.lf_get_device_status.argtypes = [_P]; L.lf_get_device_status.restype = ctypes.c_int
         L.lf_profile_enable.argtypes = [ctypes.c_int]; L.lf_profile_enable.restype = None
@@ -139,7 +142,8 @@ def exported_symbols() -> list[str]:
             "lf_profile_enable", "lf_profile_reset", "lf_profile_read", "lf_launch_count",
             "lf_lora_shrink_expand_noalloc", "lf_apply_slices_workspace_size", "lf_lora_shrink_expand_slices",
             "lf_lora_sigma_sandwich", "lf_jd_workspace_size", "lf_jd_full", "lf_route_tokens",
-            "lf_lora_shrink_expand_slices_routed", "lf_check_bounded_wait"]
+            "lf_lora_shrink_expand_slices_routed", "lf_check_bounded_wait", "lf_pool_workspace_size",
+            "lf_pool_subspace"]
 
 # Limits of lf_lora_shrink_expand_noalloc (its scratch is a fixed array in the library).
 NOALLOC_MAX_TOKENS = 16384
@@ -304,6 +308,23 @@ def _jd_tables(mods, members, probs):
 
 def lf_jd_workspace_size(mods: np.ndarray, members: np.ndarray, probs: np.ndarray) -> int:
     return lib().lf_jd_workspace_size(*_jd_tables(mods, members, probs))
+
+
+def lf_pool_workspace_size(side, ranks, offs, d) -> int:
+    rk = np.ascontiguousarray(ranks, dtype=np.int32)
+    of = np.ascontiguousarray(offs, dtype=np.int64)
+    return lib().lf_pool_workspace_size(int(side), len(rk), rk.ctypes.data, of.ctypes.data, int(d))
+
+
+def lf_pool_subspace(side, ranks, offs, d, base, num, den, k, sigma, basis, coef, resid, ws, stream=None,
+                     check=True) -> int:
+    """Pool-wide subspace of stacked factors (side 0: rows A_i; side 1: columns of B_i)."""
+    rk = np.ascontiguousarray(ranks, dtype=np.int32)
+    of = np.ascontiguousarray(offs, dtype=np.int64)
+    st = lib().lf_pool_subspace(int(side), len(rk), rk.ctypes.data, of.ctypes.data, int(d), _ptr(base), int(num),
+                                int(den), _ptr(k), _ptr(sigma), _ptr(basis), _ptr(coef), _ptr(resid), _ptr(ws),
+                                ws.numel() if ws is not None else 0, _stream(stream))
+    return _check(st, "lf_pool_subspace") if check else st
 
 
 def lf_jd_full(mods, members, probs, B_base, A_base, weights, iters, U_base, Vt_base, sigma, ws, stream=None,

@@ -287,3 +287,27 @@ def test_energy_fraction_ranks_bit_exact(num, den):
     assert not np.any(diff & (gaps > 1e-12)), (ranks_g[diff], ranks_o[diff], gaps[diff])
     for eg, eo in G.recon_errors(lay, Bh, Ah, E, sig, range(lay.n)):
         assert abs(eg - eo) <= G.RECON_TOL
+
+
+@pytest.mark.parametrize("r", [64, 36])
+def test_integer_leaf_long_rows_and_scale_fallback(r):
+    """The integer-Gram leaf takes a matrix in items of at most 24576 rows: a factor of
+    26000 rows is two items whose packed Grams are merged in item order.  A factor whose
+    first 128 rows are 1e-3 times smaller than the rest exceeds the column scale taken on
+    those rows, so the leaf leaves it to the fp64 Gram leaf.  Both must give the oracle's
+    R and sigma; the profile shows the integer leaf ran."""
+    shapes = [("long", 26000, 400), ("spike", 3000, 512), ("plain", 1000, 26000)]
+    lay = synth.fleet_layout(1, shapes=shapes, r=r, n_layers=1)
+    Bh = torch.zeros(lay.B_total); Ah = torch.zeros(lay.A_total)
+    synth.fill_fleet(lay, Bh, Ah, cfg_id=15)
+    b0 = int(lay.B_off[1])
+    Bh[b0:b0 + 128 * r] *= 1e-3
+    B, A = upload(Bh, Ah)
+    mods = api.modules_from_layout(lay)
+    lf.lf_profile_reset(); lf.lf_profile_enable(True)
+    F = api.tsqr(mods, B, A)
+    lf.lf_profile_enable(False)
+    ph = lf.lf_profile_read()
+    assert lf.lf_get_device_status() == 0
+    assert ph.get("tsqr_gram_i8", (0, 0))[1] == 1, ph
+    check_tsqr(lay, Bh, Ah, F, range(lay.n))
