@@ -20,27 +20,30 @@
 // the R of X~ to ~1e-16 kappa^2, i.e. the leaf is backward stable with a columnwise
 // backward error below 2^-27 of the column maximum.  A value at or above 2^E_j (or a
 // non-finite one) marks the matrix for the fp64 leaf instead, as does a matrix whose
-// rows the bulk copies cannot address (row or offset not 16-byte aligned).
+// rows the copies cannot address (row or offset not 16-byte aligned).
 //
 // Data flow per CTA (persistent, one per SM, static round-robin over the work items,
 // longest first):
-//   warp 0        producer: 1-D bulk copies (cp.async.bulk, no multicast) of 64-row
-//                 fp32 stages into a kI8FStages ring (B: one contiguous block; A^T:
-//                 one 256-byte run per column), completion counted in bytes;
-//   warp 1        MMA issuer (one thread): per 128-row digit stage, D1 += [P3;P2] x
-//                 [P3;P2;P1;P0]^T (M 128, N 256) and D2 += [P1;P0] x [P1;P0]^T (M 128,
-//                 N 128) in four K = 32 steps each, into 384 TMEM columns;
+//   warp 0        producer: 64-row fp32 stages into a kI8FStages ring, completion
+//                 counted in bytes: B (row-major d_out x r) by one 1-D bulk copy per
+//                 stage, A^T (A is r x d_in row-major) by two 2-D TMA copies per stage
+//                 (boxes of 32 rows x r columns of A^T, 128-byte swizzle, no multicast)
+//                 through the matrix's tensor map;
+//   warp 1        MMA issuer (one thread): per 128-row digit stage, D1 += [P0;P1] x
+//                 [P0;P1;P2;P3]^T (M 128, N 256) and D2 += [P2;P3] x [P2;P3]^T (M 128,
+//                 N 128) in four K = 32 steps each, into 384 TMEM columns (plane p =
+//                 byte 3 - p);
 //   warps 2..9    converters: column scales, fp32 -> digit planes (K-major, 128-byte
-//                 swizzle, plane p = byte 3 - p) and the planes' column sums;
-//   warps 10..13  epilogue: int32 accumulators -> signed-digit corrections ->
-//                 fp64 Gram (packed upper triangle) -> fp64 Cholesky -> R.
-// The 16 digit-pair products of a column pair live in two TMEM lanes (a column's
-// planes 0 and 2 in lane i, planes 1 and 3 in lane 64 + i) and, for four of the pairs,
-// in the transposed position; the epilogue combines them through shared memory in a
-// fixed order, so the result does not depend on scheduling.  Converters hand the fp32
-// stages back as soon as their values are in registers, so the ring keeps up to six
-// 16 KB stages of the producer's copies in flight.
+//                 swizzle) and the planes' column sums;
+//   warps 10..13  epilogue: int32 accumulators -> signed-digit corrections -> the
+//                 item's fp64 Gram (packed upper triangle) in its own global slot.
+// Operand rows interleave the planes of a column (row 2c: plane 0 or 2 of column c,
+// row 2c + 1: plane 1 or 3), so both planes of column c sit in adjacent TMEM lanes of
+// one warp and the epilogue combines them with one shuffle.  gram_i8_root_kernel then
+// sums a matrix's item Grams in item order and takes the fp64 Cholesky, so the result
+// does not depend on scheduling.
 #pragma once
+#include <cuda.h>   // CUtensorMap (type only)
 #include <float.h>
 
 #include "common.cuh"
@@ -51,7 +54,7 @@ namespace lf {
 
 constexpr int kI8Rows = 128;         // rows (the MMA's K) per digit stage
 constexpr int kI8FRows = 64;         // rows per fp32 stage (two per digit stage)
-constexpr int kI8FStages = 6;
+constexpr int kI8FStages = 7;
 constexpr int kI8DStages = 2;
 constexpr int kI8ConvWarps = 8;
 constexpr int kI8EpiWarps = 4;
@@ -62,9 +65,9 @@ constexpr int kI8HeadBits = 2;       // 2^E is 4x to 8x the largest value of the
 // Rows per work item: the largest accumulator, 255^2 * rows, stays below 2^31, and the
 // corrected top-digit product times 2^24 stays below 2^53 (exact in fp64).
 constexpr int kI8MaxRows = 24576;
-constexpr int kI8LdS = 65;           // fp64 row stride of the epilogue's row buffers
-constexpr int kI8LdA = 68;           // fp32 column stride of an A^T stage (64 rows + 4)
-constexpr int kI8FStageFloats = kI8LdA * kI8FRows;
+constexpr int kI8LdS = 65;           // fp64 row stride of the epilogue's row buffer
+constexpr int kI8FStageFloats = kI8FRows * 64;   // 16 KB: B rows (stride r) or A^T as two swizzled halves
+constexpr int kI8AHalfBytes = 64 * 128;          // one A^T half: up to 64 columns x 32 rows
 constexpr uint32_t kI8TmemCols = 512;
 
 struct GramI8Meta {
@@ -74,12 +77,9 @@ struct GramI8Meta {
 };
 
 struct GramI8Smem {
-    uint8_t dig[kI8DStages][256 * 128];     // digit stages: 4 planes x 64 columns x 128 rows (first: 1024-aligned)
-    float f32[kI8FStages][kI8FStageFloats];
-    double W[64 * kI8LdS];                  // fp64 rows: lanes i and 64 + i of the accumulators, summed
-    double G[tri_size<64>()];               // packed Gram of a one-item matrix, then its Cholesky factor
-    double diag[64];
-    uint16_t kc[tri_size<64>()];            // packed index -> (row << 8) | column
+    uint8_t dig[kI8DStages][256 * 128];     // digit stages: 4 planes x 64 columns x 128 rows (1024-aligned)
+    float f32[kI8FStages][kI8FStageFloats]; // 1024-aligned (128-byte swizzle atoms of the A^T stages)
+    double W[64 * kI8LdS];                  // fp64 row i of the column pair (i, j) sums
     GramI8Meta meta[2];
     float cmax[4][64];
     uint64_t full_f[kI8FStages], empty_f[kI8FStages];
@@ -88,8 +88,6 @@ struct GramI8Smem {
     uint64_t meta_full[2], meta_empty[2];
     uint32_t tmem;
     int abort;
-    int flag;
-    int redo;
 };
 
 constexpr size_t gram_i8_smem() { return sizeof(GramI8Smem) + 1024; }
@@ -97,18 +95,16 @@ constexpr size_t gram_i8_smem() { return sizeof(GramI8Smem) + 1024; }
 struct GramI8Args {
     const lf_module* mods;
     const float* B_base;
-    const float* A_base;
-    const TsqrWork* work;      // work items of <= kI8MaxRows rows, longest first
+    const CUtensorMap* amaps;  // per module: tensor map of its A (dims d_in x r, box 32 x r, 128-byte swizzle)
+    const TsqrWork* work;      // work items of <= kI8MaxRows rows, longest first; .slot = the item's Gram slot
     int32_t n_work;
-    const TsqrInfo* info;      // per mf: items of the matrix and its first partial slot
-    int32_t* counters;         // per mf, zero on entry
-    double* partial;           // slot s: packed Gram (tri_size<RT> doubles) of one item
+    double* gram;              // slot s: packed Gram (tri_size<RT> doubles) of one item, scaled to the input
     int32_t* fb;               // per mf: set to 1 when the matrix is left to the fp64 leaf
-    int32_t* flags;            // per mf: set to 1 when the Cholesky rejects a pivot
-    float* R_B;
-    float* R_A;
-    int32_t rs;
 };
+
+// Operand row of plane p (0 = top byte) of column c in a digit stage: planes 0, 1 of
+// the columns interleaved in rows 0..127, planes 2, 3 in rows 128..255.
+__device__ __forceinline__ int i8_row(int p, int c) { return (p >> 1) * 128 + 2 * c + (p & 1); }
 
 // Barrier among `nthreads` threads on hardware barrier `id` that also ANDs a predicate:
 // every participant gets the same answer.
@@ -135,7 +131,10 @@ __device__ __forceinline__ void planes4(const uint32_t (&u)[4], uint32_t (&w)[4]
 }
 
 // 16 values of column c, rows 16 * qs .. 16 * qs + 15 of an fp32 stage (qs in 0..3);
-// rows at or past `nvalid` and columns at or past r read as zero.
+// rows at or past `nvalid` and columns at or past r read as zero.  B stages are
+// row-major with row stride r; A^T stages are two halves of 32 rows (the second at
+// 8 KB), each r rows of 128 bytes (one column of A^T per row) with 16-byte chunks
+// XOR-swizzled by row % 8.
 __device__ __forceinline__ void i8_load_unit(float (&x)[16], const float* st, int factor, int c, int qs, int r,
                                              int nvalid) {
     if (c >= r) {
@@ -143,14 +142,15 @@ __device__ __forceinline__ void i8_load_unit(float (&x)[16], const float* st, in
         for (int e = 0; e < 16; ++e) x[e] = 0.f;
         return;
     }
-    if (factor == 0) {   // B stage: row-major, row stride r
+    if (factor == 0) {
 #pragma unroll
         for (int e = 0; e < 16; ++e) x[e] = e < nvalid ? st[(16 * qs + e) * r + c] : 0.f;
-    } else {             // A^T stage: column c at c * kI8LdA, rows contiguous
-        const float4* p = reinterpret_cast<const float4*>(st + c * kI8LdA + 16 * qs);
+    } else {
+        const char* row = reinterpret_cast<const char*>(st) + (qs >> 1) * kI8AHalfBytes + c * 128;
 #pragma unroll
         for (int v = 0; v < 4; ++v) {
-            const float4 f = p[v];
+            const int chunk = (qs & 1) * 4 + v;
+            const float4 f = *reinterpret_cast<const float4*>(row + ((chunk ^ (c & 7)) << 4));
             x[4 * v + 0] = 4 * v + 0 < nvalid ? f.x : 0.f;
             x[4 * v + 1] = 4 * v + 1 < nvalid ? f.y : 0.f;
             x[4 * v + 2] = 4 * v + 2 < nvalid ? f.z : 0.f;
@@ -159,32 +159,23 @@ __device__ __forceinline__ void i8_load_unit(float (&x)[16], const float* st, in
     }
 }
 
-// Right-looking Cholesky of the packed Gram G (r x r used, packed for RT columns) by the
-// 128 epilogue threads: per column j the pivot test (d_j <= kGramPivotTol G_jj rejects, as
-// in the fp64 leaf), row j divided by r_jj, then the trailing triangle (packed entries
-// from (j+1, j+1) on, each updated by one thread) less the outer product of row j.
-// Returns false (for every thread alike) when a pivot is rejected.
-template <int RT>
-__device__ __forceinline__ bool i8_cholesky(double* G, double* diag, const uint16_t* kc, int r, int et) {
-    constexpr int TRI = tri_size<RT>();
-    constexpr int NT = 32 * kI8EpiWarps;
-    for (int j = et; j < r; j += NT) diag[j] = G[tri_off<RT>(j, j)];
-    tc::named_sync(2, NT);
-    for (int j = 0; j < r; ++j) {
-        const double d = G[tri_off<RT>(j, j)];
-        if (!(d > kGramPivotTol * diag[j])) return false;
-        const double rjj = sqrt(d);
-        for (int c = j + 1 + et; c < r; c += NT) G[tri_off<RT>(j, c)] /= rjj;
-        tc::named_sync(2, NT);
-        if (et == 0) G[tri_off<RT>(j, j)] = rjj;
-        const double* rowj = G + tri_off<RT>(j, j) - j;   // rowj[c] = G[j][c] for c >= j
-        for (int e = (j + 1 < RT ? tri_off<RT>(j + 1, j + 1) : TRI) + et; e < TRI; e += NT) {
-            const int k = kc[e] >> 8, c = kc[e] & 255;
-            if (c < r) G[e] -= rowj[k] * rowj[c];
-        }
-        tc::named_sync(2, NT);
-    }
-    return true;
+// Each thread of a warp reads, at three TMEM column addresses, 16 consecutive 32-bit
+// columns of its own lane as integers, then waits for the loads (one asm statement, so
+// no use of v can be scheduled before the wait).
+__device__ __forceinline__ void tmem_ld16x3(uint32_t t0, uint32_t t1, uint32_t t2, int32_t (&v)[48]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%48];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%49];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47}, [%50];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+          "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]),
+          "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]),
+          "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31]),
+          "=r"(v[32]), "=r"(v[33]), "=r"(v[34]), "=r"(v[35]), "=r"(v[36]), "=r"(v[37]), "=r"(v[38]), "=r"(v[39]),
+          "=r"(v[40]), "=r"(v[41]), "=r"(v[42]), "=r"(v[43]), "=r"(v[44]), "=r"(v[45]), "=r"(v[46]), "=r"(v[47])
+        : "r"(t0), "r"(t1), "r"(t2)
+        : "memory");
 }
 
 template <int RT>
@@ -211,8 +202,6 @@ __global__ void __launch_bounds__(kI8Threads, 1) gram_i8_kernel(GramI8Args a) {
         s.abort = 0;
         fence_barrier_init();
     }
-    for (int rr = 0, e0 = 0; rr < RT; e0 += RT - rr, ++rr)
-        for (int cc = rr + tid; cc < RT; cc += kI8Threads) s.kc[e0 + cc - rr] = (uint16_t)((rr << 8) | cc);
     if (warp == 1) tc::tmem_alloc(&s.tmem, kI8TmemCols);
     tc::fence_before_sync();
     __syncthreads();
@@ -236,33 +225,37 @@ __global__ void __launch_bounds__(kI8Threads, 1) gram_i8_kernel(GramI8Args a) {
             const int factor = w.mf & 1;
             const lf_module md = a.mods[w.mf >> 1];
             const int r = md.r;
-            const float* X = factor == 0 ? a.B_base + md.B_off : a.A_base + md.A_off;
+            const float* X = a.B_base + md.B_off;
+            const CUtensorMap* amap = a.amaps + (w.mf >> 1);
             const int nf = 2 * (int)cdiv(w.nrows, kI8Rows);
             for (int f = 0; f < nf; ++f, ++g) {
                 const int slot = g % kI8FStages;
                 if (g >= kI8FStages) ok = wait(&s.empty_f[slot], (uint32_t)((g / kI8FStages - 1) & 1));
                 if (!ok) break;
                 const int rows = max(0, min(kI8FRows, w.nrows - kI8FRows * f));
-                const uint32_t bytes = (uint32_t)rows * (uint32_t)r * 4u;
+                const int64_t row = (int64_t)w.row0 + (int64_t)kI8FRows * f;
                 if (lane == 0) {
-                    if (bytes) mbar_arrive_expect_tx(&s.full_f[slot], bytes);
-                    else mbar_arrive1(&s.full_f[slot]);
-                }
-                __syncwarp();
-                if (bytes) {
-                    const int64_t row = (int64_t)w.row0 + (int64_t)kI8FRows * f;
-                    if (factor == 0) {
-                        if (lane == 0) bulk_g2s(s.f32[slot], X + row * r, bytes, &s.full_f[slot]);
+                    if (rows == 0) {
+                        mbar_arrive1(&s.full_f[slot]);   // an empty second half of the last digit stage
+                    } else if (factor == 0) {
+                        const uint32_t bytes = (uint32_t)rows * (uint32_t)r * 4u;
+                        mbar_arrive_expect_tx(&s.full_f[slot], bytes);
+                        bulk_g2s(s.f32[slot], X + row * r, bytes, &s.full_f[slot]);
                     } else {
-                        for (int c = lane; c < r; c += 32)
-                            bulk_g2s(s.f32[slot] + c * kI8LdA, X + (int64_t)c * md.d_in + row, (uint32_t)rows * 4u,
-                                     &s.full_f[slot]);
+                        // one or two boxes of 32 rows of A^T (rows past d_in read as zeros)
+                        const uint32_t nbox = rows > 32 ? 2u : 1u;
+                        mbar_arrive_expect_tx(&s.full_f[slot], nbox * 32u * (uint32_t)r * 4u);
+                        tc::tma_load_2d(s.f32[slot], amap, (int)row, 0, &s.full_f[slot]);
+                        if (nbox == 2)
+                            tc::tma_load_2d(reinterpret_cast<char*>(s.f32[slot]) + kI8AHalfBytes, amap, (int)row + 32,
+                                            0, &s.full_f[slot]);
                     }
                 }
+                __syncwarp();
             }
         }
-        // no bulk copy of this warp may still be writing shared memory when the CTA
-        // leaves (on the normal path these phases completed before their conversion)
+        // no copy of this warp may still be writing shared memory when the CTA leaves
+        // (on the normal path these phases completed before their conversion)
         for (int q = max(0, g - kI8FStages); q < g; ++q)
             mbar_wait(&s.full_f[q % kI8FStages], (uint32_t)((q / kI8FStages) & 1));
     } else if (warp == 1) {
@@ -321,7 +314,7 @@ __global__ void __launch_bounds__(kI8Threads, 1) gram_i8_kernel(GramI8Args a) {
             GramI8Meta& M = s.meta[ms];
             // this thread's column and its two 16-row chunks (q0 and q0 + 4) of every
             // digit stage: B stages are read across columns (one row per load), A^T
-            // stages across chunks of 8 columns (16-byte loads, conflict-free at stride 68)
+            // stages across 8 columns of one chunk (16-byte loads, distinct swizzled chunks)
             const int c = factor == 0 ? 32 * (cw & 1) + lane : 8 * cw + (lane & 7);
             const int q0 = factor == 0 ? (cw >> 1) : (lane >> 3);
             for (int e = ct; e < 4 * 64; e += 32 * kI8ConvWarps) (&M.colsum[0][0])[e] = 0;
@@ -398,7 +391,7 @@ __global__ void __launch_bounds__(kI8Threads, 1) gram_i8_kernel(GramI8Args a) {
                     }
 #pragma unroll
                     for (int p = 0; p < 4; ++p) {
-                        const int R = 64 * p + c;   // operand row (plane p, column c), 128 bytes
+                        const int R = i8_row(p, c);   // operand row, 128 bytes
                         *reinterpret_cast<uint4*>(dig + R * 128 + ((q ^ (R & 7)) << 4)) =
                             make_uint4(pw[p][0], pw[p][1], pw[p][2], pw[p][3]);
                     }
@@ -418,17 +411,16 @@ __global__ void __launch_bounds__(kI8Threads, 1) gram_i8_kernel(GramI8Args a) {
         // ------------------------------------------------------------ epilogue
         const int et = tid - 32 * kI8EpiWarp0;   // 0..127
         const int lq = warp & 3;                 // the TMEM lane quarter this warp may read
-        const int m = 32 * lq + lane;            // accumulator row
-        const bool hi = m >= 64;                 // planes 1 and 3 of column i (else planes 0 and 2)
-        const int i = m & 63;
+        const int m = 32 * lq + lane;            // accumulator row: plane pair member m & 1 of column m >> 1
+        const bool odd = (m & 1) != 0;           // planes 1 and 3 of column i (else planes 0 and 2)
+        const int i = m >> 1;
         constexpr int TRI = tri_size<RT>();
         int k = 0;
         bool ok = true;
         for (int it = blockIdx.x; it < a.n_work && ok; it += gridDim.x, ++k) {
             const TsqrWork w = a.work[it];
-            const int mf = w.mf, factor = mf & 1;
+            const int mf = w.mf;
             const int r = a.mods[mf >> 1].r;
-            const int nch = a.info[mf].nchunks;
             const int64_t Krows = (int64_t)cdiv(w.nrows, kI8Rows) * kI8Rows;   // zero rows included
             const int ms = k & 1;
             ok = wait(&s.acc_full, (uint32_t)(k & 1)) && wait(&s.meta_full[ms], (uint32_t)((k >> 1) & 1));
@@ -436,114 +428,123 @@ __global__ void __launch_bounds__(kI8Threads, 1) gram_i8_kernel(GramI8Args a) {
             if (!ok) break;
             tc::fence_after_sync();
             const GramI8Meta& M = s.meta[ms];
-            // row i of this lane's products -> fp64 (exact integer combination, then at
-            // most two roundings); D1 columns 0..255: column planes 0..3 (byte 3..0);
-            // D2 columns 256..383: column planes 2, 3.  Lanes 0..63 (planes 0 and 2 of
-            // column i) store W[i][j]; after a barrier lanes 64..127 (planes 1 and 3) add
-            // theirs, so W = V1 + V2 in a fixed order.
-            double* Wrow = s.W + i * kI8LdS;
+            // Row i of the column pairs (i, j): this lane's six products -> fp64 (exact
+            // integer combination, then at most two roundings); D1 columns 2j, 2j+1:
+            // planes 0, 1 of column j; 128 + 2j, +1: planes 2, 3; D2 (from column 256)
+            // 2j, 2j+1: planes 2, 3.  The even lane (row planes 0 and 2) and the odd
+            // lane (planes 1 and 3) of column i add their values in that order.
             const int64_t Si0 = M.colsum[0][i], Si1 = M.colsum[1][i];
             const uint32_t tb = tmem + ((uint32_t)(32 * lq) << 16);
-            for (int pass = 0; pass < 2; ++pass) {
-                if (pass == 1) tc::named_sync(2, 32 * kI8EpiWarps);
-                if ((int)hi != pass) continue;
-                for (int jb = 0; jb < 8; ++jb) {
-                    const uint32_t ta[6] = {tb + 8 * jb, tb + 64 + 8 * jb, tb + 128 + 8 * jb,
-                                            tb + 192 + 8 * jb, tb + 256 + 8 * jb, tb + 320 + 8 * jb};
-                    int32_t v[48];
-                    tc::tmem_ld8x6(ta, v);
+            double* Wrow = s.W + i * kI8LdS;
+            for (int jb = 0; jb < 8; ++jb) {
+                int32_t v[48];
+                tmem_ld16x3(tb + 16 * jb, tb + 128 + 16 * jb, tb + 256 + 16 * jb, v);
+                double Wv[8];
 #pragma unroll
-                    for (int jj = 0; jj < 8; ++jj) {
-                        const int j = 8 * jb + jj;
-                        const int64_t p0 = v[jj], p1 = v[8 + jj], p2 = v[16 + jj], p3 = v[24 + jj];
-                        const int64_t p4 = v[32 + jj], p5 = v[40 + jj];
-                        double H, L;
-                        if (!hi) {
-                            // row plane 0 (top digit, signed as b3 - 128) and row plane 2
-                            const int64_t q33 = p0 - 128 * (Si0 + M.colsum[0][j]) + 16384 * Krows;
-                            const int64_t q32 = p1 - 128 * (int64_t)M.colsum[1][j];
-                            const int64_t q31 = p2 - 128 * (int64_t)M.colsum[2][j];
-                            const int64_t q30 = p3 - 128 * (int64_t)M.colsum[3][j];
-                            H = (double)(q33 * (1ll << 24) + q32 * (1ll << 16) + q31 * (1ll << 8) + q30) * 0x1p24 +
-                                (double)(p4 * (1ll << 8) + p5) * 0x1p8;
-                            L = (double)(q31 * (1ll << 8) + q30) * 0x1p24;
-                        } else {
-                            // row plane 1 and row plane 3
-                            const int64_t q23 = p0 - 128 * Si1;
-                            H = (double)(q23 * (1ll << 24) + p1 * (1ll << 16) + p2 * (1ll << 8) + p3) * 0x1p16 +
-                                (double)(p4 * (1ll << 8) + p5);
-                            L = (double)(p2 * (1ll << 8) + p3) * 0x1p16;
-                        }
-                        const double V = j > i ? H : (j < i ? L : H + L);
-                        Wrow[j] = hi ? Wrow[j] + V : V;
+                for (int jj = 0; jj < 8; ++jj) {
+                    const int j = 8 * jb + jj;
+                    const int64_t p0 = v[2 * jj], p1 = v[2 * jj + 1], p2 = v[16 + 2 * jj], p3 = v[16 + 2 * jj + 1];
+                    const int64_t p4 = v[32 + 2 * jj], p5 = v[32 + 2 * jj + 1];
+                    double H, L;
+                    if (!odd) {
+                        // row plane 0 (top digit, signed as b3 - 128) and row plane 2
+                        const int64_t q33 = p0 - 128 * (Si0 + M.colsum[0][j]) + 16384 * Krows;
+                        const int64_t q32 = p1 - 128 * (int64_t)M.colsum[1][j];
+                        const int64_t q31 = p2 - 128 * (int64_t)M.colsum[2][j];
+                        const int64_t q30 = p3 - 128 * (int64_t)M.colsum[3][j];
+                        H = (double)(q33 * (1ll << 24) + q32 * (1ll << 16) + q31 * (1ll << 8) + q30) * 0x1p24 +
+                            (double)(p4 * (1ll << 8) + p5) * 0x1p8;
+                        L = (double)(q31 * (1ll << 8) + q30) * 0x1p24;
+                    } else {
+                        // row plane 1 and row plane 3
+                        const int64_t q23 = p0 - 128 * Si1;
+                        H = (double)(q23 * (1ll << 24) + p1 * (1ll << 16) + p2 * (1ll << 8) + p3) * 0x1p16 +
+                            (double)(p4 * (1ll << 8) + p5);
+                        L = (double)(p2 * (1ll << 8) + p3) * 0x1p16;
                     }
+                    const double V = j > i ? H : (j < i ? L : H + L);
+                    const double Vo = __shfl_xor_sync(0xffffffffu, V, 1);
+                    Wv[jj] = odd ? Vo + V : V + Vo;
                 }
+                // the even lane stores j = 8jb .. 8jb + 3, the odd lane 8jb + 4 .. 8jb + 7
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj) Wrow[8 * jb + 4 * odd + jj] = odd ? Wv[4 + jj] : Wv[jj];
             }
             tc::fence_before_sync();
             __syncwarp();
             if (lane == 0) mbar_arrive1(&s.acc_empty);   // the next item's MMAs may overwrite D
             tc::named_sync(2, 32 * kI8EpiWarps);
-            // packed upper triangle: G_ab = 2^(E_a + E_b - 62) (W_ab + W_ba)
-            double* dst = nch > 1 ? a.partial + (int64_t)w.slot * TRI : s.G;
+            // the item's Gram, packed upper triangle: G_ab = 2^(E_a + E_b - 62) (W_ab + W_ba)
+            double* dst = a.gram + (int64_t)w.slot * TRI;
             for (int ra = 0; ra < RT; ++ra) {
                 const int cb = ra + et;
-                if (cb < RT) {
-                    double gv = 0.0;
-                    if (ra < r && cb < r) {
-                        gv = ra == cb ? s.W[ra * kI8LdS + ra] : s.W[ra * kI8LdS + cb] + s.W[cb * kI8LdS + ra];
-                        // times 2^(E_a + E_b - 62), exact (E in [-96, 127])
-                        gv *= __longlong_as_double((long long)(M.E[ra] + M.E[cb] - 62 + 1023) << 52);
-                    }
-                    dst[tri_off<RT>(ra, cb)] = gv;
+                if (cb >= RT) continue;
+                double gv = 0.0;
+                if (cb < r) {
+                    gv = ra == cb ? s.W[ra * kI8LdS + ra] : s.W[ra * kI8LdS + cb] + s.W[cb * kI8LdS + ra];
+                    // times 2^(E_a + E_b - 62), exact (E in [-96, 127])
+                    gv *= __longlong_as_double((long long)(M.E[ra] + M.E[cb] - 62 + 1023) << 52);
                 }
+                dst[tri_off<RT>(ra, cb)] = gv;
             }
-            const int ovf = M.ovf;
+            if (et == 0 && M.ovf) atomicExch(&a.fb[mf], 1);
             __syncwarp();
             if (lane == 0) mbar_arrive1(&s.meta_empty[ms]);
-            bool redo;
-            if (nch > 1) {
-                __threadfence();
-                tc::named_sync(2, 32 * kI8EpiWarps);
-                if (et == 0) {
-                    if (ovf) atomicExch(&a.fb[mf], 1);
-                    __threadfence();
-                    s.flag = atomicAdd(&a.counters[mf], 1) == nch - 1;
-                    if (s.flag) {
-                        __threadfence();
-                        s.redo = __ldcg(&a.fb[mf]) != 0;   // any item of the matrix overflowed
-                    }
-                }
-                tc::named_sync(2, 32 * kI8EpiWarps);
-                if (!s.flag) continue;   // uniform: another CTA merges this matrix
-                redo = s.redo != 0;
-                __threadfence();
-                const double* P0 = a.partial + (int64_t)a.info[mf].slot0 * TRI;
-                for (int e = et; !redo && e < TRI; e += 32 * kI8EpiWarps) {
-                    double acc = __ldcg(P0 + e);
-                    for (int cI = 1; cI < nch; ++cI) acc += __ldcg(P0 + (int64_t)cI * TRI + e);
-                    s.G[e] = acc;
-                }
-            } else {
-                if (ovf && et == 0) a.fb[mf] = 1;
-                redo = ovf != 0;
-            }
-            tc::named_sync(2, 32 * kI8EpiWarps);
-            if (redo) continue;   // uniform: the fp64 leaf factors this matrix
-            const bool good = i8_cholesky<RT>(s.G, s.diag, s.kc, r, et);
-            if (!good) {
-                if (et == 0) a.flags[mf] = 1;   // near-dependent columns: Householder TSQR
-                continue;
-            }
-            float* out = (factor == 0 ? a.R_B : a.R_A) + (size_t)(mf >> 1) * a.rs * a.rs;
-            for (int e = et; e < a.rs * a.rs; e += 32 * kI8EpiWarps) {
-                const int jr = e / a.rs, jc = e % a.rs;
-                out[e] = (jr < r && jc < r && jc >= jr) ? (float)s.G[tri_off<RT>(jr, jc)] : 0.f;
-            }
+            tc::named_sync(2, 32 * kI8EpiWarps);   // W is rewritten by the next item
         }
     }
     tc::fence_before_sync();
     __syncthreads();
     if (warp == 1) tc::tmem_dealloc(tmem, kI8TmemCols);
+}
+
+// Root of the integer-Gram leaf: one warp per matrix (2 * module + factor).  The
+// matrix's item Grams are summed in item order, then the fp64 Cholesky gives R (fp32
+// output, zero past r); a rejected pivot marks the matrix for the Householder TSQR.
+// Matrices the fp64 leaf takes (fb) are skipped.
+struct GramI8RootArgs {
+    const lf_module* mods;
+    const TsqrInfo* info;      // per mf: item count and first slot
+    const double* gram;
+    const int32_t* fb;
+    int32_t* flags;
+    float* R_B;
+    float* R_A;
+    int32_t rs, n_mf;
+};
+constexpr int kI8RootWarps = 4;
+
+template <int RT>
+constexpr size_t gram_i8_root_smem() { return (size_t)kI8RootWarps * (tri_size<RT>() + RT) * sizeof(double); }
+
+template <int RT>
+__global__ void __launch_bounds__(32 * kI8RootWarps) gram_i8_root_kernel(GramI8RootArgs a) {
+    constexpr int TRI = tri_size<RT>();
+    extern __shared__ double root_sm[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    double* Gw = root_sm + (size_t)warp * (TRI + RT);
+    double* dg = Gw + TRI;
+    const int mf = blockIdx.x * kI8RootWarps + warp;
+    if (mf >= a.n_mf) return;
+    if (a.fb[mf]) return;   // warp-uniform
+    const TsqrInfo inf = a.info[mf];
+    const double* P0 = a.gram + (int64_t)inf.slot0 * TRI;
+    for (int e = lane; e < TRI; e += 32) {
+        double acc = P0[e];
+        for (int c = 1; c < inf.nchunks; ++c) acc += P0[(int64_t)c * TRI + e];
+        Gw[e] = acc;
+    }
+    __syncwarp();
+    const int r = a.mods[mf >> 1].r;
+    if (!gram_cholesky<RT>(Gw, dg, r, lane)) {
+        if (lane == 0) a.flags[mf] = 1;   // near-dependent columns: Householder TSQR
+        return;
+    }
+    float* out = ((mf & 1) == 0 ? a.R_B : a.R_A) + (size_t)(mf >> 1) * a.rs * a.rs;
+    for (int e = lane; e < a.rs * a.rs; e += 32) {
+        const int jr = e / a.rs, jc = e % a.rs;
+        out[e] = (jr < r && jc < r && jc >= jr) ? (float)Gw[tri_off<RT>(jr, jc)] : 0.f;
+    }
 }
 
 }  // namespace lf

@@ -159,9 +159,10 @@ static void plan_tsqr(const lf_module* mods, int32_t n, TsqrPlan& p) {
                      [](const TsqrWork& a, const TsqrWork& b) { return a.nrows > b.nrows; });
 }
 
-// Work list of the integer-Gram leaf: every matrix whose rows the bulk copies can
-// address (16-byte aligned rows and offsets) in items of at most kI8MaxRows rows,
-// longest first; fb (per matrix) starts at 1 for the others, which the fp64 leaf takes.
+// Work list of the integer-Gram leaf: every matrix whose rows the copies can address
+// (16-byte aligned rows and offsets) in items of at most kI8MaxRows rows, longest first;
+// each item has its own Gram slot, a matrix's slots consecutive in row order.  fb (per
+// matrix) starts at 1 for the others, which the fp64 leaf takes.
 struct I8Plan {
     std::vector<TsqrWork> work;
     std::vector<TsqrInfo> info;
@@ -184,12 +185,11 @@ static void plan_i8(const lf_module* mods, int32_t n, I8Plan& p) {
             const int rows = f == 0 ? mods[i].d_out : mods[i].d_in;
             const int nch = (int)cdiv(rows, kI8MaxRows);
             const int mf = 2 * i + f;
-            p.info[mf] = TsqrInfo{nch, nch > 1 ? p.slots : -1};
+            p.info[mf] = TsqrInfo{nch, p.slots};
             p.fb[mf] = 0;
             for (int c = 0; c < nch; ++c)
-                p.work.push_back(TsqrWork{mf, c * kI8MaxRows, std::min(kI8MaxRows, rows - c * kI8MaxRows),
-                                          nch > 1 ? p.slots + c : -1});
-            if (nch > 1) p.slots += nch;
+                p.work.push_back(TsqrWork{mf, c * kI8MaxRows, std::min(kI8MaxRows, rows - c * kI8MaxRows), p.slots + c});
+            p.slots += nch;
         }
     std::stable_sort(p.work.begin(), p.work.end(),
                      [](const TsqrWork& a, const TsqrWork& b) { return a.nrows > b.nrows; });
@@ -200,7 +200,7 @@ static size_t i8_slot_bytes(int RT) {
 }
 
 struct TsqrLayout {
-    size_t mods, work, nwork, info, n_dev, counters, partial, i8work, i8info, fb, i8partial, total;
+    size_t mods, work, nwork, info, n_dev, counters, partial, i8work, i8info, fb, amaps, i8gram, total;
 };
 
 // Partial-slot bytes: the fp64 packed Gram of the leaf pass or the fp32 partial R of
@@ -222,13 +222,13 @@ static TsqrLayout tsqr_layout(int32_t n, const TsqrPlan& p, const I8Plan& q) {
     LF_TAKE(nwork, int32_t, 1);
     LF_TAKE(info, TsqrInfo, p.info.size());
     LF_TAKE(n_dev, int32_t, 1);
-    // Gram counters, Householder counters, flags, integer-Gram counters (2n each)
-    LF_TAKE(counters, int32_t, (size_t)8 * n);
+    LF_TAKE(counters, int32_t, (size_t)6 * n);   // Gram counters, Householder counters, flags (2n each)
     LF_TAKE(partial, char, (size_t)p.slots * tsqr_slot_bytes(p.RT));
     LF_TAKE(i8work, TsqrWork, q.work.size());
     LF_TAKE(i8info, TsqrInfo, q.info.size());
     LF_TAKE(fb, int32_t, q.fb.size());
-    LF_TAKE(i8partial, char, (size_t)q.slots * i8_slot_bytes(p.RT));
+    LF_TAKE(amaps, CUtensorMap, (size_t)n);
+    LF_TAKE(i8gram, char, (size_t)q.slots * i8_slot_bytes(p.RT));
 #undef LF_TAKE
     L.total = c.off + 256;
     return L;
@@ -246,24 +246,33 @@ static cudaError_t launch_tsqr(const TsqrArgs<T>& a, int n_items, cudaStream_t s
 }
 
 template <int RT>
-static cudaError_t launch_gram_i8(const GramI8Args& a, cudaStream_t st) {
-    if (a.n_work <= 0) return cudaSuccess;
-    int dev = 0, sms = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+static cudaError_t launch_gram_i8(const GramI8Args& a, const GramI8RootArgs& ra, cudaStream_t st) {
+    if (a.n_work > 0) {
+        int dev = 0, sms = 0;
+        cudaError_t e = cudaGetDevice(&dev);
+        if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(gram_i8_kernel<RT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gram_i8_smem());
+        if (e != cudaSuccess) return e;
+        // one persistent CTA per SM (all of its tensor memory), static round-robin over the items
+        const int grid = std::min(a.n_work, std::max(sms, 1));
+        LF_LAUNCH("tsqr_gram_i8", gram_i8_kernel<RT>, grid, kI8Threads, gram_i8_smem(), st, a);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    constexpr size_t rsm = gram_i8_root_smem<RT>();
+    cudaError_t e = cudaFuncSetAttribute(gram_i8_root_kernel<RT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rsm);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(gram_i8_kernel<RT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gram_i8_smem());
-    if (e != cudaSuccess) return e;
-    // one persistent CTA per SM (all of its tensor memory), static round-robin over the items
-    const int grid = std::min(a.n_work, std::max(sms, 1));
-    LF_LAUNCH("tsqr_gram_i8", gram_i8_kernel<RT>, grid, kI8Threads, gram_i8_smem(), st, a);
+    if (ra.n_mf > 0)
+        LF_LAUNCH("tsqr_gram_i8_root", gram_i8_root_kernel<RT>, (unsigned)cdiv(ra.n_mf, kI8RootWarps),
+                  32 * kI8RootWarps, rsm, st, ra);
     return cudaGetLastError();
 }
 
-static cudaError_t launch_gram_i8_rt(int RT, const GramI8Args& a, cudaStream_t st) {
-    if (RT == 16) return launch_gram_i8<16>(a, st);
-    if (RT == 32) return launch_gram_i8<32>(a, st);
-    return launch_gram_i8<64>(a, st);
+static cudaError_t launch_gram_i8_rt(int RT, const GramI8Args& a, const GramI8RootArgs& ra, cudaStream_t st) {
+    if (RT == 16) return launch_gram_i8<16>(a, ra, st);
+    if (RT == 32) return launch_gram_i8<32>(a, ra, st);
+    return launch_gram_i8<64>(a, ra, st);
 }
 
 template <int RT>
@@ -474,6 +483,23 @@ static bool encode_rows_map(CUtensorMap* map, const void* base, int32_t rows, in
     const cuuint32_t box[2] = {(cuuint32_t)kTcKB, (cuuint32_t)kTcM};
     const cuuint32_t estr[2] = {1, 1};
     return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Tensor map of a module's A (r x d_in fp32, row-major) read as A^T stages: dims
+// {d_in, r}, box {32, r} (32 rows of A^T: one 128-byte run per column), 128-byte
+// swizzle, rows past d_in read as zeros.  False when the encoder is unavailable or
+// rejects the shape (the fp64 leaf then takes the matrix).
+static bool encode_a_map(CUtensorMap* map, const float* A, int32_t r, int32_t d_in) {
+    if (!aligned16(A) || (d_in & 3) || r < 1 || r > 64) return false;
+    const EncodeTiledFn fn = encode_tiled_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)d_in, (cuuint64_t)r};
+    const cuuint64_t strides[1] = {(cuuint64_t)d_in * 4};
+    const cuuint32_t box[2] = {32u, (cuuint32_t)r};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(A), dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -963,36 +989,57 @@ lf_status lf_tsqr_batched(const lf_module* mods, int32_t n, const float* B_base,
     h.put(p.info.data(), p.info.size());
     h.put(&n, 1);
     LF_CUDA_TRY(cudaMemcpyAsync(base, h.buf.data(), h.off, cudaMemcpyHostToDevice, s));
-    LF_CUDA_TRY(cudaMemsetAsync(base + L.counters, 0, (size_t)8 * n * sizeof(int32_t), s));
+    LF_CUDA_TRY(cudaMemsetAsync(base + L.counters, 0, (size_t)6 * n * sizeof(int32_t), s));
+    // tensor maps of the A factors the integer leaf reads (a matrix whose map the encoder
+    // rejects goes to the fp64 leaf with its items skipped)
+    std::vector<CUtensorMap> amaps((size_t)n);
+    std::vector<char> keep((size_t)2 * n, 1);
+    for (int32_t i = 0; i < n; ++i) {
+        std::memset(&amaps[i], 0, sizeof(CUtensorMap));
+        if (q.fb[2 * i + 1] == 0 && !encode_a_map(&amaps[i], A_base + mods[i].A_off, mods[i].r, mods[i].d_in)) {
+            q.fb[2 * i + 1] = 1;
+            keep[2 * i + 1] = 0;
+        }
+    }
+    std::vector<TsqrWork> work8;   // the items kept, then unused room up to the planned count
+    work8.reserve(q.work.size());
+    for (const TsqrWork& w : q.work)
+        if (keep[w.mf]) work8.push_back(w);
+    const int32_t n_work8 = (int32_t)work8.size();
+    work8.resize(q.work.size(), TsqrWork{0, 0, 0, 0});
     Staging h8;   // the integer-Gram tables sit after the partial slots
-    h8.put(q.work.data(), q.work.size());
+    h8.put(work8.data(), work8.size());
     h8.put(q.info.data(), q.info.size());
     h8.put(q.fb.data(), q.fb.size());
+    h8.put(amaps.data(), amaps.size());
     LF_CUDA_TRY(cudaMemcpyAsync(base + L.i8work, h8.buf.data(), h8.off, cudaMemcpyHostToDevice, s));
     int32_t* gram_counters = reinterpret_cast<int32_t*>(base + L.counters);
     int32_t* hh_counters = gram_counters + 2 * n;
     int32_t* flags = gram_counters + 4 * n;
-    int32_t* i8_counters = gram_counters + 6 * n;
     int32_t* fb = reinterpret_cast<int32_t*>(base + L.fb);
 
-    // integer Gram on the tensor cores for every addressable matrix; a matrix it leaves
-    // (unaddressable rows, a value past its column scale, a non-finite value) is marked
-    // in fb and factored by the fp64 Gram leaf below
+    // integer Gram on the tensor cores for every addressable matrix, then its root (sum of
+    // the item Grams, fp64 Cholesky); a matrix it leaves (unaddressable rows, a value past
+    // its column scale, a non-finite value) is marked in fb for the fp64 Gram leaf below
     GramI8Args ia;
     ia.mods = reinterpret_cast<const lf_module*>(base + L.mods);
     ia.B_base = B_base;
-    ia.A_base = A_base;
+    ia.amaps = reinterpret_cast<const CUtensorMap*>(base + L.amaps);
     ia.work = reinterpret_cast<const TsqrWork*>(base + L.i8work);
-    ia.n_work = (int32_t)q.work.size();
-    ia.info = reinterpret_cast<const TsqrInfo*>(base + L.i8info);
-    ia.counters = i8_counters;
-    ia.partial = reinterpret_cast<double*>(base + L.i8partial);
+    ia.n_work = n_work8;
+    ia.gram = reinterpret_cast<double*>(base + L.i8gram);
     ia.fb = fb;
-    ia.flags = flags;
-    ia.R_B = R_B;
-    ia.R_A = R_A;
-    ia.rs = p.rs;
-    LF_CUDA_TRY(launch_gram_i8_rt(p.RT, ia, s));
+    GramI8RootArgs ra;
+    ra.mods = ia.mods;
+    ra.info = reinterpret_cast<const TsqrInfo*>(base + L.i8info);
+    ra.gram = ia.gram;
+    ra.fb = fb;
+    ra.flags = flags;
+    ra.R_B = R_B;
+    ra.R_A = R_A;
+    ra.rs = p.rs;
+    ra.n_mf = 2 * n;
+    LF_CUDA_TRY(launch_gram_i8_rt(p.RT, ia, ra, s));
 
     GramArgs ga;
     ga.mods = reinterpret_cast<const lf_module*>(base + L.mods);
