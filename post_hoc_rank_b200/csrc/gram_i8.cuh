@@ -33,9 +33,10 @@
 //                 [P0;P1;P2;P3]^T (M 128, N 256) and D2 += [P2;P3] x [P2;P3]^T (M 128,
 //                 N 128) in four K = 32 steps each, into 384 TMEM columns (plane p =
 //                 byte 3 - p);
-//   warps 2..9    converters: column scales, fp32 -> digit planes (K-major, 128-byte
-//                 swizzle) and the planes' column sums;
-//   warps 10..13  epilogue: int32 accumulators -> signed-digit corrections -> the
+//   warps 2..17   converters: column scales, fp32 -> digit planes (K-major, 128-byte
+//                 swizzle) and the planes' column sums, one 16-row chunk of one
+//                 column per thread and digit stage;
+//   warps 18..21  epilogue: int32 accumulators -> signed-digit corrections -> the
 //                 item's fp64 Gram (packed upper triangle) in its own global slot.
 // Operand rows interleave the planes of a column (row 2c: plane 0 or 2 of column c,
 // row 2c + 1: plane 1 or 3), so both planes of column c sit in adjacent TMEM lanes of
@@ -56,11 +57,11 @@ constexpr int kI8Rows = 128;         // rows (the MMA's K) per digit stage
 constexpr int kI8FRows = 64;         // rows per fp32 stage (two per digit stage)
 constexpr int kI8FStages = 7;
 constexpr int kI8DStages = 2;
-constexpr int kI8ConvWarps = 8;
+constexpr int kI8ConvWarps = 16;
 constexpr int kI8EpiWarps = 4;
 constexpr int kI8ConvWarp0 = 2;
-constexpr int kI8EpiWarp0 = kI8ConvWarp0 + kI8ConvWarps;       // 10
-constexpr int kI8Threads = 32 * (kI8EpiWarp0 + kI8EpiWarps);   // 448
+constexpr int kI8EpiWarp0 = kI8ConvWarp0 + kI8ConvWarps;       // 18
+constexpr int kI8Threads = 32 * (kI8EpiWarp0 + kI8EpiWarps);   // 704
 constexpr int kI8HeadBits = 2;       // 2^E is 4x to 8x the largest value of the first 128 rows
 // Rows per work item: the largest accumulator, 255^2 * rows, stays below 2^31, and the
 // corrected top-digit product times 2^24 stays below 2^53 (exact in fp64).
@@ -81,7 +82,7 @@ struct GramI8Smem {
     float f32[kI8FStages][kI8FStageFloats]; // 1024-aligned (128-byte swizzle atoms of the A^T stages)
     double W[64 * kI8LdS];                  // fp64 row i of the column pair (i, j) sums
     GramI8Meta meta[2];
-    float cmax[4][64];
+    float cmax[8][64];
     uint64_t full_f[kI8FStages], empty_f[kI8FStages];
     uint64_t full_d[kI8DStages], empty_d[kI8DStages];
     uint64_t acc_full, acc_empty, drain;
@@ -312,11 +313,11 @@ __global__ void __launch_bounds__(kI8Threads, 1) gram_i8_kernel(GramI8Args a) {
             ok = named_and(1, 32 * kI8ConvWarps, ok);
             if (!ok) break;
             GramI8Meta& M = s.meta[ms];
-            // this thread's column and its two 16-row chunks (q0 and q0 + 4) of every
-            // digit stage: B stages are read across columns (one row per load), A^T
-            // stages across 8 columns of one chunk (16-byte loads, distinct swizzled chunks)
-            const int c = factor == 0 ? 32 * (cw & 1) + lane : 8 * cw + (lane & 7);
-            const int q0 = factor == 0 ? (cw >> 1) : (lane >> 3);
+            // this thread's column c and 16-row chunk q of every digit stage (chunk q in
+            // fp32 stage q >> 2): B stages are read across columns (one row per load),
+            // A^T stages across 8 columns of one chunk (16-byte loads, distinct swizzled chunks)
+            const int c = factor == 0 ? 32 * (cw & 1) + lane : 8 * (cw & 7) + (lane & 7);
+            const int q = factor == 0 ? (cw >> 1) : (lane >> 3) + 4 * (cw >> 3);
             for (int e = ct; e < 4 * 64; e += 32 * kI8ConvWarps) (&M.colsum[0][0])[e] = 0;
             if (ct == 0) M.ovf = 0;
             uint32_t cs[4] = {0u, 0u, 0u, 0u};
@@ -329,11 +330,10 @@ __global__ void __launch_bounds__(kI8Threads, 1) gram_i8_kernel(GramI8Args a) {
                 ok = named_and(1, 32 * kI8ConvWarps, ok);
                 if (!ok) break;
                 const int rbase = kI8Rows * ds;
-                // this thread's two 16-row chunks into registers, then the fp32 stages go
-                // back to the producer before any conversion work
-                float xv[2][16];
-                i8_load_unit(xv[0], s.f32[f0], factor, c, q0, r, w.nrows - rbase - 16 * q0);
-                i8_load_unit(xv[1], s.f32[f1], factor, c, q0, r, w.nrows - rbase - 16 * (q0 + 4));
+                // this thread's chunk into registers, then the fp32 stages go back to the
+                // producer before any conversion work
+                float xv[16];
+                i8_load_unit(xv, s.f32[q < 4 ? f0 : f1], factor, c, q & 3, r, w.nrows - rbase - 16 * q);
                 __syncwarp();
                 if (lane == 0) {
                     mbar_arrive1(&s.empty_f[f0]);
@@ -343,12 +343,12 @@ __global__ void __launch_bounds__(kI8Threads, 1) gram_i8_kernel(GramI8Args a) {
                     // column exponents from the item's first 128 rows
                     float mx = 0.f;
 #pragma unroll
-                    for (int h = 0; h < 2; ++h)
-#pragma unroll
-                        for (int e = 0; e < 16; ++e) mx = fmaxf(mx, fabsf(xv[h][e]));
-                    s.cmax[q0][c] = mx;
+                    for (int e = 0; e < 16; ++e) mx = fmaxf(mx, fabsf(xv[e]));
+                    s.cmax[q][c] = mx;
                     tc::named_sync(1, 32 * kI8ConvWarps);
-                    const float m = fmaxf(fmaxf(s.cmax[0][c], s.cmax[1][c]), fmaxf(s.cmax[2][c], s.cmax[3][c]));
+                    float m = s.cmax[0][c];
+#pragma unroll
+                    for (int h = 1; h < 8; ++h) m = fmaxf(m, s.cmax[h][c]);
                     int E = -90;   // an all-zero start: any nonzero value later overflows the scale
                     if (m > 0.f && m <= FLT_MAX) {
                         int e2;
@@ -361,40 +361,46 @@ __global__ void __launch_bounds__(kI8Threads, 1) gram_i8_kernel(GramI8Args a) {
                     }
                     mult = __int_as_float((158 - E) << 23);   // 2^(31 - E)
                     lim = __int_as_float((127 + E) << 23);    // 2^E
-                    if (q0 == 0) M.E[c] = E;
+                    if (q == 0) M.E[c] = E;
                     tc::named_sync(1, 32 * kI8ConvWarps);     // cmax is rewritten by the next item
                 }
                 if (gd >= kI8DStages) ok = wait(&s.empty_d[gd % kI8DStages], (uint32_t)((gd / kI8DStages - 1) & 1));
                 ok = named_and(1, 32 * kI8ConvWarps, ok);
                 if (!ok) break;
                 uint8_t* dig = s.dig[gd % kI8DStages];
+                uint32_t pw[4][4];
+                float amax = 0.f;
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const int q = q0 + 4 * h;   // chunk: rows 16q .. 16q + 15 of the digit stage
-                    uint32_t pw[4][4];
+                for (int j4 = 0; j4 < 4; ++j4) {
+                    uint32_t u[4];
 #pragma unroll
-                    for (int j4 = 0; j4 < 4; ++j4) {
-                        uint32_t u[4];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const float x = xv[h][4 * j4 + e];
-                            vok = vok && fabsf(x) < lim;   // false for NaN as well
-                            u[e] = (uint32_t)__float2int_rz(x * mult) ^ 0x80000000u;
-                        }
-                        uint32_t wd[4];
-                        planes4(u, wd);
-#pragma unroll
-                        for (int p = 0; p < 4; ++p) {
-                            pw[p][j4] = wd[p];
-                            cs[p] = __dp4a(wd[p], 0x01010101u, cs[p]);
-                        }
+                    for (int e = 0; e < 4; ++e) {
+                        const float x = xv[4 * j4 + e];
+                        amax = fmaxf(amax, fabsf(x));
+                        vok = vok && (x == x);   // NaN: fmaxf would drop it
+                        u[e] = (uint32_t)__float2int_rz(x * mult);
                     }
+                    uint32_t wd[4];
+                    planes4(u, wd);
+                    wd[0] ^= 0x80808080u;   // U = N + 2^31: the top byte's top bit, four rows at once
 #pragma unroll
                     for (int p = 0; p < 4; ++p) {
-                        const int R = i8_row(p, c);   // operand row, 128 bytes
-                        *reinterpret_cast<uint4*>(dig + R * 128 + ((q ^ (R & 7)) << 4)) =
-                            make_uint4(pw[p][0], pw[p][1], pw[p][2], pw[p][3]);
+                        pw[p][j4] = wd[p];
+                        cs[p] = __dp4a(wd[p], 0x01010101u, cs[p]);
                     }
+                }
+                vok = vok && amax < lim;   // false for infinities as well
+                // lanes 4..7 of each group of 8 (consecutive columns) store the other plane of
+                // the pair (0 <-> 1, 2 <-> 3) than lanes 0..3, so the eight 16-byte stores of a
+                // group land in eight different swizzled chunks (no bank conflict)
+                const int flip = (lane >> 2) & 1;
+#pragma unroll
+                for (int t = 0; t < 4; ++t) {
+                    const int p = t ^ flip;
+                    const int R = i8_row(p, c);   // operand row, 128 bytes
+                    const uint4 val = flip ? make_uint4(pw[t ^ 1][0], pw[t ^ 1][1], pw[t ^ 1][2], pw[t ^ 1][3])
+                                           : make_uint4(pw[t][0], pw[t][1], pw[t][2], pw[t][3]);
+                    *reinterpret_cast<uint4*>(dig + R * 128 + ((q ^ (R & 7)) << 4)) = val;
                 }
                 tc::fence_proxy_async();   // the digit planes, to the tensor core's proxy
                 __syncwarp();

@@ -66,9 +66,31 @@ __device__ int64_t count_ge(const SelArgs& a, int m0, int M, double t, int64_t* 
     return block_sum_i64(c, red);
 }
 
+// largest candidate energy (j >= floor, e > 0) strictly below t, 0 if there is none
+__device__ double max_below(const SelArgs& a, int m0, int M, double t, double* dred) {
+    double b = 0.0;
+    const int fl = a.pol.floor;
+    for (int q = threadIdx.x; q < M * a.rs; q += blockDim.x) {
+        const int mi = q / a.rs, j = q % a.rs;
+        const int i = a.grp_mods[m0 + mi];
+        if (j < fl || j >= a.mods[i].r) continue;
+        const double e = a.energy[(size_t)i * a.rs + j];
+        if (e > 0.0 && e < t) b = fmax(b, e);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) b = fmax(b, __shfl_xor_sync(0xffffffffu, b, o));
+    __syncthreads();
+    if ((threadIdx.x & 31) == 0) dred[threadIdx.x >> 5] = b;
+    __syncthreads();
+    double m = 0.0;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) m = fmax(m, dred[w]);
+    return m;
+}
+
 __global__ void __launch_bounds__(kSelThreads) select_kernel(SelArgs a) {
     __shared__ int64_t red[32];
-    __shared__ int64_t s_take_eq;
+    __shared__ double dred[32];
+    __shared__ int64_t s_take_eq, s_n_eq;
     __shared__ double s_theta;
     const int g = blockIdx.x;
     const int m0 = a.grp_ptr[g], m1 = a.grp_ptr[g + 1], M = m1 - m0;
@@ -150,7 +172,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelArgs a) {
     const double tiny = __longlong_as_double(1ll);
     const int64_t npos = count_ge(a, m0, M, tiny, red);
     double theta;
-    int64_t take_eq;
+    int64_t take_eq, n_eq = 0;
     if (npos <= extra) {
         theta = tiny;  // take every positive candidate
         take_eq = INT64_MAX;
@@ -165,14 +187,17 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelArgs a) {
         theta = __longlong_as_double(lo);
         const int64_t n_gt = count_ge(a, m0, M, __longlong_as_double(lo + 1), red);
         take_eq = extra - n_gt;
+        if (a.flag_list) n_eq = count_ge(a, m0, M, theta, red) - n_gt;
     }
     if (threadIdx.x == 0) {
         s_theta = theta;
         s_take_eq = take_eq;
+        s_n_eq = n_eq;
     }
     __syncthreads();
     theta = s_theta;
     take_eq = s_take_eq;
+    n_eq = s_n_eq;
     // per module: all e > theta, then the first take_eq candidates equal to theta in
     // (module, j) order.  The equal-candidate prefix over modules is taken serially.
     if (threadIdx.x == 0) {
@@ -198,6 +223,14 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelArgs a) {
         }
     }
     if (a.flag_list && npos > extra) {
+        // The selection can differ from the exact one only if the boundary is a near tie:
+        // the last selected energy theta and the first one left out (a candidate equal to
+        // theta that the tie order leaves out, else the largest below theta) closer than
+        // twice the band, the band being far above the main path's energy error.  Then
+        // the modules holding a candidate within the band of theta are refined in fp64.
+        const double below = max_below(a, m0, M, theta, dred);
+        const bool tie_out = n_eq > take_eq;
+        if (!tie_out && theta - below > 2.0 * a.band * theta) return;
         for (int mi = threadIdx.x; mi < M; mi += blockDim.x) {
             const int i = a.grp_mods[m0 + mi];
             const int r = a.mods[i].r;
@@ -205,7 +238,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelArgs a) {
             bool f = false;
             for (int j = fl; j < r; ++j) {
                 const double e = en[j];
-                if (e > 0.0 && fabs(e - theta) <= a.band * theta) f = true;
+                if (e > 0.0 && fabs(e - theta) <= 2.0 * a.band * theta) f = true;
             }
             if (f) {
                 const int slot = atomicAdd(a.flag_count, 1);
