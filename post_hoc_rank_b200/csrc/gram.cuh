@@ -172,23 +172,43 @@ __device__ __forceinline__ bool gram_cholesky(double* G, double* s_diag, int r, 
     for (int j = lane; j < r; j += 32) s_diag[j] = G[tri_off<RT>(j, j)];
     __syncwarp();
     for (int j = 0; j < r; ++j) {
-        const double d = G[tri_off<RT>(j, j)];
+        const int dj = tri_off<RT>(j, j);
+        const double d = G[dj];
         if (!(d > kGramPivotTol * s_diag[j])) return false;
         const double rjj = sqrt(d);
+        const double inv = 1.0 / rjj;   // one division per step; the row is scaled by it
         __syncwarp();
 #pragma unroll
         for (int s = 0; s < C::NS; ++s) {
             const int c = C::col(lane, s);
-            if (c > j && c < r) G[tri_off<RT>(j, c)] /= rjj;
+            if (c > j && c < r) G[dj + (c - j)] *= inv;
         }
-        if (lane == 0) G[tri_off<RT>(j, j)] = rjj;
+        if (lane == 0) G[dj] = rjj;
         __syncwarp();
+        const double* rowj = G + (dj - j);   // rowj[k] = R_jk
 #pragma unroll
         for (int s = 0; s < C::NS; ++s) {
             const int c = C::col(lane, s);
             if (c > j && c < r) {
-                const double gjc = G[tri_off<RT>(j, c)];
-                for (int k = j + 1; k <= c; ++k) G[tri_off<RT>(k, c)] -= G[tri_off<RT>(j, k)] * gjc;
+                const double gjc = rowj[c];
+                // column c, rows k = j+1..c; the packed offset of (k, c) grows by RT - k - 1
+                // from k to k + 1.  Four rows per pass: loads first, then the stores.
+                int k = j + 1;
+                int p = tri_off<RT>(k, c);
+                for (; k + 3 <= c; k += 4) {
+                    const int p1 = p + (RT - k - 1), p2 = p1 + (RT - k - 2), p3 = p2 + (RT - k - 3);
+                    const double a0 = rowj[k], a1 = rowj[k + 1], a2 = rowj[k + 2], a3 = rowj[k + 3];
+                    const double g0 = G[p], g1 = G[p1], g2 = G[p2], g3 = G[p3];
+                    G[p] = g0 - a0 * gjc;
+                    G[p1] = g1 - a1 * gjc;
+                    G[p2] = g2 - a2 * gjc;
+                    G[p3] = g3 - a3 * gjc;
+                    p = p3 + (RT - k - 4);
+                }
+                for (; k <= c; ++k) {
+                    G[p] -= rowj[k] * gjc;
+                    p += RT - k - 1;
+                }
             }
         }
         __syncwarp();

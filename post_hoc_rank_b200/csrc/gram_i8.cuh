@@ -547,9 +547,10 @@ __global__ void __launch_bounds__(32 * kI8RootWarps) gram_i8_root_kernel(GramI8R
         return;
     }
     float* out = ((mf & 1) == 0 ? a.R_B : a.R_A) + (size_t)(mf >> 1) * a.rs * a.rs;
-    for (int e = lane; e < a.rs * a.rs; e += 32) {
-        const int jr = e / a.rs, jc = e % a.rs;
-        out[e] = (jr < r && jc < r && jc >= jr) ? (float)Gw[tri_off<RT>(jr, jc)] : 0.f;
+    for (int jr = 0; jr < a.rs; ++jr) {   // row jr of R: columns jr..r-1 of the packed row, zero elsewhere
+        const double* gr = Gw + (tri_off<RT>(jr, jr) - jr);
+        for (int jc = lane; jc < a.rs; jc += 32)
+            out[(size_t)jr * a.rs + jc] = (jr < r && jc < r && jc >= jr) ? (float)gr[jc] : 0.f;
     }
 }
 

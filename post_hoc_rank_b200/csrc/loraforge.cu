@@ -333,11 +333,12 @@ static void build_groups(const lf_module* mods, int32_t n, std::vector<int32_t>&
 }
 
 // ----------------------------------------------------------- export planning
-constexpr int kRefineChunk = 1024;
+constexpr int kRefineChunk = 512;
 constexpr int kExportItem = 2048;
 
 struct ExportPlan {
     std::vector<int32_t> gptr, gmods;
+    int32_t max_cand = 0;   // largest candidate count (sum of r - floor) over the groups
     std::vector<ExportWork> ework;
     int rs = 0, RT = 16;
     int32_t refine_cap = 0;
@@ -350,6 +351,12 @@ static void plan_export(const lf_module* mods, int32_t n, ExportPlan& p) {
     p.RT = rt_bucket(p.rs);
     build_groups(mods, n, p.gptr, p.gmods);
     const int32_t ngroups = (int32_t)p.gptr.size() - 1;
+    p.max_cand = 0;
+    for (int32_t g = 0; g < ngroups; ++g) {
+        int64_t c = 0;
+        for (int32_t q = p.gptr[g]; q < p.gptr[g + 1]; ++q) c += mods[p.gmods[q]].r;
+        p.max_cand = (int32_t)std::max<int64_t>(p.max_cand, std::min<int64_t>(c, kSelMaxCand));
+    }
     p.ework.clear();
     int maxd = 1;
     for (int32_t i = 0; i < n; ++i) {
@@ -359,10 +366,10 @@ static void plan_export(const lf_module* mods, int32_t n, ExportPlan& p) {
             p.ework.push_back(ExportWork{i, 1, s, std::min(kExportItem, mods[i].d_in - s)});
         maxd = std::max(maxd, std::max(mods[i].d_out, mods[i].d_in));
     }
-    p.refine_cap = std::min<int32_t>(n, 16 * ngroups + 64);
+    p.refine_cap = std::min<int32_t>(n, 8 * ngroups + 64);
     const int per = (int)cdiv(maxd, kRefineChunk);
     p.refine_max_work = p.refine_cap * 2 * per;
-    p.refine_slots = p.refine_cap * 2 * (per > 1 ? per : 0);
+    p.refine_slots = p.refine_cap * 2 * (per > 1 ? tree_slots(per) : 0);
 }
 
 struct ExportLayout {
@@ -390,8 +397,8 @@ static ExportLayout export_layout(int32_t n, const ExportPlan& p) {
     LF_TAKE(rwork, TsqrWork, (size_t)p.refine_max_work);
     LF_TAKE(rnwork, int32_t, 1);
     LF_TAKE(rinfo, TsqrInfo, (size_t)2 * p.refine_cap);
-    LF_TAKE(rcnt, int32_t, (size_t)2 * p.refine_cap);
-    LF_TAKE(rpart, double, (size_t)p.refine_slots * p.RT * p.RT);
+    LF_TAKE(rcnt, int32_t, (size_t)p.refine_slots);
+    LF_TAKE(rpart, double, (size_t)p.refine_slots * (p.RT * (p.RT + 1) / 2));
     LF_TAKE(rRB, double, (size_t)p.refine_cap * rs2);
     LF_TAKE(rRA, double, (size_t)p.refine_cap * rs2);
     LF_TAKE(rsig, double, (size_t)p.refine_cap * p.rs);
@@ -1074,6 +1081,7 @@ lf_status lf_tsqr_batched(const lf_module* mods, int32_t n, const float* B_base,
     ta.R_A = R_A;
     ta.rs = p.rs;
     ta.only = flags;
+    ta.tree = 0;
     LF_CUDA_TRY(launch_tsqr_rt<float>(p.RT, ta, nwork, s));
 
     SvdArgs<float, float> sa;
@@ -1101,6 +1109,17 @@ size_t lf_select_workspace_size(const lf_module* mods, int32_t n) {
     c.take<int32_t>(p.gmods.size());
     c.take<double>((size_t)n * p.rs);
     return c.off + 256;
+}
+
+// One selection CTA per group, with the group's candidate list in dynamic shared memory
+// when it fits (kSelMaxCand entries at most; larger groups count from global memory).
+static cudaError_t launch_select(SelArgs a, int ng, int32_t max_cand, cudaStream_t s) {
+    a.cand_cap = std::min(max_cand, kSelMaxCand);
+    const size_t smem = (size_t)a.cand_cap * sizeof(double);
+    cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    LF_LAUNCH("select", select_kernel, ng, kSelThreads, smem, s, a);
+    return cudaGetLastError();
 }
 
 lf_status lf_select_ranks(const lf_module* mods, int32_t n, lf_policy pol, const double* sigma, int32_t* ranks,
@@ -1136,8 +1155,7 @@ lf_status lf_select_ranks(const lf_module* mods, int32_t n, lf_policy pol, const
     a.flag_list = nullptr;
     a.flag_count = nullptr;
     const int ng = (int)p.gptr.size() - 1;
-    LF_LAUNCH("select", select_kernel, ng, kSelThreads, 0, s, a);
-    LF_CUDA_TRY(cudaGetLastError());
+    LF_CUDA_TRY(launch_select(a, ng, p.max_cand, s));
     LF_LAUNCH("offsets", offsets_kernel, 1, 1024, 0, s, a.mods, n, ranks, off_A, off_Bt, INT64_MAX, INT64_MAX);
     return launch_status();
 }
@@ -1245,8 +1263,7 @@ lf_status lf_truncate_export(const lf_module* mods, int32_t n, lf_policy pol, co
         LF_CUDA_TRY(cudaMemsetAsync(fcount, 0, 2 * sizeof(int32_t), s));
         a.flag_list = flist;
         a.flag_count = fcount;
-        LF_LAUNCH("select", select_kernel, ng, kSelThreads, 0, s, a);
-        LF_CUDA_TRY(cudaGetLastError());
+        LF_CUDA_TRY(launch_select(a, ng, p.max_cand, s));
         LF_LAUNCH("refine_plan", cap_flags_kernel, 1, 32, 0, s, fcount, p.refine_cap);
         LF_CUDA_TRY(cudaGetLastError());
         TsqrWork* rwork = reinterpret_cast<TsqrWork*>(base + L.rwork);
@@ -1254,7 +1271,8 @@ lf_status lf_truncate_export(const lf_module* mods, int32_t n, lf_policy pol, co
         TsqrInfo* rinfo = reinterpret_cast<TsqrInfo*>(base + L.rinfo);
         LF_LAUNCH("refine_plan", refine_plan_kernel, 1, 32, 0, s, dmods, flist, fcount, rwork, rnwork, rinfo, kRefineChunk);
         LF_CUDA_TRY(cudaGetLastError());
-        LF_CUDA_TRY(cudaMemsetAsync(base + L.rcnt, 0, (size_t)2 * p.refine_cap * sizeof(int32_t), s));
+        if (p.refine_slots > 0)
+            LF_CUDA_TRY(cudaMemsetAsync(base + L.rcnt, 0, (size_t)p.refine_slots * sizeof(int32_t), s));
         TsqrArgs<double> ta;
         ta.mods = dmods;
         ta.mod_ids = flist;
@@ -1269,6 +1287,7 @@ lf_status lf_truncate_export(const lf_module* mods, int32_t n, lf_policy pol, co
         ta.R_A = reinterpret_cast<double*>(base + L.rRA);
         ta.rs = p.rs;
         ta.only = nullptr;
+        ta.tree = 1;
         LF_CUDA_TRY(launch_tsqr_rt<double>(p.RT, ta, p.refine_max_work, s));
         SvdArgs<double, double> sa;
         sa.mods = dmods;
@@ -1290,8 +1309,7 @@ lf_status lf_truncate_export(const lf_module* mods, int32_t n, lf_policy pol, co
         a.flag_list = nullptr;
         a.flag_count = nullptr;
     }
-    LF_LAUNCH("select", select_kernel, ng, kSelThreads, 0, s, a);
-    LF_CUDA_TRY(cudaGetLastError());
+    LF_CUDA_TRY(launch_select(a, ng, p.max_cand, s));
     LF_LAUNCH("offsets", offsets_kernel, 1, 1024, 0, s, dmods, n, ranks, off_A, off_Bt, pool_cap_A, pool_cap_Bt);
     LF_CUDA_TRY(cudaGetLastError());
     float* CA = reinterpret_cast<float*>(base + L.CA);
@@ -1640,6 +1658,7 @@ lf_status lf_jd_full(const lf_module* mods, int32_t n_mods, const int32_t* membe
         ta.R_A = RA;
         ta.rs = P.orth.rs;
         ta.only = only;
+        ta.tree = 0;
         return launch_tsqr_rt<float>(P.orth.RT, ta, onwork, s);
     };
 

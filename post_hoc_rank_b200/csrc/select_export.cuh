@@ -19,7 +19,8 @@
 
 namespace lf {
 
-constexpr int kSelThreads = 256;
+constexpr int kSelThreads = 1024;
+constexpr int kSelMaxCand = 26624;   // candidates a group keeps in shared memory (208 KB of fp64)
 
 struct SelArgs {
     const lf_module* mods;
@@ -34,6 +35,7 @@ struct SelArgs {
     double band;
     int32_t* flag_list;
     int32_t* flag_count;
+    int32_t cand_cap;          // capacity of the shared-memory candidate list (dynamic shared memory / 8)
 };
 
 __device__ __forceinline__ int64_t block_sum_i64(int64_t v, int64_t* red) {
@@ -87,7 +89,31 @@ __device__ double max_below(const SelArgs& a, int m0, int M, double t, double* d
     return m;
 }
 
+// The same two counts over the group's candidate list in shared memory (`nc` energies,
+// each > 0), when the whole list fits.
+__device__ int64_t count_ge_s(const double* c, int nc, double t, int64_t* red) {
+    int64_t n = 0;
+    for (int q = threadIdx.x; q < nc; q += blockDim.x) n += (c[q] >= t);
+    return block_sum_i64(n, red);
+}
+
+__device__ double max_below_s(const double* c, int nc, double t, double* dred) {
+    double b = 0.0;
+    for (int q = threadIdx.x; q < nc; q += blockDim.x)
+        if (c[q] < t) b = fmax(b, c[q]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) b = fmax(b, __shfl_xor_sync(0xffffffffu, b, o));
+    __syncthreads();
+    if ((threadIdx.x & 31) == 0) dred[threadIdx.x >> 5] = b;
+    __syncthreads();
+    double m = 0.0;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) m = fmax(m, dred[w]);
+    return m;
+}
+
 __global__ void __launch_bounds__(kSelThreads) select_kernel(SelArgs a) {
+    extern __shared__ double s_cand[];   // a.cand_cap entries
+    __shared__ int s_nc;
     __shared__ int64_t red[32];
     __shared__ double dred[32];
     __shared__ int64_t s_take_eq, s_n_eq;
@@ -139,7 +165,10 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelArgs a) {
         }
         return;
     }
-    // energies, one module per thread, summed in j order
+    // energies, one module per thread, summed in j order; the candidates (j >= floor,
+    // e > 0) are also copied to shared memory when the group's list fits
+    if (threadIdx.x == 0) s_nc = 0;
+    __syncthreads();
     int64_t rsum = 0;
     for (int mi = threadIdx.x; mi < M; mi += blockDim.x) {
         const int i = a.grp_mods[m0 + mi];
@@ -162,15 +191,24 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelArgs a) {
             }
             en[j] = e;
         }
+        int nv = 0;
+        for (int j = fl; j < r; ++j) nv += en[j] > 0.0;
+        const int b = atomicAdd(&s_nc, nv);
+        if (b + nv <= a.cand_cap)
+            for (int j = fl, q = b; j < r; ++j)
+                if (en[j] > 0.0) s_cand[q++] = en[j];
         a.ranks[i] = fl;
     }
-    rsum = block_sum_i64(rsum, red);
+    rsum = block_sum_i64(rsum, red);   // (synchronises the block: s_nc and s_cand are complete)
+    const int nc = s_nc;
+    const bool in_smem = nc <= a.cand_cap;
+#define LF_COUNT_GE(t) (in_smem ? count_ge_s(s_cand, nc, (t), red) : count_ge(a, m0, M, (t), red))
     const int64_t K = ((int64_t)a.pol.ratio_num * rsum) / a.pol.ratio_den;
     const int64_t extra = K - (int64_t)fl * M;
     if (extra <= 0) return;  // ranks stay at the floor
 
     const double tiny = __longlong_as_double(1ll);
-    const int64_t npos = count_ge(a, m0, M, tiny, red);
+    const int64_t npos = LF_COUNT_GE(tiny);
     double theta;
     int64_t take_eq, n_eq = 0;
     if (npos <= extra) {
@@ -181,13 +219,13 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelArgs a) {
         long long lo = 1, hi = 0x7FF0000000000000ll;
         while (lo < hi) {
             const long long mid = lo + (hi - lo + 1) / 2;
-            const int64_t c = count_ge(a, m0, M, __longlong_as_double(mid), red);
+            const int64_t c = LF_COUNT_GE(__longlong_as_double(mid));
             if (c >= extra) lo = mid; else hi = mid - 1;
         }
         theta = __longlong_as_double(lo);
-        const int64_t n_gt = count_ge(a, m0, M, __longlong_as_double(lo + 1), red);
+        const int64_t n_gt = LF_COUNT_GE(__longlong_as_double(lo + 1));
         take_eq = extra - n_gt;
-        if (a.flag_list) n_eq = count_ge(a, m0, M, theta, red) - n_gt;
+        n_eq = LF_COUNT_GE(theta) - n_gt;
     }
     if (threadIdx.x == 0) {
         s_theta = theta;
@@ -199,8 +237,23 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelArgs a) {
     take_eq = s_take_eq;
     n_eq = s_n_eq;
     // per module: all e > theta, then the first take_eq candidates equal to theta in
-    // (module, j) order.  The equal-candidate prefix over modules is taken serially.
-    if (threadIdx.x == 0) {
+    // (module, j) order.  When every candidate equal to theta is taken (the usual case)
+    // each module counts its e >= theta on its own; a tie cut by the budget takes the
+    // equal-candidate prefix over modules serially.
+    if (take_eq >= n_eq) {
+        for (int mi = threadIdx.x; mi < M; mi += blockDim.x) {
+            const int i = a.grp_mods[m0 + mi];
+            const int r = a.mods[i].r;
+            const double* en = a.energy + (size_t)i * a.rs;
+            int k = fl;
+            for (int j = fl; j < r; ++j) {
+                const double e = en[j];
+                if (e > 0.0 && e >= theta) ++k;
+                else break;
+            }
+            a.ranks[i] = k;
+        }
+    } else if (threadIdx.x == 0) {
         int64_t left = take_eq;
         for (int mi = 0; mi < M; ++mi) {
             const int i = a.grp_mods[m0 + mi];
@@ -228,7 +281,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelArgs a) {
         // theta that the tie order leaves out, else the largest below theta) closer than
         // twice the band, the band being far above the main path's energy error.  Then
         // the modules holding a candidate within the band of theta are refined in fp64.
-        const double below = max_below(a, m0, M, theta, dred);
+        const double below = in_smem ? max_below_s(s_cand, nc, theta, dred) : max_below(a, m0, M, theta, dred);
         const bool tie_out = n_eq > take_eq;
         if (!tie_out && theta - below > 2.0 * a.band * theta) return;
         for (int mi = threadIdx.x; mi < M; mi += blockDim.x) {
@@ -246,6 +299,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelArgs a) {
             }
         }
     }
+#undef LF_COUNT_GE
 }
 
 // off_A[i+1] = off_A[i] + ranks[i] * d_in, off_Bt likewise with d_out (one CTA).
@@ -307,7 +361,7 @@ __global__ void refine_plan_kernel(const lf_module* mods, const int32_t* flag_li
             const int nch = (rows + chunk - 1) / chunk;
             const int mf = 2 * l + f;
             info[mf].nchunks = nch;
-            info[mf].slot0 = nch > 1 ? slot : -1;
+            info[mf].slot0 = nch > 1 ? slot : -1;   // nch > 1: the merge tree's nodes from slot0
             for (int c = 0; c < nch; ++c) {
                 work[w].mf = mf;
                 work[w].row0 = c * chunk;
@@ -315,7 +369,7 @@ __global__ void refine_plan_kernel(const lf_module* mods, const int32_t* flag_li
                 work[w].slot = nch > 1 ? slot + c : -1;
                 ++w;
             }
-            if (nch > 1) slot += nch;
+            if (nch > 1) slot += tree_slots(nch);
         }
     }
     *n_work = w;

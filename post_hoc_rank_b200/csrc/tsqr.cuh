@@ -48,13 +48,30 @@ struct TsqrArgs {
     const TsqrWork* work;
     const int32_t* n_work;      // device scalar
     const TsqrInfo* info;       // per local mf
-    int32_t* counters;          // per local mf, zero on entry
-    T* partial;                 // slots x RT x RT
+    int32_t* counters;          // per local mf (tree: per slot), zero on entry
+    T* partial;                 // slots x RT x RT (tree: slots x packed triangle)
     T* R_B;                     // per local module, rs x rs
     T* R_A;
     int32_t rs;
     const int32_t* only;        // per local mf (nullable): nonzero = factor this matrix, zero = skip it
+    // 0: the last chunk of a matrix to finish folds every chunk R in chunk order (dense
+    //    RT x RT slots, counters per mf);
+    // 1: binary merge tree over the chunks (packed triangle slots, one slot and one
+    //    counter per tree node: see tree_slots)
+    int32_t tree;
 };
+
+// Nodes of the binary merge tree over n chunks, every level included: level 0 holds
+// the n chunks, level l + 1 the ceil(n_l / 2) merges of level l, up to one root.  Node
+// i of level l has slot (and counter) slot0 + (nodes below level l) + i.
+__host__ __device__ inline int tree_slots(int n) {
+    int t = 0;
+    for (int m = n; ; m = (m + 1) >> 1) {
+        t += m;
+        if (m == 1) break;
+    }
+    return t;
+}
 
 // Packed upper triangle of an RT x RT matrix, row-major: row j holds columns j..RT-1.
 template <int RT>
@@ -178,6 +195,22 @@ __device__ __forceinline__ void load_tri_rows(T (&x)[Cols<RT>::NS][kTsqrTM], con
 }
 
 template <typename T, int RT>
+__device__ __forceinline__ void load_packed_rows(T (&x)[Cols<RT>::NS][kTsqrTM], const T* P, int i0) {
+    // rows i0..i0+TM-1 of a packed upper triangle (zero below the diagonal)
+    const int lane = threadIdx.x & 31;
+    using C = Cols<RT>;
+#pragma unroll
+    for (int s = 0; s < C::NS; ++s) {
+        const int c = C::col(lane, s);
+#pragma unroll
+        for (int i = 0; i < kTsqrTM; ++i) {
+            const int row = i0 + i;
+            x[s][i] = (c < RT && row <= c) ? __ldcg(P + tri_off<RT>(row, c)) : T(0);
+        }
+    }
+}
+
+template <typename T, int RT>
 __device__ __forceinline__ void tsqr_item(const TsqrArgs<T>& a, int wi, T* Rp, T* vbuf, int* s_last, int lane) {
     const TsqrWork w = a.work[wi];
     if (a.only && a.only[w.mf] == 0) return;   // warp-uniform
@@ -198,7 +231,39 @@ __device__ __forceinline__ void tsqr_item(const TsqrArgs<T>& a, int wi, T* Rp, T
 
     T* out = (factor == 0 ? a.R_B : a.R_A) + (size_t)local * a.rs * a.rs;
     const TsqrInfo inf = a.info[w.mf];
-    if (inf.nchunks > 1) {
+    if (inf.nchunks > 1 && a.tree) {
+        // Each node of the tree is qr([R_left; R_right]) of its two children, formed by
+        // the second child to finish (the fixed left-right order keeps the result
+        // independent of scheduling); a node with one child passes its R up unchanged.
+        constexpr int TRI = tri_size<RT>();
+        int node = w.slot - inf.slot0, nl = inf.nchunks, off = 0;
+        while (nl > 1) {
+            const int parent = node >> 1, offp = off + nl;
+            if ((node ^ 1) < nl) {
+                T* P = a.partial + (size_t)(inf.slot0 + off + node) * TRI;
+                for (int e = lane; e < TRI; e += 32) P[e] = Rp[e];
+                __threadfence();
+                __syncwarp();
+                if (lane == 0) *s_last = (atomicAdd(&a.counters[inf.slot0 + offp + parent], 1) == 1);
+                __syncwarp();
+                if (!*s_last) return;
+                __threadfence();
+                const int left = node & ~1;
+                const T* PL = a.partial + (size_t)(inf.slot0 + off + left) * TRI;
+                const T* PR = PL + TRI;
+                if (node != left)
+                    for (int e = lane; e < TRI; e += 32) Rp[e] = __ldcg(PL + e);
+                __syncwarp();
+                for (int i0 = 0; i0 < r; i0 += kTsqrTM) {
+                    load_packed_rows<T, RT>(x, PR, i0);
+                    warp_absorb<T, RT>(x, Rp, vbuf, r);
+                }
+            }
+            node = parent;
+            nl = (nl + 1) >> 1;
+            off = offp;
+        }
+    } else if (inf.nchunks > 1) {
         T* P = a.partial + (size_t)w.slot * RT * RT;
         for (int e = lane; e < RT * RT; e += 32) {
             const int j = e / RT, c = e % RT;
@@ -315,7 +380,7 @@ __device__ __forceinline__ T svd_tol(int r) { return T(r) * (sizeof(T) == 8 ? T(
 
 // One Jacobi rotation of rows p, q of M and of columns p, q of U (fp64 refinement):
 // returns whether the pair was rotated.
-template <typename T, int RT>
+template <typename T, int RT, bool ACC>
 __device__ __forceinline__ bool svd_rotate_acc(SvdSmem<T, RT>& s, int p, int q, int r, T tol) {
     T al[4] = {0, 0, 0, 0}, be[4] = {0, 0, 0, 0}, ga[4] = {0, 0, 0, 0};
     const T* mp = s.M[p];
@@ -352,6 +417,25 @@ __device__ __forceinline__ bool svd_rotate_acc(SvdSmem<T, RT>& s, int p, int q, 
     T* Up = s.Ut[p];
     T* Uq = s.Ut[q];
     int k = 0;
+    if constexpr (!ACC) {   // singular values only: rows of M alone
+#pragma unroll 2
+        for (; k + 3 < r; k += 4) {
+            T x[4], y[4], x2[4], y2[4];
+            ld4(Mp + k, x); ld4(Mq + k, y);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                x2[e] = c * x[e] - sn * y[e];
+                y2[e] = sn * x[e] + c * y[e];
+            }
+            st4(Mp + k, x2); st4(Mq + k, y2);
+        }
+        for (; k < r; ++k) {
+            const T x = Mp[k], y = Mq[k];
+            Mp[k] = c * x - sn * y;
+            Mq[k] = sn * x + c * y;
+        }
+        return true;
+    }
 #pragma unroll 2
     for (; k + 3 < r; k += 4) {   // 16-byte loads and stores of four columns
         T x[4], y[4], u[4], v[4], x2[4], y2[4], u2[4], v2[4];
@@ -377,13 +461,15 @@ __device__ __forceinline__ bool svd_rotate_acc(SvdSmem<T, RT>& s, int p, int q, 
 
 // One Jacobi rotation of rows p, q of M only (fp32 main path): both rows are read once
 // into registers (16-byte chunks; the row padding past r is zero), the three dot
-// products and the rotation run there, and the rows are written back once.
+// products and the rotation run there on packed fp32 pairs (each component rounds as
+// fmaf), and the rows are written back once.  Each sum keeps four partial chains,
+// element e of a chunk in chain e, added as (0 + 1) + (2 + 3).
 template <typename T, int RT>
 __device__ __forceinline__ bool svd_rotate_rows(SvdSmem<T, RT>& s, int p, int q, int r, T tol) {
     static_assert(sizeof(T) == 4, "register path is fp32");
     constexpr int NC = RT / 4;
     float4 x[NC], y[NC];
-    float al[4] = {0.f, 0.f, 0.f, 0.f}, be[4] = {0.f, 0.f, 0.f, 0.f}, ga[4] = {0.f, 0.f, 0.f, 0.f};
+    float2 al01 = make_float2(0.f, 0.f), al23 = al01, be01 = al01, be23 = al01, ga01 = al01, ga23 = al01;
 #pragma unroll
     for (int c = 0; c < NC; ++c) {
         if (4 * c < r) {
@@ -392,29 +478,36 @@ __device__ __forceinline__ bool svd_rotate_rows(SvdSmem<T, RT>& s, int p, int q,
         } else {
             x[c] = y[c] = make_float4(0.f, 0.f, 0.f, 0.f);
         }
-        al[0] = fmaf(x[c].x, x[c].x, al[0]); al[1] = fmaf(x[c].y, x[c].y, al[1]);
-        al[2] = fmaf(x[c].z, x[c].z, al[2]); al[3] = fmaf(x[c].w, x[c].w, al[3]);
-        be[0] = fmaf(y[c].x, y[c].x, be[0]); be[1] = fmaf(y[c].y, y[c].y, be[1]);
-        be[2] = fmaf(y[c].z, y[c].z, be[2]); be[3] = fmaf(y[c].w, y[c].w, be[3]);
-        ga[0] = fmaf(x[c].x, y[c].x, ga[0]); ga[1] = fmaf(x[c].y, y[c].y, ga[1]);
-        ga[2] = fmaf(x[c].z, y[c].z, ga[2]); ga[3] = fmaf(x[c].w, y[c].w, ga[3]);
+        const float2 x01 = make_float2(x[c].x, x[c].y), x23 = make_float2(x[c].z, x[c].w);
+        const float2 y01 = make_float2(y[c].x, y[c].y), y23 = make_float2(y[c].z, y[c].w);
+        al01 = __ffma2_rn(x01, x01, al01);
+        al23 = __ffma2_rn(x23, x23, al23);
+        be01 = __ffma2_rn(y01, y01, be01);
+        be23 = __ffma2_rn(y23, y23, be23);
+        ga01 = __ffma2_rn(x01, y01, ga01);
+        ga23 = __ffma2_rn(x23, y23, ga23);
     }
-    const float alpha = (al[0] + al[1]) + (al[2] + al[3]);
-    const float beta_ = (be[0] + be[1]) + (be[2] + be[3]);
-    const float gamma = (ga[0] + ga[1]) + (ga[2] + ga[3]);
+    const float alpha = (al01.x + al01.y) + (al23.x + al23.y);
+    const float beta_ = (be01.x + be01.y) + (be23.x + be23.y);
+    const float gamma = (ga01.x + ga01.y) + (ga23.x + ga23.y);
     if (!(gamma != 0.f && fabsf(gamma) > tol * sqrtf(alpha * beta_))) return false;
     const float zeta = (beta_ - alpha) / (2.f * gamma);
     const float tt = (zeta >= 0.f ? 1.f : -1.f) / (fabsf(zeta) + sqrtf(1.f + zeta * zeta));
     const float cs = 1.f / sqrtf(1.f + tt * tt);
     const float sn = cs * tt;
+    const float2 c2 = make_float2(cs, cs), s2 = make_float2(sn, sn), ms2 = make_float2(-sn, -sn);
 #pragma unroll
     for (int c = 0; c < NC; ++c) {
         if (4 * c < r) {
-            const float4 a = x[c], b = y[c];
-            *reinterpret_cast<float4*>(&s.M[p][4 * c]) =
-                make_float4(cs * a.x - sn * b.x, cs * a.y - sn * b.y, cs * a.z - sn * b.z, cs * a.w - sn * b.w);
-            *reinterpret_cast<float4*>(&s.M[q][4 * c]) =
-                make_float4(sn * a.x + cs * b.x, sn * a.y + cs * b.y, sn * a.z + cs * b.z, sn * a.w + cs * b.w);
+            const float2 a01 = make_float2(x[c].x, x[c].y), a23 = make_float2(x[c].z, x[c].w);
+            const float2 b01 = make_float2(y[c].x, y[c].y), b23 = make_float2(y[c].z, y[c].w);
+            // x' = cs a - sn b,  y' = sn a + cs b  (the product with b rounded first)
+            const float2 xp01 = __ffma2_rn(c2, a01, __fmul2_rn(ms2, b01));
+            const float2 xp23 = __ffma2_rn(c2, a23, __fmul2_rn(ms2, b23));
+            const float2 yp01 = __ffma2_rn(s2, a01, __fmul2_rn(c2, b01));
+            const float2 yp23 = __ffma2_rn(s2, a23, __fmul2_rn(c2, b23));
+            *reinterpret_cast<float4*>(&s.M[p][4 * c]) = make_float4(xp01.x, xp01.y, xp23.x, xp23.y);
+            *reinterpret_cast<float4*>(&s.M[q][4 * c]) = make_float4(yp01.x, yp01.y, yp23.x, yp23.y);
         }
     }
     return true;
@@ -433,7 +526,8 @@ __global__ void __launch_bounds__(32 * svd_warps<T>()) svd_kernel(SvdArgs<TIN, T
     const TIN* RB = a.R_B + (size_t)local * rs * rs;
     const TIN* RA = a.R_A + (size_t)local * rs * rs;
 
-    // fp64 (refinement): U accumulates the rotations.  fp32 (main path): rows of M only
+    // fp64 (refinement): U accumulates the rotations when U is wanted (the refinement
+    // itself needs sigma only).  fp32 (main path): rows of M only
     // are rotated, and U = M_0 M'^T Sigma^-2 is formed at the end from M_0, which is
     // parked in the module's U output block meanwhile.
     constexpr bool kAccU = sizeof(T) == 8;
@@ -531,13 +625,16 @@ __global__ void __launch_bounds__(32 * svd_warps<T>()) svd_kernel(SvdArgs<TIN, T
                 if (lane == 0) {
                     p = rp - 1;
                     q = t;
-                } else {
-                    p = (t + lane) % (rp - 1);
-                    q = (t - lane + rp - 1) % (rp - 1);
+                } else {   // (t + lane) mod (rp - 1) and (t - lane) mod (rp - 1), both in range
+                    p = t + lane;
+                    if (p >= rp - 1) p -= rp - 1;
+                    q = t - lane;
+                    if (q < 0) q += rp - 1;
                 }
                 if (p < r && q < r) {
                     if constexpr (kAccU) {
-                        rot |= svd_rotate_acc<T, RT>(s, p, q, r, tol);
+                        rot |= a.U ? svd_rotate_acc<T, RT, true>(s, p, q, r, tol)
+                                   : svd_rotate_acc<T, RT, false>(s, p, q, r, tol);
                     } else {
                         rot |= svd_rotate_rows<T, RT>(s, p, q, r, tol);
                     }
