@@ -325,18 +325,21 @@ def apply_bytes(T, d_in, d_out, ranks_used):
     return 2 * T * d_in + 4 * T * d_out + 4 * T + sum(2 * k * (d_in + d_out) for k in ranks_used)
 
 
-def decode_bench(args, dev, stream, hbm, variant="ragged", fused=False):
+def decode_bench(args, dev, stream, hbm, variant="ragged", fused=False, per_layer=True):
     """Config 3: Llama-3-8B shapes, 32 layers x 7 projections, T=256, 128 adapters.
     variant: "ragged" (retained ranks as allocated), "padded" (every adapter's factors
     of a projection zero-padded to the largest retained rank over the 128 resident
-    adapters), "r64" (uncompressed rank-64 adapters).  fused: q/k/v and gate/up as
-    one multi-slice call each (4 calls per layer instead of 7)."""
+    adapters), "r64" (uncompressed rank-64 adapters).  per_layer: the 7 projections of
+    a layer in one lf_lora_shrink_expand_projections call (32 calls per step); else
+    fused: q/k/v and gate/up as one multi-slice call each (4 calls per layer), or one
+    call per projection (7 per layer)."""
     import torch
     from post_hoc_rank_b200 import api, synth
     from post_hoc_rank_b200 import loraforge as lf
 
     M = synth.LLAMA3_8B
     n_ad, T = 128, 256
+    per_layer = per_layer and not fused
     lay = synth.fleet_layout(n_ad, M, r=64)
     mods = api.modules_from_layout(lay)
     sig = synth.sigma_tables(n_ad, M, 64, cfg_id=3)
@@ -370,16 +373,19 @@ def decode_bench(args, dev, stream, hbm, variant="ragged", fused=False):
                 Bt.view(n_ad, kmax, d_out)[pad] = 0
             groups.append((d_in, d_out, rk, offA, offB, Ap, Bt))
             total_bytes += apply_bytes(T, d_in, d_out, [int(rk[a]) for a in distinct])
-        lc, sets = _layer_calls(groups, lambda d: x_f if d == M.ffn else x_h, ids_d, n_ad, T, dev, (3, 5, l), fused)
+        lc, sets = _layer_calls(groups, lambda d: x_f if d == M.ffn else x_h, ids_d, n_ad, T, dev, (3, 5, l), fused,
+                                per_layer=per_layer)
         calls += lc
         if fused:   # x is read once per call, not once per projection
             total_bytes -= sum(2 * T * groups[ps[0]][0] * (len(ps) - 1) for ps in sets)
     names = {"ragged": "S 1/12 floor 1 ranks (ragged)",
              "padded": "S 1/12 floor 1 ranks zero-padded to the per-projection max over resident adapters",
              "r64": "uncompressed rank-64 adapters"}
+    how = ("; q/k/v and gate/up as one slice call each" if fused else
+           ("; the 7 projections of a layer in one call" if per_layer else "; one call per projection"))
     out = _apply_run(args, calls, ids_d, n_ad, T, total_bytes, stream, hbm, dict(
         workload="decode: Llama-3-8B, 32 layers x 7 projections, 256 tokens, 128 adapters Zipf(1), "
-                 + names[variant] + ("; q/k/v and gate/up as one slice call each" if fused else ""),
+                 + names[variant] + how,
         distinct_adapters=len(distinct), mean_rank=float(ranks_all.mean())))
     del calls
     torch.cuda.empty_cache()
@@ -491,15 +497,36 @@ def _routed_call(x, y, ids_d, n_ad, slices, ws, scale=2.0):
     return run
 
 
-def _layer_calls(groups, x_of, ids_d, n_ad, T, dev, key, fused, route_once=False):
+def _projections_call(items, ids_d, n_ad, T, ws, scale=2.0):
+    """Every projection of a layer through one lf_lora_shrink_expand_projections call;
+    items: (x, y, (d_out, y_offset, ranks, off_A, off_Bt, A_pool, Bt_pool)) device tensors."""
+    from post_hoc_rank_b200 import loraforge as lf
+    projs = [lf.make_projection(x, y, lf.make_slice(*t)) for x, y, t in items]
+
+    def run(st=None, _keep=items):
+        lf.lf_lora_shrink_expand_projections(T, ids_d, n_ad, projs, scale, ws, stream=st)
+    return run
+
+
+def _layer_calls(groups, x_of, ids_d, n_ad, T, dev, key, fused, route_once=False, per_layer=False):
     """Calls of one layer.  groups: per projection (d_in, d_out, rk int64 array, offA,
     offB, Ap, Bt); fused: q/k/v and gate/up (projections reading the same x) go as
     one slice call each; route_once: one lf_route_tokens call, then routed projection
-    calls on the same workspace.  Returns (callables, the projection sets)."""
+    calls on the same workspace; per_layer: all projections in one
+    lf_lora_shrink_expand_projections call.  Returns (callables, the projection sets)."""
     import torch
     from post_hoc_rank_b200 import api, synth
     from post_hoc_rank_b200 import loraforge as lf
     sets = [[0, 1, 2], [3], [4, 5], [6]] if fused else [[p] for p in range(len(groups))]
+    if per_layer:
+        items = []
+        for p, (d_in, d_out, rk, offA, offB, Ap, Bt) in enumerate(groups):
+            y = synth.normal_bf16((T, d_out), key + (p,), device=dev)
+            items.append((x_of(d_in), y, (d_out, 0, torch.from_numpy(rk.astype(np.int32)).to(dev),
+                                          torch.from_numpy(offA[:-1]).to(dev), torch.from_numpy(offB[:-1]).to(dev),
+                                          Ap, Bt)))
+        ws = api.workspace(lf.lf_apply_workspace_size(T, n_ad), dev)
+        return [_projections_call(items, ids_d, n_ad, T, ws)], sets
     calls = []
     rws = None
     if route_once:
@@ -1126,6 +1153,7 @@ def main():
                 "decode_padded_to_max": decode_bench(args, dev, stream, hbm, "padded"),
                 "decode_uncompressed_r64": decode_bench(args, dev, stream, hbm, "r64"),
                 "decode_fused_slices": decode_bench(args, dev, stream, hbm, fused=True),
+                "decode_per_projection": decode_bench(args, dev, stream, hbm, per_layer=False),
                 "decode_sigma_sandwich_r16_diag": sandwich_bench(args, dev, stream, hbm, 16, True),
                 "decode_sigma_sandwich_r16_full": sandwich_bench(args, dev, stream, hbm, 16, False),
                 "prefill_k16": prefill_bench(args, dev, stream, hbm, 16),

@@ -233,6 +233,40 @@ lf_status lf_lora_shrink_expand_slices(int32_t T, int32_t d_in, const void* x, v
                                        float scale, const float* adapter_scale, int32_t* seg_out,
                                        void* ws, size_t ws_bytes, lf_stream_t stream);
 
+/* ---- Several projections of one batch in one call -----------------------------
+ * A decode step applies every adapted projection of a layer to the same tokens
+ * ("Compress then Serve", section 13.4: the side path per token, indexed by the
+ * token's adapter).  This call takes up to LF_MAX_PROJECTIONS projections, each
+ * with its own input x (T x d_in bf16, row-major), its own y (T rows of y_ld bf16)
+ * and its own factor tables (the lf_slice fields: d_out, y_offset, ranks, offsets,
+ * pools), and for every token t with a = ids[t] >= 0 and every projection p:
+ *   t_p    = A'_{p,a} x_{p,t}                                 (k_{p,a} fp32 values)
+ *   y_{p,t}[y_offset_p .. y_offset_p + d_out_p) =
+ *            bf16( y_{p,t}[...] + scale_a * B'_{p,a} t_p )    (one rounding)
+ * with scale_a as for lf_lora_shrink_expand_slices.  In the decode regime
+ * (T <= 8 n_adapters) every projection goes in one launch of the token-parallel
+ * kernel, and ws is not used (it may be NULL with ws_bytes 0).  Otherwise the
+ * projections are applied one after the other on the routed path: the first routes
+ * the batch into ws and the others reuse its tables, so ws must then hold
+ * lf_apply_workspace_size(T, n_adapters) bytes.  Projections must not write
+ * overlapping parts of any y, and no y may overlap an x of the same call.
+ * Per projection the argument rules of lf_lora_shrink_expand_slices with one slice
+ * apply (reserved fields 0); host errors are returned before anything is launched,
+ * and device-side errors latch as there, per (adapter, projection). */
+#define LF_MAX_PROJECTIONS 8
+typedef struct {
+    const void* x;              /* T x d_in bf16 */
+    void* y;                    /* T rows of y_ld bf16, updated in place */
+    int32_t d_in;
+    int32_t reserved;           /* 0 */
+    int64_t y_ld;               /* row stride of y (elements), multiple of 8 */
+    lf_slice slice;             /* where in y, and with which factors */
+} lf_projection;
+lf_status lf_lora_shrink_expand_projections(int32_t T, const int32_t* ids, int32_t n_adapters,
+                                            const lf_projection* projs /*[host]*/, int32_t n_proj,
+                                            float scale, const float* adapter_scale,
+                                            void* ws, size_t ws_bytes, lf_stream_t stream);
+
 /* ---- Routing once per batch ---------------------------------------------------
  * Every projection of a forward pass sees the same token ids, so the routing (the
  * stable sort of tokens by adapter, the segment table and the work items) can be

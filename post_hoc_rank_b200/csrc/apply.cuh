@@ -487,35 +487,23 @@ constexpr int kBgmvVec = 4;                                  // 8-column vectors
 constexpr int kBgmvCols = kBgmvThreads * 8 * kBgmvVec;       // d_out columns per CTA
 constexpr int kBgmvJ = 8;                                    // retained directions per shrink pass
 
-// One (token, column chunk) of the token-parallel side path; CTA-uniform control flow.
-__device__ __forceinline__ void bgmv_token(const ApplyArgs& a, int tok, float (&red)[kBgmvThreads / 32][kBgmvJ],
-                                           float* ts, float* tw) {
-    const int ad = a.ids[tok];
-    if (ad == -1) return;
-    const int sl = slice_of_chunk(a, blockIdx.y);
-    const SliceTab& S = a.sl[sl];
-    const bool lead = (int)blockIdx.y == S.chunk0 && threadIdx.x == 0;   // one CTA per (token, slice) reports
-    if (ad < -1 || ad >= a.n_adapters) {
-        if (lead && sl == 0) latch_error(LF_ERR_BAD_INDEX);
-        return;
-    }
-    int k;
-    int64_t oa, ob;
-    if (!slice_factors(a, sl, ad, lead, k, oa, ob)) return;
+// t = A' x_t for one token (k values of fp32 into ts): every thread takes 8-element
+// pieces of the row, kBgmvJ directions per pass, reduced over the warps in a fixed
+// order.  CTA-uniform control flow (block barriers inside).
+__device__ __forceinline__ void bgmv_shrink(const __nv_bfloat16* xr, int d_in, const __nv_bfloat16* Ap, int k,
+                                            float (&red)[kBgmvThreads / 32][kBgmvJ], float* ts) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const __nv_bfloat16* xr = a.x + (int64_t)tok * a.d_in;
-    const __nv_bfloat16* Ap = S.A_pool + oa;
     for (int j0 = 0; j0 < k; j0 += kBgmvJ) {
         const int nj = min(kBgmvJ, k - j0);
         float acc[kBgmvJ];
 #pragma unroll
         for (int jj = 0; jj < kBgmvJ; ++jj) acc[jj] = 0.f;
-        for (int d0 = tid * 8; d0 < a.d_in; d0 += kBgmvThreads * 8) {
+        for (int d0 = tid * 8; d0 < d_in; d0 += kBgmvThreads * 8) {
             uint4 ar[kBgmvJ];
             const uint4 xv = __ldg(reinterpret_cast<const uint4*>(xr + d0));
 #pragma unroll
             for (int jj = 0; jj < kBgmvJ; ++jj)
-                if (jj < nj) ar[jj] = __ldg(reinterpret_cast<const uint4*>(Ap + (int64_t)(j0 + jj) * a.d_in + d0));
+                if (jj < nj) ar[jj] = __ldg(reinterpret_cast<const uint4*>(Ap + (int64_t)(j0 + jj) * d_in + d0));
             float xf[8];
             bf16x8_to_f32(xv, xf);
 #pragma unroll
@@ -544,20 +532,17 @@ __device__ __forceinline__ void bgmv_token(const ApplyArgs& a, int tok, float (&
         }
         __syncthreads();
     }
-    const float* tv = ts;
-    if (a.sigma_mode) {   // Sigma-sandwich: t <- Sigma_a t
-        sigma_apply(a, ad, k, ts, tw, tid, kBgmvThreads);
-        __syncthreads();
-        tv = tw;
-    }
-    const __nv_bfloat16* Bt = S.Bt_pool + ob;
-    __nv_bfloat16* yr = a.y + (int64_t)tok * a.y_ld + S.y_off;
-    const float scale = adapter_scale(a, ad);
-    const int cbase = ((int)blockIdx.y - S.chunk0) * kBgmvCols;
+}
+
+// y[cbase .. cbase + kBgmvCols) of one token row (within d_out) += scale * B'^T tv,
+// rounded once to bf16; 16-byte loads of the k rows of B'^T.
+__device__ __forceinline__ void bgmv_expand(const float* tv, int k, const __nv_bfloat16* Bt, int d_out,
+                                            __nv_bfloat16* yr, int cbase, float scale) {
+    const int tid = threadIdx.x;
 #pragma unroll
     for (int h = 0; h < kBgmvVec; ++h) {
         const int e = cbase + h * (kBgmvThreads * 8) + tid * 8;
-        if (e >= S.d_out) break;
+        if (e >= d_out) break;
         uint4 yv = *reinterpret_cast<const uint4*>(yr + e);   // issued before the k-row loads are consumed
         float acc[8];
 #pragma unroll
@@ -565,7 +550,7 @@ __device__ __forceinline__ void bgmv_token(const ApplyArgs& a, int tok, float (&
 #pragma unroll 4
         for (int j = 0; j < k; ++j) {
             float bf[8];
-            bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(Bt + (int64_t)j * S.d_out + e)), bf);
+            bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(Bt + (int64_t)j * d_out + e)), bf);
             const float tj = tv[j];
 #pragma unroll
             for (int c = 0; c < 8; ++c) acc[c] = fmaf(tj, bf[c], acc[c]);
@@ -578,6 +563,32 @@ __device__ __forceinline__ void bgmv_token(const ApplyArgs& a, int tok, float (&
         }
         *reinterpret_cast<uint4*>(yr + e) = yv;
     }
+}
+
+// One (token, column chunk) of the token-parallel side path; CTA-uniform control flow.
+__device__ __forceinline__ void bgmv_token(const ApplyArgs& a, int tok, float (&red)[kBgmvThreads / 32][kBgmvJ],
+                                           float* ts, float* tw) {
+    const int ad = a.ids[tok];
+    if (ad == -1) return;
+    const int sl = slice_of_chunk(a, blockIdx.y);
+    const SliceTab& S = a.sl[sl];
+    const bool lead = (int)blockIdx.y == S.chunk0 && threadIdx.x == 0;   // one CTA per (token, slice) reports
+    if (ad < -1 || ad >= a.n_adapters) {
+        if (lead && sl == 0) latch_error(LF_ERR_BAD_INDEX);
+        return;
+    }
+    int k;
+    int64_t oa, ob;
+    if (!slice_factors(a, sl, ad, lead, k, oa, ob)) return;
+    bgmv_shrink(a.x + (int64_t)tok * a.d_in, a.d_in, S.A_pool + oa, k, red, ts);
+    const float* tv = ts;
+    if (a.sigma_mode) {   // Sigma-sandwich: t <- Sigma_a t
+        sigma_apply(a, ad, k, ts, tw, threadIdx.x, kBgmvThreads);
+        __syncthreads();
+        tv = tw;
+    }
+    bgmv_expand(tv, k, S.Bt_pool + ob, S.d_out, a.y + (int64_t)tok * a.y_ld + S.y_off,
+                ((int)blockIdx.y - S.chunk0) * kBgmvCols, adapter_scale(a, ad));
 }
 
 // LIST = false: CTA blockIdx.x applies token blockIdx.x (decode regime, no routing pass).
@@ -598,6 +609,34 @@ __global__ void __launch_bounds__(kBgmvThreads, 2) bgmv_kernel(ApplyArgs a) {
         bgmv_token(a, __ldg(a.tok_list + u), red, ts, tw);
         __syncthreads();   // red / ts / tw are rewritten by the next token
     }
+}
+
+// Several projections of one decode batch in one launch: CTA (token, column chunk),
+// the chunks of all projections laid end to end along grid.y (each projection's first
+// chunk at its chunk0).  Per projection the same arithmetic as bgmv_kernel<false>.
+__global__ void __launch_bounds__(kBgmvThreads, 2) bgmv_proj_kernel(ProjArgs a) {
+    __shared__ float red[kBgmvThreads / 32][kBgmvJ];
+    __shared__ float ts[kMaxRank];
+    const int tok = blockIdx.x, c = blockIdx.y;
+    int p = 0;
+#pragma unroll
+    for (int i = 1; i < kMaxProj; ++i)
+        if (i < a.n_proj && c >= a.p[i].chunk0) p = i;
+    const ProjTab& P = a.p[p];
+    const int ad = a.ids[tok];
+    if (ad == -1) return;
+    const bool lead = c == P.chunk0 && threadIdx.x == 0;   // one CTA per (token, projection) reports
+    if (ad < -1 || ad >= a.n_adapters) {
+        if (lead && p == 0) latch_error(LF_ERR_BAD_INDEX);
+        return;
+    }
+    int k;
+    int64_t oa, ob;
+    if (!factor_lookup(P.ranks, P.off_A, P.off_Bt, 0, P.d_in, P.d_out, P.pool_A, P.pool_Bt, ad, lead, k, oa, ob))
+        return;
+    bgmv_shrink(P.x + (int64_t)tok * P.d_in, P.d_in, P.A_pool + oa, k, red, ts);
+    bgmv_expand(ts, k, P.Bt_pool + ob, P.d_out, P.y + (int64_t)tok * P.y_ld + P.y_off, (c - P.chunk0) * kBgmvCols,
+                a.scales ? a.scales[ad] : a.scale);
 }
 
 // Decode regime of the no-allocation entry point (one slice, sorted items): CTA

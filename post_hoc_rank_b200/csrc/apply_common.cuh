@@ -94,23 +94,22 @@ __device__ __forceinline__ int slice_of_chunk(const ApplyArgs& a, int c) {
 // pools: k > 64 -> LF_ERR_SHAPE, offsets not 16-byte aligned -> LF_ERR_ALIGNMENT,
 // rows past a pool -> LF_ERR_WORKSPACE (latched when `report`); an invalid adapter
 // contributes nothing.  Returns true when there is work (k > 0).
-__device__ __forceinline__ bool slice_factors(const ApplyArgs& a, int s, int ad, bool report, int& k, int64_t& oa,
-                                              int64_t& ob) {
-    const SliceTab& t = a.sl[s];
-    if (t.ranks) {
-        k = t.ranks[ad];
-        oa = t.off_A[ad];
-        ob = t.off_Bt[ad];
+__device__ __forceinline__ bool factor_lookup(const int32_t* ranks, const int64_t* off_A, const int64_t* off_Bt,
+                                              int k_shared, int d_in, int d_out, int64_t pool_A, int64_t pool_Bt,
+                                              int ad, bool report, int& k, int64_t& oa, int64_t& ob) {
+    if (ranks) {
+        k = ranks[ad];
+        oa = off_A[ad];
+        ob = off_Bt[ad];
     } else {   // shared factors
-        k = t.k_shared;
+        k = k_shared;
         oa = 0;
         ob = 0;
     }
     int err = 0;
     if (k > kMaxRank) err = LF_ERR_SHAPE;
     else if (k > 0 && ((oa & 7) || (ob & 7))) err = LF_ERR_ALIGNMENT;
-    else if (k > 0 && (oa < 0 || ob < 0 || oa + (int64_t)k * a.d_in > t.pool_A ||
-                       ob + (int64_t)k * t.d_out > t.pool_Bt))
+    else if (k > 0 && (oa < 0 || ob < 0 || oa + (int64_t)k * d_in > pool_A || ob + (int64_t)k * d_out > pool_Bt))
         err = LF_ERR_WORKSPACE;
     if (err) {
         if (report) latch_error(err);
@@ -120,6 +119,38 @@ __device__ __forceinline__ bool slice_factors(const ApplyArgs& a, int s, int ad,
     if (k < 0) k = 0;
     return k > 0;
 }
+
+__device__ __forceinline__ bool slice_factors(const ApplyArgs& a, int s, int ad, bool report, int& k, int64_t& oa,
+                                              int64_t& ob) {
+    const SliceTab& t = a.sl[s];
+    return factor_lookup(t.ranks, t.off_A, t.off_Bt, t.k_shared, a.d_in, t.d_out, t.pool_A, t.pool_Bt, ad, report, k,
+                         oa, ob);
+}
+
+// Several projections of one batch (same tokens and ids), each with its own x, y and
+// factor tables, applied by one launch in the decode regime.
+constexpr int kMaxProj = 8;
+struct ProjTab {
+    const __nv_bfloat16* x;     // T x d_in
+    __nv_bfloat16* y;           // T rows of y_ld
+    int64_t y_ld, y_off;
+    int32_t d_in, d_out;
+    int32_t chunk0;             // first grid column chunk of the projection
+    int32_t pad;
+    const int32_t* ranks;
+    const int64_t* off_A;
+    const int64_t* off_Bt;
+    const __nv_bfloat16* A_pool;
+    const __nv_bfloat16* Bt_pool;
+    int64_t pool_A, pool_Bt;
+};
+struct ProjArgs {
+    int32_t T, n_adapters, n_proj, n_chunks;
+    const int32_t* ids;
+    float scale;
+    const float* scales;        // per adapter (nullable): replaces `scale`
+    ProjTab p[kMaxProj];
+};
 
 __device__ __forceinline__ float adapter_scale(const ApplyArgs& a, int ad) {
     return a.scales ? a.scales[ad] : a.scale;

@@ -543,14 +543,11 @@ struct SharedSlice {
 // adapters of 64+ tokens gather scattered rows into tensor-core tiles.
 static bool decode_regime(int64_t T, int64_t n_adapters) { return T <= (int64_t)kGemvTok * n_adapters; }
 
-static lf_status apply_impl(int32_t T, int32_t d_in, const void* x, void* y, int64_t y_ld, const int32_t* ids,
-                            int32_t n_adapters, const lf_slice* sl, int32_t ns, float scale, const float* scales,
-                            int32_t* seg_out, void* ws, size_t ws_bytes, cudaStream_t s,
-                            const SharedSlice* shared = nullptr, bool routed = false) {
-    if (T < 0 || d_in < 1 || n_adapters < 1 || n_adapters > 16384 || ns < 1 || ns > kMaxSlices || !sl)
-        return LF_ERR_INVALID_ARG;
-    if (T == 0) return LF_OK;
-    if (!x || !y || !ids || !ws) return LF_ERR_INVALID_ARG;
+// Host checks of one apply's x, y and slices (shared: factors shared by all adapters,
+// no per-adapter tables).
+static lf_status check_apply(int32_t d_in, const void* x, const void* y, int64_t y_ld, const lf_slice* sl, int32_t ns,
+                             bool shared) {
+    if (d_in < 1 || !x || !y || !sl) return LF_ERR_INVALID_ARG;
     if ((d_in & 7) || (y_ld & 7)) return LF_ERR_ALIGNMENT;
     if (!aligned16(x) || !aligned16(y)) return LF_ERR_ALIGNMENT;
     for (int q = 0; q < ns; ++q) {
@@ -562,6 +559,19 @@ static lf_status apply_impl(int32_t T, int32_t d_in, const void* x, void* y, int
         if ((t.d_out & 7) || (t.y_offset & 7)) return LF_ERR_ALIGNMENT;
         if (!aligned16(t.A_pool) || !aligned16(t.Bt_pool)) return LF_ERR_ALIGNMENT;
     }
+    return LF_OK;
+}
+
+static lf_status apply_impl(int32_t T, int32_t d_in, const void* x, void* y, int64_t y_ld, const int32_t* ids,
+                            int32_t n_adapters, const lf_slice* sl, int32_t ns, float scale, const float* scales,
+                            int32_t* seg_out, void* ws, size_t ws_bytes, cudaStream_t s,
+                            const SharedSlice* shared = nullptr, bool routed = false) {
+    if (T < 0 || d_in < 1 || n_adapters < 1 || n_adapters > 16384 || ns < 1 || ns > kMaxSlices || !sl)
+        return LF_ERR_INVALID_ARG;
+    if (T == 0) return LF_OK;
+    if (!ids || !ws) return LF_ERR_INVALID_ARG;
+    const lf_status cs = check_apply(d_in, x, y, y_ld, sl, ns, shared != nullptr);
+    if (cs != LF_OK) return cs;
     ApplyWs w;
     if (ws_bytes < carve_apply(nullptr, T, n_adapters, ns, &w)) return LF_ERR_WORKSPACE;
     carve_apply(reinterpret_cast<char*>(align_up((int64_t)reinterpret_cast<uintptr_t>(ws), 256)), T, n_adapters,
@@ -1393,6 +1403,73 @@ lf_status lf_lora_shrink_expand_slices(int32_t T, int32_t d_in, const void* x, v
                                        void* ws, size_t ws_bytes, lf_stream_t stream) {
     return apply_impl(T, d_in, x, y, y_ld, ids, n_adapters, slices, n_slices, scale, adapter_scale, seg_out, ws,
                       ws_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+static_assert(kMaxProj == LF_MAX_PROJECTIONS, "projection table size");
+
+lf_status lf_lora_shrink_expand_projections(int32_t T, const int32_t* ids, int32_t n_adapters,
+                                            const lf_projection* projs, int32_t n_proj, float scale,
+                                            const float* adapter_scale, void* ws, size_t ws_bytes,
+                                            lf_stream_t stream) {
+    if (T < 0 || n_adapters < 1 || n_adapters > 16384 || n_proj < 1 || n_proj > kMaxProj || !projs)
+        return LF_ERR_INVALID_ARG;
+    if (T == 0) return LF_OK;
+    if (!ids) return LF_ERR_INVALID_ARG;
+    for (int p = 0; p < n_proj; ++p) {
+        if (projs[p].reserved != 0 || projs[p].slice.reserved != 0) return LF_ERR_INVALID_ARG;
+        const lf_status st = check_apply(projs[p].d_in, projs[p].x, projs[p].y, projs[p].y_ld, &projs[p].slice, 1, false);
+        if (st != LF_OK) return st;
+    }
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (!decode_regime(T, n_adapters)) {
+        // routed path, projection by projection: the first call routes the batch into
+        // ws, the others reuse its tables
+        for (int p = 0; p < n_proj; ++p) {
+            const lf_projection& q = projs[p];
+            const lf_status st = apply_impl(T, q.d_in, q.x, q.y, q.y_ld, ids, n_adapters, &q.slice, 1, scale,
+                                            adapter_scale, nullptr, ws, ws_bytes, s, nullptr, p > 0);
+            if (st != LF_OK) return st;
+        }
+        return LF_OK;
+    }
+    ProjArgs A{};
+    A.T = T;
+    A.n_adapters = n_adapters;
+    A.n_proj = n_proj;
+    A.ids = ids;
+    A.scale = scale;
+    A.scales = adapter_scale;
+    // the projections with the most work per token first along grid.y, so the long
+    // CTAs start in the first waves (the table order is free: each CTA finds its
+    // projection from the chunk ranges)
+    int order[kMaxProj];
+    for (int p = 0; p < n_proj; ++p) order[p] = p;
+    std::stable_sort(order, order + n_proj, [&](int u, int v) {
+        return (int64_t)projs[u].d_in + projs[u].slice.d_out > (int64_t)projs[v].d_in + projs[v].slice.d_out;
+    });
+    int chunks = 0;
+    for (int i = 0; i < n_proj; ++i) {
+        const lf_projection& q = projs[order[i]];
+        ProjTab& t = A.p[i];
+        t.x = reinterpret_cast<const __nv_bfloat16*>(q.x);
+        t.y = reinterpret_cast<__nv_bfloat16*>(q.y);
+        t.y_ld = q.y_ld;
+        t.y_off = q.slice.y_offset;
+        t.d_in = q.d_in;
+        t.d_out = q.slice.d_out;
+        t.chunk0 = chunks;
+        t.ranks = q.slice.ranks;
+        t.off_A = q.slice.off_A;
+        t.off_Bt = q.slice.off_Bt;
+        t.A_pool = reinterpret_cast<const __nv_bfloat16*>(q.slice.A_pool);
+        t.Bt_pool = reinterpret_cast<const __nv_bfloat16*>(q.slice.Bt_pool);
+        t.pool_A = q.slice.pool_elems_A;
+        t.pool_Bt = q.slice.pool_elems_Bt;
+        chunks += (int)cdiv(q.slice.d_out, kBgmvCols);
+    }
+    A.n_chunks = chunks;
+    LF_LAUNCH("bgmv", bgmv_proj_kernel, dim3((unsigned)T, (unsigned)chunks), kBgmvThreads, 0, s, A);
+    return launch_status();
 }
 
 lf_status lf_route_tokens(int32_t T, const int32_t* ids, int32_t n_adapters, void* ws, size_t ws_bytes,

@@ -66,6 +66,15 @@ class lf_slice(ctypes.Structure):
                 ("pool_elems_A", ctypes.c_int64), ("pool_elems_Bt", ctypes.c_int64)]
 
 
+class lf_projection(ctypes.Structure):
+    """One projection of lf_lora_shrink_expand_projections (mirrors the C struct)."""
+    _fields_ = [("x", ctypes.c_void_p), ("y", ctypes.c_void_p), ("d_in", ctypes.c_int32),
+                ("reserved", ctypes.c_int32), ("y_ld", ctypes.c_int64), ("slice", lf_slice)]
+
+
+MAX_PROJECTIONS = 8
+
+
 class LFError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
@@ -115,6 +124,8 @@ def lib() -> ctypes.CDLL:
         L.lf_lora_shrink_expand_slices_routed.argtypes = [_I32, _I32, _P, _P, _I64, _P, _I32, _P, _I32,
                                                           ctypes.c_float, _P, _P, _SZ, _P]
         L.lf_lora_shrink_expand_slices_routed.restype = ctypes.c_int
+        L.lf_lora_shrink_expand_projections.argtypes = [_I32, _P, _I32, _P, _I32, ctypes.c_float, _P, _P, _SZ, _P]
+        L.lf_lora_shrink_expand_projections.restype = ctypes.c_int
         L.lf_jd_workspace_size.argtypes = [_P, _I32, _P, _I32, _P, _I32]; L.lf_jd_workspace_size.restype = _SZ
         L.lf_jd_full.argtypes = [_P, _I32, _P, _I32, _P, _I32, _P, _P, _P, _I32, _P, _P, _P, _P, _SZ, _P]
         L.lf_jd_full.restype = ctypes.c_int
@@ -143,7 +154,7 @@ def exported_symbols() -> list[str]:
             "lf_lora_shrink_expand_noalloc", "lf_apply_slices_workspace_size", "lf_lora_shrink_expand_slices",
             "lf_lora_sigma_sandwich", "lf_jd_workspace_size", "lf_jd_full", "lf_route_tokens",
             "lf_lora_shrink_expand_slices_routed", "lf_check_bounded_wait", "lf_pool_workspace_size",
-            "lf_pool_subspace"]
+            "lf_pool_subspace", "lf_lora_shrink_expand_projections"]
 
 # Limits of lf_lora_shrink_expand_noalloc (its scratch is a fixed array in the library).
 NOALLOC_MAX_TOKENS = 16384
@@ -285,6 +296,22 @@ def lf_lora_shrink_expand_slices_routed(x, y, ids, n_adapters, slices, scale, ws
                                                    len(slices), float(scale), _ptr(adapter_scale), _ptr(ws),
                                                    ws.numel() if ws is not None else 0, _stream(stream))
     return _check(st, "lf_lora_shrink_expand_slices_routed") if check else st
+
+
+def make_projection(x, y, sl: lf_slice) -> lf_projection:
+    """lf_projection from device tensors: x T x d_in bf16, y T x y_ld bf16, and the slice
+    (make_slice) saying where in y and with which factors."""
+    return lf_projection(_ptr(x), _ptr(y), int(x.shape[1]), 0, int(y.shape[1]), sl)
+
+
+def lf_lora_shrink_expand_projections(T, ids, n_adapters, projections, scale, ws=None, adapter_scale=None,
+                                      stream=None, check=True) -> int:
+    """Up to MAX_PROJECTIONS projections (make_projection) of one token batch in one call."""
+    arr = (lf_projection * len(projections))(*projections)
+    st = lib().lf_lora_shrink_expand_projections(int(T), _ptr(ids), n_adapters, arr, len(projections), float(scale),
+                                                 _ptr(adapter_scale), _ptr(ws), ws.numel() if ws is not None else 0,
+                                                 _stream(stream))
+    return _check(st, "lf_lora_shrink_expand_projections") if check else st
 
 
 def lf_lora_sigma_sandwich(x, y, ids, n_adapters, Vt, Ut, sigma, diagonal, scale, ws, stream=None,

@@ -445,3 +445,81 @@ def test_mixed_batch_with_many_resident_adapters_reaches_tensor_cores():
     check_routing(seg, ids, n)
     assert_close(y, oracle_y(x, y0, ids, ranks, offA, offB, Ap, Bt, 2.0))
     assert torch.equal(y[torch.from_numpy(ids < 0)], y0[torch.from_numpy(ids < 0)])
+
+
+def _layer_projections(T, n, key, d_h=512, d_kv=128, d_ffn=1368):
+    """A small layer: q, k, v (one y, slices with gaps), o, gate and up (one y), down; x_h
+    feeds q/k/v/gate/up, x_o feeds o, x_f feeds down.  Per projection: (x, y0, slice dict)."""
+    x_h = synth.normal_bf16((T, d_h), key + (1,))
+    x_o = synth.normal_bf16((T, d_h), key + (2,))
+    x_f = synth.normal_bf16((T, d_ffn), key + (3,))
+    out = []
+    for gi, (x, widths) in enumerate([(x_h, [d_h, d_kv, d_kv]), (x_o, [d_h]), (x_h, [d_ffn, d_ffn]), (x_f, [d_h])]):
+        sl, y_ld = make_slices(widths, n, x.shape[1], key + (4, gi))
+        y0 = synth.normal_bf16((T, y_ld), key + (5, gi))
+        out.append((x, y0, sl))
+    return out
+
+
+@pytest.mark.parametrize("regime", ["decode", "routed"])
+def test_projections_call_matches_oracle(regime):
+    """Seven projections of a layer (four inputs, four outputs, q/k/v and gate/up as slices
+    of one y) in one lf_lora_shrink_expand_projections call: the same bits as one
+    lf_lora_shrink_expand_slices call per projection, and the oracle per projection."""
+    if regime == "decode":
+        T, n = 200, 64
+        ids = synth.zipf_ids(T, n, 1.0, (15, 0)).copy()
+    else:   # T > 8 n: routed, segments long enough for the tensor-core tiles
+        T, n = 1200, 16
+        ids = np.repeat(np.arange(n, dtype=np.int32), T // n)
+        ids[:300] = synth.zipf_ids(300, n, 1.0, (15, 1))
+    ids[np.random.default_rng(15).random(T) < 0.05] = -1
+    ids_d = torch.from_numpy(ids).cuda()
+    layer = _layer_projections(T, n, (15, 2, T))
+    asc = torch.from_numpy((0.5 + np.arange(n) / n).astype(np.float32)).cuda()
+    projs, alive, ys, ys_ref = [], [], [], []
+    for x, y0, sl in layer:
+        xd = x.cuda()
+        keep, tens = _slice_tensors(sl)
+        alive += [xd, tens]
+        y = y0.cuda()
+        ys.append(y)
+        for s in keep:
+            projs.append(lf.make_projection(xd, y, s))
+        y_ref = y0.cuda()
+        lf.lf_lora_shrink_expand_slices(xd, y_ref, ids_d, n, keep, 1.0,
+                                        api.workspace(lf.lf_apply_slices_workspace_size(T, n, len(keep)), "cuda"),
+                                        adapter_scale=asc)
+        ys_ref.append(y_ref)
+    assert len(projs) == 7
+    ws = api.workspace(lf.lf_apply_workspace_size(T, n), "cuda") if regime == "routed" else None
+    l0 = lf.lf_launch_count()
+    lf.lf_lora_shrink_expand_projections(T, ids_d, n, projs, 1.0, ws, adapter_scale=asc)
+    launches = lf.lf_launch_count() - l0
+    assert lf.lf_get_device_status() == 0
+    if regime == "decode":
+        assert launches == 1
+    for (x, y0, sl), y, y_ref in zip(layer, ys, ys_ref):
+        # one projection at a time against the per-slice call and the oracle
+        assert torch.equal(y, y_ref)
+        check_slices(y.cpu(), y0, oracle_slices(x, y0, ids, sl, 1.0, asc.cpu().numpy()), sl, ids)
+
+
+def test_projections_call_host_checks():
+    """Host errors come back before anything runs: a misaligned y, too many projections,
+    a nonzero reserved field."""
+    T, n = 64, 16
+    ids_d = torch.from_numpy(synth.zipf_ids(T, n, 1.0, (16, 0))).cuda()
+    (x, y0, sl), = _layer_projections(T, n, (16, 1))[1:2]
+    keep, _alive = _slice_tensors(sl)
+    xd, y = x.cuda(), y0.cuda()
+    good = lf.make_projection(xd, y, keep[0])
+    assert lf.lf_lora_shrink_expand_projections(T, ids_d, n, [good] * 9, 1.0, check=False) == 1
+    bad = lf.make_projection(xd, y, keep[0])
+    bad.y = bad.y + 2   # not 16-byte aligned
+    assert lf.lf_lora_shrink_expand_projections(T, ids_d, n, [good, bad], 1.0, check=False) == 8   # LF_ERR_ALIGNMENT
+    res = lf.make_projection(xd, y, keep[0])
+    res.reserved = 1
+    assert lf.lf_lora_shrink_expand_projections(T, ids_d, n, [res], 1.0, check=False) == 1
+    torch.cuda.synchronize()
+    assert torch.equal(y.cpu(), y0)
