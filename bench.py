@@ -189,6 +189,13 @@ def dominant_roofline(dom, per_launch_ms, fr, hbm, peak_kind, sm_mhz):
                 "algo_flops": int(flops), "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 x SM clock",
                 "hbm": {"achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s", "frac": round(gbs / hbm, 4),
                         "algo_bytes": int(fr["bytes_in"]), "peak_source": peak_kind}}
+    if dom == "tsqr_gram_i8":
+        # every B and A^T row of the eligible matrices (all of this workload's) read once
+        b = fr["bytes_in"]
+        ach = b / (per_launch_ms * 1e-3) / 1e9
+        return {"kernel": dom, "bound": "hbm", "achieved": round(ach, 1), "peak": hbm, "unit": "GB/s",
+                "frac": round(ach / hbm, 4), "traffic": kernel_traffic(dom, n), "algo_bytes": int(b),
+                "peak_source": peak_kind}
     algo = {"export_stream": fr["bytes_in"] + fr["bytes_out"]}
     b = algo.get(dom)
     if b is None:
@@ -325,7 +332,53 @@ def apply_bytes(T, d_in, d_out, ranks_used):
     return 2 * T * d_in + 4 * T * d_out + 4 * T + sum(2 * k * (d_in + d_out) for k in ranks_used)
 
 
-def decode_bench(args, dev, stream, hbm, variant="ragged", fused=False, per_layer=True):
+def _decode_e2e(args, calls, ids, ids_d, T, stream):
+    """The decode step through the public call with host buffers: per step the token ids,
+    every layer's inputs x and outputs y go up from pinned host memory, the 32
+    lf_lora_shrink_expand_projections calls run, and every y comes back (y is updated in
+    place, so it travels both ways).  Device-timed with events around the whole step."""
+    import torch
+    xs, ys = {}, {}
+    for c in calls:
+        for x, y, _ in c.items:
+            xs.setdefault(x.data_ptr(), x)
+            ys.setdefault(y.data_ptr(), y)
+    xh = {k: v.cpu().pin_memory() for k, v in xs.items()}
+    yh = {k: v.cpu().pin_memory() for k, v in ys.items()}
+    yo = {k: torch.empty_like(v).pin_memory() for k, v in yh.items()}
+    ids_h = torch.from_numpy(np.asarray(ids, np.int32)).pin_memory()
+
+    def step():
+        with torch.cuda.stream(stream):
+            ids_d.copy_(ids_h, non_blocking=True)
+            for c in calls:
+                for p in {x.data_ptr() for x, _, _ in c.items}:
+                    xs[p].copy_(xh[p], non_blocking=True)
+                for p in {y.data_ptr() for _, y, _ in c.items}:
+                    ys[p].copy_(yh[p], non_blocking=True)
+                c(stream)
+                for p in {y.data_ptr() for _, y, _ in c.items}:
+                    yo[p].copy_(ys[p], non_blocking=True)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    reps = max(args.steps, 5)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / reps
+    h2d = ids_h.numel() * 4 + sum(v.numel() * 2 for v in xh.values()) + sum(v.numel() * 2 for v in yh.values())
+    d2h = sum(v.numel() * 2 for v in yo.values())
+    return {"value": round(T / (ms * 1e-3), 1), "unit": "tokens/s", "ms_per_step": round(ms, 3),
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+            "sample": "the whole decode step (32 layers) from pinned host memory"}
+
+
+def decode_bench(args, dev, stream, hbm, variant="ragged", fused=False, per_layer=True, e2e=False):
     """Config 3: Llama-3-8B shapes, 32 layers x 7 projections, T=256, 128 adapters.
     variant: "ragged" (retained ranks as allocated), "padded" (every adapter's factors
     of a projection zero-padded to the largest retained rank over the 128 resident
@@ -387,6 +440,8 @@ def decode_bench(args, dev, stream, hbm, variant="ragged", fused=False, per_laye
         workload="decode: Llama-3-8B, 32 layers x 7 projections, 256 tokens, 128 adapters Zipf(1), "
                  + names[variant] + how,
         distinct_adapters=len(distinct), mean_rank=float(ranks_all.mean())))
+    if e2e and per_layer:
+        out["e2e"] = _decode_e2e(args, calls, ids, ids_d, T, stream)
     del calls
     torch.cuda.empty_cache()
     return out
@@ -505,6 +560,7 @@ def _projections_call(items, ids_d, n_ad, T, ws, scale=2.0):
 
     def run(st=None, _keep=items):
         lf.lf_lora_shrink_expand_projections(T, ids_d, n_ad, projs, scale, ws, stream=st)
+    run.items = items
     return run
 
 
@@ -1149,7 +1205,7 @@ def main():
 
     lora = None
     if not args.no_apply and rank == 0:   # per-GPU side-path figures: rank 0 only
-        lora = {"decode": decode_bench(args, dev, stream, hbm),
+        lora = {"decode": decode_bench(args, dev, stream, hbm, e2e=not args.no_e2e),
                 "decode_padded_to_max": decode_bench(args, dev, stream, hbm, "padded"),
                 "decode_uncompressed_r64": decode_bench(args, dev, stream, hbm, "r64"),
                 "decode_fused_slices": decode_bench(args, dev, stream, hbm, fused=True),
