@@ -676,9 +676,19 @@ static lf_status apply_impl(int32_t T, int32_t d_in, const void* x, void* y, int
                   xmap, x_tma);
     }
     LF_CUDA_TRY(cudaGetLastError());
-    LF_CUDA_TRY(cudaFuncSetAttribute(expand_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kExpandTcSmem));
-    LF_LAUNCH("expand_tc", expand_tc_kernel, dim3(max_tc, (unsigned)A.n_chunks), kTcExpThreads, kExpandTcSmem, s, A,
-              ymap, y_tma);
+    // two expand variants over the same grid, each taking its own (item, slice) pairs:
+    // ranks up to 16 (three CTAs per SM) and the others (two), both in 64-column steps
+    {
+        constexpr size_t sm16 = expand_tc_smem<16, 64>(), sm64 = expand_tc_smem<kMaxRank, 64>();
+        LF_CUDA_TRY(cudaFuncSetAttribute(expand_tc_kernel<16, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm16));
+        LF_CUDA_TRY(cudaFuncSetAttribute(expand_tc_kernel<kMaxRank, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)sm64));
+        LF_LAUNCH("expand_tc", (expand_tc_kernel<16, 64>), dim3(max_tc, (unsigned)A.n_chunks), kTcExpThreads, sm16, s,
+                  A, ymap, y_tma);
+        LF_CUDA_TRY(cudaGetLastError());
+        LF_LAUNCH("expand_tc", (expand_tc_kernel<kMaxRank, 64>), dim3(max_tc, (unsigned)A.n_chunks), kTcExpThreads,
+                  sm64, s, A, ymap, y_tma);
+    }
     return launch_status();
 }
 

@@ -275,18 +275,21 @@ constexpr size_t shrink_tc_smem() { return sizeof(ShrinkTcSmem<MAXN>) + 1024; }
 //   back: by two TMA stores when it is a full TMA tile (128 tokens, 128 columns
 //   inside the CTA's range), else with 16-byte stores of its rows < ntok and columns
 //   in range (rows past the tile belong to other CTAs and are never written).
-constexpr int kTcN2 = 128;                  // expand step width (UMMA N)
 constexpr int kTcYBuf = 3;
 constexpr int kTcExpThreads = 256;
 constexpr uint32_t kTcYHalf = kTcM * 128;   // bytes of one 64-column half of a staged y tile
+// KMAX: largest rank the variant takes (64: every rank, 97 KB of shared memory, two CTAs
+// per SM; 16: ranks up to 16, 62 KB, three CTAs per SM); N2: expand step width (UMMA N).
+template <int KMAX, int N2>
 struct ExpandTcSmem {
-    __nv_bfloat16 ahi[kTcM * kMaxRank];          // t_hi, K-major, 16 KB
-    __nv_bfloat16 alo[kTcM * kMaxRank];          // t_lo
-    __nv_bfloat16 b[2][kMaxRank * kTcN2];        // B'^T tiles, MN-major, 16 KB each
+    __nv_bfloat16 ahi[kTcM * KMAX];              // t_hi, K-major
+    __nv_bfloat16 alo[kTcM * KMAX];              // t_lo
+    __nv_bfloat16 b[2][KMAX * N2];               // B'^T tiles, MN-major
     union {
-        __nv_bfloat16 yt[kTcYBuf][kTcM * kTcN2];     // staged y tiles, 32 KB each (64 KB into the block:
-                                                     // 1024-byte aligned when the block is; checked before TMA)
-        float tw[kTcM][kMaxRank + 1];                // summed t rows (Sigma-sandwich only, prologue), 33 KB
+        __nv_bfloat16 yt[kTcYBuf][kTcM * N2];        // staged y tiles (1024-byte aligned when the block
+                                                     // is: the members above are multiples of 1 KB;
+                                                     // checked before TMA)
+        float tw[kTcM][kMaxRank + 1];                // summed t rows (Sigma-sandwich only, prologue)
     };
     uint64_t bar;
     uint64_t ybar[kTcYBuf];   // TMA y tiles (tx bytes)
@@ -304,10 +307,14 @@ __device__ __forceinline__ uint32_t ytile_off(int row, int col) {
 }
 
 // y_tma: the caller encoded `ymap` (y as y_ld x T bf16, box 64 x 128, 128-byte swizzle).
-__global__ void __launch_bounds__(kTcExpThreads, 1) expand_tc_kernel(ApplyArgs a, const __grid_constant__ CUtensorMap ymap,
-                                                                     int y_tma) {
+// The two variants split the (item, slice) pairs between them: KMAX = 16 takes ranks up
+// to 16 (without Sigma-sandwich), KMAX = 64 the rest.
+template <int KMAX, int N2>
+__global__ void __launch_bounds__(kTcExpThreads, KMAX == 16 ? 3 : 2)
+    expand_tc_kernel(ApplyArgs a, const __grid_constant__ CUtensorMap ymap, int y_tma) {
+    static_assert(N2 % 64 == 0 && N2 <= 128, "steps of whole 64-column halves");
     extern __shared__ __align__(1024) unsigned char tc_raw[];
-    auto& s = *reinterpret_cast<ExpandTcSmem*>(tc_raw);
+    auto& s = *reinterpret_cast<ExpandTcSmem<KMAX, N2>*>(tc_raw);
     if ((int)blockIdx.x >= a.counts[3]) return;
     const TcItem it = a.tc_items[blockIdx.x];
     const int sl = slice_of_chunk(a, blockIdx.y);
@@ -315,10 +322,12 @@ __global__ void __launch_bounds__(kTcExpThreads, 1) expand_tc_kernel(ApplyArgs a
     int k;
     int64_t oa, ob;
     if (!slice_factors(a, sl, it.adapter, false, k, oa, ob)) return;   // reported by the shrink
+    const bool small = k <= 16 && a.sigma_mode == 0;
+    if (small != (KMAX == 16)) return;   // the other variant's pair
     const int e_begin = ((int)blockIdx.y - S.chunk0) * kTcCols;
     if (e_begin >= S.d_out) return;
     const int e_end = min(S.d_out, e_begin + kTcCols);
-    const int nit = (e_end - e_begin + kTcN2 - 1) / kTcN2;
+    const int nit = (e_end - e_begin + N2 - 1) / N2;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int nt = it.ntok;
     const float scale = adapter_scale(a, it.adapter);
@@ -374,7 +383,7 @@ __global__ void __launch_bounds__(kTcExpThreads, 1) expand_tc_kernel(ApplyArgs a
         *reinterpret_cast<uint4*>(reinterpret_cast<char*>(s.ahi) + off) = *reinterpret_cast<const uint4*>(hi);
         *reinterpret_cast<uint4*>(reinterpret_cast<char*>(s.alo) + off) = *reinterpret_cast<const uint4*>(lo);
     }
-    if (warp == 0) tc::tmem_alloc(&s.tmem, kTcN2);
+    if (warp == 0) tc::tmem_alloc(&s.tmem, N2);
     if (tid == 0) {
         mbar_init(&s.bar, 1);
         for (int b2 = 0; b2 < kTcYBuf; ++b2) mbar_init(&s.ybar[b2], 1);
@@ -389,32 +398,33 @@ __global__ void __launch_bounds__(kTcExpThreads, 1) expand_tc_kernel(ApplyArgs a
 
     const __nv_bfloat16* Bt = S.Bt_pool + ob;
     auto issue_y = [&](int i) {   // y rows of step i -> yt[i % 3]
-        const int e0 = e_begin + i * kTcN2;
+        const int e0 = e_begin + i * N2;
         char* dst = reinterpret_cast<char*>(s.yt[i % kTcYBuf]);
         if (ytma) {   // rows toks[0] .. +127, columns y_off + e0 .. +127 (a multiple of 8 elements)
             if (tid == 0) {
                 tc::bulk_wait_read0();   // the TMA store of the tile this buffer held has read it
                 uint64_t* bar = &s.ybar[i % kTcYBuf];
-                mbar_arrive_expect_tx(bar, 2 * kTcYHalf);
-                tc::tma_load_2d(dst, &ymap, (int)S.y_off + e0, s.toks[0], bar);
-                tc::tma_load_2d(dst + kTcYHalf, &ymap, (int)S.y_off + e0 + 64, s.toks[0], bar);
+                mbar_arrive_expect_tx(bar, (N2 / 64) * kTcYHalf);
+#pragma unroll
+                for (int hh = 0; hh < N2 / 64; ++hh)
+                    tc::tma_load_2d(dst + hh * kTcYHalf, &ymap, (int)S.y_off + e0 + 64 * hh, s.toks[0], bar);
                 ++y_issued;
             }
             return;
         }
         // rows past the tile / columns past the range zero-filled
-        for (int c = tid; c < kTcM * (kTcN2 / 8); c += kTcExpThreads) {
-            const int row = c / (kTcN2 / 8), ch = c % (kTcN2 / 8);
+        for (int c = tid; c < kTcM * (N2 / 8); c += kTcExpThreads) {
+            const int row = c / (N2 / 8), ch = c % (N2 / 8);
             const int e = e0 + ch * 8;
             const bool ok = row < nt && e < e_end;
             cp_async16_zfill(dst + ytile_off(row, ch * 8), ok ? ybase + (int64_t)s.toks[row] * a.y_ld + e : ybase, ok);
         }
     };
     auto issue_b = [&](int i) {   // B'^T rows 0..kpad-1 of step i -> b[i % 2], MN-major
-        const int e0 = e_begin + i * kTcN2;
+        const int e0 = e_begin + i * N2;
         char* dst = reinterpret_cast<char*>(s.b[i & 1]);
-        for (int c = tid; c < kpad * (kTcN2 / 8); c += kTcExpThreads) {
-            const int j = c / (kTcN2 / 8), nc = c % (kTcN2 / 8);
+        for (int c = tid; c < kpad * (N2 / 8); c += kTcExpThreads) {
+            const int j = c / (N2 / 8), nc = c % (N2 / 8);
             const int e = e0 + nc * 8;
             const bool ok = j < k && e < e_end;
             cp_async16_zfill(dst + (uint32_t)nc * sbo + (uint32_t)(j >> 3) * 128 + (uint32_t)(j & 7) * 16,
@@ -433,7 +443,7 @@ __global__ void __launch_bounds__(kTcExpThreads, 1) expand_tc_kernel(ApplyArgs a
     __syncthreads();
     tc::fence_after_sync();
     const uint32_t tmem = s.tmem;
-    const uint32_t idesc = tc::idesc_bf16(kTcM, kTcN2, 0, 1);
+    const uint32_t idesc = tc::idesc_bf16(kTcM, N2, 0, 1);
     const int q = warp & 3, h = warp >> 2;   // TMEM lane quadrant, column half
     const int m = 32 * q + lane;             // tile row of this thread in the epilogue
     bool ok = true;
@@ -463,13 +473,13 @@ __global__ void __launch_bounds__(kTcExpThreads, 1) expand_tc_kernel(ApplyArgs a
         __nv_bfloat16* yt = s.yt[i % kTcYBuf];
         if (ok) {
 #pragma unroll
-            for (int c16 = 0; c16 < kTcN2 / 32; ++c16) {
+            for (int c16 = 0; c16 < N2 / 32; ++c16) {
                 float v[16];
-                tc::tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)((kTcN2 / 2) * h + 16 * c16), v);
+                tc::tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)((N2 / 2) * h + 16 * c16), v);
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
                     uint4* yp = reinterpret_cast<uint4*>(reinterpret_cast<char*>(yt) +
-                                                         ytile_off(m, (kTcN2 / 2) * h + 16 * c16 + 8 * half));
+                                                         ytile_off(m, (N2 / 2) * h + 16 * c16 + 8 * half));
                     uint4 yv = *yp;
                     __nv_bfloat162* y2 = reinterpret_cast<__nv_bfloat162*>(&yv);
 #pragma unroll
@@ -486,17 +496,18 @@ __global__ void __launch_bounds__(kTcExpThreads, 1) expand_tc_kernel(ApplyArgs a
         tc::fence_before_sync();
         ok = __syncthreads_and(ok);          // staged tile complete; TMEM free for the next MMA
         if (ok) {
-            const int e0 = e_begin + i * kTcN2;
-            if (ytma && nt == kTcM && e0 + kTcN2 <= e_end) {   // the whole box is this CTA's
+            const int e0 = e_begin + i * N2;
+            if (ytma && nt == kTcM && e0 + N2 <= e_end) {   // the whole box is this CTA's
                 if (tid == 0) {
                     const char* src = reinterpret_cast<const char*>(yt);
-                    tc::tma_store_2d(&ymap, (int)S.y_off + e0, s.toks[0], src);
-                    tc::tma_store_2d(&ymap, (int)S.y_off + e0 + 64, s.toks[0], src + kTcYHalf);
+#pragma unroll
+                    for (int hh = 0; hh < N2 / 64; ++hh)
+                        tc::tma_store_2d(&ymap, (int)S.y_off + e0 + 64 * hh, s.toks[0], src + hh * kTcYHalf);
                     tc::bulk_commit();
                 }
             } else {
-                for (int c = tid; c < kTcM * (kTcN2 / 8); c += kTcExpThreads) {
-                    const int row = c / (kTcN2 / 8), ch = c % (kTcN2 / 8);
+                for (int c = tid; c < kTcM * (N2 / 8); c += kTcExpThreads) {
+                    const int row = c / (N2 / 8), ch = c % (N2 / 8);
                     const int e = e0 + ch * 8;
                     if (row < nt && e < e_end)
                         *reinterpret_cast<uint4*>(ybase + (int64_t)s.toks[row] * a.y_ld + e) =
@@ -515,9 +526,10 @@ __global__ void __launch_bounds__(kTcExpThreads, 1) expand_tc_kernel(ApplyArgs a
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
-    if (warp == 0) tc::tmem_dealloc(tmem, kTcN2);
+    if (warp == 0) tc::tmem_dealloc(tmem, N2);
 }
 
-constexpr size_t kExpandTcSmem = sizeof(ExpandTcSmem) + 1024;
+template <int KMAX, int N2>
+constexpr size_t expand_tc_smem() { return sizeof(ExpandTcSmem<KMAX, N2>) + 1024; }
 
 }  // namespace lf
