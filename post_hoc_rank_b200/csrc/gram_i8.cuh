@@ -55,8 +55,8 @@ namespace lf {
 
 constexpr int kI8Rows = 128;         // rows (the MMA's K) per digit stage
 constexpr int kI8FRows = 64;         // rows per fp32 stage (two per digit stage)
-constexpr int kI8FStages = 7;
-constexpr int kI8DStages = 2;
+constexpr int kI8FStages = 5;
+constexpr int kI8DStages = 3;
 constexpr int kI8ConvWarps = 16;
 constexpr int kI8EpiWarps = 4;
 constexpr int kI8ConvWarp0 = 2;
