@@ -495,18 +495,21 @@ __device__ __forceinline__ void export_stage_b(const ExportArgs& a, const lf_mod
     // directions past k are skipped without divergence (NQ covers the largest k)
     const int nq = min(NQ, max(0, (k - jbase - g + 3) / 4));
     if (nq == 0) return;
-    float acc[NQ];
+    // packed fp32 pairs: even and odd columns in two chains, added at the end
+    float2 acc[NQ];
 #pragma unroll
-    for (int q = 0; q < NQ; ++q) acc[q] = 0.f;
+    for (int q = 0; q < NQ; ++q) acc[q] = make_float2(0.f, 0.f);
     const float* row = st + e * kMaxRank;
 #pragma unroll 4
     for (int c = 0; c < 16; ++c) {
         const float4 x = *reinterpret_cast<const float4*>(row + 4 * (c ^ (e & 7)));
+        const float2 x01 = make_float2(x.x, x.y), x23 = make_float2(x.z, x.w);
 #pragma unroll
         for (int q = 0; q < NQ; ++q) {
             if (q < nq) {
                 const float4 cf = *reinterpret_cast<const float4*>(coef + (jbase + g + 4 * q) * kMaxRank + 4 * c);
-                acc[q] = fmaf(cf.x, x.x, fmaf(cf.y, x.y, fmaf(cf.z, x.z, fmaf(cf.w, x.w, acc[q]))));
+                acc[q] = __ffma2_rn(make_float2(cf.x, cf.y), x01, acc[q]);
+                acc[q] = __ffma2_rn(make_float2(cf.z, cf.w), x23, acc[q]);
             }
         }
     }
@@ -515,9 +518,10 @@ __device__ __forceinline__ void export_stage_b(const ExportArgs& a, const lf_mod
     for (int q = 0; q < NQ; ++q) {
         const int j = jbase + g + 4 * q;
         if (j < k) {
+            const float v = acc[q].x + acc[q].y;
             const int64_t o = obase + (int64_t)j * md.d_out + i0 + e;
-            a.Bt_pool[o] = acc[q];
-            if (a.Bt_pool16) a.Bt_pool16[o] = __float2bfloat16_rn(acc[q]);
+            a.Bt_pool[o] = v;
+            if (a.Bt_pool16) a.Bt_pool16[o] = __float2bfloat16_rn(v);
         }
     }
 }
@@ -568,7 +572,7 @@ __device__ void export_item_a(const ExportArgs& a, const lf_module& md, int k, c
         if (s < nst) issue(s);
         tc::cp_async_commit();
     }
-    float acc[kExpAJ];
+    float2 acc[kExpAJ / 2];   // packed pairs of retained directions (2p, 2p + 1)
     for (int t = 0; t < nst; ++t) {
         tc::cp_async_wait<kExpStages - 2>();
         __syncthreads();
@@ -579,24 +583,27 @@ __device__ void export_item_a(const ExportArgs& a, const lf_module& md, int k, c
         const int j0 = pass * kExpAJ;
         if (lq == 0) {
 #pragma unroll
-            for (int jj = 0; jj < kExpAJ; ++jj) acc[jj] = 0.f;
+            for (int jp = 0; jp < kExpAJ / 2; ++jp) acc[jp] = make_float2(0.f, 0.f);
         }
         const float* st = stages + (t % kExpStages) * kExpStageFloats;
         float x[kExpALRows];
 #pragma unroll
         for (int l = 0; l < kExpALRows; ++l) x[l] = st[l * kExpACols + tid];
         const int nj = min(kExpAJ, k - j0);
+        // coefficients pair-interleaved: float2 (C[2p][l], C[2p + 1][l]) at p * 64 + l
+        const float4* cp4 = reinterpret_cast<const float4*>(coef);
 #pragma unroll
-        for (int jj = 0; jj < kExpAJ; ++jj) {
-            if (jj < nj) {
-                const float* cr = coef + (j0 + jj) * kMaxRank + kExpALRows * lq;
-                float t4 = acc[jj];
+        for (int jp = 0; jp < kExpAJ / 2; ++jp) {
+            if (2 * jp < nj) {
+                const int p = j0 / 2 + jp;
+                float2 t2 = acc[jp];
 #pragma unroll
-                for (int l4 = 0; l4 < kExpALRows / 4; ++l4) {
-                    const float4 cf = *reinterpret_cast<const float4*>(cr + 4 * l4);
-                    t4 = fmaf(cf.x, x[4 * l4], fmaf(cf.y, x[4 * l4 + 1], fmaf(cf.z, x[4 * l4 + 2], fmaf(cf.w, x[4 * l4 + 3], t4))));
+                for (int l2 = 0; l2 < kExpALRows / 2; ++l2) {
+                    const float4 cf = cp4[p * (kMaxRank / 2) + (kExpALRows * lq) / 2 + l2];
+                    t2 = __ffma2_rn(make_float2(cf.x, cf.y), make_float2(x[2 * l2], x[2 * l2]), t2);
+                    t2 = __ffma2_rn(make_float2(cf.z, cf.w), make_float2(x[2 * l2 + 1], x[2 * l2 + 1]), t2);
                 }
-                acc[jj] = t4;
+                acc[jp] = t2;
             }
         }
         if (lq == 3) {
@@ -605,9 +612,10 @@ __device__ void export_item_a(const ExportArgs& a, const lf_module& md, int k, c
 #pragma unroll
                 for (int jj = 0; jj < kExpAJ; ++jj) {
                     if (jj < nj) {
+                        const float v = (jj & 1) ? acc[jj >> 1].y : acc[jj >> 1].x;
                         const int64_t o = obase + (int64_t)(j0 + jj) * md.d_in + d;
-                        a.A_pool[o] = acc[jj];
-                        if (a.A_pool16) a.A_pool16[o] = __float2bfloat16_rn(acc[jj]);
+                        a.A_pool[o] = v;
+                        if (a.A_pool16) a.A_pool16[o] = __float2bfloat16_rn(v);
                     }
                 }
             }
@@ -639,7 +647,11 @@ __global__ void __launch_bounds__(kExpThreads, 3) export_kernel(ExportArgs a) {
                                   : (k <= 4 ? 4 : (k <= 8 ? 8 : (k <= 16 ? 16 : kMaxRank)));   // rows the stages read
     for (int e = threadIdx.x; e < kfill * kMaxRank; e += kExpThreads) {
         const int j = e / kMaxRank, l = e % kMaxRank;
-        coef[e] = (j < k && l < r) ? C[j * a.rs + l] : 0.f;
+        const float v = (j < k && l < r) ? C[j * a.rs + l] : 0.f;
+        if (w.part == 1)   // A part: pair-interleaved, float2 (C[2p][l], C[2p + 1][l]) at p * 64 + l
+            coef[(j >> 1) * 2 * kMaxRank + 2 * l + (j & 1)] = v;
+        else
+            coef[e] = v;
     }
     const float* X = w.part == 0 ? a.B_base + md.B_off : a.A_base + md.A_off;
     // coefficient rows are read after the first barrier inside export_item_*
