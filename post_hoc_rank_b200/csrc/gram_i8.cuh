@@ -107,6 +107,13 @@ struct GramI8Args {
 // the columns interleaved in rows 0..127, planes 2, 3 in rows 128..255.
 __device__ __forceinline__ int i8_row(int p, int c) { return (p >> 1) * 128 + 2 * c + (p & 1); }
 
+// max(a, b) that returns NaN when either operand is NaN (fmaxf would return the other).
+__device__ __forceinline__ float fmax_nan(float a, float b) {
+    float d;
+    asm("max.NaN.f32 %0, %1, %2;" : "=f"(d) : "f"(a), "f"(b));
+    return d;
+}
+
 // Barrier among `nthreads` threads on hardware barrier `id` that also ANDs a predicate:
 // every participant gets the same answer.
 __device__ __forceinline__ bool named_and(int id, int nthreads, bool v) {
@@ -376,8 +383,7 @@ __global__ void __launch_bounds__(kI8Threads, 1) gram_i8_kernel(GramI8Args a) {
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const float x = xv[4 * j4 + e];
-                        amax = fmaxf(amax, fabsf(x));
-                        vok = vok && (x == x);   // NaN: fmaxf would drop it
+                        amax = fmax_nan(amax, fabsf(x));   // a NaN stays in amax
                         u[e] = (uint32_t)__float2int_rz(x * mult);
                     }
                     uint32_t wd[4];
@@ -389,7 +395,7 @@ __global__ void __launch_bounds__(kI8Threads, 1) gram_i8_kernel(GramI8Args a) {
                         cs[p] = __dp4a(wd[p], 0x01010101u, cs[p]);
                     }
                 }
-                vok = vok && amax < lim;   // false for infinities as well
+                vok = vok && amax < lim;   // false for infinities and NaN as well
                 // lanes 4..7 of each group of 8 (consecutive columns) store the other plane of
                 // the pair (0 <-> 1, 2 <-> 3) than lanes 0..3, so the eight 16-byte stores of a
                 // group land in eight different swizzled chunks (no bank conflict)
