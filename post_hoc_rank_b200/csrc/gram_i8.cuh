@@ -87,6 +87,7 @@ struct GramI8Smem {
     uint64_t full_d[kI8DStages], empty_d[kI8DStages];
     uint64_t acc_full, acc_empty, drain;
     uint64_t meta_full[2], meta_empty[2];
+    uint64_t cmax_full, cmax_empty;          // the column-maximum exchange of an item's first stage
     uint32_t tmem;
     int abort;
 };
@@ -207,6 +208,8 @@ __global__ void __launch_bounds__(kI8Threads, 1) gram_i8_kernel(GramI8Args a) {
             mbar_init(&s.meta_full[i], kI8ConvWarps);
             mbar_init(&s.meta_empty[i], kI8EpiWarps);
         }
+        mbar_init(&s.cmax_full, kI8ConvWarps);
+        mbar_init(&s.cmax_empty, kI8ConvWarps);
         s.abort = 0;
         fence_barrier_init();
     }
@@ -317,7 +320,6 @@ __global__ void __launch_bounds__(kI8Threads, 1) gram_i8_kernel(GramI8Args a) {
             const int nd = (int)cdiv(w.nrows, kI8Rows);
             const int ms = k & 1;
             if (k >= 2) ok = wait(&s.meta_empty[ms], (uint32_t)(((k >> 1) - 1) & 1));
-            ok = named_and(1, 32 * kI8ConvWarps, ok);
             if (!ok) break;
             GramI8Meta& M = s.meta[ms];
             // this thread's column c and 16-row chunk q of every digit stage (chunk q in
@@ -334,7 +336,6 @@ __global__ void __launch_bounds__(kI8Threads, 1) gram_i8_kernel(GramI8Args a) {
                 const int f0 = g % kI8FStages, f1 = (g + 1) % kI8FStages;
                 ok = wait(&s.full_f[f0], (uint32_t)((g / kI8FStages) & 1)) &&
                      wait(&s.full_f[f1], (uint32_t)(((g + 1) / kI8FStages) & 1));
-                ok = named_and(1, 32 * kI8ConvWarps, ok);
                 if (!ok) break;
                 const int rbase = kI8Rows * ds;
                 // this thread's chunk into registers, then the fp32 stages go back to the
@@ -351,11 +352,20 @@ __global__ void __launch_bounds__(kI8Threads, 1) gram_i8_kernel(GramI8Args a) {
                     float mx = 0.f;
 #pragma unroll
                     for (int e = 0; e < 16; ++e) mx = fmaxf(mx, fabsf(xv[e]));
+                    // exchanged through mbarriers (bounded waits): the previous item's
+                    // readers are done, every warp's maxima are in, then this warp is done
+                    if (k >= 1) ok = wait(&s.cmax_empty, (uint32_t)((k - 1) & 1));
+                    if (!ok) break;
                     s.cmax[q][c] = mx;
-                    tc::named_sync(1, 32 * kI8ConvWarps);
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive1(&s.cmax_full);
+                    ok = wait(&s.cmax_full, (uint32_t)(k & 1));
+                    if (!ok) break;
                     float m = s.cmax[0][c];
 #pragma unroll
                     for (int h = 1; h < 8; ++h) m = fmaxf(m, s.cmax[h][c]);
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive1(&s.cmax_empty);
                     int E = -90;   // an all-zero start: any nonzero value later overflows the scale
                     if (m > 0.f && m <= FLT_MAX) {
                         int e2;
@@ -369,10 +379,8 @@ __global__ void __launch_bounds__(kI8Threads, 1) gram_i8_kernel(GramI8Args a) {
                     mult = __int_as_float((158 - E) << 23);   // 2^(31 - E)
                     lim = __int_as_float((127 + E) << 23);    // 2^E
                     if (q == 0) M.E[c] = E;
-                    tc::named_sync(1, 32 * kI8ConvWarps);     // cmax is rewritten by the next item
                 }
                 if (gd >= kI8DStages) ok = wait(&s.empty_d[gd % kI8DStages], (uint32_t)((gd / kI8DStages - 1) & 1));
-                ok = named_and(1, 32 * kI8ConvWarps, ok);
                 if (!ok) break;
                 uint8_t* dig = s.dig[gd % kI8DStages];
                 uint32_t pw[4][4];
