@@ -77,8 +77,8 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
     if (mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
     for (int i = 0; i < max_polls; ++i) {
-        if (mbar_try_wait(bar, parity)) return true;
-        __nanosleep(32);
+        if (mbar_try_wait(bar, parity)) return true;   // try_wait itself may suspend the thread a while
+        if (i >= 1024) __nanosleep(32);                // a long wait: poll less often
         if ((i & 1023) == 1023 && clock64() - t0 > 2000000000ll) break;
     }
     latch_error(LF_ERR_TIMEOUT);
