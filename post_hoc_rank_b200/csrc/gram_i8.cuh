@@ -152,18 +152,29 @@ __device__ __forceinline__ void i8_load_unit(float (&x)[16], const float* st, in
         return;
     }
     if (factor == 0) {
+        if (nvalid >= 16) {   // every stage but a matrix's last: no row tests
 #pragma unroll
-        for (int e = 0; e < 16; ++e) x[e] = e < nvalid ? st[(16 * qs + e) * r + c] : 0.f;
+            for (int e = 0; e < 16; ++e) x[e] = st[(16 * qs + e) * r + c];
+        } else {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) x[e] = e < nvalid ? st[(16 * qs + e) * r + c] : 0.f;
+        }
     } else {
         const char* row = reinterpret_cast<const char*>(st) + (qs >> 1) * kI8AHalfBytes + c * 128;
+        float4 f[4];
+#pragma unroll
+        for (int v = 0; v < 4; ++v) f[v] = *reinterpret_cast<const float4*>(row + ((((qs & 1) * 4 + v) ^ (c & 7)) << 4));
 #pragma unroll
         for (int v = 0; v < 4; ++v) {
-            const int chunk = (qs & 1) * 4 + v;
-            const float4 f = *reinterpret_cast<const float4*>(row + ((chunk ^ (c & 7)) << 4));
-            x[4 * v + 0] = 4 * v + 0 < nvalid ? f.x : 0.f;
-            x[4 * v + 1] = 4 * v + 1 < nvalid ? f.y : 0.f;
-            x[4 * v + 2] = 4 * v + 2 < nvalid ? f.z : 0.f;
-            x[4 * v + 3] = 4 * v + 3 < nvalid ? f.w : 0.f;
+            x[4 * v + 0] = f[v].x;
+            x[4 * v + 1] = f[v].y;
+            x[4 * v + 2] = f[v].z;
+            x[4 * v + 3] = f[v].w;
+        }
+        if (nvalid < 16) {
+#pragma unroll
+            for (int e = 0; e < 16; ++e)
+                if (e >= nvalid) x[e] = 0.f;
         }
     }
 }
@@ -342,6 +353,14 @@ __global__ void __launch_bounds__(kI8Threads, 1) gram_i8_kernel(GramI8Args a) {
                 // producer before any conversion work
                 float xv[16];
                 i8_load_unit(xv, s.f32[q < 4 ? f0 : f1], factor, c, q & 3, r, w.nrows - rbase - 16 * q);
+                // the magnitude check reads every loaded value, and the empty asm pins it
+                // before the release: the stage goes back to the producer only once this
+                // thread's loads have returned (a shared-memory load still in flight at the
+                // arrive could otherwise read the producer's next copy)
+                float amax = 0.f;
+#pragma unroll
+                for (int e = 0; e < 16; ++e) amax = fmax_nan(amax, fabsf(xv[e]));   // a NaN stays in amax
+                asm volatile("" ::"f"(amax));
                 __syncwarp();
                 if (lane == 0) {
                     mbar_arrive1(&s.empty_f[f0]);
@@ -384,15 +403,12 @@ __global__ void __launch_bounds__(kI8Threads, 1) gram_i8_kernel(GramI8Args a) {
                 if (!ok) break;
                 uint8_t* dig = s.dig[gd % kI8DStages];
                 uint32_t pw[4][4];
-                float amax = 0.f;
 #pragma unroll
                 for (int j4 = 0; j4 < 4; ++j4) {
                     uint32_t u[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        const float x = xv[4 * j4 + e];
-                        amax = fmax_nan(amax, fabsf(x));   // a NaN stays in amax
-                        u[e] = (uint32_t)__float2int_rz(x * mult);
+                        u[e] = (uint32_t)__float2int_rz(xv[4 * j4 + e] * mult);
                     }
                     uint32_t wd[4];
                     planes4(u, wd);
