@@ -533,7 +533,8 @@ def _proj_call(x, y, ids_d, n_ad, rk, oa, ob, Ap, Bt, ws, scale=2.0):
 
 def _slices_call(x, y, ids_d, n_ad, slices, ws, scale=2.0):
     """Projections sharing x through one lf_lora_shrink_expand_slices call; slices:
-    (d_out, y_offset, ranks, off_A, off_Bt, A_pool, Bt_pool) device tensors."""
+    (d_out, y_offset, ranks, off_A, off_Bt, A_pool, Bt_pool, max_rank): device tensors and the
+    largest rank of the slice."""
     from post_hoc_rank_b200 import loraforge as lf
     sl = [lf.make_slice(*t) for t in slices]
 
@@ -554,7 +555,8 @@ def _routed_call(x, y, ids_d, n_ad, slices, ws, scale=2.0):
 
 def _projections_call(items, ids_d, n_ad, T, ws, scale=2.0):
     """Every projection of a layer through one lf_lora_shrink_expand_projections call;
-    items: (x, y, (d_out, y_offset, ranks, off_A, off_Bt, A_pool, Bt_pool)) device tensors."""
+    items: (x, y, (d_out, y_offset, ranks, off_A, off_Bt, A_pool, Bt_pool, max_rank)) device tensors
+    and the largest rank of the projection."""
     from post_hoc_rank_b200 import loraforge as lf
     projs = [lf.make_projection(x, y, lf.make_slice(*t)) for x, y, t in items]
 
@@ -580,7 +582,7 @@ def _layer_calls(groups, x_of, ids_d, n_ad, T, dev, key, fused, route_once=False
             y = synth.normal_bf16((T, d_out), key + (p,), device=dev)
             items.append((x_of(d_in), y, (d_out, 0, torch.from_numpy(rk.astype(np.int32)).to(dev),
                                           torch.from_numpy(offA[:-1]).to(dev), torch.from_numpy(offB[:-1]).to(dev),
-                                          Ap, Bt)))
+                                          Ap, Bt, int(rk.max()))))
         ws = api.workspace(lf.lf_apply_workspace_size(T, n_ad), dev)
         return [_projections_call(items, ids_d, n_ad, T, ws)], sets
     calls = []
@@ -601,13 +603,14 @@ def _layer_calls(groups, x_of, ids_d, n_ad, T, dev, key, fused, route_once=False
         for p in ps:
             _, d_out, rk, offA, offB, Ap, Bt = groups[p]
             tens.append((d_out, y_off, torch.from_numpy(rk.astype(np.int32)).to(dev),
-                         torch.from_numpy(offA[:-1]).to(dev), torch.from_numpy(offB[:-1]).to(dev), Ap, Bt))
+                         torch.from_numpy(offA[:-1]).to(dev), torch.from_numpy(offB[:-1]).to(dev), Ap, Bt,
+                         int(rk.max())))   # the caller's rank bound for the slice
             y_off += d_out
         if route_once:
             calls.append(_routed_call(x, y, ids_d, n_ad, tens, rws))
         elif len(ps) == 1:
             ws = api.workspace(lf.lf_apply_workspace_size(T, n_ad), dev)
-            d_out, _, rk_d, oa_d, ob_d, Ap, Bt = tens[0]
+            d_out, _, rk_d, oa_d, ob_d, Ap, Bt, _ = tens[0]
             calls.append(_proj_call(x, y, ids_d, n_ad, rk_d, oa_d, ob_d, Ap, Bt, ws))
         else:
             ws = api.workspace(lf.lf_apply_slices_workspace_size(T, n_ad, len(ps)), dev)
@@ -1148,6 +1151,8 @@ def main():
     ap.add_argument("--no-jd", action="store_true")
     ap.add_argument("--jd-only", action="store_true", help="run only the JD-Full workload and print its record")
     ap.add_argument("--large-adapters", type=int, default=1024)
+    ap.add_argument("--lora-only", choices=["decode", "decode_per_projection", "prefill_k16", "prefill_r64"],
+                    help="run only this side-path workload and print its record")
     args = ap.parse_args()
 
     rank = int(os.environ.get("RANK", "0"))
@@ -1164,6 +1169,21 @@ def main():
         torch.cuda.set_device(dev)
         hbm, _ = peaks()
         print(json.dumps(jd_bench(dev, torch.cuda.current_stream(), hbm, None, with_cpu=not args.no_cpu)))
+        return
+
+    if args.lora_only:
+        import torch
+        from post_hoc_rank_b200 import build as B
+        B.build()
+        dev = torch.device("cuda", local)
+        torch.cuda.set_device(dev)
+        hbm, _ = peaks()
+        stream = torch.cuda.Stream()
+        fn = {"decode": lambda: decode_bench(args, dev, stream, hbm),
+              "decode_per_projection": lambda: decode_bench(args, dev, stream, hbm, per_layer=False),
+              "prefill_k16": lambda: prefill_bench(args, dev, stream, hbm, 16),
+              "prefill_r64": lambda: prefill_bench(args, dev, stream, hbm, 64)}[args.lora_only]
+        print(json.dumps(fn()))
         return
 
     import torch

@@ -217,7 +217,11 @@ lf_status lf_lora_shrink_expand(int32_t T, int32_t d_in, int32_t d_out,
  * Workspace: lf_apply_slices_workspace_size(T, n_adapters, n_slices). */
 typedef struct {
     int32_t d_out;              /* output columns of the slice */
-    int32_t reserved;           /* 0 */
+    int32_t max_rank;           /* 0, or an upper bound (1..64) of every adapter's rank in this slice:
+                                   a launch may then leave out kernels sized for larger ranks (on the
+                                   tensor-core path a bound <= 16 keeps only the rank-16 expand); an
+                                   adapter whose rank exceeds it latches LF_ERR_SHAPE and its tokens
+                                   are left untouched in this slice */
     int64_t y_offset;           /* first column of the slice in each row of y */
     const int32_t* ranks;       /* per adapter: retained rank of this slice's module */
     const int64_t* off_A;       /* per adapter: element offset of A' (k x d_in) in A_pool */
@@ -251,7 +255,7 @@ lf_status lf_lora_shrink_expand_slices(int32_t T, int32_t d_in, const void* x, v
  * lf_apply_workspace_size(T, n_adapters) bytes.  Projections must not write
  * overlapping parts of any y, and no y may overlap an x of the same call.
  * Per projection the argument rules of lf_lora_shrink_expand_slices with one slice
- * apply (reserved fields 0); host errors are returned before anything is launched,
+ * apply (the projection's reserved field 0); host errors are returned before anything is launched,
  * and device-side errors latch as there, per (adapter, projection). */
 #define LF_MAX_PROJECTIONS 8
 typedef struct {

@@ -632,7 +632,8 @@ __global__ void __launch_bounds__(kBgmvThreads, 2) bgmv_proj_kernel(ProjArgs a) 
     }
     int k;
     int64_t oa, ob;
-    if (!factor_lookup(P.ranks, P.off_A, P.off_Bt, 0, P.d_in, P.d_out, P.pool_A, P.pool_Bt, ad, lead, k, oa, ob))
+    if (!factor_lookup(P.ranks, P.off_A, P.off_Bt, 0, P.max_rank, P.d_in, P.d_out, P.pool_A, P.pool_Bt, ad, lead, k,
+                       oa, ob))
         return;
     bgmv_shrink(P.x + (int64_t)tok * P.d_in, P.d_in, P.A_pool + oa, k, red, ts);
     bgmv_expand(ts, k, P.Bt_pool + ob, P.d_out, P.y + (int64_t)tok * P.y_ld + P.y_off, (c - P.chunk0) * kBgmvCols,

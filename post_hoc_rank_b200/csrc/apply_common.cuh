@@ -35,6 +35,8 @@ struct SliceTab {
     int32_t t_col;      // first column of the slice's t in the t buffers
     int32_t chunk0;     // first grid column chunk of the slice (set per expand launch)
     int32_t k_shared;   // ranks == nullptr: every adapter uses the slice's shared factors (rank k_shared, offset 0)
+    int32_t max_rank;   // 0, or the caller's bound on the slice's ranks (a rank above it is an error)
+    int32_t pad;
     int64_t y_off;      // first column of the slice in y
     const int32_t* ranks;
     const int64_t* off_A;
@@ -95,8 +97,8 @@ __device__ __forceinline__ int slice_of_chunk(const ApplyArgs& a, int c) {
 // rows past a pool -> LF_ERR_WORKSPACE (latched when `report`); an invalid adapter
 // contributes nothing.  Returns true when there is work (k > 0).
 __device__ __forceinline__ bool factor_lookup(const int32_t* ranks, const int64_t* off_A, const int64_t* off_Bt,
-                                              int k_shared, int d_in, int d_out, int64_t pool_A, int64_t pool_Bt,
-                                              int ad, bool report, int& k, int64_t& oa, int64_t& ob) {
+                                              int k_shared, int max_rank, int d_in, int d_out, int64_t pool_A,
+                                              int64_t pool_Bt, int ad, bool report, int& k, int64_t& oa, int64_t& ob) {
     if (ranks) {
         k = ranks[ad];
         oa = off_A[ad];
@@ -107,7 +109,7 @@ __device__ __forceinline__ bool factor_lookup(const int32_t* ranks, const int64_
         ob = 0;
     }
     int err = 0;
-    if (k > kMaxRank) err = LF_ERR_SHAPE;
+    if (k > kMaxRank || (max_rank > 0 && k > max_rank)) err = LF_ERR_SHAPE;
     else if (k > 0 && ((oa & 7) || (ob & 7))) err = LF_ERR_ALIGNMENT;
     else if (k > 0 && (oa < 0 || ob < 0 || oa + (int64_t)k * d_in > pool_A || ob + (int64_t)k * d_out > pool_Bt))
         err = LF_ERR_WORKSPACE;
@@ -123,8 +125,8 @@ __device__ __forceinline__ bool factor_lookup(const int32_t* ranks, const int64_
 __device__ __forceinline__ bool slice_factors(const ApplyArgs& a, int s, int ad, bool report, int& k, int64_t& oa,
                                               int64_t& ob) {
     const SliceTab& t = a.sl[s];
-    return factor_lookup(t.ranks, t.off_A, t.off_Bt, t.k_shared, a.d_in, t.d_out, t.pool_A, t.pool_Bt, ad, report, k,
-                         oa, ob);
+    return factor_lookup(t.ranks, t.off_A, t.off_Bt, t.k_shared, t.max_rank, a.d_in, t.d_out, t.pool_A, t.pool_Bt, ad,
+                         report, k, oa, ob);
 }
 
 // Several projections of one batch (same tokens and ids), each with its own x, y and
@@ -136,7 +138,7 @@ struct ProjTab {
     int64_t y_ld, y_off;
     int32_t d_in, d_out;
     int32_t chunk0;             // first grid column chunk of the projection
-    int32_t pad;
+    int32_t max_rank;           // 0, or the caller's bound on the projection's ranks
     const int32_t* ranks;
     const int64_t* off_A;
     const int64_t* off_Bt;

@@ -552,7 +552,8 @@ static lf_status check_apply(int32_t d_in, const void* x, const void* y, int64_t
     if (!aligned16(x) || !aligned16(y)) return LF_ERR_ALIGNMENT;
     for (int q = 0; q < ns; ++q) {
         const lf_slice& t = sl[q];
-        if (t.d_out < 1 || t.pool_elems_A < 0 || t.pool_elems_Bt < 0 || t.y_offset < 0 || t.y_offset + t.d_out > y_ld)
+        if (t.d_out < 1 || t.pool_elems_A < 0 || t.pool_elems_Bt < 0 || t.y_offset < 0 || t.y_offset + t.d_out > y_ld ||
+            t.max_rank < 0 || t.max_rank > kMaxRank)
             return LF_ERR_INVALID_ARG;
         if (!shared && (!t.ranks || !t.off_A || !t.off_Bt)) return LF_ERR_INVALID_ARG;
         if (!t.A_pool || !t.Bt_pool) return LF_ERR_INVALID_ARG;
@@ -597,6 +598,7 @@ static lf_status apply_impl(int32_t T, int32_t d_in, const void* x, void* y, int
         t.d_out = sl[q].d_out;
         t.t_col = kMaxRank * q;
         t.k_shared = shared ? shared->k : 0;
+        t.max_rank = shared ? 0 : sl[q].max_rank;
         t.y_off = sl[q].y_offset;
         t.ranks = sl[q].ranks;
         t.off_A = sl[q].off_A;
@@ -677,7 +679,10 @@ static lf_status apply_impl(int32_t T, int32_t d_in, const void* x, void* y, int
     }
     LF_CUDA_TRY(cudaGetLastError());
     // two expand variants over the same grid, each taking its own (item, slice) pairs:
-    // ranks up to 16 (three CTAs per SM) and the others (two), both in 64-column steps
+    // ranks up to 16 (three CTAs per SM) and the others (two), both in 64-column steps;
+    // when every slice bounds its ranks by 16 the second has nothing to take and is left out
+    bool small_only = !shared;
+    for (int q = 0; q < ns; ++q) small_only = small_only && sl[q].max_rank >= 1 && sl[q].max_rank <= 16;
     {
         constexpr size_t sm16 = expand_tc_smem<16, 64>(), sm64 = expand_tc_smem<kMaxRank, 64>();
         LF_CUDA_TRY(cudaFuncSetAttribute(expand_tc_kernel<16, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm16));
@@ -686,8 +691,9 @@ static lf_status apply_impl(int32_t T, int32_t d_in, const void* x, void* y, int
         LF_LAUNCH("expand_tc", (expand_tc_kernel<16, 64>), dim3(max_tc, (unsigned)A.n_chunks), kTcExpThreads, sm16, s,
                   A, ymap, y_tma);
         LF_CUDA_TRY(cudaGetLastError());
-        LF_LAUNCH("expand_tc", (expand_tc_kernel<kMaxRank, 64>), dim3(max_tc, (unsigned)A.n_chunks), kTcExpThreads,
-                  sm64, s, A, ymap, y_tma);
+        if (!small_only)
+            LF_LAUNCH("expand_tc", (expand_tc_kernel<kMaxRank, 64>), dim3(max_tc, (unsigned)A.n_chunks), kTcExpThreads,
+                      sm64, s, A, ymap, y_tma);
     }
     return launch_status();
 }
@@ -1426,7 +1432,7 @@ lf_status lf_lora_shrink_expand_projections(int32_t T, const int32_t* ids, int32
     if (T == 0) return LF_OK;
     if (!ids) return LF_ERR_INVALID_ARG;
     for (int p = 0; p < n_proj; ++p) {
-        if (projs[p].reserved != 0 || projs[p].slice.reserved != 0) return LF_ERR_INVALID_ARG;
+        if (projs[p].reserved != 0) return LF_ERR_INVALID_ARG;
         const lf_status st = check_apply(projs[p].d_in, projs[p].x, projs[p].y, projs[p].y_ld, &projs[p].slice, 1, false);
         if (st != LF_OK) return st;
     }
@@ -1468,6 +1474,7 @@ lf_status lf_lora_shrink_expand_projections(int32_t T, const int32_t* ids, int32
         t.d_in = q.d_in;
         t.d_out = q.slice.d_out;
         t.chunk0 = chunks;
+        t.max_rank = q.slice.max_rank;
         t.ranks = q.slice.ranks;
         t.off_A = q.slice.off_A;
         t.off_Bt = q.slice.off_Bt;

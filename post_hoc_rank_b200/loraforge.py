@@ -60,7 +60,7 @@ class lf_phase_time(ctypes.Structure):
 
 class lf_slice(ctypes.Structure):
     """One output slice of lf_lora_shrink_expand_slices (mirrors the C struct)."""
-    _fields_ = [("d_out", ctypes.c_int32), ("reserved", ctypes.c_int32), ("y_offset", ctypes.c_int64),
+    _fields_ = [("d_out", ctypes.c_int32), ("max_rank", ctypes.c_int32), ("y_offset", ctypes.c_int64),
                 ("ranks", ctypes.c_void_p), ("off_A", ctypes.c_void_p), ("off_Bt", ctypes.c_void_p),
                 ("A_pool", ctypes.c_void_p), ("Bt_pool", ctypes.c_void_p),
                 ("pool_elems_A", ctypes.c_int64), ("pool_elems_Bt", ctypes.c_int64)]
@@ -263,9 +263,10 @@ def lf_apply_slices_workspace_size(T: int, n_adapters: int, n_slices: int) -> in
     return lib().lf_apply_slices_workspace_size(T, n_adapters, n_slices)
 
 
-def make_slice(d_out, y_offset, ranks, off_A, off_Bt, A_pool, Bt_pool) -> lf_slice:
-    """lf_slice from device tensors (ranks int32, offsets int64, pools bf16)."""
-    return lf_slice(int(d_out), 0, int(y_offset), _ptr(ranks), _ptr(off_A), _ptr(off_Bt), _ptr(A_pool),
+def make_slice(d_out, y_offset, ranks, off_A, off_Bt, A_pool, Bt_pool, max_rank=0) -> lf_slice:
+    """lf_slice from device tensors (ranks int32, offsets int64, pools bf16); max_rank: 0, or
+    an upper bound of the slice's ranks the caller knows."""
+    return lf_slice(int(d_out), int(max_rank), int(y_offset), _ptr(ranks), _ptr(off_A), _ptr(off_Bt), _ptr(A_pool),
                     _ptr(Bt_pool), A_pool.numel(), Bt_pool.numel())
 
 

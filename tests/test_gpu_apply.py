@@ -523,3 +523,41 @@ def test_projections_call_host_checks():
     assert lf.lf_lora_shrink_expand_projections(T, ids_d, n, [res], 1.0, check=False) == 1
     torch.cuda.synchronize()
     assert torch.equal(y.cpu(), y0)
+
+
+def test_rank_bound_leaves_out_the_rank64_expand():
+    """A slice whose caller bounds its ranks by 16 (lf_slice.max_rank): the same bits with
+    one launch fewer on the tensor-core path; an adapter above the bound latches
+    LF_ERR_SHAPE and its rows keep y; a bound above 64 is a host error."""
+    T, n, d_in, d_out = 1024, 4, 512, 384
+    ids = np.repeat(np.arange(n, dtype=np.int32), T // n)
+    ids_d = torch.from_numpy(ids).cuda()
+    x = synth.normal_bf16((T, d_in), (17, 1)).cuda()
+    y0 = synth.normal_bf16((T, d_out), (17, 2)).cuda()
+    ws = api.workspace(lf.lf_apply_slices_workspace_size(T, n, 1), "cuda")
+
+    def run(ranks, bound):
+        offA, offB, Ap, Bt = make_pools(ranks, d_in, d_out, (17, 3, len(ranks)))
+        sl = [dict(d_out=d_out, y_off=0, ranks=np.asarray(ranks), offA=offA, offB=offB, Ap=Ap, Bt=Bt)]
+        keep, tens = _slice_tensors(sl)
+        keep[0].max_rank = bound
+        y = y0.clone()
+        l0 = lf.lf_launch_count()
+        st = lf.lf_lora_shrink_expand_slices(x, y, ids_d, n, keep, 1.0, ws, check=False)
+        return st, y, lf.lf_launch_count() - l0, sl, tens
+
+    st0, y_free, l_free, sl, _a = run([16, 8, 16, 12], 0)
+    st1, y_bound, l_bound, _, _b = run([16, 8, 16, 12], 16)
+    assert st0 == 0 and st1 == 0 and lf.lf_get_device_status() == 0
+    assert torch.equal(y_free, y_bound) and l_bound == l_free - 1
+    check_slices(y_bound.cpu(), y0.cpu(), oracle_slices(x.cpu(), y0.cpu(), ids, sl, 1.0), sl, ids)
+    st2, y_bad, _, sl2, _c = run([16, 20, 8, 4], 16)
+    assert st2 == 0 and lf.lf_get_device_status() == 2   # LF_ERR_SHAPE
+    rows = torch.from_numpy(ids == 1)
+    assert torch.equal(y_bad.cpu()[rows], y0.cpu()[rows])
+    want = oracle_slices(x.cpu(), y0.cpu(), ids, sl2, 1.0)
+    keep_rows = ids != 1   # the other adapters as usual
+    check_slices(y_bad.cpu()[torch.from_numpy(keep_rows)], y0.cpu()[torch.from_numpy(keep_rows)], want[keep_rows],
+                 sl2, ids[keep_rows])
+    st3, _, _, _, _d = run([16, 8, 16, 12], 65)
+    assert st3 == 1   # LF_ERR_INVALID_ARG before any launch
