@@ -923,7 +923,9 @@ def library_qr_context(dev, stream):
         api.tsqr(mods, B, A, out=F, ws=ws, stream=stream)
     lf.lf_profile_enable(False)
     ph = lf.lf_profile_read()
-    qr_ms = sum(ph[k][0] for k in ("tsqr_gram_leaf", "tsqr_householder") if k in ph) / reps
+    # the R factors: integer leaf + root, and the fp64 leaf / Householder routes when they run
+    qr_ms = sum(ph[k][0] for k in ("tsqr_gram_i8", "tsqr_gram_i8_root", "tsqr_gram_leaf", "tsqr_householder")
+                if k in ph) / reps
     del B, A, F, ws, groups
     torch.cuda.empty_cache()
     return {"sample": "one Qwen2.5-7B-shaped adapter, 196 modules, B and A^T (R only)",
