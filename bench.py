@@ -727,14 +727,16 @@ def large_fleet_bench(args, dev, stream, hbm):
     shapes = M.proj_shapes()
     out = {"workload": f"large fleet: {n_total} adapters x Llama-3-8B (224 modules each, r=64), LoRAForge-S "
                        "1/12 floor 1, compressed in chunks of 64 adapters; then 4096 tokens (64 prefill segments "
-                       "x 48 + 1024 decode tokens, Zipf(1.2) ids) through 32 layers x 7 projections",
+                       "x 48 + 1024 decode tokens, Zipf(1.2) ids) through 32 layers x 7 projections, one call per layer",
            "modules": int(n_mod), "compress_ms": round(compress_ms, 2),
            "modules_per_s": round(n_mod / (compress_ms * 1e-3), 1), "distinct_adapters": int(len(ref))}
+    ws = api.workspace(lf.lf_apply_workspace_size(T, n_total), dev)
     for variant in ("ragged", "padded"):
         calls, total_bytes = [], 0
         for l in range(M.layers):
             x_h = synth.normal_bf16((T, M.hidden), (5, 3, l), device=dev)
             x_f = synth.normal_bf16((T, M.ffn), (5, 4, l), device=dev)
+            items = []   # the layer's 7 projections: one lf_lora_shrink_expand_projections call
             for p, (_, d_out, d_in) in enumerate(shapes):
                 mi = (aloc * 7 + p) * M.layers + l
                 rk = np.array([ranks_c[c][m] for c, m in zip(cidx, mi)], dtype=np.int64)
@@ -761,10 +763,11 @@ def large_fleet_bench(args, dev, stream, hbm):
                     oa_d = np.zeros(n_total, dtype=np.int64); ob_d = np.zeros(n_total, dtype=np.int64)
                     oa_d[ref] = np.arange(len(ref)) * kmax * d_in; ob_d[ref] = np.arange(len(ref)) * kmax * d_out
                     k_used = np.full(len(ref), kmax)
-                ws = api.workspace(lf.lf_apply_workspace_size(T, n_total), dev)
-                calls.append(_proj_call(x, y, ids_d, n_total, torch.from_numpy(rk_d.astype(np.int32)).to(dev),
-                                        torch.from_numpy(oa_d).to(dev), torch.from_numpy(ob_d).to(dev), pa, pb, ws))
+                items.append((x, y, (d_out, 0, torch.from_numpy(rk_d.astype(np.int32)).to(dev),
+                                     torch.from_numpy(oa_d).to(dev), torch.from_numpy(ob_d).to(dev), pa, pb,
+                                     int(max(1, k_used.max())))))
                 total_bytes += apply_bytes(T, d_in, d_out, [int(k) for k in k_used])
+            calls.append(_projections_call(items, ids_d, n_total, T, ws))
         r = _apply_run(args, calls, ids_d, n_total, T, total_bytes, stream, hbm, {})
         out[variant] = {k: r[k] for k in ("tokens_per_s", "ms_per_step", "algo_bytes", "achieved_gbs", "hbm_frac",
                                           "launches_per_step", "phases_ms")}
