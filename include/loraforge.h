@@ -83,8 +83,10 @@ typedef struct {
  *     ratio_num / ratio_den (<= 1) of its spectral energy,
  *     ratio_den * sum_{j<k} sigma_j^2 >= ratio_num * sum_j sigma_j^2 (LoRASpace's
  *     minimal subspace keeping 99 % of the energy, read per module); no group budget.
- *  Spectral kinds (1-3) recompute in fp64 the modules whose decision lies within a
- *  1e-4 relative band of the threshold, so ranks match an fp64 reference.
+ *  Spectral kinds (1-3) recompute in fp64 the modules whose decision is a near tie
+ *  (kinds 1-2: the last selected energy and the first left out closer than 2e-4 of the
+ *  threshold; kind 3: a cumulative energy within 1e-4 of it), so ranks match an fp64
+ *  reference.
  * The budget scope is the module `group`: one group per adapter gives per-adapter
  * budgets, one group over all modules a fleet-wide budget. */
 typedef struct {
@@ -98,13 +100,18 @@ int32_t lf_rank_stride(const lf_module* mods /*[host]*/, int32_t n);
  * For every module i, with X_B = B_i (d_out x r) and X_A = A_i^T (d_in x r):
  *   R_B = R(X_B), R_A = R(X_A): the R factors of the thin QRs, upper triangular,
  *         diag >= 0, computed by a batched tall-skinny QR over row tiles of every
- *         module at once: each row tile contributes its Gram X_t^T X_t (fp32
- *         products, exact in fp64, fp64 sums), tile Grams are summed in a fixed
- *         order and R = chol(X^T X) in fp64 (R^T R = X^T X defines the same R as
- *         the QR).  A matrix whose Cholesky pivot falls to <= 1e-9 of its Gram
- *         diagonal (numerically rank-deficient, a zero column, non-finite input) is
- *         factored instead by structured Householder reflections of [R; tile]
- *         over the same row tiles, merged in chunk order;
+ *         module at once: each row tile (up to 24 576 rows) contributes its Gram,
+ *         tile Grams are summed in a fixed order and R = chol(X^T X) in fp64
+ *         (R^T R = X^T X defines the same R as the QR).  The tile Gram is exact for
+ *         the 32-bit fixed-point image of the tile (each column scaled by a power of
+ *         two from its first 128 rows and truncated: a columnwise error below 2^-27
+ *         of the column's largest value), formed on the int8 tensor cores from its
+ *         four byte planes.  A matrix whose rows or offset are not 16-byte aligned,
+ *         or with a value at or above its column's scale, takes an fp64 Gram of the
+ *         fp32 products instead.  A matrix whose Cholesky pivot falls to <= 1e-9 of
+ *         its Gram diagonal (numerically rank-deficient, a zero column, non-finite
+ *         input) is factored by structured Householder reflections of [R; tile]
+ *         over row chunks, merged in chunk order;
  *   M = R_B R_A^T (r x r) and its SVD M = U S V^T (one-sided Jacobi in fp32,
  *   outputs stored as fp64):
  *   sigma (descending) are the singular values of dW = B A, Q_B U its left and
@@ -136,10 +143,12 @@ lf_status lf_select_ranks(const lf_module* mods /*[host]*/, int32_t n, lf_policy
                           void* ws, size_t ws_bytes, lf_stream_t stream);
 
 /* ---- Truncation + export -----------------------------------------------------
- * Allocates ranks as lf_select_ranks does.  For LoRAForge-S, modules with a
- * candidate energy within a relative band of 1e-4 around their group's selection
- * threshold get their spectrum recomputed in fp64 from B and A before the final
- * choice, so ranks match an fp64 computation.  Then, per module with k = ranks[i]:
+ * Allocates ranks as lf_select_ranks does.  For the spectral policies, in a group
+ * whose selection boundary is a near tie (the last selected energy theta and the first
+ * one left out closer than 2e-4 theta), the modules holding a candidate within 2e-4
+ * theta of theta get their spectrum recomputed in fp64 from B and A before the final
+ * choice, so ranks match an fp64 computation; more such modules than the workspace's
+ * refinement capacity (8 per group + 64) latch LF_ERR_WORKSPACE.  Then, per module with k = ranks[i]:
  *   B'^T = (R_A^T V_k S_k^-1)^T B^T   (k x d_out, rows of the retained left
  *                                      singular vectors of dW)
  *   A'   = (U_k^T R_B) A               (k x d_in, = S_k V_k^T Q_A^T)
