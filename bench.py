@@ -1266,9 +1266,7 @@ def main():
         "metric": METRIC, "value": round(value, 1), "unit": "modules/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_step, 3), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": {"workload": f"factor construction fleet: {args.adapters} adapters x Qwen2.5-7B "
-                               f"(196 modules each, {fr['n']} modules per GPU), r=64, LoRAForge-S 1/12 floor 1",
-                   "l2": "inputs (54.9 GB fp32 per GPU) larger than L2", "parallelism": f"dp{world} (adapters)"},
+        "config": headline_config(args.adapters, world),
         "roofline": roof,
         "step_hbm": {"algo_bytes_2touch": int(step_bytes_2touch), "achieved_gbs": round(step_gbs, 1),
                      "frac": round(step_gbs / hbm, 4), "peak": hbm},
@@ -1287,6 +1285,13 @@ def main():
     print(json.dumps(line))
     if pg is not None:
         pg.destroy_process_group()
+
+
+def headline_config(n_adapters: int, world: int) -> dict:
+    """The headline workload's config record (both arms print the same one)."""
+    return {"workload": f"factor construction fleet: {n_adapters} adapters x Qwen2.5-7B (196 modules each, "
+                        f"{196 * n_adapters} modules per GPU), r=64, LoRAForge-S 1/12 floor 1",
+            "l2": "inputs (54.9 GB fp32 per GPU) larger than L2", "parallelism": f"dp{world} (adapters)"}
 
 
 def reference_arm(args, rank, world):
@@ -1313,8 +1318,7 @@ def reference_arm(args, rank, world):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * t / len(steps), 1),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic",
-            "config": {"workload": "factor construction fleet: Qwen2.5-7B-shaped adapters (196 modules each), "
-                                   "r=64, LoRAForge-S 1/12 floor 1; per step one whole adapter"},
+            "config": headline_config(args.adapters, 1),
             "cpu_baseline": {"kind": "oracle", "cores": workers, "value": round(v, 2), "unit": "modules/s",
                              "sample": "one whole adapter (196 modules, allocation over the adapter) per step; "
                                        f"spawned process pool of {workers} workers, one BLAS thread each",
