@@ -376,6 +376,7 @@ __global__ void __launch_bounds__(kI8Threads, 1) gram_i8_kernel(GramI8Args a) {
                     if (k >= 1) ok = wait(&s.cmax_empty, (uint32_t)((k - 1) & 1));
                     if (!ok) break;
                     s.cmax[q][c] = mx;
+                    __threadfence_block();
                     __syncwarp();
                     if (lane == 0) mbar_arrive1(&s.cmax_full);
                     ok = wait(&s.cmax_full, (uint32_t)(k & 1));
@@ -383,6 +384,7 @@ __global__ void __launch_bounds__(kI8Threads, 1) gram_i8_kernel(GramI8Args a) {
                     float m = s.cmax[0][c];
 #pragma unroll
                     for (int h = 1; h < 8; ++h) m = fmaxf(m, s.cmax[h][c]);
+                    asm volatile("" ::"f"(m));   // the reads have returned before the release
                     __syncwarp();
                     if (lane == 0) mbar_arrive1(&s.cmax_empty);
                     int E = -90;   // an all-zero start: any nonzero value later overflows the scale
@@ -440,6 +442,7 @@ __global__ void __launch_bounds__(kI8Threads, 1) gram_i8_kernel(GramI8Args a) {
 #pragma unroll
             for (int p = 0; p < 4; ++p) atomicAdd(&M.colsum[p][c], (int)cs[p]);
             if (!vok) M.ovf = 1;
+            __threadfence_block();   // every lane's sums and flag are in before its warp's arrive
             __syncwarp();
             if (lane == 0) mbar_arrive1(&s.meta_full[ms]);
         }
