@@ -217,3 +217,36 @@ def test_bounded_wait_check_rejects_bad_poll_counts():
     L = lf.lib()
     assert L.lf_check_bounded_wait(-1, None) == 1          # LF_ERR_INVALID_ARG, nothing launched
     assert L.lf_check_bounded_wait((1 << 20) + 1, None) == 1
+
+
+def test_slice_rank_bound_validation_on_host():
+    """lf_slice.max_rank: 0 (no bound) or 1..64; anything else is rejected before a launch."""
+    L = lf.lib()
+    for bound in (-1, 65, 1000):
+        sl = (lf.lf_slice * 1)(lf.lf_slice(64, bound, 0, 16, 16, 16, 16, 16, 1024, 1024))
+        assert L.lf_lora_shrink_expand_slices(4, 64, 16, 16, 64, 16, 2, sl, 1, 1.0, None, None, 16, 1 << 20,
+                                              None) == 1
+
+
+def test_projections_validation_on_host():
+    """lf_lora_shrink_expand_projections: host checks per projection, before any launch."""
+    L = lf.lib()
+
+    def proj(x=16, y=16, d_in=64, reserved=0, y_ld=64, bound=0):
+        return lf.lf_projection(x, y, d_in, reserved, y_ld, lf.lf_slice(64, bound, 0, 16, 16, 16, 16, 16, 1024, 1024))
+
+    def call(projs, T=4, ids=16, n=2):
+        arr = (lf.lf_projection * max(1, len(projs)))(*projs)
+        return L.lf_lora_shrink_expand_projections(T, ids, n, arr, len(projs), 1.0, None, None, 0, None)
+    assert lf.MAX_PROJECTIONS == 8
+    assert call([proj()], T=0) == 0                      # empty batch: nothing to do
+    assert call([]) == 1
+    assert call([proj()] * 9) == 1                       # more than LF_MAX_PROJECTIONS
+    assert call([proj()], T=-1) == 1
+    assert call([proj()], ids=None) == 1
+    assert call([proj(), proj(reserved=1)]) == 1
+    assert call([proj(), proj(bound=65)]) == 1
+    assert call([proj(x=18)]) == 8                       # x not 16-byte aligned
+    assert call([proj(d_in=60)]) == 8                    # d_in not a multiple of 8
+    assert call([proj(y_ld=48)]) == 1                    # the slice does not fit in y's row
+    assert call([proj(x=None)]) == 1
