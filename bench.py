@@ -1156,7 +1156,8 @@ def main():
     ap.add_argument("--no-jd", action="store_true")
     ap.add_argument("--jd-only", action="store_true", help="run only the JD-Full workload and print its record")
     ap.add_argument("--large-adapters", type=int, default=1024)
-    ap.add_argument("--lora-only", choices=["decode", "decode_per_projection", "prefill_k16", "prefill_r64"],
+    ap.add_argument("--lora-only", choices=["decode", "decode_per_projection", "prefill_k16", "prefill_r64",
+                                            "large_fleet"],
                     help="run only this side-path workload and print its record")
     args = ap.parse_args()
 
@@ -1187,7 +1188,8 @@ def main():
         fn = {"decode": lambda: decode_bench(args, dev, stream, hbm),
               "decode_per_projection": lambda: decode_bench(args, dev, stream, hbm, per_layer=False),
               "prefill_k16": lambda: prefill_bench(args, dev, stream, hbm, 16),
-              "prefill_r64": lambda: prefill_bench(args, dev, stream, hbm, 64)}[args.lora_only]
+              "prefill_r64": lambda: prefill_bench(args, dev, stream, hbm, 64),
+              "large_fleet": lambda: large_fleet_bench(args, dev, stream, hbm)}[args.lora_only]
         print(json.dumps(fn()))
         return
 

@@ -534,6 +534,20 @@ __device__ __forceinline__ void bgmv_shrink(const __nv_bfloat16* xr, int d_in, c
     }
 }
 
+// One token row's chunk y[cbase ..) and the k rows of B'^T that the expand reads, fetched
+// into L2 by bulk prefetches (one thread per row) before the shrink, so that their HBM
+// latency overlaps the shrink instead of following it.  Rows, offsets and chunk widths
+// are multiples of 8 elements (16 bytes), as the bulk copy requires.
+__device__ __forceinline__ void bgmv_prefetch(const __nv_bfloat16* yr, const __nv_bfloat16* Bt, int k, int d_out,
+                                              int cbase) {
+    const int tid = threadIdx.x;
+    const int ncols = min(kBgmvCols, d_out - cbase);
+    if (tid <= k && ncols > 0) {
+        const __nv_bfloat16* src = tid == 0 ? yr + cbase : Bt + (int64_t)(tid - 1) * d_out + cbase;
+        asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(ncols * 2) : "memory");
+    }
+}
+
 // y[cbase .. cbase + kBgmvCols) of one token row (within d_out) += scale * B'^T tv,
 // rounded once to bf16; 16-byte loads of the k rows of B'^T.
 __device__ __forceinline__ void bgmv_expand(const float* tv, int k, const __nv_bfloat16* Bt, int d_out,
@@ -580,6 +594,9 @@ __device__ __forceinline__ void bgmv_token(const ApplyArgs& a, int tok, float (&
     int k;
     int64_t oa, ob;
     if (!slice_factors(a, sl, ad, lead, k, oa, ob)) return;
+    __nv_bfloat16* yr = a.y + (int64_t)tok * a.y_ld + S.y_off;
+    const int cbase = ((int)blockIdx.y - S.chunk0) * kBgmvCols;
+    bgmv_prefetch(yr, S.Bt_pool + ob, k, S.d_out, cbase);
     bgmv_shrink(a.x + (int64_t)tok * a.d_in, a.d_in, S.A_pool + oa, k, red, ts);
     const float* tv = ts;
     if (a.sigma_mode) {   // Sigma-sandwich: t <- Sigma_a t
@@ -587,8 +604,7 @@ __device__ __forceinline__ void bgmv_token(const ApplyArgs& a, int tok, float (&
         __syncthreads();
         tv = tw;
     }
-    bgmv_expand(tv, k, S.Bt_pool + ob, S.d_out, a.y + (int64_t)tok * a.y_ld + S.y_off,
-                ((int)blockIdx.y - S.chunk0) * kBgmvCols, adapter_scale(a, ad));
+    bgmv_expand(tv, k, S.Bt_pool + ob, S.d_out, yr, cbase, adapter_scale(a, ad));
 }
 
 // LIST = false: CTA blockIdx.x applies token blockIdx.x (decode regime, no routing pass).
@@ -635,9 +651,11 @@ __global__ void __launch_bounds__(kBgmvThreads, 2) bgmv_proj_kernel(ProjArgs a) 
     if (!factor_lookup(P.ranks, P.off_A, P.off_Bt, 0, P.max_rank, P.d_in, P.d_out, P.pool_A, P.pool_Bt, ad, lead, k,
                        oa, ob))
         return;
+    __nv_bfloat16* yr = P.y + (int64_t)tok * P.y_ld + P.y_off;
+    const int cbase = (c - P.chunk0) * kBgmvCols;
+    bgmv_prefetch(yr, P.Bt_pool + ob, k, P.d_out, cbase);
     bgmv_shrink(P.x + (int64_t)tok * P.d_in, P.d_in, P.A_pool + oa, k, red, ts);
-    bgmv_expand(ts, k, P.Bt_pool + ob, P.d_out, P.y + (int64_t)tok * P.y_ld + P.y_off, (c - P.chunk0) * kBgmvCols,
-                a.scales ? a.scales[ad] : a.scale);
+    bgmv_expand(ts, k, P.Bt_pool + ob, P.d_out, yr, cbase, a.scales ? a.scales[ad] : a.scale);
 }
 
 // Decode regime of the no-allocation entry point (one slice, sorted items): CTA

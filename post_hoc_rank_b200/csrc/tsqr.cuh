@@ -434,27 +434,27 @@ __device__ __forceinline__ bool svd_rotate_acc(SvdSmem<T, RT>& s, int p, int q, 
             Mp[k] = c * x - sn * y;
             Mq[k] = sn * x + c * y;
         }
-        return true;
-    }
+    } else {
 #pragma unroll 2
-    for (; k + 3 < r; k += 4) {   // 16-byte loads and stores of four columns
-        T x[4], y[4], u[4], v[4], x2[4], y2[4], u2[4], v2[4];
-        ld4(Mp + k, x); ld4(Mq + k, y); ld4(Up + k, u); ld4(Uq + k, v);
+        for (; k + 3 < r; k += 4) {   // 16-byte loads and stores of four columns
+            T x[4], y[4], u[4], v[4], x2[4], y2[4], u2[4], v2[4];
+            ld4(Mp + k, x); ld4(Mq + k, y); ld4(Up + k, u); ld4(Uq + k, v);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            x2[e] = c * x[e] - sn * y[e];
-            y2[e] = sn * x[e] + c * y[e];
-            u2[e] = c * u[e] - sn * v[e];
-            v2[e] = sn * u[e] + c * v[e];
+            for (int e = 0; e < 4; ++e) {
+                x2[e] = c * x[e] - sn * y[e];
+                y2[e] = sn * x[e] + c * y[e];
+                u2[e] = c * u[e] - sn * v[e];
+                v2[e] = sn * u[e] + c * v[e];
+            }
+            st4(Mp + k, x2); st4(Mq + k, y2); st4(Up + k, u2); st4(Uq + k, v2);
         }
-        st4(Mp + k, x2); st4(Mq + k, y2); st4(Up + k, u2); st4(Uq + k, v2);
-    }
-    for (; k < r; ++k) {
-        const T x = Mp[k], y = Mq[k], u = Up[k], v = Uq[k];
-        Mp[k] = c * x - sn * y;
-        Mq[k] = sn * x + c * y;
-        Up[k] = c * u - sn * v;
-        Uq[k] = sn * u + c * v;
+        for (; k < r; ++k) {
+            const T x = Mp[k], y = Mq[k], u = Up[k], v = Uq[k];
+            Mp[k] = c * x - sn * y;
+            Mq[k] = sn * x + c * y;
+            Up[k] = c * u - sn * v;
+            Uq[k] = sn * u + c * v;
+        }
     }
     return true;
 }
