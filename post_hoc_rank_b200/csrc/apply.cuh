@@ -534,15 +534,18 @@ __device__ __forceinline__ void bgmv_shrink(const __nv_bfloat16* xr, int d_in, c
     }
 }
 
-// One token row's chunk y[cbase ..) and the k rows of B'^T that the expand reads, fetched
-// into L2 by bulk prefetches (one thread per row) before the shrink, so that their HBM
-// latency overlaps the shrink instead of following it.  Rows, offsets and chunk widths
-// are multiples of 8 elements (16 bytes), as the bulk copy requires.
+// The token row's chunk y[cbase ..) that the expand reads (always an HBM miss: each chunk
+// is read once) and, for ranks up to 8, the k rows of B'^T, fetched into L2 by bulk
+// prefetches (one thread per row) before the shrink, so that their latency overlaps the
+// shrink instead of following it.  Larger ranks skip the B'^T rows: those mostly come from
+// L2 already (every token of the adapter reads them), and a prefetch per CTA of up to 64
+// rows adds L2 requests that cost more than the first touch saves.  Rows, offsets and
+// chunk widths are multiples of 8 elements (16 bytes), as the bulk copy requires.
 __device__ __forceinline__ void bgmv_prefetch(const __nv_bfloat16* yr, const __nv_bfloat16* Bt, int k, int d_out,
                                               int cbase) {
     const int tid = threadIdx.x;
     const int ncols = min(kBgmvCols, d_out - cbase);
-    if (tid <= k && ncols > 0) {
+    if (tid <= (k <= 8 ? k : 0) && ncols > 0) {
         const __nv_bfloat16* src = tid == 0 ? yr + cbase : Bt + (int64_t)(tid - 1) * d_out + cbase;
         asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(ncols * 2) : "memory");
     }
@@ -594,9 +597,6 @@ __device__ __forceinline__ void bgmv_token(const ApplyArgs& a, int tok, float (&
     int k;
     int64_t oa, ob;
     if (!slice_factors(a, sl, ad, lead, k, oa, ob)) return;
-    __nv_bfloat16* yr = a.y + (int64_t)tok * a.y_ld + S.y_off;
-    const int cbase = ((int)blockIdx.y - S.chunk0) * kBgmvCols;
-    bgmv_prefetch(yr, S.Bt_pool + ob, k, S.d_out, cbase);
     bgmv_shrink(a.x + (int64_t)tok * a.d_in, a.d_in, S.A_pool + oa, k, red, ts);
     const float* tv = ts;
     if (a.sigma_mode) {   // Sigma-sandwich: t <- Sigma_a t
@@ -604,7 +604,8 @@ __device__ __forceinline__ void bgmv_token(const ApplyArgs& a, int tok, float (&
         __syncthreads();
         tv = tw;
     }
-    bgmv_expand(tv, k, S.Bt_pool + ob, S.d_out, yr, cbase, adapter_scale(a, ad));
+    bgmv_expand(tv, k, S.Bt_pool + ob, S.d_out, a.y + (int64_t)tok * a.y_ld + S.y_off,
+                ((int)blockIdx.y - S.chunk0) * kBgmvCols, adapter_scale(a, ad));
 }
 
 // LIST = false: CTA blockIdx.x applies token blockIdx.x (decode regime, no routing pass).
@@ -629,7 +630,8 @@ __global__ void __launch_bounds__(kBgmvThreads, 2) bgmv_kernel(ApplyArgs a) {
 
 // Several projections of one decode batch in one launch: CTA (token, column chunk),
 // the chunks of all projections laid end to end along grid.y (each projection's first
-// chunk at its chunk0).  Per projection the same arithmetic as bgmv_kernel<false>.
+// chunk at its chunk0).  Per projection the same arithmetic as bgmv_kernel<false>; each
+// CTA first prefetches its y chunk (and small-rank B'^T rows) into L2.
 __global__ void __launch_bounds__(kBgmvThreads, 2) bgmv_proj_kernel(ProjArgs a) {
     __shared__ float red[kBgmvThreads / 32][kBgmvJ];
     __shared__ float ts[kMaxRank];
