@@ -56,33 +56,52 @@ def peaks():
 
 
 # ----------------------------------------------------------------- clocks
+def smi_device_id(dev_index: int) -> str:
+    """nvidia-smi's --id for this process's CUDA device dev_index: its entry in
+    CUDA_VISIBLE_DEVICES (an index or a UUID, both of which nvidia-smi takes) when that is
+    set, else the index itself."""
+    vis = [p.strip() for p in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if p.strip()]
+    return vis[dev_index] if dev_index < len(vis) else str(dev_index)
+
+
 class ClockSampler:
-    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region.
+
+    The sampler is started, and its first sample awaited, on entry; the region is the
+    body of the ``with`` block, and ``summary`` keeps only the samples taken inside it."""
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
-        self.lines: list[str] = []
+    def __init__(self, gpu: str, period_ms: int = 50, exe: str = "nvidia-smi"):
+        self.gpu = gpu
+        self.period_ms = period_ms
+        self.exe = exe
+        self.samples: list[tuple[float, str]] = []
         self.proc = None
+        self.t0 = self.t1 = None
 
     def __enter__(self):
         try:
             self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                [self.exe, f"--id={self.gpu}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", str(self.period_ms)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.t = threading.Thread(target=self._read, daemon=True)
             self.t.start()
+            deadline = time.perf_counter() + 5.0
+            while not self.samples and self.proc.poll() is None and time.perf_counter() < deadline:
+                time.sleep(0.005)
         except OSError:
             self.proc = None
+        self.t0 = time.perf_counter()
         return self
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.samples.append((time.perf_counter(), line.strip()))
 
     def __exit__(self, *a):
+        self.t1 = time.perf_counter()
         if self.proc:
             self.proc.terminate()
             try:
@@ -93,7 +112,10 @@ class ClockSampler:
     def summary(self):
         sm, mx, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
+        t1 = self.t1 if self.t1 is not None else float("inf")
+        for t, ln in list(self.samples):
+            if self.t0 is None or not (self.t0 <= t <= t1):
+                continue
             f = [x.strip() for x in ln.split(",")]
             if len(f) < 9:
                 continue
@@ -105,7 +127,7 @@ class ClockSampler:
                 if v.lower() == "active":
                     reasons.add(nm)
         return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": mx,
-                "reasons": sorted(reasons), "samples": len(sm)}
+                "reasons": sorted(reasons), "samples": len(sm), "period_ms": self.period_ms}
 
 
 # ----------------------------------------------------------------- helpers
@@ -258,7 +280,7 @@ def factor_bench(args, rank, world, dev, sync_all, stream, hbm, peak_kind):
     lf.lf_profile_reset()
     lf.lf_profile_enable(True)
     launches0 = lf.lf_launch_count()
-    with ClockSampler(torch.cuda.current_device()) as clk:
+    with ClockSampler(smi_device_id(torch.cuda.current_device())) as clk:
         ms = timed(step, args.steps, sync_all, stream)
     launches = lf.lf_launch_count() - launches0
     lf.lf_profile_enable(False)
