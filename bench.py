@@ -323,16 +323,28 @@ def factor_e2e(args, dev, stream, rank=0):
     E = api.alloc_export(mods, pol, dev, bf16=True)
     ws_t = api.workspace(lf.lf_tsqr_workspace_size(mods), dev)
     ws_e = api.workspace(lf.lf_export_workspace_size(mods), dev)
+    # pinned host destinations, allocated once like the inputs: the rank table and offsets
+    # come back first (they size the pools), then the used part of each bf16 pool
+    ranks_h = torch.empty_like(E.ranks, device="cpu").pin_memory()
+    offA_h = torch.empty_like(E.off_A, device="cpu").pin_memory()
+    offB_h = torch.empty_like(E.off_Bt, device="cpu").pin_memory()
+    A16_h = torch.empty_like(E.A_pool16, device="cpu").pin_memory()
+    B16_h = torch.empty_like(E.Bt_pool16, device="cpu").pin_memory()
     outs_h = {}
 
     def step():
-        Bd.copy_(Bh, non_blocking=True); Ad.copy_(Ah, non_blocking=True)
+        with torch.cuda.stream(stream):
+            Bd.copy_(Bh, non_blocking=True); Ad.copy_(Ah, non_blocking=True)
         api.tsqr(mods, Bd, Ad, out=F, ws=ws_t, stream=stream)
         api.truncate_export(mods, pol, Bd, Ad, F, out=E, ws=ws_e, stream=stream)
-        ranks = E.ranks.cpu(); offA = E.off_A.cpu(); offB = E.off_Bt.cpu()
-        na, nb = int(offA[-1]), int(offB[-1])
-        outs_h["A"] = E.A_pool16[:na].cpu(); outs_h["B"] = E.Bt_pool16[:nb].cpu()
-        outs_h["d2h"] = ranks.numel() * 4 + (offA.numel() + offB.numel()) * 8 + 2 * (na + nb)
+        with torch.cuda.stream(stream):
+            ranks_h.copy_(E.ranks, non_blocking=True)
+            offA_h.copy_(E.off_A, non_blocking=True); offB_h.copy_(E.off_Bt, non_blocking=True)
+            stream.synchronize()
+            na, nb = int(offA_h[-1]), int(offB_h[-1])
+            A16_h[:na].copy_(E.A_pool16[:na], non_blocking=True); B16_h[:nb].copy_(E.Bt_pool16[:nb], non_blocking=True)
+            stream.synchronize()
+        outs_h["d2h"] = ranks_h.numel() * 4 + (offA_h.numel() + offB_h.numel()) * 8 + 2 * (na + nb)
 
     step()
     torch.cuda.synchronize()
@@ -344,7 +356,7 @@ def factor_e2e(args, dev, stream, rank=0):
     dt = (time.perf_counter() - t0) / k
     res = dict(value=lay.n / dt, h2d=int(4 * (lay.B_total + lay.A_total)), d2h=int(outs_h["d2h"]),
                adapters=n_ad, modules=lay.n)
-    del Bh, Ah, Bd, Ad, F, E, ws_t, ws_e
+    del Bh, Ah, Bd, Ad, F, E, ws_t, ws_e, ranks_h, offA_h, offB_h, A16_h, B16_h
     torch.cuda.empty_cache()
     return res
 
