@@ -370,7 +370,13 @@ def _decode_e2e(args, calls, ids, ids_d, T, stream):
     """The decode step through the public call with host buffers: per step the token ids,
     every layer's inputs x and outputs y go up from pinned host memory, the 32
     lf_lora_shrink_expand_projections calls run, and every y comes back (y is updated in
-    place, so it travels both ways).  Device-timed with events around the whole step."""
+    place, so it travels both ways).  Uploads, calls and read-backs run on three streams
+    ordered by events layer by layer, so the two copy directions share the PCIe link at
+    once: layer l's upload waits for the previous step's read-back of its buffers, its
+    call for its upload, its read-back for its call.  Device-timed with events on the
+    calling stream around all steps (it joins the read-back stream at the end).  One
+    step with everything on the calling stream comes first; the overlapped steps must
+    return the same bytes (``matches_serial``)."""
     import torch
     xs, ys = {}, {}
     for c in calls:
@@ -381,35 +387,77 @@ def _decode_e2e(args, calls, ids, ids_d, T, stream):
     yh = {k: v.cpu().pin_memory() for k, v in ys.items()}
     yo = {k: torch.empty_like(v).pin_memory() for k, v in yh.items()}
     ids_h = torch.from_numpy(np.asarray(ids, np.int32)).pin_memory()
+    xp = [sorted({x.data_ptr() for x, _, _ in c.items}) for c in calls]
+    yp = [sorted({y.data_ptr() for _, y, _ in c.items}) for c in calls]
 
-    def step():
+    def serial_step():
         with torch.cuda.stream(stream):
             ids_d.copy_(ids_h, non_blocking=True)
-            for c in calls:
-                for p in {x.data_ptr() for x, _, _ in c.items}:
+            for l, c in enumerate(calls):
+                for p in xp[l]:
                     xs[p].copy_(xh[p], non_blocking=True)
-                for p in {y.data_ptr() for _, y, _ in c.items}:
+                for p in yp[l]:
                     ys[p].copy_(yh[p], non_blocking=True)
                 c(stream)
-                for p in {y.data_ptr() for _, y, _ in c.items}:
+                for p in yp[l]:
                     yo[p].copy_(ys[p], non_blocking=True)
 
+    serial_step()
+    torch.cuda.synchronize()
+    ref = {k: v.clone() for k, v in yo.items()}
+
+    up, down = torch.cuda.Stream(), torch.cuda.Stream()
+    ev_up = [torch.cuda.Event() for _ in calls]
+    ev_call = [torch.cuda.Event() for _ in calls]
+    ev_down = [torch.cuda.Event() for _ in calls]
+    primed = [False]
+
+    def step():
+        with torch.cuda.stream(up):
+            if primed[0]:
+                up.wait_event(ev_call[-1])   # the previous step's calls have read ids
+            ids_d.copy_(ids_h, non_blocking=True)
+            for l in range(len(calls)):
+                if primed[0]:
+                    up.wait_event(ev_down[l])   # the previous step is done with x_l, y_l
+                for p in xp[l]:
+                    xs[p].copy_(xh[p], non_blocking=True)
+                for p in yp[l]:
+                    ys[p].copy_(yh[p], non_blocking=True)
+                ev_up[l].record(up)
+        for l, c in enumerate(calls):
+            stream.wait_event(ev_up[l])
+            c(stream)
+            ev_call[l].record(stream)
+        with torch.cuda.stream(down):
+            for l in range(len(calls)):
+                down.wait_event(ev_call[l])
+                for p in yp[l]:
+                    yo[p].copy_(ys[p], non_blocking=True)
+                ev_down[l].record(down)
+        primed[0] = True
+
+    up.wait_stream(stream)
     for _ in range(max(args.warmup, 3)):
         step()
     torch.cuda.synchronize()
     reps = max(args.steps, 5)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
+    up.wait_event(e0)
     for _ in range(reps):
         step()
+    stream.wait_stream(down)
     e1.record(stream)
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / reps
+    same = all(torch.equal(ref[k], yo[k]) for k in yo)
     h2d = ids_h.numel() * 4 + sum(v.numel() * 2 for v in xh.values()) + sum(v.numel() * 2 for v in yh.values())
     d2h = sum(v.numel() * 2 for v in yo.values())
     return {"value": round(T / (ms * 1e-3), 1), "unit": "tokens/s", "ms_per_step": round(ms, 3),
-            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-            "sample": "the whole decode step (32 layers) from pinned host memory"}
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "matches_serial": bool(same),
+            "sample": "the whole decode step (32 layers) from pinned host memory, uploads, calls and "
+                      "read-backs on three streams"}
 
 
 def decode_bench(args, dev, stream, hbm, variant="ragged", fused=False, per_layer=True, e2e=False):
