@@ -62,3 +62,34 @@ def test_device_id_follows_cuda_visible_devices(monkeypatch):
     assert bench.smi_device_id(0) == "3" and bench.smi_device_id(1) == "5"
     monkeypatch.setenv("CUDA_VISIBLE_DEVICES", "GPU-8d1c2f3e-0000-1111-2222-333344445555")
     assert bench.smi_device_id(0) == "GPU-8d1c2f3e-0000-1111-2222-333344445555"
+
+
+def _run_bench(*argv, env=None):
+    import json
+    import subprocess
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    e = dict(os.environ, **(env or {}))
+    r = subprocess.run([sys.executable, os.path.join(root, "bench.py"), *argv], capture_output=True, text=True,
+                       timeout=600, cwd=root, env=e)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.strip()]
+    return [json.loads(ln) for ln in lines[-1:]]
+
+
+def test_reference_arm_prints_the_contract_line():
+    """The reference arm (the fp64 oracle on the host cores) prints one JSON line with
+    the headline metric, unit and config of the library's own arm."""
+    (line,) = _run_bench("--impl", "reference", "--steps", "1", "--warmup", "0")
+    assert line["impl"] == "reference"
+    assert line["metric"] == bench.METRIC and line["unit"] == "modules/s" and line["value"] > 0
+    assert line["higher_is_better"] is True and line["steps"] == 1 and line["warmup"] == 0
+    assert line["config"] == bench.headline_config(bench.N_ADAPTERS, 1)
+    cb = line["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == line["value"]
+    assert line["e2e"] == {"value": line["value"], "unit": "modules/s", "h2d_bytes_per_step": 0,
+                           "d2h_bytes_per_step": 0}
+
+
+def test_reference_arm_other_ranks_do_no_work():
+    assert _run_bench("--impl", "reference", "--steps", "1", "--warmup", "0",
+                      env={"RANK": "1", "WORLD_SIZE": "2", "LOCAL_RANK": "1"}) == []
