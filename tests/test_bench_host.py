@@ -93,3 +93,29 @@ def test_reference_arm_prints_the_contract_line():
 def test_reference_arm_other_ranks_do_no_work():
     assert _run_bench("--impl", "reference", "--steps", "1", "--warmup", "0",
                       env={"RANK": "1", "WORLD_SIZE": "2", "LOCAL_RANK": "1"}) == []
+
+
+def test_traffic_record_is_dropped_once_the_kernel_source_changes(tmp_path, monkeypatch):
+    import hashlib
+    import json
+    src = tmp_path / "k.cuh"
+    src.write_text("kernel v1\n")
+    (tmp_path / "profiles").mkdir()
+    rec = {"leaf": {"bytes_per_unit": 1000.5, "source": "k.cuh",
+                    "source_sha256": hashlib.sha256(src.read_bytes()).hexdigest()}}
+    (tmp_path / "profiles" / "traffic.json").write_text(json.dumps(rec))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.kernel_traffic("leaf", 10) == 10005          # scaled by the units one launch processes
+    assert bench.kernel_traffic("other", 10) is None
+    src.write_text("kernel v2\n")                             # the kernel changed since the capture
+    assert bench.kernel_traffic("leaf", 10) is None
+
+
+def test_committed_traffic_records_name_their_captures():
+    import json
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    recs = json.load(open(os.path.join(root, "profiles", "traffic.json")))
+    for name, r in recs.items():
+        assert os.path.exists(os.path.join(root, r["capture"])), name
+        assert os.path.exists(os.path.join(root, r["source"])), name
+        assert r["bytes_per_unit"] * r["units_captured"] == pytest.approx(r["dram_read"] + r["dram_write"])
