@@ -2,8 +2,8 @@
 Python integers; nothing here imports the CUDA path or the oracle).
 
 The leaf reads each column of an item as 32-bit fixed point: the column is scaled by
-2^(31 - E), E = the exponent of its largest magnitude over the item's first 128 rows + 2,
-and truncated to an integer N.  Flipping the sign bit (U = N + 2^31) makes the four bytes
+2^(31 - E), E = the exponent of its largest magnitude over the item's first 128 rows + 2
+(that magnitude lies below 2^(E - 2)), and truncated toward zero to an integer N.  Flipping the sign bit (U = N + 2^31) makes the four bytes
 of U unsigned digits whose top digit is the signed top digit + 128, so N^T N is a sum of
 16 Grams of unsigned byte matrices, weighted by powers of 256, with column-sum
 corrections for the +128.  These tests check that this reading reproduces N^T N exactly,
@@ -20,7 +20,7 @@ def fixed_point(X, lead=128):
     """(N, E): N = trunc(X 2^(31 - E)) per column as int64; E from the first `lead` rows."""
     m = np.max(np.abs(X[:lead]), axis=0)
     _, e = np.frexp(m)                  # m = f 2^e with f in [0.5, 1)
-    E = e + 2
+    E = np.where(m > 0, e + 2, -90)     # a column whose lead rows are zero: any later nonzero value is out of range
     assert np.all(np.abs(X) < np.ldexp(1.0, E)), "a value at or above 2^E leaves the integer leaf"
     N = np.trunc(np.ldexp(X, 31 - E)).astype(np.int64)
     assert np.all(np.abs(N) < 2 ** 31)
